@@ -1,0 +1,22 @@
+"""Exact scaled dot-product attention forward for B200 (sm_100a).
+
+The compute path is the C-ABI library ``libattn.so`` (hand-written CUDA:
+TMA loads, tcgen05 MMAs into Tensor Memory, online softmax).  This package is a
+thin ctypes binding over it; PyTorch is used only for device memory and streams.
+
+The binding is loaded on first use; if ``libattn.so`` is missing the first call
+raises ImportError -- there is no fallback of any kind.
+"""
+from __future__ import annotations
+
+__all__ = [
+    "attn_fwd", "attn_fwd_config", "attn_status_sync", "attn_status_string",
+    "attn_last_error", "attn_selftest_timeout", "fwd", "AttnError",
+]
+
+
+def __getattr__(name):
+    if name in __all__:
+        from . import binding
+        return getattr(binding, name)
+    raise AttributeError(name)

@@ -1,0 +1,136 @@
+"""Seeded, counter-based synthetic inputs shared by the CUDA path's tests/bench and
+by the oracle's callers.
+
+This module holds NO attention arithmetic: it only turns (seed, tensor id, flat
+element index) into a BF16 value, and picks sampled query rows.  Because the
+generator is counter based, any subset of a tensor (one head, a few query rows)
+can be produced without generating the rest, which is how the oracle is fed at
+sizes where the full tensors would not fit its time budget.
+
+Definition (fixed here, used by every consumer):
+
+  gamma      = 0x9E3779B97F4A7C15                (SplitMix64 increment)
+  mix(z)     = SplitMix64 finaliser: z ^= z>>30; z *= 0xBF58476D1CE4E5B9;
+                                     z ^= z>>27; z *= 0x94D049BB133111EB; z ^= z>>31
+  key        = mix(mix(seed + gamma) + tensor_id)  tensor_id: Q=0, K=1, V=2
+  bits(i)    = mix(key + (i + 1) * gamma)          (all arithmetic mod 2^64)
+  normal     : u1 = (hi32 + 0.5) / 2^32, u2 = lo32 / 2^32,
+               z = sqrt(-2 ln u1) * cos(2 pi u2)   (Box-Muller, cosine branch, fp64)
+  uniform    : u = (bits >> 40) / 2^24,  z = 2u - 1  in [-1, 1)
+  value      = bf16_rne(fp32_rne(mult * z))
+
+(SplitMix64: Steele, Lea & Flood, "Fast splittable pseudorandom number
+generators", OOPSLA 2014.)
+"""
+from __future__ import annotations
+
+import numpy as np
+
+GAMMA = np.uint64(0x9E3779B97F4A7C15)
+_M1 = np.uint64(0xBF58476D1CE4E5B9)
+_M2 = np.uint64(0x94D049BB133111EB)
+
+TENSOR_ID = {"q": 0, "k": 1, "v": 2}
+
+_CHUNK = 1 << 22
+
+
+def _mix(z: np.ndarray) -> np.ndarray:
+    z = z ^ (z >> np.uint64(30))
+    z = z * _M1
+    z = z ^ (z >> np.uint64(27))
+    z = z * _M2
+    return z ^ (z >> np.uint64(31))
+
+
+def _key(seed: int, tensor_id: int) -> np.uint64:
+    with np.errstate(over="ignore"):
+        s = np.array([seed], dtype=np.uint64) + GAMMA
+        k = _mix(s) + np.uint64(tensor_id)
+        return _mix(k)[0]
+
+
+def _bits(key: np.uint64, idx: np.ndarray) -> np.ndarray:
+    with np.errstate(over="ignore"):
+        ctr = key + (idx.astype(np.uint64) + np.uint64(1)) * GAMMA
+        return _mix(ctr)
+
+
+def f32_to_bf16_bits(x: np.ndarray) -> np.ndarray:
+    """Round fp32 to BF16 (round to nearest, ties to even); returns uint16 bits."""
+    u = np.ascontiguousarray(x, dtype=np.float32).view(np.uint32)
+    rounding = ((u >> np.uint32(16)) & np.uint32(1)) + np.uint32(0x7FFF)
+    return ((u + rounding) >> np.uint32(16)).astype(np.uint16)
+
+
+def bf16_bits_to_f32(b: np.ndarray) -> np.ndarray:
+    return (np.asarray(b, dtype=np.uint16).astype(np.uint32) << np.uint32(16)).view(np.float32)
+
+
+def bf16_bits_to_f64(b: np.ndarray) -> np.ndarray:
+    """Exact widening of BF16 bit patterns to fp64."""
+    return bf16_bits_to_f32(b).astype(np.float64)
+
+
+def _values(key: np.uint64, idx: np.ndarray, dist: str, mult: float) -> np.ndarray:
+    bits = _bits(key, idx)
+    if dist == "normal":
+        hi = (bits >> np.uint64(32)).astype(np.float64)
+        lo = (bits & np.uint64(0xFFFFFFFF)).astype(np.float64)
+        u1 = (hi + 0.5) * (1.0 / 4294967296.0)
+        u2 = lo * (1.0 / 4294967296.0)
+        z = np.sqrt(-2.0 * np.log(u1)) * np.cos(2.0 * np.pi * u2)
+    elif dist == "uniform":
+        u = (bits >> np.uint64(40)).astype(np.float64) * (1.0 / 16777216.0)
+        z = 2.0 * u - 1.0
+    else:
+        raise ValueError(f"unknown distribution {dist!r}")
+    return f32_to_bf16_bits((mult * z).astype(np.float32))
+
+
+def gen_bf16_at(seed: int, tensor: str, flat_idx: np.ndarray, dist: str = "normal",
+                mult: float = 1.0) -> np.ndarray:
+    """BF16 bits of the elements with the given flat indices (any shape)."""
+    key = _key(seed, TENSOR_ID[tensor])
+    idx = np.asarray(flat_idx, dtype=np.int64)
+    flat = idx.reshape(-1)
+    out = np.empty(flat.shape, dtype=np.uint16)
+    for s in range(0, flat.size, _CHUNK):
+        out[s:s + _CHUNK] = _values(key, flat[s:s + _CHUNK], dist, mult)
+    return out.reshape(idx.shape)
+
+
+def gen_bf16(seed: int, tensor: str, shape, dist: str = "normal", mult: float = 1.0,
+             out: np.ndarray | None = None) -> np.ndarray:
+    """BF16 bits of a whole contiguous tensor of ``shape`` (flat index = C order)."""
+    n = int(np.prod(shape))
+    key = _key(seed, TENSOR_ID[tensor])
+    if out is None:
+        out = np.empty(n, dtype=np.uint16)
+    flat = out.reshape(-1)
+    assert flat.size == n
+    for s in range(0, n, _CHUNK):
+        e = min(n, s + _CHUNK)
+        flat[s:e] = _values(key, np.arange(s, e, dtype=np.int64), dist, mult)
+    return out.reshape(shape)
+
+
+def sample_rows(seed: int, bh: int, n: int, count: int) -> np.ndarray:
+    """``count`` distinct query rows of head ``bh`` (sorted), always with 0 and n-1.
+
+    Drawn with the same counter generator (tensor id 16 + bh), so they are fixed
+    by (seed, bh, n, count) alone.
+    """
+    if count >= n:
+        return np.arange(n, dtype=np.int64)
+    key = _key(seed, 16 + bh)
+    chosen = {0, n - 1}
+    ctr = 0
+    while len(chosen) < count:
+        bits = _bits(key, np.arange(ctr, ctr + 4 * count, dtype=np.int64))
+        ctr += 4 * count
+        for b in (bits % np.uint64(n)).tolist():
+            chosen.add(int(b))
+            if len(chosen) == count:
+                break
+    return np.array(sorted(chosen), dtype=np.int64)

@@ -1,0 +1,94 @@
+"""Named synthetic workloads (shapes, seeds, value distributions).
+
+No attention arithmetic here.  Each workload fixes B, H, Nq, Nk, d, causality,
+the seed and the distribution of Q, K and V; the scale is the fp32 value of
+1/sqrt(d).  The pages name no dataset or benchmark suite: their workloads are
+BF16 multi-head attention forwards on B200 at long sequence lengths, so these
+synthetic shapes stand in for them.
+"""
+from __future__ import annotations
+
+import dataclasses
+import math
+
+import numpy as np
+
+from . import inputs
+
+
+@dataclasses.dataclass(frozen=True)
+class Workload:
+    name: str
+    B: int
+    H: int
+    Nq: int
+    Nk: int
+    d: int
+    causal: bool
+    seed: int
+    q_dist: str = "normal"
+    q_mult: float = 1.0
+    k_dist: str = "normal"
+    v_dist: str = "normal"
+    oracle_rows: int | None = None  # sampled rows per head for the oracle; None = all
+
+    @property
+    def scale(self) -> float:
+        return float(np.float32(1.0 / math.sqrt(self.d)))
+
+    @property
+    def flops(self) -> float:
+        """Algorithmic FLOPs: 4*B*H*Nq*Nk*d, halved when causal."""
+        f = 4.0 * self.B * self.H * self.Nq * self.Nk * self.d
+        return f / 2 if self.causal else f
+
+    def shape(self, which: str):
+        n = self.Nq if which == "q" else self.Nk
+        return (self.B, self.H, n, self.d)
+
+    def dist(self, which: str):
+        if which == "q":
+            return self.q_dist, self.q_mult
+        if which == "k":
+            return self.k_dist, 1.0
+        return self.v_dist, 1.0
+
+    def tensor_bits(self, which: str) -> np.ndarray:
+        dist, mult = self.dist(which)
+        return inputs.gen_bf16(self.seed, which, self.shape(which), dist, mult)
+
+    def head_bits(self, which: str, bh: int) -> np.ndarray:
+        """BF16 bits of one (b, h) slice, [N, d]."""
+        dist, mult = self.dist(which)
+        n = self.Nq if which == "q" else self.Nk
+        base = bh * n * self.d
+        idx = np.arange(base, base + n * self.d, dtype=np.int64)
+        return inputs.gen_bf16_at(self.seed, which, idx, dist, mult).reshape(n, self.d)
+
+    def q_rows_bits(self, bh: int, rows: np.ndarray) -> np.ndarray:
+        dist, mult = self.dist("q")
+        base = bh * self.Nq * self.d
+        idx = base + rows.astype(np.int64)[:, None] * self.d + np.arange(self.d, dtype=np.int64)[None, :]
+        return inputs.gen_bf16_at(self.seed, "q", idx, dist, mult)
+
+    def sampled_rows(self, bh: int) -> np.ndarray:
+        if self.oracle_rows is None:
+            return np.arange(self.Nq, dtype=np.int64)
+        return inputs.sample_rows(self.seed, bh, self.Nq, self.oracle_rows)
+
+
+WORKLOADS = {
+    w.name: w
+    for w in [
+        Workload("tiny_b1h2n128d64", 1, 2, 128, 128, 64, False, seed=0),
+        Workload("mha_b4h16n1k_d128", 4, 16, 1024, 1024, 128, False, seed=1),
+        Workload("mha_b2h16n8k_d128", 2, 16, 8192, 8192, 128, False, seed=2, oracle_rows=256),
+        Workload("mha_b2h16n8k_d128_causal", 2, 16, 8192, 8192, 128, True, seed=2, oracle_rows=256),
+        Workload("wide_logits_b1h32n16k_d128_causal", 1, 32, 16384, 16384, 128, True, seed=3,
+                 q_mult=8.0, v_dist="uniform", oracle_rows=256),
+        Workload("long_b1h16n128k_d128_causal", 1, 16, 131072, 131072, 128, True, seed=4,
+                 oracle_rows=256),
+    ]
+}
+
+HEADLINE = "mha_b2h16n8k_d128"

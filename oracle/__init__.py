@@ -1,0 +1,105 @@
+"""fp64 CPU oracle for exact attention (forward).
+
+TEST INFRASTRUCTURE.  Only ``tests/``, ``__graft_entry__.smoke()`` and the
+``cpu_baseline`` / ``--impl reference`` legs of ``bench.py`` may import this
+package.  The product path (``exact_attention_152_b200``) never touches it, and
+this package never imports the product.
+
+The arithmetic lives in ``attn_oracle.c`` (plain C, fp64, one query row at a
+time, written straight from the definition -- see that file's header for the
+citations and the readings of the pages).  This module only compiles it with
+gcc, marshals numpy arrays and loops over (batch, head).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "attn_oracle.c")
+_LIB = os.path.join(_HERE, "liboracle.so")
+_lock = threading.Lock()
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile ``attn_oracle.c`` into ``liboracle.so`` (gcc, -O2, fp-contract off)."""
+    if not force and os.path.exists(_LIB) and os.path.getmtime(_LIB) >= os.path.getmtime(_SRC):
+        return _LIB
+    tmp = _LIB + f".tmp{os.getpid()}"
+    # -ffp-contract=off: no fused multiply-add, so every product and sum rounds
+    # exactly as written in fp64.
+    cmd = ["gcc", "-O2", "-ffp-contract=off", "-fPIC", "-shared", "-pthread",
+           "-o", tmp, _SRC, "-lm"]
+    subprocess.run(cmd, check=True)
+    os.replace(tmp, _LIB)
+    return _LIB
+
+
+def _load():
+    global _lib
+    with _lock:
+        if _lib is None:
+            lib = ctypes.CDLL(build())
+            f = lib.oracle_attn_rows_f64
+            f.restype = ctypes.c_int
+            f.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64,
+                          ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64,
+                          ctypes.c_double, ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p,
+                          ctypes.c_int]
+            _lib = lib
+    return _lib
+
+
+def default_threads() -> int:
+    return max(1, os.cpu_count() or 1)
+
+
+def attn_rows(q_rows, rows, k, v, scale, causal, nthreads=None):
+    """Attention of selected query rows of ONE (batch, head).
+
+    q_rows: [n, d] fp64 -- the query vectors of rows ``rows`` (int64 [n]).
+    k, v:   [Nk, d] fp64.
+    Returns (o [n, d] fp64, lse [n] fp64, natural log).
+    """
+    lib = _load()
+    q_rows = np.ascontiguousarray(q_rows, dtype=np.float64)
+    rows = np.ascontiguousarray(rows, dtype=np.int64)
+    k = np.ascontiguousarray(k, dtype=np.float64)
+    v = np.ascontiguousarray(v, dtype=np.float64)
+    n, d = q_rows.shape
+    nk = k.shape[0]
+    assert rows.shape == (n,) and k.shape == (nk, d) and v.shape == (nk, d)
+    if causal:
+        assert np.all(rows >= 0)
+    o = np.empty((n, d), dtype=np.float64)
+    lse = np.empty((n,), dtype=np.float64)
+    nt = default_threads() if nthreads is None else int(nthreads)
+    rc = lib.oracle_attn_rows_f64(q_rows.ctypes.data, rows.ctypes.data, n,
+                                  k.ctypes.data if nk else None,
+                                  v.ctypes.data if nk else None, nk, d,
+                                  float(scale), 1 if causal else 0,
+                                  o.ctypes.data, lse.ctypes.data, nt)
+    if rc != 0:
+        raise RuntimeError("oracle_attn_rows_f64 failed")
+    return o, lse
+
+
+def attn_fwd(q, k, v, scale, causal=False, nthreads=None):
+    """Full attention over [B, H, N, d] fp64 arrays -> (o [B,H,Nq,d], lse [B,H,Nq])."""
+    q = np.asarray(q, dtype=np.float64)
+    k = np.asarray(k, dtype=np.float64)
+    v = np.asarray(v, dtype=np.float64)
+    B, H, nq, d = q.shape
+    o = np.empty((B, H, nq, d), dtype=np.float64)
+    lse = np.empty((B, H, nq), dtype=np.float64)
+    rows = np.arange(nq, dtype=np.int64)
+    for b in range(B):
+        for h in range(H):
+            o[b, h], lse[b, h] = attn_rows(q[b, h], rows, k[b, h], v[b, h],
+                                           scale, causal, nthreads)
+    return o, lse

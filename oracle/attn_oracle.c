@@ -1,0 +1,164 @@
+/*
+ * Plain fp64 CPU oracle for exact scaled dot-product attention (forward).
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing in the product path may link, load or call
+ * this file; it exists so that tests, the smoke check and the CPU-baseline leg of
+ * the benchmark can compare the CUDA kernel against an obviously correct
+ * definition.  It shares no code, header, table or constant with the kernel.
+ *
+ * What it computes (the plain definition, no tiling, no online softmax):
+ *
+ *   FlashAttention 4: LLM向けのより高速でメモリ効率の良いアテンション
+ *   (ja.linux-konsole.com), section "はじめに": attention takes the queries Q,
+ *   multiplies them with the keys K, normalises the result with a softmax and
+ *   multiplies that with the values V.
+ *
+ *   Flash Attention glossary (jisaku.com), sections "主要な最適化ポイントのまとめ"
+ *   and "FAQ" (Q3): the tiled method is exact -- it equals standard attention up
+ *   to floating-point rounding -- so the oracle is the standard definition
+ *   written out.
+ *
+ * The pages print no formula (it was lost in extraction) and never mention the
+ * scale factor, causal masking or the log-sum-exp output.  This library's
+ * readings, applied identically here and in the kernel's contract:
+ *
+ *   s_j   = scale * sum_c q_c * k_jc           for j in K(i)
+ *   K(i)  = {0 .. Nk-1}, or {0 .. i} when causal (causal requires Nq == Nk)
+ *   m     = max_j s_j
+ *   e_j   = exp(s_j - m),  l = sum_j e_j
+ *   O_i   = sum_j (e_j / l) * v_j
+ *   LSE_i = m + log(l)      (natural log)
+ *   K(i) empty  ->  O_i = 0, LSE_i = -inf
+ *
+ * All arithmetic is fp64.  Inputs arrive as fp64 (the caller widens the BF16
+ * values, which is exact), so the only rounding is fp64 rounding.
+ *
+ * Parallelism: independent query rows are spread over POSIX threads.  That is
+ * not blocking or reordering of the definition -- each row is computed alone,
+ * in the order written above.
+ */
+#include <math.h>
+#include <pthread.h>
+#include <stdint.h>
+#include <stdlib.h>
+
+typedef struct {
+    const double *q;      /* [n_rows, d]  query rows to evaluate            */
+    const int64_t *rows;  /* [n_rows]     their indices i in [0, Nq)         */
+    int64_t n_rows;
+    const double *k;      /* [Nk, d]                                          */
+    const double *v;      /* [Nk, d]                                          */
+    int64_t nk;
+    int64_t d;
+    double scale;
+    int causal;
+    double *o;            /* [n_rows, d]  out                                 */
+    double *lse;          /* [n_rows]     out                                 */
+    double *s;            /* per-thread score row, [nk]                       */
+    int64_t begin, end;   /* row range handled by this thread                 */
+} oracle_job;
+
+/* One query row: full score row, then max, exp, sum, weighted sum of V. */
+static void oracle_row(const oracle_job *jb, int64_t r) {
+    const int64_t d = jb->d;
+    const double *qi = jb->q + r * d;
+    double *oi = jb->o + r * d;
+    const int64_t i = jb->rows[r];
+    /* visible keys: all of them, or the prefix 0..i when causal */
+    int64_t nvis = jb->nk;
+    if (jb->causal) nvis = (i + 1 < jb->nk) ? i + 1 : jb->nk;
+    if (nvis <= 0) {
+        for (int64_t c = 0; c < d; ++c) oi[c] = 0.0;
+        jb->lse[r] = -INFINITY;
+        return;
+    }
+    double *s = jb->s;
+    for (int64_t j = 0; j < nvis; ++j) {
+        const double *kj = jb->k + j * d;
+        double dot = 0.0;
+        for (int64_t c = 0; c < d; ++c) dot += qi[c] * kj[c];
+        s[j] = jb->scale * dot;
+    }
+    double m = s[0];
+    for (int64_t j = 1; j < nvis; ++j)
+        if (s[j] > m) m = s[j];
+    double l = 0.0;
+    for (int64_t j = 0; j < nvis; ++j) {
+        s[j] = exp(s[j] - m);
+        l += s[j];
+    }
+    for (int64_t c = 0; c < d; ++c) oi[c] = 0.0;
+    for (int64_t j = 0; j < nvis; ++j) {
+        const double p = s[j] / l;
+        const double *vj = jb->v + j * d;
+        for (int64_t c = 0; c < d; ++c) oi[c] += p * vj[c];
+    }
+    jb->lse[r] = m + log(l);
+}
+
+static void *oracle_worker(void *arg) {
+    oracle_job *jb = (oracle_job *)arg;
+    for (int64_t r = jb->begin; r < jb->end; ++r) oracle_row(jb, r);
+    return NULL;
+}
+
+/*
+ * Attention for a subset of query rows of one (batch, head).
+ *
+ * q:    [n_rows, d] fp64, the query rows to evaluate (row r has index rows[r]).
+ * k, v: [nk, d] fp64, all keys and values of that head.
+ * o:    [n_rows, d] fp64 out;  lse: [n_rows] fp64 out (natural log).
+ * nthreads <= 0 means one thread.
+ * Returns 0 on success, -1 on a bad argument or allocation failure.
+ */
+int oracle_attn_rows_f64(const double *q, const int64_t *rows, int64_t n_rows,
+                         const double *k, const double *v, int64_t nk, int64_t d,
+                         double scale, int causal, double *o, double *lse,
+                         int nthreads) {
+    if (n_rows < 0 || nk < 0 || d <= 0) return -1;
+    if (n_rows == 0) return 0;
+    if (!q || !rows || !o || !lse || (nk > 0 && (!k || !v))) return -1;
+    if (nthreads <= 0) nthreads = 1;
+    if (nthreads > n_rows) nthreads = (int)n_rows;
+
+    oracle_job *jobs = (oracle_job *)calloc((size_t)nthreads, sizeof(oracle_job));
+    pthread_t *tids = (pthread_t *)calloc((size_t)nthreads, sizeof(pthread_t));
+    if (!jobs || !tids) {
+        free(jobs);
+        free(tids);
+        return -1;
+    }
+    int rc = 0;
+    int started = 0;
+    const int64_t per = (n_rows + nthreads - 1) / nthreads;
+    for (int t = 0; t < nthreads; ++t) {
+        oracle_job *jb = &jobs[t];
+        jb->q = q; jb->rows = rows; jb->n_rows = n_rows;
+        jb->k = k; jb->v = v; jb->nk = nk; jb->d = d;
+        jb->scale = scale; jb->causal = causal;
+        jb->o = o; jb->lse = lse;
+        jb->begin = (int64_t)t * per;
+        jb->end = jb->begin + per < n_rows ? jb->begin + per : n_rows;
+        jb->s = (double *)malloc((size_t)(nk > 0 ? nk : 1) * sizeof(double));
+        if (!jb->s) { rc = -1; break; }
+    }
+    if (rc == 0) {
+        for (int t = 1; t < nthreads; ++t) {
+            if (pthread_create(&tids[t], NULL, oracle_worker, &jobs[t]) != 0) {
+                /* run it on this thread instead */
+                oracle_worker(&jobs[t]);
+                tids[t] = 0;
+            } else {
+                ++started;
+            }
+        }
+        oracle_worker(&jobs[0]);
+        for (int t = 1; t < nthreads; ++t)
+            if (tids[t]) pthread_join(tids[t], NULL);
+    }
+    (void)started;
+    for (int t = 0; t < nthreads; ++t) free(jobs[t].s);
+    free(jobs);
+    free(tids);
+    return rc;
+}

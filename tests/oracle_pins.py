@@ -1,0 +1,225 @@
+"""Pins for the fp64 oracle: checks against facts that do not come from the oracle.
+
+Each ``pin_*`` takes an ``attn_rows(q_rows, rows, k, v, scale, causal)`` callable
+(the oracle's per-head entry) and raises AssertionError when it disagrees with
+what the mathematics fixes.  ``test_oracle_pins.py`` runs them on the real
+oracle and on deliberately broken copies of it (to show each plausible mistake
+is caught by at least one pin).
+"""
+from __future__ import annotations
+
+import json
+import math
+import os
+
+import numpy as np
+
+GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden", "closed_forms.json")
+
+
+def _rng(seed):
+    return np.random.default_rng(seed)
+
+
+def _full(attn_rows, q, k, v, scale, causal):
+    rows = np.arange(q.shape[0], dtype=np.int64)
+    return attn_rows(q, rows, k, v, scale, causal)
+
+
+def brute_force_python(q, k, v, scale, causal):
+    """Textbook attention in pure Python floats: S, then softmax without any max
+    subtraction, then P.V.  Only for tiny shapes and small logits."""
+    nq, d = len(q), len(q[0])
+    nk = len(k)
+    o, lse = [], []
+    for i in range(nq):
+        keys = range(min(i + 1, nk)) if causal else range(nk)
+        w = {}
+        for j in keys:
+            w[j] = math.exp(scale * sum(q[i][c] * k[j][c] for c in range(d)))
+        z = sum(w.values())
+        o.append([sum(w[j] * v[j][c] for j in keys) / z for c in range(d)])
+        lse.append(math.log(z))
+    return np.array(o), np.array(lse)
+
+
+def pin_brute_force(attn_rows):
+    """Match a brute-force materialised softmax on tiny shapes (both maskings)."""
+    for seed, (nq, nk, d) in enumerate([(1, 1, 1), (3, 5, 2), (7, 7, 4), (9, 9, 3), (4, 13, 8)]):
+        r = _rng(seed)
+        q, k, v = (r.standard_normal((n, d)) for n in (nq, nk, nk))
+        for causal in (False, True):
+            if causal and nq != nk:
+                continue
+            scale = 0.7
+            o, lse = _full(attn_rows, q, k, v, scale, causal)
+            ob, lb = brute_force_python(q.tolist(), k.tolist(), v.tolist(), scale, causal)
+            np.testing.assert_allclose(o, ob, rtol=1e-12, atol=1e-12)
+            np.testing.assert_allclose(lse, lb, rtol=1e-12, atol=1e-12)
+
+
+def pin_golden(attn_rows):
+    """Hand-derived closed forms stored under tests/golden/."""
+    with open(GOLDEN) as f:
+        cases = json.load(f)["cases"]
+    for c in cases:
+        q, k, v = (np.array(c[x], dtype=np.float64) for x in ("q", "k", "v"))
+        o, lse = _full(attn_rows, q, k, v, c["scale"], c["causal"])
+        np.testing.assert_allclose(o, np.array(c["o"]), rtol=1e-13, atol=1e-13, err_msg=c["name"])
+        np.testing.assert_allclose(lse, np.array(c["lse"]), rtol=1e-13, atol=1e-13, err_msg=c["name"])
+
+
+def pin_single_key(attn_rows):
+    """One key: softmax weight is exactly 1, so O = V0 bit-exactly and LSE = s0."""
+    r = _rng(11)
+    q, k, v = r.standard_normal((5, 16)), r.standard_normal((1, 16)), r.standard_normal((1, 16))
+    o, lse = _full(attn_rows, q, k, v, 0.3, False)
+    assert np.array_equal(o, np.repeat(v, 5, axis=0))
+    np.testing.assert_allclose(lse, 0.3 * (q @ k[0]), rtol=1e-14, atol=1e-14)
+
+
+def pin_identical_keys(attn_rows):
+    """All keys equal: uniform weights, O = mean(V), LSE = s + log(Nk)."""
+    r = _rng(12)
+    nk, d = 37, 8
+    q = r.standard_normal((4, d))
+    k = np.repeat(r.standard_normal((1, d)), nk, axis=0)
+    v = r.standard_normal((nk, d))
+    o, lse = _full(attn_rows, q, k, v, 0.9, False)
+    np.testing.assert_allclose(o, np.repeat(v.mean(0, keepdims=True), 4, 0), rtol=1e-12, atol=1e-13)
+    np.testing.assert_allclose(lse, 0.9 * (q @ k[0]) + math.log(nk), rtol=1e-13, atol=1e-13)
+
+
+def pin_zero_scale(attn_rows):
+    """scale = 0: every logit is 0, O = mean(V), LSE = log(Nk)."""
+    r = _rng(13)
+    q, k, v = r.standard_normal((3, 8)), r.standard_normal((10, 8)), r.standard_normal((10, 8))
+    o, lse = _full(attn_rows, q, k, v, 0.0, False)
+    np.testing.assert_allclose(o, np.repeat(v.mean(0, keepdims=True), 3, 0), rtol=1e-12, atol=1e-13)
+    np.testing.assert_allclose(lse, np.full(3, math.log(10)), rtol=1e-14)
+
+
+def pin_causal_prefix(attn_rows):
+    """Causal row 0 is V0 exactly; causal row i equals unmasked attention over keys 0..i."""
+    r = _rng(14)
+    n, d = 12, 8
+    q, k, v = (r.standard_normal((n, d)) for _ in range(3))
+    o, lse = _full(attn_rows, q, k, v, 0.5, True)
+    assert np.array_equal(o[0], v[0])
+    for i in range(n):
+        oi, li = attn_rows(q[i:i + 1], np.array([0], dtype=np.int64), k[:i + 1], v[:i + 1], 0.5, False)
+        np.testing.assert_allclose(o[i], oi[0], rtol=1e-12, atol=1e-13)
+        np.testing.assert_allclose(lse[i], li[0], rtol=1e-13, atol=1e-13)
+
+
+def pin_rows_sum_to_one(attn_rows):
+    """With independently computed logits s, sum_j exp(s_j - LSE) = 1 and
+    O = sum_j exp(s_j - LSE) v_j  (normalisation and the LSE together)."""
+    r = _rng(15)
+    q, k, v = r.standard_normal((6, 8)), r.standard_normal((21, 8)), r.standard_normal((21, 8))
+    scale = 0.8
+    o, lse = _full(attn_rows, q, k, v, scale, False)
+    s = scale * np.einsum("id,jd->ij", q, k)
+    p = np.exp(s - lse[:, None])
+    np.testing.assert_allclose(p.sum(1), np.ones(6), rtol=1e-13)
+    np.testing.assert_allclose(o, p @ v, rtol=1e-12, atol=1e-13)
+
+
+def pin_shift_invariance(attn_rows):
+    """Adding one vector c to every key leaves O unchanged and shifts LSE_i by
+    scale * q_i . c (softmax is invariant to a per-row constant)."""
+    r = _rng(16)
+    q, k, v = r.standard_normal((5, 8)), r.standard_normal((9, 8)), r.standard_normal((9, 8))
+    c = r.standard_normal(8)
+    o1, l1 = _full(attn_rows, q, k, v, 0.6, False)
+    o2, l2 = _full(attn_rows, q, k + c, v, 0.6, False)
+    np.testing.assert_allclose(o2, o1, rtol=1e-11, atol=1e-12)
+    np.testing.assert_allclose(l2, l1 + 0.6 * (q @ c), rtol=1e-12, atol=1e-12)
+
+
+def pin_value_linearity(attn_rows):
+    """O is linear in V: O(V A) = O(V) A."""
+    r = _rng(17)
+    q, k, v = r.standard_normal((4, 6)), r.standard_normal((11, 6)), r.standard_normal((11, 6))
+    a = r.standard_normal((6, 6))
+    o1, _ = _full(attn_rows, q, k, v, 0.4, False)
+    o2, _ = _full(attn_rows, q, k, v @ a, 0.4, False)
+    np.testing.assert_allclose(o2, o1 @ a, rtol=1e-11, atol=1e-12)
+
+
+def pin_key_permutation(attn_rows):
+    """Unmasked attention does not depend on the order of the (key, value) pairs."""
+    r = _rng(18)
+    q, k, v = r.standard_normal((4, 8)), r.standard_normal((15, 8)), r.standard_normal((15, 8))
+    perm = r.permutation(15)
+    o1, l1 = _full(attn_rows, q, k, v, 0.5, False)
+    o2, l2 = _full(attn_rows, q, k[perm], v[perm], 0.5, False)
+    np.testing.assert_allclose(o2, o1, rtol=1e-12, atol=1e-13)
+    np.testing.assert_allclose(l2, l1, rtol=1e-13, atol=1e-13)
+
+
+def pin_split_merge(attn_rows):
+    """Attention over [K1;K2] equals the LSE-weighted merge of the two halves --
+    the algebra that lets a tiled method visit the keys block by block."""
+    r = _rng(19)
+    q, k, v = r.standard_normal((5, 8)), r.standard_normal((20, 8)), r.standard_normal((20, 8))
+    o, l = _full(attn_rows, q, k, v, 0.7, False)
+    o1, l1 = _full(attn_rows, q, k[:7], v[:7], 0.7, False)
+    o2, l2 = _full(attn_rows, q, k[7:], v[7:], 0.7, False)
+    lm = np.logaddexp(l1, l2)
+    om = np.exp(l1 - lm)[:, None] * o1 + np.exp(l2 - lm)[:, None] * o2
+    np.testing.assert_allclose(o, om, rtol=1e-12, atol=1e-13)
+    np.testing.assert_allclose(l, lm, rtol=1e-13, atol=1e-13)
+
+
+def pin_hard_max(attn_rows):
+    """As the scale grows the softmax becomes an argmax: O -> V at the largest logit.
+    Also exercises logits far beyond exp's range (the max must be subtracted)."""
+    r = _rng(20)
+    q, k, v = r.standard_normal((6, 8)), r.standard_normal((13, 8)), r.standard_normal((13, 8))
+    o, lse = _full(attn_rows, q, k, v, 1e6, False)
+    s = q @ k.T
+    best = s.argmax(1)
+    np.testing.assert_allclose(o, v[best], rtol=1e-9, atol=1e-9)
+    np.testing.assert_allclose(lse, 1e6 * s.max(1), rtol=1e-12)
+
+
+def pin_two_keys_sigmoid(attn_rows):
+    """Two keys: the weights are the logistic function of the logit difference."""
+    r = _rng(21)
+    q, k, v = r.standard_normal((8, 4)), r.standard_normal((2, 4)), r.standard_normal((2, 4))
+    o, lse = _full(attn_rows, q, k, v, 1.3, False)
+    s = 1.3 * (q @ k.T)
+    w0 = 1.0 / (1.0 + np.exp(s[:, 1] - s[:, 0]))
+    np.testing.assert_allclose(o, w0[:, None] * v[0] + (1 - w0)[:, None] * v[1], rtol=1e-12, atol=1e-13)
+    np.testing.assert_allclose(lse, np.logaddexp(s[:, 0], s[:, 1]), rtol=1e-13, atol=1e-13)
+
+
+def pin_empty_keys(attn_rows):
+    """No visible key: O = 0 and LSE = -inf (this library's definition)."""
+    q = np.ones((2, 4))
+    k = np.zeros((0, 4))
+    o, lse = attn_rows(q, np.arange(2, dtype=np.int64), k, k, 1.0, False)
+    assert np.array_equal(o, np.zeros((2, 4)))
+    assert np.all(np.isneginf(lse))
+
+
+def pin_sampled_rows(attn_rows):
+    """Evaluating a subset of rows gives the same values as evaluating all rows
+    (row sampling is how the oracle checks large problems)."""
+    r = _rng(22)
+    n, d = 30, 8
+    q, k, v = (r.standard_normal((n, d)) for _ in range(3))
+    for causal in (False, True):
+        o, lse = _full(attn_rows, q, k, v, 0.5, causal)
+        rows = np.array([0, 3, 17, 29], dtype=np.int64)
+        os_, ls_ = attn_rows(q[rows], rows, k, v, 0.5, causal)
+        assert np.array_equal(os_, o[rows]) and np.array_equal(ls_, lse[rows])
+
+
+ALL_PINS = [
+    pin_brute_force, pin_golden, pin_single_key, pin_identical_keys, pin_zero_scale,
+    pin_causal_prefix, pin_rows_sum_to_one, pin_shift_invariance, pin_value_linearity,
+    pin_key_permutation, pin_split_merge, pin_hard_max, pin_two_keys_sigmoid,
+    pin_empty_keys, pin_sampled_rows,
+]

@@ -1,0 +1,64 @@
+"""The seeded input generator (CPU only)."""
+import numpy as np
+import torch
+
+from exact_attention_152_b200 import inputs
+from exact_attention_152_b200.workloads import WORKLOADS
+
+
+def test_bf16_rounding_matches_torch():
+    r = np.random.default_rng(0)
+    x = np.concatenate([r.standard_normal(100000).astype(np.float32) * 10,
+                        np.array([1.0, -2.5, 1 + 2**-8, 1 + 3 * 2**-9, 65504.0, 1e-30], np.float32)])
+    ours = inputs.f32_to_bf16_bits(x)
+    ref = torch.from_numpy(x).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    assert np.array_equal(ours, ref)
+
+
+def test_widening_is_exact():
+    b = np.arange(0, 65536, 7, dtype=np.uint16)
+    b = b[(b & 0x7F80) != 0x7F80]  # drop inf/nan patterns
+    f = inputs.bf16_bits_to_f64(b)
+    back = inputs.f32_to_bf16_bits(f.astype(np.float32))
+    assert np.array_equal(back, b)
+
+
+def test_subset_equals_full():
+    full = inputs.gen_bf16(7, "k", (3, 50, 8))
+    idx = np.array([0, 5, 77, 1199, 600])
+    assert np.array_equal(inputs.gen_bf16_at(7, "k", idx), full.reshape(-1)[idx])
+
+
+def test_streams_differ_and_are_deterministic():
+    a = inputs.gen_bf16(1, "q", (1000,))
+    assert np.array_equal(a, inputs.gen_bf16(1, "q", (1000,)))
+    assert not np.array_equal(a, inputs.gen_bf16(1, "k", (1000,)))
+    assert not np.array_equal(a, inputs.gen_bf16(2, "q", (1000,)))
+
+
+def test_distributions():
+    z = inputs.bf16_bits_to_f64(inputs.gen_bf16(3, "q", (200000,)))
+    assert abs(z.mean()) < 0.01 and abs(z.std() - 1) < 0.01
+    z8 = inputs.bf16_bits_to_f64(inputs.gen_bf16(3, "q", (200000,), mult=8.0))
+    assert np.array_equal(z8, 8 * z)  # power-of-two scaling is exact
+    u = inputs.bf16_bits_to_f64(inputs.gen_bf16(3, "v", (200000,), dist="uniform"))
+    assert u.min() >= -1 and u.max() <= 1 and abs(u.mean()) < 0.01  # bf16 rounding may reach 1.0
+    assert abs(u.var() - 1 / 3) < 0.01
+
+
+def test_sample_rows():
+    rows = inputs.sample_rows(4, 3, 131072, 256)
+    assert len(rows) == 256 and rows[0] == 0 and rows[-1] == 131071
+    assert np.all(np.diff(rows) > 0)
+    assert np.array_equal(rows, inputs.sample_rows(4, 3, 131072, 256))
+    assert np.array_equal(inputs.sample_rows(0, 0, 10, 64), np.arange(10))
+
+
+def test_workload_slices_agree():
+    w = WORKLOADS["tiny_b1h2n128d64"]
+    q = w.tensor_bits("q")
+    assert q.shape == (1, 2, 128, 64)
+    assert np.array_equal(w.head_bits("q", 1), q[0, 1])
+    rows = np.array([0, 9, 127])
+    assert np.array_equal(w.q_rows_bits(1, rows), q[0, 1, rows])
+    assert WORKLOADS["mha_b2h16n8k_d128"].flops == 4 * 2 * 16 * 8192 * 8192 * 128
