@@ -1,0 +1,395 @@
+#!/usr/bin/env python
+"""Attention-forward benchmark on B200: one JSON line on stdout (rank 0).
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+A step is one call of the whole hot path -- one attn_fwd over the workload's full
+batch (B x H heads, Nq queries, Nk keys) -- on inputs already resident in HBM.
+The default workload is the non-causal B=2, H=16, N=8192, d=128 forward.  Its
+Q+K+V (201 MB) exceed the 126 MB L2, so L2 is not flushed between steps.
+
+Under torchrun (N > 1) every rank runs the same per-GPU workload on its own GPU
+(independent problems: weak scaling, no data-path collective); the timed region
+is bracketed by barrier + synchronize and its device time is the max over ranks.
+
+--impl reference times the fp64 CPU oracle (the reference arm: there is no
+runnable reference implementation) on bounded samples of query rows of the same
+workload, in the same metric.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "attention fwd TFLOP/s (BF16, 1×B200) and % of dense BF16 tensor peak"
+UNIT = "TFLOP/s"
+SPEC_DENSE_BF16_TFLOPS = 2250.0
+L2_BYTES = 126 * 1024 * 1024
+
+
+def parse_args(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=1000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--workload", default=None)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--e2e-steps", type=int, default=20)
+    ap.add_argument("--cpu-seconds", type=float, default=12.0,
+                    help="target CPU time of the oracle baseline sample")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--exp-mode", type=int, default=None, help="0 MUFU, 1 split, 2 polynomial")
+    ap.add_argument("--threshold", type=float, default=None, help="rescale threshold (powers of 2)")
+    return ap.parse_args(argv)
+
+
+def dist_env():
+    return (int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")),
+            int(os.environ.get("LOCAL_RANK", "0")))
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return {"burst": float(p["bf16_tflops"]), "sustained": float(p["bf16_tflops_sustained"]),
+                "hbm_gbs": float(p["hbm_gbs"]), "source": "measured"}
+    except Exception:
+        return {"burst": 1590.0, "sustained": 1400.0, "hbm_gbs": 6650.0, "source": "fallback"}
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "exact_attention_152_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        if name.endswith((".cu", ".cuh", ".h")):
+            with open(os.path.join(csrc, name), "rb") as f:
+                h.update(name.encode() + b"\0" + f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(workload_name):
+    """DRAM bytes per launch from a committed ncu summary, if it was taken on
+    the current kernel source; else None."""
+    path = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+    try:
+        with open(path) as f:
+            rec = json.load(f)
+    except Exception:
+        return None
+    e = rec.get(workload_name)
+    if not e or e.get("kernel_src_sha") != kernel_source_hash():
+        return None
+    return e.get("dram_bytes_per_launch")
+
+
+# ---------------------------------------------------------------------------
+# nvidia-smi clock sampling during the timed region
+# ---------------------------------------------------------------------------
+class ClockSampler:
+    FIELDS = ["clocks.sm", "clocks.max.sm", "power.draw", "utilization.gpu",
+              "clocks_event_reasons.hw_slowdown", "clocks_event_reasons.hw_thermal_slowdown",
+              "clocks_event_reasons.sw_thermal_slowdown", "clocks_event_reasons.sw_power_cap"]
+    REASONS = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+
+    def __init__(self, gpu_id: str):
+        self.gpu_id = gpu_id
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(prefix="clocks", suffix=".csv")
+            os.close(fd)
+            self.out = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", self.gpu_id, f"--query-gpu={','.join(self.FIELDS)}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=self.out, stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.out.close()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) != len(self.FIELDS):
+                    continue
+                try:
+                    rows.append((float(parts[0]), float(parts[1]), float(parts[2]), float(parts[3]),
+                                 parts[4:]))
+                except ValueError:
+                    continue
+        os.unlink(self.path)
+        if not rows:
+            return None
+        loaded = [r for r in rows if r[3] >= 50.0] or rows
+        reasons = sorted({self.REASONS[i] for r in loaded for i, s in enumerate(r[4])
+                          if s.lower().startswith("active")})
+        return {"sm_mhz": statistics.median(r[0] for r in loaded),
+                "sm_max_mhz": max(r[1] for r in loaded),
+                "power_w_max": max(r[2] for r in loaded),
+                "samples": len(loaded), "reasons": reasons}
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle timing (baseline / reference arm)
+# ---------------------------------------------------------------------------
+def oracle_sample_flops(w, rows):
+    if w.causal:
+        nvis = [min(int(r) + 1, w.Nk) for r in rows]
+    else:
+        nvis = [w.Nk] * len(rows)
+    return 4.0 * w.d * float(sum(nvis))
+
+
+def time_oracle_rows(w, n_rows, seed_off, bh=0):
+    import oracle
+    from exact_attention_152_b200 import inputs
+    k = inputs.bf16_bits_to_f64(w.head_bits("k", bh))
+    v = inputs.bf16_bits_to_f64(w.head_bits("v", bh))
+    rows = inputs.sample_rows(w.seed + seed_off, bh, w.Nq, n_rows)
+    q = inputs.bf16_bits_to_f64(w.q_rows_bits(bh, rows))
+    t0 = time.perf_counter()
+    oracle.attn_rows(q, rows, k, v, w.scale, w.causal)
+    dt = time.perf_counter() - t0
+    return dt, oracle_sample_flops(w, rows), len(rows)
+
+
+def calibrate_rows(w, seconds):
+    dt, _, n = time_oracle_rows(w, 64, 1000)
+    return max(16, min(w.Nq, int(n * seconds / max(dt, 1e-6))))
+
+
+def cpu_baseline(w, seconds):
+    import oracle
+    n = calibrate_rows(w, seconds)
+    dt, flops, n = time_oracle_rows(w, n, 2000)
+    return {"value": flops / dt / 1e12, "unit": UNIT, "cores": oracle.default_threads(),
+            "kind": "oracle",
+            "sample": f"{n} seeded query rows of head 0 of {w.name} (full key range{', causal' if w.causal else ''}), "
+                      f"fp64, {dt:.1f} s; value = those rows' algorithmic FLOPs / time"}
+
+
+def workload_config(w, n_gpus):
+    qkv_bytes = (w.B * w.H * (w.Nq + 2 * w.Nk) * w.d * 2)
+    return {"workload": w.name, "B": w.B, "H": w.H, "Nq": w.Nq, "Nk": w.Nk, "d": w.d,
+            "causal": w.causal, "scale": w.scale, "seed": w.seed, "per_gpu_problem": True,
+            "global_batch": w.B * n_gpus,
+            "l2": f"inputs {qkv_bytes / 1e6:.0f} MB {'>' if qkv_bytes > L2_BYTES else '<='} "
+                  f"126 MB L2; not flushed between steps",
+            "parallelism": f"independent problem per GPU x{n_gpus}"}
+
+
+def run_reference(args):
+    rank, world, _ = dist_env()
+    from exact_attention_152_b200.workloads import HEADLINE, WORKLOADS
+    if world > 1 and rank != 0:
+        return 0
+    import oracle
+    w = WORKLOADS[args.workload or HEADLINE]
+    budget = 150.0  # seconds for warmup + timed steps together
+    per_step = budget / max(1, args.steps + args.warmup)
+    n = calibrate_rows(w, per_step)
+    for i in range(args.warmup):
+        time_oracle_rows(w, n, 3000 + i)
+    tot_t, tot_f = 0.0, 0.0
+    for i in range(args.steps):
+        dt, fl, n = time_oracle_rows(w, n, 5000 + i)
+        tot_t += dt
+        tot_f += fl
+    value = tot_f / tot_t / 1e12
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": tot_t / args.steps * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": workload_config(w, 1),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": oracle.default_threads(), "kind": "oracle",
+                         "sample": f"each step: {n} seeded query rows of head 0 (full key range), fp64"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ---------------------------------------------------------------------------
+# the CUDA path
+# ---------------------------------------------------------------------------
+def run_ours(args):
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+
+    from exact_attention_152_b200 import binding
+    from exact_attention_152_b200.workloads import HEADLINE, WORKLOADS
+
+    rank, world, local_rank = dist_env()
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+    w = WORKLOADS[args.workload or HEADLINE]
+    peaks = load_peaks()
+
+    # inputs: the workload's seeded BF16 tensors, resident in HBM
+    host = {x: w.tensor_bits(x) for x in "qkv"}
+    q, k, v = (torch.from_numpy(host[x].view(np.int16)).view(torch.bfloat16).to(dev) for x in "qkv")
+    o = torch.empty((w.B, w.H, w.Nq, w.d), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((w.B, w.H, w.Nq), dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    sh = stream.cuda_stream
+    knobs = args.exp_mode is not None or args.threshold is not None
+    thr = 8.0 if args.threshold is None else args.threshold
+    em = 1 if args.exp_mode is None else args.exp_mode
+
+    def launch(qp=q, kp=k, vp=v, op=o, lp=lse):
+        if knobs:
+            rc = binding.attn_fwd_config(qp.data_ptr(), kp.data_ptr(), vp.data_ptr(), op.data_ptr(),
+                                         lp.data_ptr(), w.B, w.H, w.Nq, w.Nk, w.d, w.scale,
+                                         int(w.causal), thr, em, None, sh)
+        else:
+            rc = binding.attn_fwd(qp.data_ptr(), kp.data_ptr(), vp.data_ptr(), op.data_ptr(),
+                                  lp.data_ptr(), w.B, w.H, w.Nq, w.Nk, w.d, w.scale, int(w.causal), sh)
+        binding.check(rc, "attn_fwd")
+
+    # one checked launch before anything is timed
+    launch()
+    binding.check(binding.attn_status_sync(sh), "first launch")
+    for _ in range(args.warmup):
+        launch()
+    binding.check(binding.attn_status_sync(sh), "warm-up")
+    assert bool(torch.isfinite(o.float()).all()), "non-finite output"
+
+    gpu_id = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
+    sampler = ClockSampler(gpu_id)
+    K = args.steps
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(K + 1)]
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    sampler.start()
+    evs[0].record(stream)
+    for i in range(K):
+        launch()
+        evs[i + 1].record(stream)
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    clocks = sampler.stop()
+    binding.check(binding.attn_status_sync(sh), "timed region")
+    total_ms = evs[0].elapsed_time(evs[K])
+    per_launch = [evs[i].elapsed_time(evs[i + 1]) for i in range(K)]
+    kernel_ms = sum(per_launch) / K
+    t = torch.tensor([total_ms, kernel_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    total_ms, kernel_ms = float(t[0]), float(t[1])
+    value = world * w.flops * K / (total_ms / 1e3) / 1e12
+    achieved = w.flops / (kernel_ms / 1e3) / 1e12
+
+    # end to end through the public API: pinned host inputs -> H2D, attn_fwd, D2H
+    hq, hk, hv = (torch.from_numpy(host[x].view(np.int16)).view(torch.bfloat16).pin_memory() for x in "qkv")
+    ho = torch.empty(o.shape, dtype=torch.bfloat16).pin_memory()
+    hl = torch.empty(lse.shape, dtype=torch.float32).pin_memory()
+    qd, kd, vd = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    KE = args.e2e_steps
+
+    def e2e_step():
+        qd.copy_(hq, non_blocking=True)
+        kd.copy_(hk, non_blocking=True)
+        vd.copy_(hv, non_blocking=True)
+        launch(qd, kd, vd, o, lse)
+        ho.copy_(o, non_blocking=True)
+        hl.copy_(lse, non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    e0.record(stream)
+    for _ in range(KE):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    binding.check(binding.attn_status_sync(sh), "e2e region")
+    te = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(te, op=dist.ReduceOp.MAX)
+    e2e_value = world * w.flops * KE / (float(te[0]) / 1e3) / 1e12
+    h2d = sum(x.numel() * x.element_size() for x in (hq, hk, hv))
+    d2h = ho.numel() * ho.element_size() + hl.numel() * hl.element_size()
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(w, args.cpu_seconds)
+
+    if world > 1:
+        dist.destroy_process_group()
+    if rank != 0:
+        return 0
+    peak = peaks["sustained"]
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K,
+        "warmup": args.warmup, "ms_per_step": total_ms / K, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": workload_config(w, world),
+        "pct_of_dense_bf16_spec": 100.0 * value / world / SPEC_DENSE_BF16_TFLOPS,
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": UNIT,
+                     "frac": achieved / peak, "traffic": recorded_traffic(w.name),
+                     "peak_kind": f"bf16_tflops_sustained ({peaks['source']}): back-to-back launches for seconds under the power cap",
+                     "frac_of_burst": achieved / peaks["burst"],
+                     "frac_of_spec_2250": achieved / SPEC_DENSE_BF16_TFLOPS,
+                     "algorithmic_flops_per_launch": w.flops},
+        "cpu_baseline": cpu,
+        "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "steps": KE, "path": "pinned host Q/K/V -> H2D -> attn_fwd (C-ABI) -> D2H of O and LSE"},
+        "gpu_launches": K,
+        "clocks": clocks,
+        "kernel_src_sha": kernel_source_hash(),
+    }
+    if knobs:
+        line["config"]["rescale_threshold"] = thr
+        line["config"]["exp_mode"] = em
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,138 @@
+"""ctypes binding over libattn.so (include/attn.h).
+
+The C functions keep their names and arguments: pointers are Python ints (or
+None), sizes ints, the stream a raw ``cudaStream_t`` handle as an int.  They
+return the library's status code.  ``fwd`` is the one convenience wrapper: it
+allocates O and LSE with torch, passes ``data_ptr()`` and the current stream,
+and raises ``AttnError`` on a non-zero status.  No arithmetic happens here.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+import threading
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libattn.so")
+
+ATTN_OK = 0
+ATTN_ERR_INVALID_ARG = 1
+ATTN_ERR_UNSUPPORTED = 2
+ATTN_ERR_CUDA = 3
+ATTN_ERR_TIMEOUT = 4
+
+EXP_MUFU, EXP_SPLIT, EXP_POLY = 0, 1, 2
+
+_lock = threading.Lock()
+_lib = None
+
+_P = ctypes.c_void_p
+_I = ctypes.c_int
+
+
+def lib() -> ctypes.CDLL:
+    """Load libattn.so once; raise ImportError if it has not been built."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            if not os.path.exists(LIB_PATH):
+                raise ImportError(f"{LIB_PATH} is missing: build it with "
+                                  "`python -m exact_attention_152_b200.build` (there is no fallback)")
+            l = ctypes.CDLL(LIB_PATH)
+            l.attn_fwd.argtypes = [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, ctypes.c_float, _I, _P]
+            l.attn_fwd.restype = _I
+            l.attn_fwd_config.argtypes = [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, ctypes.c_float, _I,
+                                          ctypes.c_float, _I, _P, _P]
+            l.attn_fwd_config.restype = _I
+            l.attn_status_sync.argtypes = [_P]
+            l.attn_status_sync.restype = _I
+            l.attn_status_string.argtypes = [_I]
+            l.attn_status_string.restype = ctypes.c_char_p
+            l.attn_last_error.argtypes = []
+            l.attn_last_error.restype = ctypes.c_char_p
+            l.attn_selftest_timeout.argtypes = [ctypes.c_uint, _P]
+            l.attn_selftest_timeout.restype = _I
+            _lib = l
+    return _lib
+
+
+def attn_fwd(q, k, v, o, lse, B, H, Nq, Nk, d, scale, causal, stream) -> int:
+    return lib().attn_fwd(q, k, v, o, lse, B, H, Nq, Nk, d, scale, causal, stream)
+
+
+def attn_fwd_config(q, k, v, o, lse, B, H, Nq, Nk, d, scale, causal, rescale_threshold,
+                    exp_mode, rescale_count, stream) -> int:
+    return lib().attn_fwd_config(q, k, v, o, lse, B, H, Nq, Nk, d, scale, causal,
+                                 rescale_threshold, exp_mode, rescale_count, stream)
+
+
+def attn_status_sync(stream) -> int:
+    return lib().attn_status_sync(stream)
+
+
+def attn_status_string(code: int) -> str:
+    return lib().attn_status_string(code).decode()
+
+
+def attn_last_error() -> str:
+    return lib().attn_last_error().decode()
+
+
+def attn_selftest_timeout(timeout_us: int, stream) -> int:
+    return lib().attn_selftest_timeout(timeout_us, stream)
+
+
+class AttnError(RuntimeError):
+    def __init__(self, code: int, where: str):
+        msg = f"{where}: {attn_status_string(code)} ({code})"
+        if code == ATTN_ERR_CUDA:
+            msg += f": {attn_last_error()}"
+        super().__init__(msg)
+        self.code = code
+
+
+def check(code: int, where: str = "attn") -> None:
+    if code != ATTN_OK:
+        raise AttnError(code, where)
+
+
+def fwd(q, k, v, causal: bool = False, scale: float | None = None, *, out=None, lse=None,
+        return_lse: bool = True, rescale_threshold: float | None = None,
+        exp_mode: int | None = None, rescale_count=None):
+    """O (and LSE) for BF16 CUDA tensors q [B,H,Nq,d], k/v [B,H,Nk,d].
+
+    scale defaults to 1/sqrt(d).  Runs on torch's current stream; returns
+    (o, lse) or o.  Raises AttnError on any non-zero status.
+    """
+    import torch
+
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        if not isinstance(t, torch.Tensor) or t.dtype != torch.bfloat16 or not t.is_cuda:
+            raise TypeError(f"{name} must be a bfloat16 CUDA tensor")
+        if t.dim() != 4 or not t.is_contiguous():
+            raise ValueError(f"{name} must be contiguous [B, H, N, d]")
+    B, H, Nq, d = q.shape
+    Nk = k.shape[2]
+    if tuple(k.shape) != (B, H, Nk, d) or tuple(v.shape) != (B, H, Nk, d):
+        raise ValueError("k and v must be [B, H, Nk, d] matching q")
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if out is None:
+        out = torch.empty((B, H, Nq, d), dtype=torch.bfloat16, device=q.device)
+    if return_lse and lse is None:
+        lse = torch.empty((B, H, Nq), dtype=torch.float32, device=q.device)
+    stream = torch.cuda.current_stream(q.device).cuda_stream
+    lse_ptr = lse.data_ptr() if lse is not None else None
+    if rescale_threshold is None and exp_mode is None and rescale_count is None:
+        rc = attn_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse_ptr,
+                      B, H, Nq, Nk, d, float(scale), int(bool(causal)), stream)
+    else:
+        rc = attn_fwd_config(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse_ptr,
+                             B, H, Nq, Nk, d, float(scale), int(bool(causal)),
+                             8.0 if rescale_threshold is None else float(rescale_threshold),
+                             EXP_SPLIT if exp_mode is None else int(exp_mode),
+                             rescale_count.data_ptr() if rescale_count is not None else None,
+                             stream)
+    check(rc, "attn_fwd")
+    return (out, lse) if return_lse else out

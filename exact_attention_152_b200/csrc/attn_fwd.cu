@@ -1,0 +1,727 @@
+// Exact attention forward for B200 (sm_100a): TMA producer, tcgen05 MMAs with
+// accumulators in Tensor Memory, online softmax with adaptive rescaling and a
+// MUFU / FMA-pipe split of exp2, causal tile skipping.  Plus the C-ABI entry
+// points declared in include/attn.h.
+//
+// Method (what the pages describe; they print no formulas or code):
+//  * Tiling through on-chip memory so the Nq x Nk score matrix never reaches
+//    device memory, with a running per-row max and sum (online softmax):
+//    Flash Attention glossary (jisaku.com), sections "タイリングによるSRAMの活用"
+//    and "オンライン・ソフトマックスと再計算"; FlashAttention 4 page
+//    (ja.linux-konsole.com), section "なぜアテンションカーネルがまだLLMのコストを
+//    支配しているのか".
+//  * Warp roles -- load, tensor-core MMA, softmax, rescale, store -- each with
+//    its own asynchronous pipeline: FlashAttention 4 page, section
+//    "FlashAttention 4の新機能".
+//  * exp2 partly evaluated as a cubic polynomial on the FMA pipe to relieve the
+//    few SFUs: same page, section "CUDAコアによるソフトウェアの指数演算";
+//    FlashAttention-4 deep dive (sns.style), section 二.
+//  * Rescaling only when the new max is sufficiently larger than the old one:
+//    FlashAttention 4 page, section "よりスマートなオンラインソフトマックス再スケーリング".
+//  * Fully asynchronous MMA with Tensor Memory: FlashAttention-4 deep dive,
+//    section 二.
+//
+// Design (this library's, for sm_100a):
+//  * One CTA owns two 128-row query tiles of one (b, h) -- 256 rows -- and
+//    streams the head's K/V tiles (128 keys each) through a ring of shared
+//    memory stages filled by TMA.  Q, K and V are read through 3-D tensor maps
+//    [B*H, N, d] so out-of-range rows of one head read as zeros, never as the
+//    next head's data.
+//  * Warps 0-3 / 4-7: softmax, correction and epilogue of query tile 0 / 1
+//    (one thread = one query row = one TMEM lane).  Warp 8: TMA producer.
+//    Warp 9: TMEM allocation and the single MMA-issuing thread.
+//  * Tensor Memory (512 columns): S0 [0,128), S1 [128,256), O0 and O1 after
+//    column 256.  P (BF16) overwrites the first 64 columns of its S tile and is
+//    the A operand of O += P V straight from TMEM, so P never touches shared
+//    memory.
+//  * The MMA thread issues, per KV tile j:  O0 += P0 V_{j-1};  S0 = Q0 K_j^T;
+//    O1 += P1 V_{j-1};  S1 = Q1 K_j^T.  The commit that announces S_t(j) also
+//    covers O_t += P_t V_{j-1}, so when a softmax warp sees S_t(j) its O_t is
+//    final up to tile j-1 and it can rescale O_t in place without another wait.
+//  * Every wait is bounded (see sm100.cuh); a timeout sets the per-device
+//    status word and the CTA leaves its loops and exits cleanly.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstdint>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <string>
+
+#include "attn.h"
+#include "exp2.cuh"
+#include "sm100.cuh"
+#include "tmap.h"
+
+namespace eab {
+
+constexpr int kBlockM = 128;  // query rows per tile  (= TMEM lanes)
+constexpr int kBlockN = 128;  // keys per KV tile
+constexpr int kRowsPerCta = 2 * kBlockM;
+constexpr int kWarpLoad = 8;
+constexpr int kWarpMma = 9;
+constexpr int kNumThreads = 320;
+constexpr uint32_t kTmemCols = 512;
+constexpr uint64_t kWaitTimeoutNs = 2000000000ull;  // 2 s per pipeline wait
+constexpr float kDefaultThreshold = 8.0f;           // powers of two
+constexpr int kDefaultPoly16 = 4;                   // exp2 columns (of 16) on the FMA pipe
+constexpr float kLn2 = 0.6931471805599453f;
+constexpr float kLog2e = 1.4426950408889634f;
+
+enum : unsigned int { kStatusTimeout = 1u };
+
+// Per-device status word (each device holds its own copy of module globals).
+__device__ unsigned int g_status;
+
+template <int D>
+struct Cfg {
+  static_assert(D == 64 || D == 128, "head dim");
+  static constexpr int kBoxes = D / 64;             // 128-byte swizzle boxes across d
+  static constexpr int kBoxBytes = kBlockM * 128;   // 128 rows x 64 bf16
+  static constexpr int kTileBytes = kBoxes * kBoxBytes;
+  static constexpr int kStages = D == 128 ? 4 : 8;  // K/V ring depth
+  static constexpr int kOffQ = 0;
+  static constexpr int kOffKV = 2 * kTileBytes;
+  static constexpr int kOffBar = kOffKV + kStages * kTileBytes;
+  static constexpr int kNumBars = 2 + 2 * kStages + 2 + 2 + 2 + 1;
+  static constexpr int kOffMisc = kOffBar + kNumBars * 8;
+  static constexpr int kSmemBytes = kOffMisc + 16 + 1024;  // + slack for 1 KiB alignment
+  static constexpr uint32_t kTmemO = 256;
+};
+
+struct FwdParams {
+  float* lse;
+  unsigned long long* rescale_count;
+  uint64_t timeout_ns;
+  int Nq, Nk, BH, n_qblocks;
+  float scale_log2;  // scale * log2(e)
+  float tau;         // rescale threshold, powers of two
+};
+
+template <int POLY16>
+__device__ __forceinline__ float ex2_split(float x, int col) {
+  if ((col & 15) < POLY16) return ex2_poly(x);
+  return ex2_mufu(x);
+}
+
+// ---------------------------------------------------------------------------
+// Shared-memory / barrier map of one CTA
+// ---------------------------------------------------------------------------
+template <int D>
+struct Smem {
+  uint8_t* base;
+  uint32_t sbase;
+  __device__ __forceinline__ uint32_t q(int t) const { return sbase + Cfg<D>::kOffQ + t * Cfg<D>::kTileBytes; }
+  __device__ __forceinline__ uint32_t kv(int s) const { return sbase + Cfg<D>::kOffKV + s * Cfg<D>::kTileBytes; }
+  __device__ __forceinline__ uint32_t bar(int i) const { return sbase + Cfg<D>::kOffBar + 8 * i; }
+  __device__ __forceinline__ uint32_t q_full(int t) const { return bar(t); }
+  __device__ __forceinline__ uint32_t kv_full(int s) const { return bar(2 + s); }
+  __device__ __forceinline__ uint32_t kv_empty(int s) const { return bar(2 + Cfg<D>::kStages + s); }
+  __device__ __forceinline__ uint32_t s_full(int t) const { return bar(2 + 2 * Cfg<D>::kStages + t); }
+  __device__ __forceinline__ uint32_t p_full(int t) const { return bar(4 + 2 * Cfg<D>::kStages + t); }
+  __device__ __forceinline__ uint32_t o_full(int t) const { return bar(6 + 2 * Cfg<D>::kStages + t); }
+  __device__ __forceinline__ uint32_t mma_done() const { return bar(8 + 2 * Cfg<D>::kStages); }
+  __device__ __forceinline__ uint32_t* tmem_slot() const {
+    return reinterpret_cast<uint32_t*>(base + Cfg<D>::kOffMisc);
+  }
+};
+
+// Warp-uniform bounded wait: every lane waits, and the warp agrees on the
+// outcome so warp-collective tcgen05 instructions are never split.
+__device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, uint64_t timeout_ns) {
+  const bool ok = mbar_wait(bar, parity, timeout_ns);
+  return __all_sync(0xffffffffu, ok);
+}
+
+// ---------------------------------------------------------------------------
+// Producer: one thread, TMA loads of Q0, K0, Q1, V0, K1, V1, ...
+// ---------------------------------------------------------------------------
+template <int D>
+__device__ __forceinline__ void producer_role(const Smem<D>& sm, const CUtensorMap* tm_q,
+                                              const CUtensorMap* tm_k, const CUtensorMap* tm_v,
+                                              int bh, int qb, int n_kv, uint64_t timeout) {
+  using C = Cfg<D>;
+  uint32_t it = 0;
+  auto load_q = [&](int t) {
+    mbar_arrive_expect_tx(sm.q_full(t), C::kTileBytes);
+#pragma unroll
+    for (int b = 0; b < C::kBoxes; ++b)
+      tma_load_3d(sm.q(t) + b * C::kBoxBytes, tm_q, b * 64, qb * kRowsPerCta + t * kBlockM, bh,
+                  sm.q_full(t));
+  };
+  auto load_kv = [&](const CUtensorMap* tm, int j) -> bool {
+    const uint32_t slot = it % C::kStages;
+    const uint32_t phase = (it / C::kStages) & 1u;
+    if (!mbar_wait(sm.kv_empty(slot), phase ^ 1u, timeout)) return false;
+    mbar_arrive_expect_tx(sm.kv_full(slot), C::kTileBytes);
+#pragma unroll
+    for (int b = 0; b < C::kBoxes; ++b)
+      tma_load_3d(sm.kv(slot) + b * C::kBoxBytes, tm, b * 64, j * kBlockN, bh, sm.kv_full(slot));
+    ++it;
+    return true;
+  };
+
+  load_q(0);
+  bool ok = load_kv(tm_k, 0);
+  load_q(1);
+  ok = ok && load_kv(tm_v, 0);
+  for (int j = 1; ok && j < n_kv; ++j) ok = load_kv(tm_k, j) && load_kv(tm_v, j);
+
+  // Never leave the CTA with a copy in flight: wait for the latest fill of
+  // every slot and for both Q tiles (immediate on the normal path).
+  const uint32_t first = it > (uint32_t)C::kStages ? it - C::kStages : 0u;
+  for (uint32_t i = first; i < it; ++i) mbar_wait(sm.kv_full(i % C::kStages), (i / C::kStages) & 1u, timeout);
+  mbar_wait(sm.q_full(0), 0, timeout);
+  mbar_wait(sm.q_full(1), 0, timeout);
+  if (!ok) atomicOr(&g_status, kStatusTimeout);
+}
+
+// ---------------------------------------------------------------------------
+// MMA issuer: one thread.
+// ---------------------------------------------------------------------------
+template <int D>
+__device__ __forceinline__ void mma_role(const Smem<D>& sm, uint32_t tmem, int n_kv,
+                                         uint64_t timeout) {
+  using C = Cfg<D>;
+  constexpr uint32_t idesc_s = idesc_bf16_f32(kBlockM, kBlockN, false, false);
+  constexpr uint32_t idesc_o = idesc_bf16_f32(kBlockM, D, false, true);
+  uint32_t it = 0;
+
+  auto wait_kv = [&](uint32_t& slot) -> bool {
+    slot = it % C::kStages;
+    const uint32_t phase = (it / C::kStages) & 1u;
+    ++it;
+    return mbar_wait(sm.kv_full(slot), phase, timeout);
+  };
+  // S_t = Q_t K^T : M=128 queries, N=128 keys, K=d in steps of 16 (32 bytes of
+  // the 128-byte swizzled row; a new box every 64 columns of d).
+  auto mma_s = [&](int t, uint32_t slot) {
+    const uint32_t d_tmem = tmem + t * kBlockM;
+#pragma unroll
+    for (int kk = 0; kk < D / 16; ++kk) {
+      const uint32_t off = (kk >> 2) * C::kBoxBytes + (kk & 3) * 32;
+      mma_ss(d_tmem, sdesc_sw128(sm.q(t) + off, 16, 1024), sdesc_sw128(sm.kv(slot) + off, 16, 1024),
+             idesc_s, kk > 0 ? 1u : 0u);
+    }
+  };
+  // O_t += P_t V : M=128 queries, N=d, K=128 keys in steps of 16.  P (bf16,
+  // two per column) sits in the first 64 TMEM columns of S_t.  V is MN-major:
+  // 16 keys = 16 rows of 128 bytes = 2048 bytes; the 64-wide d boxes are
+  // kBoxBytes apart (LBO), 8-row groups 1024 bytes apart (SBO).
+  auto mma_o = [&](int t, uint32_t slot, bool acc) {
+    const uint32_t d_tmem = tmem + C::kTmemO + t * D;
+    const uint32_t a_tmem = tmem + t * kBlockM;
+#pragma unroll
+    for (int kk = 0; kk < kBlockN / 16; ++kk)
+      mma_ts(d_tmem, a_tmem + kk * 8, sdesc_sw128(sm.kv(slot) + kk * 2048, C::kBoxBytes, 1024),
+             idesc_o, (acc || kk > 0) ? 1u : 0u);
+  };
+
+  uint32_t sK = 0, sV = 0;
+  bool ok = mbar_wait(sm.q_full(0), 0, timeout) && wait_kv(sK);
+  if (ok) {
+    tc_fence_after();
+    mma_s(0, sK);
+    tc_commit(sm.s_full(0));
+    ok = mbar_wait(sm.q_full(1), 0, timeout);
+  }
+  if (ok) {
+    tc_fence_after();
+    mma_s(1, sK);
+    tc_commit(sm.s_full(1));
+    tc_commit(sm.kv_empty(sK));
+  }
+  for (int j = 1; ok && j < n_kv; ++j) {
+    const uint32_t par = (j - 1) & 1;
+    ok = wait_kv(sV) && mbar_wait(sm.p_full(0), par, timeout);
+    if (!ok) break;
+    tc_fence_after();
+    mma_o(0, sV, j > 1);
+    ok = wait_kv(sK);
+    if (!ok) break;
+    tc_fence_after();
+    mma_s(0, sK);
+    tc_commit(sm.s_full(0));
+    ok = mbar_wait(sm.p_full(1), par, timeout);
+    if (!ok) break;
+    tc_fence_after();
+    mma_o(1, sV, j > 1);
+    tc_commit(sm.kv_empty(sV));
+    mma_s(1, sK);
+    tc_commit(sm.s_full(1));
+    tc_commit(sm.kv_empty(sK));
+  }
+  if (ok) {
+    const uint32_t par = (n_kv - 1) & 1;
+    ok = wait_kv(sV) && mbar_wait(sm.p_full(0), par, timeout);
+    if (ok) {
+      tc_fence_after();
+      mma_o(0, sV, n_kv > 1);
+      tc_commit(sm.o_full(0));
+      ok = mbar_wait(sm.p_full(1), par, timeout);
+    }
+    if (ok) {
+      tc_fence_after();
+      mma_o(1, sV, n_kv > 1);
+      tc_commit(sm.o_full(1));
+      tc_commit(sm.kv_empty(sV));
+    }
+  }
+  // Everything issued must be finished before TMEM is released.
+  tc_commit(sm.mma_done());
+  mbar_wait(sm.mma_done(), 0, timeout);
+  if (!ok) atomicOr(&g_status, kStatusTimeout);
+}
+
+// ---------------------------------------------------------------------------
+// Softmax + correction + epilogue for one query tile: 4 warps, 1 row/thread.
+// ---------------------------------------------------------------------------
+template <int D, bool CAUSAL, int POLY16>
+__device__ __forceinline__ void softmax_role(const Smem<D>& sm, uint32_t tmem,
+                                             const CUtensorMap* tm_o, const FwdParams& prm,
+                                             int bh, int qb, int n_kv) {
+  using C = Cfg<D>;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int t = warp >> 2;   // query tile of this CTA
+  const int q4 = warp & 3;   // TMEM lane quarter this warp may access
+  const int r = q4 * 32 + lane;
+  const int tile_row0 = qb * kRowsPerCta + t * kBlockM;
+  const int row = tile_row0 + r;
+  const uint32_t lane_off = static_cast<uint32_t>(q4 * 32) << 16;
+  const uint32_t tS = tmem + lane_off + t * kBlockM;
+  const uint32_t tO = tmem + lane_off + C::kTmemO + t * D;
+  const uint64_t timeout = prm.timeout_ns;
+
+  // scale <= 0: apply it first, then run with an effective scale of 1 (the
+  // fast path folds a positive scale into one FFMA per score).
+  const bool prescale = !(prm.scale_log2 > 0.0f);
+  const float sl = prescale ? 1.0f : prm.scale_log2;
+  float m_run = -INFINITY;  // running reference max, log2 units of scaled scores
+  float l_run = 0.0f;       // running sum of 2^(score - m_run)
+  bool ok = true;
+
+  for (int j = 0; j < n_kv; ++j) {
+    if (!warp_wait(sm.s_full(t), j & 1, timeout)) { ok = false; break; }
+    tc_fence_after();
+    uint32_t s[4][32];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) tmem_ld32(tS + q * 32, s[q]);
+    tmem_ld_wait();
+#pragma unroll
+    for (int q = 0; q < 4; ++q) reg_fence32(s[q]);
+    float x[kBlockN];
+#pragma unroll
+    for (int c = 0; c < kBlockN; ++c) x[c] = __uint_as_float(s[c >> 5][c & 31]);
+    if (prescale) {
+#pragma unroll
+      for (int c = 0; c < kBlockN; ++c) x[c] *= prm.scale_log2;
+    }
+    // mask: key tail, and the causal diagonal (only tiles that reach past the
+    // tile's first row need it).
+    const int kv0 = j * kBlockN;
+    if (kv0 + kBlockN > prm.Nk || (CAUSAL && kv0 + kBlockN - 1 > tile_row0)) {
+#pragma unroll
+      for (int c = 0; c < kBlockN; ++c) {
+        const int key = kv0 + c;
+        if (key >= prm.Nk || (CAUSAL && key > row)) x[c] = -INFINITY;
+      }
+    }
+    float mx[8];
+#pragma unroll
+    for (int c = 0; c < 8; ++c) mx[c] = x[c];
+#pragma unroll
+    for (int c = 8; c < kBlockN; ++c) mx[c & 7] = fmaxf(mx[c & 7], x[c]);
+#pragma unroll
+    for (int w = 4; w >= 1; w >>= 1)
+#pragma unroll
+      for (int c = 0; c < w; ++c) mx[c] = fmaxf(mx[c], mx[c + w]);
+    const float m_tile = mx[0] * sl;
+
+    // adaptive rescaling: move the reference only on a jump beyond tau
+    const bool resc = m_tile > m_run + prm.tau;
+    float alpha = 1.0f;
+    if (resc) {
+      alpha = ex2_mufu(m_run - m_tile);  // 0 on the first tile
+      m_run = m_tile;
+    }
+    l_run *= alpha;
+
+    const float neg_m = (m_run == -INFINITY) ? 0.0f : -m_run;
+    float sum[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+    uint32_t p[2][32];
+#pragma unroll
+    for (int c = 0; c < kBlockN; c += 2) {
+      const float a = ex2_split<POLY16>(fmaf(x[c], sl, neg_m), c);
+      const float b = ex2_split<POLY16>(fmaf(x[c + 1], sl, neg_m), c + 1);
+      sum[(c >> 1) & 3] += a + b;
+      p[c >> 6][(c & 63) >> 1] = pack_bf16x2(a, b);
+    }
+    l_run += (sum[0] + sum[1]) + (sum[2] + sum[3]);
+    tmem_st32(tS, p[0]);
+    tmem_st32(tS + 32, p[1]);
+    // Correction: rescale this row's O accumulator (already final up to tile
+    // j-1, see the MMA order) by alpha before O += P V_j is issued.  Done after
+    // the P stores so the 128 score registers are dead by now.
+    if (j > 0 && __any_sync(0xffffffffu, resc)) {
+      if (prm.rescale_count) {
+        const unsigned n = __popc(__ballot_sync(0xffffffffu, resc));
+        if (lane == 0) atomicAdd(prm.rescale_count, static_cast<unsigned long long>(n));
+      }
+#pragma unroll
+      for (int cc = 0; cc < D / 32; ++cc) {
+        uint32_t o[32];
+        tmem_ld32(tO + cc * 32, o);
+        tmem_ld_wait();
+        reg_fence32(o);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+        tmem_st32(tO + cc * 32, o);
+      }
+    }
+    tmem_st_wait();
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(sm.p_full(t));
+  }
+
+  if (ok) ok = warp_wait(sm.o_full(t), 0, timeout);
+  if (ok) {
+    tc_fence_after();
+    // Epilogue: O / l -> BF16 -> this tile's Q buffer (its last reader, the
+    // final S MMA, finished before the last O MMA) in the 128-byte swizzled
+    // layout the O tensor map expects -> one TMA store per warp (32 rows).
+    const float inv_l = l_run > 0.0f ? 1.0f / l_run : 0.0f;
+    uint8_t* sOt = sm.base + C::kOffQ + t * C::kTileBytes;
+#pragma unroll
+    for (int cc = 0; cc < D / 32; ++cc) {
+      uint32_t o[32];
+      tmem_ld32(tO + cc * 32, o);
+      tmem_ld_wait();
+      reg_fence32(o);
+      uint32_t w[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i)
+        w[i] = pack_bf16x2(__uint_as_float(o[2 * i]) * inv_l, __uint_as_float(o[2 * i + 1]) * inv_l);
+      uint8_t* rowp = sOt + (cc >> 1) * C::kBoxBytes + r * 128;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int chunk = (((cc & 1) * 4) + i) ^ (r & 7);
+        *reinterpret_cast<uint4*>(rowp + chunk * 16) = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
+      }
+    }
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0 && tile_row0 + q4 * 32 < prm.Nq) {
+#pragma unroll
+      for (int b = 0; b < C::kBoxes; ++b)
+        tma_store_3d(tm_o, smem_u32(sOt + b * C::kBoxBytes + q4 * 32 * 128), b * 64, tile_row0 + q4 * 32, bh);
+      bulk_commit_group();
+      bulk_wait_group_read0();
+    }
+    if (prm.lse != nullptr && row < prm.Nq) {
+      const float m_use = (m_run == -INFINITY) ? 0.0f : m_run;
+      prm.lse[static_cast<size_t>(bh) * prm.Nq + row] = (m_use + log2f(l_run)) * kLn2;
+    }
+  }
+  if (!ok && lane == 0) atomicOr(&g_status, kStatusTimeout);
+}
+
+// ---------------------------------------------------------------------------
+// The kernel.  Grid: one CTA per (b*h, 256-row query block).
+// ---------------------------------------------------------------------------
+template <int D, bool CAUSAL, int POLY16>
+__global__ void __launch_bounds__(kNumThreads, 1)
+attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
+                const __grid_constant__ FwdParams prm) {
+  using C = Cfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  Smem<D> sm;
+  {
+    const uint32_t raw = smem_u32(smem_raw);
+    const uint32_t pad = (1024u - (raw & 1023u)) & 1023u;
+    sm.base = smem_raw + pad;
+    sm.sbase = raw + pad;
+  }
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  // Tile order.  Non-causal: head-major, so the CTAs resident at one time share
+  // a few heads' K/V in L2.  Causal: heaviest query blocks first across all
+  // heads, so the short blocks fill the tail.
+  const int tile = blockIdx.x;
+  int bh, qb;
+  if (CAUSAL) {
+    qb = prm.n_qblocks - 1 - tile / prm.BH;
+    bh = tile % prm.BH;
+  } else {
+    bh = tile / prm.n_qblocks;
+    qb = tile % prm.n_qblocks;
+  }
+  int n_kv = (prm.Nk + kBlockN - 1) / kBlockN;
+  if (CAUSAL) n_kv = min(n_kv, (qb + 1) * (kRowsPerCta / kBlockN));
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < C::kNumBars; ++i) {
+      const uint32_t b = sm.bar(i);
+      // p_full: one arrival per softmax warp of the tile; everything else: one.
+      mbar_init(b, (b == sm.p_full(0) || b == sm.p_full(1)) ? 4u : 1u);
+    }
+    fence_barrier_init();
+    fence_proxy_async_smem();
+  }
+  if (warp == kWarpLoad && lane == 0) {
+    tma_prefetch_desc(&tm_q);
+    tma_prefetch_desc(&tm_k);
+    tma_prefetch_desc(&tm_v);
+    tma_prefetch_desc(&tm_o);
+  }
+  if (warp == kWarpMma) {
+    tmem_alloc(smem_u32(sm.tmem_slot()), kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *sm.tmem_slot();
+
+  if (warp == kWarpLoad) {
+    if (lane == 0) producer_role<D>(sm, &tm_q, &tm_k, &tm_v, bh, qb, n_kv, prm.timeout_ns);
+    __syncwarp();
+  } else if (warp == kWarpMma) {
+    if (lane == 0) mma_role<D>(sm, tmem, n_kv, prm.timeout_ns);
+    __syncwarp();
+  } else {
+    softmax_role<D, CAUSAL, POLY16>(sm, tmem, &tm_o, prm, bh, qb, n_kv);
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == kWarpMma) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+// Nk == 0: no visible key -> O = 0 (memset by the host), LSE = -inf.
+__global__ void fill_neg_inf_kernel(float* p, size_t n) {
+  for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < n;
+       i += static_cast<size_t>(gridDim.x) * blockDim.x)
+    p[i] = -INFINITY;
+}
+
+// One thread waits on a barrier that nothing signals; the bounded wait gives
+// up and records a timeout.  Exercises the failure path without any fault.
+__global__ void selftest_timeout_kernel(uint64_t timeout_ns) {
+  __shared__ __align__(8) uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(smem_u32(&bar), 1);
+    fence_barrier_init();
+    if (!mbar_wait(smem_u32(&bar), 0, timeout_ns)) atomicOr(&g_status, kStatusTimeout);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Host side
+// ---------------------------------------------------------------------------
+thread_local std::string t_last_error;
+
+int cuda_fail(cudaError_t e, const char* what) {
+  t_last_error = std::string(what) + ": " + cudaGetErrorString(e);
+  return ATTN_ERR_CUDA;
+}
+
+constexpr int kMaxDevices = 64;
+struct DeviceInfo {
+  bool probed = false;
+  bool supported = false;
+};
+std::mutex g_dev_mu;
+DeviceInfo g_dev[kMaxDevices];
+
+template <int D, bool CAUSAL, int POLY16>
+int launch_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+               const CUtensorMap& to, const FwdParams& prm, cudaStream_t stream) {
+  auto kern = attn_fwd_kernel<D, CAUSAL, POLY16>;
+  static std::once_flag attr_once[kMaxDevices];
+  static cudaError_t attr_err[kMaxDevices];
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  std::call_once(attr_once[dev], [&] {
+    attr_err[dev] = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         Cfg<D>::kSmemBytes);
+  });
+  if (attr_err[dev] != cudaSuccess) return cuda_fail(attr_err[dev], "cudaFuncSetAttribute");
+  const unsigned grid = static_cast<unsigned>(prm.BH) * static_cast<unsigned>(prm.n_qblocks);
+  kern<<<grid, kNumThreads, Cfg<D>::kSmemBytes, stream>>>(tq, tk, tv, to, prm);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "attn_fwd_kernel launch");
+  return ATTN_OK;
+}
+
+template <int D, bool CAUSAL>
+int dispatch_exp(int exp_mode, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                 const CUtensorMap& to, const FwdParams& prm, cudaStream_t stream) {
+  switch (exp_mode) {
+    case 0: return launch_fwd<D, CAUSAL, 0>(tq, tk, tv, to, prm, stream);
+    case 1: return launch_fwd<D, CAUSAL, kDefaultPoly16>(tq, tk, tv, to, prm, stream);
+    default: return launch_fwd<D, CAUSAL, 16>(tq, tk, tv, to, prm, stream);
+  }
+}
+
+bool ranges_overlap(const void* a, size_t na, const void* b, size_t nb) {
+  if (!a || !b || na == 0 || nb == 0) return false;
+  const uintptr_t a0 = reinterpret_cast<uintptr_t>(a), b0 = reinterpret_cast<uintptr_t>(b);
+  return a0 < b0 + nb && b0 < a0 + na;
+}
+
+int check_device() {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= kMaxDevices) return ATTN_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lk(g_dev_mu);
+  DeviceInfo& di = g_dev[dev];
+  if (!di.probed) {
+    int major = 0, minor = 0;
+    e = cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceGetAttribute");
+    e = cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceGetAttribute");
+    di.supported = (major == 10 && minor == 0);
+    di.probed = true;
+  }
+  return di.supported ? ATTN_OK : ATTN_ERR_UNSUPPORTED;
+}
+
+int fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
+             int Nq, int Nk, int d, float scale, int causal, float tau, int exp_mode,
+             unsigned long long* rescale_count, cudaStream_t stream) {
+  if (B < 0 || H < 0 || Nq < 0 || Nk < 0) return ATTN_ERR_INVALID_ARG;
+  if (!std::isfinite(scale)) return ATTN_ERR_INVALID_ARG;
+  if (causal != 0 && causal != 1) return ATTN_ERR_INVALID_ARG;
+  if (!(tau >= 0.0f && tau <= 64.0f)) return ATTN_ERR_UNSUPPORTED;
+  if (exp_mode < 0 || exp_mode > 2) return ATTN_ERR_UNSUPPORTED;
+  if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
+  if (causal && Nq != Nk) return ATTN_ERR_UNSUPPORTED;
+  const long long BH = static_cast<long long>(B) * H;
+  if (BH == 0 || Nq == 0) return ATTN_OK;  // nothing to compute
+  if (BH > 0x7fffffffLL) return ATTN_ERR_INVALID_ARG;
+  if (!o || (Nk > 0 && (!q || !k || !v))) return ATTN_ERR_INVALID_ARG;
+  auto misaligned = [](const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) != 0; };
+  if (misaligned(q, 16) || misaligned(k, 16) || misaligned(v, 16) || misaligned(o, 16) ||
+      misaligned(lse, 4) || misaligned(rescale_count, 8))
+    return ATTN_ERR_INVALID_ARG;
+  const size_t o_bytes = static_cast<size_t>(BH) * Nq * d * 2;
+  const size_t kv_bytes = static_cast<size_t>(BH) * Nk * d * 2;
+  const size_t lse_bytes = lse ? static_cast<size_t>(BH) * Nq * 4 : 0;
+  if (ranges_overlap(o, o_bytes, q, o_bytes) || ranges_overlap(o, o_bytes, k, kv_bytes) ||
+      ranges_overlap(o, o_bytes, v, kv_bytes) || ranges_overlap(lse, lse_bytes, q, o_bytes) ||
+      ranges_overlap(lse, lse_bytes, k, kv_bytes) || ranges_overlap(lse, lse_bytes, v, kv_bytes) ||
+      ranges_overlap(lse, lse_bytes, o, o_bytes))
+    return ATTN_ERR_INVALID_ARG;
+  const long long n_qblocks = (Nq + kRowsPerCta - 1) / kRowsPerCta;
+  if (n_qblocks * BH > 0x7fffffffLL) return ATTN_ERR_INVALID_ARG;
+  int rc = check_device();
+  if (rc != ATTN_OK) return rc;
+
+  if (Nk == 0) {
+    cudaError_t e = cudaMemsetAsync(o, 0, o_bytes, stream);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync");
+    if (lse) {
+      const size_t n = static_cast<size_t>(BH) * Nq;
+      const unsigned blocks = static_cast<unsigned>(std::min<size_t>((n + 255) / 256, 4096));
+      fill_neg_inf_kernel<<<blocks, 256, 0, stream>>>(lse, n);
+      e = cudaGetLastError();
+      if (e != cudaSuccess) return cuda_fail(e, "fill_neg_inf_kernel launch");
+    }
+    return ATTN_OK;
+  }
+
+  CUtensorMap tq, tk, tv, to;
+  const int bh = static_cast<int>(BH);
+  if (!make_tmap_bf16_3d(&tq, q, bh, Nq, d, kBlockM, &t_last_error) ||
+      !make_tmap_bf16_3d(&tk, k, bh, Nk, d, kBlockN, &t_last_error) ||
+      !make_tmap_bf16_3d(&tv, v, bh, Nk, d, kBlockN, &t_last_error) ||
+      !make_tmap_bf16_3d(&to, o, bh, Nq, d, 32, &t_last_error))
+    return ATTN_ERR_CUDA;
+
+  FwdParams prm;
+  prm.lse = lse;
+  prm.rescale_count = rescale_count;
+  prm.timeout_ns = kWaitTimeoutNs;
+  prm.Nq = Nq;
+  prm.Nk = Nk;
+  prm.BH = static_cast<int>(BH);
+  prm.n_qblocks = static_cast<int>(n_qblocks);
+  prm.scale_log2 = scale * kLog2e;
+  prm.tau = tau;
+
+  if (d == 128) {
+    return causal ? dispatch_exp<128, true>(exp_mode, tq, tk, tv, to, prm, stream)
+                  : dispatch_exp<128, false>(exp_mode, tq, tk, tv, to, prm, stream);
+  }
+  return causal ? dispatch_exp<64, true>(exp_mode, tq, tk, tv, to, prm, stream)
+                : dispatch_exp<64, false>(exp_mode, tq, tk, tv, to, prm, stream);
+}
+
+}  // namespace eab
+
+extern "C" {
+
+int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
+             int Nq, int Nk, int d, float scale, int causal, cudaStream_t stream) {
+  return eab::fwd_impl(q, k, v, o, lse, B, H, Nq, Nk, d, scale, causal, eab::kDefaultThreshold, 1,
+                       nullptr, stream);
+}
+
+int attn_fwd_config(const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                    int H, int Nq, int Nk, int d, float scale, int causal,
+                    float rescale_threshold, int exp_mode, unsigned long long* rescale_count,
+                    cudaStream_t stream) {
+  return eab::fwd_impl(q, k, v, o, lse, B, H, Nq, Nk, d, scale, causal, rescale_threshold,
+                       exp_mode, rescale_count, stream);
+}
+
+int attn_status_sync(cudaStream_t stream) {
+  cudaError_t e = cudaStreamSynchronize(stream);
+  if (e != cudaSuccess) return eab::cuda_fail(e, "cudaStreamSynchronize");
+  unsigned int st = 0;
+  e = cudaMemcpyFromSymbolAsync(&st, eab::g_status, sizeof(st), 0, cudaMemcpyDeviceToHost, stream);
+  if (e != cudaSuccess) return eab::cuda_fail(e, "read status word");
+  const unsigned int zero = 0;
+  e = cudaMemcpyToSymbolAsync(eab::g_status, &zero, sizeof(zero), 0, cudaMemcpyHostToDevice, stream);
+  if (e != cudaSuccess) return eab::cuda_fail(e, "clear status word");
+  e = cudaStreamSynchronize(stream);
+  if (e != cudaSuccess) return eab::cuda_fail(e, "cudaStreamSynchronize");
+  return (st & eab::kStatusTimeout) ? ATTN_ERR_TIMEOUT : ATTN_OK;
+}
+
+const char* attn_status_string(int code) {
+  switch (code) {
+    case ATTN_OK: return "ok";
+    case ATTN_ERR_INVALID_ARG: return "invalid argument";
+    case ATTN_ERR_UNSUPPORTED: return "unsupported configuration";
+    case ATTN_ERR_CUDA: return "CUDA error";
+    case ATTN_ERR_TIMEOUT: return "device pipeline wait timed out";
+    default: return "unknown status";
+  }
+}
+
+const char* attn_last_error(void) { return eab::t_last_error.c_str(); }
+
+int attn_selftest_timeout(unsigned int timeout_us, cudaStream_t stream) {
+  if (timeout_us < 1 || timeout_us > 10000000u) return ATTN_ERR_INVALID_ARG;
+  int rc = eab::check_device();
+  if (rc != ATTN_OK) return rc;
+  eab::selftest_timeout_kernel<<<1, 32, 0, stream>>>(static_cast<uint64_t>(timeout_us) * 1000ull);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return eab::cuda_fail(e, "selftest_timeout_kernel launch");
+  return ATTN_OK;
+}
+
+}  // extern "C"

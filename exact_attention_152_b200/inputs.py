@@ -24,6 +24,9 @@ generators", OOPSLA 2014.)
 """
 from __future__ import annotations
 
+import concurrent.futures
+import os
+
 import numpy as np
 
 GAMMA = np.uint64(0x9E3779B97F4A7C15)
@@ -102,16 +105,29 @@ def gen_bf16_at(seed: int, tensor: str, flat_idx: np.ndarray, dist: str = "norma
 
 def gen_bf16(seed: int, tensor: str, shape, dist: str = "normal", mult: float = 1.0,
              out: np.ndarray | None = None) -> np.ndarray:
-    """BF16 bits of a whole contiguous tensor of ``shape`` (flat index = C order)."""
+    """BF16 bits of a whole contiguous tensor of ``shape`` (flat index = C order).
+
+    Chunks are independent (counter based), so they are filled by a thread pool;
+    numpy releases the GIL inside its element-wise kernels.
+    """
     n = int(np.prod(shape))
     key = _key(seed, TENSOR_ID[tensor])
     if out is None:
         out = np.empty(n, dtype=np.uint16)
     flat = out.reshape(-1)
     assert flat.size == n
-    for s in range(0, n, _CHUNK):
+
+    def fill(s):
         e = min(n, s + _CHUNK)
         flat[s:e] = _values(key, np.arange(s, e, dtype=np.int64), dist, mult)
+
+    starts = range(0, n, _CHUNK)
+    if n > 2 * _CHUNK:
+        with concurrent.futures.ThreadPoolExecutor(max_workers=min(16, os.cpu_count() or 1)) as ex:
+            list(ex.map(fill, starts))
+    else:
+        for s in starts:
+            fill(s)
     return out.reshape(shape)
 
 

@@ -1,0 +1,125 @@
+/*
+ * libattn -- exact scaled dot-product attention, forward pass, for NVIDIA B200
+ * (sm_100a).  C ABI: plain pointers, sizes and a CUDA stream; no C++ or
+ * framework types cross this boundary.
+ *
+ * What is computed.  FlashAttention 4: LLM向けのより高速でメモリ効率の良いアテンション
+ * (ja.linux-konsole.com), section "はじめに": attention multiplies the queries Q
+ * with the keys K, normalises with a softmax and multiplies by the values V.
+ * Flash Attention glossary (jisaku.com), section "タイリングによるSRAMの活用" and
+ * "オンライン・ソフトマックスと再計算": the work is tiled through on-chip memory
+ * with a running per-row max and sum, so the Nq x Nk score matrix never reaches
+ * device memory; FAQ Q3 on the same page: the result equals standard attention
+ * up to floating-point rounding.  The pages print no formula and never mention
+ * the scale, causal masking or the log-sum-exp; this library defines, per
+ * (b, h) and query row i:
+ *
+ *     s_ij   = scale * <q_i, k_j>            for j in K(i)
+ *     K(i)   = {0..Nk-1}, or {0..i} when causal (requires Nq == Nk)
+ *     O_i    = sum_j softmax_j(s_ij) * v_j
+ *     LSE_i  = log(sum_j exp(s_ij))           natural logarithm
+ *     K(i) empty (Nk == 0): O_i = 0, LSE_i = -inf
+ *
+ * Layout.  q, k, v, o are BF16, contiguous, row-major [B, H, N, d] with d
+ * fastest (N = Nq for q and o, N = Nk for k and v).  lse is FP32 [B, H, Nq].
+ * Arithmetic: BF16 products, FP32 accumulation and softmax, O rounded to BF16
+ * (round to nearest even) once at the end.
+ *
+ * Ownership.  Every pointer is a DEVICE pointer owned by the caller.  The
+ * library never allocates, frees or retains them.  o and lse must not overlap
+ * q, k, v or each other.
+ *
+ * Asynchrony.  attn_fwd() validates its arguments on the host, enqueues the
+ * work on `stream` (NULL = the legacy default stream) and returns without
+ * synchronising.  Outputs are valid once the stream reaches that point.
+ *
+ * Errors.  Argument errors are detected on the host before anything is
+ * enqueued and nothing is launched.  A device-side failure (a pipeline wait
+ * that exceeded its time limit) sets a per-device status word, reported and
+ * cleared by attn_status_sync().
+ */
+#ifndef EXACT_ATTENTION_152_B200_ATTN_H
+#define EXACT_ATTENTION_152_B200_ATTN_H
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same definition as the CUDA runtime's (an opaque driver stream handle). */
+typedef struct CUstream_st *cudaStream_t;
+
+enum {
+  ATTN_OK = 0,
+  ATTN_ERR_INVALID_ARG = 1, /* null pointer with non-empty problem, negative size,
+                               non-finite scale, misaligned pointer (q,k,v,o need
+                               16-byte alignment, lse 4-byte), overlapping outputs */
+  ATTN_ERR_UNSUPPORTED = 2, /* d not in {64,128}, causal with Nq != Nk, device is
+                               not compute capability 10.0, exp_mode/threshold out
+                               of range */
+  ATTN_ERR_CUDA = 3,        /* CUDA runtime/driver failure (text: attn_last_error) */
+  ATTN_ERR_TIMEOUT = 4      /* a device pipeline wait exceeded its limit */
+};
+
+/*
+ * Forward attention (see the definition above).
+ *   q, k, v  : device, BF16 [B,H,Nq,d], [B,H,Nk,d], [B,H,Nk,d]
+ *   o        : device, BF16 [B,H,Nq,d], written
+ *   lse      : device, FP32 [B,H,Nq], written; may be NULL (not computed)
+ *   B,H,Nq,Nk: >= 0; a problem with B*H*Nq == 0 is a no-op (pointers may be NULL)
+ *   d        : head dimension, 64 or 128
+ *   scale    : any finite float (0 gives uniform weights); not defaulted here
+ *   causal   : 0 or 1; 1 requires Nq == Nk
+ *   stream   : CUDA stream to enqueue on
+ * Returns ATTN_OK or an error code; on error nothing was enqueued.
+ */
+int attn_fwd(const void *q, const void *k, const void *v, void *o, float *lse, int B, int H,
+             int Nq, int Nk, int d, float scale, int causal, cudaStream_t stream);
+
+/*
+ * attn_fwd with the kernel's two softmax knobs exposed (same contract otherwise).
+ *
+ *   rescale_threshold : adaptive online rescaling (FlashAttention 4 page,
+ *       section "よりスマートなオンラインソフトマックス再スケーリング"): the running
+ *       max of a row is replaced -- and the accumulated output and sum rescaled
+ *       -- only when a tile's max exceeds it by more than this many powers of
+ *       two.  0 reproduces the classic always-rescale rule.  Range [0, 64].
+ *       attn_fwd uses 8.
+ *   exp_mode : where exp2 runs (same page, section "CUDAコアによるソフトウェアの
+ *       指数演算"): 0 = hardware MUFU only, 1 = the library's default split
+ *       between MUFU and a cubic polynomial on the FMA pipe, 2 = polynomial only.
+ *   rescale_count : optional device pointer (may be NULL) to one unsigned
+ *       64-bit counter; the kernel atomically adds the number of (row, tile)
+ *       events at which the output accumulator was rescaled.
+ */
+int attn_fwd_config(const void *q, const void *k, const void *v, void *o, float *lse, int B,
+                    int H, int Nq, int Nk, int d, float scale, int causal,
+                    float rescale_threshold, int exp_mode, unsigned long long *rescale_count,
+                    cudaStream_t stream);
+
+/*
+ * Synchronise `stream`, then read and clear the current device's status word.
+ * Returns ATTN_OK, ATTN_ERR_TIMEOUT (a kernel gave up on a pipeline wait since
+ * the last call; its outputs are not valid) or ATTN_ERR_CUDA.
+ */
+int attn_status_sync(cudaStream_t stream);
+
+/* Static English text for a return code. */
+const char *attn_status_string(int code);
+
+/* Text of the last ATTN_ERR_CUDA raised on the calling thread ("" if none). */
+const char *attn_last_error(void);
+
+/*
+ * Diagnostic: launch one block that waits on a pipeline barrier nothing will
+ * ever signal, with the library's bounded wait limited to `timeout_us`
+ * microseconds (1..10,000,000).  The wait runs out, the block records
+ * ATTN_ERR_TIMEOUT in the status word and exits normally, leaving the CUDA
+ * context usable.  Lets a caller check its failure handling without a fault.
+ */
+int attn_selftest_timeout(unsigned int timeout_us, cudaStream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* EXACT_ATTENTION_152_B200_ATTN_H */

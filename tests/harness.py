@@ -1,0 +1,79 @@
+"""Shared helpers for the parity tests: seeded inputs -> CUDA path and oracle.
+
+The CUDA side is reached only through the C-ABI (exact_attention_152_b200.binding);
+the oracle side only through ``oracle``.  They share nothing but the input bits.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+import oracle
+from exact_attention_152_b200 import inputs
+
+# Tolerances of the forward output against the fp64 oracle (BF16 inputs, BF16 O):
+MAX_ABS_O = 1e-2
+MEAN_ABS_O = 1e-3
+MAX_ABS_LSE = 1e-3
+
+
+def to_device_bf16(bits: np.ndarray):
+    import torch
+    t = torch.from_numpy(np.ascontiguousarray(bits).view(np.int16))
+    return t.view(torch.bfloat16).cuda()
+
+
+def run_cuda(q_bits, k_bits, v_bits, scale, causal, **kw):
+    """Run attn_fwd (or attn_fwd_config when knobs are given) via the C-ABI.
+    Returns (o fp32 numpy, lse numpy)."""
+    import torch
+
+    from exact_attention_152_b200 import binding
+    q, k, v = (to_device_bf16(x) for x in (q_bits, k_bits, v_bits))
+    o, lse = binding.fwd(q, k, v, causal=causal, scale=scale, **kw)
+    rc = binding.attn_status_sync(torch.cuda.current_stream().cuda_stream)
+    assert rc == 0, f"device status {rc}"
+    return o.float().cpu().numpy(), lse.cpu().numpy()
+
+
+def oracle_rows(q_bits, k_bits, v_bits, scale, causal, rows_per_head=None):
+    """Oracle on selected rows of every (b, h).  rows_per_head: dict bh -> rows or None (all)."""
+    B, H, Nq, d = q_bits.shape
+    out = {}
+    for b in range(B):
+        for h in range(H):
+            bh = b * H + h
+            rows = np.arange(Nq, dtype=np.int64) if rows_per_head is None else rows_per_head[bh]
+            q = inputs.bf16_bits_to_f64(q_bits[b, h, rows])
+            k = inputs.bf16_bits_to_f64(k_bits[b, h])
+            v = inputs.bf16_bits_to_f64(v_bits[b, h])
+            out[bh] = (rows,) + oracle.attn_rows(q, rows, k, v, scale, causal)
+    return out
+
+
+def compare(o_gpu, lse_gpu, ref, check_lse=True):
+    """Errors of the CUDA output against oracle rows; returns a dict of metrics."""
+    B, H = o_gpu.shape[:2]
+    errs_o, errs_l = [], []
+    for bh, (rows, o_ref, l_ref) in ref.items():
+        b, h = divmod(bh, H)
+        errs_o.append(np.abs(o_gpu[b, h, rows].astype(np.float64) - o_ref).ravel())
+        if check_lse:
+            errs_l.append(np.abs(lse_gpu[b, h, rows].astype(np.float64) - l_ref).ravel())
+    eo = np.concatenate(errs_o)
+    m = {"max_abs_o": float(eo.max()) if eo.size else 0.0, "mean_abs_o": float(eo.mean()) if eo.size else 0.0}
+    if check_lse:
+        el = np.concatenate(errs_l)
+        m["max_abs_lse"] = float(el.max()) if el.size else 0.0
+    return m
+
+
+def assert_within(m, check_lse=True):
+    assert np.isfinite(m["max_abs_o"]), m
+    assert m["max_abs_o"] <= MAX_ABS_O, m
+    assert m["mean_abs_o"] <= MEAN_ABS_O, m
+    if check_lse:
+        assert m["max_abs_lse"] <= MAX_ABS_LSE, m
+
+
+def random_bits(seed, shape, dist="normal", mult=1.0, tensor="q"):
+    return inputs.gen_bf16(seed, tensor, shape, dist, mult)

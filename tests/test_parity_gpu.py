@@ -1,0 +1,176 @@
+"""Parity of the CUDA forward (through the C-ABI) with the fp64 oracle.
+
+Bar: max|dO| <= 1e-2, mean|dO| <= 1e-3, max|dLSE| <= 1e-3 against the oracle
+evaluated on the same BF16 inputs.  Large workloads compare seeded samples of
+query rows (always including the first and last row of every head), computed
+one by one by the oracle.
+"""
+import math
+
+import numpy as np
+import pytest
+
+pytestmark = pytest.mark.gpu
+
+import harness  # noqa: E402
+from exact_attention_152_b200 import inputs  # noqa: E402
+from exact_attention_152_b200.workloads import WORKLOADS  # noqa: E402
+
+
+def _case(B, H, Nq, Nk, d, causal, seed, scale=None, q_mult=1.0, **kw):
+    q = harness.random_bits(seed, (B, H, Nq, d), mult=q_mult, tensor="q")
+    k = harness.random_bits(seed, (B, H, Nk, d), tensor="k")
+    v = harness.random_bits(seed, (B, H, Nk, d), tensor="v")
+    if scale is None:
+        scale = float(np.float32(1 / math.sqrt(d)))
+    o, lse = harness.run_cuda(q, k, v, scale, causal, **kw)
+    ref = harness.oracle_rows(q, k, v, scale, causal)
+    return o, lse, ref, (q, k, v)
+
+
+SHAPES = [
+    # B, H, Nq, Nk, d, causal
+    (1, 1, 1, 1, 64, False), (1, 1, 1, 1, 128, True), (1, 2, 17, 17, 64, True),
+    (2, 1, 128, 128, 128, True), (1, 1, 129, 129, 64, False), (1, 3, 255, 255, 128, True),
+    (1, 1, 256, 256, 64, True), (1, 1, 257, 257, 128, True), (1, 2, 1000, 1000, 128, True),
+    (1, 2, 1000, 1000, 64, False), (1, 1, 100, 300, 128, False), (1, 1, 300, 100, 64, False),
+    (1, 1, 1, 1000, 128, False), (1, 1, 1000, 1, 64, False), (3, 5, 77, 333, 128, False),
+    (1, 1, 513, 513, 128, True), (1, 1, 2048, 2048, 64, True),
+]
+
+
+@pytest.mark.parametrize("shape", SHAPES, ids=[str(s) for s in SHAPES])
+def test_shape_parity(shape):
+    B, H, Nq, Nk, d, causal = shape
+    o, lse, ref, _ = _case(B, H, Nq, Nk, d, causal, seed=sum(shape[:5]))
+    m = harness.compare(o, lse, ref)
+    harness.assert_within(m)
+
+
+@pytest.mark.parametrize("scale", [0.0, -0.2, 0.5, 1e-3])
+def test_scale_values(scale):
+    o, lse, ref, (q, k, v) = _case(1, 2, 300, 300, 128, True, seed=41, scale=scale)
+    harness.assert_within(harness.compare(o, lse, ref))
+
+
+def test_zero_scale_is_uniform():
+    o, lse, ref, (q, k, v) = _case(1, 1, 64, 200, 64, False, seed=42, scale=0.0)
+    vm = inputs.bf16_bits_to_f64(v[0, 0]).mean(0)
+    assert np.abs(o[0, 0] - vm).max() <= 4e-3
+    assert np.abs(lse[0, 0] - math.log(200)).max() <= 1e-4
+
+
+@pytest.mark.parametrize("tau", [0.0, 8.0, 20.0])
+@pytest.mark.parametrize("exp_mode", [0, 1, 2])
+@pytest.mark.parametrize("d", [64, 128])
+def test_softmax_knobs(tau, exp_mode, d):
+    # wide logits (Q x 8) so the running max moves and rescales happen
+    o, lse, ref, _ = _case(1, 2, 700, 700, d, True, seed=43, q_mult=8.0,
+                           rescale_threshold=tau, exp_mode=exp_mode)
+    harness.assert_within(harness.compare(o, lse, ref))
+
+
+def test_rescale_counter_and_reduction():
+    """Adaptive rescaling (threshold 8) must rescale far less often than the
+    classic rule (threshold 0), with the same result within tolerance."""
+    import torch
+    counts = {}
+    for tau in (0.0, 8.0):
+        cnt = torch.zeros(1, dtype=torch.int64, device="cuda")
+        o, lse, ref, _ = _case(1, 4, 4096, 4096, 128, True, seed=44, q_mult=8.0,
+                               rescale_threshold=tau, rescale_count=cnt)
+        harness.assert_within(harness.compare(o, lse, ref))
+        counts[tau] = int(cnt.item())
+    print("rescale events", counts)
+    assert counts[0.0] > 0
+    assert counts[8.0] * 4 <= counts[0.0], counts
+
+
+def test_causal_first_row_is_v0_exactly():
+    import torch
+    q = harness.random_bits(50, (1, 3, 300, 128), tensor="q")
+    k = harness.random_bits(50, (1, 3, 300, 128), tensor="k")
+    v = harness.random_bits(50, (1, 3, 300, 128), tensor="v")
+    for mode in (0, 1, 2):
+        o, _ = harness.run_cuda(q, k, v, 0.088, True, exp_mode=mode)
+        got = torch.from_numpy(o[0, :, 0]).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+        assert np.array_equal(got, v[0, :, 0])
+
+
+def test_single_key_gives_v0_exactly():
+    import torch
+    q = harness.random_bits(51, (2, 2, 130, 64), tensor="q")
+    k = harness.random_bits(51, (2, 2, 1, 64), tensor="k")
+    v = harness.random_bits(51, (2, 2, 1, 64), tensor="v")
+    o, lse = harness.run_cuda(q, k, v, 0.125, False)
+    got = torch.from_numpy(o).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    assert np.array_equal(got, np.broadcast_to(v, got.shape))
+
+
+def test_empty_keys_and_empty_problem():
+    import torch
+    from exact_attention_152_b200 import binding
+    q = torch.randn(1, 2, 5, 64, device="cuda").to(torch.bfloat16)
+    k = torch.empty(1, 2, 0, 64, device="cuda", dtype=torch.bfloat16)
+    o, lse = binding.fwd(q, k, k)
+    torch.cuda.synchronize()
+    assert torch.all(o == 0) and torch.all(torch.isneginf(lse))
+    q0 = torch.empty(0, 2, 5, 64, device="cuda", dtype=torch.bfloat16)
+    o0, l0 = binding.fwd(q0, q0, q0)
+    assert o0.numel() == 0
+
+
+def test_lse_optional_and_no_writes_outside_outputs():
+    import torch
+    from exact_attention_152_b200 import binding
+    B, H, N, d = 1, 2, 300, 128
+    q = harness.to_device_bf16(harness.random_bits(52, (B, H, N, d), tensor="q"))
+    k = harness.to_device_bf16(harness.random_bits(52, (B, H, N, d), tensor="k"))
+    v = harness.to_device_bf16(harness.random_bits(52, (B, H, N, d), tensor="v"))
+    pad = 4096
+    n_o = B * H * N * d
+    o_buf = torch.full((pad + n_o + pad,), 7.0, dtype=torch.bfloat16, device="cuda")
+    l_buf = torch.full((pad + B * H * N + pad,), 7.0, dtype=torch.float32, device="cuda")
+    o = o_buf[pad:pad + n_o].view(B, H, N, d)
+    lse = l_buf[pad:pad + B * H * N].view(B, H, N)
+    binding.fwd(q, k, v, causal=True, out=o, lse=lse)
+    o2 = binding.fwd(q, k, v, causal=True, return_lse=False)
+    assert binding.attn_status_sync(torch.cuda.current_stream().cuda_stream) == 0
+    assert torch.all(o_buf[:pad] == 7.0) and torch.all(o_buf[pad + n_o:] == 7.0)
+    assert torch.all(l_buf[:pad] == 7.0) and torch.all(l_buf[pad + B * H * N:] == 7.0)
+    assert torch.equal(o.view(torch.int16), o2.view(torch.int16))
+
+
+def test_repeatable_bitwise():
+    import torch
+    from exact_attention_152_b200 import binding
+    q = harness.to_device_bf16(harness.random_bits(53, (2, 4, 1024, 128), tensor="q"))
+    k = harness.to_device_bf16(harness.random_bits(53, (2, 4, 1024, 128), tensor="k"))
+    v = harness.to_device_bf16(harness.random_bits(53, (2, 4, 1024, 128), tensor="v"))
+    a = binding.fwd(q, k, v, causal=True)
+    b = binding.fwd(q, k, v, causal=True)
+    torch.cuda.synchronize()
+    assert torch.equal(a[0].view(torch.int16), b[0].view(torch.int16))
+    assert torch.equal(a[1], b[1])
+
+
+# Full workloads last: they are the slowest (input generation and oracle rows).
+def _workload_case(w):
+    q = w.tensor_bits("q")
+    k = w.tensor_bits("k")
+    v = w.tensor_bits("v")
+    o, lse = harness.run_cuda(q, k, v, w.scale, w.causal)
+    rows = None
+    if w.oracle_rows is not None:
+        rows = {bh: w.sampled_rows(bh) for bh in range(w.B * w.H)}
+    ref = harness.oracle_rows(q, k, v, w.scale, w.causal, rows)
+    return o, lse, ref
+
+
+@pytest.mark.parametrize("name", list(WORKLOADS))
+def test_workload_parity(name):
+    w = WORKLOADS[name]
+    o, lse, ref = _workload_case(w)
+    m = harness.compare(o, lse, ref)
+    print(name, m)
+    harness.assert_within(m)
