@@ -29,13 +29,15 @@
 //    next head's data.
 //  * Warps 0-3 / 4-7: softmax, correction and epilogue of query tile 0 / 1
 //    (one thread = one query row = one TMEM lane).  Warp 8: TMA producer.
-//    Warp 9: TMEM allocation and the single MMA-issuing thread.
+//    Warp 9: TMEM allocation and the single MMA-issuing thread.  Warps 10-11
+//    idle (they complete the third warpgroup for the setmaxnreg split).
 //  * Tensor Memory (512 columns): S0 [0,128), S1 [128,256), O0 and O1 after
 //    column 256.  P (BF16) overwrites the first 64 columns of its S tile and is
 //    the A operand of O += P V straight from TMEM, so P never touches shared
 //    memory.
 //  * The MMA thread issues, per KV tile j:  O0 += P0 V_{j-1};  S0 = Q0 K_j^T;
-//    O1 += P1 V_{j-1};  S1 = Q1 K_j^T.  The commit that announces S_t(j) also
+//    O1 += P1 V_{j-1};  S1 = Q1 K_j^T.  Each O += P V is issued in two halves
+//    of 64 keys, each as soon as the softmax warps have stored that half of P.  The commit that announces S_t(j) also
 //    covers O_t += P_t V_{j-1}, so when a softmax warp sees S_t(j) its O_t is
 //    final up to tile j-1 and it can rescale O_t in place without another wait.
 //  * Every wait is bounded (see sm100.cuh); a timeout sets the per-device
@@ -64,7 +66,9 @@ constexpr int kBlockN = 128;  // keys per KV tile
 constexpr int kRowsPerCta = 2 * kBlockM;
 constexpr int kWarpLoad = 8;
 constexpr int kWarpMma = 9;
-constexpr int kNumThreads = 320;
+constexpr int kNumThreads = 384;     // 3 warpgroups: softmax tile 0, softmax tile 1, load/MMA
+constexpr int kSoftmaxRegs = 232;    // setmaxnreg split: 2 x 128 x 232 + 128 x 40 = 384 x 168
+constexpr int kProducerRegs = 40;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint64_t kWaitTimeoutNs = 2000000000ull;  // 2 s per pipeline wait
 constexpr float kDefaultThreshold = 8.0f;           // powers of two
@@ -87,7 +91,7 @@ struct Cfg {
   static constexpr int kOffQ = 0;
   static constexpr int kOffKV = 2 * kTileBytes;
   static constexpr int kOffBar = kOffKV + kStages * kTileBytes;
-  static constexpr int kNumBars = 2 + 2 * kStages + 2 + 2 + 2 + 1;
+  static constexpr int kNumBars = 2 + 2 * kStages + 2 + 4 + 2 + 1;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
   static constexpr int kSmemBytes = kOffMisc + 16 + 1024;  // + slack for 1 KiB alignment
   static constexpr uint32_t kTmemO = 256;
@@ -122,9 +126,12 @@ struct Smem {
   __device__ __forceinline__ uint32_t kv_full(int s) const { return bar(2 + s); }
   __device__ __forceinline__ uint32_t kv_empty(int s) const { return bar(2 + Cfg<D>::kStages + s); }
   __device__ __forceinline__ uint32_t s_full(int t) const { return bar(2 + 2 * Cfg<D>::kStages + t); }
-  __device__ __forceinline__ uint32_t p_full(int t) const { return bar(4 + 2 * Cfg<D>::kStages + t); }
-  __device__ __forceinline__ uint32_t o_full(int t) const { return bar(6 + 2 * Cfg<D>::kStages + t); }
-  __device__ __forceinline__ uint32_t mma_done() const { return bar(8 + 2 * Cfg<D>::kStages); }
+  // P of tile t, keys [64*half, 64*half + 64), written to TMEM
+  __device__ __forceinline__ uint32_t p_full(int t, int half) const {
+    return bar(4 + 2 * Cfg<D>::kStages + 2 * t + half);
+  }
+  __device__ __forceinline__ uint32_t o_full(int t) const { return bar(8 + 2 * Cfg<D>::kStages + t); }
+  __device__ __forceinline__ uint32_t mma_done() const { return bar(10 + 2 * Cfg<D>::kStages); }
   __device__ __forceinline__ uint32_t* tmem_slot() const {
     return reinterpret_cast<uint32_t*>(base + Cfg<D>::kOffMisc);
   }
@@ -199,26 +206,45 @@ __device__ __forceinline__ void mma_role(const Smem<D>& sm, uint32_t tmem, int n
   };
   // S_t = Q_t K^T : M=128 queries, N=128 keys, K=d in steps of 16 (32 bytes of
   // the 128-byte swizzled row; a new box every 64 columns of d).
+  // Descriptors are built once; a K step or another stage only adds a constant
+  // to the 14-bit start-address field (addresses stay below 256 KiB).
+  const uint64_t desc_q0 = sdesc_sw128(sm.q(0), 16, 1024);
+  const uint64_t desc_kv0 = sdesc_sw128(sm.kv(0), 16, 1024);
+  const uint64_t desc_v0 = sdesc_sw128(sm.kv(0), C::kBoxBytes, 1024);
   auto mma_s = [&](int t, uint32_t slot) {
     const uint32_t d_tmem = tmem + t * kBlockM;
-#pragma unroll
+    const uint64_t a0 = desc_q0 + static_cast<uint64_t>((t * C::kTileBytes) >> 4);
+    const uint64_t b0 = desc_kv0 + static_cast<uint64_t>((slot * C::kTileBytes) >> 4);
+#pragma unroll 1  // one issuing thread: a loop keeps it within 40 registers
     for (int kk = 0; kk < D / 16; ++kk) {
-      const uint32_t off = (kk >> 2) * C::kBoxBytes + (kk & 3) * 32;
-      mma_ss(d_tmem, sdesc_sw128(sm.q(t) + off, 16, 1024), sdesc_sw128(sm.kv(slot) + off, 16, 1024),
-             idesc_s, kk > 0 ? 1u : 0u);
+      const uint32_t off = ((kk >> 2) * C::kBoxBytes + (kk & 3) * 32) >> 4;
+      mma_ss(d_tmem, a0 + off, b0 + off, idesc_s, kk > 0 ? 1u : 0u);
     }
   };
-  // O_t += P_t V : M=128 queries, N=d, K=128 keys in steps of 16.  P (bf16,
-  // two per column) sits in the first 64 TMEM columns of S_t.  V is MN-major:
-  // 16 keys = 16 rows of 128 bytes = 2048 bytes; the 64-wide d boxes are
-  // kBoxBytes apart (LBO), 8-row groups 1024 bytes apart (SBO).
-  auto mma_o = [&](int t, uint32_t slot, bool acc) {
+  // O_t += P_t V for keys [64*half, 64*half + 64): M=128 queries, N=d, K in
+  // steps of 16.  P (bf16, two per column) sits in the first 64 TMEM columns of
+  // S_t.  V is MN-major: 16 keys = 16 rows of 128 bytes = 2048 bytes; the
+  // 64-wide d boxes are kBoxBytes apart (LBO), 8-row groups 1024 bytes (SBO).
+  auto mma_o_half = [&](int t, uint32_t slot, int half, bool acc) {
     const uint32_t d_tmem = tmem + C::kTmemO + t * D;
     const uint32_t a_tmem = tmem + t * kBlockM;
-#pragma unroll
-    for (int kk = 0; kk < kBlockN / 16; ++kk)
-      mma_ts(d_tmem, a_tmem + kk * 8, sdesc_sw128(sm.kv(slot) + kk * 2048, C::kBoxBytes, 1024),
-             idesc_o, (acc || kk > 0) ? 1u : 0u);
+    const uint64_t b0 = desc_v0 + static_cast<uint64_t>((slot * C::kTileBytes) >> 4);
+#pragma unroll 1
+    for (int k4 = 0; k4 < 4; ++k4) {
+      const int kk = half * 4 + k4;
+      mma_ts(d_tmem, a_tmem + kk * 8, b0 + static_cast<uint64_t>((kk * 2048) >> 4), idesc_o,
+             (acc || kk > 0) ? 1u : 0u);
+    }
+  };
+  // Both halves of O_t += P_t V_j, each issued as soon as its P half is in TMEM.
+  auto mma_o = [&](int t, uint32_t slot, bool acc, uint32_t par) -> bool {
+    if (!mbar_wait(sm.p_full(t, 0), par, timeout)) return false;
+    tc_fence_after();
+    mma_o_half(t, slot, 0, acc);
+    if (!mbar_wait(sm.p_full(t, 1), par, timeout)) return false;
+    tc_fence_after();
+    mma_o_half(t, slot, 1, acc);
+    return true;
   };
 
   uint32_t sK = 0, sV = 0;
@@ -237,19 +263,15 @@ __device__ __forceinline__ void mma_role(const Smem<D>& sm, uint32_t tmem, int n
   }
   for (int j = 1; ok && j < n_kv; ++j) {
     const uint32_t par = (j - 1) & 1;
-    ok = wait_kv(sV) && mbar_wait(sm.p_full(0), par, timeout);
+    ok = wait_kv(sV) && mma_o(0, sV, j > 1, par);
     if (!ok) break;
-    tc_fence_after();
-    mma_o(0, sV, j > 1);
     ok = wait_kv(sK);
     if (!ok) break;
     tc_fence_after();
     mma_s(0, sK);
     tc_commit(sm.s_full(0));
-    ok = mbar_wait(sm.p_full(1), par, timeout);
+    ok = mma_o(1, sV, j > 1, par);
     if (!ok) break;
-    tc_fence_after();
-    mma_o(1, sV, j > 1);
     tc_commit(sm.kv_empty(sV));
     mma_s(1, sK);
     tc_commit(sm.s_full(1));
@@ -257,16 +279,12 @@ __device__ __forceinline__ void mma_role(const Smem<D>& sm, uint32_t tmem, int n
   }
   if (ok) {
     const uint32_t par = (n_kv - 1) & 1;
-    ok = wait_kv(sV) && mbar_wait(sm.p_full(0), par, timeout);
+    ok = wait_kv(sV) && mma_o(0, sV, n_kv > 1, par);
     if (ok) {
-      tc_fence_after();
-      mma_o(0, sV, n_kv > 1);
       tc_commit(sm.o_full(0));
-      ok = mbar_wait(sm.p_full(1), par, timeout);
+      ok = mma_o(1, sV, n_kv > 1, par);
     }
     if (ok) {
-      tc_fence_after();
-      mma_o(1, sV, n_kv > 1);
       tc_commit(sm.o_full(1));
       tc_commit(sm.kv_empty(sV));
     }
@@ -307,15 +325,15 @@ __device__ __forceinline__ void softmax_role(const Smem<D>& sm, uint32_t tmem,
   for (int j = 0; j < n_kv; ++j) {
     if (!warp_wait(sm.s_full(t), j & 1, timeout)) { ok = false; break; }
     tc_fence_after();
-    uint32_t s[4][32];
-#pragma unroll
-    for (int q = 0; q < 4; ++q) tmem_ld32(tS + q * 32, s[q]);
+    uint32_t s[kBlockN];
+    tmem_ld64(tS, s);
+    tmem_ld64(tS + 64, s + 64);
     tmem_ld_wait();
-#pragma unroll
-    for (int q = 0; q < 4; ++q) reg_fence32(s[q]);
+    reg_fence64(s);
+    reg_fence64(s + 64);
     float x[kBlockN];
 #pragma unroll
-    for (int c = 0; c < kBlockN; ++c) x[c] = __uint_as_float(s[c >> 5][c & 31]);
+    for (int c = 0; c < kBlockN; ++c) x[c] = __uint_as_float(s[c]);
     if (prescale) {
 #pragma unroll
       for (int c = 0; c < kBlockN; ++c) x[c] *= prm.scale_log2;
@@ -330,16 +348,14 @@ __device__ __forceinline__ void softmax_role(const Smem<D>& sm, uint32_t tmem,
         if (key >= prm.Nk || (CAUSAL && key > row)) x[c] = -INFINITY;
       }
     }
-    float mx[8];
+    // row max: 3-input max, four independent chains
+    float mx[4] = {x[0], x[1], x[2], x[3]};
 #pragma unroll
-    for (int c = 0; c < 8; ++c) mx[c] = x[c];
+    for (int c = 4; c < kBlockN; c += 8) {
 #pragma unroll
-    for (int c = 8; c < kBlockN; ++c) mx[c & 7] = fmaxf(mx[c & 7], x[c]);
-#pragma unroll
-    for (int w = 4; w >= 1; w >>= 1)
-#pragma unroll
-      for (int c = 0; c < w; ++c) mx[c] = fmaxf(mx[c], mx[c + w]);
-    const float m_tile = mx[0] * sl;
+      for (int a = 0; a < 4; ++a) mx[a] = fmax3(mx[a], x[c + 2 * a], x[c + 2 * a + 1]);
+    }
+    const float m_tile = fmax3(fmaxf(mx[0], mx[1]), mx[2], mx[3]) * sl;
 
     // adaptive rescaling: move the reference only on a jump beyond tau
     const bool resc = m_tile > m_run + prm.tau;
@@ -349,23 +365,8 @@ __device__ __forceinline__ void softmax_role(const Smem<D>& sm, uint32_t tmem,
       m_run = m_tile;
     }
     l_run *= alpha;
-
-    const float neg_m = (m_run == -INFINITY) ? 0.0f : -m_run;
-    float sum[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-    uint32_t p[2][32];
-#pragma unroll
-    for (int c = 0; c < kBlockN; c += 2) {
-      const float a = ex2_split<POLY16>(fmaf(x[c], sl, neg_m), c);
-      const float b = ex2_split<POLY16>(fmaf(x[c + 1], sl, neg_m), c + 1);
-      sum[(c >> 1) & 3] += a + b;
-      p[c >> 6][(c & 63) >> 1] = pack_bf16x2(a, b);
-    }
-    l_run += (sum[0] + sum[1]) + (sum[2] + sum[3]);
-    tmem_st32(tS, p[0]);
-    tmem_st32(tS + 32, p[1]);
     // Correction: rescale this row's O accumulator (already final up to tile
-    // j-1, see the MMA order) by alpha before O += P V_j is issued.  Done after
-    // the P stores so the 128 score registers are dead by now.
+    // j-1, see the MMA order) by alpha before O += P V_j is issued.
     if (j > 0 && __any_sync(0xffffffffu, resc)) {
       if (prm.rescale_count) {
         const unsigned n = __popc(__ballot_sync(0xffffffffu, resc));
@@ -382,10 +383,40 @@ __device__ __forceinline__ void softmax_role(const Smem<D>& sm, uint32_t tmem,
         tmem_st32(tO + cc * 32, o);
       }
     }
-    tmem_st_wait();
-    tc_fence_before();
-    __syncwarp();
-    if (lane == 0) mbar_arrive(sm.p_full(t));
+
+    // P = 2^(x*sl - m) in two halves of 64 keys; each half is stored to TMEM
+    // and announced on its own barrier so the MMA of the first half overlaps
+    // the exponentials of the second.
+    const float neg_m = (m_run == -INFINITY) ? 0.0f : -m_run;
+    const float2 sl2 = make_float2(sl, sl), nm2 = make_float2(neg_m, neg_m);
+    float2 sum2[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                      make_float2(0.f, 0.f)};
+#pragma unroll
+    for (int half = 0; half < 2; ++half) {
+      uint32_t p[32];
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        const int c = half * 64 + 2 * i;
+        const float2 u = ffma2(make_float2(x[c], x[c + 1]), sl2, nm2);
+        float2 e;
+        if ((c & 15) < POLY16) {
+          e = ex2_poly2(u);
+        } else {
+          e.x = ex2_mufu(u.x);
+          e.y = ex2_mufu(u.y);
+        }
+        sum2[i & 3] = fadd2(sum2[i & 3], e);
+        p[i] = pack_bf16x2(e.x, e.y);
+      }
+      tmem_st32(tS + half * 32, p);
+      tmem_st_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(sm.p_full(t, half));
+    }
+    const float2 s01 = fadd2(sum2[0], sum2[1]), s23 = fadd2(sum2[2], sum2[3]);
+    const float2 s03 = fadd2(s01, s23);
+    l_run += s03.x + s03.y;
   }
 
   if (ok) ok = warp_wait(sm.o_full(t), 0, timeout);
@@ -468,7 +499,9 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     for (int i = 0; i < C::kNumBars; ++i) {
       const uint32_t b = sm.bar(i);
       // p_full: one arrival per softmax warp of the tile; everything else: one.
-      mbar_init(b, (b == sm.p_full(0) || b == sm.p_full(1)) ? 4u : 1u);
+      const bool pf = b == sm.p_full(0, 0) || b == sm.p_full(0, 1) || b == sm.p_full(1, 0) ||
+                      b == sm.p_full(1, 1);
+      mbar_init(b, pf ? 4u : 1u);
     }
     fence_barrier_init();
     fence_proxy_async_smem();
@@ -488,13 +521,18 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   tc_fence_after();
   const uint32_t tmem = *sm.tmem_slot();
 
-  if (warp == kWarpLoad) {
-    if (lane == 0) producer_role<D>(sm, &tm_q, &tm_k, &tm_v, bh, qb, n_kv, prm.timeout_ns);
-    __syncwarp();
-  } else if (warp == kWarpMma) {
-    if (lane == 0) mma_role<D>(sm, tmem, n_kv, prm.timeout_ns);
-    __syncwarp();
+  if (warp >= kWarpLoad) {
+    // warpgroup 2: TMA producer (warp 8), MMA issuer (warp 9), two idle warps
+    setmaxnreg_dec<kProducerRegs>();
+    if (warp == kWarpLoad) {
+      if (lane == 0) producer_role<D>(sm, &tm_q, &tm_k, &tm_v, bh, qb, n_kv, prm.timeout_ns);
+      __syncwarp();
+    } else if (warp == kWarpMma) {
+      if (lane == 0) mma_role<D>(sm, tmem, n_kv, prm.timeout_ns);
+      __syncwarp();
+    }
   } else {
+    setmaxnreg_inc<kSoftmaxRegs>();
     softmax_role<D, CAUSAL, POLY16>(sm, tmem, &tm_o, prm, bh, qb, n_kv);
   }
 

@@ -2,6 +2,8 @@
 // building-block tests.
 #pragma once
 
+#include "sm100.cuh"
+
 namespace eab {
 
 // exp2 on the FMA pipe: 2^x = 2^n * p(f), n = round-to-nearest(x), f = x - n in
@@ -24,6 +26,23 @@ __device__ __forceinline__ float ex2_poly(float x) {
   p = __fmaf_rn(p, f, kExpC1);
   p = __fmaf_rn(p, f, 1.0f);
   return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
+}
+
+// The same polynomial exp2 on a pair of values with packed fp32 instructions:
+// the rounding, the reduction and the Horner steps each cost one instruction
+// for both lanes; only the clamp and the exponent insertion stay scalar.
+__device__ __forceinline__ float2 ex2_poly2(float2 x) {
+  x.x = fmaxf(x.x, -127.0f);
+  x.y = fmaxf(x.y, -127.0f);
+  const float2 kShift = make_float2(12582912.0f, 12582912.0f);
+  const float2 t = fadd2(x, kShift);
+  const float2 n = fsub2(t, kShift);
+  const float2 f = fsub2(x, n);
+  float2 p = ffma2(make_float2(kExpC3, kExpC3), f, make_float2(kExpC2, kExpC2));
+  p = ffma2(p, f, make_float2(kExpC1, kExpC1));
+  p = ffma2(p, f, make_float2(1.0f, 1.0f));
+  return make_float2(__int_as_float(__float_as_int(p.x) + (__float_as_int(t.x) << 23)),
+                     __int_as_float(__float_as_int(p.y) + (__float_as_int(t.y) << 23)));
 }
 
 }  // namespace eab

@@ -77,31 +77,41 @@ def test_softmax_knobs(tau, exp_mode, d):
 
 @pytest.mark.parametrize("exp_mode", [0, 1, 2])
 def test_peaked_softmax_relative(exp_mode):
-    """V ~ N(0,1) with logits of std 8: |O| reaches several units.  Each output
-    is then within 2^-7 relative (two BF16 half-ulps: P and O rounding) of the
-    oracle, and LSE within the absolute bar."""
-    o, lse, ref, _ = _case(1, 2, 700, 700, 128, True, seed=45, q_mult=8.0, exp_mode=exp_mode)
+    """V ~ N(0,1) with logits of std 8: |O| reaches several units, beyond what
+    the absolute bar allows for a BF16 output.  Error budget of the kernel: P is
+    rounded to BF16 (2^-9 relative per weight) and O once more (2^-9), so
+    |dO| <= 2^-8 * sum_j p_j |v_j| (+ the exp2 error, 1.1e-4); the test allows
+    twice that.  sum_j p_j |v_j| is the oracle run on |V|."""
+    d = 128
+    scale = float(np.float32(1 / math.sqrt(d)))
+    o, lse, ref, (q, k, v) = _case(1, 2, 700, 700, d, True, seed=45, q_mult=8.0, exp_mode=exp_mode)
+    v_abs = inputs.f32_to_bf16_bits(np.abs(inputs.bf16_bits_to_f32(v)))
+    ref_abs = harness.oracle_rows(q, k, v_abs, scale, True)
     for bh, (rows, o_ref, l_ref) in ref.items():
+        o_abs = ref_abs[bh][1]
         err = np.abs(o[0, bh, rows] - o_ref)
-        bound = 2.0 ** -7 * np.maximum(np.abs(o_ref), 0.25)
+        bound = 2.0 ** -7 * o_abs + 1e-6
         assert np.all(err <= bound), float((err / bound).max())
         assert np.abs(lse[0, bh, rows] - l_ref).max() <= harness.MAX_ABS_LSE
 
 
-def test_rescale_counter_and_reduction():
+@pytest.mark.parametrize("q_mult,min_ratio", [(1.0, 10.0), (8.0, 3.0)])
+def test_rescale_counter_and_reduction(q_mult, min_ratio):
     """Adaptive rescaling (threshold 8) must rescale far less often than the
-    classic rule (threshold 0), with the same result within tolerance."""
+    classic rule (threshold 0), with the same result within tolerance.  With
+    N(0,1) logits the first tile's max is almost never exceeded by 2^8; with
+    logits of std 8 the max still climbs past the threshold now and then."""
     import torch
     counts = {}
     for tau in (0.0, 8.0):
         cnt = torch.zeros(1, dtype=torch.int64, device="cuda")
-        o, lse, ref, _ = _case(1, 4, 4096, 4096, 128, True, seed=44, q_mult=8.0,
+        o, lse, ref, _ = _case(1, 4, 4096, 4096, 128, True, seed=44, q_mult=q_mult,
                                v_dist="uniform", rescale_threshold=tau, rescale_count=cnt)
         harness.assert_within(harness.compare(o, lse, ref))
         counts[tau] = int(cnt.item())
-    print("rescale events", counts)
+    print("rescale events", q_mult, counts)
     assert counts[0.0] > 0
-    assert counts[8.0] * 4 <= counts[0.0], counts
+    assert counts[8.0] * min_ratio <= counts[0.0], counts
 
 
 def test_causal_first_row_is_v0_exactly():
