@@ -348,10 +348,12 @@ __device__ __forceinline__ void softmax_role(const Smem<D>& sm, uint32_t tmem,
         if (key >= prm.Nk || (CAUSAL && key > row)) x[c] = -INFINITY;
       }
     }
-    // row max: 3-input max, four independent chains
-    float mx[4] = {x[0], x[1], x[2], x[3]};
+    // row max: 3-input max, four independent chains over columns 0..127
+    float mx[4];
 #pragma unroll
-    for (int c = 4; c < kBlockN; c += 8) {
+    for (int a = 0; a < 4; ++a) mx[a] = fmaxf(x[2 * a], x[2 * a + 1]);
+#pragma unroll
+    for (int c = 8; c < kBlockN; c += 8) {
 #pragma unroll
       for (int a = 0; a < 4; ++a) mx[a] = fmax3(mx[a], x[c + 2 * a], x[c + 2 * a + 1]);
     }
