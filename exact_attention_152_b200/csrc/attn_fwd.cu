@@ -64,10 +64,15 @@ namespace eab {
 constexpr int kBlockM = 128;  // query rows per tile  (= TMEM lanes)
 constexpr int kBlockN = 128;  // keys per KV tile
 constexpr int kRowsPerCta = 2 * kBlockM;
-constexpr int kWarpLoad = 8;
-constexpr int kWarpMma = 9;
-constexpr int kNumThreads = 384;     // 3 warpgroups: softmax tile 0, softmax tile 1, load/MMA
-constexpr int kSoftmaxRegs = 232;    // setmaxnreg split: 2 x 128 x 232 + 128 x 40 = 384 x 168
+// 5 warpgroups: 4 softmax warpgroups (tile t, key half h -> warps 8t+4h .. 8t+4h+3)
+// and one for the TMA producer (warp 16), the MMA issuer (warp 17) and two idle
+// warps that complete the group for the register split.
+constexpr int kNumSoftmaxWarps = 16;
+constexpr int kWarpLoad = 16;
+constexpr int kWarpMma = 17;
+constexpr int kNumThreads = 640;
+// setmaxnreg split of the 640 x 96 launch budget: 512 x 104 + 128 x 40 <= 61440.
+constexpr int kSoftmaxRegs = 104;
 constexpr int kProducerRegs = 40;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint64_t kWaitTimeoutNs = 2000000000ull;  // 2 s per pipeline wait
@@ -91,9 +96,13 @@ struct Cfg {
   static constexpr int kOffQ = 0;
   static constexpr int kOffKV = 2 * kTileBytes;
   static constexpr int kOffBar = kOffKV + kStages * kTileBytes;
-  static constexpr int kNumBars = 2 + 2 * kStages + 2 + 4 + 2 + 1;
+  static constexpr int kNumBars = 2 + 2 * kStages + 2 + 2 + 2 + 1;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
-  static constexpr int kSmemBytes = kOffMisc + 16 + 1024;  // + slack for 1 KiB alignment
+  // row-max / row-sum exchange between the two key halves of a row:
+  // float [tile 2][half 2][parity 2][row 128]
+  static constexpr int kOffXch = (kOffMisc + 16 + 15) / 16 * 16;
+  static constexpr int kXchBytes = 2 * 2 * 2 * kBlockM * 4;
+  static constexpr int kSmemBytes = kOffXch + kXchBytes + 1024;  // + slack for 1 KiB alignment
   static constexpr uint32_t kTmemO = 256;
 };
 
@@ -126,12 +135,13 @@ struct Smem {
   __device__ __forceinline__ uint32_t kv_full(int s) const { return bar(2 + s); }
   __device__ __forceinline__ uint32_t kv_empty(int s) const { return bar(2 + Cfg<D>::kStages + s); }
   __device__ __forceinline__ uint32_t s_full(int t) const { return bar(2 + 2 * Cfg<D>::kStages + t); }
-  // P of tile t, keys [64*half, 64*half + 64), written to TMEM
-  __device__ __forceinline__ uint32_t p_full(int t, int half) const {
-    return bar(4 + 2 * Cfg<D>::kStages + 2 * t + half);
+  // P of tile t written to TMEM (and O_t rescaled) by all 8 warps of the tile
+  __device__ __forceinline__ uint32_t p_full(int t) const { return bar(4 + 2 * Cfg<D>::kStages + t); }
+  __device__ __forceinline__ uint32_t o_full(int t) const { return bar(6 + 2 * Cfg<D>::kStages + t); }
+  __device__ __forceinline__ uint32_t mma_done() const { return bar(8 + 2 * Cfg<D>::kStages); }
+  __device__ __forceinline__ float* xch(int t, int h, int par) const {
+    return reinterpret_cast<float*>(base + Cfg<D>::kOffXch) + ((t * 2 + h) * 2 + par) * kBlockM;
   }
-  __device__ __forceinline__ uint32_t o_full(int t) const { return bar(8 + 2 * Cfg<D>::kStages + t); }
-  __device__ __forceinline__ uint32_t mma_done() const { return bar(10 + 2 * Cfg<D>::kStages); }
   __device__ __forceinline__ uint32_t* tmem_slot() const {
     return reinterpret_cast<uint32_t*>(base + Cfg<D>::kOffMisc);
   }
@@ -190,13 +200,43 @@ __device__ __forceinline__ void producer_role(const Smem<D>& sm, const CUtensorM
 // ---------------------------------------------------------------------------
 // MMA issuer: one thread.
 // ---------------------------------------------------------------------------
+template <int D, int KK>
+struct MmaUnroll {
+  // S = Q K^T, K steps KK .. D/16-1: 32 bytes along the 128-byte row, a new
+  // 64-column box every 4 steps.
+  __device__ __forceinline__ static void s(uint32_t d, uint32_t a_lo, uint32_t a_hi, uint32_t b_lo,
+                                           uint32_t b_hi, uint32_t idesc) {
+    if constexpr (KK < D / 16) {
+      constexpr uint32_t off = ((KK >> 2) * Cfg<D>::kBoxBytes + (KK & 3) * 32) >> 4;
+      mma_ss_imm<off, off, KK == 0 ? 0u : 1u>(d, a_lo, a_hi, b_lo, b_hi, idesc);
+      MmaUnroll<D, KK + 1>::s(d, a_lo, a_hi, b_lo, b_hi, idesc);
+    }
+  }
+  // O += P V, K steps KK .. 7: P of keys [64h, 64h+64) in TMEM columns
+  // [64h, 64h+32) (two bf16 per column); V rows of 16 keys = 2048 bytes.
+  __device__ __forceinline__ static void o(uint32_t d, uint32_t a_tmem, uint32_t b_lo, uint32_t b_hi,
+                                           uint32_t idesc, uint32_t acc) {
+    if constexpr (KK < kBlockN / 16) {
+      constexpr uint32_t a_off = (KK >> 2) * 64 + (KK & 3) * 8;
+      constexpr uint32_t b_off = (KK * 2048) >> 4;
+      mma_ts_imm<a_off, b_off>(d, a_tmem, b_lo, b_hi, idesc, KK == 0 ? acc : 1u);
+      MmaUnroll<D, KK + 1>::o(d, a_tmem, b_lo, b_hi, idesc, acc);
+    }
+  }
+};
+
+// ---------------------------------------------------------------------------
+// MMA issuer: one thread.  Per KV tile j it waits for V_{j-1} and K_j first
+// (normally long resident), so the only wait between a tile's P becoming
+// ready and its O += P V_{j-1}; S = Q K_j^T block is the P barrier itself.
+// ---------------------------------------------------------------------------
 template <int D>
 __device__ __forceinline__ void mma_role(const Smem<D>& sm, uint32_t tmem, int n_kv,
                                          uint64_t timeout) {
   using C = Cfg<D>;
   constexpr uint32_t idesc_s = idesc_bf16_f32(kBlockM, kBlockN, false, false);
   constexpr uint32_t idesc_o = idesc_bf16_f32(kBlockM, D, false, true);
-  uint32_t it = 0;
+  uint32_t it = 0;  // position in the K0, V0, K1, V1, ... ring order
 
   auto wait_kv = [&](uint32_t& slot) -> bool {
     slot = it % C::kStages;
@@ -204,46 +244,23 @@ __device__ __forceinline__ void mma_role(const Smem<D>& sm, uint32_t tmem, int n
     ++it;
     return mbar_wait(sm.kv_full(slot), phase, timeout);
   };
-  // S_t = Q_t K^T : M=128 queries, N=128 keys, K=d in steps of 16 (32 bytes of
-  // the 128-byte swizzled row; a new box every 64 columns of d).
-  // Descriptors are built once; a K step or another stage only adds a constant
-  // to the 14-bit start-address field (addresses stay below 256 KiB).
-  const uint64_t desc_q0 = sdesc_sw128(sm.q(0), 16, 1024);
-  const uint64_t desc_kv0 = sdesc_sw128(sm.kv(0), 16, 1024);
-  const uint64_t desc_v0 = sdesc_sw128(sm.kv(0), C::kBoxBytes, 1024);
+  // descriptors as 32-bit halves; stage and tile offsets go into the low word
+  const uint64_t dq = sdesc_sw128(sm.q(0), 16, 1024);
+  const uint64_t dk = sdesc_sw128(sm.kv(0), 16, 1024);
+  const uint64_t dv = sdesc_sw128(sm.kv(0), C::kBoxBytes, 1024);
+  const uint32_t q_lo = static_cast<uint32_t>(dq), q_hi = static_cast<uint32_t>(dq >> 32);
+  const uint32_t k_lo = static_cast<uint32_t>(dk), k_hi = static_cast<uint32_t>(dk >> 32);
+  const uint32_t v_lo = static_cast<uint32_t>(dv), v_hi = static_cast<uint32_t>(dv >> 32);
+  constexpr uint32_t kTileStep = C::kTileBytes >> 4;
   auto mma_s = [&](int t, uint32_t slot) {
-    const uint32_t d_tmem = tmem + t * kBlockM;
-    const uint64_t a0 = desc_q0 + static_cast<uint64_t>((t * C::kTileBytes) >> 4);
-    const uint64_t b0 = desc_kv0 + static_cast<uint64_t>((slot * C::kTileBytes) >> 4);
-#pragma unroll 1  // one issuing thread: a loop keeps it within 40 registers
-    for (int kk = 0; kk < D / 16; ++kk) {
-      const uint32_t off = ((kk >> 2) * C::kBoxBytes + (kk & 3) * 32) >> 4;
-      mma_ss(d_tmem, a0 + off, b0 + off, idesc_s, kk > 0 ? 1u : 0u);
-    }
+    MmaUnroll<D, 0>::s(tmem + t * kBlockM, q_lo + t * kTileStep, q_hi, k_lo + slot * kTileStep,
+                       k_hi, idesc_s);
   };
-  // O_t += P_t V for keys [64*half, 64*half + 64): M=128 queries, N=d, K in
-  // steps of 16.  P (bf16, two per column) sits in the first 64 TMEM columns of
-  // S_t.  V is MN-major: 16 keys = 16 rows of 128 bytes = 2048 bytes; the
-  // 64-wide d boxes are kBoxBytes apart (LBO), 8-row groups 1024 bytes (SBO).
-  auto mma_o_half = [&](int t, uint32_t slot, int half, bool acc) {
-    const uint32_t d_tmem = tmem + C::kTmemO + t * D;
-    const uint32_t a_tmem = tmem + t * kBlockM;
-    const uint64_t b0 = desc_v0 + static_cast<uint64_t>((slot * C::kTileBytes) >> 4);
-#pragma unroll 1
-    for (int k4 = 0; k4 < 4; ++k4) {
-      const int kk = half * 4 + k4;
-      mma_ts(d_tmem, a_tmem + kk * 8, b0 + static_cast<uint64_t>((kk * 2048) >> 4), idesc_o,
-             (acc || kk > 0) ? 1u : 0u);
-    }
-  };
-  // Both halves of O_t += P_t V_j, each issued as soon as its P half is in TMEM.
   auto mma_o = [&](int t, uint32_t slot, bool acc, uint32_t par) -> bool {
-    if (!mbar_wait(sm.p_full(t, 0), par, timeout)) return false;
+    if (!mbar_wait(sm.p_full(t), par, timeout)) return false;
     tc_fence_after();
-    mma_o_half(t, slot, 0, acc);
-    if (!mbar_wait(sm.p_full(t, 1), par, timeout)) return false;
-    tc_fence_after();
-    mma_o_half(t, slot, 1, acc);
+    MmaUnroll<D, 0>::o(tmem + C::kTmemO + t * D, tmem + t * kBlockM, v_lo + slot * kTileStep, v_hi,
+                       idesc_o, acc ? 1u : 0u);
     return true;
   };
 
@@ -263,11 +280,10 @@ __device__ __forceinline__ void mma_role(const Smem<D>& sm, uint32_t tmem, int n
   }
   for (int j = 1; ok && j < n_kv; ++j) {
     const uint32_t par = (j - 1) & 1;
-    ok = wait_kv(sV) && mma_o(0, sV, j > 1, par);
+    ok = wait_kv(sV) && wait_kv(sK);
     if (!ok) break;
-    ok = wait_kv(sK);
+    ok = mma_o(0, sV, j > 1, par);
     if (!ok) break;
-    tc_fence_after();
     mma_s(0, sK);
     tc_commit(sm.s_full(0));
     ok = mma_o(1, sV, j > 1, par);
@@ -296,22 +312,35 @@ __device__ __forceinline__ void mma_role(const Smem<D>& sm, uint32_t tmem, int n
 }
 
 // ---------------------------------------------------------------------------
-// Softmax + correction + epilogue for one query tile: 4 warps, 1 row/thread.
+// Softmax + correction + epilogue.  Tile t has 8 warps: warp (t, h, q) owns
+// TMEM lanes 32q..32q+31 (rows) and key columns [64h, 64h+64) of every S tile,
+// and output columns [h*d/2, (h+1)*d/2).  The two warps of a row pair (same t,
+// q) swap their partial row maxima (and at the end their partial sums) through
+// shared memory and a 64-thread named barrier that both reach unconditionally
+// every iteration; a failed wait travels through the same exchange as NaN, so
+// a pair always leaves its loop together.
 // ---------------------------------------------------------------------------
+__device__ __forceinline__ void pair_sync(int t, int q) {
+  asm volatile("bar.sync %0, 64;" ::"r"(1 + t * 4 + q) : "memory");
+}
+
 template <int D, bool CAUSAL, int POLY16>
 __device__ __forceinline__ void softmax_role(const Smem<D>& sm, uint32_t tmem,
                                              const CUtensorMap* tm_o, const FwdParams& prm,
                                              int bh, int qb, int n_kv) {
   using C = Cfg<D>;
+  constexpr int kCols = kBlockN / 2;  // key columns per warp
+  constexpr int kOCols = D / 2;       // output columns per warp
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int t = warp >> 2;   // query tile of this CTA
-  const int q4 = warp & 3;   // TMEM lane quarter this warp may access
+  const int t = warp >> 3;        // query tile of this CTA
+  const int h = (warp >> 2) & 1;  // key half / output-column half
+  const int q4 = warp & 3;        // TMEM lane quarter this warp may access
   const int r = q4 * 32 + lane;
   const int tile_row0 = qb * kRowsPerCta + t * kBlockM;
   const int row = tile_row0 + r;
   const uint32_t lane_off = static_cast<uint32_t>(q4 * 32) << 16;
-  const uint32_t tS = tmem + lane_off + t * kBlockM;
-  const uint32_t tO = tmem + lane_off + C::kTmemO + t * D;
+  const uint32_t tS = tmem + lane_off + t * kBlockM + h * kCols;
+  const uint32_t tO = tmem + lane_off + C::kTmemO + t * D + h * kOCols;
   const uint64_t timeout = prm.timeout_ns;
 
   // scale <= 0: apply it first, then run with an effective scale of 1 (the
@@ -319,47 +348,65 @@ __device__ __forceinline__ void softmax_role(const Smem<D>& sm, uint32_t tmem,
   const bool prescale = !(prm.scale_log2 > 0.0f);
   const float sl = prescale ? 1.0f : prm.scale_log2;
   float m_run = -INFINITY;  // running reference max, log2 units of scaled scores
-  float l_run = 0.0f;       // running sum of 2^(score - m_run)
+  float l_run = 0.0f;       // this half's running sum of 2^(score - m_run)
   bool ok = true;
 
   for (int j = 0; j < n_kv; ++j) {
-    if (!warp_wait(sm.s_full(t), j & 1, timeout)) { ok = false; break; }
-    tc_fence_after();
-    uint32_t s[kBlockN];
-    tmem_ld64(tS, s);
-    tmem_ld64(tS + 64, s + 64);
-    tmem_ld_wait();
-    reg_fence64(s);
-    reg_fence64(s + 64);
-    float x[kBlockN];
+    ok = warp_wait(sm.s_full(t), j & 1, timeout);
+    const int kv0 = j * kBlockN + h * kCols;
+    // mask needed: key tail, or the causal diagonal (only tiles that reach past
+    // the tile's first row)
+    const bool masked = kv0 + kCols > prm.Nk || (CAUSAL && kv0 + kCols - 1 > tile_row0);
+    // load 32 score columns [32*k, 32*k + 32) of this warp's half as fp32,
+    // prescaled and masked
+    auto load_scores = [&](int k, float (&x)[32]) {
+      uint32_t s[32];
+      tmem_ld32(tS + 32 * k, s);
+      tmem_ld_wait();
+      reg_fence32(s);
 #pragma unroll
-    for (int c = 0; c < kBlockN; ++c) x[c] = __uint_as_float(s[c]);
-    if (prescale) {
+      for (int c = 0; c < 32; ++c) x[c] = __uint_as_float(s[c]);
+      if (prescale) {
 #pragma unroll
-      for (int c = 0; c < kBlockN; ++c) x[c] *= prm.scale_log2;
-    }
-    // mask: key tail, and the causal diagonal (only tiles that reach past the
-    // tile's first row need it).
-    const int kv0 = j * kBlockN;
-    if (kv0 + kBlockN > prm.Nk || (CAUSAL && kv0 + kBlockN - 1 > tile_row0)) {
-#pragma unroll
-      for (int c = 0; c < kBlockN; ++c) {
-        const int key = kv0 + c;
-        if (key >= prm.Nk || (CAUSAL && key > row)) x[c] = -INFINITY;
+        for (int c = 0; c < 32; ++c) x[c] *= prm.scale_log2;
       }
-    }
-    // row max: 3-input max, four independent chains over columns 0..127
-    float mx[4];
+      if (masked) {
 #pragma unroll
-    for (int a = 0; a < 4; ++a) mx[a] = fmaxf(x[2 * a], x[2 * a + 1]);
-#pragma unroll
-    for (int c = 8; c < kBlockN; c += 8) {
-#pragma unroll
-      for (int a = 0; a < 4; ++a) mx[a] = fmax3(mx[a], x[c + 2 * a], x[c + 2 * a + 1]);
-    }
-    const float m_tile = fmax3(fmaxf(mx[0], mx[1]), mx[2], mx[3]) * sl;
+        for (int c = 0; c < 32; ++c) {
+          const int key = kv0 + 32 * k + c;
+          if (key >= prm.Nk || (CAUSAL && key > row)) x[c] = -INFINITY;
+        }
+      }
+    };
 
-    // adaptive rescaling: move the reference only on a jump beyond tau
+    // pass 1: this half's row max
+    float mloc = __int_as_float(0x7fc00000);  // NaN marks a failed wait
+    if (ok) {
+      tc_fence_after();
+      float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+      for (int k = 0; k < 2; ++k) {
+        float x[32];
+        load_scores(k, x);
+#pragma unroll
+        for (int c = 0; c < 32; c += 8) {
+#pragma unroll
+          for (int a = 0; a < 4; ++a) mx[a] = fmax3(mx[a], x[c + 2 * a], x[c + 2 * a + 1]);
+        }
+      }
+      mloc = fmax3(fmaxf(mx[0], mx[1]), mx[2], mx[3]);
+    }
+    sm.xch(t, h, j & 1)[r] = mloc;
+    pair_sync(t, q4);
+    const float mother = sm.xch(t, h ^ 1, j & 1)[r];
+    if (!ok || isnan(mother)) {  // uniform across the pair
+      ok = false;
+      break;
+    }
+    const float m_tile = fmaxf(mloc, mother) * sl;
+
+    // adaptive rescaling: move the reference only on a jump beyond tau (both
+    // warps of the pair take the same decision from the same numbers)
     const bool resc = m_tile > m_run + prm.tau;
     float alpha = 1.0f;
     if (resc) {
@@ -367,38 +414,22 @@ __device__ __forceinline__ void softmax_role(const Smem<D>& sm, uint32_t tmem,
       m_run = m_tile;
     }
     l_run *= alpha;
-    // Correction: rescale this row's O accumulator (already final up to tile
-    // j-1, see the MMA order) by alpha before O += P V_j is issued.
-    if (j > 0 && __any_sync(0xffffffffu, resc)) {
-      if (prm.rescale_count) {
-        const unsigned n = __popc(__ballot_sync(0xffffffffu, resc));
-        if (lane == 0) atomicAdd(prm.rescale_count, static_cast<unsigned long long>(n));
-      }
-#pragma unroll
-      for (int cc = 0; cc < D / 32; ++cc) {
-        uint32_t o[32];
-        tmem_ld32(tO + cc * 32, o);
-        tmem_ld_wait();
-        reg_fence32(o);
-#pragma unroll
-        for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-        tmem_st32(tO + cc * 32, o);
-      }
-    }
 
-    // P = 2^(x*sl - m) in two halves of 64 keys; each half is stored to TMEM
-    // and announced on its own barrier so the MMA of the first half overlaps
-    // the exponentials of the second.
+    // pass 2: P = 2^(x*sl - m), 32 scores at a time (re-read from TMEM) ->
+    // BF16 pairs in the first 32 TMEM columns of this warp's half of S_t.
+    // Chunk k's P lands in columns [16k, 16k+16), which chunk k has consumed.
     const float neg_m = (m_run == -INFINITY) ? 0.0f : -m_run;
     const float2 sl2 = make_float2(sl, sl), nm2 = make_float2(neg_m, neg_m);
     float2 sum2[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
                       make_float2(0.f, 0.f)};
 #pragma unroll
-    for (int half = 0; half < 2; ++half) {
-      uint32_t p[32];
+    for (int k = 0; k < 2; ++k) {
+      float x[32];
+      load_scores(k, x);
+      uint32_t p[16];
 #pragma unroll
-      for (int i = 0; i < 32; ++i) {
-        const int c = half * 64 + 2 * i;
+      for (int i = 0; i < 16; ++i) {
+        const int c = 2 * i;
         const float2 u = ffma2(make_float2(x[c], x[c + 1]), sl2, nm2);
         float2 e;
         if ((c & 15) < POLY16) {
@@ -410,27 +441,53 @@ __device__ __forceinline__ void softmax_role(const Smem<D>& sm, uint32_t tmem,
         sum2[i & 3] = fadd2(sum2[i & 3], e);
         p[i] = pack_bf16x2(e.x, e.y);
       }
-      tmem_st32(tS + half * 32, p);
-      tmem_st_wait();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(sm.p_full(t, half));
+      tmem_st16(tS + 16 * k, p);
     }
     const float2 s01 = fadd2(sum2[0], sum2[1]), s23 = fadd2(sum2[2], sum2[3]);
     const float2 s03 = fadd2(s01, s23);
     l_run += s03.x + s03.y;
+
+    // Correction: rescale this warp's half of the row's O accumulator (final up
+    // to tile j-1, see the MMA order) by alpha before O += P V_j is issued.
+    if (j > 0 && __any_sync(0xffffffffu, resc)) {
+      if (prm.rescale_count && h == 0) {
+        const unsigned n = __popc(__ballot_sync(0xffffffffu, resc));
+        if (lane == 0) atomicAdd(prm.rescale_count, static_cast<unsigned long long>(n));
+      }
+#pragma unroll
+      for (int cc = 0; cc < kOCols / 32; ++cc) {
+        uint32_t o[32];
+        tmem_ld32(tO + cc * 32, o);
+        tmem_ld_wait();
+        reg_fence32(o);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+        tmem_st32(tO + cc * 32, o);
+      }
+    }
+    tmem_st_wait();
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(sm.p_full(t));
   }
 
-  if (ok) ok = warp_wait(sm.o_full(t), 0, timeout);
-  if (ok) {
+  // Epilogue.  Both warps of the pair reach both exchanges below whatever
+  // happened above.
+  const bool ok2 = ok && warp_wait(sm.o_full(t), 0, timeout);
+  sm.xch(t, h, 0)[r] = ok2 ? l_run : __int_as_float(0x7fc00000);
+  pair_sync(t, q4);
+  const float lother = sm.xch(t, h ^ 1, 0)[r];
+  const bool ok3 = ok2 && !isnan(lother);
+  uint8_t* sOt = sm.base + C::kOffQ + t * C::kTileBytes;
+  const float l_tot = l_run + lother;
+  if (ok3) {
     tc_fence_after();
-    // Epilogue: O / l -> BF16 -> this tile's Q buffer (its last reader, the
-    // final S MMA, finished before the last O MMA) in the 128-byte swizzled
-    // layout the O tensor map expects -> one TMA store per warp (32 rows).
-    const float inv_l = l_run > 0.0f ? 1.0f / l_run : 0.0f;
-    uint8_t* sOt = sm.base + C::kOffQ + t * C::kTileBytes;
+    // O / l -> BF16 -> this tile's Q buffer (its last reader, the final S MMA,
+    // finished before the last O MMA) in the 128-byte swizzled layout the O
+    // tensor map expects.  Warp h writes output columns [h*d/2, (h+1)*d/2).
+    const float inv_l = l_tot > 0.0f ? 1.0f / l_tot : 0.0f;
 #pragma unroll
-    for (int cc = 0; cc < D / 32; ++cc) {
+    for (int cc = 0; cc < kOCols / 32; ++cc) {
       uint32_t o[32];
       tmem_ld32(tO + cc * 32, o);
       tmem_ld_wait();
@@ -439,28 +496,33 @@ __device__ __forceinline__ void softmax_role(const Smem<D>& sm, uint32_t tmem,
 #pragma unroll
       for (int i = 0; i < 16; ++i)
         w[i] = pack_bf16x2(__uint_as_float(o[2 * i]) * inv_l, __uint_as_float(o[2 * i + 1]) * inv_l);
-      uint8_t* rowp = sOt + (cc >> 1) * C::kBoxBytes + r * 128;
+      const int col0 = h * kOCols + cc * 32;  // first output column of this chunk
+      uint8_t* rowp = sOt + (col0 >> 6) * C::kBoxBytes + r * 128;
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
-        const int chunk = (((cc & 1) * 4) + i) ^ (r & 7);
-        *reinterpret_cast<uint4*>(rowp + chunk * 16) = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
+        const int chunk = (((col0 & 63) >> 3) + i) ^ (r & 7);
+        *reinterpret_cast<uint4*>(rowp + chunk * 16) =
+            make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
       }
     }
     fence_proxy_async_smem();
-    __syncwarp();
-    if (lane == 0 && tile_row0 + q4 * 32 < prm.Nq) {
-#pragma unroll
-      for (int b = 0; b < C::kBoxes; ++b)
-        tma_store_3d(tm_o, smem_u32(sOt + b * C::kBoxBytes + q4 * 32 * 128), b * 64, tile_row0 + q4 * 32, bh);
-      bulk_commit_group();
-      bulk_wait_group_read0();
-    }
-    if (prm.lse != nullptr && row < prm.Nq) {
-      const float m_use = (m_run == -INFINITY) ? 0.0f : m_run;
-      prm.lse[static_cast<size_t>(bh) * prm.Nq + row] = (m_use + log2f(l_run)) * kLn2;
-    }
   }
-  if (!ok && lane == 0) atomicOr(&g_status, kStatusTimeout);
+  // d = 128: each warp stores its own 64-column box; d = 64: the pair shares
+  // one box, stored by the h = 0 warp after both halves are written.
+  if (D == 64) pair_sync(t, q4);
+  __syncwarp();
+  if (ok3 && lane == 0 && tile_row0 + q4 * 32 < prm.Nq && (D == 128 || h == 0)) {
+    const int box = D == 128 ? h : 0;
+    tma_store_3d(tm_o, smem_u32(sOt + box * C::kBoxBytes + q4 * 32 * 128), box * 64,
+                 tile_row0 + q4 * 32, bh);
+    bulk_commit_group();
+    bulk_wait_group_read0();
+  }
+  if (ok3 && h == 0 && prm.lse != nullptr && row < prm.Nq) {
+    const float m_use = (m_run == -INFINITY) ? 0.0f : m_run;
+    prm.lse[static_cast<size_t>(bh) * prm.Nq + row] = (m_use + log2f(l_tot)) * kLn2;
+  }
+  if (!ok3 && lane == 0) atomicOr(&g_status, kStatusTimeout);
 }
 
 // ---------------------------------------------------------------------------
@@ -500,10 +562,9 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   if (threadIdx.x == 0) {
     for (int i = 0; i < C::kNumBars; ++i) {
       const uint32_t b = sm.bar(i);
-      // p_full: one arrival per softmax warp of the tile; everything else: one.
-      const bool pf = b == sm.p_full(0, 0) || b == sm.p_full(0, 1) || b == sm.p_full(1, 0) ||
-                      b == sm.p_full(1, 1);
-      mbar_init(b, pf ? 4u : 1u);
+      // p_full: one arrival per softmax warp of the tile (8); everything else: one.
+      const bool pf = b == sm.p_full(0) || b == sm.p_full(1);
+      mbar_init(b, pf ? 8u : 1u);
     }
     fence_barrier_init();
     fence_proxy_async_smem();
