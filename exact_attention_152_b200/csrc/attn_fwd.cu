@@ -96,7 +96,7 @@ struct Cfg {
   static constexpr int kOffQ = 0;
   static constexpr int kOffKV = 2 * kTileBytes;
   static constexpr int kOffBar = kOffKV + kStages * kTileBytes;
-  static constexpr int kNumBars = 2 + 2 * kStages + 2 + 2 + 2 + 1;
+  static constexpr int kNumBars = 2 + 2 * kStages + 2 + 4 + 2 + 1;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
   // row-max / row-sum exchange between the two key halves of a row:
   // float [tile 2][half 2][parity 2][row 128]
@@ -135,10 +135,13 @@ struct Smem {
   __device__ __forceinline__ uint32_t kv_full(int s) const { return bar(2 + s); }
   __device__ __forceinline__ uint32_t kv_empty(int s) const { return bar(2 + Cfg<D>::kStages + s); }
   __device__ __forceinline__ uint32_t s_full(int t) const { return bar(2 + 2 * Cfg<D>::kStages + t); }
-  // P of tile t written to TMEM (and O_t rescaled) by all 8 warps of the tile
-  __device__ __forceinline__ uint32_t p_full(int t) const { return bar(4 + 2 * Cfg<D>::kStages + t); }
-  __device__ __forceinline__ uint32_t o_full(int t) const { return bar(6 + 2 * Cfg<D>::kStages + t); }
-  __device__ __forceinline__ uint32_t mma_done() const { return bar(8 + 2 * Cfg<D>::kStages); }
+  // chunk k of P_t (keys [32k, 32k+32) and [64+32k, 96+32k)) written to TMEM by
+  // all 8 warps of the tile (chunk 0 also marks O_t as rescaled)
+  __device__ __forceinline__ uint32_t p_full(int t, int k) const {
+    return bar(4 + 2 * Cfg<D>::kStages + 2 * t + k);
+  }
+  __device__ __forceinline__ uint32_t o_full(int t) const { return bar(8 + 2 * Cfg<D>::kStages + t); }
+  __device__ __forceinline__ uint32_t mma_done() const { return bar(10 + 2 * Cfg<D>::kStages); }
   __device__ __forceinline__ float* xch(int t, int h, int par) const {
     return reinterpret_cast<float*>(base + Cfg<D>::kOffXch) + ((t * 2 + h) * 2 + par) * kBlockM;
   }
@@ -212,15 +215,19 @@ struct MmaUnroll {
       MmaUnroll<D, KK + 1>::s(d, a_lo, a_hi, b_lo, b_hi, idesc);
     }
   }
-  // O += P V, K steps KK .. 7: P of keys [64h, 64h+64) in TMEM columns
-  // [64h, 64h+32) (two bf16 per column); V rows of 16 keys = 2048 bytes.
+  // O += P V for P chunk CH: K steps {2CH, 2CH+1} (keys [32CH, 32CH+32)) and
+  // {4+2CH, 5+2CH} (keys [64+32CH, 96+32CH)).  P of keys [64h, 64h+64) sits in
+  // TMEM columns [64h, 64h+32) (two bf16 per column); V rows of 16 keys =
+  // 2048 bytes.  KK counts 0..3 within the chunk.
+  template <int CH>
   __device__ __forceinline__ static void o(uint32_t d, uint32_t a_tmem, uint32_t b_lo, uint32_t b_hi,
                                            uint32_t idesc, uint32_t acc) {
-    if constexpr (KK < kBlockN / 16) {
-      constexpr uint32_t a_off = (KK >> 2) * 64 + (KK & 3) * 8;
-      constexpr uint32_t b_off = (KK * 2048) >> 4;
-      mma_ts_imm<a_off, b_off>(d, a_tmem, b_lo, b_hi, idesc, KK == 0 ? acc : 1u);
-      MmaUnroll<D, KK + 1>::o(d, a_tmem, b_lo, b_hi, idesc, acc);
+    if constexpr (KK < 4) {
+      constexpr int step = (KK >> 1) * 4 + 2 * CH + (KK & 1);  // K step among 0..7
+      constexpr uint32_t a_off = (step >> 2) * 64 + (step & 3) * 8;
+      constexpr uint32_t b_off = (step * 2048) >> 4;
+      mma_ts_imm<a_off, b_off>(d, a_tmem, b_lo, b_hi, idesc, (CH == 0 && KK == 0) ? acc : 1u);
+      MmaUnroll<D, KK + 1>::template o<CH>(d, a_tmem, b_lo, b_hi, idesc, acc);
     }
   }
 };
@@ -256,11 +263,17 @@ __device__ __forceinline__ void mma_role(const Smem<D>& sm, uint32_t tmem, int n
     MmaUnroll<D, 0>::s(tmem + t * kBlockM, q_lo + t * kTileStep, q_hi, k_lo + slot * kTileStep,
                        k_hi, idesc_s);
   };
+  // O_t += P_t V in two chunks, each issued as soon as the softmax warps have
+  // stored it
   auto mma_o = [&](int t, uint32_t slot, bool acc, uint32_t par) -> bool {
-    if (!mbar_wait(sm.p_full(t), par, timeout)) return false;
+    const uint32_t d = tmem + C::kTmemO + t * D, a = tmem + t * kBlockM;
+    const uint32_t b_lo = v_lo + slot * kTileStep;
+    if (!mbar_wait(sm.p_full(t, 0), par, timeout)) return false;
     tc_fence_after();
-    MmaUnroll<D, 0>::o(tmem + C::kTmemO + t * D, tmem + t * kBlockM, v_lo + slot * kTileStep, v_hi,
-                       idesc_o, acc ? 1u : 0u);
+    MmaUnroll<D, 0>::template o<0>(d, a, b_lo, v_hi, idesc_o, acc ? 1u : 0u);
+    if (!mbar_wait(sm.p_full(t, 1), par, timeout)) return false;
+    tc_fence_after();
+    MmaUnroll<D, 0>::template o<1>(d, a, b_lo, v_hi, idesc_o, 1u);
     return true;
   };
 
@@ -415,9 +428,30 @@ __device__ __forceinline__ void softmax_role(const Smem<D>& sm, uint32_t tmem,
     }
     l_run *= alpha;
 
+    // Correction: rescale this warp's half of the row's O accumulator (final up
+    // to tile j-1, see the MMA order) by alpha before O += P V_j is issued.
+    if (j > 0 && __any_sync(0xffffffffu, resc)) {
+      if (prm.rescale_count && h == 0) {
+        const unsigned n = __popc(__ballot_sync(0xffffffffu, resc));
+        if (lane == 0) atomicAdd(prm.rescale_count, static_cast<unsigned long long>(n));
+      }
+#pragma unroll
+      for (int cc = 0; cc < kOCols / 32; ++cc) {
+        uint32_t o[32];
+        tmem_ld32(tO + cc * 32, o);
+        tmem_ld_wait();
+        reg_fence32(o);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+        tmem_st32(tO + cc * 32, o);
+      }
+    }
+
     // pass 2: P = 2^(x*sl - m), 32 scores at a time (re-read from TMEM) ->
     // BF16 pairs in the first 32 TMEM columns of this warp's half of S_t.
-    // Chunk k's P lands in columns [16k, 16k+16), which chunk k has consumed.
+    // Chunk k's P lands in columns [16k, 16k+16), which chunk k has consumed,
+    // and is announced on its own barrier so its O += P V can start while the
+    // next chunk is being exponentiated.
     const float neg_m = (m_run == -INFINITY) ? 0.0f : -m_run;
     const float2 sl2 = make_float2(sl, sl), nm2 = make_float2(neg_m, neg_m);
     float2 sum2[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
@@ -442,33 +476,14 @@ __device__ __forceinline__ void softmax_role(const Smem<D>& sm, uint32_t tmem,
         p[i] = pack_bf16x2(e.x, e.y);
       }
       tmem_st16(tS + 16 * k, p);
+      tmem_st_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(sm.p_full(t, k));
     }
     const float2 s01 = fadd2(sum2[0], sum2[1]), s23 = fadd2(sum2[2], sum2[3]);
     const float2 s03 = fadd2(s01, s23);
     l_run += s03.x + s03.y;
-
-    // Correction: rescale this warp's half of the row's O accumulator (final up
-    // to tile j-1, see the MMA order) by alpha before O += P V_j is issued.
-    if (j > 0 && __any_sync(0xffffffffu, resc)) {
-      if (prm.rescale_count && h == 0) {
-        const unsigned n = __popc(__ballot_sync(0xffffffffu, resc));
-        if (lane == 0) atomicAdd(prm.rescale_count, static_cast<unsigned long long>(n));
-      }
-#pragma unroll
-      for (int cc = 0; cc < kOCols / 32; ++cc) {
-        uint32_t o[32];
-        tmem_ld32(tO + cc * 32, o);
-        tmem_ld_wait();
-        reg_fence32(o);
-#pragma unroll
-        for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-        tmem_st32(tO + cc * 32, o);
-      }
-    }
-    tmem_st_wait();
-    tc_fence_before();
-    __syncwarp();
-    if (lane == 0) mbar_arrive(sm.p_full(t));
   }
 
   // Epilogue.  Both warps of the pair reach both exchanges below whatever
@@ -563,7 +578,8 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     for (int i = 0; i < C::kNumBars; ++i) {
       const uint32_t b = sm.bar(i);
       // p_full: one arrival per softmax warp of the tile (8); everything else: one.
-      const bool pf = b == sm.p_full(0) || b == sm.p_full(1);
+      const bool pf = b == sm.p_full(0, 0) || b == sm.p_full(0, 1) || b == sm.p_full(1, 0) ||
+                      b == sm.p_full(1, 1);
       mbar_init(b, pf ? 8u : 1u);
     }
     fence_barrier_init();
