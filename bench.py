@@ -73,12 +73,19 @@ def load_peaks():
 
 
 def kernel_source_hash():
+    """Hash of the CUDA sources with comments and whitespace removed, so that a
+    recorded ncu capture stays attached to the code it measured."""
+    import re
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "exact_attention_152_b200", "csrc")
     for name in sorted(os.listdir(csrc)):
         if name.endswith((".cu", ".cuh", ".h")):
-            with open(os.path.join(csrc, name), "rb") as f:
-                h.update(name.encode() + b"\0" + f.read())
+            with open(os.path.join(csrc, name)) as f:
+                src = f.read()
+            src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+            src = re.sub(r"//[^\n]*", "", src)
+            src = "".join(src.split())
+            h.update(name.encode() + b"\0" + src.encode())
     return h.hexdigest()[:16]
 
 

@@ -27,19 +27,26 @@
 //    memory stages filled by TMA.  Q, K and V are read through 3-D tensor maps
 //    [B*H, N, d] so out-of-range rows of one head read as zeros, never as the
 //    next head's data.
-//  * Warps 0-3 / 4-7: softmax, correction and epilogue of query tile 0 / 1
-//    (one thread = one query row = one TMEM lane).  Warp 8: TMA producer.
-//    Warp 9: TMEM allocation and the single MMA-issuing thread.  Warps 10-11
-//    idle (they complete the third warpgroup for the setmaxnreg split).
+//  * 20 warps.  Warps 0-15 do softmax, correction and epilogue: tile t uses
+//    warps 8t..8t+7; warp (t, h, q) owns TMEM lanes 32q..32q+31 (its 32 query
+//    rows) and the key columns [64h, 64h+64) of each S tile, and the output
+//    columns [h*d/2, (h+1)*d/2).  The two warps of a row pair swap their partial
+//    row maxima through shared memory.  Warp 16: TMA producer.  Warp 17: TMEM
+//    allocation and the single MMA-issuing thread.  Warps 18-19 idle (they
+//    complete the fifth warpgroup for the setmaxnreg split 104 / 40).
 //  * Tensor Memory (512 columns): S0 [0,128), S1 [128,256), O0 and O1 after
-//    column 256.  P (BF16) overwrites the first 64 columns of its S tile and is
-//    the A operand of O += P V straight from TMEM, so P never touches shared
-//    memory.
+//    column 256.  P (BF16 pairs) overwrites the first half of each warp's part
+//    of S and is the A operand of O += P V straight from TMEM, so P never
+//    touches shared memory.
 //  * The MMA thread issues, per KV tile j:  O0 += P0 V_{j-1};  S0 = Q0 K_j^T;
-//    O1 += P1 V_{j-1};  S1 = Q1 K_j^T.  Each O += P V is issued in two halves
-//    of 64 keys, each as soon as the softmax warps have stored that half of P.  The commit that announces S_t(j) also
-//    covers O_t += P_t V_{j-1}, so when a softmax warp sees S_t(j) its O_t is
-//    final up to tile j-1 and it can rescale O_t in place without another wait.
+//    O1 += P1 V_{j-1};  S1 = Q1 K_j^T.  Each O += P V is issued in two chunks,
+//    each as soon as the softmax warps have stored that chunk of P.  The
+//    commit that announces S_t(j) also covers O_t += P_t V_{j-1}, so when a
+//    softmax warp sees S_t(j) its O_t is final up to tile j-1 and it can
+//    rescale O_t in place without another wait.
+//  * MMAs are issued from fully unrolled code with descriptor offsets as
+//    immediates: the tensor core queues about one MMA ahead, so every cycle
+//    the issuing thread spends between MMAs is a cycle the tensor core idles.
 //  * Every wait is bounded (see sm100.cuh); a timeout sets the per-device
 //    status word and the CTA leaves its loops and exits cleanly.
 #include <cuda.h>
