@@ -57,8 +57,8 @@ def parse_args(argv=None):
 
 
 def dist_env():
-    return (int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")),
-            int(os.environ.get("LOCAL_RANK", "0")))
+    from exact_attention_152_b200 import parallel
+    return parallel.rank_env()
 
 
 def load_peaks():
@@ -262,15 +262,14 @@ def run_ours(args):
     import torch
     import torch.distributed as dist
 
-    from exact_attention_152_b200 import binding
+    from exact_attention_152_b200 import binding, parallel
     from exact_attention_152_b200.workloads import HEADLINE, WORKLOADS
 
     rank, world, local_rank = dist_env()
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
     if world > 1:
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=dev)
+        parallel.init("nccl", timeout_s=120, device=dev)
     w = WORKLOADS[args.workload or HEADLINE]
     peaks = load_peaks()
 
@@ -323,10 +322,7 @@ def run_ours(args):
     total_ms = evs[0].elapsed_time(evs[K])
     per_launch = [evs[i].elapsed_time(evs[i + 1]) for i in range(K)]
     kernel_ms = sum(per_launch) / K
-    t = torch.tensor([total_ms, kernel_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    total_ms, kernel_ms = float(t[0]), float(t[1])
+    total_ms, kernel_ms = parallel.max_over_ranks([total_ms, kernel_ms], dev)
     value = world * w.flops * K / (total_ms / 1e3) / 1e12
     achieved = w.flops / (kernel_ms / 1e3) / 1e12
 
@@ -360,10 +356,8 @@ def run_ours(args):
     if world > 1:
         dist.barrier()
     binding.check(binding.attn_status_sync(sh), "e2e region")
-    te = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(te, op=dist.ReduceOp.MAX)
-    e2e_value = world * w.flops * KE / (float(te[0]) / 1e3) / 1e12
+    (te_ms,) = parallel.max_over_ranks([e0.elapsed_time(e1)], dev)
+    e2e_value = world * w.flops * KE / (te_ms / 1e3) / 1e12
     h2d = sum(x.numel() * x.element_size() for x in (hq, hk, hv))
     d2h = ho.numel() * ho.element_size() + hl.numel() * hl.element_size()
 
