@@ -19,7 +19,6 @@ workload, in the same metric.
 from __future__ import annotations
 
 import argparse
-import datetime
 import hashlib
 import json
 import math

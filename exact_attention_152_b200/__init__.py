@@ -10,7 +10,7 @@ raises ImportError -- there is no fallback of any kind.
 from __future__ import annotations
 
 __all__ = [
-    "attn_fwd", "attn_fwd_config", "attn_status_sync", "attn_status_string",
+    "attn_fwd", "attn_fwd_config", "attn_fwd_gqa", "attn_status_sync", "attn_status_string",
     "attn_last_error", "attn_selftest_timeout", "fwd", "AttnError",
 ]
 

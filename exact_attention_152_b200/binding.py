@@ -45,6 +45,9 @@ def lib() -> ctypes.CDLL:
             l.attn_fwd_config.argtypes = [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, ctypes.c_float, _I,
                                           ctypes.c_float, _I, _P, _P]
             l.attn_fwd_config.restype = _I
+            l.attn_fwd_gqa.argtypes = [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, ctypes.c_float, _I,
+                                       _P]
+            l.attn_fwd_gqa.restype = _I
             l.attn_status_sync.argtypes = [_P]
             l.attn_status_sync.restype = _I
             l.attn_status_string.argtypes = [_I]
@@ -59,6 +62,10 @@ def lib() -> ctypes.CDLL:
 
 def attn_fwd(q, k, v, o, lse, B, H, Nq, Nk, d, scale, causal, stream) -> int:
     return lib().attn_fwd(q, k, v, o, lse, B, H, Nq, Nk, d, scale, causal, stream)
+
+
+def attn_fwd_gqa(q, k, v, o, lse, B, H, Hkv, Nq, Nk, d, scale, causal, stream) -> int:
+    return lib().attn_fwd_gqa(q, k, v, o, lse, B, H, Hkv, Nq, Nk, d, scale, causal, stream)
 
 
 def attn_fwd_config(q, k, v, o, lse, B, H, Nq, Nk, d, scale, causal, rescale_threshold,
@@ -100,8 +107,9 @@ def check(code: int, where: str = "attn") -> None:
 def fwd(q, k, v, causal: bool = False, scale: float | None = None, *, out=None, lse=None,
         return_lse: bool = True, rescale_threshold: float | None = None,
         exp_mode: int | None = None, rescale_count=None):
-    """O (and LSE) for BF16 CUDA tensors q [B,H,Nq,d], k/v [B,H,Nk,d].
+    """O (and LSE) for BF16 CUDA tensors q [B,H,Nq,d], k/v [B,Hkv,Nk,d].
 
+    Hkv < H (H % Hkv == 0) selects grouped-query attention (attn_fwd_gqa).
     scale defaults to 1/sqrt(d).  Runs on torch's current stream; returns
     (o, lse) or o.  Raises AttnError on any non-zero status.
     """
@@ -113,9 +121,9 @@ def fwd(q, k, v, causal: bool = False, scale: float | None = None, *, out=None, 
         if t.dim() != 4 or not t.is_contiguous():
             raise ValueError(f"{name} must be contiguous [B, H, N, d]")
     B, H, Nq, d = q.shape
-    Nk = k.shape[2]
-    if tuple(k.shape) != (B, H, Nk, d) or tuple(v.shape) != (B, H, Nk, d):
-        raise ValueError("k and v must be [B, H, Nk, d] matching q")
+    Hkv, Nk = k.shape[1], k.shape[2]
+    if tuple(k.shape) != (B, Hkv, Nk, d) or tuple(v.shape) != (B, Hkv, Nk, d):
+        raise ValueError("k and v must be [B, Hkv, Nk, d] matching q")
     if scale is None:
         scale = 1.0 / math.sqrt(d)
     if out is None:
@@ -124,7 +132,12 @@ def fwd(q, k, v, causal: bool = False, scale: float | None = None, *, out=None, 
         lse = torch.empty((B, H, Nq), dtype=torch.float32, device=q.device)
     stream = torch.cuda.current_stream(q.device).cuda_stream
     lse_ptr = lse.data_ptr() if lse is not None else None
-    if rescale_threshold is None and exp_mode is None and rescale_count is None:
+    if Hkv != H:
+        if rescale_threshold is not None or exp_mode is not None or rescale_count is not None:
+            raise ValueError("the softmax knobs are available for Hkv == H only")
+        rc = attn_fwd_gqa(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse_ptr,
+                          B, H, Hkv, Nq, Nk, d, float(scale), int(bool(causal)), stream)
+    elif rescale_threshold is None and exp_mode is None and rescale_count is None:
         rc = attn_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse_ptr,
                       B, H, Nq, Nk, d, float(scale), int(bool(causal)), stream)
     else:

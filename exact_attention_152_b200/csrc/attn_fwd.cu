@@ -118,6 +118,8 @@ struct FwdParams {
   unsigned long long* rescale_count;
   uint64_t timeout_ns;
   int Nq, Nk, BH, n_qblocks;
+  int H, group;      // query heads per batch; query heads per key/value head
+  int hgroup;        // causal order: heads scheduled together (their K/V fit in L2)
   float scale_log2;  // scale * log2(e)
   float tau;         // rescale threshold, powers of two
 };
@@ -170,7 +172,8 @@ __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, uint64_
 template <int D>
 __device__ __forceinline__ void producer_role(const Smem<D>& sm, const CUtensorMap* tm_q,
                                               const CUtensorMap* tm_k, const CUtensorMap* tm_v,
-                                              int bh, int qb, int n_kv, uint64_t timeout) {
+                                              int bh, int bh_kv, int qb, int n_kv,
+                                              uint64_t timeout) {
   using C = Cfg<D>;
   uint32_t it = 0;
   auto load_q = [&](int t) {
@@ -187,7 +190,7 @@ __device__ __forceinline__ void producer_role(const Smem<D>& sm, const CUtensorM
     mbar_arrive_expect_tx(sm.kv_full(slot), C::kTileBytes);
 #pragma unroll
     for (int b = 0; b < C::kBoxes; ++b)
-      tma_load_3d(sm.kv(slot) + b * C::kBoxBytes, tm, b * 64, j * kBlockN, bh, sm.kv_full(slot));
+      tma_load_3d(sm.kv(slot) + b * C::kBoxBytes, tm, b * 64, j * kBlockN, bh_kv, sm.kv_full(slot));
     ++it;
     return true;
   };
@@ -567,17 +570,25 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   // Tile order.  Non-causal: head-major, so the CTAs resident at one time share
-  // a few heads' K/V in L2.  Causal: heaviest query blocks first across all
-  // heads, so the short blocks fill the tail.
+  // a few heads' K/V in L2.  Causal: heads in groups of hgroup (sized on the
+  // host so a group's K/V fits in L2), and within a group the heaviest query
+  // blocks first, so short blocks fill the tail of each group while the next
+  // group starts.
   const int tile = blockIdx.x;
   int bh, qb;
   if (CAUSAL) {
-    qb = prm.n_qblocks - 1 - tile / prm.BH;
-    bh = tile % prm.BH;
+    const int per_group = prm.hgroup * prm.n_qblocks;
+    const int g = tile / per_group, w = tile % per_group;
+    const int gsize = min(prm.hgroup, prm.BH - g * prm.hgroup);
+    qb = prm.n_qblocks - 1 - w / gsize;
+    bh = g * prm.hgroup + w % gsize;
   } else {
     bh = tile / prm.n_qblocks;
     qb = tile % prm.n_qblocks;
   }
+  // grouped-query attention: query head h of batch b reads key/value head
+  // h / group of the same batch (group = 1: one key/value head per query head)
+  const int bh_kv = (bh / prm.H) * (prm.H / prm.group) + (bh % prm.H) / prm.group;
   int n_kv = (prm.Nk + kBlockN - 1) / kBlockN;
   if (CAUSAL) n_kv = min(n_kv, (qb + 1) * (kRowsPerCta / kBlockN));
 
@@ -611,7 +622,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     // warpgroup 2: TMA producer (warp 8), MMA issuer (warp 9), two idle warps
     setmaxnreg_dec<kProducerRegs>();
     if (warp == kWarpLoad) {
-      if (lane == 0) producer_role<D>(sm, &tm_q, &tm_k, &tm_v, bh, qb, n_kv, prm.timeout_ns);
+      if (lane == 0) producer_role<D>(sm, &tm_q, &tm_k, &tm_v, bh, bh_kv, qb, n_kv, prm.timeout_ns);
       __syncwarp();
     } else if (warp == kWarpMma) {
       if (lane == 0) mma_role<D>(sm, tmem, n_kv, prm.timeout_ns);
@@ -723,9 +734,10 @@ int check_device() {
 }
 
 int fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
-             int Nq, int Nk, int d, float scale, int causal, float tau, int exp_mode,
+             int Hkv, int Nq, int Nk, int d, float scale, int causal, float tau, int exp_mode,
              unsigned long long* rescale_count, cudaStream_t stream) {
-  if (B < 0 || H < 0 || Nq < 0 || Nk < 0) return ATTN_ERR_INVALID_ARG;
+  if (B < 0 || H < 0 || Hkv < 0 || Nq < 0 || Nk < 0) return ATTN_ERR_INVALID_ARG;
+  if (H > 0 && (Hkv == 0 || H % Hkv != 0)) return ATTN_ERR_INVALID_ARG;
   if (!std::isfinite(scale)) return ATTN_ERR_INVALID_ARG;
   if (causal != 0 && causal != 1) return ATTN_ERR_INVALID_ARG;
   if (!(tau >= 0.0f && tau <= 64.0f)) return ATTN_ERR_UNSUPPORTED;
@@ -741,7 +753,8 @@ int fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, i
       misaligned(lse, 4) || misaligned(rescale_count, 8))
     return ATTN_ERR_INVALID_ARG;
   const size_t o_bytes = static_cast<size_t>(BH) * Nq * d * 2;
-  const size_t kv_bytes = static_cast<size_t>(BH) * Nk * d * 2;
+  const long long BHkv = static_cast<long long>(B) * Hkv;
+  const size_t kv_bytes = static_cast<size_t>(BHkv) * Nk * d * 2;
   const size_t lse_bytes = lse ? static_cast<size_t>(BH) * Nq * 4 : 0;
   if (ranges_overlap(o, o_bytes, q, o_bytes) || ranges_overlap(o, o_bytes, k, kv_bytes) ||
       ranges_overlap(o, o_bytes, v, kv_bytes) || ranges_overlap(lse, lse_bytes, q, o_bytes) ||
@@ -769,8 +782,8 @@ int fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, i
   CUtensorMap tq, tk, tv, to;
   const int bh = static_cast<int>(BH);
   if (!make_tmap_bf16_3d(&tq, q, bh, Nq, d, kBlockM, &t_last_error) ||
-      !make_tmap_bf16_3d(&tk, k, bh, Nk, d, kBlockN, &t_last_error) ||
-      !make_tmap_bf16_3d(&tv, v, bh, Nk, d, kBlockN, &t_last_error) ||
+      !make_tmap_bf16_3d(&tk, k, static_cast<int>(BHkv), Nk, d, kBlockN, &t_last_error) ||
+      !make_tmap_bf16_3d(&tv, v, static_cast<int>(BHkv), Nk, d, kBlockN, &t_last_error) ||
       !make_tmap_bf16_3d(&to, o, bh, Nq, d, 32, &t_last_error))
     return ATTN_ERR_CUDA;
 
@@ -781,6 +794,16 @@ int fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, i
   prm.Nq = Nq;
   prm.Nk = Nk;
   prm.BH = static_cast<int>(BH);
+  prm.H = H;
+  prm.group = H / Hkv;
+  {
+    // causal schedule: as many heads at once as keep their K/V within ~48 MB
+    // of the 126 MB L2 (several query heads of a GQA group share one K/V head)
+    const double kv_head_bytes = 2.0 * Nk * d * 2.0 / prm.group;
+    const double budget = 48.0 * 1024 * 1024;
+    long long g = static_cast<long long>(budget / std::max(kv_head_bytes, 1.0));
+    prm.hgroup = static_cast<int>(std::max(1LL, std::min(g, BH)));
+  }
   prm.n_qblocks = static_cast<int>(n_qblocks);
   prm.scale_log2 = scale * kLog2e;
   prm.tau = tau;
@@ -799,15 +822,21 @@ extern "C" {
 
 int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
              int Nq, int Nk, int d, float scale, int causal, cudaStream_t stream) {
-  return eab::fwd_impl(q, k, v, o, lse, B, H, Nq, Nk, d, scale, causal, eab::kDefaultThreshold, 1,
-                       nullptr, stream);
+  return eab::fwd_impl(q, k, v, o, lse, B, H, H, Nq, Nk, d, scale, causal, eab::kDefaultThreshold,
+                       1, nullptr, stream);
+}
+
+int attn_fwd_gqa(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
+                 int Hkv, int Nq, int Nk, int d, float scale, int causal, cudaStream_t stream) {
+  return eab::fwd_impl(q, k, v, o, lse, B, H, Hkv, Nq, Nk, d, scale, causal,
+                       eab::kDefaultThreshold, 1, nullptr, stream);
 }
 
 int attn_fwd_config(const void* q, const void* k, const void* v, void* o, float* lse, int B,
                     int H, int Nq, int Nk, int d, float scale, int causal,
                     float rescale_threshold, int exp_mode, unsigned long long* rescale_count,
                     cudaStream_t stream) {
-  return eab::fwd_impl(q, k, v, o, lse, B, H, Nq, Nk, d, scale, causal, rescale_threshold,
+  return eab::fwd_impl(q, k, v, o, lse, B, H, H, Nq, Nk, d, scale, causal, rescale_threshold,
                        exp_mode, rescale_count, stream);
 }
 

@@ -76,6 +76,20 @@ int attn_fwd(const void *q, const void *k, const void *v, void *o, float *lse, i
              int Nq, int Nk, int d, float scale, int causal, cudaStream_t stream);
 
 /*
+ * Grouped-query / multi-query attention (same contract as attn_fwd otherwise).
+ * The pages list GQA/MQA among what FlashAttention 4's forward still lacks
+ * (FlashAttention 4 page, ja.linux-konsole.com, sections "重要ポイント" and
+ * "互換性と現状"): several query heads share one key/value head.
+ *   q, o : [B, H, Nq, d];   k, v : [B, Hkv, Nk, d];   lse : [B, H, Nq]
+ *   Hkv  : key/value heads, 1 <= Hkv <= H with H % Hkv == 0 (Hkv == 1 is
+ *          multi-query attention, Hkv == H is attn_fwd)
+ * Query head h of batch b attends to key/value head h / (H / Hkv) of batch b.
+ * H % Hkv != 0 or Hkv <= 0 with H > 0 returns ATTN_ERR_INVALID_ARG.
+ */
+int attn_fwd_gqa(const void *q, const void *k, const void *v, void *o, float *lse, int B, int H,
+                 int Hkv, int Nq, int Nk, int d, float scale, int causal, cudaStream_t stream);
+
+/*
  * attn_fwd with the kernel's two softmax knobs exposed (same contract otherwise).
  *
  *   rescale_threshold : adaptive online rescaling (FlashAttention 4 page,

@@ -48,7 +48,7 @@ def test_library_exports_every_declared_symbol(header):
 
 def test_attn_h_declares_the_contract():
     names = declared_functions(os.path.join(ROOT, "include", "attn.h"))
-    for n in ("attn_fwd", "attn_fwd_config", "attn_status_sync", "attn_status_string",
+    for n in ("attn_fwd", "attn_fwd_config", "attn_fwd_gqa", "attn_status_sync", "attn_status_string",
               "attn_last_error", "attn_selftest_timeout"):
         assert n in names
 
@@ -93,6 +93,18 @@ ALIGNED = 0x10000  # fake, never dereferenced: every case below fails validation
 ])
 def test_host_validation(args, expect):
     assert F(*args, None) == expect
+
+
+def test_gqa_validation():
+    base = (ALIGNED, ALIGNED, ALIGNED, ALIGNED * 16, None, 1)
+    # H % Hkv != 0, Hkv == 0, negative Hkv
+    assert binding.attn_fwd_gqa(*base, 6, 4, 8, 8, 64, 0.1, 0, None) == 1
+    assert binding.attn_fwd_gqa(*base, 6, 0, 8, 8, 64, 0.1, 0, None) == 1
+    assert binding.attn_fwd_gqa(*base, 6, -2, 8, 8, 64, 0.1, 0, None) == 1
+    # empty problem stays a no-op
+    assert binding.attn_fwd_gqa(None, None, None, None, None, 0, 6, 2, 8, 8, 64, 0.1, 0, None) == 0
+    # the other checks still apply
+    assert binding.attn_fwd_gqa(*base, 6, 2, 8, 8, 96, 0.1, 0, None) == 2
 
 
 def test_config_knob_validation():
