@@ -182,8 +182,8 @@ def time_oracle_rows(w, n_rows, seed_off):
     bh = 0
     while done < n_rows and bh < w.B * w.H:
         take = min(w.Nq, n_rows - done)
-        k = inputs.bf16_bits_to_f64(w.head_bits("k", bh))
-        v = inputs.bf16_bits_to_f64(w.head_bits("v", bh))
+        k = inputs.bf16_bits_to_f64(w.head_bits("k", w.kv_head_of(bh)))
+        v = inputs.bf16_bits_to_f64(w.head_bits("v", w.kv_head_of(bh)))
         rows = inputs.sample_rows(w.seed + seed_off, bh, w.Nq, take)
         q = inputs.bf16_bits_to_f64(w.q_rows_bits(bh, rows))
         t0 = time.perf_counter()
@@ -213,8 +213,8 @@ def cpu_baseline(w, seconds):
 
 
 def workload_config(w, n_gpus):
-    qkv_bytes = (w.B * w.H * (w.Nq + 2 * w.Nk) * w.d * 2)
-    return {"workload": w.name, "B": w.B, "H": w.H, "Nq": w.Nq, "Nk": w.Nk, "d": w.d,
+    qkv_bytes = (w.B * (w.H * w.Nq + 2 * w.kv_heads * w.Nk) * w.d * 2)
+    return {"workload": w.name, "B": w.B, "H": w.H, "Hkv": w.kv_heads, "Nq": w.Nq, "Nk": w.Nk, "d": w.d,
             "causal": w.causal, "scale": w.scale, "seed": w.seed, "per_gpu_problem": True,
             "global_batch": w.B * n_gpus,
             "l2": f"inputs {qkv_bytes / 1e6:.0f} MB {'>' if qkv_bytes > L2_BYTES else '<='} "
@@ -284,7 +284,11 @@ def run_ours(args):
     em = 1 if args.exp_mode is None else args.exp_mode
 
     def launch(qp=q, kp=k, vp=v, op=o, lp=lse):
-        if knobs:
+        if w.kv_heads != w.H:
+            rc = binding.attn_fwd_gqa(qp.data_ptr(), kp.data_ptr(), vp.data_ptr(), op.data_ptr(),
+                                      lp.data_ptr(), w.B, w.H, w.kv_heads, w.Nq, w.Nk, w.d, w.scale,
+                                      int(w.causal), sh)
+        elif knobs:
             rc = binding.attn_fwd_config(qp.data_ptr(), kp.data_ptr(), vp.data_ptr(), op.data_ptr(),
                                          lp.data_ptr(), w.B, w.H, w.Nq, w.Nk, w.d, w.scale,
                                          int(w.causal), thr, em, None, sh)

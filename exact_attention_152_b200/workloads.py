@@ -31,6 +31,11 @@ class Workload:
     k_dist: str = "normal"
     v_dist: str = "normal"
     oracle_rows: int | None = None  # sampled rows per head for the oracle; None = all
+    Hkv: int | None = None          # key/value heads (grouped-query attention); None = H
+
+    @property
+    def kv_heads(self) -> int:
+        return self.H if self.Hkv is None else self.Hkv
 
     @property
     def scale(self) -> float:
@@ -43,8 +48,9 @@ class Workload:
         return f / 2 if self.causal else f
 
     def shape(self, which: str):
-        n = self.Nq if which == "q" else self.Nk
-        return (self.B, self.H, n, self.d)
+        if which == "q":
+            return (self.B, self.H, self.Nq, self.d)
+        return (self.B, self.kv_heads, self.Nk, self.d)
 
     def dist(self, which: str):
         if which == "q":
@@ -58,7 +64,8 @@ class Workload:
         return inputs.gen_bf16(self.seed, which, self.shape(which), dist, mult)
 
     def head_bits(self, which: str, bh: int) -> np.ndarray:
-        """BF16 bits of one (b, h) slice, [N, d]."""
+        """BF16 bits of one (b, h) slice, [N, d]; for k/v, bh indexes the B*Hkv
+        key/value heads (see kv_head_of)."""
         dist, mult = self.dist(which)
         n = self.Nq if which == "q" else self.Nk
         base = bh * n * self.d
@@ -70,6 +77,11 @@ class Workload:
         base = bh * self.Nq * self.d
         idx = base + rows.astype(np.int64)[:, None] * self.d + np.arange(self.d, dtype=np.int64)[None, :]
         return inputs.gen_bf16_at(self.seed, "q", idx, dist, mult)
+
+    def kv_head_of(self, bh: int) -> int:
+        """Flattened key/value head read by flattened query head bh."""
+        b, h = divmod(bh, self.H)
+        return b * self.kv_heads + h // (self.H // self.kv_heads)
 
     def sampled_rows(self, bh: int) -> np.ndarray:
         if self.oracle_rows is None:
@@ -88,6 +100,10 @@ WORKLOADS = {
                  q_mult=8.0, v_dist="uniform", oracle_rows=256),
         Workload("long_b1h16n128k_d128_causal", 1, 16, 131072, 131072, 128, True, seed=4,
                  oracle_rows=256),
+        Workload("gqa_b2h32kv8n8k_d128", 2, 32, 8192, 8192, 128, False, seed=5, oracle_rows=128,
+                 Hkv=8),
+        Workload("gqa_b2h32kv8n8k_d128_causal", 2, 32, 8192, 8192, 128, True, seed=5,
+                 oracle_rows=128, Hkv=8),
     ]
 }
 

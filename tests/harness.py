@@ -35,8 +35,9 @@ def run_cuda(q_bits, k_bits, v_bits, scale, causal, **kw):
     return o.float().cpu().numpy(), lse.cpu().numpy()
 
 
-def oracle_rows(q_bits, k_bits, v_bits, scale, causal, rows_per_head=None):
-    """Oracle on selected rows of every (b, h).  rows_per_head: dict bh -> rows or None (all)."""
+def oracle_rows(q_bits, k_bits, v_bits, scale, causal, rows_per_head=None, kv_group=1):
+    """Oracle on selected rows of every (b, h).  rows_per_head: dict bh -> rows or None (all).
+    kv_group > 1: query head h reads key/value head h // kv_group."""
     B, H, Nq, d = q_bits.shape
     out = {}
     for b in range(B):
@@ -44,8 +45,8 @@ def oracle_rows(q_bits, k_bits, v_bits, scale, causal, rows_per_head=None):
             bh = b * H + h
             rows = np.arange(Nq, dtype=np.int64) if rows_per_head is None else rows_per_head[bh]
             q = inputs.bf16_bits_to_f64(q_bits[b, h, rows])
-            k = inputs.bf16_bits_to_f64(k_bits[b, h])
-            v = inputs.bf16_bits_to_f64(v_bits[b, h])
+            k = inputs.bf16_bits_to_f64(k_bits[b, h // kv_group])
+            v = inputs.bf16_bits_to_f64(v_bits[b, h // kv_group])
             out[bh] = (rows,) + oracle.attn_rows(q, rows, k, v, scale, causal)
     return out
 

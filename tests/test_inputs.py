@@ -62,3 +62,14 @@ def test_workload_slices_agree():
     rows = np.array([0, 9, 127])
     assert np.array_equal(w.q_rows_bits(1, rows), q[0, 1, rows])
     assert WORKLOADS["mha_b2h16n8k_d128"].flops == 4 * 2 * 16 * 8192 * 8192 * 128
+
+
+def test_gqa_workload_kv_heads():
+    import dataclasses
+    w = dataclasses.replace(WORKLOADS["gqa_b2h32kv8n8k_d128"], Nq=64, Nk=64)
+    assert w.shape("q") == (2, 32, 64, 128) and w.shape("k") == (2, 8, 64, 128)
+    k = w.tensor_bits("k")
+    for bh in (0, 3, 4, 31, 32, 37, 63):
+        b, h = divmod(bh, w.H)
+        assert w.kv_head_of(bh) == b * 8 + h // 4
+        assert np.array_equal(w.head_bits("k", w.kv_head_of(bh)), k[b, h // 4])

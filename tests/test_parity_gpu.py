@@ -191,7 +191,7 @@ def _workload_case(w):
     rows = None
     if w.oracle_rows is not None:
         rows = {bh: w.sampled_rows(bh) for bh in range(w.B * w.H)}
-    ref = harness.oracle_rows(q, k, v, w.scale, w.causal, rows)
+    ref = harness.oracle_rows(q, k, v, w.scale, w.causal, rows, kv_group=w.H // w.kv_heads)
     return o, lse, ref
 
 
