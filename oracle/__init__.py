@@ -51,6 +51,12 @@ def _load():
                           ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64,
                           ctypes.c_double, ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p,
                           ctypes.c_int]
+            w = lib.oracle_attn_rows_window_f64
+            w.restype = ctypes.c_int
+            w.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64,
+                          ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64,
+                          ctypes.c_double, ctypes.c_int64, ctypes.c_int64, ctypes.c_void_p,
+                          ctypes.c_void_p, ctypes.c_int]
             _lib = lib
     return _lib
 
@@ -87,6 +93,63 @@ def attn_rows(q_rows, rows, k, v, scale, causal, nthreads=None):
     if rc != 0:
         raise RuntimeError("oracle_attn_rows_f64 failed")
     return o, lse
+
+
+def attn_rows_window(q_rows, rows, k, v, scale, window_left, window_right, nthreads=None):
+    """Like ``attn_rows`` with the keys of row i limited to the band
+    [i - window_left, i + window_right] (a negative bound is unbounded; causal
+    is (-1, 0)).  Rows whose band holds no key get O = 0, LSE = -inf."""
+    lib = _load()
+    q_rows = np.ascontiguousarray(q_rows, dtype=np.float64)
+    rows = np.ascontiguousarray(rows, dtype=np.int64)
+    k = np.ascontiguousarray(k, dtype=np.float64)
+    v = np.ascontiguousarray(v, dtype=np.float64)
+    n, d = q_rows.shape
+    nk = k.shape[0]
+    assert rows.shape == (n,) and k.shape == (nk, d) and v.shape == (nk, d)
+    o = np.empty((n, d), dtype=np.float64)
+    lse = np.empty((n,), dtype=np.float64)
+    nt = default_threads() if nthreads is None else int(nthreads)
+    rc = lib.oracle_attn_rows_window_f64(q_rows.ctypes.data, rows.ctypes.data, n,
+                                         k.ctypes.data if nk else None,
+                                         v.ctypes.data if nk else None, nk, d, float(scale),
+                                         int(window_left), int(window_right),
+                                         o.ctypes.data, lse.ctypes.data, nt)
+    if rc != 0:
+        raise RuntimeError("oracle_attn_rows_window_f64 failed")
+    return o, lse
+
+
+def attn_varlen(q, k, v, cu_seqlens_q, cu_seqlens_k, scale, window_left=-1, window_right=-1,
+                rows_per_seq=None, nthreads=None):
+    """Variable-length batch: sequences packed back to back without padding
+    (FlashAttention 4 page, ja.linux-konsole.com, section "互換性と現状": batching
+    sequences of different lengths efficiently, with no padding).
+
+    q: [total_q, H, d], k/v: [total_k, Hkv, d] fp64 (H % Hkv == 0; query head h
+    reads key/value head h // (H // Hkv)); sequence s owns query rows
+    cu_seqlens_q[s] .. cu_seqlens_q[s+1]-1 and keys cu_seqlens_k[s] ..
+    cu_seqlens_k[s+1]-1, positions counted from 0 within the sequence; the band
+    applies to those positions.  rows_per_seq: optional dict s -> local rows to
+    evaluate (default all).  Returns {(s, h): (local rows, o [n, d], lse [n])}.
+    """
+    q = np.asarray(q, dtype=np.float64)
+    k = np.asarray(k, dtype=np.float64)
+    v = np.asarray(v, dtype=np.float64)
+    H, Hkv = q.shape[1], k.shape[1]
+    assert H % Hkv == 0
+    out = {}
+    for s in range(len(cu_seqlens_q) - 1):
+        q0, q1 = int(cu_seqlens_q[s]), int(cu_seqlens_q[s + 1])
+        k0, k1 = int(cu_seqlens_k[s]), int(cu_seqlens_k[s + 1])
+        rows = np.arange(q1 - q0, dtype=np.int64) if rows_per_seq is None else \
+            np.asarray(rows_per_seq[s], dtype=np.int64)
+        for h in range(H):
+            hk = h // (H // Hkv)
+            out[(s, h)] = (rows,) + attn_rows_window(q[q0 + rows, h], rows, k[k0:k1, hk],
+                                                     v[k0:k1, hk], scale, window_left,
+                                                     window_right, nthreads)
+    return out
 
 
 def attn_fwd(q, k, v, scale, causal=False, nthreads=None):

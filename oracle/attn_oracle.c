@@ -30,6 +30,17 @@
  *   LSE_i = m + log(l)      (natural log)
  *   K(i) empty  ->  O_i = 0, LSE_i = -inf
  *
+ * Sliding-window (local) masks.  The pages only name richer masks: "AIの
+ * 「脳の回転」を1.8倍高速化？FlashAttentionの秘密" (gipyeong-lee.github.io),
+ * section "今後はどうなるか？", points to FlashMask.  This library's reading is
+ * the band of keys around the query's own position:
+ *
+ *   K(i)  = {j : 0 <= j < Nk,  j >= i - window_left,  j <= i + window_right}
+ *
+ * with a negative window bound meaning "unbounded on that side".  Causal is the
+ * band (-1, 0); no mask is (-1, -1).  A row whose band holds no key gets
+ * O_i = 0, LSE_i = -inf, as for Nk == 0.
+ *
  * All arithmetic is fp64.  Inputs arrive as fp64 (the caller widens the BF16
  * values, which is exact), so the only rounding is fp64 rounding.
  *
@@ -51,7 +62,8 @@ typedef struct {
     int64_t nk;
     int64_t d;
     double scale;
-    int causal;
+    int64_t window_left;  /* keys j >= i - window_left (negative: no bound)  */
+    int64_t window_right; /* keys j <= i + window_right (negative: no bound) */
     double *o;            /* [n_rows, d]  out                                 */
     double *lse;          /* [n_rows]     out                                 */
     double *s;            /* per-thread score row, [nk]                       */
@@ -64,20 +76,22 @@ static void oracle_row(const oracle_job *jb, int64_t r) {
     const double *qi = jb->q + r * d;
     double *oi = jb->o + r * d;
     const int64_t i = jb->rows[r];
-    /* visible keys: all of them, or the prefix 0..i when causal */
-    int64_t nvis = jb->nk;
-    if (jb->causal) nvis = (i + 1 < jb->nk) ? i + 1 : jb->nk;
+    /* visible keys: the contiguous range lo..hi of the band around i */
+    int64_t lo = 0, hi = jb->nk - 1;
+    if (jb->window_left >= 0 && i - jb->window_left > lo) lo = i - jb->window_left;
+    if (jb->window_right >= 0 && i + jb->window_right < hi) hi = i + jb->window_right;
+    const int64_t nvis = hi - lo + 1;
     if (nvis <= 0) {
         for (int64_t c = 0; c < d; ++c) oi[c] = 0.0;
         jb->lse[r] = -INFINITY;
         return;
     }
-    double *s = jb->s;
-    for (int64_t j = 0; j < nvis; ++j) {
+    double *s = jb->s; /* s[j - lo] holds the score of key j */
+    for (int64_t j = lo; j <= hi; ++j) {
         const double *kj = jb->k + j * d;
         double dot = 0.0;
         for (int64_t c = 0; c < d; ++c) dot += qi[c] * kj[c];
-        s[j] = jb->scale * dot;
+        s[j - lo] = jb->scale * dot;
     }
     double m = s[0];
     for (int64_t j = 1; j < nvis; ++j)
@@ -90,7 +104,7 @@ static void oracle_row(const oracle_job *jb, int64_t r) {
     for (int64_t c = 0; c < d; ++c) oi[c] = 0.0;
     for (int64_t j = 0; j < nvis; ++j) {
         const double p = s[j] / l;
-        const double *vj = jb->v + j * d;
+        const double *vj = jb->v + (lo + j) * d;
         for (int64_t c = 0; c < d; ++c) oi[c] += p * vj[c];
     }
     jb->lse[r] = m + log(l);
@@ -103,7 +117,8 @@ static void *oracle_worker(void *arg) {
 }
 
 /*
- * Attention for a subset of query rows of one (batch, head).
+ * Attention for a subset of query rows of one (batch, head), keys limited to
+ * the band [i - window_left, i + window_right] (negative bound: unbounded).
  *
  * q:    [n_rows, d] fp64, the query rows to evaluate (row r has index rows[r]).
  * k, v: [nk, d] fp64, all keys and values of that head.
@@ -111,10 +126,10 @@ static void *oracle_worker(void *arg) {
  * nthreads <= 0 means one thread.
  * Returns 0 on success, -1 on a bad argument or allocation failure.
  */
-int oracle_attn_rows_f64(const double *q, const int64_t *rows, int64_t n_rows,
-                         const double *k, const double *v, int64_t nk, int64_t d,
-                         double scale, int causal, double *o, double *lse,
-                         int nthreads) {
+int oracle_attn_rows_window_f64(const double *q, const int64_t *rows, int64_t n_rows,
+                                const double *k, const double *v, int64_t nk, int64_t d,
+                                double scale, int64_t window_left, int64_t window_right,
+                                double *o, double *lse, int nthreads) {
     if (n_rows < 0 || nk < 0 || d <= 0) return -1;
     if (n_rows == 0) return 0;
     if (!q || !rows || !o || !lse || (nk > 0 && (!k || !v))) return -1;
@@ -135,7 +150,8 @@ int oracle_attn_rows_f64(const double *q, const int64_t *rows, int64_t n_rows,
         oracle_job *jb = &jobs[t];
         jb->q = q; jb->rows = rows; jb->n_rows = n_rows;
         jb->k = k; jb->v = v; jb->nk = nk; jb->d = d;
-        jb->scale = scale; jb->causal = causal;
+        jb->scale = scale;
+        jb->window_left = window_left; jb->window_right = window_right;
         jb->o = o; jb->lse = lse;
         jb->begin = (int64_t)t * per;
         jb->end = jb->begin + per < n_rows ? jb->begin + per : n_rows;
@@ -161,4 +177,13 @@ int oracle_attn_rows_f64(const double *q, const int64_t *rows, int64_t n_rows,
     free(jobs);
     free(tids);
     return rc;
+}
+
+/* The same without a window: all keys, or the prefix 0..i when causal. */
+int oracle_attn_rows_f64(const double *q, const int64_t *rows, int64_t n_rows,
+                         const double *k, const double *v, int64_t nk, int64_t d,
+                         double scale, int causal, double *o, double *lse,
+                         int nthreads) {
+    return oracle_attn_rows_window_f64(q, rows, n_rows, k, v, nk, d, scale, -1,
+                                       causal ? 0 : -1, o, lse, nthreads);
 }

@@ -217,9 +217,143 @@ def pin_sampled_rows(attn_rows):
         assert np.array_equal(os_, o[rows]) and np.array_equal(ls_, lse[rows])
 
 
+# ---------------------------------------------------------------------------
+# Sliding-window band.  These take ``attn_rows_window(q_rows, rows, k, v, scale,
+# window_left, window_right)``.
+# ---------------------------------------------------------------------------
+def band_mask_numpy(nq, nk, wl, wr):
+    """Visible (i, j) pairs built from numpy's triangle helpers: np.triu(., -wl)
+    keeps j - i >= -wl, np.tril(., wr) keeps j - i <= wr."""
+    m = np.ones((nq, nk), dtype=bool)
+    if wl >= 0:
+        m = np.triu(m, -wl)
+    if wr >= 0:
+        m = np.tril(m, wr)
+    return m
+
+
+def masked_softmax_numpy(q, k, v, scale, mask):
+    """Dense masked attention: materialised scores, -inf outside the mask."""
+    s = np.where(mask, scale * (q @ k.T), -np.inf)
+    o = np.zeros((q.shape[0], v.shape[1]))
+    lse = np.full(q.shape[0], -np.inf)
+    for i in range(q.shape[0]):
+        if not mask[i].any():
+            continue
+        m = s[i].max()
+        e = np.exp(s[i] - m)
+        o[i] = (e / e.sum()) @ v
+        lse[i] = m + np.log(e.sum())
+    return o, lse
+
+
+WINDOWS = [(0, 0), (2, 1), (-1, 0), (3, -1), (-1, -1), (1, 5), (20, 20), (0, 3), (4, 0)]
+
+
+def pin_window_brute_force(attn_rows_window):
+    """Match materialised masked attention for many bands, Nq != Nk, and rows
+    whose band holds no key."""
+    for seed, (nq, nk, d) in enumerate([(7, 7, 4), (9, 13, 3), (12, 5, 8), (1, 1, 2)]):
+        r = _rng(100 + seed)
+        q, k, v = (r.standard_normal((n, d)) for n in (nq, nk, nk))
+        for wl, wr in WINDOWS:
+            o, lse = attn_rows_window(q, np.arange(nq, dtype=np.int64), k, v, 0.6, wl, wr)
+            ob, lb = masked_softmax_numpy(q, k, v, 0.6, band_mask_numpy(nq, nk, wl, wr))
+            np.testing.assert_allclose(o, ob, rtol=1e-12, atol=1e-12, err_msg=str((nq, nk, wl, wr)))
+            np.testing.assert_allclose(lse, lb, rtol=1e-12, atol=1e-12, err_msg=str((nq, nk, wl, wr)))
+
+
+def pin_window_diagonal(attn_rows_window):
+    """Band (0, 0): each row sees only its own key, so O_i = v_i exactly and
+    LSE_i = scale * q_i . k_i."""
+    r = _rng(110)
+    n, d = 10, 8
+    q, k, v = (r.standard_normal((n, d)) for _ in range(3))
+    o, lse = attn_rows_window(q, np.arange(n, dtype=np.int64), k, v, 0.45, 0, 0)
+    assert np.array_equal(o, v)
+    np.testing.assert_allclose(lse, 0.45 * np.einsum("id,id->i", q, k), rtol=1e-14, atol=1e-14)
+
+
+def pin_window_is_a_key_slice(attn_rows_window):
+    """Row i under band (wl, wr) equals unmasked attention over the key slice
+    [max(0, i-wl), min(Nk-1, i+wr)] given to the oracle as the whole key set."""
+    r = _rng(111)
+    n, d = 16, 4
+    q, k, v = (r.standard_normal((n, d)) for _ in range(3))
+    for wl, wr in [(3, 2), (0, 5), (6, 0)]:
+        o, lse = attn_rows_window(q, np.arange(n, dtype=np.int64), k, v, 0.8, wl, wr)
+        for i in range(n):
+            lo, hi = max(0, i - wl), min(n - 1, i + wr)
+            oi, li = attn_rows_window(q[i:i + 1], np.array([0], dtype=np.int64), k[lo:hi + 1],
+                                      v[lo:hi + 1], 0.8, -1, -1)
+            np.testing.assert_allclose(o[i], oi[0], rtol=1e-12, atol=1e-13)
+            np.testing.assert_allclose(lse[i], li[0], rtol=1e-13, atol=1e-13)
+
+
+WINDOW_PINS = [pin_window_brute_force, pin_window_diagonal, pin_window_is_a_key_slice]
+
+
 ALL_PINS = [
     pin_brute_force, pin_golden, pin_single_key, pin_identical_keys, pin_zero_scale,
     pin_causal_prefix, pin_rows_sum_to_one, pin_shift_invariance, pin_value_linearity,
     pin_key_permutation, pin_split_merge, pin_hard_max, pin_two_keys_sigmoid,
     pin_empty_keys, pin_sampled_rows,
 ]
+
+
+# ---------------------------------------------------------------------------
+# Variable-length batches.  These take ``attn_varlen(q, k, v, cu_q, cu_k, scale,
+# window_left, window_right)`` returning {(s, h): (rows, o, lse)}.
+# ---------------------------------------------------------------------------
+def pin_varlen_block_diagonal(attn_varlen):
+    """Packed sequences equal one dense masked attention over the whole packed
+    index space whose mask is block-diagonal (same sequence) and banded on the
+    positions within the sequence; includes an empty sequence, Nq != Nk per
+    sequence and grouped key/value heads."""
+    r = _rng(120)
+    lens_q = [5, 0, 9, 3]
+    lens_k = [7, 2, 9, 1]
+    H, Hkv, d = 4, 2, 4
+    cu_q = np.concatenate([[0], np.cumsum(lens_q)])
+    cu_k = np.concatenate([[0], np.cumsum(lens_k)])
+    q = r.standard_normal((cu_q[-1], H, d))
+    k = r.standard_normal((cu_k[-1], Hkv, d))
+    v = r.standard_normal((cu_k[-1], Hkv, d))
+    seq_q = np.repeat(np.arange(len(lens_q)), lens_q)
+    seq_k = np.repeat(np.arange(len(lens_k)), lens_k)
+    pos_q = np.arange(cu_q[-1]) - cu_q[seq_q]
+    pos_k = np.arange(cu_k[-1]) - cu_k[seq_k]
+    for wl, wr in [(-1, -1), (-1, 0), (1, 1)]:
+        got = attn_varlen(q, k, v, cu_q, cu_k, 0.7, wl, wr)
+        rel = pos_k[None, :] - pos_q[:, None]
+        mask = seq_q[:, None] == seq_k[None, :]
+        if wl >= 0:
+            mask &= rel >= -wl
+        if wr >= 0:
+            mask &= rel <= wr
+        for h in range(H):
+            hk = h // (H // Hkv)
+            ob, lb = masked_softmax_numpy(q[:, h], k[:, hk], v[:, hk], 0.7, mask)
+            for s in range(len(lens_q)):
+                rows, o, lse = got[(s, h)]
+                np.testing.assert_allclose(o, ob[cu_q[s] + rows], rtol=1e-12, atol=1e-12)
+                np.testing.assert_allclose(lse, lb[cu_q[s] + rows], rtol=1e-12, atol=1e-12)
+
+
+def pin_varlen_neighbours_do_not_leak(attn_varlen):
+    """A sequence's output does not change when the other sequences' data does."""
+    r = _rng(121)
+    cu = np.array([0, 6, 10, 19])
+    q, k, v = (r.standard_normal((19, 2, 4)) for _ in range(3))
+    a = attn_varlen(q, k, v, cu, cu, 0.5, -1, 0)
+    q2, k2, v2 = q.copy(), k.copy(), v.copy()
+    for x in (q2, k2, v2):
+        x[:6] += 3.0
+        x[10:] -= 2.0
+    b = attn_varlen(q2, k2, v2, cu, cu, 0.5, -1, 0)
+    for h in range(2):
+        assert np.array_equal(a[(1, h)][1], b[(1, h)][1])
+        assert np.array_equal(a[(1, h)][2], b[(1, h)][2])
+
+
+VARLEN_PINS = [pin_varlen_block_diagonal, pin_varlen_neighbours_do_not_leak]

@@ -17,6 +17,16 @@ def test_oracle_pin(pin):
     pin(oracle.attn_rows)
 
 
+@pytest.mark.parametrize("pin", pins.WINDOW_PINS, ids=[p.__name__ for p in pins.WINDOW_PINS])
+def test_oracle_window_pin(pin):
+    pin(oracle.attn_rows_window)
+
+
+@pytest.mark.parametrize("pin", pins.VARLEN_PINS, ids=[p.__name__ for p in pins.VARLEN_PINS])
+def test_oracle_varlen_pin(pin):
+    pin(oracle.attn_varlen)
+
+
 def test_full_tensor_wrapper_matches_rows():
     r = np.random.default_rng(5)
     q, k, v = (r.standard_normal((2, 3, 9, 4)) for _ in range(3))
@@ -41,14 +51,19 @@ def test_thread_count_does_not_change_result():
 # The mutants are built in a temporary directory; the real oracle is untouched.
 # ---------------------------------------------------------------------------
 MUTANTS = {
-    "dropped_scale": ("s[j] = jb->scale * dot;", "s[j] = dot;"),
-    "causal_off_by_one": ("nvis = (i + 1 < jb->nk) ? i + 1 : jb->nk;",
-                          "nvis = (i < jb->nk) ? i : jb->nk;"),
+    "dropped_scale": ("s[j - lo] = jb->scale * dot;", "s[j - lo] = dot;"),
+    "causal_off_by_one": ("hi = i + jb->window_right;", "hi = i + jb->window_right - 1;"),
+    "window_left_off_by_one": ("lo = i - jb->window_left;", "lo = i - jb->window_left + 1;"),
+    "window_right_ignored": ("if (jb->window_right >= 0 && i + jb->window_right < hi)",
+                             "if (0 && i + jb->window_right < hi)"),
     "lse_without_max": ("jb->lse[r] = m + log(l);", "jb->lse[r] = log(l);"),
     "unnormalised_weights": ("const double p = s[j] / l;", "const double p = s[j];"),
     "transposed_key_index": ("const double *kj = jb->k + j * d;", "const double *kj = jb->k + j;"),
     "max_sign_flip": ("if (s[j] > m) m = s[j];", "if (s[j] < m) m = s[j];"),
-    "wrong_value_row": ("const double *vj = jb->v + j * d;", "const double *vj = jb->v + (nvis - 1 - j) * d;"),
+    "wrong_value_row": ("const double *vj = jb->v + (lo + j) * d;",
+                        "const double *vj = jb->v + (hi - j) * d;"),
+    "value_row_not_offset": ("const double *vj = jb->v + (lo + j) * d;",
+                             "const double *vj = jb->v + j * d;"),
 }
 
 
@@ -67,7 +82,13 @@ def _build_mutant(tmp_path, name, old, new):
                   ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64, ctypes.c_double,
                   ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int]
 
-    def attn_rows(q_rows, rows, k, v, scale, causal):
+    w = cdll.oracle_attn_rows_window_f64
+    w.restype = ctypes.c_int
+    w.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p,
+                  ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64, ctypes.c_double,
+                  ctypes.c_int64, ctypes.c_int64, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int]
+
+    def call(fn, q_rows, rows, k, v, scale, *mask):
         q_rows = np.ascontiguousarray(q_rows, dtype=np.float64)
         rows = np.ascontiguousarray(rows, dtype=np.int64)
         k = np.ascontiguousarray(k, dtype=np.float64)
@@ -75,22 +96,29 @@ def _build_mutant(tmp_path, name, old, new):
         n, d = q_rows.shape
         o = np.empty((n, d))
         lse = np.empty(n)
-        f(q_rows.ctypes.data, rows.ctypes.data, n, k.ctypes.data if len(k) else None,
-          v.ctypes.data if len(v) else None, k.shape[0], d, float(scale), int(causal),
-          o.ctypes.data, lse.ctypes.data, 2)
+        fn(q_rows.ctypes.data, rows.ctypes.data, n, k.ctypes.data if len(k) else None,
+           v.ctypes.data if len(v) else None, k.shape[0], d, float(scale), *mask,
+           o.ctypes.data, lse.ctypes.data, 2)
         return o, lse
 
-    return attn_rows
+    def attn_rows(q_rows, rows, k, v, scale, causal):
+        return call(f, q_rows, rows, k, v, scale, int(causal))
+
+    def attn_rows_window(q_rows, rows, k, v, scale, wl, wr):
+        return call(w, q_rows, rows, k, v, scale, int(wl), int(wr))
+
+    return attn_rows, attn_rows_window
 
 
 @pytest.mark.parametrize("name", sorted(MUTANTS))
 def test_planted_mistake_is_caught(tmp_path, name):
     old, new = MUTANTS[name]
-    mutant = _build_mutant(tmp_path, name, old, new)
+    rows_fn, window_fn = _build_mutant(tmp_path, name, old, new)
     failed = []
-    for pin in PINS:
-        try:
-            pin(mutant)
-        except AssertionError:
-            failed.append(pin.__name__)
+    for pin_set, fn in ((PINS, rows_fn), (pins.WINDOW_PINS, window_fn)):
+        for pin in pin_set:
+            try:
+                pin(fn)
+            except AssertionError:
+                failed.append(pin.__name__)
     assert failed, f"no pin catches the planted mistake {name}"
