@@ -57,6 +57,10 @@ def _load():
                           ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64,
                           ctypes.c_double, ctypes.c_int64, ctypes.c_int64, ctypes.c_void_p,
                           ctypes.c_void_p, ctypes.c_int]
+            b = lib.oracle_attn_bwd_f64
+            b.restype = ctypes.c_int
+            b.argtypes = [ctypes.c_void_p] * 4 + [ctypes.c_int64] * 3 + [ctypes.c_double] + \
+                [ctypes.c_int64] * 2 + [ctypes.c_void_p] * 3
             _lib = lib
     return _lib
 
@@ -166,3 +170,49 @@ def attn_fwd(q, k, v, scale, causal=False, nthreads=None):
             o[b, h], lse[b, h] = attn_rows(q[b, h], rows, k[b, h], v[b, h],
                                            scale, causal, nthreads)
     return o, lse
+
+
+def attn_bwd_head(q, k, v, dout, scale, window_left=-1, window_right=-1):
+    """Gradients of one (batch, head): returns (dq [nq, d], dk [nk, d], dv [nk, d])
+    fp64 for the cotangent dout [nq, d] (see oracle_attn_bwd_f64)."""
+    lib = _load()
+    q, k, v, dout = (np.ascontiguousarray(x, dtype=np.float64) for x in (q, k, v, dout))
+    nq, d = q.shape
+    nk = k.shape[0]
+    assert k.shape == (nk, d) and v.shape == (nk, d) and dout.shape == (nq, d)
+    dq = np.empty((nq, d))
+    dk = np.empty((nk, d))
+    dv = np.empty((nk, d))
+    ptr = lambda a: a.ctypes.data if a.size else None  # noqa: E731
+    rc = lib.oracle_attn_bwd_f64(ptr(q), ptr(k), ptr(v), ptr(dout), nq, nk, d, float(scale),
+                                 int(window_left), int(window_right), ptr(dq), ptr(dk), ptr(dv))
+    if rc != 0:
+        raise RuntimeError("oracle_attn_bwd_f64 failed")
+    return dq, dk, dv
+
+
+def attn_bwd(q, k, v, dout, scale, window_left=-1, window_right=-1, nthreads=None):
+    """Gradients over [B, H, Nq, d] q/dout and [B, Hkv, Nk, d] k/v (fp64).
+    Query head h reads key/value head h // (H // Hkv); the key/value gradients
+    of a shared head are the sum over its query heads.  Heads run on a thread
+    pool (the C routine releases the GIL); the group sums are added in head
+    order, so the result does not depend on the thread count."""
+    import concurrent.futures
+    q, k, v, dout = (np.asarray(x, dtype=np.float64) for x in (q, k, v, dout))
+    B, H = q.shape[:2]
+    Hkv = k.shape[1]
+    g = H // Hkv
+    jobs = [(b, h) for b in range(B) for h in range(H)]
+    nt = default_threads() if nthreads is None else int(nthreads)
+    with concurrent.futures.ThreadPoolExecutor(max_workers=max(1, nt)) as ex:
+        res = list(ex.map(lambda bh: attn_bwd_head(q[bh[0], bh[1]], k[bh[0], bh[1] // g],
+                                                   v[bh[0], bh[1] // g], dout[bh[0], bh[1]],
+                                                   scale, window_left, window_right), jobs))
+    dq = np.empty(q.shape)
+    dk = np.zeros(k.shape)
+    dv = np.zeros(v.shape)
+    for (b, h), (a, bk, bv) in zip(jobs, res):
+        dq[b, h] = a
+        dk[b, h // g] += bk
+        dv[b, h // g] += bv
+    return dq, dk, dv

@@ -187,3 +187,74 @@ int oracle_attn_rows_f64(const double *q, const int64_t *rows, int64_t n_rows,
     return oracle_attn_rows_window_f64(q, rows, n_rows, k, v, nk, d, scale, -1,
                                        causal ? 0 : -1, o, lse, nthreads);
 }
+
+/*
+ * Backward pass of one (batch, head): the vector-Jacobian product of the
+ * forward map above with the output cotangent dO.  FlashAttention 4 page
+ * (ja.linux-konsole.com), sections "重要ポイント" and "互換性と現状", and
+ * "FlashAttention-4 deep dive" (sns.style), section 二: the backward pass --
+ * the gradients needed for training -- is what FA4 still lacks.  The pages give
+ * no formulas; this is the chain rule through s -> softmax -> P.V, per query
+ * row i over its visible keys j:
+ *
+ *   p_j   = softmax_j(s_ij)                      (as in the forward)
+ *   dp_j  = <dO_i, v_j>
+ *   D_i   = sum_j p_j * dp_j                     (= <dO_i, O_i>)
+ *   ds_j  = p_j * (dp_j - D_i)                   (softmax Jacobian)
+ *   dQ_i  = scale * sum_j ds_j * k_j
+ *   dK_j += scale * ds_j * q_i
+ *   dV_j += p_j * dO_i
+ *
+ * q, dout, dq: [nq, d]; k, v, dk, dv: [nk, d]; all fp64, rows in order, one
+ * thread.  dq, dk, dv are overwritten.  Band as in oracle_attn_rows_window_f64.
+ * Returns 0, or -1 on a bad argument or allocation failure.
+ */
+int oracle_attn_bwd_f64(const double *q, const double *k, const double *v,
+                        const double *dout, int64_t nq, int64_t nk, int64_t d,
+                        double scale, int64_t window_left, int64_t window_right,
+                        double *dq, double *dk, double *dv) {
+    if (nq < 0 || nk < 0 || d <= 0) return -1;
+    for (int64_t x = 0; x < nk * d; ++x) { dk[x] = 0.0; dv[x] = 0.0; }
+    for (int64_t x = 0; x < nq * d; ++x) dq[x] = 0.0;
+    if (nq == 0 || nk == 0) return 0;
+    double *p = (double *)malloc((size_t)nk * sizeof(double));
+    double *dp = (double *)malloc((size_t)nk * sizeof(double));
+    if (!p || !dp) { free(p); free(dp); return -1; }
+    for (int64_t i = 0; i < nq; ++i) {
+        const double *qi = q + i * d, *gi = dout + i * d;
+        int64_t lo = 0, hi = nk - 1;
+        if (window_left >= 0 && i - window_left > lo) lo = i - window_left;
+        if (window_right >= 0 && i + window_right < hi) hi = i + window_right;
+        if (hi < lo) continue; /* no visible key: O_i = 0 does not depend on the inputs */
+        /* forward probabilities of the row */
+        double m = -INFINITY;
+        for (int64_t j = lo; j <= hi; ++j) {
+            double dot = 0.0;
+            for (int64_t c = 0; c < d; ++c) dot += qi[c] * k[j * d + c];
+            p[j] = scale * dot;
+            if (p[j] > m) m = p[j];
+        }
+        double l = 0.0;
+        for (int64_t j = lo; j <= hi; ++j) { p[j] = exp(p[j] - m); l += p[j]; }
+        for (int64_t j = lo; j <= hi; ++j) p[j] /= l;
+        /* dp and D */
+        double D = 0.0;
+        for (int64_t j = lo; j <= hi; ++j) {
+            double dot = 0.0;
+            for (int64_t c = 0; c < d; ++c) dot += gi[c] * v[j * d + c];
+            dp[j] = dot;
+            D += p[j] * dot;
+        }
+        for (int64_t j = lo; j <= hi; ++j) {
+            const double ds = p[j] * (dp[j] - D);
+            for (int64_t c = 0; c < d; ++c) {
+                dq[i * d + c] += scale * ds * k[j * d + c];
+                dk[j * d + c] += scale * ds * qi[c];
+                dv[j * d + c] += p[j] * gi[c];
+            }
+        }
+    }
+    free(p);
+    free(dp);
+    return 0;
+}

@@ -357,3 +357,91 @@ def pin_varlen_neighbours_do_not_leak(attn_varlen):
 
 
 VARLEN_PINS = [pin_varlen_block_diagonal, pin_varlen_neighbours_do_not_leak]
+
+
+
+# ---------------------------------------------------------------------------
+# Backward pass.  These take ``bwd(q, k, v, dout, scale, wl, wr) -> (dq, dk, dv)``
+# for one head and ``fwd(q_rows, rows, k, v, scale, wl, wr) -> (o, lse)``.
+# ---------------------------------------------------------------------------
+def _loss(fwd, q, k, v, dout, scale, wl, wr):
+    o, _ = fwd(q, np.arange(q.shape[0], dtype=np.int64), k, v, scale, wl, wr)
+    return float((o * dout).sum())
+
+
+def pin_bwd_finite_differences(bwd, fwd):
+    """Each gradient element equals the central difference of
+    L(Q, K, V) = sum(dO * O(Q, K, V)) computed with the forward definition
+    (step 1e-5 in fp64: truncation ~1e-10, rounding ~1e-11)."""
+    h = 1e-5
+    for seed, (nq, nk, d, wl, wr) in enumerate([(4, 6, 3, -1, -1), (5, 5, 2, -1, 0),
+                                                 (6, 4, 3, 1, 1), (3, 7, 2, 0, 2)]):
+        r = _rng(300 + seed)
+        q, k, v, dout = (r.standard_normal(s) for s in ((nq, d), (nk, d), (nk, d), (nq, d)))
+        grads = bwd(q, k, v, dout, 0.8, wl, wr)
+        for which, x in enumerate((q, k, v)):
+            num = np.zeros_like(x)
+            for idx in np.ndindex(*x.shape):
+                args = [q.copy(), k.copy(), v.copy()]
+                args[which][idx] += h
+                lp = _loss(fwd, *args, dout, 0.8, wl, wr)
+                args[which][idx] -= 2 * h
+                lm = _loss(fwd, *args, dout, 0.8, wl, wr)
+                num[idx] = (lp - lm) / (2 * h)
+            np.testing.assert_allclose(grads[which], num, rtol=1e-6, atol=1e-8,
+                                       err_msg=f"grad {'qkv'[which]} band {(wl, wr)}")
+
+
+def pin_bwd_single_key(bwd, fwd):
+    """One key: the softmax is constant 1, so dQ = dK = 0 exactly and
+    dV = sum_i dO_i."""
+    r = _rng(310)
+    q, dout = r.standard_normal((5, 4)), r.standard_normal((5, 4))
+    k, v = r.standard_normal((1, 4)), r.standard_normal((1, 4))
+    dq, dk, dv = bwd(q, k, v, dout, 0.6, -1, -1)
+    assert np.array_equal(dq, np.zeros_like(dq)) and np.array_equal(dk, np.zeros_like(dk))
+    np.testing.assert_allclose(dv[0], dout.sum(0), rtol=1e-14, atol=1e-14)
+
+
+def pin_bwd_sums(bwd, fwd):
+    """Rows of the softmax Jacobian sum to zero, so sum_j dK_j = 0; weights
+    sum to one, so sum_j dV_j = sum_i dO_i (unmasked and causal)."""
+    r = _rng(311)
+    n, d = 9, 5
+    q, k, v, dout = (r.standard_normal((n, d)) for _ in range(4))
+    for wl, wr in [(-1, -1), (-1, 0), (2, 1)]:
+        dq, dk, dv = bwd(q, k, v, dout, 0.7, wl, wr)
+        np.testing.assert_allclose(dk.sum(0), np.zeros(d), atol=1e-12)
+        np.testing.assert_allclose(dv.sum(0), dout.sum(0), rtol=1e-12, atol=1e-12)
+
+
+def pin_bwd_linear_in_cotangent(bwd, fwd):
+    """The gradients are linear in dO."""
+    r = _rng(312)
+    q, k, v = r.standard_normal((6, 4)), r.standard_normal((8, 4)), r.standard_normal((8, 4))
+    g1, g2 = r.standard_normal((6, 4)), r.standard_normal((6, 4))
+    a = bwd(q, k, v, g1, 0.5, -1, -1)
+    b = bwd(q, k, v, g2, 0.5, -1, -1)
+    c = bwd(q, k, v, 2.0 * g1 - 3.0 * g2, 0.5, -1, -1)
+    for x, y, z in zip(a, b, c):
+        np.testing.assert_allclose(z, 2.0 * x - 3.0 * y, rtol=1e-11, atol=1e-12)
+
+
+def pin_bwd_dv_is_pt_dout(bwd, fwd):
+    """dV = P^T dO with P the materialised softmax of the (independent)
+    numpy masked-attention construction."""
+    r = _rng(313)
+    nq, nk, d = 7, 9, 3
+    q, k, v = r.standard_normal((nq, d)), r.standard_normal((nk, d)), r.standard_normal((nk, d))
+    dout = r.standard_normal((nq, d))
+    for wl, wr in [(-1, -1), (3, 0)]:
+        mask = band_mask_numpy(nq, nk, wl, wr)
+        s = np.where(mask, 0.9 * (q @ k.T), -np.inf)
+        p = np.exp(s - s.max(1, keepdims=True))
+        p /= p.sum(1, keepdims=True)
+        _, _, dv = bwd(q, k, v, dout, 0.9, wl, wr)
+        np.testing.assert_allclose(dv, p.T @ dout, rtol=1e-12, atol=1e-12)
+
+
+BWD_PINS = [pin_bwd_finite_differences, pin_bwd_single_key, pin_bwd_sums,
+            pin_bwd_linear_in_cotangent, pin_bwd_dv_is_pt_dout]

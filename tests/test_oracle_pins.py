@@ -27,6 +27,28 @@ def test_oracle_varlen_pin(pin):
     pin(oracle.attn_varlen)
 
 
+@pytest.mark.parametrize("pin", pins.BWD_PINS, ids=[p.__name__ for p in pins.BWD_PINS])
+def test_oracle_bwd_pin(pin):
+    pin(oracle.attn_bwd_head, oracle.attn_rows_window)
+
+
+def test_bwd_group_sum_and_threads():
+    """Grouped key/value heads: the shared head's gradients are the sums over its
+    query heads, whatever the thread count."""
+    r = np.random.default_rng(7)
+    q, g = r.standard_normal((2, 4, 6, 3)), r.standard_normal((2, 4, 6, 3))
+    k, v = r.standard_normal((2, 2, 5, 3)), r.standard_normal((2, 2, 5, 3))
+    dq, dk, dv = oracle.attn_bwd(q, k, v, g, 0.5, -1, 0, nthreads=1)
+    dq2, dk2, dv2 = oracle.attn_bwd(q, k, v, g, 0.5, -1, 0, nthreads=5)
+    assert np.array_equal(dk, dk2) and np.array_equal(dv, dv2) and np.array_equal(dq, dq2)
+    for b in range(2):
+        for hk in range(2):
+            parts = [oracle.attn_bwd_head(q[b, h], k[b, hk], v[b, hk], g[b, h], 0.5, -1, 0)
+                     for h in (2 * hk, 2 * hk + 1)]
+            np.testing.assert_allclose(dk[b, hk], parts[0][1] + parts[1][1], rtol=1e-15, atol=1e-15)
+            np.testing.assert_allclose(dv[b, hk], parts[0][2] + parts[1][2], rtol=1e-15, atol=1e-15)
+
+
 def test_full_tensor_wrapper_matches_rows():
     r = np.random.default_rng(5)
     q, k, v = (r.standard_normal((2, 3, 9, 4)) for _ in range(3))
@@ -64,6 +86,15 @@ MUTANTS = {
                         "const double *vj = jb->v + (hi - j) * d;"),
     "value_row_not_offset": ("const double *vj = jb->v + (lo + j) * d;",
                              "const double *vj = jb->v + j * d;"),
+    "bwd_dropped_D": ("const double ds = p[j] * (dp[j] - D);", "const double ds = p[j] * dp[j];"),
+    "bwd_dk_without_scale": ("dk[j * d + c] += scale * ds * qi[c];", "dk[j * d + c] += ds * qi[c];"),
+    "bwd_dq_wrong_operand": ("dq[i * d + c] += scale * ds * k[j * d + c];",
+                             "dq[i * d + c] += scale * ds * v[j * d + c];"),
+    "bwd_dv_with_ds": ("dv[j * d + c] += p[j] * gi[c];", "dv[j * d + c] += ds * gi[c];"),
+    "bwd_dp_against_k": ("for (int64_t c = 0; c < d; ++c) dot += gi[c] * v[j * d + c];",
+                         "for (int64_t c = 0; c < d; ++c) dot += gi[c] * k[j * d + c];"),
+    "bwd_band_ignored": ("if (window_right >= 0 && i + window_right < hi) hi = i + window_right;",
+                         "if (0) hi = i + window_right;"),
 }
 
 
@@ -107,18 +138,33 @@ def _build_mutant(tmp_path, name, old, new):
     def attn_rows_window(q_rows, rows, k, v, scale, wl, wr):
         return call(w, q_rows, rows, k, v, scale, int(wl), int(wr))
 
-    return attn_rows, attn_rows_window
+    b = cdll.oracle_attn_bwd_f64
+    b.restype = ctypes.c_int
+    b.argtypes = [ctypes.c_void_p] * 4 + [ctypes.c_int64] * 3 + [ctypes.c_double] + \
+        [ctypes.c_int64] * 2 + [ctypes.c_void_p] * 3
+
+    def attn_bwd_head(q, k, v, dout, scale, wl, wr):
+        q, k, v, dout = (np.ascontiguousarray(x, dtype=np.float64) for x in (q, k, v, dout))
+        nq, d = q.shape
+        nk = k.shape[0]
+        dq, dk, dv = np.empty((nq, d)), np.empty((nk, d)), np.empty((nk, d))
+        b(q.ctypes.data, k.ctypes.data, v.ctypes.data, dout.ctypes.data, nq, nk, d, float(scale),
+          int(wl), int(wr), dq.ctypes.data, dk.ctypes.data, dv.ctypes.data)
+        return dq, dk, dv
+
+    return attn_rows, attn_rows_window, attn_bwd_head
 
 
 @pytest.mark.parametrize("name", sorted(MUTANTS))
 def test_planted_mistake_is_caught(tmp_path, name):
     old, new = MUTANTS[name]
-    rows_fn, window_fn = _build_mutant(tmp_path, name, old, new)
+    rows_fn, window_fn, bwd_fn = _build_mutant(tmp_path, name, old, new)
     failed = []
-    for pin_set, fn in ((PINS, rows_fn), (pins.WINDOW_PINS, window_fn)):
+    for pin_set, args in ((PINS, (rows_fn,)), (pins.WINDOW_PINS, (window_fn,)),
+                          (pins.BWD_PINS, (bwd_fn, window_fn))):
         for pin in pin_set:
             try:
-                pin(fn)
+                pin(*args)
             except AssertionError:
                 failed.append(pin.__name__)
     assert failed, f"no pin catches the planted mistake {name}"
