@@ -29,11 +29,14 @@ import sys
 import tempfile
 import time
 
+import numpy as np
+
 ROOT = os.path.dirname(os.path.abspath(__file__))
 if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
 METRIC = "attention fwd TFLOP/s (BF16, 1×B200) and % of dense BF16 tensor peak"
+METRIC_BWD = "attention bwd TFLOP/s (BF16, 1×B200; 2.5x the forward's FLOPs)"
 UNIT = "TFLOP/s"
 SPEC_DENSE_BF16_TFLOPS = 2250.0
 L2_BYTES = 126 * 1024 * 1024
@@ -52,6 +55,8 @@ def parse_args(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--exp-mode", type=int, default=None, help="0 MUFU, 1 split, 2 polynomial")
     ap.add_argument("--threshold", type=float, default=None, help="rescale threshold (powers of 2)")
+    ap.add_argument("--pass", dest="which", choices=["fwd", "bwd"], default="fwd",
+                    help="time the forward (default) or the backward pass")
     return ap.parse_args(argv)
 
 
@@ -165,40 +170,57 @@ class ClockSampler:
 # ---------------------------------------------------------------------------
 # CPU oracle timing (baseline / reference arm)
 # ---------------------------------------------------------------------------
-def oracle_sample_flops(w, rows):
-    if w.causal:
-        nvis = [min(int(r) + 1, w.Nk) for r in rows]
+def oracle_units(w):
+    """The oracle's units of work for a workload, one (batch, head) or one
+    (sequence, head) at a time: yields (tag, Nq, Nk, key/value loader)."""
+    from exact_attention_152_b200 import inputs
+    if w.packed:
+        kvh = w.H // w.kv_heads
+        for s, n in enumerate(w.seqlens):
+            if n == 0:
+                continue
+            for h in range(w.H):
+                yield (s, h), n, n, (lambda s=s, h=h: tuple(
+                    inputs.bf16_bits_to_f64(w.seq_head_bits(x, s, h // kvh)) for x in "kv"))
     else:
-        nvis = [w.Nk] * len(rows)
-    return 4.0 * w.d * float(sum(nvis))
+        for bh in range(w.B * w.H):
+            yield bh, w.Nq, w.Nk, (lambda bh=bh: tuple(
+                inputs.bf16_bits_to_f64(w.head_bits(x, w.kv_head_of(bh))) for x in "kv"))
 
 
 def time_oracle_rows(w, n_rows, seed_off):
-    """Time the oracle on n_rows seeded query rows, taken head by head (all rows
+    """Time the oracle on n_rows seeded query rows, taken unit by unit (all rows
     of a head, then the next) so large samples span several heads."""
     import oracle
     from exact_attention_152_b200 import inputs
-    tot_t, tot_f, done, heads = 0.0, 0.0, 0, 0
-    bh = 0
-    while done < n_rows and bh < w.B * w.H:
-        take = min(w.Nq, n_rows - done)
-        k = inputs.bf16_bits_to_f64(w.head_bits("k", w.kv_head_of(bh)))
-        v = inputs.bf16_bits_to_f64(w.head_bits("v", w.kv_head_of(bh)))
-        rows = inputs.sample_rows(w.seed + seed_off, bh, w.Nq, take)
-        q = inputs.bf16_bits_to_f64(w.q_rows_bits(bh, rows))
+    from exact_attention_152_b200.workloads import visible_keys
+    tot_t, tot_f, done, units = 0.0, 0.0, 0, 0
+    wl, wr = w.band
+    for i, (tag, nq, nk, load_kv) in enumerate(oracle_units(w)):
+        if done >= n_rows:
+            break
+        k, v = load_kv()
+        rows = inputs.sample_rows(w.seed + seed_off, i, nq, min(nq, n_rows - done))
+        if w.packed:
+            q = inputs.bf16_bits_to_f64(w.seq_head_bits("q", tag[0], tag[1], rows))
+        else:
+            q = inputs.bf16_bits_to_f64(w.q_rows_bits(tag, rows))
         t0 = time.perf_counter()
-        oracle.attn_rows(q, rows, k, v, w.scale, w.causal)
+        oracle.attn_rows_window(q, rows, k, v, w.scale, wl, wr)
         tot_t += time.perf_counter() - t0
-        tot_f += oracle_sample_flops(w, rows)
+        tot_f += 4.0 * w.d * float(visible_keys(rows, nk, wl, wr).sum())
         done += len(rows)
-        heads += 1
-        bh += 1
-    return tot_t, tot_f, done, heads
+        units += 1
+    return tot_t, tot_f, done, units
+
+
+def total_rows(w):
+    return (w.total if w.packed else w.B * w.Nq) * w.H
 
 
 def calibrate_rows(w, seconds):
     dt, _, n, _ = time_oracle_rows(w, 256, 1000)
-    return max(16, min(w.B * w.H * w.Nq, int(n * seconds / max(dt, 1e-6))))
+    return max(16, min(total_rows(w), int(n * seconds / max(dt, 1e-6))))
 
 
 def cpu_baseline(w, seconds):
@@ -207,19 +229,34 @@ def cpu_baseline(w, seconds):
     dt, flops, n, heads = time_oracle_rows(w, n, 2000)
     return {"value": flops / dt / 1e12, "unit": UNIT, "cores": oracle.default_threads(),
             "kind": "oracle",
-            "sample": f"{n} seeded query rows over {heads} head(s) of {w.name} (full key range"
-                      f"{', causal' if w.causal else ''}), fp64, {dt:.1f} s of oracle time; "
+            "sample": f"{n} seeded query rows over {heads} head(s) of {w.name} (visible keys "
+                      f"of band {w.band}), fp64, {dt:.1f} s of oracle time; "
                       f"value = those rows' algorithmic FLOPs / time"}
 
 
 def workload_config(w, n_gpus):
-    qkv_bytes = (w.B * (w.H * w.Nq + 2 * w.kv_heads * w.Nk) * w.d * 2)
-    return {"workload": w.name, "B": w.B, "H": w.H, "Hkv": w.kv_heads, "Nq": w.Nq, "Nk": w.Nk, "d": w.d,
-            "causal": w.causal, "scale": w.scale, "seed": w.seed, "per_gpu_problem": True,
-            "global_batch": w.B * n_gpus,
-            "l2": f"inputs {qkv_bytes / 1e6:.0f} MB {'>' if qkv_bytes > L2_BYTES else '<='} "
-                  f"126 MB L2; not flushed between steps",
-            "parallelism": f"independent problem per GPU x{n_gpus}"}
+    rows_q = w.total if w.packed else w.B * w.Nq
+    rows_k = w.total if w.packed else w.B * w.Nk
+    qkv_bytes = (w.H * rows_q + 2 * w.kv_heads * rows_k) * w.d * 2
+    cfg = {"workload": w.name, "B": w.B, "H": w.H, "Hkv": w.kv_heads, "Nq": w.Nq, "Nk": w.Nk, "d": w.d,
+           "causal": w.causal, "band": list(w.band), "scale": w.scale, "seed": w.seed,
+           "per_gpu_problem": True, "global_batch": w.B * n_gpus,
+           "l2": f"inputs {qkv_bytes / 1e6:.0f} MB {'>' if qkv_bytes > L2_BYTES else '<='} "
+                 f"126 MB L2; not flushed between steps",
+           "parallelism": f"independent problem per GPU x{n_gpus}"}
+    if w.packed:
+        cfg.update({"layout": "packed [total, H, d]", "num_seqs": len(w.seqlens),
+                    "total_tokens": w.total, "seqlen_min": min(w.seqlens),
+                    "seqlen_max": max(w.seqlens)})
+    return cfg
+
+
+def launch_name(w):
+    if w.packed:
+        return "attn_fwd_varlen"
+    if w.window is not None:
+        return "attn_fwd_window"
+    return "attn_fwd_gqa" if w.kv_heads != w.H else "attn_fwd"
 
 
 def run_reference(args):
@@ -246,7 +283,7 @@ def run_reference(args):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic", "config": workload_config(w, 1),
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": oracle.default_threads(), "kind": "oracle",
-                         "sample": f"each step: {n} seeded query rows (head by head, full key range), fp64"},
+                         "sample": f"each step: {n} seeded query rows (head by head, visible keys of band {w.band}), fp64"},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -275,16 +312,34 @@ def run_ours(args):
     # inputs: the workload's seeded BF16 tensors, resident in HBM
     host = {x: w.tensor_bits(x) for x in "qkv"}
     q, k, v = (torch.from_numpy(host[x].view(np.int16)).view(torch.bfloat16).to(dev) for x in "qkv")
-    o = torch.empty((w.B, w.H, w.Nq, w.d), dtype=torch.bfloat16, device=dev)
-    lse = torch.empty((w.B, w.H, w.Nq), dtype=torch.float32, device=dev)
+    if w.packed:
+        o = torch.empty((w.total, w.H, w.d), dtype=torch.bfloat16, device=dev)
+        lse = torch.empty((w.H, w.total), dtype=torch.float32, device=dev)
+        host_cu = torch.from_numpy(w.cu_seqlens)
+        cu = host_cu.to(dev)
+    else:
+        o = torch.empty((w.B, w.H, w.Nq, w.d), dtype=torch.bfloat16, device=dev)
+        lse = torch.empty((w.B, w.H, w.Nq), dtype=torch.float32, device=dev)
+        host_cu = cu = None
     stream = torch.cuda.current_stream(dev)
     sh = stream.cuda_stream
     knobs = args.exp_mode is not None or args.threshold is not None
     thr = 8.0 if args.threshold is None else args.threshold
     em = 1 if args.exp_mode is None else args.exp_mode
+    if knobs and (w.packed or w.window is not None or w.kv_heads != w.H):
+        raise SystemExit("--exp-mode/--threshold apply to dense workloads without a band only")
 
-    def launch(qp=q, kp=k, vp=v, op=o, lp=lse):
-        if w.kv_heads != w.H:
+    def launch(qp=q, kp=k, vp=v, op=o, lp=lse, cp=cu):
+        if w.packed:
+            rc = binding.attn_fwd_varlen(qp.data_ptr(), kp.data_ptr(), vp.data_ptr(), op.data_ptr(),
+                                         lp.data_ptr(), cp.data_ptr(), cp.data_ptr(), len(w.seqlens),
+                                         max(w.seqlens), w.total, w.total, w.H, w.kv_heads, w.d,
+                                         w.scale, w.band[0], w.band[1], sh)
+        elif w.window is not None:
+            rc = binding.attn_fwd_window(qp.data_ptr(), kp.data_ptr(), vp.data_ptr(), op.data_ptr(),
+                                         lp.data_ptr(), w.B, w.H, w.kv_heads, w.Nq, w.Nk, w.d,
+                                         w.scale, w.band[0], w.band[1], sh)
+        elif w.kv_heads != w.H:
             rc = binding.attn_fwd_gqa(qp.data_ptr(), kp.data_ptr(), vp.data_ptr(), op.data_ptr(),
                                       lp.data_ptr(), w.B, w.H, w.kv_heads, w.Nq, w.Nk, w.d, w.scale,
                                       int(w.causal), sh)
@@ -334,13 +389,17 @@ def run_ours(args):
     ho = torch.empty(o.shape, dtype=torch.bfloat16).pin_memory()
     hl = torch.empty(lse.shape, dtype=torch.float32).pin_memory()
     qd, kd, vd = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    hc = host_cu.pin_memory() if w.packed else None
+    cd = torch.empty_like(cu) if w.packed else None
     KE = args.e2e_steps
 
     def e2e_step():
         qd.copy_(hq, non_blocking=True)
         kd.copy_(hk, non_blocking=True)
         vd.copy_(hv, non_blocking=True)
-        launch(qd, kd, vd, o, lse)
+        if w.packed:
+            cd.copy_(hc, non_blocking=True)
+        launch(qd, kd, vd, o, lse, cd)
         ho.copy_(o, non_blocking=True)
         hl.copy_(lse, non_blocking=True)
 
@@ -361,7 +420,7 @@ def run_ours(args):
     binding.check(binding.attn_status_sync(sh), "e2e region")
     (te_ms,) = parallel.max_over_ranks([e0.elapsed_time(e1)], dev)
     e2e_value = world * w.flops * KE / (te_ms / 1e3) / 1e12
-    h2d = sum(x.numel() * x.element_size() for x in (hq, hk, hv))
+    h2d = sum(x.numel() * x.element_size() for x in (hq, hk, hv) + ((hc,) if w.packed else ()))
     d2h = ho.numel() * ho.element_size() + hl.numel() * hl.element_size()
 
     cpu = None
@@ -387,7 +446,8 @@ def run_ours(args):
                      "algorithmic_flops_per_launch": w.flops},
         "cpu_baseline": cpu,
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                "steps": KE, "path": "pinned host Q/K/V -> H2D -> attn_fwd (C-ABI) -> D2H of O and LSE"},
+                "steps": KE, "path": f"pinned host Q/K/V{' + offsets' if w.packed else ''} -> H2D -> "
+                        f"{launch_name(w)} (C-ABI) -> D2H of O and LSE"},
         "gpu_launches": K,
         "clocks": clocks,
         "kernel_src_sha": kernel_source_hash(),
@@ -399,10 +459,151 @@ def run_ours(args):
     return 0
 
 
+def bwd_cpu_baseline(w, seconds):
+    """The oracle's backward on the first n query rows of one head (all of its
+    keys), n sized to about `seconds` of CPU time; FLOPs counted as 2.5x the
+    forward's 4*d per visible pair."""
+    import oracle
+    from exact_attention_152_b200 import inputs
+    from exact_attention_152_b200.workloads import visible_keys
+    wl, wr = w.band
+    k, v = (inputs.bf16_bits_to_f64(w.head_bits(x, w.kv_head_of(0))) for x in "kv")
+    n, dt = 64, 0.0
+    while True:
+        rows = np.arange(n, dtype=np.int64)
+        q = inputs.bf16_bits_to_f64(w.q_rows_bits(0, rows))
+        g = inputs.bf16_bits_to_f64(inputs.gen_bf16_at(w.seed + 1, "q", rows[:, None] * w.d
+                                                       + np.arange(w.d)[None, :]))
+        t0 = time.perf_counter()
+        oracle.attn_bwd_head(q, k, v, g, w.scale, wl, wr)
+        dt = time.perf_counter() - t0
+        if dt > seconds / 4 or n >= w.Nq:
+            break
+        n = min(w.Nq, n * 4)
+    flops = 2.5 * 4.0 * w.d * float(visible_keys(rows, w.Nk, wl, wr).sum())
+    return {"value": flops / dt / 1e12, "unit": UNIT, "cores": 1, "kind": "oracle",
+            "sample": f"backward of the first {n} query rows of head 0 of {w.name} against all "
+                      f"its keys, fp64, one thread, {dt:.1f} s"}
+
+
+def run_ours_bwd(args):
+    """The backward pass: each step is one attn_bwd call (row sums, main
+    kernel, dQ rounding) over the whole workload, with O and LSE from one
+    forward call before timing."""
+    import torch
+
+    from exact_attention_152_b200 import binding, inputs
+    from exact_attention_152_b200.workloads import HEADLINE, WORKLOADS
+
+    rank, world, local_rank = dist_env()
+    if world > 1:
+        raise SystemExit("--pass bwd runs on one GPU")
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    w = WORKLOADS[args.workload or HEADLINE]
+    if w.packed or w.window is not None:
+        raise SystemExit("--pass bwd supports dense workloads, causal or not")
+    peaks = load_peaks()
+    host = {x: w.tensor_bits(x) for x in "qkv"}
+    host["do"] = inputs.gen_bf16(w.seed + 1, "q", w.shape("q"))
+    to_dev = lambda a: torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).to(dev)  # noqa: E731
+    q, k, v, do = (to_dev(host[x]) for x in ("q", "k", "v", "do"))
+    o, lse = binding.fwd(q, k, v, causal=w.causal, scale=w.scale)
+    stream = torch.cuda.current_stream(dev)
+    sh = stream.cuda_stream
+    ws_bytes = binding.attn_bwd_workspace_size(w.B, w.H, w.Nq, w.d)
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+
+    def launch(ins=(q, k, v, o, do, lse), outs=(dq, dk, dv)):
+        rc = binding.attn_bwd(*(t.data_ptr() for t in ins), *(t.data_ptr() for t in outs),
+                              ws.data_ptr(), ws_bytes, w.B, w.H, w.kv_heads, w.Nq, w.Nk, w.d,
+                              w.scale, int(w.causal), sh)
+        binding.check(rc, "attn_bwd")
+
+    launch()
+    binding.check(binding.attn_status_sync(sh), "first launch")
+    for _ in range(args.warmup):
+        launch()
+    binding.check(binding.attn_status_sync(sh), "warm-up")
+    for t in (dq, dk, dv):
+        assert bool(torch.isfinite(t.float()).all()), "non-finite gradient"
+    flops = 2.5 * w.flops
+    sampler = ClockSampler("GPU-" + str(torch.cuda.get_device_properties(dev).uuid))
+    K = args.steps
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(K + 1)]
+    torch.cuda.synchronize(dev)
+    sampler.start()
+    evs[0].record(stream)
+    for i in range(K):
+        launch()
+        evs[i + 1].record(stream)
+    torch.cuda.synchronize(dev)
+    clocks = sampler.stop()
+    binding.check(binding.attn_status_sync(sh), "timed region")
+    total_ms = evs[0].elapsed_time(evs[K])
+    call_ms = total_ms / K
+    value = flops * K / (total_ms / 1e3) / 1e12
+
+    # end to end: pinned host Q, K, V, O, dO, LSE -> H2D -> attn_bwd -> D2H dQ, dK, dV
+    pin = lambda t: t.cpu().pin_memory()  # noqa: E731
+    h_in = [pin(t) for t in (q, k, v, o, do, lse)]
+    h_out = [torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in (dq, dk, dv)]
+    d_in = [torch.empty_like(t) for t in (q, k, v, o, do, lse)]
+
+    def e2e_step():
+        for d_, h_ in zip(d_in, h_in):
+            d_.copy_(h_, non_blocking=True)
+        launch(tuple(d_in))
+        for h_, d_ in zip(h_out, (dq, dk, dv)):
+            h_.copy_(d_, non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    binding.check(binding.attn_status_sync(sh), "e2e region")
+    e2e_value = flops * args.e2e_steps / (e0.elapsed_time(e1) / 1e3) / 1e12
+    cpu = None if args.no_cpu_baseline else bwd_cpu_baseline(w, args.cpu_seconds)
+    peak = peaks["sustained"]
+    achieved = flops / (call_ms / 1e3) / 1e12
+    line = {
+        "metric": METRIC_BWD, "value": value, "unit": UNIT, "n_gpus": 1, "steps": K,
+        "warmup": args.warmup, "ms_per_step": call_ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": dict(workload_config(w, 1), **{"pass": "bwd", "dO": "N(0,1), seed + 1"}),
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": UNIT,
+                     "frac": achieved / peak, "traffic": None,
+                     "peak_kind": f"bf16_tflops_sustained ({peaks['source']})",
+                     "frac_of_burst": achieved / peaks["burst"],
+                     "frac_of_spec_2250": achieved / SPEC_DENSE_BF16_TFLOPS,
+                     "algorithmic_flops_per_launch": flops,
+                     "timed": "the whole attn_bwd call: row sums + main kernel + dQ rounding"},
+        "cpu_baseline": cpu,
+        "e2e": {"value": e2e_value, "unit": UNIT,
+                "h2d_bytes_per_step": sum(t.numel() * t.element_size() for t in h_in),
+                "d2h_bytes_per_step": sum(t.numel() * t.element_size() for t in h_out),
+                "steps": args.e2e_steps,
+                "path": "pinned host Q/K/V/O/dO/LSE -> H2D -> attn_bwd (C-ABI) -> D2H of dQ/dK/dV"},
+        "gpu_launches": 3 * K,
+        "clocks": clocks,
+        "kernel_src_sha": kernel_source_hash(),
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main(argv=None):
     args = parse_args(argv)
     if args.impl == "reference":
         return run_reference(args)
+    if args.which == "bwd":
+        return run_ours_bwd(args)
     return run_ours(args)
 
 

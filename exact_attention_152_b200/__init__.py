@@ -10,8 +10,9 @@ raises ImportError -- there is no fallback of any kind.
 from __future__ import annotations
 
 __all__ = [
-    "attn_fwd", "attn_fwd_config", "attn_fwd_gqa", "attn_status_sync", "attn_status_string",
-    "attn_last_error", "attn_selftest_timeout", "fwd", "AttnError",
+    "attn_fwd", "attn_fwd_config", "attn_fwd_gqa", "attn_fwd_window", "attn_fwd_varlen",
+    "attn_status_sync", "attn_status_string", "attn_last_error", "attn_selftest_timeout", "fwd",
+    "fwd_varlen", "attn_bwd", "attn_bwd_workspace_size", "bwd", "AttnError",
 ]
 
 

@@ -48,6 +48,16 @@ def lib() -> ctypes.CDLL:
             l.attn_fwd_gqa.argtypes = [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, ctypes.c_float, _I,
                                        _P]
             l.attn_fwd_gqa.restype = _I
+            l.attn_fwd_window.argtypes = [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I,
+                                          ctypes.c_float, _I, _I, _P]
+            l.attn_fwd_window.restype = _I
+            l.attn_fwd_varlen.argtypes = [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I,
+                                          ctypes.c_float, _I, _I, _P]
+            l.attn_fwd_varlen.restype = _I
+            l.attn_bwd.argtypes = [_P] * 10 + [ctypes.c_size_t] + [_I] * 6 + [ctypes.c_float, _I, _P]
+            l.attn_bwd.restype = _I
+            l.attn_bwd_workspace_size.argtypes = [_I, _I, _I, _I]
+            l.attn_bwd_workspace_size.restype = ctypes.c_size_t
             l.attn_status_sync.argtypes = [_P]
             l.attn_status_sync.restype = _I
             l.attn_status_string.argtypes = [_I]
@@ -68,10 +78,33 @@ def attn_fwd_gqa(q, k, v, o, lse, B, H, Hkv, Nq, Nk, d, scale, causal, stream) -
     return lib().attn_fwd_gqa(q, k, v, o, lse, B, H, Hkv, Nq, Nk, d, scale, causal, stream)
 
 
+def attn_fwd_window(q, k, v, o, lse, B, H, Hkv, Nq, Nk, d, scale, window_left, window_right,
+                    stream) -> int:
+    return lib().attn_fwd_window(q, k, v, o, lse, B, H, Hkv, Nq, Nk, d, scale, window_left,
+                                 window_right, stream)
+
+
+def attn_fwd_varlen(q, k, v, o, lse, cu_seqlens_q, cu_seqlens_k, num_seqs, max_seqlen_q, total_q,
+                    total_k, H, Hkv, d, scale, window_left, window_right, stream) -> int:
+    return lib().attn_fwd_varlen(q, k, v, o, lse, cu_seqlens_q, cu_seqlens_k, num_seqs,
+                                 max_seqlen_q, total_q, total_k, H, Hkv, d, scale, window_left,
+                                 window_right, stream)
+
+
 def attn_fwd_config(q, k, v, o, lse, B, H, Nq, Nk, d, scale, causal, rescale_threshold,
                     exp_mode, rescale_count, stream) -> int:
     return lib().attn_fwd_config(q, k, v, o, lse, B, H, Nq, Nk, d, scale, causal,
                                  rescale_threshold, exp_mode, rescale_count, stream)
+
+
+def attn_bwd(q, k, v, o, dout, lse, dq, dk, dv, workspace, workspace_bytes, B, H, Hkv, Nq, Nk, d,
+             scale, causal, stream) -> int:
+    return lib().attn_bwd(q, k, v, o, dout, lse, dq, dk, dv, workspace, workspace_bytes, B, H, Hkv,
+                          Nq, Nk, d, scale, causal, stream)
+
+
+def attn_bwd_workspace_size(B, H, Nq, d) -> int:
+    return lib().attn_bwd_workspace_size(B, H, Nq, d)
 
 
 def attn_status_sync(stream) -> int:
@@ -104,14 +137,24 @@ def check(code: int, where: str = "attn") -> None:
         raise AttnError(code, where)
 
 
-def fwd(q, k, v, causal: bool = False, scale: float | None = None, *, out=None, lse=None,
-        return_lse: bool = True, rescale_threshold: float | None = None,
+def _check_bf16(**tensors):
+    import torch
+    for name, t in tensors.items():
+        if not isinstance(t, torch.Tensor) or t.dtype != torch.bfloat16 or not t.is_cuda:
+            raise TypeError(f"{name} must be a bfloat16 CUDA tensor")
+        if not t.is_contiguous():
+            raise ValueError(f"{name} must be contiguous")
+
+
+def fwd(q, k, v, causal: bool = False, scale: float | None = None, *, window=None, out=None,
+        lse=None, return_lse: bool = True, rescale_threshold: float | None = None,
         exp_mode: int | None = None, rescale_count=None):
     """O (and LSE) for BF16 CUDA tensors q [B,H,Nq,d], k/v [B,Hkv,Nk,d].
 
     Hkv < H (H % Hkv == 0) selects grouped-query attention (attn_fwd_gqa).
-    scale defaults to 1/sqrt(d).  Runs on torch's current stream; returns
-    (o, lse) or o.  Raises AttnError on any non-zero status.
+    window=(left, right) selects the key band of attn_fwd_window (-1: no bound;
+    it replaces ``causal``).  scale defaults to 1/sqrt(d).  Runs on torch's
+    current stream; returns (o, lse) or o.  Raises AttnError on any non-zero status.
     """
     import torch
 
@@ -132,6 +175,15 @@ def fwd(q, k, v, causal: bool = False, scale: float | None = None, *, out=None, 
         lse = torch.empty((B, H, Nq), dtype=torch.float32, device=q.device)
     stream = torch.cuda.current_stream(q.device).cuda_stream
     lse_ptr = lse.data_ptr() if lse is not None else None
+    knobs = rescale_threshold is not None or exp_mode is not None or rescale_count is not None
+    if window is not None:
+        if causal or knobs:
+            raise ValueError("window replaces causal and takes no softmax knobs")
+        rc = attn_fwd_window(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse_ptr,
+                             B, H, Hkv, Nq, Nk, d, float(scale), int(window[0]), int(window[1]),
+                             stream)
+        check(rc, "attn_fwd_window")
+        return (out, lse) if return_lse else out
     if Hkv != H:
         if rescale_threshold is not None or exp_mode is not None or rescale_count is not None:
             raise ValueError("the softmax knobs are available for Hkv == H only")
@@ -149,3 +201,79 @@ def fwd(q, k, v, causal: bool = False, scale: float | None = None, *, out=None, 
                              stream)
     check(rc, "attn_fwd")
     return (out, lse) if return_lse else out
+
+
+def fwd_varlen(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q: int, causal: bool = False,
+               scale: float | None = None, *, window=None, out=None, lse=None,
+               return_lse: bool = True):
+    """Packed variable-length batch: q [total_q, H, d], k/v [total_k, Hkv, d]
+    BF16 CUDA tensors, cu_seqlens_* int32 CUDA tensors of num_seqs + 1 offsets.
+    Returns (o [total_q, H, d], lse [H, total_q]) or o.  ``window`` = (left,
+    right) band over positions within each sequence (replaces ``causal``)."""
+    import torch
+
+    _check_bf16(q=q, k=k, v=v)
+    if q.dim() != 3 or k.dim() != 3 or v.dim() != 3:
+        raise ValueError("q, k, v must be [total, heads, d]")
+    total_q, H, d = q.shape
+    total_k, Hkv = k.shape[0], k.shape[1]
+    if tuple(k.shape) != (total_k, Hkv, d) or tuple(v.shape) != (total_k, Hkv, d):
+        raise ValueError("k and v must be [total_k, Hkv, d] matching q")
+    for name, c in (("cu_seqlens_q", cu_seqlens_q), ("cu_seqlens_k", cu_seqlens_k)):
+        if not isinstance(c, torch.Tensor) or c.dtype != torch.int32 or not c.is_cuda \
+                or c.dim() != 1 or not c.is_contiguous():
+            raise TypeError(f"{name} must be a contiguous int32 CUDA vector")
+    if cu_seqlens_q.numel() != cu_seqlens_k.numel() or cu_seqlens_q.numel() < 1:
+        raise ValueError("cu_seqlens_q and cu_seqlens_k need the same num_seqs + 1 entries")
+    num_seqs = cu_seqlens_q.numel() - 1
+    if window is None:
+        window = (-1, 0) if causal else (-1, -1)
+    elif causal:
+        raise ValueError("window replaces causal")
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if out is None:
+        out = torch.empty((total_q, H, d), dtype=torch.bfloat16, device=q.device)
+    if return_lse and lse is None:
+        lse = torch.empty((H, total_q), dtype=torch.float32, device=q.device)
+    stream = torch.cuda.current_stream(q.device).cuda_stream
+    rc = attn_fwd_varlen(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                         lse.data_ptr() if lse is not None else None, cu_seqlens_q.data_ptr(),
+                         cu_seqlens_k.data_ptr(), num_seqs, int(max_seqlen_q), total_q, total_k,
+                         H, Hkv, d, float(scale), int(window[0]), int(window[1]), stream)
+    check(rc, "attn_fwd_varlen")
+    return (out, lse) if return_lse else out
+
+
+def bwd(q, k, v, o, dout, lse, causal: bool = False, scale: float | None = None, *,
+        workspace=None):
+    """Gradients (dq, dk, dv) for BF16 CUDA tensors q/o/dout [B,H,Nq,d], k/v
+    [B,Hkv,Nk,d] and the forward's fp32 lse [B,H,Nq].  The workspace (a uint8
+    CUDA tensor of at least attn_bwd_workspace_size bytes) is allocated with
+    torch when not given.  Runs on torch's current stream."""
+    import torch
+
+    _check_bf16(q=q, k=k, v=v, o=o, dout=dout)
+    B, H, Nq, d = q.shape
+    Hkv, Nk = k.shape[1], k.shape[2]
+    if tuple(o.shape) != tuple(q.shape) or tuple(dout.shape) != tuple(q.shape):
+        raise ValueError("o and dout must match q")
+    if tuple(k.shape) != (B, Hkv, Nk, d) or tuple(v.shape) != (B, Hkv, Nk, d):
+        raise ValueError("k and v must be [B, Hkv, Nk, d] matching q")
+    if lse.dtype != torch.float32 or not lse.is_contiguous() or tuple(lse.shape) != (B, H, Nq):
+        raise ValueError("lse must be contiguous float32 [B, H, Nq]")
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    need = attn_bwd_workspace_size(B, H, Nq, d)
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
+    dq = torch.empty_like(q)
+    dk = torch.empty_like(k)
+    dv = torch.empty_like(v)
+    stream = torch.cuda.current_stream(q.device).cuda_stream
+    rc = attn_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), dout.data_ptr(),
+                  lse.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), workspace.data_ptr(),
+                  workspace.numel() * workspace.element_size(), B, H, Hkv, Nq, Nk, d, float(scale),
+                  int(bool(causal)), stream)
+    check(rc, "attn_bwd")
+    return dq, dk, dv

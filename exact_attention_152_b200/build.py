@@ -24,7 +24,7 @@ BUILD = os.path.join(HERE, "_build")
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 TARGETS = {
-    "libattn.so": ["attn_fwd.cu"],
+    "libattn.so": ["attn_fwd.cu", "attn_bwd.cu"],
     "libattn_blocks.so": ["blocks.cu"],
 }
 

@@ -1,0 +1,752 @@
+// Exact attention backward for B200 (sm_100a): dQ, dK, dV from Q, K, V, O, dO
+// and the forward's log-sum-exp, with the score matrix recomputed tile by tile
+// on the tensor cores (tcgen05, accumulators in Tensor Memory) and never stored.
+//
+// What is computed (the pages name the backward pass as what FlashAttention 4
+// still lacks -- FlashAttention 4 page, ja.linux-konsole.com, sections
+// "重要ポイント" and "互換性と現状"; "FlashAttention-4：非対称ハードウェアスケーリング…" (sns.style),
+// section 二 -- and give no formula): the chain rule through the forward
+// definition of include/attn.h, per (b, h), query row i, visible key j:
+//
+//   P_ij  = exp(scale * <q_i, k_j> - LSE_i)
+//   dP_ij = <dO_i, v_j>,   D_i = <dO_i, O_i>,   dS_ij = P_ij (dP_ij - D_i)
+//   dV_j  = sum_i P_ij dO_i
+//   dK_j  = scale * sum_i dS_ij q_i
+//   dQ_i  = scale * sum_j dS_ij k_j
+//
+// Design (this library's, for sm_100a):
+//  * Three launches: a row-sum kernel for D (and dQ's fp32 accumulator is
+//    zeroed), the main kernel, and a kernel that scales and rounds dQ to BF16.
+//    D and the dQ accumulator live in a caller-provided workspace.
+//  * Main kernel: one CTA per (b, key/value head, 128-key block).  K and V of
+//    the block stay in shared memory; the CTA walks every query tile (128
+//    rows) of every query head that reads this key/value head (causal: only
+//    tiles at or below the diagonal), double-buffering Q and dO by TMA.
+//  * Per query tile, five BF16 GEMMs on the tensor cores, all with M = 128
+//    keys or queries:
+//        S^T  = K Q^T          (keys x queries, TMEM columns [0, 128))
+//        dP^T = V dO^T         (TMEM columns [128, 256))
+//        dV  += P^T dO         (A = P^T straight from TMEM; TMEM [256, 256+d))
+//        dK  += dS^T Q         (A = dS^T from TMEM;          TMEM [256+d, 256+2d))
+//        dQ_i = dS K           (A = dS from shared memory, MN-major; TMEM [0, d))
+//    Because the tiles are computed transposed (keys on the TMEM lanes), P^T
+//    and dS^T are the A operands of the dV and dK GEMMs as they stand.
+//  * Warps 0-7 turn S^T and dP^T into P^T and dS^T (one key row per thread,
+//    half of the query columns per warp) and write them back to TMEM as BF16
+//    pairs over the first half of their own columns; dS also goes to shared
+//    memory for the dQ GEMM.  Warps 8-11 drain each dQ tile from TMEM into the
+//    fp32 accumulator with vector reductions.  Warp 12 loads (TMA), warp 13
+//    issues the MMAs from one thread.
+//  * Every wait is bounded; a timeout sets this file's status word and the CTA
+//    leaves its loops and exits cleanly.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstdint>
+#include <mutex>
+
+#include "attn.h"
+#include "host_common.h"
+#include "sm100.cuh"
+#include "tmap.h"
+
+namespace eab {
+namespace bwd {
+
+constexpr int kBlockK = 128;  // keys per CTA (TMEM lanes of S^T, dP^T, dV, dK)
+constexpr int kBlockQ = 128;  // queries per tile
+constexpr int kWarpDrain = 8;
+constexpr int kWarpLoad = 12;
+constexpr int kWarpMma = 13;
+constexpr int kNumThreads = 512;
+constexpr uint32_t kTmemCols = 512;
+constexpr uint64_t kWaitTimeoutNs = 2000000000ull;
+constexpr float kLog2e = 1.4426950408889634f;
+
+constexpr unsigned int kStatusTimeout = kStatusWordTimeout;
+constexpr unsigned int kStatusSmemAlign = 4u;  // mapped to kStatusWordLaunch on the host
+
+__device__ unsigned int g_status_bwd;
+
+template <int D>
+struct Cfg {
+  static_assert(D == 64 || D == 128, "head dim");
+  static constexpr int kBoxes = D / 64;
+  static constexpr int kBoxBytes = 128 * 128;       // 128 rows x 64 bf16
+  static constexpr int kTileBytes = kBoxes * kBoxBytes;
+  static constexpr int kOffK = 0;
+  static constexpr int kOffV = kTileBytes;
+  static constexpr int kOffQ = 2 * kTileBytes;      // 2 stages
+  static constexpr int kOffDO = 4 * kTileBytes;     // 2 stages
+  static constexpr int kOffDS = 6 * kTileBytes;     // dS, 128 queries x 128 keys, MN-major
+  static constexpr int kDSBytes = 2 * kBoxBytes;
+  static constexpr int kOffRow = kOffDS + kDSBytes; // per stage: LSE*log2e [128], D [128]
+  static constexpr int kRowBytes = 2 * 2 * kBlockQ * 4;
+  static constexpr int kNumBars = 11;
+  static constexpr int kOffBar = kOffRow + kRowBytes;
+  static constexpr int kOffMisc = kOffBar + kNumBars * 8;
+  static constexpr int kSmemBytes = kOffMisc + 16;
+  static constexpr uint32_t kTmemDP = 128;
+  static constexpr uint32_t kTmemDV = 256;
+  static constexpr uint32_t kTmemDK = 256 + D;
+  static_assert(kSmemBytes <= 232448, "shared memory");
+};
+
+struct BwdParams {
+  const float* lse;    // [B*H, Nq], natural log
+  const float* dsum;   // D = rowsum(dO * O), [B*H, Nq]
+  float* dq_acc;       // [B*H, Nq, d] fp32, zeroed before the launch
+  uint64_t timeout_ns;
+  int Nq, Nk, H, group, n_kblocks, n_qtiles;
+  int causal;
+  float scale_log2;    // scale * log2(e)
+  float scale;
+};
+
+template <int D>
+struct Smem {
+  uint8_t* base;
+  uint32_t sbase;
+  __device__ __forceinline__ uint32_t k() const { return sbase + Cfg<D>::kOffK; }
+  __device__ __forceinline__ uint32_t v() const { return sbase + Cfg<D>::kOffV; }
+  __device__ __forceinline__ uint32_t q(int s) const { return sbase + Cfg<D>::kOffQ + s * Cfg<D>::kTileBytes; }
+  __device__ __forceinline__ uint32_t dout(int s) const { return sbase + Cfg<D>::kOffDO + s * Cfg<D>::kTileBytes; }
+  __device__ __forceinline__ uint32_t ds() const { return sbase + Cfg<D>::kOffDS; }
+  __device__ __forceinline__ float* lse2(int s) const {
+    return reinterpret_cast<float*>(base + Cfg<D>::kOffRow) + s * 2 * kBlockQ;
+  }
+  __device__ __forceinline__ float* dsum(int s) const { return lse2(s) + kBlockQ; }
+  __device__ __forceinline__ uint32_t bar(int i) const { return sbase + Cfg<D>::kOffBar + 8 * i; }
+  __device__ __forceinline__ uint32_t kv_full() const { return bar(0); }
+  __device__ __forceinline__ uint32_t q_full(int s) const { return bar(1 + s); }
+  __device__ __forceinline__ uint32_t q_empty(int s) const { return bar(3 + s); }
+  __device__ __forceinline__ uint32_t s_full() const { return bar(5); }
+  __device__ __forceinline__ uint32_t dp_full() const { return bar(6); }
+  __device__ __forceinline__ uint32_t p_ready() const { return bar(7); }
+  __device__ __forceinline__ uint32_t dq_full() const { return bar(8); }
+  __device__ __forceinline__ uint32_t dq_free() const { return bar(9); }
+  __device__ __forceinline__ uint32_t done() const { return bar(10); }
+  __device__ __forceinline__ uint32_t* tmem_slot() const {
+    return reinterpret_cast<uint32_t*>(base + Cfg<D>::kOffMisc);
+  }
+};
+
+// The work of one CTA: key block j of key/value head bh_kv; iterations walk the
+// group's query heads, and within each its query tiles i_lo .. n_qtiles-1.
+struct Work {
+  int bh_kv, j, b, hkv, i_lo, tiles_per_head, n_it;
+  __device__ __forceinline__ int head_of(int it) const { return it / tiles_per_head; }
+  __device__ __forceinline__ int tile_of(int it) const { return i_lo + it % tiles_per_head; }
+};
+
+__device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, uint64_t timeout_ns) {
+  const bool ok = mbar_wait(bar, parity, timeout_ns);
+  return __all_sync(0xffffffffu, ok);
+}
+
+// ---------------------------------------------------------------------------
+// MMA issue (one thread), fully unrolled with immediate descriptor offsets.
+// ---------------------------------------------------------------------------
+template <int D, int KK>
+struct Mma {
+  // K-major A and B, K = d: 32 bytes per K step in a 128-byte row, a new
+  // 64-column box every 4 steps (S^T = K Q^T, dP^T = V dO^T).
+  __device__ __forceinline__ static void kmajor(uint32_t d, uint32_t a_lo, uint32_t a_hi, uint32_t b_lo,
+                                                uint32_t b_hi, uint32_t idesc) {
+    if constexpr (KK < D / 16) {
+      constexpr uint32_t off = ((KK >> 2) * Cfg<D>::kBoxBytes + (KK & 3) * 32) >> 4;
+      mma_ss_imm<off, off, KK == 0 ? 0u : 1u>(d, a_lo, a_hi, b_lo, b_hi, idesc);
+      Mma<D, KK + 1>::kmajor(d, a_lo, a_hi, b_lo, b_hi, idesc);
+    }
+  }
+  // A from TMEM (BF16 pairs; queries [64h, 64h+64) in columns [64h, 64h+32)),
+  // B MN-major (rows of 16 queries = 2048 bytes per K step): dV, dK.
+  __device__ __forceinline__ static void tmem_a(uint32_t d, uint32_t a_tmem, uint32_t b_lo,
+                                                uint32_t b_hi, uint32_t idesc, uint32_t acc) {
+    if constexpr (KK < kBlockQ / 16) {
+      constexpr uint32_t a_off = (KK >> 2) * 64 + (KK & 3) * 8;
+      constexpr uint32_t b_off = (KK * 2048) >> 4;
+      mma_ts_imm<a_off, b_off>(d, a_tmem, b_lo, b_hi, idesc, KK == 0 ? acc : 1u);
+      Mma<D, KK + 1>::tmem_a(d, a_tmem, b_lo, b_hi, idesc, acc);
+    }
+  }
+  // A and B both MN-major, K = 128 keys, 2048 bytes per K step: dQ = dS K.
+  __device__ __forceinline__ static void mnmajor(uint32_t d, uint32_t a_lo, uint32_t a_hi, uint32_t b_lo,
+                                                 uint32_t b_hi, uint32_t idesc) {
+    if constexpr (KK < kBlockK / 16) {
+      constexpr uint32_t off = (KK * 2048) >> 4;
+      mma_ss_imm<off, off, KK == 0 ? 0u : 1u>(d, a_lo, a_hi, b_lo, b_hi, idesc);
+      Mma<D, KK + 1>::mnmajor(d, a_lo, a_hi, b_lo, b_hi, idesc);
+    }
+  }
+};
+
+// ---------------------------------------------------------------------------
+// Producer warp: K, V once; then Q, dO (TMA) and LSE, D (plain loads) per tile.
+// ---------------------------------------------------------------------------
+template <int D>
+__device__ __forceinline__ void producer_role(const Smem<D>& sm, const CUtensorMap* tm_q,
+                                              const CUtensorMap* tm_k, const CUtensorMap* tm_v,
+                                              const CUtensorMap* tm_do, const BwdParams& prm,
+                                              const Work& w, int lane) {
+  using C = Cfg<D>;
+  if (lane == 0) {
+    mbar_arrive_expect_tx(sm.kv_full(), 2 * C::kTileBytes);
+#pragma unroll
+    for (int b = 0; b < C::kBoxes; ++b) {
+      tma_load_3d(sm.k() + b * C::kBoxBytes, tm_k, b * 64, w.j * kBlockK, w.bh_kv, sm.kv_full());
+      tma_load_3d(sm.v() + b * C::kBoxBytes, tm_v, b * 64, w.j * kBlockK, w.bh_kv, sm.kv_full());
+    }
+  }
+  bool ok = true;
+  int it = 0;
+  for (; it < w.n_it; ++it) {
+    const int s = it & 1;
+    const uint32_t ph = (it >> 1) & 1;
+    ok = warp_wait(sm.q_empty(s), ph ^ 1u, prm.timeout_ns);
+    if (!ok) break;
+    const int bh = w.b * prm.H + w.hkv * prm.group + w.head_of(it);
+    const int q0 = w.tile_of(it) * kBlockQ;
+    // rows past Nq: LSE = +inf makes P = 0 there; D = 0
+    float* l2 = sm.lse2(s);
+    float* dd = sm.dsum(s);
+#pragma unroll
+    for (int r = lane; r < kBlockQ; r += 32) {
+      const int q = q0 + r;
+      const bool in = q < prm.Nq;
+      const size_t row = static_cast<size_t>(bh) * prm.Nq + q;
+      l2[r] = in ? prm.lse[row] * kLog2e : INFINITY;
+      dd[r] = in ? prm.dsum[row] : 0.0f;
+    }
+    if (lane == 0) {
+      mbar_arrive_expect_tx(sm.q_full(s), 2 * C::kTileBytes);
+#pragma unroll
+      for (int b = 0; b < C::kBoxes; ++b) {
+        tma_load_3d(sm.q(s) + b * C::kBoxBytes, tm_q, b * 64, q0, bh, sm.q_full(s));
+        tma_load_3d(sm.dout(s) + b * C::kBoxBytes, tm_do, b * 64, q0, bh, sm.q_full(s));
+      }
+    } else {
+      mbar_arrive(sm.q_full(s));
+    }
+  }
+  // never leave with a copy in flight
+  if (lane == 0) {
+    mbar_wait(sm.kv_full(), 0, prm.timeout_ns);
+    for (int i = it > 2 ? it - 2 : 0; i < it; ++i)
+      mbar_wait(sm.q_full(i & 1), (i >> 1) & 1, prm.timeout_ns);
+    if (!ok) atomicOr(&g_status_bwd, kStatusTimeout);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// MMA issuer: one thread.
+// ---------------------------------------------------------------------------
+template <int D>
+__device__ __forceinline__ void mma_role(const Smem<D>& sm, uint32_t tmem, const Work& w,
+                                         uint64_t timeout) {
+  using C = Cfg<D>;
+  constexpr uint32_t id_sq = idesc_bf16_f32(kBlockK, kBlockQ, false, false);  // S^T, dP^T
+  constexpr uint32_t id_kv = idesc_bf16_f32(kBlockK, D, false, true);         // dV, dK
+  constexpr uint32_t id_q = idesc_bf16_f32(kBlockQ, D, true, true);           // dQ
+  const uint64_t dk_ = sdesc_sw128(sm.k(), 16, 1024), dv_ = sdesc_sw128(sm.v(), 16, 1024);
+  const uint64_t dq_ = sdesc_sw128(sm.q(0), 16, 1024), do_ = sdesc_sw128(sm.dout(0), 16, 1024);
+  // MN-major views: Q, dO and K as B operands along d; dS as the A operand
+  const uint64_t qmn = sdesc_sw128(sm.q(0), C::kBoxBytes, 1024);
+  const uint64_t domn = sdesc_sw128(sm.dout(0), C::kBoxBytes, 1024);
+  const uint64_t kmn = sdesc_sw128(sm.k(), C::kBoxBytes, 1024);
+  const uint64_t dsmn = sdesc_sw128(sm.ds(), Cfg<D>::kBoxBytes, 1024);
+  auto lo = [](uint64_t x) { return static_cast<uint32_t>(x); };
+  auto hi = [](uint64_t x) { return static_cast<uint32_t>(x >> 32); };
+  constexpr uint32_t kStageStep = C::kTileBytes >> 4;
+
+  bool ok = mbar_wait(sm.kv_full(), 0, timeout);
+  for (int it = 0; ok && it < w.n_it; ++it) {
+    const int s = it & 1;
+    ok = mbar_wait(sm.q_full(s), (it >> 1) & 1, timeout);
+    if (!ok) break;
+    tc_fence_after();
+    // dP^T = V dO^T (its columns were last read by dK of the previous tile,
+    // issued earlier by this thread: MMAs execute in issue order)
+    Mma<D, 0>::kmajor(tmem + C::kTmemDP, lo(dv_), hi(dv_), lo(do_) + s * kStageStep, hi(do_), id_sq);
+    tc_commit(sm.dp_full());
+    // S^T = K Q^T into the columns of the previous dQ tile, once it is drained
+    if (it > 0) {
+      ok = mbar_wait(sm.dq_free(), (it - 1) & 1, timeout);
+      if (!ok) break;
+      tc_fence_after();
+    }
+    Mma<D, 0>::kmajor(tmem, lo(dk_), hi(dk_), lo(dq_) + s * kStageStep, hi(dq_), id_sq);
+    tc_commit(sm.s_full());
+    ok = mbar_wait(sm.p_ready(), it & 1, timeout);
+    if (!ok) break;
+    tc_fence_after();
+    const uint32_t acc = it > 0 ? 1u : 0u;
+    Mma<D, 0>::tmem_a(tmem + C::kTmemDV, tmem, lo(domn) + s * kStageStep, hi(domn), id_kv, acc);
+    Mma<D, 0>::tmem_a(tmem + C::kTmemDK, tmem + C::kTmemDP, lo(qmn) + s * kStageStep, hi(qmn), id_kv,
+                      acc);
+    tc_commit(sm.q_empty(s));
+    Mma<D, 0>::mnmajor(tmem, lo(dsmn), hi(dsmn), lo(kmn), hi(kmn), id_q);
+    tc_commit(sm.dq_full());
+  }
+  tc_commit(sm.done());
+  mbar_wait(sm.done(), 0, timeout);
+  if (!ok) atomicOr(&g_status_bwd, kStatusTimeout);
+}
+
+// ---------------------------------------------------------------------------
+// Warps 0-7: P^T and dS^T from S^T and dP^T.  Warp (c, q) owns TMEM lanes
+// 32q..32q+31 (keys) and query columns [64c, 64c+64).
+// ---------------------------------------------------------------------------
+template <int D, bool CAUSAL>
+__device__ __forceinline__ bool softmax_grad_role(const Smem<D>& sm, uint32_t tmem,
+                                                  const BwdParams& prm, const Work& w) {
+  using C = Cfg<D>;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int q4 = warp & 3, c = warp >> 2;
+  const int r = q4 * 32 + lane;          // key row within the block
+  const int key = w.j * kBlockK + r;
+  const bool key_in = key < prm.Nk;
+  const uint32_t lane_off = static_cast<uint32_t>(q4 * 32) << 16;
+  const uint32_t tS = tmem + lane_off + c * 64;
+  const uint32_t tP = tmem + lane_off + C::kTmemDP + c * 64;
+  uint8_t* ds_row = sm.base + C::kOffDS + c * C::kBoxBytes + r * 128;
+  bool ok = true;
+  for (int it = 0; it < w.n_it; ++it) {
+    const int s = it & 1;
+    // q_full orders the producer's LSE / D rows of this stage before the reads
+    // below (long complete by now); it cannot run two phases ahead, since the
+    // stage is refilled only after this tile's p_ready.
+    ok = warp_wait(sm.q_full(s), (it >> 1) & 1, prm.timeout_ns) &&
+         warp_wait(sm.s_full(), it & 1, prm.timeout_ns) &&
+         warp_wait(sm.dp_full(), it & 1, prm.timeout_ns);
+    if (!ok) break;
+    tc_fence_after();
+    const int q_base = w.tile_of(it) * kBlockQ + c * 64;  // first query of this warp's columns
+    // masking: key tail, or (causal) a key past some query of the block
+    const bool masked = !key_in || (CAUSAL && w.j * kBlockK + q4 * 32 + 31 > q_base);
+    const float* l2 = sm.lse2(s) + c * 64;
+    const float* dd = sm.dsum(s) + c * 64;
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+      uint32_t sv[32], pv[32];
+      tmem_ld32(tS + 32 * k, sv);
+      tmem_ld32(tP + 32 * k, pv);
+      tmem_ld_wait();
+      reg_fence32(sv);
+      reg_fence32(pv);
+      uint32_t pp[16], dsp[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        float p2[2], d2[2];
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const int col = 32 * k + 2 * i + e;
+          float x = fmaf(__uint_as_float(sv[2 * i + e]), prm.scale_log2, -l2[col]);
+          if (masked && (!key_in || (CAUSAL && key > q_base + col))) x = -INFINITY;
+          const float p = ex2_mufu(x);
+          p2[e] = p;
+          d2[e] = p * (__uint_as_float(pv[2 * i + e]) - dd[col]);
+        }
+        pp[i] = pack_bf16x2(p2[0], p2[1]);
+        dsp[i] = pack_bf16x2(d2[0], d2[1]);
+      }
+      tmem_st16(tS + 16 * k, pp);
+      tmem_st16(tP + 16 * k, dsp);
+      // dS for the dQ GEMM: key row r of the 64-query block c, columns
+      // [32k, 32k+32) = 16-byte chunks 4k..4k+3, 128-byte swizzle
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int chunk = (4 * k + i) ^ (r & 7);
+        *reinterpret_cast<uint4*>(ds_row + chunk * 16) =
+            make_uint4(dsp[4 * i], dsp[4 * i + 1], dsp[4 * i + 2], dsp[4 * i + 3]);
+      }
+    }
+    tmem_st_wait();
+    fence_proxy_async_smem();
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(sm.p_ready());
+  }
+  return ok;
+}
+
+// Warps 8-11: dQ tile (queries on the TMEM lanes) -> fp32 accumulator.
+template <int D>
+__device__ __forceinline__ bool dq_drain_role(const Smem<D>& sm, uint32_t tmem, const BwdParams& prm,
+                                              const Work& w) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int q4 = warp & 3;
+  const uint32_t tQ = tmem + (static_cast<uint32_t>(q4 * 32) << 16);
+  bool ok = true;
+  for (int it = 0; it < w.n_it; ++it) {
+    ok = warp_wait(sm.dq_full(), it & 1, prm.timeout_ns);
+    if (!ok) break;
+    tc_fence_after();
+    const int bh = w.b * prm.H + w.hkv * prm.group + w.head_of(it);
+    const int q = w.tile_of(it) * kBlockQ + q4 * 32 + lane;
+    float* dst = prm.dq_acc + (static_cast<size_t>(bh) * prm.Nq + q) * D;
+#pragma unroll
+    for (int cc = 0; cc < D / 32; ++cc) {
+      uint32_t v[32];
+      tmem_ld32(tQ + 32 * cc, v);
+      tmem_ld_wait();
+      reg_fence32(v);
+      if (q < prm.Nq) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+          asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(dst + 32 * cc + 4 * i),
+                       "f"(__uint_as_float(v[4 * i])), "f"(__uint_as_float(v[4 * i + 1])),
+                       "f"(__uint_as_float(v[4 * i + 2])), "f"(__uint_as_float(v[4 * i + 3]))
+                       : "memory");
+      }
+    }
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(sm.dq_free());
+  }
+  return ok;
+}
+
+// Warps 0-7 after the last tile: dV and scale * dK -> BF16 -> shared memory ->
+// TMA store.  d = 128: warp (c, q) stores output columns [64c, 64c+64) of both;
+// d = 64: warp (0, q) stores dV, warp (1, q) stores dK.
+template <int D>
+__device__ __forceinline__ bool epilogue(const Smem<D>& sm, uint32_t tmem, const CUtensorMap* tm_dk,
+                                         const CUtensorMap* tm_dv, const BwdParams& prm,
+                                         const Work& w, bool ok) {
+  using C = Cfg<D>;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int q4 = warp & 3, c = warp >> 2;
+  ok = ok && warp_wait(sm.done(), 0, prm.timeout_ns);
+  if (!ok) return false;
+  tc_fence_after();
+  const uint32_t lane_off = static_cast<uint32_t>(q4 * 32) << 16;
+  constexpr int kBoxesPerWarp = D == 128 ? 2 : 1;
+#pragma unroll
+  for (int bx = 0; bx < kBoxesPerWarp; ++bx) {
+    // which tensor and which 64 columns
+    const bool is_k = D == 128 ? bx == 1 : c == 1;
+    const int col0 = D == 128 ? c * 64 : 0;
+    const uint32_t src = tmem + lane_off + (is_k ? C::kTmemDK : C::kTmemDV) + col0;
+    const float mul = is_k ? prm.scale : 1.0f;
+    // staging: 4 KiB per (warp, box) inside the Q stages (free by now)
+    uint8_t* stage = sm.base + C::kOffQ + (warp * kBoxesPerWarp + bx) * 4096;
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      uint32_t v[32];
+      tmem_ld32(src + 32 * h, v);
+      tmem_ld_wait();
+      reg_fence32(v);
+      uint32_t wv[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i)
+        wv[i] = pack_bf16x2(__uint_as_float(v[2 * i]) * mul, __uint_as_float(v[2 * i + 1]) * mul);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int chunk = (4 * h + i) ^ (lane & 7);
+        *reinterpret_cast<uint4*>(stage + lane * 128 + chunk * 16) =
+            make_uint4(wv[4 * i], wv[4 * i + 1], wv[4 * i + 2], wv[4 * i + 3]);
+      }
+    }
+    fence_proxy_async_smem();
+    __syncwarp();
+    const int row0 = w.j * kBlockK + q4 * 32;
+    if (lane == 0 && row0 < prm.Nk) {
+      tma_store_3d(is_k ? tm_dk : tm_dv, smem_u32(stage), col0, row0, w.bh_kv);
+      bulk_commit_group();
+    }
+  }
+  if (lane == 0) bulk_wait_group0();
+  return true;
+}
+
+template <int D, bool CAUSAL>
+__global__ void __launch_bounds__(kNumThreads, 1)
+attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
+                const __grid_constant__ CUtensorMap tm_dk, const __grid_constant__ CUtensorMap tm_dv,
+                const __grid_constant__ BwdParams prm) {
+  using C = Cfg<D>;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  // The 128-byte swizzled tiles need 1 KiB-aligned shared memory; there is no
+  // room for alignment slack, so a misaligned window is reported, not used.
+  if ((smem_u32(smem_raw) & 1023u) != 0) {
+    if (threadIdx.x == 0) atomicOr(&g_status_bwd, kStatusSmemAlign);
+    return;
+  }
+  Smem<D> sm;
+  sm.base = smem_raw;
+  sm.sbase = smem_u32(smem_raw);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  Work w;
+  w.bh_kv = blockIdx.x / prm.n_kblocks;
+  w.j = blockIdx.x % prm.n_kblocks;
+  const int hkv_per_b = prm.H / prm.group;
+  w.b = w.bh_kv / hkv_per_b;
+  w.hkv = w.bh_kv % hkv_per_b;
+  // causal: query tiles from the diagonal on (tile i holds a visible pair iff
+  // its last query >= the block's first key)
+  w.i_lo = CAUSAL ? (w.j * kBlockK) / kBlockQ : 0;
+  w.tiles_per_head = prm.n_qtiles - w.i_lo;
+  w.n_it = prm.group * w.tiles_per_head;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < C::kNumBars; ++i) {
+      const uint32_t b = sm.bar(i);
+      uint32_t count = 1;
+      if (b == sm.q_full(0) || b == sm.q_full(1)) count = 32;  // every producer lane
+      if (b == sm.p_ready()) count = 8;
+      if (b == sm.dq_free()) count = 4;
+      mbar_init(b, count);
+    }
+    fence_barrier_init();
+    fence_proxy_async_smem();
+  }
+  if (warp == kWarpLoad && lane == 0) {
+    tma_prefetch_desc(&tm_q);
+    tma_prefetch_desc(&tm_k);
+    tma_prefetch_desc(&tm_v);
+    tma_prefetch_desc(&tm_do);
+  }
+  if (warp == kWarpMma) {
+    tmem_alloc(smem_u32(sm.tmem_slot()), kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *sm.tmem_slot();
+
+  if (warp < kWarpDrain) {
+    bool ok = softmax_grad_role<D, CAUSAL>(sm, tmem, prm, w);
+    ok = epilogue<D>(sm, tmem, &tm_dk, &tm_dv, prm, w, ok);
+    if (!ok && lane == 0) atomicOr(&g_status_bwd, kStatusTimeout);
+  } else if (warp < kWarpLoad) {
+    const bool ok = dq_drain_role<D>(sm, tmem, prm, w);
+    if (!ok && lane == 0) atomicOr(&g_status_bwd, kStatusTimeout);
+  } else if (warp == kWarpLoad) {
+    producer_role<D>(sm, &tm_q, &tm_k, &tm_v, &tm_do, prm, w, lane);
+  } else if (warp == kWarpMma) {
+    if (lane == 0) mma_role<D>(sm, tmem, w, prm.timeout_ns);
+    __syncwarp();
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == kWarpMma) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+// D_i = <dO_i, O_i> in fp32, one warp per row.
+template <int D>
+__global__ void row_dot_kernel(const __nv_bfloat16* __restrict__ o, const __nv_bfloat16* __restrict__ dout,
+                               float* __restrict__ dsum, size_t rows) {
+  const int lane = threadIdx.x & 31;
+  const size_t warps = static_cast<size_t>(gridDim.x) * (blockDim.x >> 5);
+  for (size_t row = blockIdx.x * static_cast<size_t>(blockDim.x >> 5) + (threadIdx.x >> 5); row < rows;
+       row += warps) {
+    float acc = 0.0f;
+#pragma unroll
+    for (int c = lane * 2; c < D; c += 64) {
+      const __nv_bfloat162 a = *reinterpret_cast<const __nv_bfloat162*>(o + row * D + c);
+      const __nv_bfloat162 g = *reinterpret_cast<const __nv_bfloat162*>(dout + row * D + c);
+      acc = fmaf(__low2float(a), __low2float(g), acc);
+      acc = fmaf(__high2float(a), __high2float(g), acc);
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+    if (lane == 0) dsum[row] = acc;
+  }
+}
+
+// dQ = BF16(scale * accumulator), 4 elements per thread per step.
+__global__ void dq_finish_kernel(const float4* __restrict__ acc, uint2* __restrict__ dq, float scale,
+                                 size_t n4) {
+  for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < n4;
+       i += static_cast<size_t>(gridDim.x) * blockDim.x) {
+    const float4 a = acc[i];
+    dq[i] = make_uint2(pack_bf16x2(a.x * scale, a.y * scale), pack_bf16x2(a.z * scale, a.w * scale));
+  }
+}
+
+template <int D, bool CAUSAL>
+int launch_main(const CUtensorMap* maps, const BwdParams& prm, int grid, cudaStream_t stream) {
+  auto kern = attn_bwd_kernel<D, CAUSAL>;
+  static std::once_flag once[kMaxDeviceCount];
+  static cudaError_t err[kMaxDeviceCount];
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  std::call_once(once[dev], [&] {
+    err[dev] = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg<D>::kSmemBytes);
+  });
+  if (err[dev] != cudaSuccess) return cuda_fail(err[dev], "cudaFuncSetAttribute");
+  kern<<<grid, kNumThreads, Cfg<D>::kSmemBytes, stream>>>(maps[0], maps[1], maps[2], maps[3], maps[4],
+                                                          maps[5], prm);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "attn_bwd_kernel launch");
+  return ATTN_OK;
+}
+
+size_t align256(size_t x) { return (x + 255) / 256 * 256; }
+
+size_t workspace_bytes(long long BH, long long Nq, int d) {
+  return align256(static_cast<size_t>(BH) * Nq * 4) + static_cast<size_t>(BH) * Nq * d * 4;
+}
+
+int bwd_impl(const void* q, const void* k, const void* v, const void* o, const void* dout,
+             const float* lse, void* dq, void* dk, void* dv, void* workspace, size_t ws_bytes, int B,
+             int H, int Hkv, int Nq, int Nk, int d, float scale, int causal, cudaStream_t stream) {
+  if (B < 0 || H < 0 || Hkv < 0 || Nq < 0 || Nk < 0) return ATTN_ERR_INVALID_ARG;
+  if (H > 0 && (Hkv == 0 || H % Hkv != 0)) return ATTN_ERR_INVALID_ARG;
+  if (!std::isfinite(scale)) return ATTN_ERR_INVALID_ARG;
+  if (causal != 0 && causal != 1) return ATTN_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
+  if (causal && Nq != Nk) return ATTN_ERR_UNSUPPORTED;
+  const long long BH = static_cast<long long>(B) * H, BHkv = static_cast<long long>(B) * Hkv;
+  if (BH > 0x7fffffffLL) return ATTN_ERR_INVALID_ARG;
+  const size_t q_bytes = static_cast<size_t>(BH) * Nq * d * 2;
+  const size_t kv_bytes = static_cast<size_t>(BHkv) * Nk * d * 2;
+  if (BH == 0 || (Nq == 0 && Nk == 0)) return ATTN_OK;
+  const bool any_q = Nq > 0, any_k = Nk > 0;
+  if ((any_q && (!q || !o || !dout || !lse || !dq)) || (any_k && (!k || !v || !dk || !dv)))
+    return ATTN_ERR_INVALID_ARG;
+  const size_t need = workspace_bytes(BH, Nq, d);
+  if (any_q && any_k && (!workspace || ws_bytes < need)) return ATTN_ERR_INVALID_ARG;
+  if (misaligned(q, 16) || misaligned(k, 16) || misaligned(v, 16) || misaligned(o, 16) ||
+      misaligned(dout, 16) || misaligned(dq, 16) || misaligned(dk, 16) || misaligned(dv, 16) ||
+      misaligned(lse, 4) || misaligned(workspace, 256))
+    return ATTN_ERR_INVALID_ARG;
+  // outputs may not overlap each other, any input, or the workspace
+  const size_t lse_bytes = static_cast<size_t>(BH) * Nq * 4;
+  const void* ins[6] = {q, k, v, o, dout, lse};
+  const size_t in_bytes[6] = {q_bytes, kv_bytes, kv_bytes, q_bytes, q_bytes, lse_bytes};
+  void* outs[4] = {dq, dk, dv, workspace};
+  const size_t out_bytes[4] = {q_bytes, kv_bytes, kv_bytes, any_q && any_k ? need : 0};
+  for (int a = 0; a < 4; ++a) {
+    for (int b = 0; b < 6; ++b)
+      if (ranges_overlap(outs[a], out_bytes[a], ins[b], in_bytes[b])) return ATTN_ERR_INVALID_ARG;
+    for (int b = a + 1; b < 4; ++b)
+      if (ranges_overlap(outs[a], out_bytes[a], outs[b], out_bytes[b])) return ATTN_ERR_INVALID_ARG;
+  }
+  const long long n_kblocks = (Nk + kBlockK - 1) / kBlockK;
+  if (n_kblocks * BHkv > 0x7fffffffLL) return ATTN_ERR_INVALID_ARG;
+  int rc = check_device();
+  if (rc != ATTN_OK) return rc;
+
+  cudaError_t e;
+  // no keys: every gradient is 0 (O = 0 does not depend on the inputs);
+  // no queries: dK = dV = 0
+  if (!any_k || !any_q) {
+    if (any_q && (e = cudaMemsetAsync(dq, 0, q_bytes, stream)) != cudaSuccess)
+      return cuda_fail(e, "cudaMemsetAsync");
+    if (any_k && (e = cudaMemsetAsync(dk, 0, kv_bytes, stream)) != cudaSuccess)
+      return cuda_fail(e, "cudaMemsetAsync");
+    if (any_k && (e = cudaMemsetAsync(dv, 0, kv_bytes, stream)) != cudaSuccess)
+      return cuda_fail(e, "cudaMemsetAsync");
+    return ATTN_OK;
+  }
+
+  CUtensorMap maps[6];
+  const int bh = static_cast<int>(BH), bhkv = static_cast<int>(BHkv);
+  if (!make_tmap_bf16_3d(&maps[0], q, bh, Nq, d, kBlockQ, &t_last_error) ||
+      !make_tmap_bf16_3d(&maps[1], k, bhkv, Nk, d, kBlockK, &t_last_error) ||
+      !make_tmap_bf16_3d(&maps[2], v, bhkv, Nk, d, kBlockK, &t_last_error) ||
+      !make_tmap_bf16_3d(&maps[3], dout, bh, Nq, d, kBlockQ, &t_last_error) ||
+      !make_tmap_bf16_3d(&maps[4], dk, bhkv, Nk, d, 32, &t_last_error) ||
+      !make_tmap_bf16_3d(&maps[5], dv, bhkv, Nk, d, 32, &t_last_error))
+    return ATTN_ERR_CUDA;
+
+  float* dsum = static_cast<float*>(workspace);
+  float* dq_acc = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) +
+                                           align256(static_cast<size_t>(BH) * Nq * 4));
+  const size_t rows = static_cast<size_t>(BH) * Nq;
+  e = cudaMemsetAsync(dq_acc, 0, rows * d * 4, stream);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync");
+  {
+    const unsigned blocks = static_cast<unsigned>(std::min<size_t>((rows + 7) / 8, 148 * 16));
+    if (d == 128)
+      row_dot_kernel<128><<<blocks, 256, 0, stream>>>(static_cast<const __nv_bfloat16*>(o),
+                                                      static_cast<const __nv_bfloat16*>(dout), dsum, rows);
+    else
+      row_dot_kernel<64><<<blocks, 256, 0, stream>>>(static_cast<const __nv_bfloat16*>(o),
+                                                     static_cast<const __nv_bfloat16*>(dout), dsum, rows);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "row_dot_kernel launch");
+  }
+
+  BwdParams prm = {};
+  prm.lse = lse;
+  prm.dsum = dsum;
+  prm.dq_acc = dq_acc;
+  prm.timeout_ns = kWaitTimeoutNs;
+  prm.Nq = Nq;
+  prm.Nk = Nk;
+  prm.H = H;
+  prm.group = H / Hkv;
+  prm.n_kblocks = static_cast<int>(n_kblocks);
+  prm.n_qtiles = (Nq + kBlockQ - 1) / kBlockQ;
+  prm.causal = causal;
+  prm.scale_log2 = scale * kLog2e;
+  prm.scale = scale;
+  const int grid = static_cast<int>(n_kblocks * BHkv);
+  if (d == 128)
+    rc = causal ? launch_main<128, true>(maps, prm, grid, stream) : launch_main<128, false>(maps, prm, grid, stream);
+  else
+    rc = causal ? launch_main<64, true>(maps, prm, grid, stream) : launch_main<64, false>(maps, prm, grid, stream);
+  if (rc != ATTN_OK) return rc;
+
+  const size_t n4 = rows * d / 4;
+  const unsigned blocks = static_cast<unsigned>(std::min<size_t>((n4 + 255) / 256, 148 * 32));
+  dq_finish_kernel<<<blocks, 256, 0, stream>>>(reinterpret_cast<const float4*>(dq_acc),
+                                               static_cast<uint2*>(dq), scale, n4);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "dq_finish_kernel launch");
+  return ATTN_OK;
+}
+
+}  // namespace bwd
+
+int bwd_status_take(cudaStream_t stream, unsigned int* status) {
+  unsigned int st = 0;
+  cudaError_t e = cudaMemcpyFromSymbolAsync(&st, bwd::g_status_bwd, sizeof(st), 0,
+                                            cudaMemcpyDeviceToHost, stream);
+  if (e != cudaSuccess) return cuda_fail(e, "read backward status word");
+  const unsigned int zero = 0;
+  e = cudaMemcpyToSymbolAsync(bwd::g_status_bwd, &zero, sizeof(zero), 0, cudaMemcpyHostToDevice, stream);
+  if (e != cudaSuccess) return cuda_fail(e, "clear backward status word");
+  e = cudaStreamSynchronize(stream);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+  // a misaligned shared-memory window is a launch problem, reported as CUDA
+  if (st & bwd::kStatusSmemAlign) {
+    t_last_error = "attn_bwd_kernel: dynamic shared memory not 1 KiB aligned";
+    st = (st & ~bwd::kStatusSmemAlign) | kStatusWordLaunch;
+  }
+  *status = st;
+  return ATTN_OK;
+}
+
+}  // namespace eab
+
+extern "C" {
+
+size_t attn_bwd_workspace_size(int B, int H, int Nq, int d) {
+  if (B < 0 || H < 0 || Nq < 0 || (d != 64 && d != 128)) return 0;
+  return eab::bwd::workspace_bytes(static_cast<long long>(B) * H, Nq, d);
+}
+
+int attn_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout,
+             const float* lse, void* dq, void* dk, void* dv, void* workspace,
+             size_t workspace_bytes, int B, int H, int Hkv, int Nq, int Nk, int d, float scale,
+             int causal, cudaStream_t stream) {
+  return eab::bwd::bwd_impl(q, k, v, o, dout, lse, dq, dk, dv, workspace, workspace_bytes, B, H, Hkv,
+                            Nq, Nk, d, scale, causal, stream);
+}
+
+}  // extern "C"

@@ -6,7 +6,7 @@
 // Method (what the pages describe; they print no formulas or code):
 //  * Tiling through on-chip memory so the Nq x Nk score matrix never reaches
 //    device memory, with a running per-row max and sum (online softmax):
-//    Flash Attention glossary (jisaku.com), sections "タイリングによるSRAMの活用"
+//    "Flash Attention（Flash Attention）" (jisaku.com glossary), sections "タイリングによるSRAMの活用"
 //    and "オンライン・ソフトマックスと再計算"; FlashAttention 4 page
 //    (ja.linux-konsole.com), section "なぜアテンションカーネルがまだLLMのコストを
 //    支配しているのか".
@@ -15,11 +15,11 @@
 //    "FlashAttention 4の新機能".
 //  * exp2 partly evaluated as a cubic polynomial on the FMA pipe to relieve the
 //    few SFUs: same page, section "CUDAコアによるソフトウェアの指数演算";
-//    FlashAttention-4 deep dive (sns.style), section 二.
+//    "FlashAttention-4：非対称ハードウェアスケーリング…" (sns.style), section 二.
 //  * Rescaling only when the new max is sufficiently larger than the old one:
 //    FlashAttention 4 page, section "よりスマートなオンラインソフトマックス再スケーリング".
-//  * Fully asynchronous MMA with Tensor Memory: FlashAttention-4 deep dive,
-//    section 二.
+//  * Fully asynchronous MMA with Tensor Memory: "FlashAttention-4：非対称ハードウェア
+//    スケーリング…" (sns.style), section 二.
 //
 // Design (this library's, for sm_100a):
 //  * One CTA owns two 128-row query tiles of one (b, h) -- 256 rows -- and
@@ -64,6 +64,7 @@
 #include "attn.h"
 #include "exp2.cuh"
 #include "sm100.cuh"
+#include "host_common.h"
 #include "tmap.h"
 
 namespace eab {
@@ -88,7 +89,11 @@ constexpr int kDefaultPoly16 = 4;                   // exp2 columns (of 16) on t
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kLog2e = 1.4426950408889634f;
 
-enum : unsigned int { kStatusTimeout = 1u };
+constexpr unsigned int kStatusTimeout = kStatusWordTimeout;
+constexpr unsigned int kStatusBadSeqlens = kStatusWordBadSeqlens;
+// "no bound" for a side of the key band; large enough for any sequence, small
+// enough that row +- bound stays inside int.
+constexpr int kUnbounded = 1 << 30;
 
 // Per-device status word (each device holds its own copy of module globals).
 __device__ unsigned int g_status;
@@ -109,20 +114,47 @@ struct Cfg {
   // float [tile 2][half 2][parity 2][row 128]
   static constexpr int kOffXch = (kOffMisc + 16 + 15) / 16 * 16;
   static constexpr int kXchBytes = 2 * 2 * 2 * kBlockM * 4;
-  static constexpr int kSmemBytes = kOffXch + kXchBytes + 1024;  // + slack for 1 KiB alignment
+  static constexpr int kOffSeq = kOffXch + kXchBytes;  // this CTA's SeqView
+  static constexpr int kSeqBytes = 64;
+  static constexpr int kSmemBytes = kOffSeq + kSeqBytes + 1024;  // + slack for 1 KiB alignment
   static constexpr uint32_t kTmemO = 256;
 };
 
 struct FwdParams {
   float* lse;
   unsigned long long* rescale_count;
+  __nv_bfloat16* o;  // output base (packed layout: ragged row blocks are stored directly)
+  const int* cu_q;   // packed variable-length batch: sequence starts (num_seqs + 1), else null
+  const int* cu_k;
   uint64_t timeout_ns;
-  int Nq, Nk, BH, n_qblocks;
+  int Nq, Nk;        // dense: sequence lengths; packed: total_q, total_k
+  int BH, n_qblocks; // grid = BH * n_qblocks (packed: BH = num_seqs * H)
   int H, group;      // query heads per batch; query heads per key/value head
-  int hgroup;        // causal order: heads scheduled together (their K/V fit in L2)
+  int wl, wr;        // key band: i - wl <= j <= i + wr (kUnbounded: no bound)
+  int grouped;       // causal band: heads in L2-sized groups, heaviest blocks first
+  int hgroup;        // heads scheduled together (their K/V fit in L2)
   float scale_log2;  // scale * log2(e)
   float tau;         // rescale threshold, powers of two
 };
+
+// Where one CTA's sequence lives: lengths, first packed row (packed layout),
+// tensor-map head coordinates and the KV tile range it visits.
+struct SeqView {
+  int Nq, Nk;        // this sequence's lengths
+  int q0, k0;        // first row of the sequence in the packed layout (0 dense)
+  int head_q, head_kv;  // tensor-map head coordinate of Q/O and of K/V
+  int j_lo, n_kv;    // KV tiles j_lo .. j_lo + n_kv - 1
+  bool packed;
+  float* lse_row0;   // LSE of this sequence's row 0 (null: not computed)
+};
+
+// Tensor-map coordinates (column, row, head) -> the map's dimension order:
+// dense maps are [BH, N, d], packed maps [total, H, d].
+__device__ __forceinline__ void tma_load_rows(uint32_t dst, const CUtensorMap* tm, int col, int row,
+                                              int head, bool packed, uint32_t bar) {
+  if (packed) tma_load_3d(dst, tm, col, head, row, bar);
+  else tma_load_3d(dst, tm, col, row, head, bar);
+}
 
 template <int POLY16>
 __device__ __forceinline__ float ex2_split(float x, int col) {
@@ -157,6 +189,11 @@ struct Smem {
   __device__ __forceinline__ uint32_t* tmem_slot() const {
     return reinterpret_cast<uint32_t*>(base + Cfg<D>::kOffMisc);
   }
+  // kept in shared memory rather than registers: the softmax warps need most of
+  // it only in the epilogue
+  __device__ __forceinline__ SeqView* seq() const {
+    return reinterpret_cast<SeqView*>(base + Cfg<D>::kOffSeq);
+  }
 };
 
 // Warp-uniform bounded wait: every lane waits, and the warp agrees on the
@@ -172,16 +209,15 @@ __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, uint64_
 template <int D>
 __device__ __forceinline__ void producer_role(const Smem<D>& sm, const CUtensorMap* tm_q,
                                               const CUtensorMap* tm_k, const CUtensorMap* tm_v,
-                                              int bh, int bh_kv, int qb, int n_kv,
-                                              uint64_t timeout) {
+                                              const SeqView& sv, int qb, uint64_t timeout) {
   using C = Cfg<D>;
   uint32_t it = 0;
   auto load_q = [&](int t) {
     mbar_arrive_expect_tx(sm.q_full(t), C::kTileBytes);
 #pragma unroll
     for (int b = 0; b < C::kBoxes; ++b)
-      tma_load_3d(sm.q(t) + b * C::kBoxBytes, tm_q, b * 64, qb * kRowsPerCta + t * kBlockM, bh,
-                  sm.q_full(t));
+      tma_load_rows(sm.q(t) + b * C::kBoxBytes, tm_q, b * 64, sv.q0 + qb * kRowsPerCta + t * kBlockM,
+                    sv.head_q, sv.packed, sm.q_full(t));
   };
   auto load_kv = [&](const CUtensorMap* tm, int j) -> bool {
     const uint32_t slot = it % C::kStages;
@@ -190,16 +226,17 @@ __device__ __forceinline__ void producer_role(const Smem<D>& sm, const CUtensorM
     mbar_arrive_expect_tx(sm.kv_full(slot), C::kTileBytes);
 #pragma unroll
     for (int b = 0; b < C::kBoxes; ++b)
-      tma_load_3d(sm.kv(slot) + b * C::kBoxBytes, tm, b * 64, j * kBlockN, bh_kv, sm.kv_full(slot));
+      tma_load_rows(sm.kv(slot) + b * C::kBoxBytes, tm, b * 64, sv.k0 + j * kBlockN, sv.head_kv,
+                    sv.packed, sm.kv_full(slot));
     ++it;
     return true;
   };
 
   load_q(0);
-  bool ok = load_kv(tm_k, 0);
+  bool ok = load_kv(tm_k, sv.j_lo);
   load_q(1);
-  ok = ok && load_kv(tm_v, 0);
-  for (int j = 1; ok && j < n_kv; ++j) ok = load_kv(tm_k, j) && load_kv(tm_v, j);
+  ok = ok && load_kv(tm_v, sv.j_lo);
+  for (int j = sv.j_lo + 1; ok && j < sv.j_lo + sv.n_kv; ++j) ok = load_kv(tm_k, j) && load_kv(tm_v, j);
 
   // Never leave the CTA with a copy in flight: wait for the latest fill of
   // every slot and for both Q tiles (immediate on the normal path).
@@ -347,10 +384,10 @@ __device__ __forceinline__ void pair_sync(int t, int q) {
   asm volatile("bar.sync %0, 64;" ::"r"(1 + t * 4 + q) : "memory");
 }
 
-template <int D, bool CAUSAL, int POLY16>
+template <int D, bool MASK, int POLY16>
 __device__ __forceinline__ void softmax_role(const Smem<D>& sm, uint32_t tmem,
                                              const CUtensorMap* tm_o, const FwdParams& prm,
-                                             int bh, int qb, int n_kv) {
+                                             const SeqView& sv, int qb) {
   using C = Cfg<D>;
   constexpr int kCols = kBlockN / 2;  // key columns per warp
   constexpr int kOCols = D / 2;       // output columns per warp
@@ -361,6 +398,8 @@ __device__ __forceinline__ void softmax_role(const Smem<D>& sm, uint32_t tmem,
   const int r = q4 * 32 + lane;
   const int tile_row0 = qb * kRowsPerCta + t * kBlockM;
   const int row = tile_row0 + r;
+  const int rw0 = tile_row0 + q4 * 32;  // first row of this warp
+  const int Nk = sv.Nk;
   const uint32_t lane_off = static_cast<uint32_t>(q4 * 32) << 16;
   const uint32_t tS = tmem + lane_off + t * kBlockM + h * kCols;
   const uint32_t tO = tmem + lane_off + C::kTmemO + t * D + h * kOCols;
@@ -374,12 +413,12 @@ __device__ __forceinline__ void softmax_role(const Smem<D>& sm, uint32_t tmem,
   float l_run = 0.0f;       // this half's running sum of 2^(score - m_run)
   bool ok = true;
 
-  for (int j = 0; j < n_kv; ++j) {
+  for (int j = 0; j < sv.n_kv; ++j) {
     ok = warp_wait(sm.s_full(t), j & 1, timeout);
-    const int kv0 = j * kBlockN + h * kCols;
-    // mask needed: key tail, or the causal diagonal (only tiles that reach past
-    // the tile's first row)
-    const bool masked = kv0 + kCols > prm.Nk || (CAUSAL && kv0 + kCols - 1 > tile_row0);
+    const int kv0 = (sv.j_lo + j) * kBlockN + h * kCols;
+    // mask needed: key tail, or a band edge crossing this warp's 64 x 32 block
+    const bool masked = kv0 + kCols > Nk ||
+                        (MASK && (kv0 + kCols - 1 - rw0 > prm.wr || rw0 + 31 - kv0 > prm.wl));
     // load 32 score columns [32*k, 32*k + 32) of this warp's half as fp32,
     // prescaled and masked
     auto load_scores = [&](int k, float (&x)[32]) {
@@ -397,7 +436,7 @@ __device__ __forceinline__ void softmax_role(const Smem<D>& sm, uint32_t tmem,
 #pragma unroll
         for (int c = 0; c < 32; ++c) {
           const int key = kv0 + 32 * k + c;
-          if (key >= prm.Nk || (CAUSAL && key > row)) x[c] = -INFINITY;
+          if (key >= Nk || (MASK && (key - row > prm.wr || row - key > prm.wl))) x[c] = -INFINITY;
         }
       }
     };
@@ -505,6 +544,7 @@ __device__ __forceinline__ void softmax_role(const Smem<D>& sm, uint32_t tmem,
   const bool ok3 = ok2 && !isnan(lother);
   uint8_t* sOt = sm.base + C::kOffQ + t * C::kTileBytes;
   const float l_tot = l_run + lother;
+  const bool ragged = sv.packed && rw0 + 32 > sv.Nq;
   if (ok3) {
     tc_fence_after();
     // O / l -> BF16 -> this tile's Q buffer (its last reader, the final S MMA,
@@ -522,12 +562,23 @@ __device__ __forceinline__ void softmax_role(const Smem<D>& sm, uint32_t tmem,
       for (int i = 0; i < 16; ++i)
         w[i] = pack_bf16x2(__uint_as_float(o[2 * i]) * inv_l, __uint_as_float(o[2 * i + 1]) * inv_l);
       const int col0 = h * kOCols + cc * 32;  // first output column of this chunk
-      uint8_t* rowp = sOt + (col0 >> 6) * C::kBoxBytes + r * 128;
+      if (ragged) {
+        // the warp's 32 rows cross the end of a packed sequence: a TMA store
+        // would write into the next sequence, so each row stores itself
+        if (row < sv.Nq) {
+          uint4* dst = reinterpret_cast<uint4*>(
+              prm.o + (static_cast<size_t>(sv.q0 + row) * prm.H + sv.head_q) * D + col0);
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const int chunk = (((col0 & 63) >> 3) + i) ^ (r & 7);
-        *reinterpret_cast<uint4*>(rowp + chunk * 16) =
-            make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
+          for (int i = 0; i < 4; ++i) dst[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
+        }
+      } else {
+        uint8_t* rowp = sOt + (col0 >> 6) * C::kBoxBytes + r * 128;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int chunk = (((col0 & 63) >> 3) + i) ^ (r & 7);
+          *reinterpret_cast<uint4*>(rowp + chunk * 16) =
+              make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
+        }
       }
     }
     fence_proxy_async_smem();
@@ -536,16 +587,17 @@ __device__ __forceinline__ void softmax_role(const Smem<D>& sm, uint32_t tmem,
   // one box, stored by the h = 0 warp after both halves are written.
   if (D == 64) pair_sync(t, q4);
   __syncwarp();
-  if (ok3 && lane == 0 && tile_row0 + q4 * 32 < prm.Nq && (D == 128 || h == 0)) {
+  if (ok3 && !ragged && lane == 0 && rw0 < sv.Nq && (D == 128 || h == 0)) {
     const int box = D == 128 ? h : 0;
-    tma_store_3d(tm_o, smem_u32(sOt + box * C::kBoxBytes + q4 * 32 * 128), box * 64,
-                 tile_row0 + q4 * 32, bh);
+    const uint32_t src = smem_u32(sOt + box * C::kBoxBytes + q4 * 32 * 128);
+    if (sv.packed) tma_store_3d(tm_o, src, box * 64, sv.head_q, sv.q0 + rw0);
+    else tma_store_3d(tm_o, src, box * 64, rw0, sv.head_q);
     bulk_commit_group();
     bulk_wait_group_read0();
   }
-  if (ok3 && h == 0 && prm.lse != nullptr && row < prm.Nq) {
+  if (ok3 && h == 0 && sv.lse_row0 != nullptr && row < sv.Nq) {
     const float m_use = (m_run == -INFINITY) ? 0.0f : m_run;
-    prm.lse[static_cast<size_t>(bh) * prm.Nq + row] = (m_use + log2f(l_tot)) * kLn2;
+    sv.lse_row0[row] = (m_use + log2f(l_tot)) * kLn2;
   }
   if (!ok3 && lane == 0) atomicOr(&g_status, kStatusTimeout);
 }
@@ -553,7 +605,7 @@ __device__ __forceinline__ void softmax_role(const Smem<D>& sm, uint32_t tmem,
 // ---------------------------------------------------------------------------
 // The kernel.  Grid: one CTA per (b*h, 256-row query block).
 // ---------------------------------------------------------------------------
-template <int D, bool CAUSAL, int POLY16>
+template <int D, bool MASK, int POLY16>
 __global__ void __launch_bounds__(kNumThreads, 1)
 attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                 const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
@@ -569,14 +621,14 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   }
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-  // Tile order.  Non-causal: head-major, so the CTAs resident at one time share
-  // a few heads' K/V in L2.  Causal: heads in groups of hgroup (sized on the
+  // Tile order.  Default: head-major, so the CTAs resident at one time share a
+  // few heads' K/V in L2.  Causal band: heads in groups of hgroup (sized on the
   // host so a group's K/V fits in L2), and within a group the heaviest query
   // blocks first, so short blocks fill the tail of each group while the next
   // group starts.
   const int tile = blockIdx.x;
   int bh, qb;
-  if (CAUSAL) {
+  if (prm.grouped) {
     const int per_group = prm.hgroup * prm.n_qblocks;
     const int g = tile / per_group, w = tile % per_group;
     const int gsize = min(prm.hgroup, prm.BH - g * prm.hgroup);
@@ -586,11 +638,66 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     bh = tile / prm.n_qblocks;
     qb = tile % prm.n_qblocks;
   }
-  // grouped-query attention: query head h of batch b reads key/value head
-  // h / group of the same batch (group = 1: one key/value head per query head)
-  const int bh_kv = (bh / prm.H) * (prm.H / prm.group) + (bh % prm.H) / prm.group;
-  int n_kv = (prm.Nk + kBlockN - 1) / kBlockN;
-  if (CAUSAL) n_kv = min(n_kv, (qb + 1) * (kRowsPerCta / kBlockN));
+  // grouped-query attention: query head h reads key/value head h / group of the
+  // same batch entry (group = 1: one key/value head per query head)
+  const int hq = bh % prm.H, seq = bh / prm.H;
+  SeqView sv;
+  static_assert(sizeof(SeqView) <= Cfg<D>::kSeqBytes, "SeqView slot");
+  sv.packed = prm.cu_q != nullptr;
+  if (sv.packed) {
+    // packed variable-length batch: sequence `seq` owns rows cu_q[seq] ..
+    // cu_q[seq+1]-1 of the [total, H, d] tensors.  Offsets that do not describe
+    // sequences inside the tensors, or a sequence longer than the grid covers,
+    // are reported and the CTA does nothing (every access stays in bounds).
+    const int a = __ldg(prm.cu_q + seq), b = __ldg(prm.cu_q + seq + 1);
+    const int c = __ldg(prm.cu_k + seq), e = __ldg(prm.cu_k + seq + 1);
+    if (a < 0 || b < a || b > prm.Nq || c < 0 || e < c || e > prm.Nk ||
+        b - a > prm.n_qblocks * kRowsPerCta) {
+      if (threadIdx.x == 0 && qb == 0) atomicOr(&g_status, kStatusBadSeqlens);
+      return;
+    }
+    sv.Nq = b - a;
+    sv.Nk = e - c;
+    sv.q0 = a;
+    sv.k0 = c;
+    sv.head_q = hq;
+    sv.head_kv = hq / prm.group;
+    sv.lse_row0 = prm.lse ? prm.lse + static_cast<size_t>(hq) * prm.Nq + a : nullptr;
+    if (qb * kRowsPerCta >= sv.Nq) return;  // this sequence is shorter than the grid
+  } else {
+    sv.Nq = prm.Nq;
+    sv.Nk = prm.Nk;
+    sv.q0 = 0;
+    sv.k0 = 0;
+    sv.head_q = bh;
+    sv.head_kv = seq * (prm.H / prm.group) + hq / prm.group;
+    sv.lse_row0 = prm.lse ? prm.lse + static_cast<size_t>(bh) * prm.Nq : nullptr;
+  }
+  {
+    // KV tiles that hold a visible key for some row of this block; a block with
+    // none (an empty band, an empty key set) still runs one fully masked tile,
+    // which yields O = 0 and LSE = -inf.
+    const int n_all = max((sv.Nk + kBlockN - 1) / kBlockN, 1);
+    int j_lo = 0, j_hi = n_all;
+    if (MASK) {
+      // rows and bounds are below 2^31 and 2^30: the sums stay inside 64 bits
+      const long long r_lo = static_cast<long long>(qb) * kRowsPerCta;
+      const long long r_end = r_lo + kRowsPerCta < sv.Nq ? r_lo + kRowsPerCta : sv.Nq;
+      const long long r_hi = r_end - 1;
+      if (prm.wr < kUnbounded) {
+        const long long last = (r_hi + prm.wr) / kBlockN + 1;
+        if (last < j_hi) j_hi = static_cast<int>(last);
+      }
+      if (prm.wl < kUnbounded && r_lo - prm.wl > 0) j_lo = static_cast<int>((r_lo - prm.wl) / kBlockN);
+      if (j_lo >= j_hi) {
+        j_lo = min(j_lo, n_all - 1);
+        j_hi = j_lo + 1;
+      }
+    }
+    sv.j_lo = j_lo;
+    sv.n_kv = j_hi - j_lo;
+  }
+  if (threadIdx.x == 0) *sm.seq() = sv;
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < C::kNumBars; ++i) {
@@ -617,20 +724,21 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *sm.tmem_slot();
+  const SeqView& seqv = *sm.seq();
 
   if (warp >= kWarpLoad) {
     // warpgroup 2: TMA producer (warp 8), MMA issuer (warp 9), two idle warps
     setmaxnreg_dec<kProducerRegs>();
     if (warp == kWarpLoad) {
-      if (lane == 0) producer_role<D>(sm, &tm_q, &tm_k, &tm_v, bh, bh_kv, qb, n_kv, prm.timeout_ns);
+      if (lane == 0) producer_role<D>(sm, &tm_q, &tm_k, &tm_v, seqv, qb, prm.timeout_ns);
       __syncwarp();
     } else if (warp == kWarpMma) {
-      if (lane == 0) mma_role<D>(sm, tmem, n_kv, prm.timeout_ns);
+      if (lane == 0) mma_role<D>(sm, tmem, seqv.n_kv, prm.timeout_ns);
       __syncwarp();
     }
   } else {
     setmaxnreg_inc<kSoftmaxRegs>();
-    softmax_role<D, CAUSAL, POLY16>(sm, tmem, &tm_o, prm, bh, qb, n_kv);
+    softmax_role<D, MASK, POLY16>(sm, tmem, &tm_o, prm, seqv, qb);
   }
 
   tc_fence_before();
@@ -662,25 +770,12 @@ __global__ void selftest_timeout_kernel(uint64_t timeout_ns) {
 // ---------------------------------------------------------------------------
 // Host side
 // ---------------------------------------------------------------------------
-thread_local std::string t_last_error;
+constexpr int kMaxDevices = kMaxDeviceCount;
 
-int cuda_fail(cudaError_t e, const char* what) {
-  t_last_error = std::string(what) + ": " + cudaGetErrorString(e);
-  return ATTN_ERR_CUDA;
-}
-
-constexpr int kMaxDevices = 64;
-struct DeviceInfo {
-  bool probed = false;
-  bool supported = false;
-};
-std::mutex g_dev_mu;
-DeviceInfo g_dev[kMaxDevices];
-
-template <int D, bool CAUSAL, int POLY16>
+template <int D, bool MASK, int POLY16>
 int launch_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                const CUtensorMap& to, const FwdParams& prm, cudaStream_t stream) {
-  auto kern = attn_fwd_kernel<D, CAUSAL, POLY16>;
+  auto kern = attn_fwd_kernel<D, MASK, POLY16>;
   static std::once_flag attr_once[kMaxDevices];
   static cudaError_t attr_err[kMaxDevices];
   int dev = 0;
@@ -698,57 +793,86 @@ int launch_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& 
   return ATTN_OK;
 }
 
-template <int D, bool CAUSAL>
+template <int D, bool MASK>
 int dispatch_exp(int exp_mode, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                  const CUtensorMap& to, const FwdParams& prm, cudaStream_t stream) {
   switch (exp_mode) {
-    case 0: return launch_fwd<D, CAUSAL, 0>(tq, tk, tv, to, prm, stream);
-    case 1: return launch_fwd<D, CAUSAL, kDefaultPoly16>(tq, tk, tv, to, prm, stream);
-    default: return launch_fwd<D, CAUSAL, 16>(tq, tk, tv, to, prm, stream);
+    case 0: return launch_fwd<D, MASK, 0>(tq, tk, tv, to, prm, stream);
+    case 1: return launch_fwd<D, MASK, kDefaultPoly16>(tq, tk, tv, to, prm, stream);
+    default: return launch_fwd<D, MASK, 16>(tq, tk, tv, to, prm, stream);
   }
 }
 
-bool ranges_overlap(const void* a, size_t na, const void* b, size_t nb) {
-  if (!a || !b || na == 0 || nb == 0) return false;
-  const uintptr_t a0 = reinterpret_cast<uintptr_t>(a), b0 = reinterpret_cast<uintptr_t>(b);
-  return a0 < b0 + nb && b0 < a0 + na;
+
+
+// Key band from the C-ABI's (window_left, window_right), -1 = no bound.
+bool band_from_window(int window_left, int window_right, int* wl, int* wr) {
+  if (window_left < -1 || window_right < -1) return false;
+  *wl = window_left < 0 ? kUnbounded : std::min(window_left, kUnbounded);
+  *wr = window_right < 0 ? kUnbounded : std::min(window_right, kUnbounded);
+  return true;
 }
 
-int check_device() {
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
-  if (dev < 0 || dev >= kMaxDevices) return ATTN_ERR_UNSUPPORTED;
-  std::lock_guard<std::mutex> lk(g_dev_mu);
-  DeviceInfo& di = g_dev[dev];
-  if (!di.probed) {
-    int major = 0, minor = 0;
-    e = cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
-    if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceGetAttribute");
-    e = cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
-    if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceGetAttribute");
-    di.supported = (major == 10 && minor == 0);
-    di.probed = true;
+// Heads scheduled together under the causal order: as many as keep their K/V
+// within ~48 MB of the 126 MB L2 (several query heads of a GQA group share one
+// K/V head).
+int heads_per_l2_group(double keys_per_head, int d, int group, long long BH) {
+  const double kv_head_bytes = 2.0 * keys_per_head * d * 2.0 / group;
+  const double budget = 48.0 * 1024 * 1024;
+  const long long g = static_cast<long long>(budget / std::max(kv_head_bytes, 1.0));
+  return static_cast<int>(std::max(1LL, std::min(g, BH)));
+}
+
+int launch_any(int d, int exp_mode, const CUtensorMap& tq, const CUtensorMap& tk,
+               const CUtensorMap& tv, const CUtensorMap& to, const FwdParams& prm,
+               cudaStream_t stream) {
+  const bool mask = prm.wl < kUnbounded || prm.wr < kUnbounded;
+  if (d == 128) {
+    return mask ? dispatch_exp<128, true>(exp_mode, tq, tk, tv, to, prm, stream)
+                : dispatch_exp<128, false>(exp_mode, tq, tk, tv, to, prm, stream);
   }
-  return di.supported ? ATTN_OK : ATTN_ERR_UNSUPPORTED;
+  return mask ? dispatch_exp<64, true>(exp_mode, tq, tk, tv, to, prm, stream)
+              : dispatch_exp<64, false>(exp_mode, tq, tk, tv, to, prm, stream);
+}
+
+// No key at all: O = 0, LSE = -inf.
+int fill_empty(void* o, size_t o_bytes, float* lse, size_t n_lse, cudaStream_t stream) {
+  cudaError_t e = cudaMemsetAsync(o, 0, o_bytes, stream);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync");
+  if (lse && n_lse) {
+    const unsigned blocks = static_cast<unsigned>(std::min<size_t>((n_lse + 255) / 256, 4096));
+    fill_neg_inf_kernel<<<blocks, 256, 0, stream>>>(lse, n_lse);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "fill_neg_inf_kernel launch");
+  }
+  return ATTN_OK;
+}
+
+
+// Outputs may not overlap any input or each other.
+bool outputs_overlap(const void* q, size_t q_bytes, const void* k, const void* v, size_t kv_bytes,
+                     const void* o, size_t o_bytes, const void* lse, size_t lse_bytes) {
+  return ranges_overlap(o, o_bytes, q, q_bytes) || ranges_overlap(o, o_bytes, k, kv_bytes) ||
+         ranges_overlap(o, o_bytes, v, kv_bytes) || ranges_overlap(lse, lse_bytes, q, q_bytes) ||
+         ranges_overlap(lse, lse_bytes, k, kv_bytes) || ranges_overlap(lse, lse_bytes, v, kv_bytes) ||
+         ranges_overlap(lse, lse_bytes, o, o_bytes);
 }
 
 int fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
-             int Hkv, int Nq, int Nk, int d, float scale, int causal, float tau, int exp_mode,
-             unsigned long long* rescale_count, cudaStream_t stream) {
+             int Hkv, int Nq, int Nk, int d, float scale, int window_left, int window_right,
+             float tau, int exp_mode, unsigned long long* rescale_count, cudaStream_t stream) {
+  int wl = 0, wr = 0;
   if (B < 0 || H < 0 || Hkv < 0 || Nq < 0 || Nk < 0) return ATTN_ERR_INVALID_ARG;
   if (H > 0 && (Hkv == 0 || H % Hkv != 0)) return ATTN_ERR_INVALID_ARG;
   if (!std::isfinite(scale)) return ATTN_ERR_INVALID_ARG;
-  if (causal != 0 && causal != 1) return ATTN_ERR_INVALID_ARG;
+  if (!band_from_window(window_left, window_right, &wl, &wr)) return ATTN_ERR_INVALID_ARG;
   if (!(tau >= 0.0f && tau <= 64.0f)) return ATTN_ERR_UNSUPPORTED;
   if (exp_mode < 0 || exp_mode > 2) return ATTN_ERR_UNSUPPORTED;
   if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
-  if (causal && Nq != Nk) return ATTN_ERR_UNSUPPORTED;
   const long long BH = static_cast<long long>(B) * H;
   if (BH == 0 || Nq == 0) return ATTN_OK;  // nothing to compute
   if (BH > 0x7fffffffLL) return ATTN_ERR_INVALID_ARG;
   if (!o || (Nk > 0 && (!q || !k || !v))) return ATTN_ERR_INVALID_ARG;
-  auto misaligned = [](const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) != 0; };
   if (misaligned(q, 16) || misaligned(k, 16) || misaligned(v, 16) || misaligned(o, 16) ||
       misaligned(lse, 4) || misaligned(rescale_count, 8))
     return ATTN_ERR_INVALID_ARG;
@@ -756,28 +880,14 @@ int fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, i
   const long long BHkv = static_cast<long long>(B) * Hkv;
   const size_t kv_bytes = static_cast<size_t>(BHkv) * Nk * d * 2;
   const size_t lse_bytes = lse ? static_cast<size_t>(BH) * Nq * 4 : 0;
-  if (ranges_overlap(o, o_bytes, q, o_bytes) || ranges_overlap(o, o_bytes, k, kv_bytes) ||
-      ranges_overlap(o, o_bytes, v, kv_bytes) || ranges_overlap(lse, lse_bytes, q, o_bytes) ||
-      ranges_overlap(lse, lse_bytes, k, kv_bytes) || ranges_overlap(lse, lse_bytes, v, kv_bytes) ||
-      ranges_overlap(lse, lse_bytes, o, o_bytes))
+  if (outputs_overlap(q, o_bytes, k, v, kv_bytes, o, o_bytes, lse, lse_bytes))
     return ATTN_ERR_INVALID_ARG;
   const long long n_qblocks = (Nq + kRowsPerCta - 1) / kRowsPerCta;
   if (n_qblocks * BH > 0x7fffffffLL) return ATTN_ERR_INVALID_ARG;
   int rc = check_device();
   if (rc != ATTN_OK) return rc;
 
-  if (Nk == 0) {
-    cudaError_t e = cudaMemsetAsync(o, 0, o_bytes, stream);
-    if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync");
-    if (lse) {
-      const size_t n = static_cast<size_t>(BH) * Nq;
-      const unsigned blocks = static_cast<unsigned>(std::min<size_t>((n + 255) / 256, 4096));
-      fill_neg_inf_kernel<<<blocks, 256, 0, stream>>>(lse, n);
-      e = cudaGetLastError();
-      if (e != cudaSuccess) return cuda_fail(e, "fill_neg_inf_kernel launch");
-    }
-    return ATTN_OK;
-  }
+  if (Nk == 0) return fill_empty(o, o_bytes, lse, static_cast<size_t>(BH) * Nq, stream);
 
   CUtensorMap tq, tk, tv, to;
   const int bh = static_cast<int>(BH);
@@ -787,33 +897,87 @@ int fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, i
       !make_tmap_bf16_3d(&to, o, bh, Nq, d, 32, &t_last_error))
     return ATTN_ERR_CUDA;
 
-  FwdParams prm;
+  FwdParams prm = {};
   prm.lse = lse;
   prm.rescale_count = rescale_count;
+  prm.o = static_cast<__nv_bfloat16*>(o);
   prm.timeout_ns = kWaitTimeoutNs;
   prm.Nq = Nq;
   prm.Nk = Nk;
-  prm.BH = static_cast<int>(BH);
+  prm.BH = bh;
   prm.H = H;
   prm.group = H / Hkv;
-  {
-    // causal schedule: as many heads at once as keep their K/V within ~48 MB
-    // of the 126 MB L2 (several query heads of a GQA group share one K/V head)
-    const double kv_head_bytes = 2.0 * Nk * d * 2.0 / prm.group;
-    const double budget = 48.0 * 1024 * 1024;
-    long long g = static_cast<long long>(budget / std::max(kv_head_bytes, 1.0));
-    prm.hgroup = static_cast<int>(std::max(1LL, std::min(g, BH)));
-  }
+  prm.wl = wl;
+  prm.wr = wr;
+  prm.grouped = (wl == kUnbounded && wr == 0) ? 1 : 0;
+  prm.hgroup = heads_per_l2_group(Nk, d, prm.group, BH);
   prm.n_qblocks = static_cast<int>(n_qblocks);
   prm.scale_log2 = scale * kLog2e;
   prm.tau = tau;
+  return launch_any(d, exp_mode, tq, tk, tv, to, prm, stream);
+}
 
-  if (d == 128) {
-    return causal ? dispatch_exp<128, true>(exp_mode, tq, tk, tv, to, prm, stream)
-                  : dispatch_exp<128, false>(exp_mode, tq, tk, tv, to, prm, stream);
-  }
-  return causal ? dispatch_exp<64, true>(exp_mode, tq, tk, tv, to, prm, stream)
-                : dispatch_exp<64, false>(exp_mode, tq, tk, tv, to, prm, stream);
+int varlen_impl(const void* q, const void* k, const void* v, void* o, float* lse,
+                const int* cu_q, const int* cu_k, int num_seqs, int max_seqlen_q, int total_q,
+                int total_k, int H, int Hkv, int d, float scale, int window_left,
+                int window_right, cudaStream_t stream) {
+  int wl = 0, wr = 0;
+  if (num_seqs < 0 || max_seqlen_q < 0 || total_q < 0 || total_k < 0 || H < 0 || Hkv < 0)
+    return ATTN_ERR_INVALID_ARG;
+  if (H > 0 && (Hkv == 0 || H % Hkv != 0)) return ATTN_ERR_INVALID_ARG;
+  if (!std::isfinite(scale)) return ATTN_ERR_INVALID_ARG;
+  if (!band_from_window(window_left, window_right, &wl, &wr)) return ATTN_ERR_INVALID_ARG;
+  if (max_seqlen_q > total_q) return ATTN_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
+  if (num_seqs == 0 || H == 0 || total_q == 0) return ATTN_OK;  // nothing to compute
+  if (max_seqlen_q == 0) return ATTN_ERR_INVALID_ARG;  // rows exist but no sequence may hold one
+  if (!o || !q || !cu_q || !cu_k || (total_k > 0 && (!k || !v))) return ATTN_ERR_INVALID_ARG;
+  if (misaligned(q, 16) || misaligned(k, 16) || misaligned(v, 16) || misaligned(o, 16) ||
+      misaligned(lse, 4) || misaligned(cu_q, 4) || misaligned(cu_k, 4))
+    return ATTN_ERR_INVALID_ARG;
+  const size_t q_bytes = static_cast<size_t>(total_q) * H * d * 2;
+  const size_t kv_bytes = static_cast<size_t>(total_k) * Hkv * d * 2;
+  const size_t lse_bytes = lse ? static_cast<size_t>(total_q) * H * 4 : 0;
+  if (outputs_overlap(q, q_bytes, k, v, kv_bytes, o, q_bytes, lse, lse_bytes) ||
+      ranges_overlap(o, q_bytes, cu_q, (num_seqs + 1) * 4ull) ||
+      ranges_overlap(o, q_bytes, cu_k, (num_seqs + 1) * 4ull) ||
+      ranges_overlap(lse, lse_bytes, cu_q, (num_seqs + 1) * 4ull) ||
+      ranges_overlap(lse, lse_bytes, cu_k, (num_seqs + 1) * 4ull))
+    return ATTN_ERR_INVALID_ARG;
+  const long long BH = static_cast<long long>(num_seqs) * H;
+  const long long n_qblocks = (max_seqlen_q + kRowsPerCta - 1) / kRowsPerCta;
+  if (BH > 0x7fffffffLL || n_qblocks * BH > 0x7fffffffLL) return ATTN_ERR_INVALID_ARG;
+  int rc = check_device();
+  if (rc != ATTN_OK) return rc;
+
+  if (total_k == 0) return fill_empty(o, q_bytes, lse, static_cast<size_t>(total_q) * H, stream);
+
+  CUtensorMap tq, tk, tv, to;
+  if (!make_tmap_bf16_packed(&tq, q, total_q, H, d, kBlockM, &t_last_error) ||
+      !make_tmap_bf16_packed(&tk, k, total_k, Hkv, d, kBlockN, &t_last_error) ||
+      !make_tmap_bf16_packed(&tv, v, total_k, Hkv, d, kBlockN, &t_last_error) ||
+      !make_tmap_bf16_packed(&to, o, total_q, H, d, 32, &t_last_error))
+    return ATTN_ERR_CUDA;
+
+  FwdParams prm = {};
+  prm.lse = lse;
+  prm.o = static_cast<__nv_bfloat16*>(o);
+  prm.cu_q = cu_q;
+  prm.cu_k = cu_k;
+  prm.timeout_ns = kWaitTimeoutNs;
+  prm.Nq = total_q;
+  prm.Nk = total_k;
+  prm.BH = static_cast<int>(BH);
+  prm.H = H;
+  prm.group = H / Hkv;
+  prm.wl = wl;
+  prm.wr = wr;
+  prm.grouped = (wl == kUnbounded && wr == 0) ? 1 : 0;
+  prm.hgroup = heads_per_l2_group(static_cast<double>(total_k) / num_seqs, d, prm.group, BH);
+  prm.n_qblocks = static_cast<int>(n_qblocks);
+  prm.scale_log2 = scale * kLog2e;
+  prm.tau = kDefaultThreshold;
+  return launch_any(d, 1, tq, tk, tv, to, prm, stream);
 }
 
 }  // namespace eab
@@ -822,22 +986,43 @@ extern "C" {
 
 int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
              int Nq, int Nk, int d, float scale, int causal, cudaStream_t stream) {
-  return eab::fwd_impl(q, k, v, o, lse, B, H, H, Nq, Nk, d, scale, causal, eab::kDefaultThreshold,
-                       1, nullptr, stream);
+  if (causal != 0 && causal != 1) return ATTN_ERR_INVALID_ARG;
+  if (causal && Nq != Nk) return ATTN_ERR_UNSUPPORTED;
+  return eab::fwd_impl(q, k, v, o, lse, B, H, H, Nq, Nk, d, scale, -1, causal ? 0 : -1,
+                       eab::kDefaultThreshold, 1, nullptr, stream);
 }
 
 int attn_fwd_gqa(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
                  int Hkv, int Nq, int Nk, int d, float scale, int causal, cudaStream_t stream) {
-  return eab::fwd_impl(q, k, v, o, lse, B, H, Hkv, Nq, Nk, d, scale, causal,
+  if (causal != 0 && causal != 1) return ATTN_ERR_INVALID_ARG;
+  if (causal && Nq != Nk) return ATTN_ERR_UNSUPPORTED;
+  return eab::fwd_impl(q, k, v, o, lse, B, H, Hkv, Nq, Nk, d, scale, -1, causal ? 0 : -1,
                        eab::kDefaultThreshold, 1, nullptr, stream);
+}
+
+int attn_fwd_window(const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                    int H, int Hkv, int Nq, int Nk, int d, float scale, int window_left,
+                    int window_right, cudaStream_t stream) {
+  return eab::fwd_impl(q, k, v, o, lse, B, H, Hkv, Nq, Nk, d, scale, window_left, window_right,
+                       eab::kDefaultThreshold, 1, nullptr, stream);
+}
+
+int attn_fwd_varlen(const void* q, const void* k, const void* v, void* o, float* lse,
+                    const int* cu_seqlens_q, const int* cu_seqlens_k, int num_seqs,
+                    int max_seqlen_q, int total_q, int total_k, int H, int Hkv, int d,
+                    float scale, int window_left, int window_right, cudaStream_t stream) {
+  return eab::varlen_impl(q, k, v, o, lse, cu_seqlens_q, cu_seqlens_k, num_seqs, max_seqlen_q,
+                          total_q, total_k, H, Hkv, d, scale, window_left, window_right, stream);
 }
 
 int attn_fwd_config(const void* q, const void* k, const void* v, void* o, float* lse, int B,
                     int H, int Nq, int Nk, int d, float scale, int causal,
                     float rescale_threshold, int exp_mode, unsigned long long* rescale_count,
                     cudaStream_t stream) {
-  return eab::fwd_impl(q, k, v, o, lse, B, H, H, Nq, Nk, d, scale, causal, rescale_threshold,
-                       exp_mode, rescale_count, stream);
+  if (causal != 0 && causal != 1) return ATTN_ERR_INVALID_ARG;
+  if (causal && Nq != Nk) return ATTN_ERR_UNSUPPORTED;
+  return eab::fwd_impl(q, k, v, o, lse, B, H, H, Nq, Nk, d, scale, -1, causal ? 0 : -1,
+                       rescale_threshold, exp_mode, rescale_count, stream);
 }
 
 int attn_status_sync(cudaStream_t stream) {
@@ -851,7 +1036,14 @@ int attn_status_sync(cudaStream_t stream) {
   if (e != cudaSuccess) return eab::cuda_fail(e, "clear status word");
   e = cudaStreamSynchronize(stream);
   if (e != cudaSuccess) return eab::cuda_fail(e, "cudaStreamSynchronize");
-  return (st & eab::kStatusTimeout) ? ATTN_ERR_TIMEOUT : ATTN_OK;
+  unsigned int st_bwd = 0;
+  const int rc = eab::bwd_status_take(stream, &st_bwd);
+  if (rc != ATTN_OK) return rc;
+  st |= st_bwd;
+  if (st & eab::kStatusWordTimeout) return ATTN_ERR_TIMEOUT;
+  if (st & eab::kStatusWordLaunch) return ATTN_ERR_CUDA;
+  if (st & eab::kStatusWordBadSeqlens) return ATTN_ERR_INVALID_ARG;
+  return ATTN_OK;
 }
 
 const char* attn_status_string(int code) {

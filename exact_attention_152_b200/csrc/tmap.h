@@ -1,4 +1,5 @@
-// Host-side TMA tensor-map construction for BF16 [B*H, N, d] tensors.
+// Host-side TMA tensor-map construction for BF16 tensors: dense [B*H, N, d]
+// and packed variable-length [total, H, d].
 #pragma once
 
 #include <cuda.h>
@@ -30,21 +31,19 @@ inline EncodeTiledFn get_encode_fn() {
   return fn;
 }
 
-// 3-D view [BH, N, d] of a contiguous BF16 tensor; box = 64 columns of d
-// (128 bytes, 128-byte swizzle) x box_rows rows x 1.  Rows past N read as zero
-// and are clipped on store, per head.  Returns false (and a message) on failure.
-inline bool make_tmap_bf16_3d(CUtensorMap* tm, const void* base, int BH, int N, int d,
-                              int box_rows, std::string* err) {
+// Encodes a 3-D BF16 tensor map: dims innermost first (dims[0] = d, 2-byte
+// elements, contiguous), byte strides of dims 1 and 2, box = 64 columns of d
+// (128 bytes, 128-byte swizzle) x box1 x box2.  Coordinates outside the dims
+// read as zero and are clipped on store.  Returns false (and a message) on failure.
+inline bool encode_bf16_3d(CUtensorMap* tm, const void* base, const cuuint64_t dims[3],
+                           const cuuint64_t strides[2], cuuint32_t box1, cuuint32_t box2,
+                           std::string* err) {
   EncodeTiledFn enc = get_encode_fn();
   if (!enc) {
     *err = "cuTensorMapEncodeTiled unavailable";
     return false;
   }
-  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(N),
-                              static_cast<cuuint64_t>(BH)};
-  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2,
-                                 static_cast<cuuint64_t>(N) * static_cast<cuuint64_t>(d) * 2};
-  const cuuint32_t box[3] = {64u, static_cast<cuuint32_t>(box_rows), 1u};
+  const cuuint32_t box[3] = {64u, box1, box2};
   const cuuint32_t estr[3] = {1u, 1u, 1u};
   CUresult r = enc(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides,
                    box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -54,6 +53,30 @@ inline bool make_tmap_bf16_3d(CUtensorMap* tm, const void* base, int BH, int N, 
     return false;
   }
   return true;
+}
+
+// Dense [BH, N, d]: coordinates (column, row, head); rows past N of one head
+// read as zero (never as the next head's rows) and are clipped on store.
+inline bool make_tmap_bf16_3d(CUtensorMap* tm, const void* base, int BH, int N, int d,
+                              int box_rows, std::string* err) {
+  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(N),
+                              static_cast<cuuint64_t>(BH)};
+  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2,
+                                 static_cast<cuuint64_t>(N) * static_cast<cuuint64_t>(d) * 2};
+  return encode_bf16_3d(tm, base, dims, strides, static_cast<cuuint32_t>(box_rows), 1u, err);
+}
+
+// Packed [total, H, d] (sequences back to back): coordinates (column, head,
+// row); a box is box_rows consecutive rows of one head.  Rows past `total`
+// read as zero and are clipped on store; rows past the end of one sequence are
+// the next sequence's, so the kernel masks them (keys) or stores around them (O).
+inline bool make_tmap_bf16_packed(CUtensorMap* tm, const void* base, int total, int H, int d,
+                                  int box_rows, std::string* err) {
+  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(H),
+                              static_cast<cuuint64_t>(total)};
+  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2,
+                                 static_cast<cuuint64_t>(H) * static_cast<cuuint64_t>(d) * 2};
+  return encode_bf16_3d(tm, base, dims, strides, 1u, static_cast<cuuint32_t>(box_rows), err);
 }
 
 }  // namespace eab

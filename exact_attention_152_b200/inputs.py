@@ -18,6 +18,7 @@ Definition (fixed here, used by every consumer):
                z = sqrt(-2 ln u1) * cos(2 pi u2)   (Box-Muller, cosine branch, fp64)
   uniform    : u = (bits >> 40) / 2^24,  z = 2u - 1  in [-1, 1)
   value      = bf16_rne(fp32_rne(mult * z))
+  unit draw  : (bits >> 11) / 2^53 in [0, 1), fp64 (sequence lengths; id 3)
 
 (SplitMix64: Steele, Lea & Flood, "Fast splittable pseudorandom number
 generators", OOPSLA 2014.)
@@ -33,7 +34,7 @@ GAMMA = np.uint64(0x9E3779B97F4A7C15)
 _M1 = np.uint64(0xBF58476D1CE4E5B9)
 _M2 = np.uint64(0x94D049BB133111EB)
 
-TENSOR_ID = {"q": 0, "k": 1, "v": 2}
+TENSOR_ID = {"q": 0, "k": 1, "v": 2, "len": 3}  # "len": sequence lengths of a packed batch
 
 _CHUNK = 1 << 22
 
@@ -101,6 +102,12 @@ def gen_bf16_at(seed: int, tensor: str, flat_idx: np.ndarray, dist: str = "norma
     for s in range(0, flat.size, _CHUNK):
         out[s:s + _CHUNK] = _values(key, flat[s:s + _CHUNK], dist, mult)
     return out.reshape(idx.shape)
+
+
+def uniform_at(seed: int, tensor: str, idx: np.ndarray) -> np.ndarray:
+    """fp64 draws in [0, 1) at the given counter indices of stream ``tensor``."""
+    bits = _bits(_key(seed, TENSOR_ID[tensor]), np.asarray(idx, dtype=np.int64))
+    return (bits >> np.uint64(11)).astype(np.float64) * (1.0 / 9007199254740992.0)
 
 
 def gen_bf16(seed: int, tensor: str, shape, dist: str = "normal", mult: float = 1.0,

@@ -32,6 +32,28 @@ class Workload:
     v_dist: str = "normal"
     oracle_rows: int | None = None  # sampled rows per head for the oracle; None = all
     Hkv: int | None = None          # key/value heads (grouped-query attention); None = H
+    window: tuple | None = None     # key band (left, right), -1 = no bound; replaces causal
+    seqlens: tuple | None = None    # packed variable-length batch: one length per sequence
+                                    # (queries and keys alike); B = len(seqlens)
+
+    @property
+    def packed(self) -> bool:
+        return self.seqlens is not None
+
+    @property
+    def band(self) -> tuple:
+        """(window_left, window_right) of the mask: -1 = no bound."""
+        if self.window is not None:
+            return tuple(self.window)
+        return (-1, 0) if self.causal else (-1, -1)
+
+    @property
+    def cu_seqlens(self) -> np.ndarray:
+        return np.concatenate([[0], np.cumsum(self.seqlens)]).astype(np.int32)
+
+    @property
+    def total(self) -> int:
+        return int(sum(self.seqlens))
 
     @property
     def kv_heads(self) -> int:
@@ -43,11 +65,20 @@ class Workload:
 
     @property
     def flops(self) -> float:
-        """Algorithmic FLOPs: 4*B*H*Nq*Nk*d, halved when causal."""
-        f = 4.0 * self.B * self.H * self.Nq * self.Nk * self.d
-        return f / 2 if self.causal else f
+        """Algorithmic FLOPs, 4*d per visible (query, key) pair: 4*B*H*Nq*Nk*d
+        without a mask, half of that for causal (the usual convention), and the
+        exact count of visible pairs for a band or a packed batch."""
+        if self.window is None and not self.packed:
+            f = 4.0 * self.B * self.H * self.Nq * self.Nk * self.d
+            return f / 2 if self.causal else f
+        lens = self.seqlens if self.packed else [self.Nq] * self.B
+        pairs = sum(float(visible_keys(np.arange(n), n, *self.band).sum()) for n in lens)
+        return 4.0 * self.d * self.H * pairs
 
     def shape(self, which: str):
+        heads = self.H if which == "q" else self.kv_heads
+        if self.packed:
+            return (self.total, heads, self.d)
         if which == "q":
             return (self.B, self.H, self.Nq, self.d)
         return (self.B, self.kv_heads, self.Nk, self.d)
@@ -83,10 +114,37 @@ class Workload:
         b, h = divmod(bh, self.H)
         return b * self.kv_heads + h // (self.H // self.kv_heads)
 
+    def seq_head_bits(self, which: str, s: int, h: int, rows=None) -> np.ndarray:
+        """Packed batch: BF16 bits of sequence s, head h (a key/value head for
+        k and v), rows `rows` of the sequence (default all) -> [n, d]."""
+        dist, mult = self.dist(which)
+        heads = self.H if which == "q" else self.kv_heads
+        start = int(self.cu_seqlens[s])
+        if rows is None:
+            rows = np.arange(self.seqlens[s], dtype=np.int64)
+        idx = ((start + np.asarray(rows, dtype=np.int64))[:, None] * heads + h) * self.d \
+            + np.arange(self.d, dtype=np.int64)[None, :]
+        return inputs.gen_bf16_at(self.seed, which, idx, dist, mult)
+
     def sampled_rows(self, bh: int) -> np.ndarray:
         if self.oracle_rows is None:
             return np.arange(self.Nq, dtype=np.int64)
         return inputs.sample_rows(self.seed, bh, self.Nq, self.oracle_rows)
+
+
+def visible_keys(rows, nk, window_left, window_right) -> np.ndarray:
+    """Number of keys in the band [i - left, i + right] of each query row i,
+    clipped to 0 .. nk-1 (-1 = no bound)."""
+    rows = np.asarray(rows, dtype=np.int64)
+    lo = np.zeros_like(rows) if window_left < 0 else np.maximum(rows - window_left, 0)
+    hi = np.full_like(rows, nk - 1) if window_right < 0 else np.minimum(rows + window_right, nk - 1)
+    return np.maximum(hi - lo + 1, 0)
+
+
+def _mixed_lengths(seed, n, lo, hi):
+    """n sequence lengths, uniform in [lo, hi], from the counter-based generator."""
+    u = inputs.uniform_at(seed, "len", np.arange(n, dtype=np.int64))
+    return tuple(int(lo + (hi - lo) * x) for x in u)
 
 
 WORKLOADS = {
@@ -104,6 +162,12 @@ WORKLOADS = {
                  Hkv=8),
         Workload("gqa_b2h32kv8n8k_d128_causal", 2, 32, 8192, 8192, 128, True, seed=5,
                  oracle_rows=128, Hkv=8),
+        # causal sliding window over the last 4096 keys
+        Workload("swa_b1h32n32k_w4k_d128", 1, 32, 32768, 32768, 128, False, seed=6,
+                 oracle_rows=128, window=(4095, 0)),
+        # 16 sequences of mixed length (512 .. 16384 tokens), packed, causal
+        Workload("varlen16_h16_d128_causal", 16, 16, 0, 0, 128, True, seed=7, oracle_rows=64,
+                 seqlens=_mixed_lengths(7, 16, 512, 16384)),
     ]
 }
 

@@ -6,7 +6,7 @@
  * What is computed.  FlashAttention 4: LLM向けのより高速でメモリ効率の良いアテンション
  * (ja.linux-konsole.com), section "はじめに": attention multiplies the queries Q
  * with the keys K, normalises with a softmax and multiplies by the values V.
- * Flash Attention glossary (jisaku.com), section "タイリングによるSRAMの活用" and
+ * "Flash Attention（Flash Attention）" (jisaku.com glossary), section "タイリングによるSRAMの活用" and
  * "オンライン・ソフトマックスと再計算": the work is tiled through on-chip memory
  * with a running per-row max and sum, so the Nq x Nk score matrix never reaches
  * device memory; FAQ Q3 on the same page: the result equals standard attention
@@ -44,6 +44,8 @@
 #ifdef __cplusplus
 extern "C" {
 #endif
+
+#include <stddef.h>
 
 /* Same definition as the CUDA runtime's (an opaque driver stream handle). */
 typedef struct CUstream_st *cudaStream_t;
@@ -90,6 +92,55 @@ int attn_fwd_gqa(const void *q, const void *k, const void *v, void *o, float *ls
                  int Hkv, int Nq, int Nk, int d, float scale, int causal, cudaStream_t stream);
 
 /*
+ * Sliding-window (local) attention: each query sees a band of keys around its
+ * own position.  The pages only name richer masks than causal ("AIの「脳の回転」
+ * を1.8倍高速化？FlashAttentionの秘密", gipyeong-lee.github.io, section
+ * "今後はどうなるか？", pointing to FlashMask); this library's reading is
+ *
+ *     K(i) = { j : 0 <= j < Nk,  i - window_left <= j <= i + window_right }
+ *
+ * with -1 for "no bound on that side": (-1, -1) is attn_fwd non-causal,
+ * (-1, 0) is causal, (w, 0) is causal attention over the last w+1 keys.
+ * Positions of queries and keys both count from 0, so Nq != Nk is allowed; a
+ * row whose band holds no key gets O = 0, LSE = -inf.
+ *   q, o : [B, H, Nq, d];  k, v : [B, Hkv, Nk, d];  lse : [B, H, Nq] (may be NULL)
+ *   Hkv  : as attn_fwd_gqa (Hkv == H: one key/value head per query head)
+ *   window_left, window_right : >= -1; anything below -1 is ATTN_ERR_INVALID_ARG
+ * Only KV tiles that hold a visible key are read.
+ */
+int attn_fwd_window(const void *q, const void *k, const void *v, void *o, float *lse, int B,
+                    int H, int Hkv, int Nq, int Nk, int d, float scale, int window_left,
+                    int window_right, cudaStream_t stream);
+
+/*
+ * Variable-length batch: sequences of different lengths packed back to back,
+ * with no padding (FlashAttention 4 page, ja.linux-konsole.com, section
+ * "互換性と現状", lists this among what FA4's forward lacks).
+ *   q, o : BF16 [total_q, H, d]    k, v : BF16 [total_k, Hkv, d]   (d fastest)
+ *   lse  : FP32 [H, total_q], may be NULL
+ *   cu_seqlens_q, cu_seqlens_k : DEVICE int32 arrays of num_seqs + 1 entries;
+ *       sequence s owns query rows cu_seqlens_q[s] .. cu_seqlens_q[s+1]-1 and
+ *       key/value rows cu_seqlens_k[s] .. cu_seqlens_k[s+1]-1 (non-decreasing,
+ *       starting at >= 0, ending at <= total_q / total_k; a sequence may be
+ *       empty, and its query and key lengths may differ)
+ *   max_seqlen_q : an upper bound on every sequence's query length (sizes the
+ *       grid), 1 <= max_seqlen_q <= total_q when total_q > 0
+ *   H, Hkv, d, scale : as attn_fwd_gqa
+ *   window_left, window_right : the band of attn_fwd_window over positions
+ *       counted from 0 within each sequence; (-1, 0) is causal, (-1, -1) none
+ * Each sequence is attended independently: no query sees another sequence's
+ * keys.  The offsets live on the device and are not read by the host: offsets
+ * that break the rules above (or a sequence longer than max_seqlen_q rounded up
+ * to 256) make the kernel skip that sequence and record the fact, which the next
+ * attn_status_sync() returns as ATTN_ERR_INVALID_ARG; no access goes outside
+ * the tensors.  All other errors are detected on the host as for attn_fwd.
+ */
+int attn_fwd_varlen(const void *q, const void *k, const void *v, void *o, float *lse,
+                    const int *cu_seqlens_q, const int *cu_seqlens_k, int num_seqs,
+                    int max_seqlen_q, int total_q, int total_k, int H, int Hkv, int d,
+                    float scale, int window_left, int window_right, cudaStream_t stream);
+
+/*
  * attn_fwd with the kernel's two softmax knobs exposed (same contract otherwise).
  *
  *   rescale_threshold : adaptive online rescaling (FlashAttention 4 page,
@@ -111,9 +162,46 @@ int attn_fwd_config(const void *q, const void *k, const void *v, void *o, float 
                     cudaStream_t stream);
 
 /*
+ * Backward pass: the gradients dQ, dK, dV of the forward above (causal or not,
+ * grouped key/value heads allowed) for the output cotangent dO.  The pages name
+ * the backward pass as what FlashAttention 4 lacks (FlashAttention 4 page,
+ * ja.linux-konsole.com, sections "重要ポイント" and "互換性と現状";
+ * "FlashAttention-4：非対称ハードウェアスケーリング…" (sns.style), section 二) and give no formula; this
+ * library computes the chain rule through the definition above:
+ *
+ *     P_ij  = exp(scale * <q_i, k_j> - LSE_i)      (j visible to i, else 0)
+ *     dS_ij = P_ij * (<dO_i, v_j> - <dO_i, O_i>)
+ *     dV_j  = sum_i P_ij dO_i
+ *     dK_j  = scale * sum_i dS_ij q_i,   dQ_i = scale * sum_j dS_ij k_j
+ *
+ * summed over the query heads that share a key/value head.
+ *   q, o, dout : BF16 [B, H, Nq, d]      k, v : BF16 [B, Hkv, Nk, d]
+ *   lse        : FP32 [B, H, Nq], the forward's log-sum-exp (natural log)
+ *   dq         : BF16 [B, H, Nq, d] written;  dk, dv : BF16 [B, Hkv, Nk, d] written
+ *   workspace  : DEVICE scratch of at least attn_bwd_workspace_size(B, H, Nq, d)
+ *                bytes, 256-byte aligned, owned by the caller, not overlapping
+ *                any other argument; its contents are overwritten (the row sums
+ *                <dO_i, O_i> and dQ's fp32 accumulator)
+ *   B, H, Hkv, Nq, Nk, d, scale, causal : as attn_fwd_gqa
+ * All pointers 16-byte aligned (lse 4).  Outputs may not overlap inputs or each
+ * other.  Nk == 0 gives dQ = 0; Nq == 0 gives dK = dV = 0.  Asynchronous on
+ * `stream` like attn_fwd; argument errors are returned before anything is
+ * enqueued, device-side failures through attn_status_sync().
+ */
+int attn_bwd(const void *q, const void *k, const void *v, const void *o, const void *dout,
+             const float *lse, void *dq, void *dk, void *dv, void *workspace,
+             size_t workspace_bytes, int B, int H, int Hkv, int Nq, int Nk, int d, float scale,
+             int causal, cudaStream_t stream);
+
+/* Workspace bytes attn_bwd needs (0 for d not in {64, 128} or negative sizes). */
+size_t attn_bwd_workspace_size(int B, int H, int Nq, int d);
+
+/*
  * Synchronise `stream`, then read and clear the current device's status word.
  * Returns ATTN_OK, ATTN_ERR_TIMEOUT (a kernel gave up on a pipeline wait since
- * the last call; its outputs are not valid) or ATTN_ERR_CUDA.
+ * the last call; its outputs are not valid), ATTN_ERR_INVALID_ARG (an
+ * attn_fwd_varlen call met bad sequence offsets on the device; the outputs of
+ * those sequences were not written) or ATTN_ERR_CUDA.
  */
 int attn_status_sync(cudaStream_t stream);
 

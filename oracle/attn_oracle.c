@@ -13,7 +13,7 @@
  *   multiplies them with the keys K, normalises the result with a softmax and
  *   multiplies that with the values V.
  *
- *   Flash Attention glossary (jisaku.com), sections "主要な最適化ポイントのまとめ"
+ *   "Flash Attention（Flash Attention）" (jisaku.com glossary), sections "主要な最適化ポイントのまとめ"
  *   and "FAQ" (Q3): the tiled method is exact -- it equals standard attention up
  *   to floating-point rounding -- so the oracle is the standard definition
  *   written out.
@@ -192,7 +192,7 @@ int oracle_attn_rows_f64(const double *q, const int64_t *rows, int64_t n_rows,
  * Backward pass of one (batch, head): the vector-Jacobian product of the
  * forward map above with the output cotangent dO.  FlashAttention 4 page
  * (ja.linux-konsole.com), sections "重要ポイント" and "互換性と現状", and
- * "FlashAttention-4 deep dive" (sns.style), section 二: the backward pass --
+ * "FlashAttention-4：非対称ハードウェアスケーリング…" (sns.style), section 二: the backward pass --
  * the gradients needed for training -- is what FA4 still lacks.  The pages give
  * no formulas; this is the chain rule through s -> softmax -> P.V, per query
  * row i over its visible keys j:

@@ -48,7 +48,8 @@ def test_library_exports_every_declared_symbol(header):
 
 def test_attn_h_declares_the_contract():
     names = declared_functions(os.path.join(ROOT, "include", "attn.h"))
-    for n in ("attn_fwd", "attn_fwd_config", "attn_fwd_gqa", "attn_status_sync", "attn_status_string",
+    for n in ("attn_fwd", "attn_fwd_config", "attn_fwd_gqa", "attn_fwd_window", "attn_fwd_varlen",
+              "attn_bwd", "attn_bwd_workspace_size", "attn_status_sync", "attn_status_string",
               "attn_last_error", "attn_selftest_timeout"):
         assert n in names
 
@@ -105,6 +106,61 @@ def test_gqa_validation():
     assert binding.attn_fwd_gqa(None, None, None, None, None, 0, 6, 2, 8, 8, 64, 0.1, 0, None) == 0
     # the other checks still apply
     assert binding.attn_fwd_gqa(*base, 6, 2, 8, 8, 96, 0.1, 0, None) == 2
+
+
+def test_window_validation():
+    W = binding.attn_fwd_window
+    base = (ALIGNED, ALIGNED, ALIGNED, ALIGNED * 16, None, 1, 4, 2, 8, 8, 64, 0.1)
+    assert W(*base, -2, 0, None) == 1        # bounds below -1
+    assert W(*base, 0, -5, None) == 1
+    assert W(ALIGNED, ALIGNED, ALIGNED, ALIGNED * 16, None, 1, 4, 3, 8, 8, 64, 0.1, 3, 3, None) == 1
+    assert W(*base[:10], 96, 0.1, 3, 3, None) == 2
+    assert W(*base[:11], math.nan, 3, 3, None) == 1
+    # empty problems are a no-op whatever the band
+    assert W(None, None, None, None, None, 0, 4, 2, 8, 8, 64, 0.1, 3, 0, None) == 0
+
+
+def test_varlen_validation():
+    V = binding.attn_fwd_varlen
+    P = (ALIGNED, ALIGNED, ALIGNED, ALIGNED * 16, None, ALIGNED * 64, ALIGNED * 65)
+    ok_sizes = (2, 100, 150, 150, 4, 2, 64, 0.1, -1, 0)   # seqs, max_q, total_q, total_k, H, Hkv, d, ...
+    def call(ptrs=P, sizes=ok_sizes):
+        return V(*ptrs, *sizes, None)
+    assert call(sizes=(-1,) + ok_sizes[1:]) == 1                      # negative num_seqs
+    assert call(sizes=ok_sizes[:1] + (200,) + ok_sizes[2:]) == 1      # max_seqlen_q > total_q
+    assert call(sizes=ok_sizes[:1] + (0,) + ok_sizes[2:]) == 1        # rows but no room for them
+    assert call(sizes=ok_sizes[:5] + (3,) + ok_sizes[6:]) == 1        # H % Hkv != 0
+    assert call(sizes=ok_sizes[:6] + (80,) + ok_sizes[7:]) == 2       # head dim
+    assert call(sizes=ok_sizes[:7] + (math.inf,) + ok_sizes[8:]) == 1
+    assert call(sizes=ok_sizes[:8] + (-3, 0)) == 1                    # band
+    assert call(ptrs=P[:5] + (None,) + P[6:]) == 1                    # null offsets
+    assert call(ptrs=P[:5] + (ALIGNED * 64 + 2,) + P[6:]) == 1        # misaligned offsets
+    assert call(ptrs=(ALIGNED + 8,) + P[1:]) == 1                     # misaligned q
+    assert call(ptrs=P[:3] + (ALIGNED,) + P[4:]) == 1                 # o overlaps q
+    assert call(ptrs=P[:5] + (ALIGNED * 16,) + P[6:]) == 1            # offsets inside o
+    # nothing to compute: a no-op even with null pointers
+    assert V(None, None, None, None, None, None, None, 0, 0, 0, 0, 4, 2, 64, 0.1, -1, 0, None) == 0
+    assert V(None, None, None, None, None, None, None, 3, 0, 0, 0, 4, 2, 64, 0.1, -1, 0, None) == 0
+
+
+def test_bwd_validation():
+    Bw = binding.attn_bwd
+    A = ALIGNED
+    ptrs = (A, A * 2, A * 3, A * 4, A * 5, A * 6, A * 7, A * 8, A * 9, A * 16)
+    need = binding.attn_bwd_workspace_size(1, 2, 64, 64)
+    assert need == 512 + 1 * 2 * 64 * 64 * 4   # row sums (256-aligned) + fp32 dQ
+    assert binding.attn_bwd_workspace_size(1, 2, 64, 96) == 0
+    sizes = (1, 2, 2, 64, 64, 64, 0.1, 0)
+    assert Bw(*ptrs, need - 1, *sizes, None) == 1                # workspace too small
+    assert Bw(*ptrs[:9], None, need, *sizes, None) == 1          # no workspace
+    assert Bw(*ptrs[:9], A * 16 + 16, need, *sizes, None) == 1   # workspace misaligned (256)
+    assert Bw(*ptrs, need, 1, 2, 2, 64, 64, 80, 0.1, 0, None) == 2
+    assert Bw(*ptrs, need, 1, 2, 2, 64, 32, 64, 0.1, 1, None) == 2   # causal Nq != Nk
+    assert Bw(*ptrs, need, 1, 3, 2, 64, 64, 64, 0.1, 0, None) == 1   # H % Hkv
+    assert Bw(*ptrs, need, 1, 2, 2, 64, 64, 64, math.inf, 0, None) == 1
+    assert Bw(*ptrs[:6], A, *ptrs[7:], need, *sizes, None) == 1   # dq overlaps q
+    assert Bw(*ptrs[:9], A * 9, need, *sizes, None) == 1         # workspace overlaps dv
+    assert Bw(*(None,) * 10, 0, 0, 2, 2, 64, 64, 64, 0.1, 0, None) == 0   # empty batch
 
 
 def test_config_knob_validation():

@@ -13,6 +13,7 @@ import pytest
 pytestmark = pytest.mark.gpu
 
 import harness  # noqa: E402
+import oracle  # noqa: E402
 from exact_attention_152_b200 import inputs  # noqa: E402
 from exact_attention_152_b200.workloads import WORKLOADS  # noqa: E402
 
@@ -187,18 +188,37 @@ def _workload_case(w):
     q = w.tensor_bits("q")
     k = w.tensor_bits("k")
     v = w.tensor_bits("v")
-    o, lse = harness.run_cuda(q, k, v, w.scale, w.causal)
+    if w.window is not None:
+        o, lse = harness.run_cuda(q, k, v, w.scale, False, window=w.band)
+    else:
+        o, lse = harness.run_cuda(q, k, v, w.scale, w.causal)
     rows = None
     if w.oracle_rows is not None:
         rows = {bh: w.sampled_rows(bh) for bh in range(w.B * w.H)}
-    ref = harness.oracle_rows(q, k, v, w.scale, w.causal, rows, kv_group=w.H // w.kv_heads)
+    ref = harness.oracle_rows(q, k, v, w.scale, w.causal, rows, kv_group=w.H // w.kv_heads,
+                              band=w.band)
     return o, lse, ref
+
+
+def _packed_case(w):
+    q, k, v = (w.tensor_bits(x) for x in "qkv")
+    cu = w.cu_seqlens
+    o, lse = harness.run_varlen(q, k, v, cu, cu, max(w.seqlens), w.scale, w.band)
+    rows = {s: inputs.sample_rows(w.seed, s, n, w.oracle_rows or n)
+            for s, n in enumerate(w.seqlens)}
+    ref = oracle.attn_varlen(inputs.bf16_bits_to_f64(q), inputs.bf16_bits_to_f64(k),
+                             inputs.bf16_bits_to_f64(v), cu, cu, w.scale, *w.band,
+                             rows_per_seq=rows)
+    return harness.compare_varlen(o, lse, ref, cu)
 
 
 @pytest.mark.parametrize("name", list(WORKLOADS))
 def test_workload_parity(name):
     w = WORKLOADS[name]
-    o, lse, ref = _workload_case(w)
-    m = harness.compare(o, lse, ref)
+    if w.packed:
+        m = _packed_case(w)
+    else:
+        o, lse, ref = _workload_case(w)
+        m = harness.compare(o, lse, ref)
     print(name, m)
     harness.assert_within(m)
