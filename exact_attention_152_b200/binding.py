@@ -56,6 +56,8 @@ def lib() -> ctypes.CDLL:
             l.attn_fwd_varlen.restype = _I
             l.attn_bwd.argtypes = [_P] * 10 + [ctypes.c_size_t] + [_I] * 6 + [ctypes.c_float, _I, _P]
             l.attn_bwd.restype = _I
+            l.attn_bwd_noalloc.argtypes = [_P] * 9 + [_I] * 6 + [ctypes.c_float, _I, _P]
+            l.attn_bwd_noalloc.restype = _I
             l.attn_bwd_workspace_size.argtypes = [_I, _I, _I, _I]
             l.attn_bwd_workspace_size.restype = ctypes.c_size_t
             l.attn_status_sync.argtypes = [_P]
@@ -101,6 +103,12 @@ def attn_bwd(q, k, v, o, dout, lse, dq, dk, dv, workspace, workspace_bytes, B, H
              scale, causal, stream) -> int:
     return lib().attn_bwd(q, k, v, o, dout, lse, dq, dk, dv, workspace, workspace_bytes, B, H, Hkv,
                           Nq, Nk, d, scale, causal, stream)
+
+
+def attn_bwd_noalloc(q, k, v, o, dout, lse, dq, dk, dv, B, H, Hkv, Nq, Nk, d, scale, causal,
+                     stream) -> int:
+    return lib().attn_bwd_noalloc(q, k, v, o, dout, lse, dq, dk, dv, B, H, Hkv, Nq, Nk, d, scale,
+                                  causal, stream)
 
 
 def attn_bwd_workspace_size(B, H, Nq, d) -> int:

@@ -711,6 +711,26 @@ int bwd_impl(const void* q, const void* k, const void* v, const void* o, const v
   return ATTN_OK;
 }
 
+// attn_bwd_noalloc: the same computation with its workspace in a file-scope
+// device array, so the call itself allocates no memory.
+constexpr size_t kStaticScratchBytes = size_t(96) << 20;  // 96 MiB per device
+__device__ __align__(256) unsigned char g_bwd_scratch[kStaticScratchBytes];
+
+// Device address of g_bwd_scratch on the current device, looked up once per device.
+int static_scratch(void** ptr) {
+  static std::once_flag once[kMaxDeviceCount];
+  static void* addr[kMaxDeviceCount];
+  static cudaError_t err[kMaxDeviceCount];
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= kMaxDeviceCount) return ATTN_ERR_UNSUPPORTED;
+  std::call_once(once[dev], [&] { err[dev] = cudaGetSymbolAddress(&addr[dev], g_bwd_scratch); });
+  if (err[dev] != cudaSuccess) return cuda_fail(err[dev], "cudaGetSymbolAddress");
+  *ptr = addr[dev];
+  return ATTN_OK;
+}
+
 }  // namespace bwd
 
 int bwd_status_take(cudaStream_t stream, unsigned int* status) {
@@ -747,6 +767,20 @@ int attn_bwd(const void* q, const void* k, const void* v, const void* o, const v
              int causal, cudaStream_t stream) {
   return eab::bwd::bwd_impl(q, k, v, o, dout, lse, dq, dk, dv, workspace, workspace_bytes, B, H, Hkv,
                             Nq, Nk, d, scale, causal, stream);
+}
+
+int attn_bwd_noalloc(const void* q, const void* k, const void* v, const void* o, const void* dout,
+                     const float* lse, void* dq, void* dk, void* dv, int B, int H, int Hkv, int Nq,
+                     int Nk, int d, float scale, int causal, cudaStream_t stream) {
+  // sizes beyond the static scratch are refused before anything else happens
+  if (B >= 0 && H >= 0 && Nq >= 0 && (d == 64 || d == 128) &&
+      eab::bwd::workspace_bytes(static_cast<long long>(B) * H, Nq, d) > eab::bwd::kStaticScratchBytes)
+    return ATTN_ERR_UNSUPPORTED;
+  void* ws = nullptr;
+  const int rc = eab::bwd::static_scratch(&ws);
+  if (rc != ATTN_OK) return rc;
+  return eab::bwd::bwd_impl(q, k, v, o, dout, lse, dq, dk, dv, ws, eab::bwd::kStaticScratchBytes, B, H,
+                            Hkv, Nq, Nk, d, scale, causal, stream);
 }
 
 }  // extern "C"

@@ -197,6 +197,19 @@ int attn_bwd(const void *q, const void *k, const void *v, const void *o, const v
 size_t attn_bwd_workspace_size(int B, int H, int Nq, int d);
 
 /*
+ * attn_bwd without a workspace argument: the workspace is a file-scope device
+ * array of 96 MiB (100663296 bytes) per device inside the library, so the call
+ * allocates no memory (no cudaMalloc / cudaFree).  Problems whose
+ * attn_bwd_workspace_size exceeds 96 MiB return ATTN_ERR_UNSUPPORTED before
+ * anything else is done.  Every call on a device uses the same array: calls
+ * must be ordered (one stream, or synchronised between streams).  Arguments
+ * and results are otherwise those of attn_bwd.
+ */
+int attn_bwd_noalloc(const void *q, const void *k, const void *v, const void *o, const void *dout,
+                     const float *lse, void *dq, void *dk, void *dv, int B, int H, int Hkv, int Nq,
+                     int Nk, int d, float scale, int causal, cudaStream_t stream);
+
+/*
  * Synchronise `stream`, then read and clear the current device's status word.
  * Returns ATTN_OK, ATTN_ERR_TIMEOUT (a kernel gave up on a pipeline wait since
  * the last call; its outputs are not valid), ATTN_ERR_INVALID_ARG (an

@@ -49,7 +49,7 @@ def test_library_exports_every_declared_symbol(header):
 def test_attn_h_declares_the_contract():
     names = declared_functions(os.path.join(ROOT, "include", "attn.h"))
     for n in ("attn_fwd", "attn_fwd_config", "attn_fwd_gqa", "attn_fwd_window", "attn_fwd_varlen",
-              "attn_bwd", "attn_bwd_workspace_size", "attn_status_sync", "attn_status_string",
+              "attn_bwd", "attn_bwd_noalloc", "attn_bwd_workspace_size", "attn_status_sync", "attn_status_string",
               "attn_last_error", "attn_selftest_timeout"):
         assert n in names
 
