@@ -54,6 +54,8 @@ def lib() -> ctypes.CDLL:
             l.attn_fwd_varlen.argtypes = [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I,
                                           ctypes.c_float, _I, _I, _P]
             l.attn_fwd_varlen.restype = _I
+            l.attn_fwd_fp8.argtypes = [_P, _P, _P, _P, _P] + [_I] * 6 + [ctypes.c_float] * 4 + [_I, _P]
+            l.attn_fwd_fp8.restype = _I
             l.attn_bwd.argtypes = [_P] * 10 + [ctypes.c_size_t] + [_I] * 6 + [ctypes.c_float, _I, _P]
             l.attn_bwd.restype = _I
             l.attn_bwd_noalloc.argtypes = [_P] * 9 + [_I] * 6 + [ctypes.c_float, _I, _P]
@@ -91,6 +93,12 @@ def attn_fwd_varlen(q, k, v, o, lse, cu_seqlens_q, cu_seqlens_k, num_seqs, max_s
     return lib().attn_fwd_varlen(q, k, v, o, lse, cu_seqlens_q, cu_seqlens_k, num_seqs,
                                  max_seqlen_q, total_q, total_k, H, Hkv, d, scale, window_left,
                                  window_right, stream)
+
+
+def attn_fwd_fp8(q, k, v, o, lse, B, H, Hkv, Nq, Nk, d, scale, q_descale, k_descale, v_descale,
+                 causal, stream) -> int:
+    return lib().attn_fwd_fp8(q, k, v, o, lse, B, H, Hkv, Nq, Nk, d, scale, q_descale, k_descale,
+                              v_descale, causal, stream)
 
 
 def attn_fwd_config(q, k, v, o, lse, B, H, Nq, Nk, d, scale, causal, rescale_threshold,
@@ -285,3 +293,29 @@ def bwd(q, k, v, o, dout, lse, causal: bool = False, scale: float | None = None,
                   int(bool(causal)), stream)
     check(rc, "attn_bwd")
     return dq, dk, dv
+
+
+def fwd_fp8(q, k, v, descale=(1.0, 1.0, 1.0), causal: bool = False, scale: float | None = None):
+    """FP8 forward: q [B,H,Nq,d], k/v [B,Hkv,Nk,d] uint8 CUDA tensors of E4M3
+    codes (or torch.float8_e4m3fn), descale = (q, k, v) scale factors.
+    Returns (o BF16 [B,H,Nq,d], lse fp32 [B,H,Nq])."""
+    import torch
+
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        if not isinstance(t, torch.Tensor) or not t.is_cuda or t.element_size() != 1 \
+                or t.dim() != 4 or not t.is_contiguous():
+            raise TypeError(f"{name} must be a contiguous 4-D one-byte CUDA tensor of E4M3 codes")
+    B, H, Nq, d = q.shape
+    Hkv, Nk = k.shape[1], k.shape[2]
+    if tuple(k.shape) != (B, Hkv, Nk, d) or tuple(v.shape) != (B, Hkv, Nk, d):
+        raise ValueError("k and v must be [B, Hkv, Nk, d] matching q")
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    o = torch.empty((B, H, Nq, d), dtype=torch.bfloat16, device=q.device)
+    lse = torch.empty((B, H, Nq), dtype=torch.float32, device=q.device)
+    stream = torch.cuda.current_stream(q.device).cuda_stream
+    rc = attn_fwd_fp8(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), B, H,
+                      Hkv, Nq, Nk, d, float(scale), *(float(x) for x in descale), int(bool(causal)),
+                      stream)
+    check(rc, "attn_fwd_fp8")
+    return o, lse

@@ -26,6 +26,9 @@ def lib() -> ctypes.CDLL:
                                ("blocks_mma_ts", [_P, _P, _P, _I, _P]),
                                ("blocks_swizzle_roundtrip", [_P, _P, _P, _I, _P]),
                                ("blocks_exp2", [_P, _P, _P, _I, _P]),
+                               ("blocks_mma_e4m3_ss", [_P, _P, _P, _P]),
+                               ("blocks_mma_e4m3_ts", [_P, _P, _P, _P]),
+                               ("blocks_pack_e4m3", [_P, _P, _I, _P]),
                                ("blocks_status_sync", [_P])):
                 f = getattr(l, name)
                 f.argtypes = args
@@ -48,6 +51,18 @@ def blocks_swizzle_roundtrip(x, y_tma, y_plain, d, stream) -> int:
 
 def blocks_exp2(x, y_mufu, y_poly, n, stream) -> int:
     return lib().blocks_exp2(x, y_mufu, y_poly, n, stream)
+
+
+def blocks_mma_e4m3_ss(a, b, c, stream) -> int:
+    return lib().blocks_mma_e4m3_ss(a, b, c, stream)
+
+
+def blocks_mma_e4m3_ts(p, v, c, stream) -> int:
+    return lib().blocks_mma_e4m3_ts(p, v, c, stream)
+
+
+def blocks_pack_e4m3(x, y, n4, stream) -> int:
+    return lib().blocks_pack_e4m3(x, y, n4, stream)
 
 
 def blocks_status_sync(stream) -> int:

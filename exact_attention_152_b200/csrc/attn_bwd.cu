@@ -85,7 +85,7 @@ struct Cfg {
   static constexpr int kDSBytes = 2 * kBoxBytes;
   static constexpr int kOffRow = kOffDS + kDSBytes; // per stage: LSE*log2e [128], D [128]
   static constexpr int kRowBytes = 2 * 2 * kBlockQ * 4;
-  static constexpr int kNumBars = 11;
+  static constexpr int kNumBars = 12;
   static constexpr int kOffBar = kOffRow + kRowBytes;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
   static constexpr int kSmemBytes = kOffMisc + 16;
@@ -129,6 +129,8 @@ struct Smem {
   __device__ __forceinline__ uint32_t dq_full() const { return bar(8); }
   __device__ __forceinline__ uint32_t dq_free() const { return bar(9); }
   __device__ __forceinline__ uint32_t done() const { return bar(10); }
+  // the dQ drain no longer stages in the dS buffer (its reductions have read it)
+  __device__ __forceinline__ uint32_t ds_free() const { return bar(11); }
   __device__ __forceinline__ uint32_t* tmem_slot() const {
     return reinterpret_cast<uint32_t*>(base + Cfg<D>::kOffMisc);
   }
@@ -327,6 +329,11 @@ __device__ __forceinline__ bool softmax_grad_role(const Smem<D>& sm, uint32_t tm
     const int q_base = w.tile_of(it) * kBlockQ + c * 64;  // first query of this warp's columns
     // masking: key tail, or (causal) a key past some query of the block
     const bool masked = !key_in || (CAUSAL && w.j * kBlockK + q4 * 32 + 31 > q_base);
+    // the dS buffer doubled as the previous dQ tile's staging
+    if (it > 0 && !warp_wait(sm.ds_free(), (it - 1) & 1, prm.timeout_ns)) {
+      ok = false;
+      break;
+    }
     const float* l2 = sm.lse2(s) + c * 64;
     const float* dd = sm.dsum(s) + c * 64;
 #pragma unroll
@@ -373,40 +380,66 @@ __device__ __forceinline__ bool softmax_grad_role(const Smem<D>& sm, uint32_t tm
   return ok;
 }
 
-// Warps 8-11: dQ tile (queries on the TMEM lanes) -> fp32 accumulator.
+// Warps 8-11: dQ tile (queries on the TMEM lanes) -> fp32 accumulator by TMA
+// reduce-add.  Each warp stages its 32 rows, 64 columns at a time, as two
+// 32-column x 32-row boxes (128-byte swizzle) in its 8 KiB of the dS buffer,
+// which the dQ GEMM has finished reading and the next dS is not written until
+// ds_free.  TMEM is released (dq_free) as soon as the last columns are in
+// registers, so the next S^T GEMM overlaps the reductions.
 template <int D>
-__device__ __forceinline__ bool dq_drain_role(const Smem<D>& sm, uint32_t tmem, const BwdParams& prm,
-                                              const Work& w) {
+__device__ __forceinline__ bool dq_drain_role(const Smem<D>& sm, uint32_t tmem, const CUtensorMap* tm_dq,
+                                              const BwdParams& prm, const Work& w) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int q4 = warp & 3;
   const uint32_t tQ = tmem + (static_cast<uint32_t>(q4 * 32) << 16);
+  uint8_t* stage = sm.base + Cfg<D>::kOffDS + q4 * 8192;
+  const uint32_t stage_s = smem_u32(stage);
+  constexpr int kHalves = D / 64;
   bool ok = true;
   for (int it = 0; it < w.n_it; ++it) {
     ok = warp_wait(sm.dq_full(), it & 1, prm.timeout_ns);
     if (!ok) break;
     tc_fence_after();
     const int bh = w.b * prm.H + w.hkv * prm.group + w.head_of(it);
-    const int q = w.tile_of(it) * kBlockQ + q4 * 32 + lane;
-    float* dst = prm.dq_acc + (static_cast<size_t>(bh) * prm.Nq + q) * D;
+    const int row0 = w.tile_of(it) * kBlockQ + q4 * 32;
 #pragma unroll
-    for (int cc = 0; cc < D / 32; ++cc) {
-      uint32_t v[32];
-      tmem_ld32(tQ + 32 * cc, v);
+    for (int hf = 0; hf < kHalves; ++hf) {
+      uint32_t v0[32], v1[32];
+      tmem_ld32(tQ + 64 * hf, v0);
+      tmem_ld32(tQ + 64 * hf + 32, v1);
       tmem_ld_wait();
-      reg_fence32(v);
-      if (q < prm.Nq) {
+      reg_fence32(v0);
+      reg_fence32(v1);
+      if (hf == kHalves - 1) {
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(sm.dq_free());
+      }
+      if (hf > 0) {  // the previous half's reductions must have read the staging
+        if (lane == 0) bulk_wait_group_read0();
+        __syncwarp();
+      }
+      uint8_t* row = stage + lane * 128;
 #pragma unroll
-        for (int i = 0; i < 8; ++i)
-          asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(dst + 32 * cc + 4 * i),
-                       "f"(__uint_as_float(v[4 * i])), "f"(__uint_as_float(v[4 * i + 1])),
-                       "f"(__uint_as_float(v[4 * i + 2])), "f"(__uint_as_float(v[4 * i + 3]))
-                       : "memory");
+      for (int c = 0; c < 8; ++c) {
+        *reinterpret_cast<uint4*>(row + ((c ^ (lane & 7)) * 16)) =
+            make_uint4(v0[4 * c], v0[4 * c + 1], v0[4 * c + 2], v0[4 * c + 3]);
+        *reinterpret_cast<uint4*>(row + 4096 + ((c ^ (lane & 7)) * 16)) =
+            make_uint4(v1[4 * c], v1[4 * c + 1], v1[4 * c + 2], v1[4 * c + 3]);
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) {
+        tma_reduce_add_3d(tm_dq, stage_s, 64 * hf, row0, bh);
+        tma_reduce_add_3d(tm_dq, stage_s + 4096, 64 * hf + 32, row0, bh);
+        bulk_commit_group();
       }
     }
-    tc_fence_before();
+    if (lane == 0) bulk_wait_group_read0();
     __syncwarp();
-    if (lane == 0) mbar_arrive(sm.dq_free());
+    if (lane == 0) mbar_arrive(sm.ds_free());
   }
+  if (lane == 0) bulk_wait_group0();  // every reduction complete before the CTA exits
   return ok;
 }
 
@@ -468,7 +501,7 @@ __global__ void __launch_bounds__(kNumThreads, 1)
 attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                 const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
                 const __grid_constant__ CUtensorMap tm_dk, const __grid_constant__ CUtensorMap tm_dv,
-                const __grid_constant__ BwdParams prm) {
+                const __grid_constant__ CUtensorMap tm_dq, const __grid_constant__ BwdParams prm) {
   using C = Cfg<D>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   // The 128-byte swizzled tiles need 1 KiB-aligned shared memory; there is no
@@ -500,7 +533,7 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       uint32_t count = 1;
       if (b == sm.q_full(0) || b == sm.q_full(1)) count = 32;  // every producer lane
       if (b == sm.p_ready()) count = 8;
-      if (b == sm.dq_free()) count = 4;
+      if (b == sm.dq_free() || b == sm.ds_free()) count = 4;
       mbar_init(b, count);
     }
     fence_barrier_init();
@@ -526,7 +559,7 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     ok = epilogue<D>(sm, tmem, &tm_dk, &tm_dv, prm, w, ok);
     if (!ok && lane == 0) atomicOr(&g_status_bwd, kStatusTimeout);
   } else if (warp < kWarpLoad) {
-    const bool ok = dq_drain_role<D>(sm, tmem, prm, w);
+    const bool ok = dq_drain_role<D>(sm, tmem, &tm_dq, prm, w);
     if (!ok && lane == 0) atomicOr(&g_status_bwd, kStatusTimeout);
   } else if (warp == kWarpLoad) {
     producer_role<D>(sm, &tm_q, &tm_k, &tm_v, &tm_do, prm, w, lane);
@@ -588,7 +621,7 @@ int launch_main(const CUtensorMap* maps, const BwdParams& prm, int grid, cudaStr
   });
   if (err[dev] != cudaSuccess) return cuda_fail(err[dev], "cudaFuncSetAttribute");
   kern<<<grid, kNumThreads, Cfg<D>::kSmemBytes, stream>>>(maps[0], maps[1], maps[2], maps[3], maps[4],
-                                                          maps[5], prm);
+                                                          maps[5], maps[6], prm);
   e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "attn_bwd_kernel launch");
   return ATTN_OK;
@@ -653,7 +686,7 @@ int bwd_impl(const void* q, const void* k, const void* v, const void* o, const v
     return ATTN_OK;
   }
 
-  CUtensorMap maps[6];
+  CUtensorMap maps[7];
   const int bh = static_cast<int>(BH), bhkv = static_cast<int>(BHkv);
   if (!make_tmap_bf16_3d(&maps[0], q, bh, Nq, d, kBlockQ, &t_last_error) ||
       !make_tmap_bf16_3d(&maps[1], k, bhkv, Nk, d, kBlockK, &t_last_error) ||
@@ -666,6 +699,7 @@ int bwd_impl(const void* q, const void* k, const void* v, const void* o, const v
   float* dsum = static_cast<float*>(workspace);
   float* dq_acc = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) +
                                            align256(static_cast<size_t>(BH) * Nq * 4));
+  if (!make_tmap_f32_3d(&maps[6], dq_acc, bh, Nq, d, 32, &t_last_error)) return ATTN_ERR_CUDA;
   const size_t rows = static_cast<size_t>(BH) * Nq;
   e = cudaMemsetAsync(dq_acc, 0, rows * d * 4, stream);
   if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync");

@@ -86,6 +86,12 @@ constexpr uint32_t kTmemCols = 512;
 constexpr uint64_t kWaitTimeoutNs = 2000000000ull;  // 2 s per pipeline wait
 constexpr float kDefaultThreshold = 8.0f;           // powers of two
 constexpr int kDefaultPoly16 = 4;                   // exp2 columns (of 16) on the FMA pipe
+// E4M3 P: the exponent is raised by kP8Offset powers of two and the rescale
+// threshold lowered to kP8Tau, so P stays within [0, 2^(kP8Tau + kP8Offset)] =
+// [0, 256] (E4M3 saturates at 448) while small weights keep 4 more binades
+// above E4M3's smallest subnormal.  Both cancel in O / l; LSE subtracts the offset.
+constexpr float kP8Offset = 4.0f;
+constexpr float kP8Tau = 4.0f;
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kLog2e = 1.4426950408889634f;
 
@@ -98,16 +104,26 @@ constexpr int kUnbounded = 1 << 30;
 // Per-device status word (each device holds its own copy of module globals).
 __device__ unsigned int g_status;
 
-template <int D>
+// F8: Q, K, V (and P) in E4M3 bytes instead of BF16.
+template <int D, bool F8>
 struct Cfg {
   static_assert(D == 64 || D == 128, "head dim");
-  static constexpr int kBoxes = D / 64;             // 128-byte swizzle boxes across d
-  static constexpr int kBoxBytes = kBlockM * 128;   // 128 rows x 64 bf16
+  static_assert(!F8 || D == 128, "E4M3 inputs: d = 128 (one 128-byte row)");
+  static constexpr int kElem = F8 ? 1 : 2;          // bytes per element
+  static constexpr int kBoxCols = 128 / kElem;      // elements per 128-byte swizzle row
+  static constexpr int kBoxes = D / kBoxCols;       // 128-byte swizzle boxes across d
+  static constexpr int kBoxBytes = kBlockM * 128;   // 128 rows x 128 bytes
   static constexpr int kTileBytes = kBoxes * kBoxBytes;
-  static constexpr int kStages = D == 128 ? 4 : 8;  // K/V ring depth
+  static constexpr int kKStep = 32 / kElem;         // MMA K per instruction (32 bytes)
+  static constexpr int kStages = F8 ? 6 : (D == 64 ? 8 : 4);  // K/V ring depth
   static constexpr int kOffQ = 0;
   static constexpr int kOffKV = 2 * kTileBytes;
-  static constexpr int kOffBar = kOffKV + kStages * kTileBytes;
+  // BF16 O of one tile (128 rows x d) is staged for its TMA store in that
+  // tile's Q buffer when it fits (BF16 inputs: same size); E4M3 Q tiles are
+  // half as large, so O gets its own area after the K/V ring.
+  static constexpr int kOTileBytes = kBlockM * D * 2;
+  static constexpr int kOffO = F8 ? kOffKV + kStages * kTileBytes : kOffQ;
+  static constexpr int kOffBar = F8 ? kOffO + 2 * kOTileBytes : kOffKV + kStages * kTileBytes;
   static constexpr int kNumBars = 2 + 2 * kStages + 2 + 4 + 2 + 1;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
   // row-max / row-sum exchange between the two key halves of a row:
@@ -117,6 +133,7 @@ struct Cfg {
   static constexpr int kOffSeq = kOffXch + kXchBytes;  // this CTA's SeqView
   static constexpr int kSeqBytes = 64;
   static constexpr int kSmemBytes = kOffSeq + kSeqBytes + 1024;  // + slack for 1 KiB alignment
+  static_assert(kSmemBytes <= 232448, "shared memory per CTA");
   static constexpr uint32_t kTmemO = 256;
 };
 
@@ -133,8 +150,9 @@ struct FwdParams {
   int wl, wr;        // key band: i - wl <= j <= i + wr (kUnbounded: no bound)
   int grouped;       // causal band: heads in L2-sized groups, heaviest blocks first
   int hgroup;        // heads scheduled together (their K/V fit in L2)
-  float scale_log2;  // scale * log2(e)
+  float scale_log2;  // scale * log2(e) (E4M3: times the Q and K scale factors)
   float tau;         // rescale threshold, powers of two
+  float o_scale;     // multiplies O / l (E4M3: the V scale factor; else 1)
 };
 
 // Where one CTA's sequence lives: lengths, first packed row (packed layout),
@@ -165,34 +183,34 @@ __device__ __forceinline__ float ex2_split(float x, int col) {
 // ---------------------------------------------------------------------------
 // Shared-memory / barrier map of one CTA
 // ---------------------------------------------------------------------------
-template <int D>
+template <int D, bool F8>
 struct Smem {
   uint8_t* base;
   uint32_t sbase;
-  __device__ __forceinline__ uint32_t q(int t) const { return sbase + Cfg<D>::kOffQ + t * Cfg<D>::kTileBytes; }
-  __device__ __forceinline__ uint32_t kv(int s) const { return sbase + Cfg<D>::kOffKV + s * Cfg<D>::kTileBytes; }
-  __device__ __forceinline__ uint32_t bar(int i) const { return sbase + Cfg<D>::kOffBar + 8 * i; }
+  __device__ __forceinline__ uint32_t q(int t) const { return sbase + Cfg<D, F8>::kOffQ + t * Cfg<D, F8>::kTileBytes; }
+  __device__ __forceinline__ uint32_t kv(int s) const { return sbase + Cfg<D, F8>::kOffKV + s * Cfg<D, F8>::kTileBytes; }
+  __device__ __forceinline__ uint32_t bar(int i) const { return sbase + Cfg<D, F8>::kOffBar + 8 * i; }
   __device__ __forceinline__ uint32_t q_full(int t) const { return bar(t); }
   __device__ __forceinline__ uint32_t kv_full(int s) const { return bar(2 + s); }
-  __device__ __forceinline__ uint32_t kv_empty(int s) const { return bar(2 + Cfg<D>::kStages + s); }
-  __device__ __forceinline__ uint32_t s_full(int t) const { return bar(2 + 2 * Cfg<D>::kStages + t); }
+  __device__ __forceinline__ uint32_t kv_empty(int s) const { return bar(2 + Cfg<D, F8>::kStages + s); }
+  __device__ __forceinline__ uint32_t s_full(int t) const { return bar(2 + 2 * Cfg<D, F8>::kStages + t); }
   // chunk k of P_t (keys [32k, 32k+32) and [64+32k, 96+32k)) written to TMEM by
   // all 8 warps of the tile (chunk 0 also marks O_t as rescaled)
   __device__ __forceinline__ uint32_t p_full(int t, int k) const {
-    return bar(4 + 2 * Cfg<D>::kStages + 2 * t + k);
+    return bar(4 + 2 * Cfg<D, F8>::kStages + 2 * t + k);
   }
-  __device__ __forceinline__ uint32_t o_full(int t) const { return bar(8 + 2 * Cfg<D>::kStages + t); }
-  __device__ __forceinline__ uint32_t mma_done() const { return bar(10 + 2 * Cfg<D>::kStages); }
+  __device__ __forceinline__ uint32_t o_full(int t) const { return bar(8 + 2 * Cfg<D, F8>::kStages + t); }
+  __device__ __forceinline__ uint32_t mma_done() const { return bar(10 + 2 * Cfg<D, F8>::kStages); }
   __device__ __forceinline__ float* xch(int t, int h, int par) const {
-    return reinterpret_cast<float*>(base + Cfg<D>::kOffXch) + ((t * 2 + h) * 2 + par) * kBlockM;
+    return reinterpret_cast<float*>(base + Cfg<D, F8>::kOffXch) + ((t * 2 + h) * 2 + par) * kBlockM;
   }
   __device__ __forceinline__ uint32_t* tmem_slot() const {
-    return reinterpret_cast<uint32_t*>(base + Cfg<D>::kOffMisc);
+    return reinterpret_cast<uint32_t*>(base + Cfg<D, F8>::kOffMisc);
   }
   // kept in shared memory rather than registers: the softmax warps need most of
   // it only in the epilogue
   __device__ __forceinline__ SeqView* seq() const {
-    return reinterpret_cast<SeqView*>(base + Cfg<D>::kOffSeq);
+    return reinterpret_cast<SeqView*>(base + Cfg<D, F8>::kOffSeq);
   }
 };
 
@@ -206,17 +224,17 @@ __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, uint64_
 // ---------------------------------------------------------------------------
 // Producer: one thread, TMA loads of Q0, K0, Q1, V0, K1, V1, ...
 // ---------------------------------------------------------------------------
-template <int D>
-__device__ __forceinline__ void producer_role(const Smem<D>& sm, const CUtensorMap* tm_q,
+template <int D, bool F8>
+__device__ __forceinline__ void producer_role(const Smem<D, F8>& sm, const CUtensorMap* tm_q,
                                               const CUtensorMap* tm_k, const CUtensorMap* tm_v,
                                               const SeqView& sv, int qb, uint64_t timeout) {
-  using C = Cfg<D>;
+  using C = Cfg<D, F8>;
   uint32_t it = 0;
   auto load_q = [&](int t) {
     mbar_arrive_expect_tx(sm.q_full(t), C::kTileBytes);
 #pragma unroll
     for (int b = 0; b < C::kBoxes; ++b)
-      tma_load_rows(sm.q(t) + b * C::kBoxBytes, tm_q, b * 64, sv.q0 + qb * kRowsPerCta + t * kBlockM,
+      tma_load_rows(sm.q(t) + b * C::kBoxBytes, tm_q, b * C::kBoxCols, sv.q0 + qb * kRowsPerCta + t * kBlockM,
                     sv.head_q, sv.packed, sm.q_full(t));
   };
   auto load_kv = [&](const CUtensorMap* tm, int j) -> bool {
@@ -226,7 +244,7 @@ __device__ __forceinline__ void producer_role(const Smem<D>& sm, const CUtensorM
     mbar_arrive_expect_tx(sm.kv_full(slot), C::kTileBytes);
 #pragma unroll
     for (int b = 0; b < C::kBoxes; ++b)
-      tma_load_rows(sm.kv(slot) + b * C::kBoxBytes, tm, b * 64, sv.k0 + j * kBlockN, sv.head_kv,
+      tma_load_rows(sm.kv(slot) + b * C::kBoxBytes, tm, b * C::kBoxCols, sv.k0 + j * kBlockN, sv.head_kv,
                     sv.packed, sm.kv_full(slot));
     ++it;
     return true;
@@ -250,31 +268,45 @@ __device__ __forceinline__ void producer_role(const Smem<D>& sm, const CUtensorM
 // ---------------------------------------------------------------------------
 // MMA issuer: one thread.
 // ---------------------------------------------------------------------------
-template <int D, int KK>
+template <int D, bool F8, int KK>
 struct MmaUnroll {
-  // S = Q K^T, K steps KK .. D/16-1: 32 bytes along the 128-byte row, a new
-  // 64-column box every 4 steps.
+  // S = Q K^T, K steps KK .. : 32 bytes along the 128-byte row, a new box
+  // every 4 steps (BF16: 16 elements per step; E4M3: 32).
   __device__ __forceinline__ static void s(uint32_t d, uint32_t a_lo, uint32_t a_hi, uint32_t b_lo,
                                            uint32_t b_hi, uint32_t idesc) {
-    if constexpr (KK < D / 16) {
-      constexpr uint32_t off = ((KK >> 2) * Cfg<D>::kBoxBytes + (KK & 3) * 32) >> 4;
-      mma_ss_imm<off, off, KK == 0 ? 0u : 1u>(d, a_lo, a_hi, b_lo, b_hi, idesc);
-      MmaUnroll<D, KK + 1>::s(d, a_lo, a_hi, b_lo, b_hi, idesc);
+    if constexpr (KK < D / Cfg<D, F8>::kKStep) {
+      constexpr uint32_t off = ((KK >> 2) * Cfg<D, F8>::kBoxBytes + (KK & 3) * 32) >> 4;
+      if constexpr (F8)
+        mma_ss_imm_f8<off, off, KK == 0 ? 0u : 1u>(d, a_lo, a_hi, b_lo, b_hi, idesc);
+      else
+        mma_ss_imm<off, off, KK == 0 ? 0u : 1u>(d, a_lo, a_hi, b_lo, b_hi, idesc);
+      MmaUnroll<D, F8, KK + 1>::s(d, a_lo, a_hi, b_lo, b_hi, idesc);
     }
   }
-  // O += P V for P chunk CH: K steps {2CH, 2CH+1} (keys [32CH, 32CH+32)) and
-  // {4+2CH, 5+2CH} (keys [64+32CH, 96+32CH)).  P of keys [64h, 64h+64) sits in
-  // TMEM columns [64h, 64h+32) (two bf16 per column); V rows of 16 keys =
-  // 2048 bytes.  KK counts 0..3 within the chunk.
+  // O += P V for P chunk CH.  BF16: K steps {2CH, 2CH+1} (keys [32CH, 32CH+32))
+  // and {4+2CH, 5+2CH} (keys [64+32CH, 96+32CH)); P of keys [64h, 64h+64) sits
+  // in TMEM columns [64h, 64h+32) (two per column); V rows of 16 keys = 2048
+  // bytes.  E4M3: K steps CH (keys [32CH, 32CH+32)) and 2+CH (keys
+  // [64+32CH, 96+32CH)); P of keys [64h, 64h+64) in columns [64h, 64h+16)
+  // (four per column); V rows of 32 keys = 4096 bytes.  KK counts the steps
+  // of the chunk.
   template <int CH>
   __device__ __forceinline__ static void o(uint32_t d, uint32_t a_tmem, uint32_t b_lo, uint32_t b_hi,
                                            uint32_t idesc, uint32_t acc) {
-    if constexpr (KK < 4) {
+    if constexpr (F8) {
+      if constexpr (KK < 2) {
+        constexpr int step = 2 * KK + CH;  // K step among 0..3, 32 keys each
+        constexpr uint32_t a_off = (step >> 1) * 64 + (step & 1) * 8;
+        constexpr uint32_t b_off = (step * 4096) >> 4;
+        mma_ts_imm_f8<a_off, b_off>(d, a_tmem, b_lo, b_hi, idesc, (CH == 0 && KK == 0) ? acc : 1u);
+        MmaUnroll<D, F8, KK + 1>::template o<CH>(d, a_tmem, b_lo, b_hi, idesc, acc);
+      }
+    } else if constexpr (KK < 4) {
       constexpr int step = (KK >> 1) * 4 + 2 * CH + (KK & 1);  // K step among 0..7
       constexpr uint32_t a_off = (step >> 2) * 64 + (step & 3) * 8;
       constexpr uint32_t b_off = (step * 2048) >> 4;
       mma_ts_imm<a_off, b_off>(d, a_tmem, b_lo, b_hi, idesc, (CH == 0 && KK == 0) ? acc : 1u);
-      MmaUnroll<D, KK + 1>::template o<CH>(d, a_tmem, b_lo, b_hi, idesc, acc);
+      MmaUnroll<D, F8, KK + 1>::template o<CH>(d, a_tmem, b_lo, b_hi, idesc, acc);
     }
   }
 };
@@ -284,12 +316,14 @@ struct MmaUnroll {
 // (normally long resident), so the only wait between a tile's P becoming
 // ready and its O += P V_{j-1}; S = Q K_j^T block is the P barrier itself.
 // ---------------------------------------------------------------------------
-template <int D>
-__device__ __forceinline__ void mma_role(const Smem<D>& sm, uint32_t tmem, int n_kv,
+template <int D, bool F8>
+__device__ __forceinline__ void mma_role(const Smem<D, F8>& sm, uint32_t tmem, int n_kv,
                                          uint64_t timeout) {
-  using C = Cfg<D>;
-  constexpr uint32_t idesc_s = idesc_bf16_f32(kBlockM, kBlockN, false, false);
-  constexpr uint32_t idesc_o = idesc_bf16_f32(kBlockM, D, false, true);
+  using C = Cfg<D, F8>;
+  constexpr uint32_t idesc_s = F8 ? idesc_e4m3_f32(kBlockM, kBlockN, false, false)
+                                  : idesc_bf16_f32(kBlockM, kBlockN, false, false);
+  constexpr uint32_t idesc_o = F8 ? idesc_e4m3_f32(kBlockM, D, false, true)
+                                  : idesc_bf16_f32(kBlockM, D, false, true);
   uint32_t it = 0;  // position in the K0, V0, K1, V1, ... ring order
 
   auto wait_kv = [&](uint32_t& slot) -> bool {
@@ -307,7 +341,7 @@ __device__ __forceinline__ void mma_role(const Smem<D>& sm, uint32_t tmem, int n
   const uint32_t v_lo = static_cast<uint32_t>(dv), v_hi = static_cast<uint32_t>(dv >> 32);
   constexpr uint32_t kTileStep = C::kTileBytes >> 4;
   auto mma_s = [&](int t, uint32_t slot) {
-    MmaUnroll<D, 0>::s(tmem + t * kBlockM, q_lo + t * kTileStep, q_hi, k_lo + slot * kTileStep,
+    MmaUnroll<D, F8, 0>::s(tmem + t * kBlockM, q_lo + t * kTileStep, q_hi, k_lo + slot * kTileStep,
                        k_hi, idesc_s);
   };
   // O_t += P_t V in two chunks, each issued as soon as the softmax warps have
@@ -317,10 +351,10 @@ __device__ __forceinline__ void mma_role(const Smem<D>& sm, uint32_t tmem, int n
     const uint32_t b_lo = v_lo + slot * kTileStep;
     if (!mbar_wait(sm.p_full(t, 0), par, timeout)) return false;
     tc_fence_after();
-    MmaUnroll<D, 0>::template o<0>(d, a, b_lo, v_hi, idesc_o, acc ? 1u : 0u);
+    MmaUnroll<D, F8, 0>::template o<0>(d, a, b_lo, v_hi, idesc_o, acc ? 1u : 0u);
     if (!mbar_wait(sm.p_full(t, 1), par, timeout)) return false;
     tc_fence_after();
-    MmaUnroll<D, 0>::template o<1>(d, a, b_lo, v_hi, idesc_o, 1u);
+    MmaUnroll<D, F8, 0>::template o<1>(d, a, b_lo, v_hi, idesc_o, 1u);
     return true;
   };
 
@@ -384,11 +418,11 @@ __device__ __forceinline__ void pair_sync(int t, int q) {
   asm volatile("bar.sync %0, 64;" ::"r"(1 + t * 4 + q) : "memory");
 }
 
-template <int D, bool MASK, int POLY16>
-__device__ __forceinline__ void softmax_role(const Smem<D>& sm, uint32_t tmem,
+template <int D, bool MASK, int POLY16, bool F8>
+__device__ __forceinline__ void softmax_role(const Smem<D, F8>& sm, uint32_t tmem,
                                              const CUtensorMap* tm_o, const FwdParams& prm,
                                              const SeqView& sv, int qb) {
-  using C = Cfg<D>;
+  using C = Cfg<D, F8>;
   constexpr int kCols = kBlockN / 2;  // key columns per warp
   constexpr int kOCols = D / 2;       // output columns per warp
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -501,7 +535,8 @@ __device__ __forceinline__ void softmax_role(const Smem<D>& sm, uint32_t tmem,
     // Chunk k's P lands in columns [16k, 16k+16), which chunk k has consumed,
     // and is announced on its own barrier so its O += P V can start while the
     // next chunk is being exponentiated.
-    const float neg_m = (m_run == -INFINITY) ? 0.0f : -m_run;
+    constexpr float kOff = F8 ? kP8Offset : 0.0f;
+    const float neg_m = (m_run == -INFINITY) ? 0.0f : kOff - m_run;
     const float2 sl2 = make_float2(sl, sl), nm2 = make_float2(neg_m, neg_m);
     float2 sum2[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
                       make_float2(0.f, 0.f)};
@@ -510,6 +545,7 @@ __device__ __forceinline__ void softmax_role(const Smem<D>& sm, uint32_t tmem,
       float x[32];
       load_scores(k, x);
       uint32_t p[16];
+      float2 prev = make_float2(0.f, 0.f);
 #pragma unroll
       for (int i = 0; i < 16; ++i) {
         const int c = 2 * i;
@@ -522,9 +558,18 @@ __device__ __forceinline__ void softmax_role(const Smem<D>& sm, uint32_t tmem,
           e.y = ex2_mufu(u.y);
         }
         sum2[i & 3] = fadd2(sum2[i & 3], e);
-        p[i] = pack_bf16x2(e.x, e.y);
+        if constexpr (F8) {
+          // four E4M3 per TMEM column, key 4w in the low byte of word w
+          if (i & 1) p[i >> 1] = pack_e4m3x4(prev.x, prev.y, e.x, e.y);
+          prev = e;
+        } else {
+          p[i] = pack_bf16x2(e.x, e.y);
+        }
       }
-      tmem_st16(tS + 16 * k, p);
+      if constexpr (F8)
+        tmem_st8(tS + 8 * k, p);
+      else
+        tmem_st16(tS + 16 * k, p);
       tmem_st_wait();
       tc_fence_before();
       __syncwarp();
@@ -542,15 +587,16 @@ __device__ __forceinline__ void softmax_role(const Smem<D>& sm, uint32_t tmem,
   pair_sync(t, q4);
   const float lother = sm.xch(t, h ^ 1, 0)[r];
   const bool ok3 = ok2 && !isnan(lother);
-  uint8_t* sOt = sm.base + C::kOffQ + t * C::kTileBytes;
+  uint8_t* sOt = sm.base + C::kOffO + t * C::kOTileBytes;
   const float l_tot = l_run + lother;
   const bool ragged = sv.packed && rw0 + 32 > sv.Nq;
   if (ok3) {
     tc_fence_after();
-    // O / l -> BF16 -> this tile's Q buffer (its last reader, the final S MMA,
-    // finished before the last O MMA) in the 128-byte swizzled layout the O
-    // tensor map expects.  Warp h writes output columns [h*d/2, (h+1)*d/2).
-    const float inv_l = l_tot > 0.0f ? 1.0f / l_tot : 0.0f;
+    // O / l -> BF16 -> the tile's O staging (BF16 inputs: the tile's Q buffer,
+    // whose last reader, the final S MMA, finished before the last O MMA) in
+    // the 128-byte swizzled layout the O tensor map expects.  Warp h writes
+    // output columns [h*d/2, (h+1)*d/2).
+    const float inv_l = l_tot > 0.0f ? prm.o_scale / l_tot : 0.0f;
 #pragma unroll
     for (int cc = 0; cc < kOCols / 32; ++cc) {
       uint32_t o[32];
@@ -596,7 +642,8 @@ __device__ __forceinline__ void softmax_role(const Smem<D>& sm, uint32_t tmem,
     bulk_wait_group_read0();
   }
   if (ok3 && h == 0 && sv.lse_row0 != nullptr && row < sv.Nq) {
-    const float m_use = (m_run == -INFINITY) ? 0.0f : m_run;
+    // P carried 2^kOff: LSE = ln 2 * (m - kOff + log2 l)
+    const float m_use = (m_run == -INFINITY) ? 0.0f : m_run - (F8 ? kP8Offset : 0.0f);
     sv.lse_row0[row] = (m_use + log2f(l_tot)) * kLn2;
   }
   if (!ok3 && lane == 0) atomicOr(&g_status, kStatusTimeout);
@@ -605,14 +652,14 @@ __device__ __forceinline__ void softmax_role(const Smem<D>& sm, uint32_t tmem,
 // ---------------------------------------------------------------------------
 // The kernel.  Grid: one CTA per (b*h, 256-row query block).
 // ---------------------------------------------------------------------------
-template <int D, bool MASK, int POLY16>
+template <int D, bool MASK, int POLY16, bool F8>
 __global__ void __launch_bounds__(kNumThreads, 1)
 attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                 const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
                 const __grid_constant__ FwdParams prm) {
-  using C = Cfg<D>;
+  using C = Cfg<D, F8>;
   extern __shared__ uint8_t smem_raw[];
-  Smem<D> sm;
+  Smem<D, F8> sm;
   {
     const uint32_t raw = smem_u32(smem_raw);
     const uint32_t pad = (1024u - (raw & 1023u)) & 1023u;
@@ -642,7 +689,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   // same batch entry (group = 1: one key/value head per query head)
   const int hq = bh % prm.H, seq = bh / prm.H;
   SeqView sv;
-  static_assert(sizeof(SeqView) <= Cfg<D>::kSeqBytes, "SeqView slot");
+  static_assert(sizeof(SeqView) <= Cfg<D, F8>::kSeqBytes, "SeqView slot");
   sv.packed = prm.cu_q != nullptr;
   if (sv.packed) {
     // packed variable-length batch: sequence `seq` owns rows cu_q[seq] ..
@@ -730,15 +777,15 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     // warpgroup 2: TMA producer (warp 8), MMA issuer (warp 9), two idle warps
     setmaxnreg_dec<kProducerRegs>();
     if (warp == kWarpLoad) {
-      if (lane == 0) producer_role<D>(sm, &tm_q, &tm_k, &tm_v, seqv, qb, prm.timeout_ns);
+      if (lane == 0) producer_role<D, F8>(sm, &tm_q, &tm_k, &tm_v, seqv, qb, prm.timeout_ns);
       __syncwarp();
     } else if (warp == kWarpMma) {
-      if (lane == 0) mma_role<D>(sm, tmem, seqv.n_kv, prm.timeout_ns);
+      if (lane == 0) mma_role<D, F8>(sm, tmem, seqv.n_kv, prm.timeout_ns);
       __syncwarp();
     }
   } else {
     setmaxnreg_inc<kSoftmaxRegs>();
-    softmax_role<D, MASK, POLY16>(sm, tmem, &tm_o, prm, seqv, qb);
+    softmax_role<D, MASK, POLY16, F8>(sm, tmem, &tm_o, prm, seqv, qb);
   }
 
   tc_fence_before();
@@ -772,10 +819,10 @@ __global__ void selftest_timeout_kernel(uint64_t timeout_ns) {
 // ---------------------------------------------------------------------------
 constexpr int kMaxDevices = kMaxDeviceCount;
 
-template <int D, bool MASK, int POLY16>
+template <int D, bool MASK, int POLY16, bool F8 = false>
 int launch_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                const CUtensorMap& to, const FwdParams& prm, cudaStream_t stream) {
-  auto kern = attn_fwd_kernel<D, MASK, POLY16>;
+  auto kern = attn_fwd_kernel<D, MASK, POLY16, F8>;
   static std::once_flag attr_once[kMaxDevices];
   static cudaError_t attr_err[kMaxDevices];
   int dev = 0;
@@ -783,11 +830,11 @@ int launch_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& 
   if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
   std::call_once(attr_once[dev], [&] {
     attr_err[dev] = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         Cfg<D>::kSmemBytes);
+                                         Cfg<D, F8>::kSmemBytes);
   });
   if (attr_err[dev] != cudaSuccess) return cuda_fail(attr_err[dev], "cudaFuncSetAttribute");
   const unsigned grid = static_cast<unsigned>(prm.BH) * static_cast<unsigned>(prm.n_qblocks);
-  kern<<<grid, kNumThreads, Cfg<D>::kSmemBytes, stream>>>(tq, tk, tv, to, prm);
+  kern<<<grid, kNumThreads, Cfg<D, F8>::kSmemBytes, stream>>>(tq, tk, tv, to, prm);
   e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "attn_fwd_kernel launch");
   return ATTN_OK;
@@ -914,6 +961,7 @@ int fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, i
   prm.n_qblocks = static_cast<int>(n_qblocks);
   prm.scale_log2 = scale * kLog2e;
   prm.tau = tau;
+  prm.o_scale = 1.0f;
   return launch_any(d, exp_mode, tq, tk, tv, to, prm, stream);
 }
 
@@ -977,7 +1025,73 @@ int varlen_impl(const void* q, const void* k, const void* v, void* o, float* lse
   prm.n_qblocks = static_cast<int>(n_qblocks);
   prm.scale_log2 = scale * kLog2e;
   prm.tau = kDefaultThreshold;
+  prm.o_scale = 1.0f;
   return launch_any(d, 1, tq, tk, tv, to, prm, stream);
+}
+
+int fp8_impl(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int Hkv,
+             int Nq, int Nk, int d, float scale, float q_descale, float k_descale, float v_descale,
+             int causal, cudaStream_t stream) {
+  if (B < 0 || H < 0 || Hkv < 0 || Nq < 0 || Nk < 0) return ATTN_ERR_INVALID_ARG;
+  if (H > 0 && (Hkv == 0 || H % Hkv != 0)) return ATTN_ERR_INVALID_ARG;
+  if (!std::isfinite(scale) || !std::isfinite(q_descale) || !std::isfinite(k_descale) ||
+      !std::isfinite(v_descale))
+    return ATTN_ERR_INVALID_ARG;
+  const float s_eff = scale * q_descale * k_descale;
+  if (!std::isfinite(s_eff)) return ATTN_ERR_INVALID_ARG;
+  if (causal != 0 && causal != 1) return ATTN_ERR_INVALID_ARG;
+  if (d != 128) return ATTN_ERR_UNSUPPORTED;
+  if (causal && Nq != Nk) return ATTN_ERR_UNSUPPORTED;
+  const long long BH = static_cast<long long>(B) * H;
+  if (BH == 0 || Nq == 0) return ATTN_OK;
+  if (BH > 0x7fffffffLL) return ATTN_ERR_INVALID_ARG;
+  if (!o || (Nk > 0 && (!q || !k || !v))) return ATTN_ERR_INVALID_ARG;
+  if (misaligned(q, 16) || misaligned(k, 16) || misaligned(v, 16) || misaligned(o, 16) ||
+      misaligned(lse, 4))
+    return ATTN_ERR_INVALID_ARG;
+  const long long BHkv = static_cast<long long>(B) * Hkv;
+  const size_t q_bytes = static_cast<size_t>(BH) * Nq * d;
+  const size_t kv_bytes = static_cast<size_t>(BHkv) * Nk * d;
+  const size_t o_bytes = static_cast<size_t>(BH) * Nq * d * 2;
+  const size_t lse_bytes = lse ? static_cast<size_t>(BH) * Nq * 4 : 0;
+  if (ranges_overlap(o, o_bytes, q, q_bytes) || ranges_overlap(o, o_bytes, k, kv_bytes) ||
+      ranges_overlap(o, o_bytes, v, kv_bytes) || ranges_overlap(lse, lse_bytes, q, q_bytes) ||
+      ranges_overlap(lse, lse_bytes, k, kv_bytes) || ranges_overlap(lse, lse_bytes, v, kv_bytes) ||
+      ranges_overlap(lse, lse_bytes, o, o_bytes))
+    return ATTN_ERR_INVALID_ARG;
+  const long long n_qblocks = (Nq + kRowsPerCta - 1) / kRowsPerCta;
+  if (n_qblocks * BH > 0x7fffffffLL) return ATTN_ERR_INVALID_ARG;
+  int rc = check_device();
+  if (rc != ATTN_OK) return rc;
+  if (Nk == 0) return fill_empty(o, o_bytes, lse, static_cast<size_t>(BH) * Nq, stream);
+
+  CUtensorMap tq, tk, tv, to;
+  const int bh = static_cast<int>(BH);
+  if (!make_tmap_u8_3d(&tq, q, bh, Nq, d, kBlockM, &t_last_error) ||
+      !make_tmap_u8_3d(&tk, k, static_cast<int>(BHkv), Nk, d, kBlockN, &t_last_error) ||
+      !make_tmap_u8_3d(&tv, v, static_cast<int>(BHkv), Nk, d, kBlockN, &t_last_error) ||
+      !make_tmap_bf16_3d(&to, o, bh, Nq, d, 32, &t_last_error))
+    return ATTN_ERR_CUDA;
+
+  FwdParams prm = {};
+  prm.lse = lse;
+  prm.o = static_cast<__nv_bfloat16*>(o);
+  prm.timeout_ns = kWaitTimeoutNs;
+  prm.Nq = Nq;
+  prm.Nk = Nk;
+  prm.BH = bh;
+  prm.H = H;
+  prm.group = H / Hkv;
+  prm.wl = kUnbounded;
+  prm.wr = causal ? 0 : kUnbounded;
+  prm.grouped = causal;
+  prm.hgroup = heads_per_l2_group(Nk / 2.0, d, prm.group, BH);  // one byte per element
+  prm.n_qblocks = static_cast<int>(n_qblocks);
+  prm.scale_log2 = s_eff * kLog2e;
+  prm.tau = kP8Tau;
+  prm.o_scale = v_descale;
+  return causal ? launch_fwd<128, true, kDefaultPoly16, true>(tq, tk, tv, to, prm, stream)
+                : launch_fwd<128, false, kDefaultPoly16, true>(tq, tk, tv, to, prm, stream);
 }
 
 }  // namespace eab
@@ -1013,6 +1127,13 @@ int attn_fwd_varlen(const void* q, const void* k, const void* v, void* o, float*
                     float scale, int window_left, int window_right, cudaStream_t stream) {
   return eab::varlen_impl(q, k, v, o, lse, cu_seqlens_q, cu_seqlens_k, num_seqs, max_seqlen_q,
                           total_q, total_k, H, Hkv, d, scale, window_left, window_right, stream);
+}
+
+int attn_fwd_fp8(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
+                 int Hkv, int Nq, int Nk, int d, float scale, float q_descale, float k_descale,
+                 float v_descale, int causal, cudaStream_t stream) {
+  return eab::fp8_impl(q, k, v, o, lse, B, H, Hkv, Nq, Nk, d, scale, q_descale, k_descale,
+                       v_descale, causal, stream);
 }
 
 int attn_fwd_config(const void* q, const void* k, const void* v, void* o, float* lse, int B,

@@ -222,6 +222,101 @@ swizzle_kernel(const __grid_constant__ CUtensorMap tx, const __grid_constant__ C
   __syncthreads();
 }
 
+// 8-bit operands (kind::f8f6f4, E4M3).  SS: c[128][128] = a[128][128] *
+// b[128][128]^T, both K-major (one 128-byte box per row, K steps of 32 bytes).
+// TS: c[128][128] = p[128][128 keys] * v[128 keys][128]; P written to TMEM by
+// the threads, four E4M3 per column (key 4i in the low byte of column i), V
+// MN-major (rows of 128 bytes along d, 32 key rows = 4096 bytes per K step).
+template <bool TS>
+__global__ void __launch_bounds__(128, 1)
+mma_e4m3_kernel(const __grid_constant__ CUtensorMap ta, const __grid_constant__ CUtensorMap tb,
+                const uint32_t* p, float* c) {
+  extern __shared__ uint8_t raw[];
+  uint8_t* base = align1024(raw);
+  const uint32_t sA = smem_u32(base), sB = sA + kBox;
+  const uint32_t full = sB + kBox, done = full + 8;
+  uint32_t* slot = reinterpret_cast<uint32_t*>(base + 2 * kBox + 16);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  if (tid == 0) {
+    mbar_init(full, 1);
+    mbar_init(done, 1);
+    fence_barrier_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(smem_u32(slot), 256);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *slot;
+  const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
+  const int row = warp * 32 + lane;
+  if (TS) {
+    uint32_t pr[32];
+    for (int i = 0; i < 32; ++i) pr[i] = p[row * 32 + i];
+    tmem_st32(tmem + lane_off + 128, pr);
+    tmem_st_wait();
+  }
+  tc_fence_before();
+  __syncthreads();
+  bool ok = true;
+  if (tid == 0) {
+    tc_fence_after();
+    mbar_arrive_expect_tx(full, TS ? kBox : 2 * kBox);
+    if (!TS) tma_load_3d(sA, &ta, 0, 0, 0, full);
+    tma_load_3d(sB, &tb, 0, 0, 0, full);
+    ok = mbar_wait(full, 0, kTimeoutNs);
+    if (ok) {
+      if (TS) {
+        constexpr uint32_t idesc = idesc_e4m3_f32(128, 128, false, true);
+        const uint64_t bd = sdesc_sw128(sB, kBox, 1024);
+        const uint32_t b_lo = static_cast<uint32_t>(bd), b_hi = static_cast<uint32_t>(bd >> 32);
+        mma_ts_imm_f8<0, 0>(tmem, tmem + 128, b_lo, b_hi, idesc, 0u);
+        mma_ts_imm_f8<8, (4096 >> 4)>(tmem, tmem + 128, b_lo, b_hi, idesc, 1u);
+        mma_ts_imm_f8<16, (8192 >> 4)>(tmem, tmem + 128, b_lo, b_hi, idesc, 1u);
+        mma_ts_imm_f8<24, (12288 >> 4)>(tmem, tmem + 128, b_lo, b_hi, idesc, 1u);
+      } else {
+        constexpr uint32_t idesc = idesc_e4m3_f32(128, 128, false, false);
+        const uint64_t ad = sdesc_sw128(sA, 16, 1024), bd = sdesc_sw128(sB, 16, 1024);
+        const uint32_t a_lo = static_cast<uint32_t>(ad), a_hi = static_cast<uint32_t>(ad >> 32);
+        const uint32_t b_lo = static_cast<uint32_t>(bd), b_hi = static_cast<uint32_t>(bd >> 32);
+        mma_ss_imm_f8<0, 0, 0u>(tmem, a_lo, a_hi, b_lo, b_hi, idesc);
+        mma_ss_imm_f8<2, 2, 1u>(tmem, a_lo, a_hi, b_lo, b_hi, idesc);
+        mma_ss_imm_f8<4, 4, 1u>(tmem, a_lo, a_hi, b_lo, b_hi, idesc);
+        mma_ss_imm_f8<6, 6, 1u>(tmem, a_lo, a_hi, b_lo, b_hi, idesc);
+      }
+    } else {
+      mbar_wait(full, 0, kTimeoutNs);
+    }
+    tc_commit(done);
+  }
+  __syncwarp();
+  const bool ok2 = warp_wait(done, 0);
+  if (ok2) {
+    tc_fence_after();
+    for (int q = 0; q < 4; ++q) {
+      uint32_t r[32];
+      tmem_ld32(tmem + lane_off + q * 32, r);
+      tmem_ld_wait();
+      reg_fence32(r);
+      for (int i = 0; i < 32; ++i) c[row * 128 + q * 32 + i] = __uint_as_float(r[i]);
+    }
+  }
+  if (!ok || !ok2) atomicOr(&g_blk_status, 1u);
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 256);
+  }
+}
+
+__global__ void pack_e4m3_kernel(const float* x, uint32_t* y, int n4) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < n4) y[i] = pack_e4m3x4(x[4 * i], x[4 * i + 1], x[4 * i + 2], x[4 * i + 3]);
+}
+
 __global__ void exp2_kernel(const float* x, float* y_mufu, float* y_poly, int n) {
   const int i = blockIdx.x * blockDim.x + threadIdx.x;
   if (i < n) {
@@ -315,6 +410,41 @@ int blocks_exp2(const float* x, float* y_mufu, float* y_poly, int n, cudaStream_
   exp2_kernel<<<(n + 255) / 256, 256, 0, stream>>>(x, y_mufu, y_poly, n);
   cudaError_t e = cudaGetLastError();
   return e == cudaSuccess ? BLOCKS_OK : fail(e, "exp2_kernel launch");
+}
+
+int blocks_mma_e4m3_ss(const void* a, const void* b, float* c, cudaStream_t stream) {
+  if (bad_ptr(a) || bad_ptr(b) || bad_ptr(c)) return BLOCKS_ERR_INVALID_ARG;
+  CUtensorMap ta, tb;
+  if (!eab::make_tmap_u8_3d(&ta, a, 1, 128, 128, 128, &t_err) ||
+      !eab::make_tmap_u8_3d(&tb, b, 1, 128, 128, 128, &t_err))
+    return BLOCKS_ERR_CUDA;
+  const int smem = 2 * kBox + 1024 + 64;
+  int rc;
+  if ((rc = set_smem((const void*)mma_e4m3_kernel<false>, smem)) != BLOCKS_OK) return rc;
+  mma_e4m3_kernel<false><<<1, 128, smem, stream>>>(ta, tb, nullptr, c);
+  cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? BLOCKS_OK : fail(e, "mma_e4m3_kernel launch");
+}
+
+int blocks_mma_e4m3_ts(const void* p, const void* v, float* c, cudaStream_t stream) {
+  if (bad_ptr(p) || bad_ptr(v) || bad_ptr(c)) return BLOCKS_ERR_INVALID_ARG;
+  CUtensorMap tv;
+  if (!eab::make_tmap_u8_3d(&tv, v, 1, 128, 128, 128, &t_err)) return BLOCKS_ERR_CUDA;
+  const int smem = 2 * kBox + 1024 + 64;
+  int rc;
+  if ((rc = set_smem((const void*)mma_e4m3_kernel<true>, smem)) != BLOCKS_OK) return rc;
+  mma_e4m3_kernel<true><<<1, 128, smem, stream>>>(tv, tv, static_cast<const uint32_t*>(p), c);
+  cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? BLOCKS_OK : fail(e, "mma_e4m3_kernel launch");
+}
+
+int blocks_pack_e4m3(const float* x, void* y, int n4, cudaStream_t stream) {
+  if (n4 < 0) return BLOCKS_ERR_INVALID_ARG;
+  if (n4 == 0) return BLOCKS_OK;
+  if (!x || !y) return BLOCKS_ERR_INVALID_ARG;
+  pack_e4m3_kernel<<<(n4 + 255) / 256, 256, 0, stream>>>(x, static_cast<uint32_t*>(y), n4);
+  cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? BLOCKS_OK : fail(e, "pack_e4m3_kernel launch");
 }
 
 int blocks_status_sync(cudaStream_t stream) {

@@ -55,6 +55,56 @@ inline bool encode_bf16_3d(CUtensorMap* tm, const void* base, const cuuint64_t d
   return true;
 }
 
+// 8-bit elements: a 3-D map [BH, N, d] of bytes, box = 128 columns (128 bytes,
+// 128-byte swizzle) x box_rows rows x 1; coordinates (column, row, head).
+inline bool make_tmap_u8_3d(CUtensorMap* tm, const void* base, int BH, int N, int d, int box_rows,
+                            std::string* err) {
+  EncodeTiledFn enc = get_encode_fn();
+  if (!enc) {
+    *err = "cuTensorMapEncodeTiled unavailable";
+    return false;
+  }
+  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(N),
+                              static_cast<cuuint64_t>(BH)};
+  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(d),
+                                 static_cast<cuuint64_t>(N) * static_cast<cuuint64_t>(d)};
+  const cuuint32_t box[3] = {128u, static_cast<cuuint32_t>(box_rows), 1u};
+  const cuuint32_t estr[3] = {1u, 1u, 1u};
+  CUresult r = enc(tm, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides, box,
+                   estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) {
+    *err = "cuTensorMapEncodeTiled failed (CUresult " + std::to_string(static_cast<int>(r)) + ")";
+    return false;
+  }
+  return true;
+}
+
+// FP32 [BH, N, d] with 32-column (128-byte, 128-byte swizzle) x box_rows boxes;
+// coordinates (column, row, head).  Used for reductions into an accumulator.
+inline bool make_tmap_f32_3d(CUtensorMap* tm, const void* base, int BH, int N, int d, int box_rows,
+                             std::string* err) {
+  EncodeTiledFn enc = get_encode_fn();
+  if (!enc) {
+    *err = "cuTensorMapEncodeTiled unavailable";
+    return false;
+  }
+  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(N),
+                              static_cast<cuuint64_t>(BH)};
+  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 4,
+                                 static_cast<cuuint64_t>(N) * static_cast<cuuint64_t>(d) * 4};
+  const cuuint32_t box[3] = {32u, static_cast<cuuint32_t>(box_rows), 1u};
+  const cuuint32_t estr[3] = {1u, 1u, 1u};
+  CUresult r = enc(tm, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<void*>(base), dims, strides, box,
+                   estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) {
+    *err = "cuTensorMapEncodeTiled failed (CUresult " + std::to_string(static_cast<int>(r)) + ")";
+    return false;
+  }
+  return true;
+}
+
 // Dense [BH, N, d]: coordinates (column, row, head); rows past N of one head
 // read as zero (never as the next head's rows) and are clipped on store.
 inline bool make_tmap_bf16_3d(CUtensorMap* tm, const void* base, int BH, int N, int d,

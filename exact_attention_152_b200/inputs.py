@@ -76,7 +76,8 @@ def bf16_bits_to_f64(b: np.ndarray) -> np.ndarray:
     return bf16_bits_to_f32(b).astype(np.float64)
 
 
-def _values(key: np.uint64, idx: np.ndarray, dist: str, mult: float) -> np.ndarray:
+def _draw(key: np.uint64, idx: np.ndarray, dist: str) -> np.ndarray:
+    """fp64 draws z (before the multiplier and rounding)."""
     bits = _bits(key, idx)
     if dist == "normal":
         hi = (bits >> np.uint64(32)).astype(np.float64)
@@ -89,7 +90,11 @@ def _values(key: np.uint64, idx: np.ndarray, dist: str, mult: float) -> np.ndarr
         z = 2.0 * u - 1.0
     else:
         raise ValueError(f"unknown distribution {dist!r}")
-    return f32_to_bf16_bits((mult * z).astype(np.float32))
+    return z
+
+
+def _values(key: np.uint64, idx: np.ndarray, dist: str, mult: float) -> np.ndarray:
+    return f32_to_bf16_bits((mult * _draw(key, idx, dist)).astype(np.float32))
 
 
 def gen_bf16_at(seed: int, tensor: str, flat_idx: np.ndarray, dist: str = "normal",
@@ -136,6 +141,72 @@ def gen_bf16(seed: int, tensor: str, shape, dist: str = "normal", mult: float = 
         for s in starts:
             fill(s)
     return out.reshape(shape)
+
+
+# ---------------------------------------------------------------------------
+# FP8 E4M3 (the OCP "E4M3FN" format): 1 sign bit, 4 exponent bits (bias 7),
+# 3 mantissa bits; exponent field 0 holds the subnormals m/8 * 2^-6; code
+# S.1111.111 is NaN and there is no infinity, so the largest finite value is
+# 1.75 * 2^8 = 448.
+# ---------------------------------------------------------------------------
+def e4m3_decode_table() -> np.ndarray:
+    """fp64 value of each of the 256 codes (NaN for the two NaN codes)."""
+    vals = np.empty(256, dtype=np.float64)
+    for code in range(256):
+        sign = -1.0 if code & 0x80 else 1.0
+        e, m = (code >> 3) & 0xF, code & 0x7
+        if e == 0xF and m == 0x7:
+            vals[code] = np.nan
+        elif e == 0:
+            vals[code] = sign * (m / 8.0) * 2.0 ** -6
+        else:
+            vals[code] = sign * (1.0 + m / 8.0) * 2.0 ** (e - 7)
+    return vals
+
+
+_E4M3 = e4m3_decode_table()
+_E4M3_POS = _E4M3[:127]  # codes 0 .. 126: +0 .. 448, increasing
+
+
+def e4m3_from_f32(x: np.ndarray) -> np.ndarray:
+    """Round fp32 values to the nearest E4M3 code (ties to the even code),
+    saturating at +-448.  Returns uint8 codes."""
+    x = np.asarray(x, dtype=np.float32).astype(np.float64)
+    a = np.minimum(np.abs(x), 448.0)
+    hi = np.searchsorted(_E4M3_POS, a, side="left")      # first code with value >= a
+    hi = np.minimum(hi, 126)
+    lo = np.maximum(hi - 1, 0)
+    d_lo = a - _E4M3_POS[lo]
+    d_hi = _E4M3_POS[hi] - a
+    pick_hi = (d_hi < d_lo) | ((d_hi == d_lo) & (hi % 2 == 0))
+    code = np.where(pick_hi, hi, lo).astype(np.uint8)
+    return np.where(np.signbit(x), code | np.uint8(0x80), code).astype(np.uint8)
+
+
+def e4m3_to_f64(codes: np.ndarray) -> np.ndarray:
+    return _E4M3[np.asarray(codes, dtype=np.uint8)]
+
+
+def gen_e4m3(seed: int, tensor: str, shape, dist: str = "normal", mult: float = 1.0) -> np.ndarray:
+    """E4M3 codes of a whole tensor: the BF16 generator's fp32 draw (mult * z)
+    rounded to E4M3 instead of BF16."""
+    n = int(np.prod(shape))
+    key = _key(seed, TENSOR_ID[tensor])
+    out = np.empty(n, dtype=np.uint8)
+    for s in range(0, n, _CHUNK):
+        e = min(n, s + _CHUNK)
+        out[s:e] = e4m3_from_f32((mult * _draw(key, np.arange(s, e, dtype=np.int64), dist))
+                                 .astype(np.float32))
+    return out.reshape(shape)
+
+
+def e4m3_at(seed: int, tensor: str, flat_idx: np.ndarray, dist: str = "normal",
+            mult: float = 1.0) -> np.ndarray:
+    """E4M3 codes of the elements with the given flat indices (any shape)."""
+    key = _key(seed, TENSOR_ID[tensor])
+    idx = np.asarray(flat_idx, dtype=np.int64)
+    z = _draw(key, idx.reshape(-1), dist)
+    return e4m3_from_f32((mult * z).astype(np.float32)).reshape(idx.shape)
 
 
 def sample_rows(seed: int, bh: int, n: int, count: int) -> np.ndarray:

@@ -35,6 +35,8 @@ class Workload:
     window: tuple | None = None     # key band (left, right), -1 = no bound; replaces causal
     seqlens: tuple | None = None    # packed variable-length batch: one length per sequence
                                     # (queries and keys alike); B = len(seqlens)
+    fp8: bool = False               # Q, K, V as E4M3 codes times the descale factors below
+    descale: tuple = (1.0, 1.0, 1.0)  # (q, k, v) scale factors of the E4M3 codes
 
     @property
     def packed(self) -> bool:
@@ -91,8 +93,17 @@ class Workload:
         return self.v_dist, 1.0
 
     def tensor_bits(self, which: str) -> np.ndarray:
+        """BF16 bits (uint16), or E4M3 codes (uint8) for an FP8 workload."""
         dist, mult = self.dist(which)
+        if self.fp8:
+            return inputs.gen_e4m3(self.seed, which, self.shape(which), dist, mult)
         return inputs.gen_bf16(self.seed, which, self.shape(which), dist, mult)
+
+    def to_f64(self, which: str, bits: np.ndarray) -> np.ndarray:
+        """The values the stored bits stand for (E4M3 codes times their descale)."""
+        if self.fp8:
+            return inputs.e4m3_to_f64(bits) * self.descale["qkv".index(which)]
+        return inputs.bf16_bits_to_f64(bits)
 
     def head_bits(self, which: str, bh: int) -> np.ndarray:
         """BF16 bits of one (b, h) slice, [N, d]; for k/v, bh indexes the B*Hkv
@@ -101,12 +112,16 @@ class Workload:
         n = self.Nq if which == "q" else self.Nk
         base = bh * n * self.d
         idx = np.arange(base, base + n * self.d, dtype=np.int64)
+        if self.fp8:
+            return inputs.e4m3_at(self.seed, which, idx, dist, mult).reshape(n, self.d)
         return inputs.gen_bf16_at(self.seed, which, idx, dist, mult).reshape(n, self.d)
 
     def q_rows_bits(self, bh: int, rows: np.ndarray) -> np.ndarray:
         dist, mult = self.dist("q")
         base = bh * self.Nq * self.d
         idx = base + rows.astype(np.int64)[:, None] * self.d + np.arange(self.d, dtype=np.int64)[None, :]
+        if self.fp8:
+            return inputs.e4m3_at(self.seed, "q", idx, dist, mult)
         return inputs.gen_bf16_at(self.seed, "q", idx, dist, mult)
 
     def kv_head_of(self, bh: int) -> int:
@@ -165,6 +180,11 @@ WORKLOADS = {
         # causal sliding window over the last 4096 keys
         Workload("swa_b1h32n32k_w4k_d128", 1, 32, 32768, 32768, 128, False, seed=6,
                  oracle_rows=128, window=(4095, 0)),
+        # E4M3 inputs (the FP8 forward)
+        Workload("fp8_b2h16n8k_d128", 2, 16, 8192, 8192, 128, False, seed=8, oracle_rows=128,
+                 fp8=True),
+        Workload("fp8_b2h16n8k_d128_causal", 2, 16, 8192, 8192, 128, True, seed=8, oracle_rows=128,
+                 fp8=True),
         # 16 sequences of mixed length (512 .. 16384 tokens), packed, causal
         Workload("varlen16_h16_d128_causal", 16, 16, 0, 0, 128, True, seed=7, oracle_rows=64,
                  seqlens=_mixed_lengths(7, 16, 512, 16384)),

@@ -141,6 +141,31 @@ int attn_fwd_varlen(const void *q, const void *k, const void *v, void *o, float 
                     float scale, int window_left, int window_right, cudaStream_t stream);
 
 /*
+ * FP8 forward: Q, K, V given as E4M3 bytes (OCP E4M3FN: 4 exponent bits with
+ * bias 7, 3 mantissa bits, largest finite value 448) with one scale factor per
+ * tensor, so the attended values are q_descale * Q8, k_descale * K8 and
+ * v_descale * V8.  The pages name the FP8 forward among FlashAttention 3's
+ * improvements ("Flash Attention（Flash Attention）", jisaku.com glossary,
+ * sections "ハードウェアへの影響と推奨スペック" and "FlashAttention-3とFP8の時代");
+ * the definition is that of
+ * attn_fwd on those values:
+ *
+ *     s_ij = scale * q_descale * k_descale * <Q8_i, K8_j>
+ *     O_i  = v_descale * sum_j softmax_j(s_ij) * V8_j,   LSE_i as in attn_fwd
+ *
+ * Q.K^T and P.V run on the tensor cores in E4M3 (kind::f8f6f4) with FP32
+ * accumulation; P is rounded to E4M3 for P.V (O's error is therefore of the
+ * order of E4M3's 2^-4 relative rounding of the weights, not BF16's 2^-9).
+ *   q : [B, H, Nq, d] bytes;  k, v : [B, Hkv, Nk, d] bytes;  d must be 128
+ *   o : BF16 [B, H, Nq, d];   lse : FP32 [B, H, Nq] (may be NULL)
+ *   q_descale, k_descale, v_descale : finite floats
+ *   Hkv, causal and everything else as attn_fwd_gqa.
+ */
+int attn_fwd_fp8(const void *q, const void *k, const void *v, void *o, float *lse, int B, int H,
+                 int Hkv, int Nq, int Nk, int d, float scale, float q_descale, float k_descale,
+                 float v_descale, int causal, cudaStream_t stream);
+
+/*
  * attn_fwd with the kernel's two softmax knobs exposed (same contract otherwise).
  *
  *   rescale_threshold : adaptive online rescaling (FlashAttention 4 page,

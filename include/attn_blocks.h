@@ -54,6 +54,19 @@ int blocks_swizzle_roundtrip(const void *x, void *y_tma, void *y_plain, int d,
 /* y_mufu[i] = hardware ex2.approx(x[i]); y_poly[i] = polynomial exp2(x[i]). */
 int blocks_exp2(const float *x, float *y_mufu, float *y_poly, int n, cudaStream_t stream);
 
+/* E4M3 (kind::f8f6f4) tile, both operands K-major: c[128][128] (fp32) =
+ * a[128][128] * b[128][128]^T, a and b row-major E4M3 bytes. */
+int blocks_mma_e4m3_ss(const void *a, const void *b, float *c, cudaStream_t stream);
+
+/* E4M3 tile with A from Tensor Memory: c[128][128] = P[128][128] * v[128][128],
+ * p = 128 rows x 32 words, four E4M3 per word (key 4i in the low byte of word i),
+ * v row-major E4M3 [keys][d], read MN-major. */
+int blocks_mma_e4m3_ts(const void *p, const void *v, float *c, cudaStream_t stream);
+
+/* y[i] = the four E4M3 codes of x[4i..4i+3] (x[4i] in the low byte), round to
+ * nearest even, saturating at +-448; n4 words. */
+int blocks_pack_e4m3(const float *x, void *y, int n4, cudaStream_t stream);
+
 /* Synchronise `stream`, read and clear this library's status word. */
 int blocks_status_sync(cudaStream_t stream);
 

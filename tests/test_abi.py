@@ -49,7 +49,7 @@ def test_library_exports_every_declared_symbol(header):
 def test_attn_h_declares_the_contract():
     names = declared_functions(os.path.join(ROOT, "include", "attn.h"))
     for n in ("attn_fwd", "attn_fwd_config", "attn_fwd_gqa", "attn_fwd_window", "attn_fwd_varlen",
-              "attn_bwd", "attn_bwd_noalloc", "attn_bwd_workspace_size", "attn_status_sync", "attn_status_string",
+              "attn_fwd_fp8", "attn_bwd", "attn_bwd_noalloc", "attn_bwd_workspace_size", "attn_status_sync", "attn_status_string",
               "attn_last_error", "attn_selftest_timeout"):
         assert n in names
 
@@ -141,6 +141,19 @@ def test_varlen_validation():
     # nothing to compute: a no-op even with null pointers
     assert V(None, None, None, None, None, None, None, 0, 0, 0, 0, 4, 2, 64, 0.1, -1, 0, None) == 0
     assert V(None, None, None, None, None, None, None, 3, 0, 0, 0, 4, 2, 64, 0.1, -1, 0, None) == 0
+
+
+def test_fp8_validation():
+    F8 = binding.attn_fwd_fp8
+    P = (ALIGNED, ALIGNED * 2, ALIGNED * 3, ALIGNED * 16, None)
+    assert F8(*P, 1, 2, 2, 64, 64, 64, 0.1, 1.0, 1.0, 1.0, 0, None) == 2      # d must be 128
+    assert F8(*P, 1, 2, 2, 64, 32, 128, 0.1, 1.0, 1.0, 1.0, 1, None) == 2     # causal Nq != Nk
+    assert F8(*P, 1, 2, 2, 64, 64, 128, 0.1, math.nan, 1.0, 1.0, 0, None) == 1
+    assert F8(*P, 1, 2, 2, 64, 64, 128, 0.1, 1.0, 1.0, math.inf, 0, None) == 1
+    assert F8(*P, 1, 2, 2, 64, 64, 128, 1e30, 1e30, 1.0, 1.0, 0, None) == 1  # scale product overflows
+    assert F8(*P, 1, 3, 2, 64, 64, 128, 0.1, 1.0, 1.0, 1.0, 0, None) == 1     # H % Hkv
+    assert F8(ALIGNED + 1, *P[1:], 1, 2, 2, 64, 64, 128, 0.1, 1.0, 1.0, 1.0, 0, None) == 1
+    assert F8(None, None, None, None, None, 0, 2, 2, 64, 64, 128, 0.1, 1.0, 1.0, 1.0, 0, None) == 0
 
 
 def test_bwd_validation():

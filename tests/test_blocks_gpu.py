@@ -86,3 +86,46 @@ def test_exp2_mufu_and_polynomial():
     # far below the range (masked scores) -> exactly +0
     assert np.all(yp[xs <= -127.0] == 0.0)
     assert np.all(ym[xs <= -127.0] < 1e-37)
+
+
+def _dev_u8(codes):
+    import torch
+    return torch.from_numpy(np.ascontiguousarray(codes)).cuda()
+
+
+def test_pack_e4m3_order_and_rounding():
+    """Four fp32 -> four E4M3 bytes, x[4i] in the low byte, rounded as the
+    host encoder rounds (nearest even, saturating)."""
+    import torch
+    x = np.random.default_rng(7).standard_normal(4096).astype(np.float32) * np.float32(50)
+    x[:8] = [0.0, -0.0, 2.0 ** -10, 1.5 * 2.0 ** -9, 1.0625, 1.1875, 448.0, 1000.0]
+    y = torch.zeros(1024, dtype=torch.int32, device="cuda")
+    assert bb.blocks_pack_e4m3(torch.from_numpy(x).cuda().data_ptr(), y.data_ptr(), 1024, _stream()) == 0
+    assert bb.blocks_status_sync(_stream()) == 0
+    got = y.cpu().numpy().view(np.uint8)
+    assert np.array_equal(got, inputs.e4m3_from_f32(x))
+
+
+def test_mma_e4m3_ss_tile():
+    import torch
+    a = inputs.gen_e4m3(500, "q", (128, 128))
+    b = inputs.gen_e4m3(500, "k", (128, 128))
+    c = torch.full((128, 128), float("nan"), dtype=torch.float32, device="cuda")
+    assert bb.blocks_mma_e4m3_ss(_dev_u8(a).data_ptr(), _dev_u8(b).data_ptr(), c.data_ptr(), _stream()) == 0
+    assert bb.blocks_status_sync(_stream()) == 0
+    ref = inputs.e4m3_to_f64(a) @ inputs.e4m3_to_f64(b).T
+    got = c.cpu().numpy().astype(np.float64)
+    # E4M3 products are exact in fp32; only the accumulation order differs
+    np.testing.assert_allclose(got, ref, rtol=0, atol=1e-5 * np.abs(ref).max())
+
+
+def test_mma_e4m3_ts_tile():
+    import torch
+    p = inputs.gen_e4m3(510, "q", (128, 128), dist="uniform", mult=4.0)
+    v = inputs.gen_e4m3(510, "v", (128, 128))
+    c = torch.full((128, 128), float("nan"), dtype=torch.float32, device="cuda")
+    assert bb.blocks_mma_e4m3_ts(_dev_u8(p).data_ptr(), _dev_u8(v).data_ptr(), c.data_ptr(), _stream()) == 0
+    assert bb.blocks_status_sync(_stream()) == 0
+    ref = inputs.e4m3_to_f64(p) @ inputs.e4m3_to_f64(v)
+    got = c.cpu().numpy().astype(np.float64)
+    np.testing.assert_allclose(got, ref, rtol=0, atol=1e-5 * np.abs(ref).max())

@@ -73,3 +73,23 @@ def test_gqa_workload_kv_heads():
         b, h = divmod(bh, w.H)
         assert w.kv_head_of(bh) == b * 8 + h // 4
         assert np.array_equal(w.head_bits("k", w.kv_head_of(bh)), k[b, h // 4])
+
+
+def test_e4m3_codes():
+    """The E4M3 table follows the format's definition, and rounding to it agrees
+    with torch's float8_e4m3fn conversion inside the finite range (torch does
+    not saturate beyond it; this generator does, to +-448)."""
+    import torch
+    from exact_attention_152_b200 import inputs
+    t = inputs.e4m3_decode_table()
+    assert t[0x00] == 0.0 and t[0x01] == 2.0 ** -9 and t[0x08] == 2.0 ** -6
+    assert t[0x38] == 1.0 and t[0x7E] == 448.0 and np.isnan(t[0x7F]) and t[0xB8] == -1.0
+    x = np.random.default_rng(3).standard_normal(100000).astype(np.float32) * np.float32(40)
+    x = np.concatenate([x, np.float32([0.0, -0.0, 2.0 ** -10, 1.5 * 2.0 ** -9, 1.0625, 1.1875, 448])])
+    x = x[np.abs(x) <= 448]
+    ours = inputs.e4m3_from_f32(x)
+    ref = torch.from_numpy(x).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    assert np.array_equal(ours, ref)
+    assert inputs.e4m3_from_f32(np.float32([1000.0, -500.0])).tolist() == [0x7E, 0xFE]
+    codes = inputs.gen_e4m3(5, "q", (4, 8))
+    assert codes.dtype == np.uint8 and codes.shape == (4, 8)

@@ -212,8 +212,9 @@ def _packed_case(w):
     return harness.compare_varlen(o, lse, ref, cu)
 
 
-@pytest.mark.parametrize("name", list(WORKLOADS))
+@pytest.mark.parametrize("name", [n for n, w in WORKLOADS.items() if not w.fp8])
 def test_workload_parity(name):
+    """Every BF16 workload (the E4M3 ones have their own bound: test_fp8_gpu.py)."""
     w = WORKLOADS[name]
     if w.packed:
         m = _packed_case(w)
