@@ -49,6 +49,7 @@
 #include <mutex>
 
 #include "attn.h"
+#include "exp2.cuh"
 #include "host_common.h"
 #include "sm100.cuh"
 #include "tmap.h"
@@ -85,7 +86,7 @@ struct Cfg {
   static constexpr int kDSBytes = 2 * kBoxBytes;
   static constexpr int kOffRow = kOffDS + kDSBytes; // per stage: LSE*log2e [128], D [128]
   static constexpr int kRowBytes = 2 * 2 * kBlockQ * 4;
-  static constexpr int kNumBars = 12;
+  static constexpr int kNumBars = 13;
   static constexpr int kOffBar = kOffRow + kRowBytes;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
   static constexpr int kSmemBytes = kOffMisc + 16;
@@ -115,6 +116,7 @@ struct Smem {
   __device__ __forceinline__ uint32_t q(int s) const { return sbase + Cfg<D>::kOffQ + s * Cfg<D>::kTileBytes; }
   __device__ __forceinline__ uint32_t dout(int s) const { return sbase + Cfg<D>::kOffDO + s * Cfg<D>::kTileBytes; }
   __device__ __forceinline__ uint32_t ds() const { return sbase + Cfg<D>::kOffDS; }
+  // -LSE * log2(e) of the stage's 128 query rows, then their D
   __device__ __forceinline__ float* lse2(int s) const {
     return reinterpret_cast<float*>(base + Cfg<D>::kOffRow) + s * 2 * kBlockQ;
   }
@@ -131,6 +133,8 @@ struct Smem {
   __device__ __forceinline__ uint32_t done() const { return bar(10); }
   // the dQ drain no longer stages in the dS buffer (its reductions have read it)
   __device__ __forceinline__ uint32_t ds_free() const { return bar(11); }
+  // dS of the current tile is in shared memory (the dQ GEMM may start)
+  __device__ __forceinline__ uint32_t ds_ready() const { return bar(12); }
   __device__ __forceinline__ uint32_t* tmem_slot() const {
     return reinterpret_cast<uint32_t*>(base + Cfg<D>::kOffMisc);
   }
@@ -212,15 +216,15 @@ __device__ __forceinline__ void producer_role(const Smem<D>& sm, const CUtensorM
     if (!ok) break;
     const int bh = w.b * prm.H + w.hkv * prm.group + w.head_of(it);
     const int q0 = w.tile_of(it) * kBlockQ;
-    // rows past Nq: LSE = +inf makes P = 0 there; D = 0
-    float* l2 = sm.lse2(s);
+    // -LSE * log2(e) per query row (rows past Nq: -inf, so P = 0 there), and D
+    float* nl = sm.lse2(s);
     float* dd = sm.dsum(s);
 #pragma unroll
     for (int r = lane; r < kBlockQ; r += 32) {
       const int q = q0 + r;
       const bool in = q < prm.Nq;
       const size_t row = static_cast<size_t>(bh) * prm.Nq + q;
-      l2[r] = in ? prm.lse[row] * kLog2e : INFINITY;
+      nl[r] = in ? -prm.lse[row] * kLog2e : -INFINITY;
       dd[r] = in ? prm.dsum[row] : 0.0f;
     }
     if (lane == 0) {
@@ -290,6 +294,9 @@ __device__ __forceinline__ void mma_role(const Smem<D>& sm, uint32_t tmem, const
     Mma<D, 0>::tmem_a(tmem + C::kTmemDK, tmem + C::kTmemDP, lo(qmn) + s * kStageStep, hi(qmn), id_kv,
                       acc);
     tc_commit(sm.q_empty(s));
+    ok = mbar_wait(sm.ds_ready(), it & 1, timeout);
+    if (!ok) break;
+    tc_fence_after();
     Mma<D, 0>::mnmajor(tmem, lo(dsmn), hi(dsmn), lo(kmn), hi(kmn), id_q);
     tc_commit(sm.dq_full());
   }
@@ -329,13 +336,10 @@ __device__ __forceinline__ bool softmax_grad_role(const Smem<D>& sm, uint32_t tm
     const int q_base = w.tile_of(it) * kBlockQ + c * 64;  // first query of this warp's columns
     // masking: key tail, or (causal) a key past some query of the block
     const bool masked = !key_in || (CAUSAL && w.j * kBlockK + q4 * 32 + 31 > q_base);
-    // the dS buffer doubled as the previous dQ tile's staging
-    if (it > 0 && !warp_wait(sm.ds_free(), (it - 1) & 1, prm.timeout_ns)) {
-      ok = false;
-      break;
-    }
-    const float* l2 = sm.lse2(s) + c * 64;
-    const float* dd = sm.dsum(s) + c * 64;
+    const float4* nl4 = reinterpret_cast<const float4*>(sm.lse2(s) + c * 64);
+    const float4* dd4 = reinterpret_cast<const float4*>(sm.dsum(s) + c * 64);
+    const float2 sl2 = make_float2(prm.scale_log2, prm.scale_log2);
+    uint32_t dsk[2][16];  // this thread's dS row (BF16 pairs), written to shared memory last
 #pragma unroll
     for (int k = 0; k < 2; ++k) {
       uint32_t sv[32], pv[32];
@@ -346,36 +350,66 @@ __device__ __forceinline__ bool softmax_grad_role(const Smem<D>& sm, uint32_t tm
       reg_fence32(pv);
       uint32_t pp[16], dsp[16];
 #pragma unroll
-      for (int i = 0; i < 16; ++i) {
-        float p2[2], d2[2];
-#pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          const int col = 32 * k + 2 * i + e;
-          float x = fmaf(__uint_as_float(sv[2 * i + e]), prm.scale_log2, -l2[col]);
-          if (masked && (!key_in || (CAUSAL && key > q_base + col))) x = -INFINITY;
-          const float p = ex2_mufu(x);
-          p2[e] = p;
-          d2[e] = p * (__uint_as_float(pv[2 * i + e]) - dd[col]);
+      for (int g = 0; g < 8; ++g) {  // query columns 32k + 4g .. 32k + 4g + 3
+        const float4 nl = nl4[8 * k + g], dv = dd4[8 * k + g];
+        float2 xa = ffma2(make_float2(__uint_as_float(sv[4 * g]), __uint_as_float(sv[4 * g + 1])), sl2,
+                          make_float2(nl.x, nl.y));
+        float2 xb = ffma2(make_float2(__uint_as_float(sv[4 * g + 2]), __uint_as_float(sv[4 * g + 3])),
+                          sl2, make_float2(nl.z, nl.w));
+        if (masked) {
+          const int col = q_base + 32 * k + 4 * g;
+          if (!key_in || (CAUSAL && key > col)) xa.x = -INFINITY;
+          if (!key_in || (CAUSAL && key > col + 1)) xa.y = -INFINITY;
+          if (!key_in || (CAUSAL && key > col + 2)) xb.x = -INFINITY;
+          if (!key_in || (CAUSAL && key > col + 3)) xb.y = -INFINITY;
         }
-        pp[i] = pack_bf16x2(p2[0], p2[1]);
-        dsp[i] = pack_bf16x2(d2[0], d2[1]);
+        float2 pa, pb;
+        if ((g & 3) == 0) {  // a quarter of the exponentials on the FMA pipe
+          pa = ex2_poly2(xa);
+          pb = ex2_poly2(xb);
+        } else {
+          pa = make_float2(ex2_mufu(xa.x), ex2_mufu(xa.y));
+          pb = make_float2(ex2_mufu(xb.x), ex2_mufu(xb.y));
+        }
+        const float2 da = fmul2(pa, fsub2(make_float2(__uint_as_float(pv[4 * g]), __uint_as_float(pv[4 * g + 1])),
+                                          make_float2(dv.x, dv.y)));
+        const float2 db = fmul2(pb, fsub2(make_float2(__uint_as_float(pv[4 * g + 2]),
+                                                      __uint_as_float(pv[4 * g + 3])),
+                                          make_float2(dv.z, dv.w)));
+        pp[2 * g] = pack_bf16x2(pa.x, pa.y);
+        pp[2 * g + 1] = pack_bf16x2(pb.x, pb.y);
+        dsp[2 * g] = pack_bf16x2(da.x, da.y);
+        dsp[2 * g + 1] = pack_bf16x2(db.x, db.y);
       }
       tmem_st16(tS + 16 * k, pp);
       tmem_st16(tP + 16 * k, dsp);
-      // dS for the dQ GEMM: key row r of the 64-query block c, columns
-      // [32k, 32k+32) = 16-byte chunks 4k..4k+3, 128-byte swizzle
+#pragma unroll
+      for (int i = 0; i < 16; ++i) dsk[k][i] = dsp[i];
+    }
+    // P^T and dS^T are in TMEM: the dV and dK GEMMs may start
+    tmem_st_wait();
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(sm.p_ready());
+    // dS for the dQ GEMM, once the previous dQ tile's reductions have read the
+    // buffer they staged in: key row r of the 64-query block c, 16-byte chunks,
+    // 128-byte swizzle
+    if (it > 0 && !warp_wait(sm.ds_free(), (it - 1) & 1, prm.timeout_ns)) {
+      ok = false;
+      break;
+    }
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
         const int chunk = (4 * k + i) ^ (r & 7);
         *reinterpret_cast<uint4*>(ds_row + chunk * 16) =
-            make_uint4(dsp[4 * i], dsp[4 * i + 1], dsp[4 * i + 2], dsp[4 * i + 3]);
+            make_uint4(dsk[k][4 * i], dsk[k][4 * i + 1], dsk[k][4 * i + 2], dsk[k][4 * i + 3]);
       }
     }
-    tmem_st_wait();
     fence_proxy_async_smem();
-    tc_fence_before();
     __syncwarp();
-    if (lane == 0) mbar_arrive(sm.p_ready());
+    if (lane == 0) mbar_arrive(sm.ds_ready());
   }
   return ok;
 }
@@ -402,19 +436,24 @@ __device__ __forceinline__ bool dq_drain_role(const Smem<D>& sm, uint32_t tmem, 
     tc_fence_after();
     const int bh = w.b * prm.H + w.hkv * prm.group + w.head_of(it);
     const int row0 = w.tile_of(it) * kBlockQ + q4 * 32;
+    // all of this warp's dQ columns into registers, then TMEM is free
+    uint32_t v[kHalves][2][32];
 #pragma unroll
     for (int hf = 0; hf < kHalves; ++hf) {
-      uint32_t v0[32], v1[32];
-      tmem_ld32(tQ + 64 * hf, v0);
-      tmem_ld32(tQ + 64 * hf + 32, v1);
-      tmem_ld_wait();
-      reg_fence32(v0);
-      reg_fence32(v1);
-      if (hf == kHalves - 1) {
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(sm.dq_free());
-      }
+      tmem_ld32(tQ + 64 * hf, v[hf][0]);
+      tmem_ld32(tQ + 64 * hf + 32, v[hf][1]);
+    }
+    tmem_ld_wait();
+#pragma unroll
+    for (int hf = 0; hf < kHalves; ++hf) {
+      reg_fence32(v[hf][0]);
+      reg_fence32(v[hf][1]);
+    }
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(sm.dq_free());
+#pragma unroll
+    for (int hf = 0; hf < kHalves; ++hf) {
       if (hf > 0) {  // the previous half's reductions must have read the staging
         if (lane == 0) bulk_wait_group_read0();
         __syncwarp();
@@ -423,9 +462,9 @@ __device__ __forceinline__ bool dq_drain_role(const Smem<D>& sm, uint32_t tmem, 
 #pragma unroll
       for (int c = 0; c < 8; ++c) {
         *reinterpret_cast<uint4*>(row + ((c ^ (lane & 7)) * 16)) =
-            make_uint4(v0[4 * c], v0[4 * c + 1], v0[4 * c + 2], v0[4 * c + 3]);
+            make_uint4(v[hf][0][4 * c], v[hf][0][4 * c + 1], v[hf][0][4 * c + 2], v[hf][0][4 * c + 3]);
         *reinterpret_cast<uint4*>(row + 4096 + ((c ^ (lane & 7)) * 16)) =
-            make_uint4(v1[4 * c], v1[4 * c + 1], v1[4 * c + 2], v1[4 * c + 3]);
+            make_uint4(v[hf][1][4 * c], v[hf][1][4 * c + 1], v[hf][1][4 * c + 2], v[hf][1][4 * c + 3]);
       }
       fence_proxy_async_smem();
       __syncwarp();
@@ -532,7 +571,7 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       const uint32_t b = sm.bar(i);
       uint32_t count = 1;
       if (b == sm.q_full(0) || b == sm.q_full(1)) count = 32;  // every producer lane
-      if (b == sm.p_ready()) count = 8;
+      if (b == sm.p_ready() || b == sm.ds_ready()) count = 8;
       if (b == sm.dq_free() || b == sm.ds_free()) count = 4;
       mbar_init(b, count);
     }
@@ -554,18 +593,26 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   tc_fence_after();
   const uint32_t tmem = *sm.tmem_slot();
 
+  // register split of the 512 x 128 launch budget: element-wise warpgroups 144,
+  // the drain 176 (a whole dQ row in registers), load/MMA 48
+  // (2 x 128 x 144 + 128 x 176 + 128 x 48 = 65536)
   if (warp < kWarpDrain) {
+    setmaxnreg_inc<144>();
     bool ok = softmax_grad_role<D, CAUSAL>(sm, tmem, prm, w);
     ok = epilogue<D>(sm, tmem, &tm_dk, &tm_dv, prm, w, ok);
     if (!ok && lane == 0) atomicOr(&g_status_bwd, kStatusTimeout);
   } else if (warp < kWarpLoad) {
+    setmaxnreg_inc<176>();
     const bool ok = dq_drain_role<D>(sm, tmem, &tm_dq, prm, w);
     if (!ok && lane == 0) atomicOr(&g_status_bwd, kStatusTimeout);
-  } else if (warp == kWarpLoad) {
-    producer_role<D>(sm, &tm_q, &tm_k, &tm_v, &tm_do, prm, w, lane);
-  } else if (warp == kWarpMma) {
-    if (lane == 0) mma_role<D>(sm, tmem, w, prm.timeout_ns);
-    __syncwarp();
+  } else {
+    setmaxnreg_dec<48>();
+    if (warp == kWarpLoad) {
+      producer_role<D>(sm, &tm_q, &tm_k, &tm_v, &tm_do, prm, w, lane);
+    } else if (warp == kWarpMma) {
+      if (lane == 0) mma_role<D>(sm, tmem, w, prm.timeout_ns);
+      __syncwarp();
+    }
   }
 
   tc_fence_before();

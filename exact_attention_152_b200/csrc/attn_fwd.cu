@@ -1021,7 +1021,9 @@ int varlen_impl(const void* q, const void* k, const void* v, void* o, float* lse
   prm.wl = wl;
   prm.wr = wr;
   prm.grouped = (wl == kUnbounded && wr == 0) ? 1 : 0;
-  prm.hgroup = heads_per_l2_group(static_cast<double>(total_k) / num_seqs, d, prm.group, BH);
+  // L2 grouping sized by the longest sequence (max_seqlen_q bounds the causal
+  // key count; the average would let groups of long sequences overflow L2)
+  prm.hgroup = heads_per_l2_group(static_cast<double>(std::min(max_seqlen_q, total_k)), d, prm.group, BH);
   prm.n_qblocks = static_cast<int>(n_qblocks);
   prm.scale_log2 = scale * kLog2e;
   prm.tau = kDefaultThreshold;
