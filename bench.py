@@ -76,34 +76,40 @@ def load_peaks():
         return {"burst": 1590.0, "sustained": 1400.0, "hbm_gbs": 6650.0, "source": "fallback"}
 
 
-def kernel_source_hash():
-    """Hash of the CUDA sources with comments and whitespace removed, so that a
-    recorded ncu capture stays attached to the code it measured."""
+# The sources each timed kernel is built from: a recorded ncu capture stays
+# attached to exactly this code.
+KERNEL_SOURCES = {
+    "fwd": ("attn_fwd.cu", "sm100.cuh", "exp2.cuh", "tmap.h", "host_common.h"),
+    "bwd": ("attn_bwd.cu", "sm100.cuh", "exp2.cuh", "tmap.h", "host_common.h"),
+}
+
+
+def kernel_source_hash(kind="fwd"):
+    """Hash of a kernel's CUDA sources with comments and whitespace removed."""
     import re
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "exact_attention_152_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
-        if name.endswith((".cu", ".cuh", ".h")):
-            with open(os.path.join(csrc, name)) as f:
-                src = f.read()
-            src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
-            src = re.sub(r"//[^\n]*", "", src)
-            src = "".join(src.split())
-            h.update(name.encode() + b"\0" + src.encode())
+    for name in KERNEL_SOURCES[kind]:
+        with open(os.path.join(csrc, name)) as f:
+            src = f.read()
+        src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+        src = re.sub(r"//[^\n]*", "", src)
+        src = "".join(src.split())
+        h.update(name.encode() + b"\0" + src.encode())
     return h.hexdigest()[:16]
 
 
-def recorded_traffic(workload_name):
-    """DRAM bytes per launch from a committed ncu summary, if it was taken on
-    the current kernel source; else None."""
+def recorded_traffic(workload_name, kind="fwd"):
+    """DRAM bytes per launch of the timed kernel from a committed ncu summary,
+    if it was taken on the current kernel source; else None."""
     path = os.path.join(ROOT, "profiles", "ncu_traffic.json")
     try:
         with open(path) as f:
             rec = json.load(f)
     except Exception:
         return None
-    e = rec.get(workload_name)
-    if not e or e.get("kernel_src_sha") != kernel_source_hash():
+    e = rec.get(f"{kind}:{workload_name}")
+    if not e or e.get("kernel_src_sha") != kernel_source_hash(kind):
         return None
     return e.get("dram_bytes_per_launch")
 
@@ -455,7 +461,7 @@ def run_ours(args):
         "config": workload_config(w, world),
         "pct_of_dense_spec": 100.0 * value / world / (SPEC_DENSE_BF16_TFLOPS * ratio),
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": UNIT,
-                     "frac": achieved / peak, "traffic": recorded_traffic(w.name),
+                     "frac": achieved / peak, "traffic": recorded_traffic(w.name, "fwd"),
                      "peak_kind": (f"bf16_tflops_sustained ({peaks['source']})"
                                    + (" x 2 (nominal E4M3/BF16 dense ratio)" if w.fp8 else "")
                                    + ": back-to-back launches for seconds under the power cap"),
@@ -468,7 +474,7 @@ def run_ours(args):
                         f"{launch_name(w)} (C-ABI) -> D2H of O and LSE"},
         "gpu_launches": K,
         "clocks": clocks,
-        "kernel_src_sha": kernel_source_hash(),
+        "kernel_src_sha": kernel_source_hash("fwd"),
     }
     if knobs:
         line["config"]["rescale_threshold"] = thr
@@ -596,7 +602,7 @@ def run_ours_bwd(args):
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": dict(workload_config(w, 1), **{"pass": "bwd", "dO": "N(0,1), seed + 1"}),
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": UNIT,
-                     "frac": achieved / peak, "traffic": None,
+                     "frac": achieved / peak, "traffic": recorded_traffic(w.name, "bwd"),
                      "peak_kind": f"bf16_tflops_sustained ({peaks['source']})",
                      "frac_of_burst": achieved / peaks["burst"],
                      "frac_of_spec_2250": achieved / SPEC_DENSE_BF16_TFLOPS,
@@ -610,7 +616,7 @@ def run_ours_bwd(args):
                 "path": "pinned host Q/K/V/O/dO/LSE -> H2D -> attn_bwd (C-ABI) -> D2H of dQ/dK/dV"},
         "gpu_launches": 3 * K,
         "clocks": clocks,
-        "kernel_src_sha": kernel_source_hash(),
+        "kernel_src_sha": kernel_source_hash("bwd"),
     }
     print(json.dumps(line), flush=True)
     return 0
