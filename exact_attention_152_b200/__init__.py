@@ -12,7 +12,7 @@ from __future__ import annotations
 __all__ = [
     "attn_fwd", "attn_fwd_config", "attn_fwd_gqa", "attn_fwd_window", "attn_fwd_varlen",
     "attn_status_sync", "attn_status_string", "attn_last_error", "attn_selftest_timeout", "fwd",
-    "fwd_varlen", "attn_fwd_fp8", "fwd_fp8", "attn_bwd", "attn_bwd_workspace_size", "bwd", "AttnError",
+    "fwd_varlen", "attn_fwd_fp8", "fwd_fp8", "attn_bwd", "attn_bwd_window", "attn_bwd_workspace_size", "bwd", "AttnError",
 ]
 
 

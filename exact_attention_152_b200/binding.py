@@ -58,6 +58,8 @@ def lib() -> ctypes.CDLL:
             l.attn_fwd_fp8.restype = _I
             l.attn_bwd.argtypes = [_P] * 10 + [ctypes.c_size_t] + [_I] * 6 + [ctypes.c_float, _I, _P]
             l.attn_bwd.restype = _I
+            l.attn_bwd_window.argtypes = [_P] * 10 + [ctypes.c_size_t] + [_I] * 6 + [ctypes.c_float, _I, _I, _P]
+            l.attn_bwd_window.restype = _I
             l.attn_bwd_noalloc.argtypes = [_P] * 9 + [_I] * 6 + [ctypes.c_float, _I, _P]
             l.attn_bwd_noalloc.restype = _I
             l.attn_bwd_workspace_size.argtypes = [_I, _I, _I, _I]
@@ -111,6 +113,12 @@ def attn_bwd(q, k, v, o, dout, lse, dq, dk, dv, workspace, workspace_bytes, B, H
              scale, causal, stream) -> int:
     return lib().attn_bwd(q, k, v, o, dout, lse, dq, dk, dv, workspace, workspace_bytes, B, H, Hkv,
                           Nq, Nk, d, scale, causal, stream)
+
+
+def attn_bwd_window(q, k, v, o, dout, lse, dq, dk, dv, workspace, workspace_bytes, B, H, Hkv, Nq, Nk,
+                    d, scale, window_left, window_right, stream) -> int:
+    return lib().attn_bwd_window(q, k, v, o, dout, lse, dq, dk, dv, workspace, workspace_bytes, B, H,
+                                 Hkv, Nq, Nk, d, scale, window_left, window_right, stream)
 
 
 def attn_bwd_noalloc(q, k, v, o, dout, lse, dq, dk, dv, B, H, Hkv, Nq, Nk, d, scale, causal,
@@ -262,11 +270,12 @@ def fwd_varlen(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q: int, causal: b
 
 
 def bwd(q, k, v, o, dout, lse, causal: bool = False, scale: float | None = None, *,
-        workspace=None):
+        window=None, workspace=None):
     """Gradients (dq, dk, dv) for BF16 CUDA tensors q/o/dout [B,H,Nq,d], k/v
-    [B,Hkv,Nk,d] and the forward's fp32 lse [B,H,Nq].  The workspace (a uint8
-    CUDA tensor of at least attn_bwd_workspace_size bytes) is allocated with
-    torch when not given.  Runs on torch's current stream."""
+    [B,Hkv,Nk,d] and the forward's fp32 lse [B,H,Nq].  window=(left, right)
+    selects the key band of attn_bwd_window (it replaces ``causal``).  The
+    workspace (a uint8 CUDA tensor of at least attn_bwd_workspace_size bytes)
+    is allocated with torch when not given.  Runs on torch's current stream."""
     import torch
 
     _check_bf16(q=q, k=k, v=v, o=o, dout=dout)
@@ -287,11 +296,18 @@ def bwd(q, k, v, o, dout, lse, causal: bool = False, scale: float | None = None,
     dk = torch.empty_like(k)
     dv = torch.empty_like(v)
     stream = torch.cuda.current_stream(q.device).cuda_stream
-    rc = attn_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), dout.data_ptr(),
-                  lse.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), workspace.data_ptr(),
-                  workspace.numel() * workspace.element_size(), B, H, Hkv, Nq, Nk, d, float(scale),
-                  int(bool(causal)), stream)
-    check(rc, "attn_bwd")
+    ptrs = (q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), dout.data_ptr(), lse.data_ptr(),
+            dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), workspace.data_ptr(),
+            workspace.numel() * workspace.element_size())
+    if window is not None:
+        if causal:
+            raise ValueError("window replaces causal")
+        rc = attn_bwd_window(*ptrs, B, H, Hkv, Nq, Nk, d, float(scale), int(window[0]),
+                             int(window[1]), stream)
+        check(rc, "attn_bwd_window")
+    else:
+        rc = attn_bwd(*ptrs, B, H, Hkv, Nq, Nk, d, float(scale), int(bool(causal)), stream)
+        check(rc, "attn_bwd")
     return dq, dk, dv
 
 

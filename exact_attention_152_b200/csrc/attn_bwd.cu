@@ -20,8 +20,9 @@
 //    D and the dQ accumulator live in a caller-provided workspace.
 //  * Main kernel: one CTA per (b, key/value head, 128-key block).  K and V of
 //    the block stay in shared memory; the CTA walks every query tile (128
-//    rows) of every query head that reads this key/value head (causal: only
-//    tiles at or below the diagonal), double-buffering Q and dO by TMA.
+//    rows) of every query head that reads this key/value head (with a key
+//    band such as causal, only the tiles whose queries see one of the block's
+//    keys), double-buffering Q and dO by TMA.
 //  * Per query tile, five BF16 GEMMs on the tensor cores, all with M = 128
 //    keys or queries:
 //        S^T  = K Q^T          (keys x queries, TMEM columns [0, 128))
@@ -66,6 +67,7 @@ constexpr int kNumThreads = 512;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint64_t kWaitTimeoutNs = 2000000000ull;
 constexpr float kLog2e = 1.4426950408889634f;
+constexpr int kUnbounded = 1 << 30;  // "no bound" for a side of the key band
 
 constexpr unsigned int kStatusTimeout = kStatusWordTimeout;
 constexpr unsigned int kStatusSmemAlign = 4u;  // mapped to kStatusWordLaunch on the host
@@ -102,7 +104,7 @@ struct BwdParams {
   float* dq_acc;       // [B*H, Nq, d] fp32, zeroed before the launch
   uint64_t timeout_ns;
   int Nq, Nk, H, group, n_kblocks, n_qtiles;
-  int causal;
+  int wl, wr;          // key band i - wl <= j <= i + wr (kUnbounded: no bound)
   float scale_log2;    // scale * log2(e)
   float scale;
 };
@@ -141,7 +143,8 @@ struct Smem {
 };
 
 // The work of one CTA: key block j of key/value head bh_kv; iterations walk the
-// group's query heads, and within each its query tiles i_lo .. n_qtiles-1.
+// group's query heads, and within each the query tiles i_lo .. i_lo +
+// tiles_per_head - 1 that can see one of the block's keys.
 struct Work {
   int bh_kv, j, b, hkv, i_lo, tiles_per_head, n_it;
   __device__ __forceinline__ int head_of(int it) const { return it / tiles_per_head; }
@@ -309,7 +312,7 @@ __device__ __forceinline__ void mma_role(const Smem<D>& sm, uint32_t tmem, const
 // Warps 0-7: P^T and dS^T from S^T and dP^T.  Warp (c, q) owns TMEM lanes
 // 32q..32q+31 (keys) and query columns [64c, 64c+64).
 // ---------------------------------------------------------------------------
-template <int D, bool CAUSAL>
+template <int D, bool MASK>
 __device__ __forceinline__ bool softmax_grad_role(const Smem<D>& sm, uint32_t tmem,
                                                   const BwdParams& prm, const Work& w) {
   using C = Cfg<D>;
@@ -334,8 +337,10 @@ __device__ __forceinline__ bool softmax_grad_role(const Smem<D>& sm, uint32_t tm
     if (!ok) break;
     tc_fence_after();
     const int q_base = w.tile_of(it) * kBlockQ + c * 64;  // first query of this warp's columns
-    // masking: key tail, or (causal) a key past some query of the block
-    const bool masked = !key_in || (CAUSAL && w.j * kBlockK + q4 * 32 + 31 > q_base);
+    // masking: key tail, or a band edge crossing this warp's 32 keys x 64 queries
+    const int k_lo = w.j * kBlockK + q4 * 32;
+    const bool masked = !key_in ||
+                        (MASK && (k_lo + 31 - q_base > prm.wr || q_base + 63 - k_lo > prm.wl));
     const float4* nl4 = reinterpret_cast<const float4*>(sm.lse2(s) + c * 64);
     const float4* dd4 = reinterpret_cast<const float4*>(sm.dsum(s) + c * 64);
     const float2 sl2 = make_float2(prm.scale_log2, prm.scale_log2);
@@ -357,11 +362,15 @@ __device__ __forceinline__ bool softmax_grad_role(const Smem<D>& sm, uint32_t tm
         float2 xb = ffma2(make_float2(__uint_as_float(sv[4 * g + 2]), __uint_as_float(sv[4 * g + 3])),
                           sl2, make_float2(nl.z, nl.w));
         if (masked) {
-          const int col = q_base + 32 * k + 4 * g;
-          if (!key_in || (CAUSAL && key > col)) xa.x = -INFINITY;
-          if (!key_in || (CAUSAL && key > col + 1)) xa.y = -INFINITY;
-          if (!key_in || (CAUSAL && key > col + 2)) xb.x = -INFINITY;
-          if (!key_in || (CAUSAL && key > col + 3)) xb.y = -INFINITY;
+          // query q = q_base + 32k + 4g + e is outside the band of this key when
+          // key - q > wr or q - key > wl; with d0 = key - (q_base + 32k + 4g):
+          // d0 - e > wr or e - d0 > wl
+          const int d0 = key - (q_base + 32 * k + 4 * g);
+          const int hi = prm.wr, lo = -prm.wl;  // visible iff lo <= d0 - e <= hi
+          if (!key_in || d0 > hi || d0 < lo) xa.x = -INFINITY;
+          if (!key_in || d0 - 1 > hi || d0 - 1 < lo) xa.y = -INFINITY;
+          if (!key_in || d0 - 2 > hi || d0 - 2 < lo) xb.x = -INFINITY;
+          if (!key_in || d0 - 3 > hi || d0 - 3 < lo) xb.y = -INFINITY;
         }
         float2 pa, pb;
         if ((g & 3) == 0) {  // a quarter of the exponentials on the FMA pipe
@@ -535,7 +544,7 @@ __device__ __forceinline__ bool epilogue(const Smem<D>& sm, uint32_t tmem, const
   return true;
 }
 
-template <int D, bool CAUSAL>
+template <int D, bool MASK>
 __global__ void __launch_bounds__(kNumThreads, 1)
 attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                 const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
@@ -560,10 +569,23 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   const int hkv_per_b = prm.H / prm.group;
   w.b = w.bh_kv / hkv_per_b;
   w.hkv = w.bh_kv % hkv_per_b;
-  // causal: query tiles from the diagonal on (tile i holds a visible pair iff
-  // its last query >= the block's first key)
-  w.i_lo = CAUSAL ? (w.j * kBlockK) / kBlockQ : 0;
-  w.tiles_per_head = prm.n_qtiles - w.i_lo;
+  // query tiles that can see a key of this block: i - wl <= j <= i + wr for
+  // some key j in [j0, j0 + 127] and query i of the tile; a block no query
+  // sees still runs one fully masked tile, so dK = dV = 0 come out of TMEM
+  w.i_lo = 0;
+  w.tiles_per_head = prm.n_qtiles;
+  if (MASK) {
+    const long long j0 = static_cast<long long>(w.j) * kBlockK;
+    long long lo = 0, hi = prm.n_qtiles - 1;
+    if (prm.wr < kUnbounded && j0 - prm.wr > 0) lo = (j0 - prm.wr) / kBlockQ;
+    if (prm.wl < kUnbounded) {
+      const long long last = (j0 + kBlockK - 1 + prm.wl) / kBlockQ;
+      if (last < hi) hi = last;
+    }
+    if (lo > hi) lo = hi = (lo < prm.n_qtiles - 1 ? lo : prm.n_qtiles - 1);
+    w.i_lo = static_cast<int>(lo);
+    w.tiles_per_head = static_cast<int>(hi - lo + 1);
+  }
   w.n_it = prm.group * w.tiles_per_head;
 
   if (threadIdx.x == 0) {
@@ -598,7 +620,7 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   // (2 x 128 x 144 + 128 x 176 + 128 x 48 = 65536)
   if (warp < kWarpDrain) {
     setmaxnreg_inc<144>();
-    bool ok = softmax_grad_role<D, CAUSAL>(sm, tmem, prm, w);
+    bool ok = softmax_grad_role<D, MASK>(sm, tmem, prm, w);
     ok = epilogue<D>(sm, tmem, &tm_dk, &tm_dv, prm, w, ok);
     if (!ok && lane == 0) atomicOr(&g_status_bwd, kStatusTimeout);
   } else if (warp < kWarpLoad) {
@@ -655,9 +677,9 @@ __global__ void dq_finish_kernel(const float4* __restrict__ acc, uint2* __restri
   }
 }
 
-template <int D, bool CAUSAL>
+template <int D, bool MASK>
 int launch_main(const CUtensorMap* maps, const BwdParams& prm, int grid, cudaStream_t stream) {
-  auto kern = attn_bwd_kernel<D, CAUSAL>;
+  auto kern = attn_bwd_kernel<D, MASK>;
   static std::once_flag once[kMaxDeviceCount];
   static cudaError_t err[kMaxDeviceCount];
   int dev = 0;
@@ -680,15 +702,16 @@ size_t workspace_bytes(long long BH, long long Nq, int d) {
   return align256(static_cast<size_t>(BH) * Nq * 4) + static_cast<size_t>(BH) * Nq * d * 4;
 }
 
+// window_left / window_right: the key band of the forward (-1 = no bound).
 int bwd_impl(const void* q, const void* k, const void* v, const void* o, const void* dout,
              const float* lse, void* dq, void* dk, void* dv, void* workspace, size_t ws_bytes, int B,
-             int H, int Hkv, int Nq, int Nk, int d, float scale, int causal, cudaStream_t stream) {
+             int H, int Hkv, int Nq, int Nk, int d, float scale, int window_left, int window_right,
+             cudaStream_t stream) {
   if (B < 0 || H < 0 || Hkv < 0 || Nq < 0 || Nk < 0) return ATTN_ERR_INVALID_ARG;
   if (H > 0 && (Hkv == 0 || H % Hkv != 0)) return ATTN_ERR_INVALID_ARG;
   if (!std::isfinite(scale)) return ATTN_ERR_INVALID_ARG;
-  if (causal != 0 && causal != 1) return ATTN_ERR_INVALID_ARG;
+  if (window_left < -1 || window_right < -1) return ATTN_ERR_INVALID_ARG;
   if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
-  if (causal && Nq != Nk) return ATTN_ERR_UNSUPPORTED;
   const long long BH = static_cast<long long>(B) * H, BHkv = static_cast<long long>(B) * Hkv;
   if (BH > 0x7fffffffLL) return ATTN_ERR_INVALID_ARG;
   const size_t q_bytes = static_cast<size_t>(BH) * Nq * d * 2;
@@ -773,14 +796,16 @@ int bwd_impl(const void* q, const void* k, const void* v, const void* o, const v
   prm.group = H / Hkv;
   prm.n_kblocks = static_cast<int>(n_kblocks);
   prm.n_qtiles = (Nq + kBlockQ - 1) / kBlockQ;
-  prm.causal = causal;
+  prm.wl = window_left < 0 ? kUnbounded : std::min(window_left, kUnbounded);
+  prm.wr = window_right < 0 ? kUnbounded : std::min(window_right, kUnbounded);
+  const bool mask = prm.wl < kUnbounded || prm.wr < kUnbounded;
   prm.scale_log2 = scale * kLog2e;
   prm.scale = scale;
   const int grid = static_cast<int>(n_kblocks * BHkv);
   if (d == 128)
-    rc = causal ? launch_main<128, true>(maps, prm, grid, stream) : launch_main<128, false>(maps, prm, grid, stream);
+    rc = mask ? launch_main<128, true>(maps, prm, grid, stream) : launch_main<128, false>(maps, prm, grid, stream);
   else
-    rc = causal ? launch_main<64, true>(maps, prm, grid, stream) : launch_main<64, false>(maps, prm, grid, stream);
+    rc = mask ? launch_main<64, true>(maps, prm, grid, stream) : launch_main<64, false>(maps, prm, grid, stream);
   if (rc != ATTN_OK) return rc;
 
   const size_t n4 = rows * d / 4;
@@ -846,8 +871,18 @@ int attn_bwd(const void* q, const void* k, const void* v, const void* o, const v
              const float* lse, void* dq, void* dk, void* dv, void* workspace,
              size_t workspace_bytes, int B, int H, int Hkv, int Nq, int Nk, int d, float scale,
              int causal, cudaStream_t stream) {
+  if (causal != 0 && causal != 1) return ATTN_ERR_INVALID_ARG;
+  if (causal && Nq != Nk) return ATTN_ERR_UNSUPPORTED;
   return eab::bwd::bwd_impl(q, k, v, o, dout, lse, dq, dk, dv, workspace, workspace_bytes, B, H, Hkv,
-                            Nq, Nk, d, scale, causal, stream);
+                            Nq, Nk, d, scale, -1, causal ? 0 : -1, stream);
+}
+
+int attn_bwd_window(const void* q, const void* k, const void* v, const void* o, const void* dout,
+                    const float* lse, void* dq, void* dk, void* dv, void* workspace,
+                    size_t workspace_bytes, int B, int H, int Hkv, int Nq, int Nk, int d,
+                    float scale, int window_left, int window_right, cudaStream_t stream) {
+  return eab::bwd::bwd_impl(q, k, v, o, dout, lse, dq, dk, dv, workspace, workspace_bytes, B, H, Hkv,
+                            Nq, Nk, d, scale, window_left, window_right, stream);
 }
 
 int attn_bwd_noalloc(const void* q, const void* k, const void* v, const void* o, const void* dout,
@@ -857,11 +892,13 @@ int attn_bwd_noalloc(const void* q, const void* k, const void* v, const void* o,
   if (B >= 0 && H >= 0 && Nq >= 0 && (d == 64 || d == 128) &&
       eab::bwd::workspace_bytes(static_cast<long long>(B) * H, Nq, d) > eab::bwd::kStaticScratchBytes)
     return ATTN_ERR_UNSUPPORTED;
+  if (causal != 0 && causal != 1) return ATTN_ERR_INVALID_ARG;
+  if (causal && Nq != Nk) return ATTN_ERR_UNSUPPORTED;
   void* ws = nullptr;
   const int rc = eab::bwd::static_scratch(&ws);
   if (rc != ATTN_OK) return rc;
   return eab::bwd::bwd_impl(q, k, v, o, dout, lse, dq, dk, dv, ws, eab::bwd::kStaticScratchBytes, B, H,
-                            Hkv, Nq, Nk, d, scale, causal, stream);
+                            Hkv, Nq, Nk, d, scale, -1, causal ? 0 : -1, stream);
 }
 
 }  // extern "C"

@@ -218,6 +218,19 @@ int attn_bwd(const void *q, const void *k, const void *v, const void *o, const v
              size_t workspace_bytes, int B, int H, int Hkv, int Nq, int Nk, int d, float scale,
              int causal, cudaStream_t stream);
 
+/*
+ * attn_bwd for the key band of attn_fwd_window: key j is visible to query i
+ * when i - window_left <= j <= i + window_right (-1: no bound on that side;
+ * (-1, 0) is causal, (-1, -1) unmasked), positions counted from 0 for queries
+ * and keys alike, so Nq != Nk is allowed.  Keys no query sees get dK = dV = 0.
+ * window_left, window_right below -1 return ATTN_ERR_INVALID_ARG; everything
+ * else is as attn_bwd (lse must come from attn_fwd_window with the same band).
+ */
+int attn_bwd_window(const void *q, const void *k, const void *v, const void *o, const void *dout,
+                    const float *lse, void *dq, void *dk, void *dv, void *workspace,
+                    size_t workspace_bytes, int B, int H, int Hkv, int Nq, int Nk, int d,
+                    float scale, int window_left, int window_right, cudaStream_t stream);
+
 /* Workspace bytes attn_bwd needs (0 for d not in {64, 128} or negative sizes). */
 size_t attn_bwd_workspace_size(int B, int H, int Nq, int d);
 

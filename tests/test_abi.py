@@ -49,7 +49,7 @@ def test_library_exports_every_declared_symbol(header):
 def test_attn_h_declares_the_contract():
     names = declared_functions(os.path.join(ROOT, "include", "attn.h"))
     for n in ("attn_fwd", "attn_fwd_config", "attn_fwd_gqa", "attn_fwd_window", "attn_fwd_varlen",
-              "attn_fwd_fp8", "attn_bwd", "attn_bwd_noalloc", "attn_bwd_workspace_size", "attn_status_sync", "attn_status_string",
+              "attn_fwd_fp8", "attn_bwd", "attn_bwd_window", "attn_bwd_noalloc", "attn_bwd_workspace_size", "attn_status_sync", "attn_status_string",
               "attn_last_error", "attn_selftest_timeout"):
         assert n in names
 
@@ -174,6 +174,10 @@ def test_bwd_validation():
     assert Bw(*ptrs[:6], A, *ptrs[7:], need, *sizes, None) == 1   # dq overlaps q
     assert Bw(*ptrs[:9], A * 9, need, *sizes, None) == 1         # workspace overlaps dv
     assert Bw(*(None,) * 10, 0, 0, 2, 2, 64, 64, 64, 0.1, 0, None) == 0   # empty batch
+    BW = binding.attn_bwd_window
+    assert BW(*ptrs, need, 1, 2, 2, 64, 64, 64, 0.1, -2, 0, None) == 1    # band below -1
+    assert BW(*ptrs, need, 1, 2, 2, 64, 64, 64, 0.1, 0, -3, None) == 1
+    assert BW(*ptrs, need - 1, 1, 2, 2, 64, 64, 64, 0.1, 8, 0, None) == 1  # workspace too small
 
 
 def test_config_knob_validation():

@@ -47,6 +47,12 @@ def run_fwd_bwd(q_bits, k_bits, v_bits, do_bits, scale, causal):
 
 
 def check_grads(got, ref, label=""):
+    """Norm-wise and element-wise bounds per gradient.  A gradient that is zero
+    in exact arithmetic (a band where every query sees one key: the softmax is
+    constant) still carries fp32 rounding from P and D = <dO, O>; the floor of
+    each bound is therefore 1e-4 of the largest gradient of the problem."""
+    scale_nrm = max(np.linalg.norm(r) for r in ref)
+    scale_max = max(np.abs(r).max() if r.size else 0.0 for r in ref)
     for name, g, r in zip(("dq", "dk", "dv"), got, ref):
         g = g.astype(np.float64)
         err = np.linalg.norm(g - r)
@@ -54,8 +60,8 @@ def check_grads(got, ref, label=""):
         mx = np.abs(g - r).max() if r.size else 0.0
         print(label, name, "rel_fro", err / max(nrm, 1e-30), "max_abs", mx, "ref_max", np.abs(r).max())
         assert np.all(np.isfinite(g)), name
-        assert err <= REL_FRO * nrm + 1e-6, (label, name, err, nrm)
-        assert mx <= REL_MAX * np.abs(r).max() + 1e-6, (label, name, mx)
+        assert err <= REL_FRO * nrm + 1e-4 * scale_nrm + 1e-6, (label, name, err, nrm)
+        assert mx <= REL_MAX * np.abs(r).max() + 1e-4 * scale_max + 1e-6, (label, name, mx)
 
 
 @pytest.mark.parametrize("case", CASES, ids=[str(c) for c in CASES])
@@ -129,3 +135,54 @@ def test_bwd_workload_sampled():
         ref = oracle.attn_bwd(f(q[b:b + 1, h:h + 1]), f(k[b:b + 1, h:h + 1]), f(v[b:b + 1, h:h + 1]),
                               f(do[b:b + 1, h:h + 1]), scale, -1, 0)
         check_grads(tuple(g[b:b + 1, h:h + 1] for g in got), ref, f"head {(b, h)}")
+
+
+BAND_CASES = [
+    # B, H, Hkv, Nq, Nk, d, (window_left, window_right)
+    (1, 2, 2, 384, 384, 128, (63, 0)),        # causal sliding window
+    (1, 2, 2, 300, 300, 64, (100, 50)),
+    (1, 2, 2, 257, 257, 128, (0, 0)),          # diagonal only
+    (1, 4, 2, 520, 520, 128, (-1, 10)),
+    (1, 2, 2, 200, 517, 128, (10, 300)),       # Nq < Nk
+    (1, 2, 2, 600, 100, 64, (50, 0)),          # Nq > Nk: rows >= 150 and some keys see nothing
+    (2, 2, 1, 1024, 1024, 128, (255, 0)),
+]
+
+
+@pytest.mark.parametrize("case", BAND_CASES, ids=[str(c) for c in BAND_CASES])
+def test_bwd_band_parity(case):
+    import torch
+    from exact_attention_152_b200 import binding
+    B, H, Hkv, Nq, Nk, d, (wl, wr) = case
+    seed = 340 + Nq + Nk + d + wl
+    q = harness.random_bits(seed, (B, H, Nq, d), tensor="q")
+    k = harness.random_bits(seed, (B, Hkv, Nk, d), tensor="k")
+    v = harness.random_bits(seed, (B, Hkv, Nk, d), tensor="v")
+    do = harness.random_bits(seed + 1, (B, H, Nq, d), tensor="q")
+    scale = float(np.float32(1 / math.sqrt(d)))
+    qd, kd, vd, dod = (harness.to_device_bf16(x) for x in (q, k, v, do))
+    o, lse = binding.fwd(qd, kd, vd, scale=scale, window=(wl, wr))
+    got = binding.bwd(qd, kd, vd, o, dod, lse, scale=scale, window=(wl, wr))
+    assert binding.attn_status_sync(torch.cuda.current_stream().cuda_stream) == 0
+    got = tuple(x.float().cpu().numpy() for x in got)
+    f = inputs.bf16_bits_to_f64
+    ref = oracle.attn_bwd(f(q), f(k), f(v), f(do), scale, wl, wr)
+    check_grads(got, ref, str(case))
+
+
+def test_bwd_band_limits_equal_causal_and_full_bitwise():
+    """Band (-1, 0) is the causal backward and (-1, -1) the unmasked one, bit for
+    bit for dK and dV (dQ: the fp32 reductions may reorder)."""
+    import torch
+    from exact_attention_152_b200 import binding
+    B, H, N, d = 1, 4, 640, 128
+    q, k, v, do = (harness.to_device_bf16(harness.random_bits(350, (B, H, N, d), tensor=t))
+                   for t in ("q", "k", "v", "v"))
+    for causal, band in ((True, (-1, 0)), (False, (-1, -1))):
+        o, lse = binding.fwd(q, k, v, causal=causal)
+        a = binding.bwd(q, k, v, o, do, lse, causal=causal)
+        b = binding.bwd(q, k, v, o, do, lse, window=band)
+        torch.cuda.synchronize()
+        assert torch.equal(a[1].view(torch.int16), b[1].view(torch.int16))
+        assert torch.equal(a[2].view(torch.int16), b[2].view(torch.int16))
+        assert torch.allclose(a[0].float(), b[0].float(), rtol=1e-2, atol=1e-3)
