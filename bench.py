@@ -257,6 +257,33 @@ def workload_config(w, n_gpus):
     return cfg
 
 
+def run_reference_bwd(args, w, per_step):
+    """Reference arm of --pass bwd: the oracle's backward, each step on the
+    first n query rows of one head against all its keys (n sized to about
+    per_step seconds), in the same metric (2.5x the forward's FLOPs)."""
+    import oracle
+    for _ in range(args.warmup):
+        bwd_cpu_baseline(w, per_step)
+    vals, secs = [], []
+    for _ in range(args.steps):
+        t0 = time.perf_counter()
+        r = bwd_cpu_baseline(w, per_step)
+        secs.append(time.perf_counter() - t0)
+        vals.append(r["value"])
+    value = statistics.mean(vals)
+    line = {
+        "impl": "reference", "metric": METRIC_BWD, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": statistics.mean(secs) * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": dict(workload_config(w, 1), **{"pass": "bwd"}),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle",
+                         "sample": r["sample"]},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def launch_name(w):
     if w.fp8:
         return "attn_fwd_fp8"
@@ -276,6 +303,8 @@ def run_reference(args):
     w = WORKLOADS[args.workload or HEADLINE]
     budget = 150.0  # seconds for warmup + timed steps together
     per_step = budget / max(1, args.steps + args.warmup)
+    if args.which == "bwd":
+        return run_reference_bwd(args, w, per_step)
     n = calibrate_rows(w, per_step)
     for i in range(args.warmup):
         time_oracle_rows(w, n, 3000 + i)

@@ -75,7 +75,6 @@ constexpr int kRowsPerCta = 2 * kBlockM;
 // 5 warpgroups: 4 softmax warpgroups (tile t, key half h -> warps 8t+4h .. 8t+4h+3)
 // and one for the TMA producer (warp 16), the MMA issuer (warp 17) and two idle
 // warps that complete the group for the register split.
-constexpr int kNumSoftmaxWarps = 16;
 constexpr int kWarpLoad = 16;
 constexpr int kWarpMma = 17;
 constexpr int kNumThreads = 640;
@@ -172,12 +171,6 @@ __device__ __forceinline__ void tma_load_rows(uint32_t dst, const CUtensorMap* t
                                               int head, bool packed, uint32_t bar) {
   if (packed) tma_load_3d(dst, tm, col, head, row, bar);
   else tma_load_3d(dst, tm, col, row, head, bar);
-}
-
-template <int POLY16>
-__device__ __forceinline__ float ex2_split(float x, int col) {
-  if ((col & 15) < POLY16) return ex2_poly(x);
-  return ex2_mufu(x);
 }
 
 // ---------------------------------------------------------------------------
