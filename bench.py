@@ -198,10 +198,11 @@ def time_oracle_rows(w, n_rows, seed_off):
     """Time the oracle on n_rows seeded query rows, taken unit by unit (all rows
     of a head, then the next) so large samples span several heads."""
     import oracle
-    from exact_attention_152_b200 import inputs
+    from exact_attention_152_b200 import inputs, masks
     from exact_attention_152_b200.workloads import visible_keys
     tot_t, tot_f, done, units = 0.0, 0.0, 0, 0
     wl, wr = w.band
+    cols_all = w.colmask_array() if w.colmask else None
     for i, (tag, nq, nk, load_kv) in enumerate(oracle_units(w)):
         if done >= n_rows:
             break
@@ -211,10 +212,17 @@ def time_oracle_rows(w, n_rows, seed_off):
             q = w.to_f64("q", w.seq_head_bits("q", tag[0], tag[1], rows))
         else:
             q = w.to_f64("q", w.q_rows_bits(tag, rows))
-        t0 = time.perf_counter()
-        oracle.attn_rows_window(q, rows, k, v, w.scale, wl, wr)
-        tot_t += time.perf_counter() - t0
-        tot_f += 4.0 * w.d * float(visible_keys(rows, nk, wl, wr).sum())
+        if cols_all is not None:
+            cols = cols_all[tag // w.H, 0]
+            t0 = time.perf_counter()
+            oracle.attn_rows_colmask(q, rows, k, v, w.scale, w.causal, cols)
+            tot_t += time.perf_counter() - t0
+            tot_f += 4.0 * w.d * float(masks.visible_per_row(cols, rows, w.causal).sum())
+        else:
+            t0 = time.perf_counter()
+            oracle.attn_rows_window(q, rows, k, v, w.scale, wl, wr)
+            tot_t += time.perf_counter() - t0
+            tot_f += 4.0 * w.d * float(visible_keys(rows, nk, wl, wr).sum())
         done += len(rows)
         units += 1
     return tot_t, tot_f, done, units
@@ -236,8 +244,15 @@ def cpu_baseline(w, seconds):
     return {"value": flops / dt / 1e12, "unit": UNIT, "cores": oracle.default_threads(),
             "kind": "oracle",
             "sample": f"{n} seeded query rows over {heads} head(s) of {w.name} (visible keys "
-                      f"of band {w.band}), fp64, {dt:.1f} s of oracle time; "
+                      f"of {mask_words(w)}), fp64, {dt:.1f} s of oracle time; "
                       f"value = those rows' algorithmic FLOPs / time"}
+
+
+def mask_words(w):
+    if w.colmask:
+        return f"column-interval document mask, documents of {w.docs[0]}..{w.docs[1]} tokens" + \
+            (", causal" if w.causal else "")
+    return f"band {w.band}"
 
 
 def workload_config(w, n_gpus):
@@ -250,6 +265,9 @@ def workload_config(w, n_gpus):
            "l2": f"inputs {qkv_bytes / 1e6:.0f} MB {'>' if qkv_bytes > L2_BYTES else '<='} "
                  f"126 MB L2; not flushed between steps",
            "parallelism": f"independent problem per GPU x{n_gpus}"}
+    if w.colmask:
+        cfg.update({"mask": mask_words(w), "mask_layout": "int32 [B, 1, Nk, 4]",
+                    "doc_lengths": [w.doc_lengths(b) for b in range(w.B)]})
     if w.packed:
         cfg.update({"layout": "packed [total, H, d]", "num_seqs": len(w.seqlens),
                     "total_tokens": w.total, "seqlen_min": min(w.seqlens),
@@ -285,6 +303,8 @@ def run_reference_bwd(args, w, per_step):
 
 
 def launch_name(w):
+    if w.colmask:
+        return "attn_fwd_colmask"
     if w.fp8:
         return "attn_fwd_fp8"
     if w.packed:
@@ -320,7 +340,7 @@ def run_reference(args):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic", "config": workload_config(w, 1),
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": oracle.default_threads(), "kind": "oracle",
-                         "sample": f"each step: {n} seeded query rows (head by head, visible keys of band {w.band}), fp64"},
+                         "sample": f"each step: {n} seeded query rows (head by head, visible keys of {mask_words(w)}), fp64"},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -364,16 +384,28 @@ def run_ours(args):
         o = torch.empty((w.B, w.H, w.Nq, w.d), dtype=torch.bfloat16, device=dev)
         lse = torch.empty((w.B, w.H, w.Nq), dtype=torch.float32, device=dev)
         host_cu = cu = None
+    if w.colmask:
+        host_mask = torch.from_numpy(w.colmask_array())
+        mask = host_mask.to(dev)
+        ws_bytes = binding.attn_colmask_workspace_size(w.B, 1, w.Nk)
+        ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+    else:
+        host_mask = mask = None
     stream = torch.cuda.current_stream(dev)
     sh = stream.cuda_stream
     knobs = args.exp_mode is not None or args.threshold is not None
     thr = 8.0 if args.threshold is None else args.threshold
     em = 1 if args.exp_mode is None else args.exp_mode
-    if knobs and (w.packed or w.window is not None or w.kv_heads != w.H or w.fp8):
+    if knobs and (w.packed or w.window is not None or w.kv_heads != w.H or w.fp8 or w.colmask):
         raise SystemExit("--exp-mode/--threshold apply to dense workloads without a band only")
 
-    def launch(qp=q, kp=k, vp=v, op=o, lp=lse, cp=cu):
-        if w.fp8:
+    def launch(qp=q, kp=k, vp=v, op=o, lp=lse, cp=cu, mp=mask):
+        if w.colmask:
+            rc = binding.attn_fwd_colmask(qp.data_ptr(), kp.data_ptr(), vp.data_ptr(), op.data_ptr(),
+                                          lp.data_ptr(), w.B, w.H, w.kv_heads, w.Nq, w.Nk, w.d,
+                                          w.scale, int(w.causal), mp.data_ptr(), 1, ws.data_ptr(),
+                                          ws_bytes, sh)
+        elif w.fp8:
             rc = binding.attn_fwd_fp8(qp.data_ptr(), kp.data_ptr(), vp.data_ptr(), op.data_ptr(),
                                       lp.data_ptr(), w.B, w.H, w.kv_heads, w.Nq, w.Nk, w.d, w.scale,
                                       *w.descale, int(w.causal), sh)
@@ -438,6 +470,8 @@ def run_ours(args):
     qd, kd, vd = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
     hc = host_cu.pin_memory() if w.packed else None
     cd = torch.empty_like(cu) if w.packed else None
+    hm = host_mask.pin_memory() if w.colmask else None
+    md = torch.empty_like(mask) if w.colmask else None
     KE = args.e2e_steps
 
     def e2e_step():
@@ -446,7 +480,9 @@ def run_ours(args):
         vd.copy_(hv, non_blocking=True)
         if w.packed:
             cd.copy_(hc, non_blocking=True)
-        launch(qd, kd, vd, o, lse, cd)
+        if w.colmask:
+            md.copy_(hm, non_blocking=True)
+        launch(qd, kd, vd, o, lse, cd, md)
         ho.copy_(o, non_blocking=True)
         hl.copy_(lse, non_blocking=True)
 
@@ -467,7 +503,8 @@ def run_ours(args):
     binding.check(binding.attn_status_sync(sh), "e2e region")
     (te_ms,) = parallel.max_over_ranks([e0.elapsed_time(e1)], dev)
     e2e_value = world * w.flops * KE / (te_ms / 1e3) / 1e12
-    h2d = sum(x.numel() * x.element_size() for x in (hq, hk, hv) + ((hc,) if w.packed else ()))
+    h2d = sum(x.numel() * x.element_size()
+              for x in (hq, hk, hv) + ((hc,) if w.packed else ()) + ((hm,) if w.colmask else ()))
     d2h = ho.numel() * ho.element_size() + hl.numel() * hl.element_size()
 
     cpu = None
@@ -496,12 +533,16 @@ def run_ours(args):
                                    + ": back-to-back launches for seconds under the power cap"),
                      "frac_of_burst": achieved / (peaks["burst"] * ratio),
                      "frac_of_spec": achieved / (SPEC_DENSE_BF16_TFLOPS * ratio),
-                     "algorithmic_flops_per_launch": w.flops},
+                     "algorithmic_flops_per_launch": w.flops,
+                     "timed_window": ("mask-summary + attention kernels" if w.colmask
+                                      else "attention kernel")},
         "cpu_baseline": cpu,
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                "steps": KE, "path": f"pinned host Q/K/V{' + offsets' if w.packed else ''} -> H2D -> "
+                "steps": KE, "path": f"pinned host Q/K/V{' + offsets' if w.packed else ''}"
+                        f"{' + mask' if w.colmask else ''} -> H2D -> "
                         f"{launch_name(w)} (C-ABI) -> D2H of O and LSE"},
-        "gpu_launches": K,
+        # attn_fwd_colmask launches a summary kernel before the attention kernel
+        "gpu_launches": 2 * K if w.colmask else K,
         "clocks": clocks,
         "kernel_src_sha": kernel_source_hash("fwd"),
     }

@@ -51,6 +51,11 @@ def lib() -> ctypes.CDLL:
             l.attn_fwd_window.argtypes = [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I,
                                           ctypes.c_float, _I, _I, _P]
             l.attn_fwd_window.restype = _I
+            l.attn_fwd_colmask.argtypes = [_P, _P, _P, _P, _P] + [_I] * 6 + [ctypes.c_float, _I, _P, _I,
+                                                                          _P, ctypes.c_size_t, _P]
+            l.attn_fwd_colmask.restype = _I
+            l.attn_colmask_workspace_size.argtypes = [_I, _I, _I]
+            l.attn_colmask_workspace_size.restype = ctypes.c_size_t
             l.attn_fwd_varlen.argtypes = [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I,
                                           ctypes.c_float, _I, _I, _P]
             l.attn_fwd_varlen.restype = _I
@@ -88,6 +93,16 @@ def attn_fwd_window(q, k, v, o, lse, B, H, Hkv, Nq, Nk, d, scale, window_left, w
                     stream) -> int:
     return lib().attn_fwd_window(q, k, v, o, lse, B, H, Hkv, Nq, Nk, d, scale, window_left,
                                  window_right, stream)
+
+
+def attn_fwd_colmask(q, k, v, o, lse, B, H, Hkv, Nq, Nk, d, scale, causal, mask, Hm, workspace,
+                     workspace_bytes, stream) -> int:
+    return lib().attn_fwd_colmask(q, k, v, o, lse, B, H, Hkv, Nq, Nk, d, scale, causal, mask, Hm,
+                                  workspace, workspace_bytes, stream)
+
+
+def attn_colmask_workspace_size(B, Hm, Nk) -> int:
+    return lib().attn_colmask_workspace_size(B, Hm, Nk)
 
 
 def attn_fwd_varlen(q, k, v, o, lse, cu_seqlens_q, cu_seqlens_k, num_seqs, max_seqlen_q, total_q,
@@ -225,6 +240,44 @@ def fwd(q, k, v, causal: bool = False, scale: float | None = None, *, window=Non
                              stream)
     check(rc, "attn_fwd")
     return (out, lse) if return_lse else out
+
+
+def fwd_colmask(q, k, v, mask, causal: bool = False, scale: float | None = None, *,
+                workspace=None, out=None, lse=None):
+    """attn_fwd_colmask on BF16 CUDA tensors q [B,H,Nq,d], k/v [B,Hkv,Nk,d] and
+    an int32 CUDA mask [B, Hm, Nk, 4] (Hm = 1 or H): key j is hidden from query
+    rows [mask[..., j, 0], mask[..., j, 1]) and [mask[..., j, 2], mask[..., j, 3]),
+    and from rows i < j when causal.  workspace: a uint8 CUDA tensor of at least
+    attn_colmask_workspace_size(B, Hm, Nk) bytes (allocated when None).
+    Returns (o, lse) on torch's current stream."""
+    import torch
+
+    _check_bf16(q=q, k=k, v=v)
+    B, H, Nq, d = q.shape
+    Hkv, Nk = k.shape[1], k.shape[2]
+    if tuple(k.shape) != (B, Hkv, Nk, d) or tuple(v.shape) != (B, Hkv, Nk, d):
+        raise ValueError("k and v must be [B, Hkv, Nk, d] matching q")
+    if not isinstance(mask, torch.Tensor) or mask.dtype != torch.int32 or not mask.is_cuda:
+        raise TypeError("mask must be an int32 CUDA tensor")
+    if mask.dim() != 4 or mask.shape[0] != B or mask.shape[2] != Nk or mask.shape[3] != 4 \
+            or not mask.is_contiguous():
+        raise ValueError("mask must be contiguous [B, Hm, Nk, 4]")
+    Hm = mask.shape[1]
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    ws_bytes = attn_colmask_workspace_size(B, Hm, Nk)
+    if workspace is None:
+        workspace = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=q.device)
+    if out is None:
+        out = torch.empty((B, H, Nq, d), dtype=torch.bfloat16, device=q.device)
+    if lse is None:
+        lse = torch.empty((B, H, Nq), dtype=torch.float32, device=q.device)
+    stream = torch.cuda.current_stream(q.device).cuda_stream
+    rc = attn_fwd_colmask(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
+                          B, H, Hkv, Nq, Nk, d, float(scale), int(bool(causal)), mask.data_ptr(), Hm,
+                          workspace.data_ptr(), workspace.numel(), stream)
+    check(rc, "attn_fwd_colmask")
+    return out, lse
 
 
 def fwd_varlen(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q: int, causal: bool = False,

@@ -54,6 +54,7 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <climits>
 #include <cmath>
 #include <cstdint>
 #include <cstdio>
@@ -99,6 +100,15 @@ constexpr unsigned int kStatusBadSeqlens = kStatusWordBadSeqlens;
 // "no bound" for a side of the key band; large enough for any sequence, small
 // enough that row +- bound stays inside int.
 constexpr int kUnbounded = 1 << 30;
+
+// Mask kinds (kernel template argument).  kMaskBand: the key band
+// i - wl <= j <= i + wr (causal is wl unbounded, wr = 0).  kMaskCols: the band
+// plus a column-interval mask -- per key column j up to two query-row
+// intervals [lo1, hi1) and [lo2, hi2) that do not see key j -- with key blocks
+// that hide all of a CTA's rows skipped altogether.
+constexpr int kMaskNone = 0;
+constexpr int kMaskBand = 1;
+constexpr int kMaskCols = 2;
 
 // Per-device status word (each device holds its own copy of module globals).
 __device__ unsigned int g_status;
@@ -152,6 +162,13 @@ struct FwdParams {
   float scale_log2;  // scale * log2(e) (E4M3: times the Q and K scale factors)
   float tau;         // rescale threshold, powers of two
   float o_scale;     // multiplies O / l (E4M3: the V scale factor; else 1)
+  // column-interval mask (kMaskCols): per key column (lo1, hi1, lo2, hi2),
+  // [B * mask_heads, Nk]; per 128-key block two summaries,
+  // [B * mask_heads, n_kblocks, 2] (see colmask_summary_kernel)
+  const int4* colmask;
+  const int4* colsum;
+  int mask_heads;    // 1 (one mask for all heads of a batch entry) or H
+  int n_kblocks;     // key blocks per head: ceil(Nk / 128)
 };
 
 // Where one CTA's sequence lives: lengths, first packed row (packed layout),
@@ -160,8 +177,11 @@ struct SeqView {
   int Nq, Nk;        // this sequence's lengths
   int q0, k0;        // first row of the sequence in the packed layout (0 dense)
   int head_q, head_kv;  // tensor-map head coordinate of Q/O and of K/V
-  int j_lo, n_kv;    // KV tiles j_lo .. j_lo + n_kv - 1
+  int j_lo, n_kv;    // KV tiles visited: n_kv of j_lo .. j_end - 1 (all of them
+  int j_end;         // unless a column-interval mask skips some)
+  int mrow;          // column-interval mask: row of [B * mask_heads] to use
   bool packed;
+  bool none_visible; // column-interval mask hides every block: visit j_lo, fully masked
   float* lse_row0;   // LSE of this sequence's row 0 (null: not computed)
 };
 
@@ -171,6 +191,42 @@ __device__ __forceinline__ void tma_load_rows(uint32_t dst, const CUtensorMap* t
                                               int head, bool packed, uint32_t bar) {
   if (packed) tma_load_3d(dst, tm, col, head, row, bar);
   else tma_load_3d(dst, tm, col, row, head, bar);
+}
+
+// Column-interval mask, block summaries (colmask_summary_kernel):
+//   a = (max lo1, min hi1, max lo2, min hi2) over the block's keys, with an
+//       empty interval counting as (INT_MAX, INT_MIN): one interval of every
+//       key hides rows [r0, r1) iff a.x <= r0 && a.y >= r1 (or a.z / a.w);
+//   b = (min lo1, max hi1, min lo2, max hi2): no key's interval meets [r0, r1)
+//       iff b.y <= r0 || b.x >= r1 (and likewise b.z / b.w).
+__device__ __forceinline__ bool cols_hide_all(const FwdParams& prm, int mrow, int blk, int r0,
+                                              int r1) {
+  const int4 a = __ldg(prm.colsum + (static_cast<size_t>(mrow) * prm.n_kblocks + blk) * 2);
+  return (a.x <= r0 && a.y >= r1) || (a.z <= r0 && a.w >= r1);
+}
+__device__ __forceinline__ bool cols_touch(const FwdParams& prm, int mrow, int blk, int r0,
+                                           int r1) {
+  const int4 b = __ldg(prm.colsum + (static_cast<size_t>(mrow) * prm.n_kblocks + blk) * 2 + 1);
+  return !(b.y <= r0 || b.x >= r1) || !(b.w <= r0 || b.z >= r1);
+}
+
+// Query rows [r0, r1) of a CTA's block qb (r1 clipped to the sequence).
+__device__ __forceinline__ int cta_row_end(int qb, int Nq) {
+  const long long e = static_cast<long long>(qb) * kRowsPerCta + kRowsPerCta;
+  return e < Nq ? static_cast<int>(e) : Nq;
+}
+
+// KV tile visited after tile blk (first: blk = j_lo - 1).  Every role of the
+// CTA walks the same sequence, so they agree on it without communicating.
+template <int MASK>
+__device__ __forceinline__ int next_block(const FwdParams& prm, const SeqView& sv, int qb, int blk) {
+  ++blk;
+  if constexpr (MASK == kMaskCols) {
+    if (sv.none_visible) return sv.j_lo;
+    const int r0 = qb * kRowsPerCta, r1 = cta_row_end(qb, sv.Nq);
+    while (blk < sv.j_end - 1 && cols_hide_all(prm, sv.mrow, blk, r0, r1)) ++blk;
+  }
+  return blk;
 }
 
 // ---------------------------------------------------------------------------
@@ -217,10 +273,11 @@ __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, uint64_
 // ---------------------------------------------------------------------------
 // Producer: one thread, TMA loads of Q0, K0, Q1, V0, K1, V1, ...
 // ---------------------------------------------------------------------------
-template <int D, bool F8>
+template <int D, int MASK, bool F8>
 __device__ __forceinline__ void producer_role(const Smem<D, F8>& sm, const CUtensorMap* tm_q,
                                               const CUtensorMap* tm_k, const CUtensorMap* tm_v,
-                                              const SeqView& sv, int qb, uint64_t timeout) {
+                                              const SeqView& sv, const FwdParams& prm, int qb,
+                                              uint64_t timeout) {
   using C = Cfg<D, F8>;
   uint32_t it = 0;
   auto load_q = [&](int t) {
@@ -243,11 +300,15 @@ __device__ __forceinline__ void producer_role(const Smem<D, F8>& sm, const CUten
     return true;
   };
 
+  int blk = next_block<MASK>(prm, sv, qb, sv.j_lo - 1);
   load_q(0);
-  bool ok = load_kv(tm_k, sv.j_lo);
+  bool ok = load_kv(tm_k, blk);
   load_q(1);
-  ok = ok && load_kv(tm_v, sv.j_lo);
-  for (int j = sv.j_lo + 1; ok && j < sv.j_lo + sv.n_kv; ++j) ok = load_kv(tm_k, j) && load_kv(tm_v, j);
+  ok = ok && load_kv(tm_v, blk);
+  for (int j = 1; ok && j < sv.n_kv; ++j) {
+    blk = next_block<MASK>(prm, sv, qb, blk);
+    ok = load_kv(tm_k, blk) && load_kv(tm_v, blk);
+  }
 
   // Never leave the CTA with a copy in flight: wait for the latest fill of
   // every slot and for both Q tiles (immediate on the normal path).
@@ -411,7 +472,7 @@ __device__ __forceinline__ void pair_sync(int t, int q) {
   asm volatile("bar.sync %0, 64;" ::"r"(1 + t * 4 + q) : "memory");
 }
 
-template <int D, bool MASK, int POLY16, bool F8>
+template <int D, int MASK, int POLY16, bool F8>
 __device__ __forceinline__ void softmax_role(const Smem<D, F8>& sm, uint32_t tmem,
                                              const CUtensorMap* tm_o, const FwdParams& prm,
                                              const SeqView& sv, int qb) {
@@ -440,12 +501,37 @@ __device__ __forceinline__ void softmax_role(const Smem<D, F8>& sm, uint32_t tme
   float l_run = 0.0f;       // this half's running sum of 2^(score - m_run)
   bool ok = true;
 
+  int blk = sv.j_lo - 1;
   for (int j = 0; j < sv.n_kv; ++j) {
+    blk = next_block<MASK>(prm, sv, qb, blk);
+    const int kv0 = blk * kBlockN + h * kCols;
+    // mask needed: key tail, a band edge crossing this warp's 64 x 32 block, or
+    // a column interval meeting the warp's rows
+    bool masked = kv0 + kCols > Nk ||
+                  (MASK != kMaskNone && (kv0 + kCols - 1 - rw0 > prm.wr || rw0 + 31 - kv0 > prm.wl));
+    // column-interval mask: bit c of hid[k] = key kv0 + 32k + c hidden from this row
+    uint32_t hid[2] = {0u, 0u};
+    if constexpr (MASK == kMaskCols) {
+      if (cols_touch(prm, sv.mrow, blk, rw0, rw0 + 32)) {
+        masked = true;
+        const int4* cm = prm.colmask + static_cast<size_t>(sv.mrow) * Nk + kv0;
+        const int n_in = min(kCols, Nk - kv0);
+#pragma unroll
+        for (int k = 0; k < 2; ++k) {
+          uint32_t bits = 0u;
+#pragma unroll 8
+          for (int c = 0; c < 32; ++c) {
+            if (32 * k + c < n_in) {
+              const int4 iv = __ldg(cm + 32 * k + c);
+              const bool hide = (iv.x <= row && row < iv.y) || (iv.z <= row && row < iv.w);
+              bits |= static_cast<uint32_t>(hide) << c;
+            }
+          }
+          hid[k] = bits;
+        }
+      }
+    }
     ok = warp_wait(sm.s_full(t), j & 1, timeout);
-    const int kv0 = (sv.j_lo + j) * kBlockN + h * kCols;
-    // mask needed: key tail, or a band edge crossing this warp's 64 x 32 block
-    const bool masked = kv0 + kCols > Nk ||
-                        (MASK && (kv0 + kCols - 1 - rw0 > prm.wr || rw0 + 31 - kv0 > prm.wl));
     // load 32 score columns [32*k, 32*k + 32) of this warp's half as fp32,
     // prescaled and masked
     auto load_scores = [&](int k, float (&x)[32]) {
@@ -463,7 +549,9 @@ __device__ __forceinline__ void softmax_role(const Smem<D, F8>& sm, uint32_t tme
 #pragma unroll
         for (int c = 0; c < 32; ++c) {
           const int key = kv0 + 32 * k + c;
-          if (key >= Nk || (MASK && (key - row > prm.wr || row - key > prm.wl))) x[c] = -INFINITY;
+          if (key >= Nk || (MASK != kMaskNone && (key - row > prm.wr || row - key > prm.wl)) ||
+              (MASK == kMaskCols && ((hid[k] >> c) & 1u)))
+            x[c] = -INFINITY;
         }
       }
     };
@@ -645,7 +733,7 @@ __device__ __forceinline__ void softmax_role(const Smem<D, F8>& sm, uint32_t tme
 // ---------------------------------------------------------------------------
 // The kernel.  Grid: one CTA per (b*h, 256-row query block).
 // ---------------------------------------------------------------------------
-template <int D, bool MASK, int POLY16, bool F8>
+template <int D, int MASK, int POLY16, bool F8>
 __global__ void __launch_bounds__(kNumThreads, 1)
 attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                 const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
@@ -719,7 +807,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     // which yields O = 0 and LSE = -inf.
     const int n_all = max((sv.Nk + kBlockN - 1) / kBlockN, 1);
     int j_lo = 0, j_hi = n_all;
-    if (MASK) {
+    if (MASK != kMaskNone) {
       // rows and bounds are below 2^31 and 2^30: the sums stay inside 64 bits
       const long long r_lo = static_cast<long long>(qb) * kRowsPerCta;
       const long long r_end = r_lo + kRowsPerCta < sv.Nq ? r_lo + kRowsPerCta : sv.Nq;
@@ -735,7 +823,26 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       }
     }
     sv.j_lo = j_lo;
+    sv.j_end = j_hi;
     sv.n_kv = j_hi - j_lo;
+    sv.mrow = 0;
+    sv.none_visible = false;
+    if constexpr (MASK == kMaskCols) {
+      // count the tiles that some row of this block sees (warp 0, 32 tiles a
+      // step); none: visit tile j_lo fully masked, as for an empty band
+      sv.mrow = seq * prm.mask_heads + (prm.mask_heads == 1 ? 0 : hq);
+      if (warp == 0) {
+        const int r0 = qb * kRowsPerCta, r1 = cta_row_end(qb, sv.Nq);
+        int cnt = 0;
+        for (int base = j_lo; base < j_hi; base += 32) {
+          const int blk = base + lane;
+          const bool vis = blk < j_hi && !cols_hide_all(prm, sv.mrow, blk, r0, r1);
+          cnt += __popc(__ballot_sync(0xffffffffu, vis));
+        }
+        sv.none_visible = cnt == 0;
+        sv.n_kv = cnt > 0 ? cnt : 1;
+      }
+    }
   }
   if (threadIdx.x == 0) *sm.seq() = sv;
 
@@ -770,7 +877,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     // warpgroup 2: TMA producer (warp 8), MMA issuer (warp 9), two idle warps
     setmaxnreg_dec<kProducerRegs>();
     if (warp == kWarpLoad) {
-      if (lane == 0) producer_role<D, F8>(sm, &tm_q, &tm_k, &tm_v, seqv, qb, prm.timeout_ns);
+      if (lane == 0) producer_role<D, MASK, F8>(sm, &tm_q, &tm_k, &tm_v, seqv, prm, qb, prm.timeout_ns);
       __syncwarp();
     } else if (warp == kWarpMma) {
       if (lane == 0) mma_role<D, F8>(sm, tmem, seqv.n_kv, prm.timeout_ns);
@@ -796,6 +903,62 @@ __global__ void fill_neg_inf_kernel(float* p, size_t n) {
     p[i] = -INFINITY;
 }
 
+// Column-interval mask summaries: one 128-thread CTA per (mask row, key block)
+// reduces the block's intervals to the two int4 that cols_hide_all and
+// cols_touch read.  Keys past Nk take no part; an empty interval (lo >= hi)
+// counts as (INT_MAX, INT_MIN), so it neither hides a row nor meets one.
+__global__ void __launch_bounds__(128) colmask_summary_kernel(const int4* __restrict__ mask,
+                                                              int4* __restrict__ sum, int Nk,
+                                                              int n_kblocks) {
+  const int blk = static_cast<int>(blockIdx.x % static_cast<unsigned>(n_kblocks));
+  const size_t mrow = blockIdx.x / static_cast<unsigned>(n_kblocks);
+  const int key = blk * kBlockN + static_cast<int>(threadIdx.x);
+  // a: max lo1, min hi1, max lo2, min hi2;  b: min lo1, max hi1, min lo2, max hi2
+  int a[4] = {INT_MIN, INT_MAX, INT_MIN, INT_MAX};
+  int b[4] = {INT_MAX, INT_MIN, INT_MAX, INT_MIN};
+  if (key < Nk) {
+    const int4 iv = mask[mrow * Nk + key];
+    const bool e1 = iv.x >= iv.y, e2 = iv.z >= iv.w;
+    a[0] = b[0] = e1 ? INT_MAX : iv.x;
+    a[1] = b[1] = e1 ? INT_MIN : iv.y;
+    a[2] = b[2] = e2 ? INT_MAX : iv.z;
+    a[3] = b[3] = e2 ? INT_MIN : iv.w;
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int oa = __shfl_xor_sync(0xffffffffu, a[i], off);
+      const int ob = __shfl_xor_sync(0xffffffffu, b[i], off);
+      a[i] = (i & 1) ? min(a[i], oa) : max(a[i], oa);
+      b[i] = (i & 1) ? max(b[i], ob) : min(b[i], ob);
+    }
+  }
+  __shared__ int red[4][8];
+  const int warp = threadIdx.x >> 5;
+  if ((threadIdx.x & 31) == 0) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      red[warp][i] = a[i];
+      red[warp][4 + i] = b[i];
+    }
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+#pragma unroll
+    for (int w = 1; w < 4; ++w) {
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        a[i] = (i & 1) ? min(a[i], red[w][i]) : max(a[i], red[w][i]);
+        b[i] = (i & 1) ? max(b[i], red[w][4 + i]) : min(b[i], red[w][4 + i]);
+      }
+    }
+    int4* dst = sum + (mrow * n_kblocks + blk) * 2;
+    dst[0] = make_int4(a[0], a[1], a[2], a[3]);
+    dst[1] = make_int4(b[0], b[1], b[2], b[3]);
+  }
+}
+
 // One thread waits on a barrier that nothing signals; the bounded wait gives
 // up and records a timeout.  Exercises the failure path without any fault.
 __global__ void selftest_timeout_kernel(uint64_t timeout_ns) {
@@ -812,7 +975,7 @@ __global__ void selftest_timeout_kernel(uint64_t timeout_ns) {
 // ---------------------------------------------------------------------------
 constexpr int kMaxDevices = kMaxDeviceCount;
 
-template <int D, bool MASK, int POLY16, bool F8 = false>
+template <int D, int MASK, int POLY16, bool F8 = false>
 int launch_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                const CUtensorMap& to, const FwdParams& prm, cudaStream_t stream) {
   auto kern = attn_fwd_kernel<D, MASK, POLY16, F8>;
@@ -833,7 +996,7 @@ int launch_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& 
   return ATTN_OK;
 }
 
-template <int D, bool MASK>
+template <int D, int MASK>
 int dispatch_exp(int exp_mode, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                  const CUtensorMap& to, const FwdParams& prm, cudaStream_t stream) {
   switch (exp_mode) {
@@ -866,13 +1029,17 @@ int heads_per_l2_group(double keys_per_head, int d, int group, long long BH) {
 int launch_any(int d, int exp_mode, const CUtensorMap& tq, const CUtensorMap& tk,
                const CUtensorMap& tv, const CUtensorMap& to, const FwdParams& prm,
                cudaStream_t stream) {
+  if (prm.colmask != nullptr) {  // default exp2 split only
+    return d == 128 ? launch_fwd<128, kMaskCols, kDefaultPoly16>(tq, tk, tv, to, prm, stream)
+                    : launch_fwd<64, kMaskCols, kDefaultPoly16>(tq, tk, tv, to, prm, stream);
+  }
   const bool mask = prm.wl < kUnbounded || prm.wr < kUnbounded;
   if (d == 128) {
-    return mask ? dispatch_exp<128, true>(exp_mode, tq, tk, tv, to, prm, stream)
-                : dispatch_exp<128, false>(exp_mode, tq, tk, tv, to, prm, stream);
+    return mask ? dispatch_exp<128, kMaskBand>(exp_mode, tq, tk, tv, to, prm, stream)
+                : dispatch_exp<128, kMaskNone>(exp_mode, tq, tk, tv, to, prm, stream);
   }
-  return mask ? dispatch_exp<64, true>(exp_mode, tq, tk, tv, to, prm, stream)
-              : dispatch_exp<64, false>(exp_mode, tq, tk, tv, to, prm, stream);
+  return mask ? dispatch_exp<64, kMaskBand>(exp_mode, tq, tk, tv, to, prm, stream)
+              : dispatch_exp<64, kMaskNone>(exp_mode, tq, tk, tv, to, prm, stream);
 }
 
 // No key at all: O = 0, LSE = -inf.
@@ -898,9 +1065,24 @@ bool outputs_overlap(const void* q, size_t q_bytes, const void* k, const void* v
          ranges_overlap(lse, lse_bytes, o, o_bytes);
 }
 
+// Column-interval mask of attn_fwd_colmask: int32 [B, Hm, Nk, 4] and the
+// caller's workspace for the per-block summaries.
+struct ColMaskArgs {
+  const int* mask;
+  int Hm;
+  void* workspace;
+  size_t workspace_bytes;
+};
+
+size_t colmask_workspace_bytes(long long BHm, int Nk) {
+  const long long n_kblocks = (static_cast<long long>(Nk) + kBlockN - 1) / kBlockN;
+  return static_cast<size_t>(BHm * n_kblocks) * 2 * sizeof(int4);
+}
+
 int fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
              int Hkv, int Nq, int Nk, int d, float scale, int window_left, int window_right,
-             float tau, int exp_mode, unsigned long long* rescale_count, cudaStream_t stream) {
+             float tau, int exp_mode, unsigned long long* rescale_count, cudaStream_t stream,
+             const ColMaskArgs* cm = nullptr) {
   int wl = 0, wr = 0;
   if (B < 0 || H < 0 || Hkv < 0 || Nq < 0 || Nk < 0) return ATTN_ERR_INVALID_ARG;
   if (H > 0 && (Hkv == 0 || H % Hkv != 0)) return ATTN_ERR_INVALID_ARG;
@@ -924,6 +1106,27 @@ int fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, i
     return ATTN_ERR_INVALID_ARG;
   const long long n_qblocks = (Nq + kRowsPerCta - 1) / kRowsPerCta;
   if (n_qblocks * BH > 0x7fffffffLL) return ATTN_ERR_INVALID_ARG;
+  long long BHm = 0;
+  size_t mask_bytes = 0, ws_need = 0;
+  if (cm) {
+    if (cm->Hm != 1 && cm->Hm != H) return ATTN_ERR_INVALID_ARG;
+    BHm = static_cast<long long>(B) * cm->Hm;
+    mask_bytes = static_cast<size_t>(BHm) * Nk * sizeof(int4);
+    ws_need = colmask_workspace_bytes(BHm, Nk);
+    if (Nk > 0 && (!cm->mask || !cm->workspace)) return ATTN_ERR_INVALID_ARG;
+    if (misaligned(cm->mask, 16) || misaligned(cm->workspace, 16)) return ATTN_ERR_INVALID_ARG;
+    if (cm->workspace_bytes < ws_need) return ATTN_ERR_INVALID_ARG;
+    if (BHm * ((Nk + kBlockN - 1) / kBlockN) > 0x7fffffffLL) return ATTN_ERR_INVALID_ARG;
+    // the workspace is written: it may overlap no input or output
+    const void* ws = cm->workspace;
+    if (ranges_overlap(ws, ws_need, q, o_bytes) || ranges_overlap(ws, ws_need, k, kv_bytes) ||
+        ranges_overlap(ws, ws_need, v, kv_bytes) || ranges_overlap(ws, ws_need, o, o_bytes) ||
+        ranges_overlap(ws, ws_need, lse, lse_bytes) ||
+        ranges_overlap(ws, ws_need, cm->mask, mask_bytes) ||
+        ranges_overlap(o, o_bytes, cm->mask, mask_bytes) ||
+        ranges_overlap(lse, lse_bytes, cm->mask, mask_bytes))
+      return ATTN_ERR_INVALID_ARG;
+  }
   int rc = check_device();
   if (rc != ATTN_OK) return rc;
 
@@ -955,6 +1158,17 @@ int fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, i
   prm.scale_log2 = scale * kLog2e;
   prm.tau = tau;
   prm.o_scale = 1.0f;
+  if (cm) {
+    prm.colmask = reinterpret_cast<const int4*>(cm->mask);
+    prm.colsum = static_cast<const int4*>(cm->workspace);
+    prm.mask_heads = cm->Hm;
+    prm.n_kblocks = (Nk + kBlockN - 1) / kBlockN;
+    const unsigned grid = static_cast<unsigned>(BHm * prm.n_kblocks);
+    colmask_summary_kernel<<<grid, 128, 0, stream>>>(prm.colmask, static_cast<int4*>(cm->workspace),
+                                                     Nk, prm.n_kblocks);
+    const cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "colmask_summary_kernel launch");
+  }
   return launch_any(d, exp_mode, tq, tk, tv, to, prm, stream);
 }
 
@@ -1085,8 +1299,8 @@ int fp8_impl(const void* q, const void* k, const void* v, void* o, float* lse, i
   prm.scale_log2 = s_eff * kLog2e;
   prm.tau = kP8Tau;
   prm.o_scale = v_descale;
-  return causal ? launch_fwd<128, true, kDefaultPoly16, true>(tq, tk, tv, to, prm, stream)
-                : launch_fwd<128, false, kDefaultPoly16, true>(tq, tk, tv, to, prm, stream);
+  return causal ? launch_fwd<128, kMaskBand, kDefaultPoly16, true>(tq, tk, tv, to, prm, stream)
+                : launch_fwd<128, kMaskNone, kDefaultPoly16, true>(tq, tk, tv, to, prm, stream);
 }
 
 }  // namespace eab
@@ -1114,6 +1328,21 @@ int attn_fwd_window(const void* q, const void* k, const void* v, void* o, float*
                     int window_right, cudaStream_t stream) {
   return eab::fwd_impl(q, k, v, o, lse, B, H, Hkv, Nq, Nk, d, scale, window_left, window_right,
                        eab::kDefaultThreshold, 1, nullptr, stream);
+}
+
+size_t attn_colmask_workspace_size(int B, int Hm, int Nk) {
+  if (B < 0 || Hm < 0 || Nk < 0) return 0;
+  return eab::colmask_workspace_bytes(static_cast<long long>(B) * Hm, Nk);
+}
+
+int attn_fwd_colmask(const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                     int H, int Hkv, int Nq, int Nk, int d, float scale, int causal,
+                     const int* mask, int Hm, void* workspace, size_t workspace_bytes,
+                     cudaStream_t stream) {
+  if (causal != 0 && causal != 1) return ATTN_ERR_INVALID_ARG;
+  const eab::ColMaskArgs cm = {mask, Hm, workspace, workspace_bytes};
+  return eab::fwd_impl(q, k, v, o, lse, B, H, Hkv, Nq, Nk, d, scale, -1, causal ? 0 : -1,
+                       eab::kDefaultThreshold, 1, nullptr, stream, &cm);
 }
 
 int attn_fwd_varlen(const void* q, const void* k, const void* v, void* o, float* lse,

@@ -18,7 +18,8 @@ Definition (fixed here, used by every consumer):
                z = sqrt(-2 ln u1) * cos(2 pi u2)   (Box-Muller, cosine branch, fp64)
   uniform    : u = (bits >> 40) / 2^24,  z = 2u - 1  in [-1, 1)
   value      = bf16_rne(fp32_rne(mult * z))
-  unit draw  : (bits >> 11) / 2^53 in [0, 1), fp64 (sequence lengths; id 3)
+  unit draw  : (bits >> 11) / 2^53 in [0, 1), fp64 (sequence lengths, id 3;
+               column-interval masks, id 4)
 
 (SplitMix64: Steele, Lea & Flood, "Fast splittable pseudorandom number
 generators", OOPSLA 2014.)
@@ -34,7 +35,8 @@ GAMMA = np.uint64(0x9E3779B97F4A7C15)
 _M1 = np.uint64(0xBF58476D1CE4E5B9)
 _M2 = np.uint64(0x94D049BB133111EB)
 
-TENSOR_ID = {"q": 0, "k": 1, "v": 2, "len": 3}  # "len": sequence lengths of a packed batch
+# "len": sequence / document lengths; "mask": column-interval stress masks
+TENSOR_ID = {"q": 0, "k": 1, "v": 2, "len": 3, "mask": 4}
 
 _CHUNK = 1 << 22
 

@@ -13,7 +13,7 @@ import math
 
 import numpy as np
 
-from . import inputs
+from . import inputs, masks
 
 
 @dataclasses.dataclass(frozen=True)
@@ -37,6 +37,19 @@ class Workload:
                                     # (queries and keys alike); B = len(seqlens)
     fp8: bool = False               # Q, K, V as E4M3 codes times the descale factors below
     descale: tuple = (1.0, 1.0, 1.0)  # (q, k, v) scale factors of the E4M3 codes
+    docs: tuple | None = None       # column-interval document mask: lengths uniform in
+                                    # [lo, hi] per batch entry (with causal: block-diagonal causal)
+
+    @property
+    def colmask(self) -> bool:
+        return self.docs is not None
+
+    def doc_lengths(self, b: int) -> list:
+        return masks.document_lengths(self.seed * 1000 + b, self.Nk, *self.docs)
+
+    def colmask_array(self) -> np.ndarray:
+        """int32 [B, 1, Nk, 4] column intervals of the document mask."""
+        return masks.documents([self.doc_lengths(b) for b in range(self.B)], self.Nk)
 
     @property
     def packed(self) -> bool:
@@ -70,6 +83,9 @@ class Workload:
         """Algorithmic FLOPs, 4*d per visible (query, key) pair: 4*B*H*Nq*Nk*d
         without a mask, half of that for causal (the usual convention), and the
         exact count of visible pairs for a band or a packed batch."""
+        if self.colmask:
+            pairs = masks.visible_pairs(self.colmask_array(), self.Nq, self.causal)
+            return 4.0 * self.d * self.H * float(pairs.sum())
         if self.window is None and not self.packed:
             f = 4.0 * self.B * self.H * self.Nq * self.Nk * self.d
             return f / 2 if self.causal else f
@@ -185,6 +201,9 @@ WORKLOADS = {
                  fp8=True),
         Workload("fp8_b2h16n8k_d128_causal", 2, 16, 8192, 8192, 128, True, seed=8, oracle_rows=128,
                  fp8=True),
+        # causal document mask (column intervals): documents of 256 .. 4096 tokens
+        Workload("docs_b2h16n8k_d128_causal", 2, 16, 8192, 8192, 128, True, seed=9,
+                 oracle_rows=128, docs=(256, 4096)),
         # 16 sequences of mixed length (512 .. 16384 tokens), packed, causal
         Workload("varlen16_h16_d128_causal", 16, 16, 0, 0, 128, True, seed=7, oracle_rows=64,
                  seqlens=_mixed_lengths(7, 16, 512, 16384)),

@@ -113,6 +113,43 @@ int attn_fwd_window(const void *q, const void *k, const void *v, void *o, float 
                     int window_right, cudaStream_t stream);
 
 /*
+ * Column-interval ("FlashMask-style") masks.  The same page that points to
+ * FlashMask ("AIの「脳の回転」を1.8倍高速化？FlashAttentionの秘密",
+ * gipyeong-lee.github.io, section "今後はどうなるか？") names it only as an
+ * extension that handles masks more precisely; it gives no representation.
+ * This library's reading: for every key column j, up to two intervals of query
+ * rows that do not see key j,
+ *
+ *     K(i) = { j : 0 <= j < Nk,  not (lo1_j <= i < hi1_j),  not (lo2_j <= i < hi2_j),
+ *                 and j <= i if causal }
+ *
+ * which holds document (block-diagonal) masks, prefix-LM masks, shared-prefix
+ * masks and bands in O(Nk) memory.  An interval with lo >= hi is empty.  A row
+ * that sees no key gets O = 0, LSE = -inf.
+ *   q, o : [B, H, Nq, d];  k, v : [B, Hkv, Nk, d];  lse : [B, H, Nq] (may be NULL)
+ *   Hkv, d, scale : as attn_fwd_gqa;  causal : 0 or 1 (j <= i, any Nq, Nk)
+ *   mask : DEVICE int32 [B, Hm, Nk, 4], each key's (lo1, hi1, lo2, hi2), 16-byte
+ *          aligned; Hm == 1 (one mask per batch entry, shared by all heads) or
+ *          Hm == H (one per query head).  Read only.
+ *   workspace : DEVICE, 16-byte aligned, at least
+ *          attn_colmask_workspace_size(B, Hm, Nk) bytes, owned by the caller;
+ *          overwritten with per-128-key-block summaries of the mask, so it may
+ *          not overlap any other argument.  Calls on different streams need
+ *          different workspaces.
+ * The call launches two kernels on `stream`: the block summaries, then the
+ * attention kernel, which skips every 128-key block that hides all 256 query
+ * rows of a CTA and masks element-wise only in blocks whose intervals meet a
+ * warp's 32 rows.  Errors as attn_fwd_gqa, plus ATTN_ERR_INVALID_ARG for a NULL
+ * or misaligned mask or workspace, a workspace that is too small or overlaps
+ * another argument, or Hm not in {1, H}.
+ */
+size_t attn_colmask_workspace_size(int B, int Hm, int Nk);
+int attn_fwd_colmask(const void *q, const void *k, const void *v, void *o, float *lse, int B,
+                     int H, int Hkv, int Nq, int Nk, int d, float scale, int causal,
+                     const int *mask, int Hm, void *workspace, size_t workspace_bytes,
+                     cudaStream_t stream);
+
+/*
  * Variable-length batch: sequences of different lengths packed back to back,
  * with no padding (FlashAttention 4 page, ja.linux-konsole.com, section
  * "互換性と現状", lists this among what FA4's forward lacks).

@@ -57,6 +57,12 @@ def _load():
                           ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64,
                           ctypes.c_double, ctypes.c_int64, ctypes.c_int64, ctypes.c_void_p,
                           ctypes.c_void_p, ctypes.c_int]
+            c = lib.oracle_attn_rows_colmask_f64
+            c.restype = ctypes.c_int
+            c.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64,
+                          ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64,
+                          ctypes.c_double, ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p,
+                          ctypes.c_void_p, ctypes.c_int]
             b = lib.oracle_attn_bwd_f64
             b.restype = ctypes.c_int
             b.argtypes = [ctypes.c_void_p] * 4 + [ctypes.c_int64] * 3 + [ctypes.c_double] + \
@@ -121,6 +127,34 @@ def attn_rows_window(q_rows, rows, k, v, scale, window_left, window_right, nthre
                                          o.ctypes.data, lse.ctypes.data, nt)
     if rc != 0:
         raise RuntimeError("oracle_attn_rows_window_f64 failed")
+    return o, lse
+
+
+def attn_rows_colmask(q_rows, rows, k, v, scale, causal, cols, nthreads=None):
+    """Like ``attn_rows`` under column intervals: ``cols`` is [Nk, 4] integers,
+    key j's (lo1, hi1, lo2, hi2); row i does not see key j when
+    lo1 <= i < hi1 or lo2 <= i < hi2 (or j > i when causal).  Rows that see no
+    key get O = 0, LSE = -inf."""
+    lib = _load()
+    q_rows = np.ascontiguousarray(q_rows, dtype=np.float64)
+    rows = np.ascontiguousarray(rows, dtype=np.int64)
+    k = np.ascontiguousarray(k, dtype=np.float64)
+    v = np.ascontiguousarray(v, dtype=np.float64)
+    cols = np.ascontiguousarray(cols, dtype=np.int64)
+    n, d = q_rows.shape
+    nk = k.shape[0]
+    assert rows.shape == (n,) and k.shape == (nk, d) and v.shape == (nk, d)
+    assert cols.shape == (nk, 4)
+    o = np.empty((n, d), dtype=np.float64)
+    lse = np.empty((n,), dtype=np.float64)
+    nt = default_threads() if nthreads is None else int(nthreads)
+    rc = lib.oracle_attn_rows_colmask_f64(q_rows.ctypes.data, rows.ctypes.data, n,
+                                          k.ctypes.data if nk else None,
+                                          v.ctypes.data if nk else None, nk, d, float(scale),
+                                          1 if causal else 0, cols.ctypes.data if nk else None,
+                                          o.ctypes.data, lse.ctypes.data, nt)
+    if rc != 0:
+        raise RuntimeError("oracle_attn_rows_colmask_f64 failed")
     return o, lse
 
 

@@ -41,6 +41,16 @@
  * band (-1, 0); no mask is (-1, -1).  A row whose band holds no key gets
  * O_i = 0, LSE_i = -inf, as for Nk == 0.
  *
+ * Column-interval masks.  The same page names FlashMask only as an extension
+ * that handles masks more precisely, with no representation.  This library's
+ * reading: every key j carries two intervals of query rows that do not see it,
+ *
+ *   K(i)  = {j : 0 <= j < Nk,  not lo1_j <= i < hi1_j,  not lo2_j <= i < hi2_j,
+ *                and j <= i when causal}
+ *
+ * (an interval with lo >= hi is empty); the visible keys need not be
+ * contiguous.  Same empty-row rule.
+ *
  * All arithmetic is fp64.  Inputs arrive as fp64 (the caller widens the BF16
  * values, which is exact), so the only rounding is fp64 rounding.
  *
@@ -64,6 +74,9 @@ typedef struct {
     double scale;
     int64_t window_left;  /* keys j >= i - window_left (negative: no bound)  */
     int64_t window_right; /* keys j <= i + window_right (negative: no bound) */
+    const int64_t *cols;  /* [Nk, 4] column intervals, or NULL: band only      */
+    int causal;           /* with cols: also hide keys j > i                   */
+    int64_t *vis;         /* per-thread visible-key list, [nk]                 */
     double *o;            /* [n_rows, d]  out                                 */
     double *lse;          /* [n_rows]     out                                 */
     double *s;            /* per-thread score row, [nk]                       */
@@ -110,9 +123,55 @@ static void oracle_row(const oracle_job *jb, int64_t r) {
     jb->lse[r] = m + log(l);
 }
 
+/* One query row under column intervals: list the visible keys, then the same
+ * steps as oracle_row over that list. */
+static void oracle_row_cols(const oracle_job *jb, int64_t r) {
+    const int64_t d = jb->d;
+    const double *qi = jb->q + r * d;
+    double *oi = jb->o + r * d;
+    const int64_t i = jb->rows[r];
+    int64_t nvis = 0;
+    for (int64_t j = 0; j < jb->nk; ++j) {
+        const int64_t *c = jb->cols + 4 * j;
+        const int hidden = (jb->causal && j > i) || (c[0] <= i && i < c[1]) ||
+                           (c[2] <= i && i < c[3]);
+        if (!hidden) jb->vis[nvis++] = j;
+    }
+    if (nvis == 0) {
+        for (int64_t c = 0; c < d; ++c) oi[c] = 0.0;
+        jb->lse[r] = -INFINITY;
+        return;
+    }
+    double *s = jb->s; /* s[t] holds the score of key vis[t] */
+    for (int64_t t = 0; t < nvis; ++t) {
+        const double *kj = jb->k + jb->vis[t] * d;
+        double dot = 0.0;
+        for (int64_t c = 0; c < d; ++c) dot += qi[c] * kj[c];
+        s[t] = jb->scale * dot;
+    }
+    double m = s[0];
+    for (int64_t t = 1; t < nvis; ++t)
+        if (s[t] > m) m = s[t];
+    double l = 0.0;
+    for (int64_t t = 0; t < nvis; ++t) {
+        s[t] = exp(s[t] - m);
+        l += s[t];
+    }
+    for (int64_t c = 0; c < d; ++c) oi[c] = 0.0;
+    for (int64_t t = 0; t < nvis; ++t) {
+        const double p = s[t] / l;
+        const double *vj = jb->v + jb->vis[t] * d;
+        for (int64_t c = 0; c < d; ++c) oi[c] += p * vj[c];
+    }
+    jb->lse[r] = m + log(l);
+}
+
 static void *oracle_worker(void *arg) {
     oracle_job *jb = (oracle_job *)arg;
-    for (int64_t r = jb->begin; r < jb->end; ++r) oracle_row(jb, r);
+    for (int64_t r = jb->begin; r < jb->end; ++r) {
+        if (jb->cols) oracle_row_cols(jb, r);
+        else oracle_row(jb, r);
+    }
     return NULL;
 }
 
@@ -126,10 +185,10 @@ static void *oracle_worker(void *arg) {
  * nthreads <= 0 means one thread.
  * Returns 0 on success, -1 on a bad argument or allocation failure.
  */
-int oracle_attn_rows_window_f64(const double *q, const int64_t *rows, int64_t n_rows,
-                                const double *k, const double *v, int64_t nk, int64_t d,
-                                double scale, int64_t window_left, int64_t window_right,
-                                double *o, double *lse, int nthreads) {
+static int run_rows(const double *q, const int64_t *rows, int64_t n_rows, const double *k,
+                    const double *v, int64_t nk, int64_t d, double scale, int64_t window_left,
+                    int64_t window_right, const int64_t *cols, int causal, double *o,
+                    double *lse, int nthreads) {
     if (n_rows < 0 || nk < 0 || d <= 0) return -1;
     if (n_rows == 0) return 0;
     if (!q || !rows || !o || !lse || (nk > 0 && (!k || !v))) return -1;
@@ -152,11 +211,13 @@ int oracle_attn_rows_window_f64(const double *q, const int64_t *rows, int64_t n_
         jb->k = k; jb->v = v; jb->nk = nk; jb->d = d;
         jb->scale = scale;
         jb->window_left = window_left; jb->window_right = window_right;
+        jb->cols = cols; jb->causal = causal;
         jb->o = o; jb->lse = lse;
         jb->begin = (int64_t)t * per;
         jb->end = jb->begin + per < n_rows ? jb->begin + per : n_rows;
         jb->s = (double *)malloc((size_t)(nk > 0 ? nk : 1) * sizeof(double));
-        if (!jb->s) { rc = -1; break; }
+        jb->vis = (int64_t *)malloc((size_t)(nk > 0 ? nk : 1) * sizeof(int64_t));
+        if (!jb->s || !jb->vis) { rc = -1; break; }
     }
     if (rc == 0) {
         for (int t = 1; t < nthreads; ++t) {
@@ -173,10 +234,34 @@ int oracle_attn_rows_window_f64(const double *q, const int64_t *rows, int64_t n_
             if (tids[t]) pthread_join(tids[t], NULL);
     }
     (void)started;
-    for (int t = 0; t < nthreads; ++t) free(jobs[t].s);
+    for (int t = 0; t < nthreads; ++t) {
+        free(jobs[t].s);
+        free(jobs[t].vis);
+    }
     free(jobs);
     free(tids);
     return rc;
+}
+
+int oracle_attn_rows_window_f64(const double *q, const int64_t *rows, int64_t n_rows,
+                                const double *k, const double *v, int64_t nk, int64_t d,
+                                double scale, int64_t window_left, int64_t window_right,
+                                double *o, double *lse, int nthreads) {
+    return run_rows(q, rows, n_rows, k, v, nk, d, scale, window_left, window_right, NULL, 0, o,
+                    lse, nthreads);
+}
+
+/*
+ * Attention for a subset of query rows of one (batch, head) under column
+ * intervals: cols is [nk, 4] int64, key j's (lo1, hi1, lo2, hi2); causal also
+ * hides keys j > i.  Other arguments and the return value as above.
+ */
+int oracle_attn_rows_colmask_f64(const double *q, const int64_t *rows, int64_t n_rows,
+                                 const double *k, const double *v, int64_t nk, int64_t d,
+                                 double scale, int causal, const int64_t *cols, double *o,
+                                 double *lse, int nthreads) {
+    if (nk > 0 && !cols) return -1;
+    return run_rows(q, rows, n_rows, k, v, nk, d, scale, -1, -1, cols, causal, o, lse, nthreads);
 }
 
 /* The same without a window: all keys, or the prefix 0..i when causal. */

@@ -293,6 +293,111 @@ def pin_window_is_a_key_slice(attn_rows_window):
 WINDOW_PINS = [pin_window_brute_force, pin_window_diagonal, pin_window_is_a_key_slice]
 
 
+# ---------------------------------------------------------------------------
+# Column-interval masks.  These take ``attn_rows_colmask(q_rows, rows, k, v,
+# scale, causal, cols)`` with cols [Nk, 4] = (lo1, hi1, lo2, hi2) per key.
+# ---------------------------------------------------------------------------
+BIG = 1 << 20  # beyond every row index used here
+
+
+def band_as_columns(nk, wl, wr):
+    """Column intervals of the band (wl, wr): key j is hidden from rows
+    i > j + wl (first interval) and from rows i < j - wr (second)."""
+    j = np.arange(nk, dtype=np.int64)
+    cols = np.zeros((nk, 4), dtype=np.int64)  # (0, 0): empty
+    if wl >= 0:
+        cols[:, 0], cols[:, 1] = j + wl + 1, BIG
+    if wr >= 0:
+        cols[:, 2], cols[:, 3] = -BIG, j - wr
+    return cols
+
+
+def pin_colmask_band(attn_rows_colmask):
+    """Column intervals that spell a band give the band's materialised masked
+    attention (the mask built from numpy's triangle helpers)."""
+    for seed, (nq, nk, d) in enumerate([(7, 7, 4), (9, 13, 3), (12, 5, 8)]):
+        r = _rng(200 + seed)
+        q, k, v = (r.standard_normal((n, d)) for n in (nq, nk, nk))
+        for wl, wr in WINDOWS:
+            o, lse = attn_rows_colmask(q, np.arange(nq, dtype=np.int64), k, v, 0.6, False,
+                                       band_as_columns(nk, wl, wr))
+            ob, lb = masked_softmax_numpy(q, k, v, 0.6, band_mask_numpy(nq, nk, wl, wr))
+            np.testing.assert_allclose(o, ob, rtol=1e-12, atol=1e-12, err_msg=str((nq, nk, wl, wr)))
+            np.testing.assert_allclose(lse, lb, rtol=1e-12, atol=1e-12, err_msg=str((nq, nk, wl, wr)))
+
+
+def pin_colmask_documents(attn_rows_colmask):
+    """Document mask: keys of a document are hidden from every later row; with
+    causal on, each document's rows equal causal attention within that document
+    alone (textbook brute force on the slice)."""
+    r = _rng(210)
+    lens = [3, 5, 1, 4, 2]
+    n, d = sum(lens), 4
+    q, k, v = (r.standard_normal((n, d)) for _ in range(3))
+    cols = np.zeros((n, 4), dtype=np.int64)
+    start = 0
+    for ln in lens:
+        cols[start:start + ln, 0] = start + ln
+        cols[start:start + ln, 1] = n
+        start += ln
+    o, lse = attn_rows_colmask(q, np.arange(n, dtype=np.int64), k, v, 0.9, True, cols)
+    start = 0
+    for ln in lens:
+        sl = slice(start, start + ln)
+        ob, lb = brute_force_python(q[sl].tolist(), k[sl].tolist(), v[sl].tolist(), 0.9, True)
+        np.testing.assert_allclose(o[sl], ob, rtol=1e-12, atol=1e-12)
+        np.testing.assert_allclose(lse[sl], lb, rtol=1e-12, atol=1e-12)
+        start += ln
+
+
+def pin_colmask_empty_intervals(attn_rows_colmask):
+    """Empty intervals (lo >= hi, in several spellings) hide nothing: the result
+    is textbook attention, causal or not."""
+    r = _rng(220)
+    n, d = 9, 3
+    q, k, v = (r.standard_normal((n, d)) for _ in range(3))
+    cols = np.array([[0, 0, 5, 5], [7, 2, 3, 3], [9, 9, 100, -100]] * 3, dtype=np.int64)
+    for causal in (False, True):
+        o, lse = attn_rows_colmask(q, np.arange(n, dtype=np.int64), k, v, 0.7, causal, cols)
+        ob, lb = brute_force_python(q.tolist(), k.tolist(), v.tolist(), 0.7, causal)
+        np.testing.assert_allclose(o, ob, rtol=1e-12, atol=1e-12)
+        np.testing.assert_allclose(lse, lb, rtol=1e-12, atol=1e-12)
+
+
+def pin_colmask_two_intervals(attn_rows_colmask):
+    """Row i sees exactly the keys outside both of their intervals: each row
+    equals unmasked attention over that key subset, given as the whole key set
+    (so the second interval, the half-open ends and non-contiguous key sets are
+    all exercised), and rows that see nothing get O = 0, LSE = -inf."""
+    r = _rng(230)
+    n, nk, d = 11, 10, 3
+    q, k, v = (r.standard_normal((n, d)) for n in (n, nk, nk))
+    cols = np.array([[2, 5, 8, 11], [0, 3, 3, 3], [4, 4, 0, 6], [1, 9, 10, 11], [0, 11, 0, 0],
+                     [6, 7, 2, 3], [0, 2, 9, 11], [3, 8, 8, 10], [5, 11, 0, 5], [7, 10, 1, 2]],
+                    dtype=np.int64)
+    rows = np.arange(n, dtype=np.int64)
+    # second set: every key's second interval is [8, 11), so rows 8..10 see nothing
+    cols_b = cols.copy()
+    cols_b[:, 2], cols_b[:, 3] = 8, 11
+    for c in (cols, cols_b):
+        o, lse = attn_rows_colmask(q, rows, k, v, 0.5, False, c)
+        for i in range(n):
+            keep = [j for j in range(nk)
+                    if not (c[j, 0] <= i < c[j, 1]) and not (c[j, 2] <= i < c[j, 3])]
+            if not keep:
+                assert np.all(o[i] == 0.0) and lse[i] == -np.inf, i
+                continue
+            ob, lb = brute_force_python(q[i:i + 1].tolist(), k[keep].tolist(), v[keep].tolist(),
+                                        0.5, False)
+            np.testing.assert_allclose(o[i], ob[0], rtol=1e-12, atol=1e-12, err_msg=str(i))
+            np.testing.assert_allclose(lse[i], lb[0], rtol=1e-12, atol=1e-12, err_msg=str(i))
+    assert np.all(o[8:] == 0.0) and np.all(lse[8:] == -np.inf)
+
+
+COLMASK_PINS = [pin_colmask_band, pin_colmask_documents, pin_colmask_empty_intervals,
+                pin_colmask_two_intervals]
+
+
 ALL_PINS = [
     pin_brute_force, pin_golden, pin_single_key, pin_identical_keys, pin_zero_scale,
     pin_causal_prefix, pin_rows_sum_to_one, pin_shift_invariance, pin_value_linearity,

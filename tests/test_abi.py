@@ -49,7 +49,7 @@ def test_library_exports_every_declared_symbol(header):
 def test_attn_h_declares_the_contract():
     names = declared_functions(os.path.join(ROOT, "include", "attn.h"))
     for n in ("attn_fwd", "attn_fwd_config", "attn_fwd_gqa", "attn_fwd_window", "attn_fwd_varlen",
-              "attn_fwd_fp8", "attn_bwd", "attn_bwd_window", "attn_bwd_noalloc", "attn_bwd_workspace_size", "attn_status_sync", "attn_status_string",
+              "attn_fwd_fp8", "attn_fwd_colmask", "attn_colmask_workspace_size", "attn_bwd", "attn_bwd_window", "attn_bwd_noalloc", "attn_bwd_workspace_size", "attn_status_sync", "attn_status_string",
               "attn_last_error", "attn_selftest_timeout"):
         assert n in names
 
@@ -118,6 +118,34 @@ def test_window_validation():
     assert W(*base[:11], math.nan, 3, 3, None) == 1
     # empty problems are a no-op whatever the band
     assert W(None, None, None, None, None, 0, 4, 2, 8, 8, 64, 0.1, 3, 0, None) == 0
+
+
+def test_colmask_validation():
+    C = binding.attn_fwd_colmask
+    P = (ALIGNED, ALIGNED * 2, ALIGNED * 3, ALIGNED * 16, None)
+    sizes = (1, 4, 2, 8, 8, 64, 0.1, 0)            # B, H, Hkv, Nq, Nk, d, scale, causal
+    M, WS = ALIGNED * 40, ALIGNED * 48
+    need = binding.attn_colmask_workspace_size(1, 1, 8)
+    assert need == 32                              # one key block: two int4 summaries
+    assert binding.attn_colmask_workspace_size(2, 4, 129) == 2 * 4 * 2 * 32
+    assert binding.attn_colmask_workspace_size(-1, 1, 8) == 0
+
+    def call(ptrs=P, sz=sizes, mask=M, hm=1, ws=WS, ws_bytes=need):
+        return C(*ptrs, *sz, mask, hm, ws, ws_bytes, None)
+    assert call(sz=sizes[:7] + (2,)) == 1          # causal flag
+    assert call(hm=3) == 1                         # Hm not in {1, H}
+    assert call(mask=None) == 1
+    assert call(ws=None) == 1
+    assert call(mask=M + 4) == 1                   # misaligned mask
+    assert call(ws=WS + 8) == 1                    # misaligned workspace
+    assert call(ws_bytes=need - 16) == 1           # workspace too small
+    assert call(ws=ALIGNED * 16) == 1              # workspace inside o
+    assert call(ws=M) == 1                         # workspace over the mask
+    assert call(mask=ALIGNED * 16) == 1            # mask inside o
+    assert call(sz=(1, 4, 3) + sizes[3:]) == 1     # H % Hkv
+    assert call(sz=sizes[:5] + (96,) + sizes[6:]) == 2
+    # nothing to compute: a no-op even with null pointers
+    assert C(None, None, None, None, None, 0, 4, 2, 8, 8, 64, 0.1, 0, None, 1, None, 0, None) == 0
 
 
 def test_varlen_validation():

@@ -1,0 +1,72 @@
+"""Column-interval mask builders and their visible-pair counts (CPU)."""
+import numpy as np
+import pytest
+
+from exact_attention_152_b200 import masks
+
+
+def dense_visible(cols, nq, causal):
+    """Boolean [Nq, Nk] visibility of one mask row, element by element."""
+    nk = cols.shape[0]
+    vis = np.ones((nq, nk), dtype=bool)
+    for j in range(nk):
+        lo1, hi1, lo2, hi2 = (int(x) for x in cols[j])
+        for i in range(nq):
+            if lo1 <= i < hi1 or lo2 <= i < hi2 or (causal and j > i):
+                vis[i, j] = False
+    return vis
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_visible_pairs_match_dense_count(causal):
+    m = masks.random_intervals(3, 2, 3, 37, 29)
+    got = masks.visible_pairs(m, 37, causal)
+    for b in range(2):
+        for h in range(3):
+            assert got[b, h] == dense_visible(m[b, h], 37, causal).sum()
+
+
+def test_visible_per_row_matches_dense():
+    m = masks.random_intervals(4, 1, 1, 50, 33)[0, 0]
+    rows = np.array([0, 3, 17, 49])
+    for causal in (False, True):
+        want = dense_visible(m, 50, causal)[rows].sum(axis=1)
+        assert np.array_equal(masks.visible_per_row(m, rows, causal), want)
+
+
+def test_random_intervals_cover_the_cases():
+    m = masks.random_intervals(5, 1, 1, 64, 4096).reshape(-1, 4).astype(np.int64)
+    assert np.all(m[:, 0] <= m[:, 1]) and np.all(m[:, 2] <= m[:, 3])
+    assert np.any(m[:, 0] == m[:, 1]) or np.any(m[:, 0] > 63)        # some empty for all rows
+    assert np.any((m[:, 0] <= 0) & (m[:, 1] >= 64))                   # some hide every row
+    assert np.any((m[:, 0] > 0) & (m[:, 1] < 64))                     # some cut rows in the middle
+
+
+def test_band_columns_are_the_band():
+    for wl, wr in [(3, 0), (-1, 0), (2, 5), (-1, 4), (0, 0)]:
+        m = masks.band(1, 20, wl, wr)[0, 0]
+        vis = dense_visible(m, 20, False)
+        i, j = np.meshgrid(np.arange(20), np.arange(20), indexing="ij")
+        want = np.ones((20, 20), dtype=bool)
+        if wl >= 0:
+            want &= j >= i - wl
+        if wr >= 0:
+            want &= j <= i + wr
+        assert np.array_equal(vis, want), (wl, wr)
+
+
+def test_documents_are_block_diagonal():
+    lens = [5, 1, 7, 3]
+    m = masks.documents([lens], 16)[0, 0]
+    doc = np.repeat(np.arange(len(lens)), lens)
+    i, j = np.meshgrid(np.arange(16), np.arange(16), indexing="ij")
+    assert np.array_equal(dense_visible(m, 16, True), (doc[i] == doc[j]) & (j <= i))
+    mb = masks.documents([lens], 16, bidirectional=True)[0, 0]
+    assert np.array_equal(dense_visible(mb, 16, False), doc[i] == doc[j])
+    assert masks.visible_pairs(m[None, None], 16, True)[0, 0] == sum(n * (n + 1) // 2 for n in lens)
+
+
+def test_prefix_lm():
+    m = masks.prefix_lm(1, 12, 4)[0, 0]
+    i, j = np.meshgrid(np.arange(12), np.arange(12), indexing="ij")
+    assert np.array_equal(dense_visible(m, 12, False), (j < 4) | (j <= i))

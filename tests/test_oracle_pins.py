@@ -17,6 +17,11 @@ def test_oracle_pin(pin):
     pin(oracle.attn_rows)
 
 
+@pytest.mark.parametrize("pin", pins.COLMASK_PINS, ids=[p.__name__ for p in pins.COLMASK_PINS])
+def test_oracle_colmask_pin(pin):
+    pin(oracle.attn_rows_colmask)
+
+
 @pytest.mark.parametrize("pin", pins.WINDOW_PINS, ids=[p.__name__ for p in pins.WINDOW_PINS])
 def test_oracle_window_pin(pin):
     pin(oracle.attn_rows_window)
@@ -93,6 +98,11 @@ MUTANTS = {
     "bwd_dv_with_ds": ("dv[j * d + c] += p[j] * gi[c];", "dv[j * d + c] += ds * gi[c];"),
     "bwd_dp_against_k": ("for (int64_t c = 0; c < d; ++c) dot += gi[c] * v[j * d + c];",
                          "for (int64_t c = 0; c < d; ++c) dot += gi[c] * k[j * d + c];"),
+    "cols_hi_inclusive": ("(c[0] <= i && i < c[1])", "(c[0] <= i && i <= c[1])"),
+    "cols_second_interval_ignored": ("(c[2] <= i && i < c[3])", "(0 && i < c[3])"),
+    "cols_causal_ignored": ("(jb->causal && j > i)", "(0 && j > i)"),
+    "cols_value_not_gathered": ("const double *vj = jb->v + jb->vis[t] * d;",
+                                "const double *vj = jb->v + t * d;"),
     "bwd_band_ignored": ("if (window_right >= 0 && i + window_right < hi) hi = i + window_right;",
                          "if (0) hi = i + window_right;"),
 }
@@ -138,6 +148,16 @@ def _build_mutant(tmp_path, name, old, new):
     def attn_rows_window(q_rows, rows, k, v, scale, wl, wr):
         return call(w, q_rows, rows, k, v, scale, int(wl), int(wr))
 
+    cm = cdll.oracle_attn_rows_colmask_f64
+    cm.restype = ctypes.c_int
+    cm.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p,
+                   ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64, ctypes.c_double,
+                   ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int]
+
+    def attn_rows_colmask(q_rows, rows, k, v, scale, causal, cols):
+        cols = np.ascontiguousarray(cols, dtype=np.int64)
+        return call(cm, q_rows, rows, k, v, scale, int(causal), cols.ctypes.data)
+
     b = cdll.oracle_attn_bwd_f64
     b.restype = ctypes.c_int
     b.argtypes = [ctypes.c_void_p] * 4 + [ctypes.c_int64] * 3 + [ctypes.c_double] + \
@@ -152,16 +172,17 @@ def _build_mutant(tmp_path, name, old, new):
           int(wl), int(wr), dq.ctypes.data, dk.ctypes.data, dv.ctypes.data)
         return dq, dk, dv
 
-    return attn_rows, attn_rows_window, attn_bwd_head
+    return attn_rows, attn_rows_window, attn_bwd_head, attn_rows_colmask
 
 
 @pytest.mark.parametrize("name", sorted(MUTANTS))
 def test_planted_mistake_is_caught(tmp_path, name):
     old, new = MUTANTS[name]
-    rows_fn, window_fn, bwd_fn = _build_mutant(tmp_path, name, old, new)
+    rows_fn, window_fn, bwd_fn, colmask_fn = _build_mutant(tmp_path, name, old, new)
     failed = []
     for pin_set, args in ((PINS, (rows_fn,)), (pins.WINDOW_PINS, (window_fn,)),
-                          (pins.BWD_PINS, (bwd_fn, window_fn))):
+                          (pins.BWD_PINS, (bwd_fn, window_fn)),
+                          (pins.COLMASK_PINS, (colmask_fn,))):
         for pin in pin_set:
             try:
                 pin(*args)
