@@ -302,6 +302,12 @@ def run_reference_bwd(args, w, per_step):
     return 0
 
 
+def bwd_launch_name(w):
+    if w.packed:
+        return "attn_bwd_varlen"
+    return "attn_bwd_window" if w.window is not None else "attn_bwd"
+
+
 def launch_name(w):
     if w.colmask:
         return "attn_fwd_colmask"
@@ -561,23 +567,32 @@ def bwd_cpu_baseline(w, seconds):
     from exact_attention_152_b200 import inputs
     from exact_attention_152_b200.workloads import visible_keys
     wl, wr = w.band
-    k, v = (inputs.bf16_bits_to_f64(w.head_bits(x, w.kv_head_of(0))) for x in "kv")
+    if w.packed:  # sequence 0, head 0
+        nq = nk = w.seqlens[0]
+        k, v = (inputs.bf16_bits_to_f64(w.seq_head_bits(x, 0, 0)) for x in "kv")
+        q_of = lambda rows: w.seq_head_bits("q", 0, 0, rows)  # noqa: E731
+        flat = lambda rows: (rows[:, None] * w.H) * w.d + np.arange(w.d)[None, :]  # noqa: E731
+    else:
+        nq, nk = w.Nq, w.Nk
+        k, v = (inputs.bf16_bits_to_f64(w.head_bits(x, w.kv_head_of(0))) for x in "kv")
+        q_of = lambda rows: w.q_rows_bits(0, rows)  # noqa: E731
+        flat = lambda rows: rows[:, None] * w.d + np.arange(w.d)[None, :]  # noqa: E731
     n, dt = 64, 0.0
     while True:
-        rows = np.arange(n, dtype=np.int64)
-        q = inputs.bf16_bits_to_f64(w.q_rows_bits(0, rows))
-        g = inputs.bf16_bits_to_f64(inputs.gen_bf16_at(w.seed + 1, "q", rows[:, None] * w.d
-                                                       + np.arange(w.d)[None, :]))
+        rows = np.arange(min(n, nq), dtype=np.int64)
+        q = inputs.bf16_bits_to_f64(q_of(rows))
+        g = inputs.bf16_bits_to_f64(inputs.gen_bf16_at(w.seed + 1, "q", flat(rows)))
         t0 = time.perf_counter()
         oracle.attn_bwd_head(q, k, v, g, w.scale, wl, wr)
         dt = time.perf_counter() - t0
-        if dt > seconds / 4 or n >= w.Nq:
+        if dt > seconds / 4 or n >= nq:
             break
-        n = min(w.Nq, n * 4)
-    flops = 2.5 * 4.0 * w.d * float(visible_keys(rows, w.Nk, wl, wr).sum())
+        n = min(nq, n * 4)
+    flops = 2.5 * 4.0 * w.d * float(visible_keys(rows, nk, wl, wr).sum())
+    where = "sequence 0, head 0" if w.packed else "head 0"
     return {"value": flops / dt / 1e12, "unit": UNIT, "cores": 1, "kind": "oracle",
-            "sample": f"backward of the first {n} query rows of head 0 of {w.name} against all "
-                      f"its keys, fp64, one thread, {dt:.1f} s"}
+            "sample": f"backward of the first {len(rows)} query rows of {where} of {w.name} against "
+                      f"all its keys, fp64, one thread, {dt:.1f} s"}
 
 
 def run_ours_bwd(args):
@@ -595,24 +610,39 @@ def run_ours_bwd(args):
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
     w = WORKLOADS[args.workload or HEADLINE]
-    if w.packed or w.window is not None:
-        raise SystemExit("--pass bwd supports dense workloads, causal or not")
+    if w.fp8 or w.colmask:
+        raise SystemExit("--pass bwd: no backward for E4M3 or column-interval workloads")
     peaks = load_peaks()
     host = {x: w.tensor_bits(x) for x in "qkv"}
     host["do"] = inputs.gen_bf16(w.seed + 1, "q", w.shape("q"))
     to_dev = lambda a: torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).to(dev)  # noqa: E731
     q, k, v, do = (to_dev(host[x]) for x in ("q", "k", "v", "do"))
-    o, lse = binding.fwd(q, k, v, causal=w.causal, scale=w.scale)
+    if w.packed:
+        cu = torch.from_numpy(w.cu_seqlens).to(dev)
+        o, lse = binding.fwd_varlen(q, k, v, cu, cu, max(w.seqlens), scale=w.scale, window=w.band)
+        ws_bytes = binding.attn_bwd_workspace_size(1, w.H, w.total, w.d)
+    else:
+        cu = None
+        o, lse = binding.fwd(q, k, v, causal=w.causal, scale=w.scale, window=w.window)
+        ws_bytes = binding.attn_bwd_workspace_size(w.B, w.H, w.Nq, w.d)
     stream = torch.cuda.current_stream(dev)
     sh = stream.cuda_stream
-    ws_bytes = binding.attn_bwd_workspace_size(w.B, w.H, w.Nq, w.d)
     ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
     dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
 
-    def launch(ins=(q, k, v, o, do, lse), outs=(dq, dk, dv)):
-        rc = binding.attn_bwd(*(t.data_ptr() for t in ins), *(t.data_ptr() for t in outs),
-                              ws.data_ptr(), ws_bytes, w.B, w.H, w.kv_heads, w.Nq, w.Nk, w.d,
-                              w.scale, int(w.causal), sh)
+    def launch(ins=(q, k, v, o, do, lse, cu), outs=(dq, dk, dv)):
+        ptrs = [t.data_ptr() for t in ins[:6]] + [t.data_ptr() for t in outs]
+        if w.packed:
+            c = ins[6].data_ptr()
+            rc = binding.attn_bwd_varlen(*ptrs, ws.data_ptr(), ws_bytes, c, c, len(w.seqlens),
+                                         max(w.seqlens), w.total, w.total, w.H, w.kv_heads, w.d,
+                                         w.scale, w.band[0], w.band[1], sh)
+        elif w.window is not None:
+            rc = binding.attn_bwd_window(*ptrs, ws.data_ptr(), ws_bytes, w.B, w.H, w.kv_heads,
+                                         w.Nq, w.Nk, w.d, w.scale, w.band[0], w.band[1], sh)
+        else:
+            rc = binding.attn_bwd(*ptrs, ws.data_ptr(), ws_bytes, w.B, w.H, w.kv_heads, w.Nq, w.Nk,
+                                  w.d, w.scale, int(w.causal), sh)
         binding.check(rc, "attn_bwd")
 
     launch()
@@ -641,14 +671,15 @@ def run_ours_bwd(args):
 
     # end to end: pinned host Q, K, V, O, dO, LSE -> H2D -> attn_bwd -> D2H dQ, dK, dV
     pin = lambda t: t.cpu().pin_memory()  # noqa: E731
-    h_in = [pin(t) for t in (q, k, v, o, do, lse)]
+    ins = (q, k, v, o, do, lse) + ((cu,) if w.packed else ())
+    h_in = [pin(t) for t in ins]
     h_out = [torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in (dq, dk, dv)]
-    d_in = [torch.empty_like(t) for t in (q, k, v, o, do, lse)]
+    d_in = [torch.empty_like(t) for t in ins]
 
     def e2e_step():
         for d_, h_ in zip(d_in, h_in):
             d_.copy_(h_, non_blocking=True)
-        launch(tuple(d_in))
+        launch(tuple(d_in) + ((None,) if not w.packed else ()))
         for h_, d_ in zip(h_out, (dq, dk, dv)):
             h_.copy_(d_, non_blocking=True)
 
@@ -683,7 +714,8 @@ def run_ours_bwd(args):
                 "h2d_bytes_per_step": sum(t.numel() * t.element_size() for t in h_in),
                 "d2h_bytes_per_step": sum(t.numel() * t.element_size() for t in h_out),
                 "steps": args.e2e_steps,
-                "path": "pinned host Q/K/V/O/dO/LSE -> H2D -> attn_bwd (C-ABI) -> D2H of dQ/dK/dV"},
+                "path": f"pinned host Q/K/V/O/dO/LSE{' + offsets' if w.packed else ''} -> H2D -> "
+                        f"{bwd_launch_name(w)} (C-ABI) -> D2H of dQ/dK/dV"},
         "gpu_launches": 3 * K,
         "clocks": clocks,
         "kernel_src_sha": kernel_source_hash("bwd"),

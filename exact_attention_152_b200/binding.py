@@ -65,6 +65,9 @@ def lib() -> ctypes.CDLL:
             l.attn_bwd.restype = _I
             l.attn_bwd_window.argtypes = [_P] * 10 + [ctypes.c_size_t] + [_I] * 6 + [ctypes.c_float, _I, _I, _P]
             l.attn_bwd_window.restype = _I
+            l.attn_bwd_varlen.argtypes = [_P] * 10 + [ctypes.c_size_t, _P, _P] + [_I] * 7 + \
+                [ctypes.c_float, _I, _I, _P]
+            l.attn_bwd_varlen.restype = _I
             l.attn_bwd_noalloc.argtypes = [_P] * 9 + [_I] * 6 + [ctypes.c_float, _I, _P]
             l.attn_bwd_noalloc.restype = _I
             l.attn_bwd_workspace_size.argtypes = [_I, _I, _I, _I]
@@ -134,6 +137,14 @@ def attn_bwd_window(q, k, v, o, dout, lse, dq, dk, dv, workspace, workspace_byte
                     d, scale, window_left, window_right, stream) -> int:
     return lib().attn_bwd_window(q, k, v, o, dout, lse, dq, dk, dv, workspace, workspace_bytes, B, H,
                                  Hkv, Nq, Nk, d, scale, window_left, window_right, stream)
+
+
+def attn_bwd_varlen(q, k, v, o, dout, lse, dq, dk, dv, workspace, workspace_bytes, cu_seqlens_q,
+                    cu_seqlens_k, num_seqs, max_seqlen_k, total_q, total_k, H, Hkv, d, scale,
+                    window_left, window_right, stream) -> int:
+    return lib().attn_bwd_varlen(q, k, v, o, dout, lse, dq, dk, dv, workspace, workspace_bytes,
+                                 cu_seqlens_q, cu_seqlens_k, num_seqs, max_seqlen_k, total_q, total_k,
+                                 H, Hkv, d, scale, window_left, window_right, stream)
 
 
 def attn_bwd_noalloc(q, k, v, o, dout, lse, dq, dk, dv, B, H, Hkv, Nq, Nk, d, scale, causal,
@@ -361,6 +372,57 @@ def bwd(q, k, v, o, dout, lse, causal: bool = False, scale: float | None = None,
     else:
         rc = attn_bwd(*ptrs, B, H, Hkv, Nq, Nk, d, float(scale), int(bool(causal)), stream)
         check(rc, "attn_bwd")
+    return dq, dk, dv
+
+
+def bwd_varlen(q, k, v, o, dout, lse, cu_seqlens_q, cu_seqlens_k, max_seqlen_k: int,
+               causal: bool = False, scale: float | None = None, *, window=None, workspace=None):
+    """Gradients (dq, dk, dv) of fwd_varlen: q/o/dout [total_q, H, d], k/v
+    [total_k, Hkv, d] BF16 CUDA tensors, lse [H, total_q] fp32, int32 CUDA
+    offsets.  ``window`` = (left, right) replaces ``causal``.  The workspace
+    (attn_bwd_workspace_size(1, H, total_q, d) bytes) is allocated when not
+    given.  Key rows that belong to no sequence are left as torch.empty made
+    them.  Runs on torch's current stream."""
+    import torch
+
+    _check_bf16(q=q, k=k, v=v, o=o, dout=dout)
+    if q.dim() != 3 or k.dim() != 3 or v.dim() != 3:
+        raise ValueError("q, k, v must be [total, heads, d]")
+    total_q, H, d = q.shape
+    total_k, Hkv = k.shape[0], k.shape[1]
+    if tuple(o.shape) != tuple(q.shape) or tuple(dout.shape) != tuple(q.shape):
+        raise ValueError("o and dout must match q")
+    if tuple(k.shape) != (total_k, Hkv, d) or tuple(v.shape) != (total_k, Hkv, d):
+        raise ValueError("k and v must be [total_k, Hkv, d] matching q")
+    if lse.dtype != torch.float32 or not lse.is_contiguous() or tuple(lse.shape) != (H, total_q):
+        raise ValueError("lse must be contiguous float32 [H, total_q]")
+    for name, c in (("cu_seqlens_q", cu_seqlens_q), ("cu_seqlens_k", cu_seqlens_k)):
+        if not isinstance(c, torch.Tensor) or c.dtype != torch.int32 or not c.is_cuda \
+                or c.dim() != 1 or not c.is_contiguous():
+            raise TypeError(f"{name} must be a contiguous int32 CUDA vector")
+    if cu_seqlens_q.numel() != cu_seqlens_k.numel() or cu_seqlens_q.numel() < 1:
+        raise ValueError("cu_seqlens_q and cu_seqlens_k need the same num_seqs + 1 entries")
+    num_seqs = cu_seqlens_q.numel() - 1
+    if window is None:
+        window = (-1, 0) if causal else (-1, -1)
+    elif causal:
+        raise ValueError("window replaces causal")
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    need = attn_bwd_workspace_size(1, H, total_q, d)
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
+    dq = torch.empty_like(q)
+    dk = torch.empty_like(k)
+    dv = torch.empty_like(v)
+    stream = torch.cuda.current_stream(q.device).cuda_stream
+    rc = attn_bwd_varlen(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), dout.data_ptr(),
+                         lse.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(),
+                         workspace.data_ptr(), workspace.numel() * workspace.element_size(),
+                         cu_seqlens_q.data_ptr(), cu_seqlens_k.data_ptr(), num_seqs,
+                         int(max_seqlen_k), total_q, total_k, H, Hkv, d, float(scale),
+                         int(window[0]), int(window[1]), stream)
+    check(rc, "attn_bwd_varlen")
     return dq, dk, dv
 
 

@@ -99,11 +99,15 @@ struct Cfg {
 };
 
 struct BwdParams {
-  const float* lse;    // [B*H, Nq], natural log
-  const float* dsum;   // D = rowsum(dO * O), [B*H, Nq]
-  float* dq_acc;       // [B*H, Nq, d] fp32, zeroed before the launch
+  const float* lse;    // [B*H, Nq], natural log (packed: [H, total_q])
+  const float* dsum;   // D = rowsum(dO * O), [B*H, Nq] (packed: [total_q, H])
+  float* dq_acc;       // [B*H, Nq, d] fp32 (packed: [total_q, H, d]), zeroed before the launch
+  const int* cu_q;     // packed variable-length batch: sequence starts (B + 1), else null
+  const int* cu_k;
+  __nv_bfloat16* dk;   // packed outputs, for rows stored one by one at a sequence's end
+  __nv_bfloat16* dv;
   uint64_t timeout_ns;
-  int Nq, Nk, H, group, n_kblocks, n_qtiles;
+  int Nq, Nk, H, group, n_kblocks, n_qtiles;  // packed: Nq, Nk = total_q, total_k
   int wl, wr;          // key band i - wl <= j <= i + wr (kUnbounded: no bound)
   float scale_log2;    // scale * log2(e)
   float scale;
@@ -147,8 +151,16 @@ struct Smem {
 // tiles_per_head - 1 that can see one of the block's keys.
 struct Work {
   int bh_kv, j, b, hkv, i_lo, tiles_per_head, n_it;
+  bool packed;   // a compile-time constant per kernel instance
+  int Nq, Nk;    // packed: the sequence's lengths
+  int q0, k0;    // packed: the sequence's first rows
   __device__ __forceinline__ int head_of(int it) const { return it / tiles_per_head; }
   __device__ __forceinline__ int tile_of(int it) const { return i_lo + it % tiles_per_head; }
+  // lengths and first rows of this CTA's problem (dense: the launch's, from 0)
+  __device__ __forceinline__ int nq(const BwdParams& p) const { return packed ? Nq : p.Nq; }
+  __device__ __forceinline__ int nk(const BwdParams& p) const { return packed ? Nk : p.Nk; }
+  __device__ __forceinline__ int row_q0() const { return packed ? q0 : 0; }
+  __device__ __forceinline__ int row_k0() const { return packed ? k0 : 0; }
 };
 
 __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, uint64_t timeout_ns) {
@@ -193,6 +205,14 @@ struct Mma {
   }
 };
 
+// Tensor-map coordinates (column, row, head) in the map's dimension order:
+// dense maps are [BH, N, d], packed maps [total, H, d].
+__device__ __forceinline__ void load_rows(uint32_t dst, const CUtensorMap* tm, int col, int row, int head,
+                                          bool packed, uint32_t bar) {
+  if (packed) tma_load_3d(dst, tm, col, head, row, bar);
+  else tma_load_3d(dst, tm, col, row, head, bar);
+}
+
 // ---------------------------------------------------------------------------
 // Producer warp: K, V once; then Q, dO (TMA) and LSE, D (plain loads) per tile.
 // ---------------------------------------------------------------------------
@@ -206,8 +226,11 @@ __device__ __forceinline__ void producer_role(const Smem<D>& sm, const CUtensorM
     mbar_arrive_expect_tx(sm.kv_full(), 2 * C::kTileBytes);
 #pragma unroll
     for (int b = 0; b < C::kBoxes; ++b) {
-      tma_load_3d(sm.k() + b * C::kBoxBytes, tm_k, b * 64, w.j * kBlockK, w.bh_kv, sm.kv_full());
-      tma_load_3d(sm.v() + b * C::kBoxBytes, tm_v, b * 64, w.j * kBlockK, w.bh_kv, sm.kv_full());
+      const int kh = w.packed ? w.hkv : w.bh_kv;
+      load_rows(sm.k() + b * C::kBoxBytes, tm_k, b * 64, w.row_k0() + w.j * kBlockK, kh, w.packed,
+                sm.kv_full());
+      load_rows(sm.v() + b * C::kBoxBytes, tm_v, b * 64, w.row_k0() + w.j * kBlockK, kh, w.packed,
+                sm.kv_full());
     }
   }
   bool ok = true;
@@ -217,25 +240,42 @@ __device__ __forceinline__ void producer_role(const Smem<D>& sm, const CUtensorM
     const uint32_t ph = (it >> 1) & 1;
     ok = warp_wait(sm.q_empty(s), ph ^ 1u, prm.timeout_ns);
     if (!ok) break;
-    const int bh = w.b * prm.H + w.hkv * prm.group + w.head_of(it);
+    const int h = w.hkv * prm.group + w.head_of(it);  // query head within the batch entry
+    const int bh = w.b * prm.H + h;
     const int q0 = w.tile_of(it) * kBlockQ;
-    // -LSE * log2(e) per query row (rows past Nq: -inf, so P = 0 there), and D
+    // -LSE * log2(e) per query row (rows past the sequence: -inf, so P = 0
+    // there), and D.  Dense: both [B*H, Nq]; packed: LSE [H, total_q], D
+    // [total_q, H].
     float* nl = sm.lse2(s);
     float* dd = sm.dsum(s);
+    if (w.packed) {
+      const size_t lse0 = static_cast<size_t>(h) * prm.Nq + w.q0;
+      const size_t d0 = static_cast<size_t>(w.q0) * prm.H + h;
 #pragma unroll
-    for (int r = lane; r < kBlockQ; r += 32) {
-      const int q = q0 + r;
-      const bool in = q < prm.Nq;
-      const size_t row = static_cast<size_t>(bh) * prm.Nq + q;
-      nl[r] = in ? -prm.lse[row] * kLog2e : -INFINITY;
-      dd[r] = in ? prm.dsum[row] : 0.0f;
+      for (int r = lane; r < kBlockQ; r += 32) {
+        const int q = q0 + r;
+        const bool in = q < w.Nq;
+        nl[r] = in ? -prm.lse[lse0 + q] * kLog2e : -INFINITY;
+        dd[r] = in ? prm.dsum[d0 + static_cast<size_t>(q) * prm.H] : 0.0f;
+      }
+    } else {
+#pragma unroll
+      for (int r = lane; r < kBlockQ; r += 32) {
+        const int q = q0 + r;
+        const bool in = q < prm.Nq;
+        const size_t row = static_cast<size_t>(bh) * prm.Nq + q;
+        nl[r] = in ? -prm.lse[row] * kLog2e : -INFINITY;
+        dd[r] = in ? prm.dsum[row] : 0.0f;
+      }
     }
     if (lane == 0) {
       mbar_arrive_expect_tx(sm.q_full(s), 2 * C::kTileBytes);
+      const int qh = w.packed ? h : bh;
 #pragma unroll
       for (int b = 0; b < C::kBoxes; ++b) {
-        tma_load_3d(sm.q(s) + b * C::kBoxBytes, tm_q, b * 64, q0, bh, sm.q_full(s));
-        tma_load_3d(sm.dout(s) + b * C::kBoxBytes, tm_do, b * 64, q0, bh, sm.q_full(s));
+        load_rows(sm.q(s) + b * C::kBoxBytes, tm_q, b * 64, w.row_q0() + q0, qh, w.packed, sm.q_full(s));
+        load_rows(sm.dout(s) + b * C::kBoxBytes, tm_do, b * 64, w.row_q0() + q0, qh, w.packed,
+                  sm.q_full(s));
       }
     } else {
       mbar_arrive(sm.q_full(s));
@@ -320,7 +360,7 @@ __device__ __forceinline__ bool softmax_grad_role(const Smem<D>& sm, uint32_t tm
   const int q4 = warp & 3, c = warp >> 2;
   const int r = q4 * 32 + lane;          // key row within the block
   const int key = w.j * kBlockK + r;
-  const bool key_in = key < prm.Nk;
+  const bool key_in = key < w.nk(prm);
   const uint32_t lane_off = static_cast<uint32_t>(q4 * 32) << 16;
   const uint32_t tS = tmem + lane_off + c * 64;
   const uint32_t tP = tmem + lane_off + C::kTmemDP + c * 64;
@@ -443,8 +483,11 @@ __device__ __forceinline__ bool dq_drain_role(const Smem<D>& sm, uint32_t tmem, 
     ok = warp_wait(sm.dq_full(), it & 1, prm.timeout_ns);
     if (!ok) break;
     tc_fence_after();
-    const int bh = w.b * prm.H + w.hkv * prm.group + w.head_of(it);
-    const int row0 = w.tile_of(it) * kBlockQ + q4 * 32;
+    const int h = w.hkv * prm.group + w.head_of(it);
+    const int qh = w.packed ? h : w.b * prm.H + h;
+    // rows past a packed sequence's end reduce exact zeros (P = 0 there) into
+    // the next sequence's rows, which leaves them unchanged
+    const int row0 = w.row_q0() + w.tile_of(it) * kBlockQ + q4 * 32;
     // all of this warp's dQ columns into registers, then TMEM is free
     uint32_t v[kHalves][2][32];
 #pragma unroll
@@ -478,8 +521,13 @@ __device__ __forceinline__ bool dq_drain_role(const Smem<D>& sm, uint32_t tmem, 
       fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) {
-        tma_reduce_add_3d(tm_dq, stage_s, 64 * hf, row0, bh);
-        tma_reduce_add_3d(tm_dq, stage_s + 4096, 64 * hf + 32, row0, bh);
+        if (w.packed) {
+          tma_reduce_add_3d(tm_dq, stage_s, 64 * hf, qh, row0);
+          tma_reduce_add_3d(tm_dq, stage_s + 4096, 64 * hf + 32, qh, row0);
+        } else {
+          tma_reduce_add_3d(tm_dq, stage_s, 64 * hf, row0, qh);
+          tma_reduce_add_3d(tm_dq, stage_s + 4096, 64 * hf + 32, row0, qh);
+        }
         bulk_commit_group();
       }
     }
@@ -506,6 +554,9 @@ __device__ __forceinline__ bool epilogue(const Smem<D>& sm, uint32_t tmem, const
   tc_fence_after();
   const uint32_t lane_off = static_cast<uint32_t>(q4 * 32) << 16;
   constexpr int kBoxesPerWarp = D == 128 ? 2 : 1;
+  // a packed sequence ending inside this warp's 32 rows: a TMA store would
+  // write into the next sequence, so each row stores itself
+  const bool ragged = w.packed && w.j * kBlockK + q4 * 32 + 32 > w.Nk;
 #pragma unroll
   for (int bx = 0; bx < kBoxesPerWarp; ++bx) {
     // which tensor and which 64 columns
@@ -525,18 +576,33 @@ __device__ __forceinline__ bool epilogue(const Smem<D>& sm, uint32_t tmem, const
 #pragma unroll
       for (int i = 0; i < 16; ++i)
         wv[i] = pack_bf16x2(__uint_as_float(v[2 * i]) * mul, __uint_as_float(v[2 * i + 1]) * mul);
+      if (ragged) {
+        const int key = w.j * kBlockK + q4 * 32 + lane;
+        if (key < w.Nk) {
+          const int hkv_all = prm.H / prm.group;
+          __nv_bfloat16* out = (is_k ? prm.dk : prm.dv) +
+                               (static_cast<size_t>(w.k0 + key) * hkv_all + w.hkv) * D + col0 + 32 * h;
+          uint4* dst = reinterpret_cast<uint4*>(out);
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const int chunk = (4 * h + i) ^ (lane & 7);
-        *reinterpret_cast<uint4*>(stage + lane * 128 + chunk * 16) =
-            make_uint4(wv[4 * i], wv[4 * i + 1], wv[4 * i + 2], wv[4 * i + 3]);
+          for (int i = 0; i < 4; ++i) dst[i] = make_uint4(wv[4 * i], wv[4 * i + 1], wv[4 * i + 2], wv[4 * i + 3]);
+        }
+      } else {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int chunk = (4 * h + i) ^ (lane & 7);
+          *reinterpret_cast<uint4*>(stage + lane * 128 + chunk * 16) =
+              make_uint4(wv[4 * i], wv[4 * i + 1], wv[4 * i + 2], wv[4 * i + 3]);
+        }
       }
     }
     fence_proxy_async_smem();
     __syncwarp();
     const int row0 = w.j * kBlockK + q4 * 32;
-    if (lane == 0 && row0 < prm.Nk) {
-      tma_store_3d(is_k ? tm_dk : tm_dv, smem_u32(stage), col0, row0, w.bh_kv);
+    if (lane == 0 && !ragged && row0 < w.nk(prm)) {
+      if (w.packed)
+        tma_store_3d(is_k ? tm_dk : tm_dv, smem_u32(stage), col0, w.hkv, w.k0 + row0);
+      else
+        tma_store_3d(is_k ? tm_dk : tm_dv, smem_u32(stage), col0, row0, w.bh_kv);
       bulk_commit_group();
     }
   }
@@ -544,7 +610,7 @@ __device__ __forceinline__ bool epilogue(const Smem<D>& sm, uint32_t tmem, const
   return true;
 }
 
-template <int D, bool MASK>
+template <int D, bool MASK, bool PACKED>
 __global__ void __launch_bounds__(kNumThreads, 1)
 attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                 const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
@@ -569,20 +635,46 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   const int hkv_per_b = prm.H / prm.group;
   w.b = w.bh_kv / hkv_per_b;
   w.hkv = w.bh_kv % hkv_per_b;
+  // a compile-time constant in each instance, so the dense kernel carries none
+  // of the packed layout's bookkeeping
+  w.packed = PACKED;
+  if (PACKED) {
+    // packed variable-length batch: sequence b owns query rows cu_q[b] ..
+    // cu_q[b+1]-1 and key rows cu_k[b] .. cu_k[b+1]-1.  Offsets that do not
+    // describe sequences inside the tensors, or a key length beyond the grid,
+    // are reported and the CTA does nothing (every access stays in bounds).
+    const int a = __ldg(prm.cu_q + w.b), e = __ldg(prm.cu_q + w.b + 1);
+    const int c = __ldg(prm.cu_k + w.b), f = __ldg(prm.cu_k + w.b + 1);
+    if (a < 0 || e < a || e > prm.Nq || c < 0 || f < c || f > prm.Nk ||
+        f - c > prm.n_kblocks * kBlockK) {
+      if (threadIdx.x == 0 && w.j == 0 && w.hkv == 0) atomicOr(&g_status_bwd, kStatusWordBadSeqlens);
+      return;
+    }
+    w.Nq = e - a;
+    w.Nk = f - c;
+    w.q0 = a;
+    w.k0 = c;
+    if (w.j * kBlockK >= w.Nk) return;  // this sequence has no key in the block
+  } else {
+    w.Nq = w.Nk = w.q0 = w.k0 = 0;  // unused: the launch's sizes apply
+  }
+  // query tiles (packed: at least one -- a sequence without queries still runs
+  // one fully masked tile, so dK = dV = 0 come out of TMEM)
+  const int n_qtiles = PACKED ? (w.Nq > 0 ? (w.Nq + kBlockQ - 1) / kBlockQ : 1) : prm.n_qtiles;
   // query tiles that can see a key of this block: i - wl <= j <= i + wr for
   // some key j in [j0, j0 + 127] and query i of the tile; a block no query
   // sees still runs one fully masked tile, so dK = dV = 0 come out of TMEM
   w.i_lo = 0;
-  w.tiles_per_head = prm.n_qtiles;
+  w.tiles_per_head = n_qtiles;
   if (MASK) {
     const long long j0 = static_cast<long long>(w.j) * kBlockK;
-    long long lo = 0, hi = prm.n_qtiles - 1;
+    long long lo = 0, hi = n_qtiles - 1;
     if (prm.wr < kUnbounded && j0 - prm.wr > 0) lo = (j0 - prm.wr) / kBlockQ;
     if (prm.wl < kUnbounded) {
       const long long last = (j0 + kBlockK - 1 + prm.wl) / kBlockQ;
       if (last < hi) hi = last;
     }
-    if (lo > hi) lo = hi = (lo < prm.n_qtiles - 1 ? lo : prm.n_qtiles - 1);
+    if (lo > hi) lo = hi = (lo < n_qtiles - 1 ? lo : n_qtiles - 1);
     w.i_lo = static_cast<int>(lo);
     w.tiles_per_head = static_cast<int>(hi - lo + 1);
   }
@@ -677,9 +769,9 @@ __global__ void dq_finish_kernel(const float4* __restrict__ acc, uint2* __restri
   }
 }
 
-template <int D, bool MASK>
+template <int D, bool MASK, bool PACKED>
 int launch_main(const CUtensorMap* maps, const BwdParams& prm, int grid, cudaStream_t stream) {
-  auto kern = attn_bwd_kernel<D, MASK>;
+  auto kern = attn_bwd_kernel<D, MASK, PACKED>;
   static std::once_flag once[kMaxDeviceCount];
   static cudaError_t err[kMaxDeviceCount];
   int dev = 0;
@@ -700,6 +792,51 @@ size_t align256(size_t x) { return (x + 255) / 256 * 256; }
 
 size_t workspace_bytes(long long BH, long long Nq, int d) {
   return align256(static_cast<size_t>(BH) * Nq * 4) + static_cast<size_t>(BH) * Nq * d * 4;
+}
+
+// D rows, the main kernel and dQ's conversion, shared by the dense and packed
+// entries once the tensor maps and parameters are set up.
+int run_bwd(const CUtensorMap* maps, BwdParams& prm, const void* o, const void* dout, void* dq,
+            size_t rows, int d, bool mask, int grid, cudaStream_t stream) {
+  cudaError_t e = cudaMemsetAsync(prm.dq_acc, 0, rows * d * 4, stream);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync");
+  {
+    const unsigned blocks = static_cast<unsigned>(std::min<size_t>((rows + 7) / 8, 148 * 16));
+    float* dsum = const_cast<float*>(prm.dsum);
+    if (d == 128)
+      row_dot_kernel<128><<<blocks, 256, 0, stream>>>(static_cast<const __nv_bfloat16*>(o),
+                                                      static_cast<const __nv_bfloat16*>(dout), dsum, rows);
+    else
+      row_dot_kernel<64><<<blocks, 256, 0, stream>>>(static_cast<const __nv_bfloat16*>(o),
+                                                     static_cast<const __nv_bfloat16*>(dout), dsum, rows);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "row_dot_kernel launch");
+  }
+  int rc;
+  const bool packed = prm.cu_q != nullptr;
+  if (d == 128) {
+    if (packed)
+      rc = mask ? launch_main<128, true, true>(maps, prm, grid, stream)
+                : launch_main<128, false, true>(maps, prm, grid, stream);
+    else
+      rc = mask ? launch_main<128, true, false>(maps, prm, grid, stream)
+                : launch_main<128, false, false>(maps, prm, grid, stream);
+  } else {
+    if (packed)
+      rc = mask ? launch_main<64, true, true>(maps, prm, grid, stream)
+                : launch_main<64, false, true>(maps, prm, grid, stream);
+    else
+      rc = mask ? launch_main<64, true, false>(maps, prm, grid, stream)
+                : launch_main<64, false, false>(maps, prm, grid, stream);
+  }
+  if (rc != ATTN_OK) return rc;
+  const size_t n4 = rows * d / 4;
+  const unsigned blocks = static_cast<unsigned>(std::min<size_t>((n4 + 255) / 256, 148 * 32));
+  dq_finish_kernel<<<blocks, 256, 0, stream>>>(reinterpret_cast<const float4*>(prm.dq_acc),
+                                               static_cast<uint2*>(dq), prm.scale, n4);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "dq_finish_kernel launch");
+  return ATTN_OK;
 }
 
 // window_left / window_right: the key band of the forward (-1 = no bound).
@@ -770,20 +907,6 @@ int bwd_impl(const void* q, const void* k, const void* v, const void* o, const v
   float* dq_acc = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) +
                                            align256(static_cast<size_t>(BH) * Nq * 4));
   if (!make_tmap_f32_3d(&maps[6], dq_acc, bh, Nq, d, 32, &t_last_error)) return ATTN_ERR_CUDA;
-  const size_t rows = static_cast<size_t>(BH) * Nq;
-  e = cudaMemsetAsync(dq_acc, 0, rows * d * 4, stream);
-  if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync");
-  {
-    const unsigned blocks = static_cast<unsigned>(std::min<size_t>((rows + 7) / 8, 148 * 16));
-    if (d == 128)
-      row_dot_kernel<128><<<blocks, 256, 0, stream>>>(static_cast<const __nv_bfloat16*>(o),
-                                                      static_cast<const __nv_bfloat16*>(dout), dsum, rows);
-    else
-      row_dot_kernel<64><<<blocks, 256, 0, stream>>>(static_cast<const __nv_bfloat16*>(o),
-                                                     static_cast<const __nv_bfloat16*>(dout), dsum, rows);
-    e = cudaGetLastError();
-    if (e != cudaSuccess) return cuda_fail(e, "row_dot_kernel launch");
-  }
 
   BwdParams prm = {};
   prm.lse = lse;
@@ -801,20 +924,103 @@ int bwd_impl(const void* q, const void* k, const void* v, const void* o, const v
   const bool mask = prm.wl < kUnbounded || prm.wr < kUnbounded;
   prm.scale_log2 = scale * kLog2e;
   prm.scale = scale;
-  const int grid = static_cast<int>(n_kblocks * BHkv);
-  if (d == 128)
-    rc = mask ? launch_main<128, true>(maps, prm, grid, stream) : launch_main<128, false>(maps, prm, grid, stream);
-  else
-    rc = mask ? launch_main<64, true>(maps, prm, grid, stream) : launch_main<64, false>(maps, prm, grid, stream);
+  return run_bwd(maps, prm, o, dout, dq, static_cast<size_t>(BH) * Nq, d, mask,
+                 static_cast<int>(n_kblocks * BHkv), stream);
+}
+
+// Packed variable-length batch: q, o, dout, dq [total_q, H, d]; k, v, dk, dv
+// [total_k, Hkv, d]; lse [H, total_q]; device offsets cu_q, cu_k.  Positions
+// count from 0 within each sequence (the band is applied to them).
+int bwd_varlen_impl(const void* q, const void* k, const void* v, const void* o, const void* dout,
+                    const float* lse, void* dq, void* dk, void* dv, void* workspace, size_t ws_bytes,
+                    const int* cu_q, const int* cu_k, int num_seqs, int max_seqlen_k, int total_q,
+                    int total_k, int H, int Hkv, int d, float scale, int window_left,
+                    int window_right, cudaStream_t stream) {
+  if (num_seqs < 0 || max_seqlen_k < 0 || total_q < 0 || total_k < 0 || H < 0 || Hkv < 0)
+    return ATTN_ERR_INVALID_ARG;
+  if (H > 0 && (Hkv == 0 || H % Hkv != 0)) return ATTN_ERR_INVALID_ARG;
+  if (!std::isfinite(scale)) return ATTN_ERR_INVALID_ARG;
+  if (window_left < -1 || window_right < -1) return ATTN_ERR_INVALID_ARG;
+  if (max_seqlen_k > total_k) return ATTN_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
+  if (num_seqs == 0 || H == 0 || (total_q == 0 && total_k == 0)) return ATTN_OK;
+  const bool any_q = total_q > 0, any_k = total_k > 0;
+  if (any_k && max_seqlen_k == 0) return ATTN_ERR_INVALID_ARG;  // keys exist but no sequence may hold one
+  if ((any_q && (!q || !o || !dout || !lse || !dq)) || (any_k && (!k || !v || !dk || !dv)) ||
+      !cu_q || !cu_k)
+    return ATTN_ERR_INVALID_ARG;
+  const size_t need = workspace_bytes(H, total_q, d);
+  if (any_q && any_k && (!workspace || ws_bytes < need)) return ATTN_ERR_INVALID_ARG;
+  if (misaligned(q, 16) || misaligned(k, 16) || misaligned(v, 16) || misaligned(o, 16) ||
+      misaligned(dout, 16) || misaligned(dq, 16) || misaligned(dk, 16) || misaligned(dv, 16) ||
+      misaligned(lse, 4) || misaligned(workspace, 256) || misaligned(cu_q, 4) || misaligned(cu_k, 4))
+    return ATTN_ERR_INVALID_ARG;
+  const size_t q_bytes = static_cast<size_t>(total_q) * H * d * 2;
+  const size_t kv_bytes = static_cast<size_t>(total_k) * Hkv * d * 2;
+  const size_t lse_bytes = static_cast<size_t>(total_q) * H * 4;
+  const size_t cu_bytes = (static_cast<size_t>(num_seqs) + 1) * 4;
+  const void* ins[8] = {q, k, v, o, dout, lse, cu_q, cu_k};
+  const size_t in_bytes[8] = {q_bytes, kv_bytes, kv_bytes, q_bytes, q_bytes, lse_bytes, cu_bytes, cu_bytes};
+  void* outs[4] = {dq, dk, dv, workspace};
+  const size_t out_bytes[4] = {q_bytes, kv_bytes, kv_bytes, any_q && any_k ? need : 0};
+  for (int a = 0; a < 4; ++a) {
+    for (int b = 0; b < 8; ++b)
+      if (ranges_overlap(outs[a], out_bytes[a], ins[b], in_bytes[b])) return ATTN_ERR_INVALID_ARG;
+    for (int b = a + 1; b < 4; ++b)
+      if (ranges_overlap(outs[a], out_bytes[a], outs[b], out_bytes[b])) return ATTN_ERR_INVALID_ARG;
+  }
+  const long long n_kblocks = (static_cast<long long>(max_seqlen_k) + kBlockK - 1) / kBlockK;
+  const long long BHkv = static_cast<long long>(num_seqs) * Hkv;
+  if (static_cast<long long>(num_seqs) * H > 0x7fffffffLL || n_kblocks * BHkv > 0x7fffffffLL)
+    return ATTN_ERR_INVALID_ARG;
+  int rc = check_device();
   if (rc != ATTN_OK) return rc;
 
-  const size_t n4 = rows * d / 4;
-  const unsigned blocks = static_cast<unsigned>(std::min<size_t>((n4 + 255) / 256, 148 * 32));
-  dq_finish_kernel<<<blocks, 256, 0, stream>>>(reinterpret_cast<const float4*>(dq_acc),
-                                               static_cast<uint2*>(dq), scale, n4);
-  e = cudaGetLastError();
-  if (e != cudaSuccess) return cuda_fail(e, "dq_finish_kernel launch");
-  return ATTN_OK;
+  cudaError_t e;
+  if (!any_k || !any_q) {
+    if (any_q && (e = cudaMemsetAsync(dq, 0, q_bytes, stream)) != cudaSuccess)
+      return cuda_fail(e, "cudaMemsetAsync");
+    if (any_k && (e = cudaMemsetAsync(dk, 0, kv_bytes, stream)) != cudaSuccess)
+      return cuda_fail(e, "cudaMemsetAsync");
+    if (any_k && (e = cudaMemsetAsync(dv, 0, kv_bytes, stream)) != cudaSuccess)
+      return cuda_fail(e, "cudaMemsetAsync");
+    return ATTN_OK;
+  }
+  CUtensorMap maps[7];
+  float* dsum = static_cast<float*>(workspace);
+  float* dq_acc = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) +
+                                           align256(static_cast<size_t>(H) * total_q * 4));
+  if (!make_tmap_bf16_packed(&maps[0], q, total_q, H, d, kBlockQ, &t_last_error) ||
+      !make_tmap_bf16_packed(&maps[1], k, total_k, Hkv, d, kBlockK, &t_last_error) ||
+      !make_tmap_bf16_packed(&maps[2], v, total_k, Hkv, d, kBlockK, &t_last_error) ||
+      !make_tmap_bf16_packed(&maps[3], dout, total_q, H, d, kBlockQ, &t_last_error) ||
+      !make_tmap_bf16_packed(&maps[4], dk, total_k, Hkv, d, 32, &t_last_error) ||
+      !make_tmap_bf16_packed(&maps[5], dv, total_k, Hkv, d, 32, &t_last_error) ||
+      !make_tmap_f32_packed(&maps[6], dq_acc, total_q, H, d, 32, &t_last_error))
+    return ATTN_ERR_CUDA;
+
+  BwdParams prm = {};
+  prm.lse = lse;
+  prm.dsum = dsum;
+  prm.dq_acc = dq_acc;
+  prm.cu_q = cu_q;
+  prm.cu_k = cu_k;
+  prm.dk = static_cast<__nv_bfloat16*>(dk);
+  prm.dv = static_cast<__nv_bfloat16*>(dv);
+  prm.timeout_ns = kWaitTimeoutNs;
+  prm.Nq = total_q;
+  prm.Nk = total_k;
+  prm.H = H;
+  prm.group = H / Hkv;
+  prm.n_kblocks = static_cast<int>(n_kblocks);
+  prm.n_qtiles = 0;  // per sequence
+  prm.wl = window_left < 0 ? kUnbounded : std::min(window_left, kUnbounded);
+  prm.wr = window_right < 0 ? kUnbounded : std::min(window_right, kUnbounded);
+  const bool mask = prm.wl < kUnbounded || prm.wr < kUnbounded;
+  prm.scale_log2 = scale * kLog2e;
+  prm.scale = scale;
+  return run_bwd(maps, prm, o, dout, dq, static_cast<size_t>(total_q) * H, d, mask,
+                 static_cast<int>(n_kblocks * BHkv), stream);
 }
 
 // attn_bwd_noalloc: the same computation with its workspace in a file-scope
@@ -883,6 +1089,16 @@ int attn_bwd_window(const void* q, const void* k, const void* v, const void* o, 
                     float scale, int window_left, int window_right, cudaStream_t stream) {
   return eab::bwd::bwd_impl(q, k, v, o, dout, lse, dq, dk, dv, workspace, workspace_bytes, B, H, Hkv,
                             Nq, Nk, d, scale, window_left, window_right, stream);
+}
+
+int attn_bwd_varlen(const void* q, const void* k, const void* v, const void* o, const void* dout,
+                    const float* lse, void* dq, void* dk, void* dv, void* workspace,
+                    size_t workspace_bytes, const int* cu_seqlens_q, const int* cu_seqlens_k,
+                    int num_seqs, int max_seqlen_k, int total_q, int total_k, int H, int Hkv, int d,
+                    float scale, int window_left, int window_right, cudaStream_t stream) {
+  return eab::bwd::bwd_varlen_impl(q, k, v, o, dout, lse, dq, dk, dv, workspace, workspace_bytes,
+                                   cu_seqlens_q, cu_seqlens_k, num_seqs, max_seqlen_k, total_q,
+                                   total_k, H, Hkv, d, scale, window_left, window_right, stream);
 }
 
 int attn_bwd_noalloc(const void* q, const void* k, const void* v, const void* o, const void* dout,

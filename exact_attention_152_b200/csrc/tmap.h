@@ -105,6 +105,31 @@ inline bool make_tmap_f32_3d(CUtensorMap* tm, const void* base, int BH, int N, i
   return true;
 }
 
+// FP32 packed [total, H, d] with 32-column x 1-head x box_rows boxes (the same
+// shared-memory layout as make_tmap_f32_3d's); coordinates (column, head, row).
+inline bool make_tmap_f32_packed(CUtensorMap* tm, const void* base, int total, int H, int d,
+                                 int box_rows, std::string* err) {
+  EncodeTiledFn enc = get_encode_fn();
+  if (!enc) {
+    *err = "cuTensorMapEncodeTiled unavailable";
+    return false;
+  }
+  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(H),
+                              static_cast<cuuint64_t>(total)};
+  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 4,
+                                 static_cast<cuuint64_t>(H) * static_cast<cuuint64_t>(d) * 4};
+  const cuuint32_t box[3] = {32u, 1u, static_cast<cuuint32_t>(box_rows)};
+  const cuuint32_t estr[3] = {1u, 1u, 1u};
+  CUresult r = enc(tm, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<void*>(base), dims, strides, box,
+                   estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) {
+    *err = "cuTensorMapEncodeTiled failed (CUresult " + std::to_string(static_cast<int>(r)) + ")";
+    return false;
+  }
+  return true;
+}
+
 // Dense [BH, N, d]: coordinates (column, row, head); rows past N of one head
 // read as zero (never as the next head's rows) and are clipped on store.
 inline bool make_tmap_bf16_3d(CUtensorMap* tm, const void* base, int BH, int N, int d,

@@ -268,6 +268,31 @@ int attn_bwd_window(const void *q, const void *k, const void *v, const void *o, 
                     size_t workspace_bytes, int B, int H, int Hkv, int Nq, int Nk, int d,
                     float scale, int window_left, int window_right, cudaStream_t stream);
 
+/*
+ * Backward of attn_fwd_varlen: a packed variable-length batch (sequences back
+ * to back, no padding; FlashAttention 4 page, ja.linux-konsole.com, section
+ * "互換性と現状", names variable-length batches and the backward pass among
+ * what FA4 lacks), the same chain rule as attn_bwd within each sequence.
+ *   q, o, dout, dq : BF16 [total_q, H, d]    k, v, dk, dv : BF16 [total_k, Hkv, d]
+ *   lse  : FP32 [H, total_q], attn_fwd_varlen's log-sum-exp
+ *   cu_seqlens_q, cu_seqlens_k, num_seqs : as attn_fwd_varlen (DEVICE int32)
+ *   max_seqlen_k : an upper bound on every sequence's key length (sizes the
+ *       grid), 1 <= max_seqlen_k <= total_k when total_k > 0
+ *   workspace : DEVICE scratch of at least attn_bwd_workspace_size(1, H, total_q, d)
+ *       bytes, 256-byte aligned, owned by the caller, overwritten
+ *   H, Hkv, d, scale, window_left, window_right : as attn_fwd_varlen
+ * Query rows that belong to no sequence get dQ = 0; key rows that belong to no
+ * sequence are not written.  Offsets that break attn_fwd_varlen's rules, or a
+ * key length beyond max_seqlen_k rounded up to 128, make the kernel skip that
+ * sequence and record the fact, which the next attn_status_sync() returns as
+ * ATTN_ERR_INVALID_ARG.  Other errors as attn_bwd.
+ */
+int attn_bwd_varlen(const void *q, const void *k, const void *v, const void *o, const void *dout,
+                    const float *lse, void *dq, void *dk, void *dv, void *workspace,
+                    size_t workspace_bytes, const int *cu_seqlens_q, const int *cu_seqlens_k,
+                    int num_seqs, int max_seqlen_k, int total_q, int total_k, int H, int Hkv, int d,
+                    float scale, int window_left, int window_right, cudaStream_t stream);
+
 /* Workspace bytes attn_bwd needs (0 for d not in {64, 128} or negative sizes). */
 size_t attn_bwd_workspace_size(int B, int H, int Nq, int d);
 

@@ -250,3 +250,25 @@ def attn_bwd(q, k, v, dout, scale, window_left=-1, window_right=-1, nthreads=Non
         dk[b, h // g] += bk
         dv[b, h // g] += bv
     return dq, dk, dv
+
+
+def attn_bwd_varlen(q, k, v, dout, cu_seqlens_q, cu_seqlens_k, scale, window_left=-1,
+                    window_right=-1, nthreads=None):
+    """Gradients of ``attn_varlen``: q/dout [total_q, H, d], k/v [total_k, Hkv, d]
+    fp64, each sequence taken alone (positions from 0 within it) and its heads
+    through ``attn_bwd``.  Returns (dq, dk, dv) in the packed layouts; rows that
+    belong to no sequence are 0 in dq and NaN in dk, dv (not defined)."""
+    q, k, v, dout = (np.asarray(x, dtype=np.float64) for x in (q, k, v, dout))
+    dq = np.zeros(q.shape)
+    dk = np.full(k.shape, np.nan)
+    dv = np.full(v.shape, np.nan)
+    for s in range(len(cu_seqlens_q) - 1):
+        q0, q1 = int(cu_seqlens_q[s]), int(cu_seqlens_q[s + 1])
+        k0, k1 = int(cu_seqlens_k[s]), int(cu_seqlens_k[s + 1])
+        per_head = lambda x, a, b: x[a:b].transpose(1, 0, 2)[None]  # noqa: E731  [1, heads, n, d]
+        g = attn_bwd(per_head(q, q0, q1), per_head(k, k0, k1), per_head(v, k0, k1),
+                     per_head(dout, q0, q1), scale, window_left, window_right, nthreads)
+        dq[q0:q1] = g[0][0].transpose(1, 0, 2)
+        dk[k0:k1] = g[1][0].transpose(1, 0, 2)
+        dv[k0:k1] = g[2][0].transpose(1, 0, 2)
+    return dq, dk, dv

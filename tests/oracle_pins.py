@@ -550,3 +550,65 @@ def pin_bwd_dv_is_pt_dout(bwd, fwd):
 
 BWD_PINS = [pin_bwd_finite_differences, pin_bwd_single_key, pin_bwd_sums,
             pin_bwd_linear_in_cotangent, pin_bwd_dv_is_pt_dout]
+
+
+# ---------------------------------------------------------------------------
+# Backward of a packed variable-length batch.  These take
+# ``attn_bwd_varlen(q, k, v, dout, cu_q, cu_k, scale, wl, wr)`` and
+# ``attn_varlen(q, k, v, cu_q, cu_k, scale, wl, wr)``.
+# ---------------------------------------------------------------------------
+def _varlen_loss(attn_varlen, q, k, v, dout, cu_q, cu_k, scale, wl, wr):
+    total = 0.0
+    for (s, h), (rows, o, _) in attn_varlen(q, k, v, cu_q, cu_k, scale, wl, wr).items():
+        total += float((o * dout[int(cu_q[s]) + rows, h]).sum())
+    return total
+
+
+def pin_bwd_varlen_finite_differences(attn_bwd_varlen, attn_varlen):
+    """Every owned gradient element of a packed batch (an empty sequence, a
+    sequence without keys, Nq != Nk per sequence, two query heads on one
+    key/value head, causal and a band) equals the central difference of
+    L = sum(dO * O) through the packed forward definition."""
+    h = 1e-5
+    cu_q = np.array([0, 3, 3, 7, 9])
+    cu_k = np.array([0, 4, 6, 9, 9])
+    r = _rng(330)
+    d = 2
+    q, dout = r.standard_normal((9, 2, d)), r.standard_normal((9, 2, d))
+    k, v = r.standard_normal((9, 1, d)), r.standard_normal((9, 1, d))
+    for wl, wr in [(-1, 0), (1, 1)]:
+        grads = attn_bwd_varlen(q, k, v, dout, cu_q, cu_k, 0.7, wl, wr)
+        for which, x in enumerate((q, k, v)):
+            num = np.zeros_like(x)
+            for idx in np.ndindex(*x.shape):
+                args = [q.copy(), k.copy(), v.copy()]
+                args[which][idx] += h
+                lp = _varlen_loss(attn_varlen, *args, dout, cu_q, cu_k, 0.7, wl, wr)
+                args[which][idx] -= 2 * h
+                lm = _varlen_loss(attn_varlen, *args, dout, cu_q, cu_k, 0.7, wl, wr)
+                num[idx] = (lp - lm) / (2 * h)
+            np.testing.assert_allclose(grads[which], num, rtol=1e-6, atol=1e-8,
+                                       err_msg=f"grad {'qkv'[which]} band {(wl, wr)}")
+
+
+def pin_bwd_varlen_rows_outside_sequences(attn_bwd_varlen, attn_varlen):
+    """Rows no sequence owns: dQ = 0 there, and the owned gradients do not
+    depend on their data (the outside rows are refilled with other values)."""
+    cu_q = np.array([1, 4, 6])
+    cu_k = np.array([0, 3, 5])
+    r = _rng(331)
+    q, dout = r.standard_normal((8, 1, 3)), r.standard_normal((8, 1, 3))
+    k, v = r.standard_normal((7, 1, 3)), r.standard_normal((7, 1, 3))
+    dq, dk, dv = attn_bwd_varlen(q, k, v, dout, cu_q, cu_k, 0.5, -1, 0)
+    assert np.all(dq[[0, 6, 7]] == 0.0)
+    q2, k2, v2, do2 = q.copy(), k.copy(), v.copy(), dout.copy()
+    q2[[0, 6, 7]] += 5.0
+    do2[[0, 6, 7]] -= 3.0
+    k2[5:] *= -2.0
+    v2[5:] += 1.0
+    dq2, dk2, dv2 = attn_bwd_varlen(q2, k2, v2, do2, cu_q, cu_k, 0.5, -1, 0)
+    assert np.array_equal(dq[1:6], dq2[1:6])
+    assert np.array_equal(dk[:5], dk2[:5]) and np.array_equal(dv[:5], dv2[:5])
+
+
+BWD_VARLEN_PINS = [pin_bwd_varlen_finite_differences, pin_bwd_varlen_rows_outside_sequences]

@@ -49,7 +49,7 @@ def test_library_exports_every_declared_symbol(header):
 def test_attn_h_declares_the_contract():
     names = declared_functions(os.path.join(ROOT, "include", "attn.h"))
     for n in ("attn_fwd", "attn_fwd_config", "attn_fwd_gqa", "attn_fwd_window", "attn_fwd_varlen",
-              "attn_fwd_fp8", "attn_fwd_colmask", "attn_colmask_workspace_size", "attn_bwd", "attn_bwd_window", "attn_bwd_noalloc", "attn_bwd_workspace_size", "attn_status_sync", "attn_status_string",
+              "attn_fwd_fp8", "attn_fwd_colmask", "attn_colmask_workspace_size", "attn_bwd", "attn_bwd_window", "attn_bwd_varlen", "attn_bwd_noalloc", "attn_bwd_workspace_size", "attn_status_sync", "attn_status_string",
               "attn_last_error", "attn_selftest_timeout"):
         assert n in names
 
@@ -206,6 +206,29 @@ def test_bwd_validation():
     assert BW(*ptrs, need, 1, 2, 2, 64, 64, 64, 0.1, -2, 0, None) == 1    # band below -1
     assert BW(*ptrs, need, 1, 2, 2, 64, 64, 64, 0.1, 0, -3, None) == 1
     assert BW(*ptrs, need - 1, 1, 2, 2, 64, 64, 64, 0.1, 8, 0, None) == 1  # workspace too small
+
+
+def test_bwd_varlen_validation():
+    BV = binding.attn_bwd_varlen
+    A = ALIGNED
+    ptrs = (A, A * 2, A * 3, A * 4, A * 5, A * 6, A * 7, A * 8, A * 9, A * 16)
+    need = binding.attn_bwd_workspace_size(1, 2, 150, 64)
+    cu = (A * 64, A * 65)
+    sizes = (2, 100, 150, 150, 2, 2, 64, 0.1, -1, 0)  # seqs, max_k, total_q, total_k, H, Hkv, d, ...
+
+    def call(p=ptrs, ws=need, c=cu, sz=sizes):
+        return BV(*p, ws, *c, *sz, None)
+    assert call(ws=need - 1) == 1                                   # workspace too small
+    assert call(c=(None, A * 65)) == 1                              # null offsets
+    assert call(c=(A * 64 + 2, A * 65)) == 1                        # misaligned offsets
+    assert call(sz=(2, 200) + sizes[2:]) == 1                       # max_seqlen_k > total_k
+    assert call(sz=(2, 0) + sizes[2:]) == 1                         # keys but max_seqlen_k 0
+    assert call(sz=sizes[:5] + (3,) + sizes[6:]) == 1               # H % Hkv
+    assert call(sz=sizes[:6] + (96,) + sizes[7:]) == 2              # head dim
+    assert call(sz=sizes[:8] + (-2, 0)) == 1                        # band
+    assert call(p=ptrs[:6] + (A,) + ptrs[7:]) == 1                  # dq overlaps q
+    assert call(c=(A * 7, A * 65)) == 1                             # offsets inside dq
+    assert BV(*(None,) * 10, 0, None, None, 0, 0, 0, 0, 2, 2, 64, 0.1, -1, 0, None) == 0
 
 
 def test_config_knob_validation():

@@ -17,6 +17,21 @@ def test_oracle_pin(pin):
     pin(oracle.attn_rows)
 
 
+@pytest.mark.parametrize("pin", pins.BWD_VARLEN_PINS, ids=[p.__name__ for p in pins.BWD_VARLEN_PINS])
+def test_oracle_bwd_varlen_pin(pin):
+    pin(oracle.attn_bwd_varlen, oracle.attn_varlen)
+
+
+def test_bwd_varlen_pin_catches_wrong_offsets():
+    """A packed backward that reads each sequence's keys one row too late is
+    caught by the finite-difference pin."""
+    def shifted(q, k, v, dout, cu_q, cu_k, scale, wl, wr):
+        return oracle.attn_bwd_varlen(q, k, v, dout, cu_q, np.minimum(np.asarray(cu_k) + 1, k.shape[0]),
+                                      scale, wl, wr)
+    with pytest.raises(AssertionError):
+        pins.pin_bwd_varlen_finite_differences(shifted, oracle.attn_varlen)
+
+
 @pytest.mark.parametrize("pin", pins.COLMASK_PINS, ids=[p.__name__ for p in pins.COLMASK_PINS])
 def test_oracle_colmask_pin(pin):
     pin(oracle.attn_rows_colmask)
