@@ -109,6 +109,7 @@ constexpr int kUnbounded = 1 << 30;
 constexpr int kMaskNone = 0;
 constexpr int kMaskBand = 1;
 constexpr int kMaskCols = 2;
+constexpr int kMaxMaskBlocks = 65536;  // key blocks per sequence under a column-interval mask
 
 // Per-device status word (each device holds its own copy of module globals).
 __device__ unsigned int g_status;
@@ -141,7 +142,11 @@ struct Cfg {
   static constexpr int kXchBytes = 2 * 2 * 2 * kBlockM * 4;
   static constexpr int kOffSeq = kOffXch + kXchBytes;  // this CTA's SeqView
   static constexpr int kSeqBytes = 64;
-  static constexpr int kSmemBytes = kOffSeq + kSeqBytes + 1024;  // + slack for 1 KiB alignment
+  // column-interval mask: one bit per 128-key block, set when the block is
+  // visited (kMaxMaskBlocks blocks = 8M keys)
+  static constexpr int kOffVis = kOffSeq + kSeqBytes;
+  static constexpr int kVisBytes = kMaxMaskBlocks / 8;
+  static constexpr int kSmemBytes = kOffVis + kVisBytes + 1024;  // + slack for 1 KiB alignment
   static_assert(kSmemBytes <= 232448, "shared memory per CTA");
   static constexpr uint32_t kTmemO = 256;
 };
@@ -177,11 +182,10 @@ struct SeqView {
   int Nq, Nk;        // this sequence's lengths
   int q0, k0;        // first row of the sequence in the packed layout (0 dense)
   int head_q, head_kv;  // tensor-map head coordinate of Q/O and of K/V
-  int j_lo, n_kv;    // KV tiles visited: n_kv of j_lo .. j_end - 1 (all of them
-  int j_end;         // unless a column-interval mask skips some)
+  int j_lo, n_kv;    // KV tiles visited: n_kv of them from j_lo on (consecutive
+                     // unless a column-interval mask skips some)
   int mrow;          // column-interval mask: row of [B * mask_heads] to use
   bool packed;
-  bool none_visible; // column-interval mask hides every block: visit j_lo, fully masked
   float* lse_row0;   // LSE of this sequence's row 0 (null: not computed)
 };
 
@@ -216,17 +220,30 @@ __device__ __forceinline__ int cta_row_end(int qb, int Nq) {
   return e < Nq ? static_cast<int>(e) : Nq;
 }
 
-// KV tile visited after tile blk (first: blk = j_lo - 1).  Every role of the
-// CTA walks the same sequence, so they agree on it without communicating.
+// KV tile visited after tile blk (first: blk = j_lo - 1).  Column-interval
+// mask: the next set bit of the CTA's visited-block bitmap in shared memory
+// (written once by warp 0; every role reads the same bits, so they agree on
+// the sequence without communicating).  The caller asks only for tiles that
+// exist (n_kv of them), so the search ends inside the bitmap.
 template <int MASK>
-__device__ __forceinline__ int next_block(const FwdParams& prm, const SeqView& sv, int qb, int blk) {
+__device__ __forceinline__ int next_block(const uint32_t* vis, int blk) {
   ++blk;
   if constexpr (MASK == kMaskCols) {
-    if (sv.none_visible) return sv.j_lo;
-    const int r0 = qb * kRowsPerCta, r1 = cta_row_end(qb, sv.Nq);
-    while (blk < sv.j_end - 1 && cols_hide_all(prm, sv.mrow, blk, r0, r1)) ++blk;
+    int wi = blk >> 5;
+    uint32_t bits = vis[wi] & (0xffffffffu << (blk & 31));
+    while (bits == 0u && wi < kMaxMaskBlocks / 32 - 1) bits = vis[++wi];
+    blk = wi * 32 + __ffs(bits) - 1;
   }
   return blk;
+}
+
+// Rows [lo, hi) of a warp's 32 rows starting at w0, as bits (lo, hi any ints).
+__device__ __forceinline__ uint32_t row_bits(int lo, int hi, int w0) {
+  const long long a = max(static_cast<long long>(lo) - w0, 0LL);
+  const long long b = min(static_cast<long long>(hi) - w0, 32LL);
+  if (b <= a) return 0u;
+  const uint32_t upto = b >= 32 ? 0xffffffffu : ((1u << b) - 1u);
+  return upto & ~((1u << a) - 1u);
 }
 
 // ---------------------------------------------------------------------------
@@ -260,6 +277,9 @@ struct Smem {
   // it only in the epilogue
   __device__ __forceinline__ SeqView* seq() const {
     return reinterpret_cast<SeqView*>(base + Cfg<D, F8>::kOffSeq);
+  }
+  __device__ __forceinline__ uint32_t* vis() const {
+    return reinterpret_cast<uint32_t*>(base + Cfg<D, F8>::kOffVis);
   }
 };
 
@@ -300,13 +320,14 @@ __device__ __forceinline__ void producer_role(const Smem<D, F8>& sm, const CUten
     return true;
   };
 
-  int blk = next_block<MASK>(prm, sv, qb, sv.j_lo - 1);
+  const uint32_t* vis = sm.vis();
+  int blk = next_block<MASK>(vis, sv.j_lo - 1);
   load_q(0);
   bool ok = load_kv(tm_k, blk);
   load_q(1);
   ok = ok && load_kv(tm_v, blk);
   for (int j = 1; ok && j < sv.n_kv; ++j) {
-    blk = next_block<MASK>(prm, sv, qb, blk);
+    blk = next_block<MASK>(vis, blk);
     ok = load_kv(tm_k, blk) && load_kv(tm_v, blk);
   }
 
@@ -503,7 +524,7 @@ __device__ __forceinline__ void softmax_role(const Smem<D, F8>& sm, uint32_t tme
 
   int blk = sv.j_lo - 1;
   for (int j = 0; j < sv.n_kv; ++j) {
-    blk = next_block<MASK>(prm, sv, qb, blk);
+    blk = next_block<MASK>(sm.vis(), blk);
     const int kv0 = blk * kBlockN + h * kCols;
     // mask needed: key tail, a band edge crossing this warp's 64 x 32 block, or
     // a column interval meeting the warp's rows
@@ -514,20 +535,24 @@ __device__ __forceinline__ void softmax_role(const Smem<D, F8>& sm, uint32_t tme
     if constexpr (MASK == kMaskCols) {
       if (cols_touch(prm, sv.mrow, blk, rw0, rw0 + 32)) {
         masked = true;
+        // lane l reads keys kv0 + l and kv0 + 32 + l (coalesced) and turns each
+        // into the set of the warp's 32 rows it is hidden from; 32 ballots
+        // transpose those into per-row words (bit c of row r: key 32k + c)
         const int4* cm = prm.colmask + static_cast<size_t>(sv.mrow) * Nk + kv0;
         const int n_in = min(kCols, Nk - kv0);
+        const int4 none = make_int4(0, 0, 0, 0);
+        const int4 ia = lane < n_in ? __ldg(cm + lane) : none;
+        const int4 ib = lane + 32 < n_in ? __ldg(cm + 32 + lane) : none;
+        const uint32_t ca = row_bits(ia.x, ia.y, rw0) | row_bits(ia.z, ia.w, rw0);
+        const uint32_t cb = row_bits(ib.x, ib.y, rw0) | row_bits(ib.z, ib.w, rw0);
 #pragma unroll
-        for (int k = 0; k < 2; ++k) {
-          uint32_t bits = 0u;
-#pragma unroll 8
-          for (int c = 0; c < 32; ++c) {
-            if (32 * k + c < n_in) {
-              const int4 iv = __ldg(cm + 32 * k + c);
-              const bool hide = (iv.x <= row && row < iv.y) || (iv.z <= row && row < iv.w);
-              bits |= static_cast<uint32_t>(hide) << c;
-            }
+        for (int rr = 0; rr < 32; ++rr) {
+          const uint32_t wa = __ballot_sync(0xffffffffu, (ca >> rr) & 1u);
+          const uint32_t wb = __ballot_sync(0xffffffffu, (cb >> rr) & 1u);
+          if (lane == rr) {
+            hid[0] = wa;
+            hid[1] = wb;
           }
-          hid[k] = bits;
         }
       }
     }
@@ -823,23 +848,26 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       }
     }
     sv.j_lo = j_lo;
-    sv.j_end = j_hi;
     sv.n_kv = j_hi - j_lo;
     sv.mrow = 0;
-    sv.none_visible = false;
     if constexpr (MASK == kMaskCols) {
-      // count the tiles that some row of this block sees (warp 0, 32 tiles a
-      // step); none: visit tile j_lo fully masked, as for an empty band
+      // the bitmap of tiles that some row of this block sees (warp 0, 32 tiles
+      // a step, bit b of word w = tile 32w + b); none: visit tile j_lo fully
+      // masked, as for an empty band
       sv.mrow = seq * prm.mask_heads + (prm.mask_heads == 1 ? 0 : hq);
       if (warp == 0) {
         const int r0 = qb * kRowsPerCta, r1 = cta_row_end(qb, sv.Nq);
+        uint32_t* vis = sm.vis();
         int cnt = 0;
-        for (int base = j_lo; base < j_hi; base += 32) {
-          const int blk = base + lane;
-          const bool vis = blk < j_hi && !cols_hide_all(prm, sv.mrow, blk, r0, r1);
-          cnt += __popc(__ballot_sync(0xffffffffu, vis));
+#pragma unroll 4
+        for (int w = j_lo >> 5; w <= (j_hi - 1) >> 5; ++w) {
+          const int blk = w * 32 + lane;
+          const bool v = blk >= j_lo && blk < j_hi && !cols_hide_all(prm, sv.mrow, blk, r0, r1);
+          const uint32_t word = __ballot_sync(0xffffffffu, v);
+          if (lane == 0) vis[w] = word;
+          cnt += __popc(word);
         }
-        sv.none_visible = cnt == 0;
+        if (cnt == 0 && lane == 0) vis[j_lo >> 5] = 1u << (j_lo & 31);
         sv.n_kv = cnt > 0 ? cnt : 1;
       }
     }
@@ -1117,6 +1145,7 @@ int fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, i
     if (misaligned(cm->mask, 16) || misaligned(cm->workspace, 16)) return ATTN_ERR_INVALID_ARG;
     if (cm->workspace_bytes < ws_need) return ATTN_ERR_INVALID_ARG;
     if (BHm * ((Nk + kBlockN - 1) / kBlockN) > 0x7fffffffLL) return ATTN_ERR_INVALID_ARG;
+    if ((static_cast<long long>(Nk) + kBlockN - 1) / kBlockN > kMaxMaskBlocks) return ATTN_ERR_UNSUPPORTED;
     // the workspace is written: it may overlap no input or output
     const void* ws = cm->workspace;
     if (ranges_overlap(ws, ws_need, q, o_bytes) || ranges_overlap(ws, ws_need, k, kv_bytes) ||
