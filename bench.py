@@ -305,6 +305,8 @@ def run_reference_bwd(args, w, per_step):
 
 
 def bwd_launch_name(w):
+    if w.colmask:
+        return "attn_bwd_colmask"
     if w.packed:
         return "attn_bwd_varlen"
     return "attn_bwd_window" if w.window is not None else "attn_bwd"
@@ -579,18 +581,27 @@ def bwd_cpu_baseline(w, seconds):
         k, v = (inputs.bf16_bits_to_f64(w.head_bits(x, w.kv_head_of(0))) for x in "kv")
         q_of = lambda rows: w.q_rows_bits(0, rows)  # noqa: E731
         flat = lambda rows: rows[:, None] * w.d + np.arange(w.d)[None, :]  # noqa: E731
+    cols = w.colmask_array()[0, 0] if w.colmask else None
     n, dt = 64, 0.0
     while True:
         rows = np.arange(min(n, nq), dtype=np.int64)
         q = inputs.bf16_bits_to_f64(q_of(rows))
         g = inputs.bf16_bits_to_f64(inputs.gen_bf16_at(w.seed + 1, "q", flat(rows)))
         t0 = time.perf_counter()
-        oracle.attn_bwd_head(q, k, v, g, w.scale, wl, wr)
+        if cols is not None:
+            oracle.attn_bwd_colmask_head(q, k, v, g, w.scale, w.causal, cols)
+        else:
+            oracle.attn_bwd_head(q, k, v, g, w.scale, wl, wr)
         dt = time.perf_counter() - t0
         if dt > seconds / 4 or n >= nq:
             break
         n = min(nq, n * 4)
-    flops = 2.5 * 4.0 * w.d * float(visible_keys(rows, nk, wl, wr).sum())
+    if cols is not None:
+        from exact_attention_152_b200 import masks
+        pairs = float(masks.visible_per_row(cols, rows, w.causal).sum())
+    else:
+        pairs = float(visible_keys(rows, nk, wl, wr).sum())
+    flops = 2.5 * 4.0 * w.d * pairs
     where = "sequence 0, head 0" if w.packed else "head 0"
     return {"value": flops / dt / 1e12, "unit": UNIT, "cores": 1, "kind": "oracle",
             "sample": f"backward of the first {len(rows)} query rows of {where} of {w.name} against "
@@ -612,17 +623,23 @@ def run_ours_bwd(args):
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
     w = WORKLOADS[args.workload or HEADLINE]
-    if w.fp8 or w.colmask:
-        raise SystemExit("--pass bwd: no backward for E4M3 or column-interval workloads")
+    if w.fp8:
+        raise SystemExit("--pass bwd: no backward for E4M3 workloads")
     peaks = load_peaks()
     host = {x: w.tensor_bits(x) for x in "qkv"}
     host["do"] = inputs.gen_bf16(w.seed + 1, "q", w.shape("q"))
     to_dev = lambda a: torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).to(dev)  # noqa: E731
     q, k, v, do = (to_dev(host[x]) for x in ("q", "k", "v", "do"))
+    mask = None
     if w.packed:
         cu = torch.from_numpy(w.cu_seqlens).to(dev)
         o, lse = binding.fwd_varlen(q, k, v, cu, cu, max(w.seqlens), scale=w.scale, window=w.band)
         ws_bytes = binding.attn_bwd_workspace_size(1, w.H, w.total, w.d)
+    elif w.colmask:
+        cu = None
+        mask = torch.from_numpy(w.colmask_array()).to(dev)
+        o, lse = binding.fwd_colmask(q, k, v, mask, causal=w.causal, scale=w.scale)
+        ws_bytes = binding.attn_bwd_colmask_workspace_size(w.B, w.H, w.Nq, w.d, 1, w.Nk)
     else:
         cu = None
         o, lse = binding.fwd(q, k, v, causal=w.causal, scale=w.scale, window=w.window)
@@ -632,9 +649,12 @@ def run_ours_bwd(args):
     ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
     dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
 
-    def launch(ins=(q, k, v, o, do, lse, cu), outs=(dq, dk, dv)):
+    def launch(ins=(q, k, v, o, do, lse, cu if w.packed else mask), outs=(dq, dk, dv)):
         ptrs = [t.data_ptr() for t in ins[:6]] + [t.data_ptr() for t in outs]
-        if w.packed:
+        if w.colmask:
+            rc = binding.attn_bwd_colmask(*ptrs, ws.data_ptr(), ws_bytes, w.B, w.H, w.kv_heads, w.Nq,
+                                          w.Nk, w.d, w.scale, int(w.causal), ins[6].data_ptr(), 1, sh)
+        elif w.packed:
             c = ins[6].data_ptr()
             rc = binding.attn_bwd_varlen(*ptrs, ws.data_ptr(), ws_bytes, c, c, len(w.seqlens),
                                          max(w.seqlens), w.total, w.total, w.H, w.kv_heads, w.d,
@@ -673,7 +693,7 @@ def run_ours_bwd(args):
 
     # end to end: pinned host Q, K, V, O, dO, LSE -> H2D -> attn_bwd -> D2H dQ, dK, dV
     pin = lambda t: t.cpu().pin_memory()  # noqa: E731
-    ins = (q, k, v, o, do, lse) + ((cu,) if w.packed else ())
+    ins = (q, k, v, o, do, lse) + ((cu,) if w.packed else ()) + ((mask,) if w.colmask else ())
     h_in = [pin(t) for t in ins]
     h_out = [torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in (dq, dk, dv)]
     d_in = [torch.empty_like(t) for t in ins]
@@ -681,7 +701,7 @@ def run_ours_bwd(args):
     def e2e_step():
         for d_, h_ in zip(d_in, h_in):
             d_.copy_(h_, non_blocking=True)
-        launch(tuple(d_in) + ((None,) if not w.packed else ()))
+        launch(tuple(d_in) + ((None,) if not (w.packed or w.colmask) else ()))
         for h_, d_ in zip(h_out, (dq, dk, dv)):
             h_.copy_(d_, non_blocking=True)
 
@@ -716,9 +736,11 @@ def run_ours_bwd(args):
                 "h2d_bytes_per_step": sum(t.numel() * t.element_size() for t in h_in),
                 "d2h_bytes_per_step": sum(t.numel() * t.element_size() for t in h_out),
                 "steps": args.e2e_steps,
-                "path": f"pinned host Q/K/V/O/dO/LSE{' + offsets' if w.packed else ''} -> H2D -> "
+                "path": f"pinned host Q/K/V/O/dO/LSE{' + offsets' if w.packed else ''}"
+                        f"{' + mask' if w.colmask else ''} -> H2D -> "
                         f"{bwd_launch_name(w)} (C-ABI) -> D2H of dQ/dK/dV"},
-        "gpu_launches": 3 * K,
+        # row sums, main kernel, dQ rounding (+ the mask summaries for column intervals)
+        "gpu_launches": (4 if w.colmask else 3) * K,
         "clocks": clocks,
         "kernel_src_sha": kernel_source_hash("bwd"),
     }

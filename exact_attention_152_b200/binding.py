@@ -68,6 +68,11 @@ def lib() -> ctypes.CDLL:
             l.attn_bwd_varlen.argtypes = [_P] * 10 + [ctypes.c_size_t, _P, _P] + [_I] * 7 + \
                 [ctypes.c_float, _I, _I, _P]
             l.attn_bwd_varlen.restype = _I
+            l.attn_bwd_colmask.argtypes = [_P] * 10 + [ctypes.c_size_t] + [_I] * 6 + \
+                [ctypes.c_float, _I, _P, _I, _P]
+            l.attn_bwd_colmask.restype = _I
+            l.attn_bwd_colmask_workspace_size.argtypes = [_I] * 6
+            l.attn_bwd_colmask_workspace_size.restype = ctypes.c_size_t
             l.attn_bwd_noalloc.argtypes = [_P] * 9 + [_I] * 6 + [ctypes.c_float, _I, _P]
             l.attn_bwd_noalloc.restype = _I
             l.attn_bwd_workspace_size.argtypes = [_I, _I, _I, _I]
@@ -137,6 +142,16 @@ def attn_bwd_window(q, k, v, o, dout, lse, dq, dk, dv, workspace, workspace_byte
                     d, scale, window_left, window_right, stream) -> int:
     return lib().attn_bwd_window(q, k, v, o, dout, lse, dq, dk, dv, workspace, workspace_bytes, B, H,
                                  Hkv, Nq, Nk, d, scale, window_left, window_right, stream)
+
+
+def attn_bwd_colmask(q, k, v, o, dout, lse, dq, dk, dv, workspace, workspace_bytes, B, H, Hkv, Nq, Nk,
+                     d, scale, causal, mask, Hm, stream) -> int:
+    return lib().attn_bwd_colmask(q, k, v, o, dout, lse, dq, dk, dv, workspace, workspace_bytes, B, H,
+                                  Hkv, Nq, Nk, d, scale, causal, mask, Hm, stream)
+
+
+def attn_bwd_colmask_workspace_size(B, H, Nq, d, Hm, Nk) -> int:
+    return lib().attn_bwd_colmask_workspace_size(B, H, Nq, d, Hm, Nk)
 
 
 def attn_bwd_varlen(q, k, v, o, dout, lse, dq, dk, dv, workspace, workspace_bytes, cu_seqlens_q,
@@ -372,6 +387,45 @@ def bwd(q, k, v, o, dout, lse, causal: bool = False, scale: float | None = None,
     else:
         rc = attn_bwd(*ptrs, B, H, Hkv, Nq, Nk, d, float(scale), int(bool(causal)), stream)
         check(rc, "attn_bwd")
+    return dq, dk, dv
+
+
+def bwd_colmask(q, k, v, o, dout, lse, mask, causal: bool = False, scale: float | None = None, *,
+                workspace=None):
+    """Gradients (dq, dk, dv) of fwd_colmask for BF16 CUDA tensors q/o/dout
+    [B,H,Nq,d], k/v [B,Hkv,Nk,d], fp32 lse [B,H,Nq] and the int32 CUDA mask
+    [B, Hm, Nk, 4].  The workspace is allocated when not given.  Runs on
+    torch's current stream."""
+    import torch
+
+    _check_bf16(q=q, k=k, v=v, o=o, dout=dout)
+    B, H, Nq, d = q.shape
+    Hkv, Nk = k.shape[1], k.shape[2]
+    if tuple(o.shape) != tuple(q.shape) or tuple(dout.shape) != tuple(q.shape):
+        raise ValueError("o and dout must match q")
+    if tuple(k.shape) != (B, Hkv, Nk, d) or tuple(v.shape) != (B, Hkv, Nk, d):
+        raise ValueError("k and v must be [B, Hkv, Nk, d] matching q")
+    if lse.dtype != torch.float32 or not lse.is_contiguous() or tuple(lse.shape) != (B, H, Nq):
+        raise ValueError("lse must be contiguous float32 [B, H, Nq]")
+    if not isinstance(mask, torch.Tensor) or mask.dtype != torch.int32 or not mask.is_cuda \
+            or mask.dim() != 4 or mask.shape[0] != B or mask.shape[2] != Nk or mask.shape[3] != 4 \
+            or not mask.is_contiguous():
+        raise ValueError("mask must be a contiguous int32 CUDA tensor [B, Hm, Nk, 4]")
+    Hm = mask.shape[1]
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    need = attn_bwd_colmask_workspace_size(B, H, Nq, d, Hm, Nk)
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
+    dq = torch.empty_like(q)
+    dk = torch.empty_like(k)
+    dv = torch.empty_like(v)
+    stream = torch.cuda.current_stream(q.device).cuda_stream
+    rc = attn_bwd_colmask(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), dout.data_ptr(),
+                          lse.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(),
+                          workspace.data_ptr(), workspace.numel() * workspace.element_size(), B, H,
+                          Hkv, Nq, Nk, d, float(scale), int(bool(causal)), mask.data_ptr(), Hm, stream)
+    check(rc, "attn_bwd_colmask")
     return dq, dk, dv
 
 

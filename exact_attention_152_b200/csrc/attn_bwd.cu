@@ -56,6 +56,13 @@
 #include "tmap.h"
 
 namespace eab {
+
+// Column-interval mask summaries (attn_fwd.cu): for each of the BHm mask rows
+// and each 128-key block, two int4 -- (max lo1, min hi1, max lo2, min hi2) and
+// (min lo1, max hi1, min lo2, max hi2), an empty interval counting as
+// (INT_MAX, INT_MIN) -- written to sum ([BHm, ceil(Nk / 128), 2] int4).
+int launch_colmask_summary(const int* mask, void* sum, long long BHm, int Nk, cudaStream_t stream);
+
 namespace bwd {
 
 constexpr int kBlockK = 128;  // keys per CTA (TMEM lanes of S^T, dP^T, dV, dK)
@@ -68,6 +75,12 @@ constexpr uint32_t kTmemCols = 512;
 constexpr uint64_t kWaitTimeoutNs = 2000000000ull;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr int kUnbounded = 1 << 30;  // "no bound" for a side of the key band
+// mask kinds (kernel template argument): none; the key band i - wl <= j <= i + wr
+// (causal: wl unbounded, wr = 0); the band plus column intervals (each key j
+// hidden from query rows [lo1_j, hi1_j) and [lo2_j, hi2_j))
+constexpr int kMaskNone = 0;
+constexpr int kMaskBand = 1;
+constexpr int kMaskCols = 2;
 
 constexpr unsigned int kStatusTimeout = kStatusWordTimeout;
 constexpr unsigned int kStatusSmemAlign = 4u;  // mapped to kStatusWordLaunch on the host
@@ -106,6 +119,11 @@ struct BwdParams {
   const int* cu_k;
   __nv_bfloat16* dk;   // packed outputs, for rows stored one by one at a sequence's end
   __nv_bfloat16* dv;
+  // column intervals (kMaskCols): per key (lo1, hi1, lo2, hi2), [B * mask_heads, Nk];
+  // per 128-key block two summaries, [B * mask_heads, n_kblocks, 2]
+  const int4* colmask;
+  const int4* colsum;
+  int mask_heads;      // 1 or H
   uint64_t timeout_ns;
   int Nq, Nk, H, group, n_kblocks, n_qtiles;  // packed: Nq, Nk = total_q, total_k
   int wl, wr;          // key band i - wl <= j <= i + wr (kUnbounded: no bound)
@@ -152,10 +170,10 @@ struct Smem {
 struct Work {
   int bh_kv, j, b, hkv, i_lo, tiles_per_head, n_it;
   bool packed;   // a compile-time constant per kernel instance
+  bool force;    // column intervals hide every tile: visit (head 0, i_lo) fully masked
   int Nq, Nk;    // packed: the sequence's lengths
   int q0, k0;    // packed: the sequence's first rows
-  __device__ __forceinline__ int head_of(int it) const { return it / tiles_per_head; }
-  __device__ __forceinline__ int tile_of(int it) const { return i_lo + it % tiles_per_head; }
+  int n_qtiles;  // query tiles of the problem
   // lengths and first rows of this CTA's problem (dense: the launch's, from 0)
   __device__ __forceinline__ int nq(const BwdParams& p) const { return packed ? Nq : p.Nq; }
   __device__ __forceinline__ int nk(const BwdParams& p) const { return packed ? Nk : p.Nk; }
@@ -205,6 +223,85 @@ struct Mma {
   }
 };
 
+// Which (query head, query tile) iteration `it` works on.  Without column
+// intervals: head it / tiles_per_head, tile i_lo + it % tiles_per_head.  With
+// them, the query tiles of one head that every key of this block hides form at
+// most two ranges (one per interval, from the block's summary), which the walk
+// steps over; every role walks the same sequence, so they agree on it.
+struct Walk {
+  int hh, t;           // query head within the group, query tile
+  int a1, b1, a2, b2;  // hidden tiles [a1, b1] and [a2, b2] of head hh (a > b: none)
+};
+
+// mask row of query head hh of the CTA's group
+__device__ __forceinline__ int mask_row(const BwdParams& prm, const Work& w, int hh) {
+  return w.b * prm.mask_heads + (prm.mask_heads == 1 ? 0 : w.hkv * prm.group + hh);
+}
+
+// Tiles t whose rows [128t, min(128t + 128, Nq)) lie inside [lo, hi) for every
+// key of the block: lo = the block's max lo, hi = its min hi.
+__device__ __forceinline__ void hidden_range(int lo, int hi, int Nq, int n_qtiles, int* a, int* b) {
+  const long long first = lo <= 0 ? 0 : (static_cast<long long>(lo) + kBlockQ - 1) / kBlockQ;
+  const long long last = hi >= Nq ? n_qtiles - 1 : static_cast<long long>(hi) / kBlockQ - 1;
+  *a = static_cast<int>(first < n_qtiles ? first : n_qtiles);
+  *b = static_cast<int>(last < n_qtiles - 1 ? last : n_qtiles - 1);
+}
+
+__device__ __forceinline__ void walk_head(Walk& k, const BwdParams& prm, const Work& w, int n_qtiles) {
+  const int4 a = __ldg(prm.colsum + (static_cast<size_t>(mask_row(prm, w, k.hh)) * prm.n_kblocks + w.j) * 2);
+  hidden_range(a.x, a.y, prm.Nq, n_qtiles, &k.a1, &k.b1);
+  hidden_range(a.z, a.w, prm.Nq, n_qtiles, &k.a2, &k.b2);
+}
+
+// Visible tiles of head hh in [i_lo, i_hi]: the range minus the two hidden ones.
+__device__ __forceinline__ int visible_count(const Walk& k, int i_lo, int i_hi) {
+  auto inter = [](int a, int b, int c, int e) { const int lo = max(a, c), hi = min(b, e); return hi >= lo ? hi - lo + 1 : 0; };
+  const int both = inter(max(k.a1, k.a2), min(k.b1, k.b2), i_lo, i_hi);
+  return (i_hi - i_lo + 1) - inter(k.a1, k.b1, i_lo, i_hi) - inter(k.a2, k.b2, i_lo, i_hi) + both;
+}
+
+// Move (hh, t) forward to the first visible tile at or after it.
+template <int MASK>
+__device__ __forceinline__ void walk_settle(Walk& k, const BwdParams& prm, const Work& w, int n_qtiles) {
+  if constexpr (MASK == kMaskCols) {
+    if (w.force) return;
+    const int i_hi = w.i_lo + w.tiles_per_head - 1;
+    for (int guard = 0; guard <= prm.group; ++guard) {
+      for (int rep = 0; rep < 2; ++rep) {
+        if (k.t >= k.a1 && k.t <= k.b1) k.t = k.b1 + 1;
+        if (k.t >= k.a2 && k.t <= k.b2) k.t = k.b2 + 1;
+      }
+      if (k.t <= i_hi || k.hh + 1 >= prm.group) break;
+      ++k.hh;
+      k.t = w.i_lo;
+      walk_head(k, prm, w, n_qtiles);
+    }
+  } else {
+    if (k.t >= w.i_lo + w.tiles_per_head) {
+      ++k.hh;
+      k.t = w.i_lo;
+    }
+  }
+}
+
+template <int MASK>
+__device__ __forceinline__ void walk_start(Walk& k, const BwdParams& prm, const Work& w, int n_qtiles) {
+  k.hh = 0;
+  k.t = w.i_lo;
+  k.a1 = k.a2 = 1;
+  k.b1 = k.b2 = 0;
+  if constexpr (MASK == kMaskCols) {
+    if (!w.force) walk_head(k, prm, w, n_qtiles);
+  }
+  walk_settle<MASK>(k, prm, w, n_qtiles);
+}
+
+template <int MASK>
+__device__ __forceinline__ void walk_next(Walk& k, const BwdParams& prm, const Work& w, int n_qtiles) {
+  ++k.t;
+  walk_settle<MASK>(k, prm, w, n_qtiles);
+}
+
 // Tensor-map coordinates (column, row, head) in the map's dimension order:
 // dense maps are [BH, N, d], packed maps [total, H, d].
 __device__ __forceinline__ void load_rows(uint32_t dst, const CUtensorMap* tm, int col, int row, int head,
@@ -216,7 +313,7 @@ __device__ __forceinline__ void load_rows(uint32_t dst, const CUtensorMap* tm, i
 // ---------------------------------------------------------------------------
 // Producer warp: K, V once; then Q, dO (TMA) and LSE, D (plain loads) per tile.
 // ---------------------------------------------------------------------------
-template <int D>
+template <int D, int MASK>
 __device__ __forceinline__ void producer_role(const Smem<D>& sm, const CUtensorMap* tm_q,
                                               const CUtensorMap* tm_k, const CUtensorMap* tm_v,
                                               const CUtensorMap* tm_do, const BwdParams& prm,
@@ -235,14 +332,17 @@ __device__ __forceinline__ void producer_role(const Smem<D>& sm, const CUtensorM
   }
   bool ok = true;
   int it = 0;
+  Walk wk;
+  walk_start<MASK>(wk, prm, w, w.n_qtiles);
   for (; it < w.n_it; ++it) {
+    if (it > 0) walk_next<MASK>(wk, prm, w, w.n_qtiles);
     const int s = it & 1;
     const uint32_t ph = (it >> 1) & 1;
     ok = warp_wait(sm.q_empty(s), ph ^ 1u, prm.timeout_ns);
     if (!ok) break;
-    const int h = w.hkv * prm.group + w.head_of(it);  // query head within the batch entry
+    const int h = w.hkv * prm.group + wk.hh;  // query head within the batch entry
     const int bh = w.b * prm.H + h;
-    const int q0 = w.tile_of(it) * kBlockQ;
+    const int q0 = wk.t * kBlockQ;
     // -LSE * log2(e) per query row (rows past the sequence: -inf, so P = 0
     // there), and D.  Dense: both [B*H, Nq]; packed: LSE [H, total_q], D
     // [total_q, H].
@@ -352,7 +452,7 @@ __device__ __forceinline__ void mma_role(const Smem<D>& sm, uint32_t tmem, const
 // Warps 0-7: P^T and dS^T from S^T and dP^T.  Warp (c, q) owns TMEM lanes
 // 32q..32q+31 (keys) and query columns [64c, 64c+64).
 // ---------------------------------------------------------------------------
-template <int D, bool MASK>
+template <int D, int MASK>
 __device__ __forceinline__ bool softmax_grad_role(const Smem<D>& sm, uint32_t tmem,
                                                   const BwdParams& prm, const Work& w) {
   using C = Cfg<D>;
@@ -366,7 +466,17 @@ __device__ __forceinline__ bool softmax_grad_role(const Smem<D>& sm, uint32_t tm
   const uint32_t tP = tmem + lane_off + C::kTmemDP + c * 64;
   uint8_t* ds_row = sm.base + C::kOffDS + c * C::kBoxBytes + r * 128;
   bool ok = true;
+  Walk wk;
+  walk_start<MASK>(wk, prm, w, w.n_qtiles);
+  int4 kiv = make_int4(0, 0, 0, 0);  // this thread's key intervals (column mask)
+  int kiv_head = -1;
   for (int it = 0; it < w.n_it; ++it) {
+    if (it > 0) walk_next<MASK>(wk, prm, w, w.n_qtiles);
+    if (MASK == kMaskCols && wk.hh != kiv_head) {
+      kiv_head = wk.hh;
+      kiv = key_in ? __ldg(prm.colmask + static_cast<size_t>(mask_row(prm, w, wk.hh)) * prm.Nk + key)
+                   : make_int4(0, 0, 0, 0);
+    }
     const int s = it & 1;
     // q_full orders the producer's LSE / D rows of this stage before the reads
     // below (long complete by now); it cannot run two phases ahead, since the
@@ -376,11 +486,16 @@ __device__ __forceinline__ bool softmax_grad_role(const Smem<D>& sm, uint32_t tm
          warp_wait(sm.dp_full(), it & 1, prm.timeout_ns);
     if (!ok) break;
     tc_fence_after();
-    const int q_base = w.tile_of(it) * kBlockQ + c * 64;  // first query of this warp's columns
-    // masking: key tail, or a band edge crossing this warp's 32 keys x 64 queries
+    const int q_base = wk.t * kBlockQ + c * 64;  // first query of this warp's columns
+    // masking: key tail, a band edge crossing this warp's 32 keys x 64 queries,
+    // or a key interval meeting the warp's queries
     const int k_lo = w.j * kBlockK + q4 * 32;
-    const bool masked = !key_in ||
-                        (MASK && (k_lo + 31 - q_base > prm.wr || q_base + 63 - k_lo > prm.wl));
+    bool masked = !key_in || (MASK != kMaskNone && (k_lo + 31 - q_base > prm.wr || q_base + 63 - k_lo > prm.wl));
+    if (MASK == kMaskCols) {
+      const bool meets = (kiv.x < q_base + 64 && kiv.y > q_base && kiv.x < kiv.y) ||
+                         (kiv.z < q_base + 64 && kiv.w > q_base && kiv.z < kiv.w);
+      masked = masked || meets;
+    }
     const float4* nl4 = reinterpret_cast<const float4*>(sm.lse2(s) + c * 64);
     const float4* dd4 = reinterpret_cast<const float4*>(sm.dsum(s) + c * 64);
     const float2 sl2 = make_float2(prm.scale_log2, prm.scale_log2);
@@ -411,6 +526,17 @@ __device__ __forceinline__ bool softmax_grad_role(const Smem<D>& sm, uint32_t tm
           if (!key_in || d0 - 1 > hi || d0 - 1 < lo) xa.y = -INFINITY;
           if (!key_in || d0 - 2 > hi || d0 - 2 < lo) xb.x = -INFINITY;
           if (!key_in || d0 - 3 > hi || d0 - 3 < lo) xb.y = -INFINITY;
+          if (MASK == kMaskCols) {
+            // query q0 + e hidden from this key by one of its intervals
+            const int q0 = q_base + 32 * k + 4 * g;
+            auto hid = [&](int e) {
+              return (kiv.x <= q0 + e && q0 + e < kiv.y) || (kiv.z <= q0 + e && q0 + e < kiv.w);
+            };
+            if (hid(0)) xa.x = -INFINITY;
+            if (hid(1)) xa.y = -INFINITY;
+            if (hid(2)) xb.x = -INFINITY;
+            if (hid(3)) xb.y = -INFINITY;
+          }
         }
         float2 pa, pb;
         if ((g & 3) == 0) {  // a quarter of the exponentials on the FMA pipe
@@ -469,7 +595,7 @@ __device__ __forceinline__ bool softmax_grad_role(const Smem<D>& sm, uint32_t tm
 // which the dQ GEMM has finished reading and the next dS is not written until
 // ds_free.  TMEM is released (dq_free) as soon as the last columns are in
 // registers, so the next S^T GEMM overlaps the reductions.
-template <int D>
+template <int D, int MASK>
 __device__ __forceinline__ bool dq_drain_role(const Smem<D>& sm, uint32_t tmem, const CUtensorMap* tm_dq,
                                               const BwdParams& prm, const Work& w) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -479,15 +605,18 @@ __device__ __forceinline__ bool dq_drain_role(const Smem<D>& sm, uint32_t tmem, 
   const uint32_t stage_s = smem_u32(stage);
   constexpr int kHalves = D / 64;
   bool ok = true;
+  Walk wk;
+  walk_start<MASK>(wk, prm, w, w.n_qtiles);
   for (int it = 0; it < w.n_it; ++it) {
+    if (it > 0) walk_next<MASK>(wk, prm, w, w.n_qtiles);
     ok = warp_wait(sm.dq_full(), it & 1, prm.timeout_ns);
     if (!ok) break;
     tc_fence_after();
-    const int h = w.hkv * prm.group + w.head_of(it);
+    const int h = w.hkv * prm.group + wk.hh;
     const int qh = w.packed ? h : w.b * prm.H + h;
     // rows past a packed sequence's end reduce exact zeros (P = 0 there) into
     // the next sequence's rows, which leaves them unchanged
-    const int row0 = w.row_q0() + w.tile_of(it) * kBlockQ + q4 * 32;
+    const int row0 = w.row_q0() + wk.t * kBlockQ + q4 * 32;
     // all of this warp's dQ columns into registers, then TMEM is free
     uint32_t v[kHalves][2][32];
 #pragma unroll
@@ -610,7 +739,7 @@ __device__ __forceinline__ bool epilogue(const Smem<D>& sm, uint32_t tmem, const
   return true;
 }
 
-template <int D, bool MASK, bool PACKED>
+template <int D, int MASK, bool PACKED>
 __global__ void __launch_bounds__(kNumThreads, 1)
 attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                 const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
@@ -664,9 +793,11 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   // query tiles that can see a key of this block: i - wl <= j <= i + wr for
   // some key j in [j0, j0 + 127] and query i of the tile; a block no query
   // sees still runs one fully masked tile, so dK = dV = 0 come out of TMEM
+  w.n_qtiles = n_qtiles;
+  w.force = false;
   w.i_lo = 0;
   w.tiles_per_head = n_qtiles;
-  if (MASK) {
+  if (MASK != kMaskNone) {
     const long long j0 = static_cast<long long>(w.j) * kBlockK;
     long long lo = 0, hi = n_qtiles - 1;
     if (prm.wr < kUnbounded && j0 - prm.wr > 0) lo = (j0 - prm.wr) / kBlockQ;
@@ -679,6 +810,20 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     w.tiles_per_head = static_cast<int>(hi - lo + 1);
   }
   w.n_it = prm.group * w.tiles_per_head;
+  if constexpr (MASK == kMaskCols) {
+    // visible (head, tile) pairs: per head, the band's tiles minus the ones
+    // every key of this block hides; none at all: one fully masked tile, so
+    // dK = dV = 0 come out of TMEM
+    const int i_hi = w.i_lo + w.tiles_per_head - 1;
+    int n = 0;
+    Walk k;
+    for (k.hh = 0; k.hh < prm.group; ++k.hh) {
+      walk_head(k, prm, w, n_qtiles);
+      n += visible_count(k, w.i_lo, i_hi);
+    }
+    w.force = n == 0;
+    w.n_it = n > 0 ? n : 1;
+  }
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < C::kNumBars; ++i) {
@@ -717,12 +862,12 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     if (!ok && lane == 0) atomicOr(&g_status_bwd, kStatusTimeout);
   } else if (warp < kWarpLoad) {
     setmaxnreg_inc<176>();
-    const bool ok = dq_drain_role<D>(sm, tmem, &tm_dq, prm, w);
+    const bool ok = dq_drain_role<D, MASK>(sm, tmem, &tm_dq, prm, w);
     if (!ok && lane == 0) atomicOr(&g_status_bwd, kStatusTimeout);
   } else {
     setmaxnreg_dec<48>();
     if (warp == kWarpLoad) {
-      producer_role<D>(sm, &tm_q, &tm_k, &tm_v, &tm_do, prm, w, lane);
+      producer_role<D, MASK>(sm, &tm_q, &tm_k, &tm_v, &tm_do, prm, w, lane);
     } else if (warp == kWarpMma) {
       if (lane == 0) mma_role<D>(sm, tmem, w, prm.timeout_ns);
       __syncwarp();
@@ -769,7 +914,7 @@ __global__ void dq_finish_kernel(const float4* __restrict__ acc, uint2* __restri
   }
 }
 
-template <int D, bool MASK, bool PACKED>
+template <int D, int MASK, bool PACKED>
 int launch_main(const CUtensorMap* maps, const BwdParams& prm, int grid, cudaStream_t stream) {
   auto kern = attn_bwd_kernel<D, MASK, PACKED>;
   static std::once_flag once[kMaxDeviceCount];
@@ -798,6 +943,7 @@ size_t workspace_bytes(long long BH, long long Nq, int d) {
 // entries once the tensor maps and parameters are set up.
 int run_bwd(const CUtensorMap* maps, BwdParams& prm, const void* o, const void* dout, void* dq,
             size_t rows, int d, bool mask, int grid, cudaStream_t stream) {
+  const bool cols = prm.colmask != nullptr;
   cudaError_t e = cudaMemsetAsync(prm.dq_acc, 0, rows * d * 4, stream);
   if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync");
   {
@@ -815,19 +961,23 @@ int run_bwd(const CUtensorMap* maps, BwdParams& prm, const void* o, const void* 
   int rc;
   const bool packed = prm.cu_q != nullptr;
   if (d == 128) {
-    if (packed)
-      rc = mask ? launch_main<128, true, true>(maps, prm, grid, stream)
-                : launch_main<128, false, true>(maps, prm, grid, stream);
+    if (cols)
+      rc = launch_main<128, kMaskCols, false>(maps, prm, grid, stream);
+    else if (packed)
+      rc = mask ? launch_main<128, kMaskBand, true>(maps, prm, grid, stream)
+                : launch_main<128, kMaskNone, true>(maps, prm, grid, stream);
     else
-      rc = mask ? launch_main<128, true, false>(maps, prm, grid, stream)
-                : launch_main<128, false, false>(maps, prm, grid, stream);
+      rc = mask ? launch_main<128, kMaskBand, false>(maps, prm, grid, stream)
+                : launch_main<128, kMaskNone, false>(maps, prm, grid, stream);
   } else {
-    if (packed)
-      rc = mask ? launch_main<64, true, true>(maps, prm, grid, stream)
-                : launch_main<64, false, true>(maps, prm, grid, stream);
+    if (cols)
+      rc = launch_main<64, kMaskCols, false>(maps, prm, grid, stream);
+    else if (packed)
+      rc = mask ? launch_main<64, kMaskBand, true>(maps, prm, grid, stream)
+                : launch_main<64, kMaskNone, true>(maps, prm, grid, stream);
     else
-      rc = mask ? launch_main<64, true, false>(maps, prm, grid, stream)
-                : launch_main<64, false, false>(maps, prm, grid, stream);
+      rc = mask ? launch_main<64, kMaskBand, false>(maps, prm, grid, stream)
+                : launch_main<64, kMaskNone, false>(maps, prm, grid, stream);
   }
   if (rc != ATTN_OK) return rc;
   const size_t n4 = rows * d / 4;
@@ -840,10 +990,21 @@ int run_bwd(const CUtensorMap* maps, BwdParams& prm, const void* o, const void* 
 }
 
 // window_left / window_right: the key band of the forward (-1 = no bound).
+// Column intervals of attn_bwd_colmask: int32 [B, Hm, Nk, 4]; their block
+// summaries go to the end of the workspace.
+struct ColMaskArgs {
+  const int* mask;
+  int Hm;
+};
+
+size_t colmask_workspace_bytes(long long BH, long long Nq, int d, long long BHm, long long Nk) {
+  return align256(workspace_bytes(BH, Nq, d)) + static_cast<size_t>(BHm * ((Nk + kBlockK - 1) / kBlockK)) * 32;
+}
+
 int bwd_impl(const void* q, const void* k, const void* v, const void* o, const void* dout,
              const float* lse, void* dq, void* dk, void* dv, void* workspace, size_t ws_bytes, int B,
              int H, int Hkv, int Nq, int Nk, int d, float scale, int window_left, int window_right,
-             cudaStream_t stream) {
+             cudaStream_t stream, const ColMaskArgs* cm = nullptr) {
   if (B < 0 || H < 0 || Hkv < 0 || Nq < 0 || Nk < 0) return ATTN_ERR_INVALID_ARG;
   if (H > 0 && (Hkv == 0 || H % Hkv != 0)) return ATTN_ERR_INVALID_ARG;
   if (!std::isfinite(scale)) return ATTN_ERR_INVALID_ARG;
@@ -857,20 +1018,24 @@ int bwd_impl(const void* q, const void* k, const void* v, const void* o, const v
   const bool any_q = Nq > 0, any_k = Nk > 0;
   if ((any_q && (!q || !o || !dout || !lse || !dq)) || (any_k && (!k || !v || !dk || !dv)))
     return ATTN_ERR_INVALID_ARG;
-  const size_t need = workspace_bytes(BH, Nq, d);
+  if (cm && cm->Hm != 1 && cm->Hm != H) return ATTN_ERR_INVALID_ARG;
+  const long long BHm = cm ? static_cast<long long>(B) * cm->Hm : 0;
+  const size_t need = cm ? colmask_workspace_bytes(BH, Nq, d, BHm, Nk) : workspace_bytes(BH, Nq, d);
   if (any_q && any_k && (!workspace || ws_bytes < need)) return ATTN_ERR_INVALID_ARG;
+  if (cm && any_k && (!cm->mask || misaligned(cm->mask, 16))) return ATTN_ERR_INVALID_ARG;
   if (misaligned(q, 16) || misaligned(k, 16) || misaligned(v, 16) || misaligned(o, 16) ||
       misaligned(dout, 16) || misaligned(dq, 16) || misaligned(dk, 16) || misaligned(dv, 16) ||
       misaligned(lse, 4) || misaligned(workspace, 256))
     return ATTN_ERR_INVALID_ARG;
   // outputs may not overlap each other, any input, or the workspace
   const size_t lse_bytes = static_cast<size_t>(BH) * Nq * 4;
-  const void* ins[6] = {q, k, v, o, dout, lse};
-  const size_t in_bytes[6] = {q_bytes, kv_bytes, kv_bytes, q_bytes, q_bytes, lse_bytes};
+  const size_t mask_bytes = static_cast<size_t>(BHm) * Nk * 16;
+  const void* ins[7] = {q, k, v, o, dout, lse, cm ? cm->mask : nullptr};
+  const size_t in_bytes[7] = {q_bytes, kv_bytes, kv_bytes, q_bytes, q_bytes, lse_bytes, mask_bytes};
   void* outs[4] = {dq, dk, dv, workspace};
   const size_t out_bytes[4] = {q_bytes, kv_bytes, kv_bytes, any_q && any_k ? need : 0};
   for (int a = 0; a < 4; ++a) {
-    for (int b = 0; b < 6; ++b)
+    for (int b = 0; b < 7; ++b)
       if (ranges_overlap(outs[a], out_bytes[a], ins[b], in_bytes[b])) return ATTN_ERR_INVALID_ARG;
     for (int b = a + 1; b < 4; ++b)
       if (ranges_overlap(outs[a], out_bytes[a], outs[b], out_bytes[b])) return ATTN_ERR_INVALID_ARG;
@@ -924,6 +1089,14 @@ int bwd_impl(const void* q, const void* k, const void* v, const void* o, const v
   const bool mask = prm.wl < kUnbounded || prm.wr < kUnbounded;
   prm.scale_log2 = scale * kLog2e;
   prm.scale = scale;
+  if (cm) {
+    void* sum = static_cast<uint8_t*>(workspace) + align256(workspace_bytes(BH, Nq, d));
+    prm.colmask = reinterpret_cast<const int4*>(cm->mask);
+    prm.colsum = static_cast<const int4*>(sum);
+    prm.mask_heads = cm->Hm;
+    rc = launch_colmask_summary(cm->mask, sum, BHm, Nk, stream);
+    if (rc != ATTN_OK) return rc;
+  }
   return run_bwd(maps, prm, o, dout, dq, static_cast<size_t>(BH) * Nq, d, mask,
                  static_cast<int>(n_kblocks * BHkv), stream);
 }
@@ -1089,6 +1262,22 @@ int attn_bwd_window(const void* q, const void* k, const void* v, const void* o, 
                     float scale, int window_left, int window_right, cudaStream_t stream) {
   return eab::bwd::bwd_impl(q, k, v, o, dout, lse, dq, dk, dv, workspace, workspace_bytes, B, H, Hkv,
                             Nq, Nk, d, scale, window_left, window_right, stream);
+}
+
+size_t attn_bwd_colmask_workspace_size(int B, int H, int Nq, int d, int Hm, int Nk) {
+  if (B < 0 || H < 0 || Nq < 0 || Hm < 0 || Nk < 0 || (d != 64 && d != 128)) return 0;
+  return eab::bwd::colmask_workspace_bytes(static_cast<long long>(B) * H, Nq, d,
+                                           static_cast<long long>(B) * Hm, Nk);
+}
+
+int attn_bwd_colmask(const void* q, const void* k, const void* v, const void* o, const void* dout,
+                     const float* lse, void* dq, void* dk, void* dv, void* workspace,
+                     size_t workspace_bytes, int B, int H, int Hkv, int Nq, int Nk, int d, float scale,
+                     int causal, const int* mask, int Hm, cudaStream_t stream) {
+  if (causal != 0 && causal != 1) return ATTN_ERR_INVALID_ARG;
+  const eab::bwd::ColMaskArgs cm = {mask, Hm};
+  return eab::bwd::bwd_impl(q, k, v, o, dout, lse, dq, dk, dv, workspace, workspace_bytes, B, H, Hkv,
+                            Nq, Nk, d, scale, -1, causal ? 0 : -1, stream, &cm);
 }
 
 int attn_bwd_varlen(const void* q, const void* k, const void* v, const void* o, const void* dout,

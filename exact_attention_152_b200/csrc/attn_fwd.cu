@@ -987,6 +987,17 @@ __global__ void __launch_bounds__(128) colmask_summary_kernel(const int4* __rest
   }
 }
 
+int launch_colmask_summary(const int* mask, void* sum, long long BHm, int Nk, cudaStream_t stream) {
+  const int n_kblocks = (Nk + kBlockN - 1) / kBlockN;
+  const unsigned grid = static_cast<unsigned>(BHm * n_kblocks);
+  if (grid == 0) return ATTN_OK;
+  colmask_summary_kernel<<<grid, 128, 0, stream>>>(reinterpret_cast<const int4*>(mask),
+                                                   static_cast<int4*>(sum), Nk, n_kblocks);
+  const cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "colmask_summary_kernel launch");
+  return ATTN_OK;
+}
+
 // One thread waits on a barrier that nothing signals; the bounded wait gives
 // up and records a timeout.  Exercises the failure path without any fault.
 __global__ void selftest_timeout_kernel(uint64_t timeout_ns) {
@@ -1192,11 +1203,8 @@ int fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, i
     prm.colsum = static_cast<const int4*>(cm->workspace);
     prm.mask_heads = cm->Hm;
     prm.n_kblocks = (Nk + kBlockN - 1) / kBlockN;
-    const unsigned grid = static_cast<unsigned>(BHm * prm.n_kblocks);
-    colmask_summary_kernel<<<grid, 128, 0, stream>>>(prm.colmask, static_cast<int4*>(cm->workspace),
-                                                     Nk, prm.n_kblocks);
-    const cudaError_t e = cudaGetLastError();
-    if (e != cudaSuccess) return cuda_fail(e, "colmask_summary_kernel launch");
+    const int rc2 = launch_colmask_summary(cm->mask, cm->workspace, BHm, Nk, stream);
+    if (rc2 != ATTN_OK) return rc2;
   }
   return launch_any(d, exp_mode, tq, tk, tv, to, prm, stream);
 }

@@ -287,6 +287,26 @@ int attn_bwd_window(const void *q, const void *k, const void *v, const void *o, 
  * sequence and record the fact, which the next attn_status_sync() returns as
  * ATTN_ERR_INVALID_ARG.  Other errors as attn_bwd.
  */
+/*
+ * Backward of attn_fwd_colmask (column intervals; see that call for the mask):
+ * the chain rule of attn_bwd over the visible (query, key) pairs.
+ *   q, o, dout, dq : BF16 [B, H, Nq, d]    k, v, dk, dv : BF16 [B, Hkv, Nk, d]
+ *   lse  : FP32 [B, H, Nq] from attn_fwd_colmask
+ *   mask, Hm, causal : as attn_fwd_colmask
+ *   workspace : DEVICE, 256-byte aligned, at least
+ *       attn_bwd_colmask_workspace_size(B, H, Nq, d, Hm, Nk) bytes (attn_bwd's
+ *       workspace followed by the mask's block summaries), overwritten
+ * Each CTA owns a 128-key block; the query tiles that every key of the block
+ * hides form at most two ranges per query head, which are skipped outright.
+ * Errors as attn_bwd, plus ATTN_ERR_INVALID_ARG for a NULL or misaligned mask,
+ * Hm not in {1, H}, or a mask overlapping an output or the workspace.
+ */
+size_t attn_bwd_colmask_workspace_size(int B, int H, int Nq, int d, int Hm, int Nk);
+int attn_bwd_colmask(const void *q, const void *k, const void *v, const void *o, const void *dout,
+                     const float *lse, void *dq, void *dk, void *dv, void *workspace,
+                     size_t workspace_bytes, int B, int H, int Hkv, int Nq, int Nk, int d, float scale,
+                     int causal, const int *mask, int Hm, cudaStream_t stream);
+
 int attn_bwd_varlen(const void *q, const void *k, const void *v, const void *o, const void *dout,
                     const float *lse, void *dq, void *dk, void *dv, void *workspace,
                     size_t workspace_bytes, const int *cu_seqlens_q, const int *cu_seqlens_k,

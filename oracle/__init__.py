@@ -63,6 +63,10 @@ def _load():
                           ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64,
                           ctypes.c_double, ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p,
                           ctypes.c_void_p, ctypes.c_int]
+            bc = lib.oracle_attn_bwd_colmask_f64
+            bc.restype = ctypes.c_int
+            bc.argtypes = [ctypes.c_void_p] * 4 + [ctypes.c_int64] * 3 + [ctypes.c_double, ctypes.c_int] + \
+                [ctypes.c_void_p] * 4
             b = lib.oracle_attn_bwd_f64
             b.restype = ctypes.c_int
             b.argtypes = [ctypes.c_void_p] * 4 + [ctypes.c_int64] * 3 + [ctypes.c_double] + \
@@ -271,4 +275,48 @@ def attn_bwd_varlen(q, k, v, dout, cu_seqlens_q, cu_seqlens_k, scale, window_lef
         dq[q0:q1] = g[0][0].transpose(1, 0, 2)
         dk[k0:k1] = g[1][0].transpose(1, 0, 2)
         dv[k0:k1] = g[2][0].transpose(1, 0, 2)
+    return dq, dk, dv
+
+
+def attn_bwd_colmask_head(q, k, v, dout, scale, causal, cols):
+    """Gradients of one (batch, head) under column intervals (cols [Nk, 4]:
+    key j hidden from rows [lo1, hi1) and [lo2, hi2), and from rows i < j when
+    causal); see oracle_attn_bwd_colmask_f64."""
+    lib = _load()
+    q, k, v, dout = (np.ascontiguousarray(x, dtype=np.float64) for x in (q, k, v, dout))
+    cols = np.ascontiguousarray(cols, dtype=np.int64)
+    nq, d = q.shape
+    nk = k.shape[0]
+    assert cols.shape == (nk, 4)
+    dq, dk, dv = np.empty((nq, d)), np.empty((nk, d)), np.empty((nk, d))
+    ptr = lambda a: a.ctypes.data if a.size else None  # noqa: E731
+    rc = lib.oracle_attn_bwd_colmask_f64(ptr(q), ptr(k), ptr(v), ptr(dout), nq, nk, d, float(scale),
+                                         1 if causal else 0, ptr(cols), ptr(dq), ptr(dk), ptr(dv))
+    if rc != 0:
+        raise RuntimeError("oracle_attn_bwd_colmask_f64 failed")
+    return dq, dk, dv
+
+
+def attn_bwd_colmask(q, k, v, dout, scale, causal, mask, nthreads=None):
+    """Gradients over [B, H, Nq, d] q/dout and [B, Hkv, Nk, d] k/v under the
+    column intervals mask [B, Hm, Nk, 4] (Hm = 1: shared by the heads of a
+    batch entry); key/value gradients of a shared head summed in head order."""
+    import concurrent.futures
+    q, k, v, dout = (np.asarray(x, dtype=np.float64) for x in (q, k, v, dout))
+    B, H = q.shape[:2]
+    g = H // k.shape[1]
+    hm = mask.shape[1]
+    jobs = [(b, h) for b in range(B) for h in range(H)]
+    nt = default_threads() if nthreads is None else int(nthreads)
+    with concurrent.futures.ThreadPoolExecutor(max_workers=max(1, nt)) as ex:
+        res = list(ex.map(lambda bh: attn_bwd_colmask_head(
+            q[bh[0], bh[1]], k[bh[0], bh[1] // g], v[bh[0], bh[1] // g], dout[bh[0], bh[1]], scale,
+            causal, mask[bh[0], bh[1] if hm > 1 else 0]), jobs))
+    dq = np.empty(q.shape)
+    dk = np.zeros(k.shape)
+    dv = np.zeros(v.shape)
+    for (b, h), (a, bk, bv) in zip(jobs, res):
+        dq[b, h] = a
+        dk[b, h // g] += bk
+        dv[b, h // g] += bv
     return dq, dk, dv

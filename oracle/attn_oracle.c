@@ -343,3 +343,66 @@ int oracle_attn_bwd_f64(const double *q, const double *k, const double *v,
     free(dp);
     return 0;
 }
+
+/*
+ * The same backward under column intervals (cols [nk, 4] int64, key j's
+ * (lo1, hi1, lo2, hi2); causal also hides keys j > i): the visible keys of a
+ * row need not be contiguous, so they are listed first, then the steps above
+ * run over the list.
+ */
+int oracle_attn_bwd_colmask_f64(const double *q, const double *k, const double *v,
+                                const double *dout, int64_t nq, int64_t nk, int64_t d,
+                                double scale, int causal, const int64_t *cols,
+                                double *dq, double *dk, double *dv) {
+    if (nq < 0 || nk < 0 || d <= 0 || (nk > 0 && !cols)) return -1;
+    for (int64_t x = 0; x < nk * d; ++x) { dk[x] = 0.0; dv[x] = 0.0; }
+    for (int64_t x = 0; x < nq * d; ++x) dq[x] = 0.0;
+    if (nq == 0 || nk == 0) return 0;
+    double *p = (double *)malloc((size_t)nk * sizeof(double));
+    double *dp = (double *)malloc((size_t)nk * sizeof(double));
+    int64_t *vis = (int64_t *)malloc((size_t)nk * sizeof(int64_t));
+    if (!p || !dp || !vis) { free(p); free(dp); free(vis); return -1; }
+    for (int64_t i = 0; i < nq; ++i) {
+        const double *qi = q + i * d, *gi = dout + i * d;
+        int64_t n = 0;
+        for (int64_t j = 0; j < nk; ++j) {
+            const int64_t *c = cols + 4 * j;
+            const int hidden = (causal && j > i) || (c[0] <= i && i < c[1]) ||
+                               (c[2] <= i && i < c[3]);
+            if (!hidden) vis[n++] = j;
+        }
+        if (n == 0) continue; /* no visible key: O_i = 0 does not depend on the inputs */
+        double m = -INFINITY;
+        for (int64_t t = 0; t < n; ++t) {
+            const int64_t j = vis[t];
+            double dot = 0.0;
+            for (int64_t c = 0; c < d; ++c) dot += qi[c] * k[j * d + c];
+            p[t] = scale * dot;
+            if (p[t] > m) m = p[t];
+        }
+        double l = 0.0;
+        for (int64_t t = 0; t < n; ++t) { p[t] = exp(p[t] - m); l += p[t]; }
+        for (int64_t t = 0; t < n; ++t) p[t] /= l;
+        double D = 0.0;
+        for (int64_t t = 0; t < n; ++t) {
+            const int64_t j = vis[t];
+            double dot = 0.0;
+            for (int64_t c = 0; c < d; ++c) dot += gi[c] * v[j * d + c];
+            dp[t] = dot;
+            D += p[t] * dot;
+        }
+        for (int64_t t = 0; t < n; ++t) {
+            const int64_t j = vis[t];
+            const double ds = p[t] * (dp[t] - D);
+            for (int64_t c = 0; c < d; ++c) {
+                dq[i * d + c] += scale * ds * k[j * d + c];
+                dk[j * d + c] += scale * ds * qi[c];
+                dv[j * d + c] += p[t] * gi[c];
+            }
+        }
+    }
+    free(p);
+    free(dp);
+    free(vis);
+    return 0;
+}

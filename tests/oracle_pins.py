@@ -398,6 +398,58 @@ COLMASK_PINS = [pin_colmask_band, pin_colmask_documents, pin_colmask_empty_inter
                 pin_colmask_two_intervals]
 
 
+def pin_bwd_colmask_finite_differences(attn_bwd_colmask_head, attn_rows_colmask):
+    """Every gradient element under column intervals (two intervals per key,
+    some rows seeing no key, causal or not) equals the central difference of
+    L = sum(dO * O) through the column-interval forward definition."""
+    h = 1e-5
+    r = _rng(340)
+    nq, nk, d = 6, 7, 2
+    cols = np.array([[2, 4, 5, 6], [0, 1, 3, 3], [4, 4, 0, 2], [1, 6, 0, 0], [5, 9, 1, 2],
+                     [0, 0, 0, 0], [3, 5, 0, 1]], dtype=np.int64)
+    rows = np.arange(nq, dtype=np.int64)
+    for causal in (False, True):
+        q, k, v, dout = (r.standard_normal(s) for s in ((nq, d), (nk, d), (nk, d), (nq, d)))
+        grads = attn_bwd_colmask_head(q, k, v, dout, 0.9, causal, cols)
+
+        def loss(q_, k_, v_):
+            o, _ = attn_rows_colmask(q_, rows, k_, v_, 0.9, causal, cols)
+            return float((o * dout).sum())
+        for which, x in enumerate((q, k, v)):
+            num = np.zeros_like(x)
+            for idx in np.ndindex(*x.shape):
+                args = [q.copy(), k.copy(), v.copy()]
+                args[which][idx] += h
+                lp = loss(*args)
+                args[which][idx] -= 2 * h
+                lm = loss(*args)
+                num[idx] = (lp - lm) / (2 * h)
+            np.testing.assert_allclose(grads[which], num, rtol=1e-6, atol=1e-8,
+                                       err_msg=f"grad {'qkv'[which]} causal {causal}")
+
+
+def pin_bwd_colmask_band_is_the_band(attn_bwd_colmask_head, attn_rows_colmask):
+    """Intervals that spell a band give the band's gradients (numpy softmax
+    Jacobian on the triu/tril mask: dV = P^T dO, dS = P (dP - rowsum(P dP)))."""
+    r = _rng(341)
+    n, d = 8, 3
+    q, k, v, dout = (r.standard_normal((n, d)) for _ in range(4))
+    for wl, wr in [(2, 1), (-1, 0), (0, 3)]:
+        dq, dk, dv = attn_bwd_colmask_head(q, k, v, dout, 0.6, False, band_as_columns(n, wl, wr))
+        m = band_mask_numpy(n, n, wl, wr)
+        s = np.where(m, 0.6 * q @ k.T, -np.inf)
+        p = np.exp(s - s.max(1, keepdims=True))
+        p /= p.sum(1, keepdims=True)
+        dp = dout @ v.T
+        ds = p * (dp - (p * dp).sum(1, keepdims=True))
+        np.testing.assert_allclose(dv, p.T @ dout, rtol=1e-12, atol=1e-12)
+        np.testing.assert_allclose(dq, 0.6 * ds @ k, rtol=1e-12, atol=1e-12)
+        np.testing.assert_allclose(dk, 0.6 * ds.T @ q, rtol=1e-12, atol=1e-12)
+
+
+BWD_COLMASK_PINS = [pin_bwd_colmask_finite_differences, pin_bwd_colmask_band_is_the_band]
+
+
 ALL_PINS = [
     pin_brute_force, pin_golden, pin_single_key, pin_identical_keys, pin_zero_scale,
     pin_causal_prefix, pin_rows_sum_to_one, pin_shift_invariance, pin_value_linearity,

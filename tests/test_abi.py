@@ -49,7 +49,7 @@ def test_library_exports_every_declared_symbol(header):
 def test_attn_h_declares_the_contract():
     names = declared_functions(os.path.join(ROOT, "include", "attn.h"))
     for n in ("attn_fwd", "attn_fwd_config", "attn_fwd_gqa", "attn_fwd_window", "attn_fwd_varlen",
-              "attn_fwd_fp8", "attn_fwd_colmask", "attn_colmask_workspace_size", "attn_bwd", "attn_bwd_window", "attn_bwd_varlen", "attn_bwd_noalloc", "attn_bwd_workspace_size", "attn_status_sync", "attn_status_string",
+              "attn_fwd_fp8", "attn_fwd_colmask", "attn_colmask_workspace_size", "attn_bwd", "attn_bwd_window", "attn_bwd_varlen", "attn_bwd_colmask", "attn_bwd_colmask_workspace_size", "attn_bwd_noalloc", "attn_bwd_workspace_size", "attn_status_sync", "attn_status_string",
               "attn_last_error", "attn_selftest_timeout"):
         assert n in names
 
@@ -206,6 +206,29 @@ def test_bwd_validation():
     assert BW(*ptrs, need, 1, 2, 2, 64, 64, 64, 0.1, -2, 0, None) == 1    # band below -1
     assert BW(*ptrs, need, 1, 2, 2, 64, 64, 64, 0.1, 0, -3, None) == 1
     assert BW(*ptrs, need - 1, 1, 2, 2, 64, 64, 64, 0.1, 8, 0, None) == 1  # workspace too small
+
+
+def test_bwd_colmask_validation():
+    BC = binding.attn_bwd_colmask
+    A = ALIGNED
+    ptrs = (A, A * 2, A * 3, A * 4, A * 5, A * 6, A * 7, A * 8, A * 9, A * 16)
+    base = binding.attn_bwd_workspace_size(1, 2, 64, 64)
+    need = binding.attn_bwd_colmask_workspace_size(1, 2, 64, 64, 1, 64)
+    assert need == (base + 255) // 256 * 256 + 32     # + one key block's two int4 summaries
+    assert binding.attn_bwd_colmask_workspace_size(1, 2, 64, 96, 1, 64) == 0
+    M = A * 40
+    sizes = (1, 2, 2, 64, 64, 64, 0.1, 0)
+
+    def call(ws=need, mask=M, hm=1, sz=sizes, p=ptrs):
+        return BC(*p, ws, *sz, mask, hm, None)
+    assert call(ws=need - 1) == 1                      # workspace too small
+    assert call(ws=base) == 1                          # room for attn_bwd only
+    assert call(mask=None) == 1
+    assert call(mask=M + 4) == 1                       # misaligned mask
+    assert call(hm=3) == 1                             # Hm not in {1, H}
+    assert call(mask=A * 7) == 1                       # mask inside dq
+    assert call(sz=sizes[:7] + (2,)) == 1              # causal flag
+    assert call(sz=sizes[:5] + (80,) + sizes[6:]) == 2
 
 
 def test_bwd_varlen_validation():

@@ -141,3 +141,92 @@ def test_colmask_documents_sampled_rows_long():
     scale = float(np.float32(1 / math.sqrt(d)))
     o, lse = _run(q, k, v, mask, True, scale)
     harness.assert_within(harness.compare(o, lse, _oracle(q, k, v, mask, True, scale, 96, 313)))
+
+
+BWD_CASES = [
+    # kind, B, H, Hkv, Nq, Nk, d
+    ("docs", 1, 2, 2, 1000, 1000, 128),
+    ("docs_bidir", 1, 2, 1, 777, 777, 64),
+    ("prefix", 1, 2, 2, 900, 900, 128),
+    ("random", 1, 2, 2, 520, 520, 128),
+    ("random", 1, 2, 2, 300, 1000, 64),          # Nq < Nk
+    ("random_heads", 1, 4, 2, 600, 600, 128),    # one mask per head, grouped K/V
+    ("random_causal", 1, 2, 2, 700, 700, 128),
+    ("random", 1, 2, 2, 1000, 130, 128),         # Nq > Nk, one ragged key block
+]
+
+
+@pytest.mark.parametrize("case", BWD_CASES, ids=[str(c) for c in BWD_CASES])
+def test_colmask_bwd_parity(case):
+    """attn_bwd_colmask against the oracle's chain rule under the same intervals
+    (tolerance as the dense backward's)."""
+    import torch
+    from exact_attention_152_b200 import binding
+    from test_bwd_gpu import check_grads
+    kind, B, H, Hkv, Nq, Nk, d = case
+    seed = 320 + Nq + d
+    q = harness.random_bits(seed, (B, H, Nq, d), tensor="q")
+    k = harness.random_bits(seed, (B, Hkv, Nk, d), tensor="k")
+    v = harness.random_bits(seed, (B, Hkv, Nk, d), tensor="v")
+    do = harness.random_bits(seed + 1, (B, H, Nq, d), tensor="q")
+    mask, causal = _mask(kind, seed, B, H, Nq, Nk)
+    scale = float(np.float32(1 / math.sqrt(d)))
+    qd, kd, vd, dod = (harness.to_device_bf16(x) for x in (q, k, v, do))
+    md = torch.from_numpy(mask).cuda()
+    o, lse = binding.fwd_colmask(qd, kd, vd, md, causal=causal, scale=scale)
+    grads = binding.bwd_colmask(qd, kd, vd, o, dod, lse, md, causal=causal, scale=scale)
+    assert binding.attn_status_sync(torch.cuda.current_stream().cuda_stream) == 0
+    got = tuple(x.float().cpu().numpy() for x in grads)
+    f = inputs.bf16_bits_to_f64
+    ref = oracle.attn_bwd_colmask(f(q), f(k), f(v), f(do), scale, causal, mask)
+    check_grads(got, ref, str(case))
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_colmask_bwd_equals_band_and_plain(d):
+    """An all-empty mask gives attn_bwd's dK and dV bit for bit (causal or not),
+    and a band spelled as intervals gives attn_bwd_window's: the same query
+    tiles are visited and the same pairs masked.  dQ, reduced in no fixed
+    order, agrees to fp32 rounding."""
+    import torch
+    from exact_attention_152_b200 import binding
+    B, H, N = 1, 2, 900
+    q, k, v = (harness.to_device_bf16(harness.random_bits(330, (B, H, N, d), tensor=t)) for t in "qkv")
+    do = harness.to_device_bf16(harness.random_bits(331, (B, H, N, d), tensor="q"))
+    cases = [(masks.empty(B, 1, N), False, dict(causal=False)),
+             (masks.empty(B, 1, N), True, dict(causal=True)),
+             (masks.band(B, N, 200, 0), False, dict(window=(200, 0))),
+             (masks.band(B, N, 100, 300), False, dict(window=(100, 300)))]
+    for mask, causal, kw in cases:
+        o, lse = binding.fwd(q, k, v, **kw)
+        ref = binding.bwd(q, k, v, o, do, lse, **kw)
+        got = binding.bwd_colmask(q, k, v, o, do, lse, torch.from_numpy(mask).cuda(), causal=causal)
+        torch.cuda.synchronize()
+        assert torch.equal(got[1].view(torch.int16), ref[1].view(torch.int16)), kw
+        assert torch.equal(got[2].view(torch.int16), ref[2].view(torch.int16)), kw
+        torch.testing.assert_close(got[0].float(), ref[0].float(), rtol=1e-2, atol=1e-3)
+
+
+def test_colmask_bwd_hidden_blocks():
+    """Every key hides rows [200, 520) and keys 300..427 hide every row: the
+    hidden query tiles are skipped, keys no query sees get dK = dV = 0, and the
+    rest matches the oracle."""
+    import torch
+    from exact_attention_152_b200 import binding
+    from test_bwd_gpu import check_grads
+    B, H, N, d = 1, 2, 700, 128
+    q, k, v = (harness.random_bits(332, (B, H, N, d), tensor=t) for t in "qkv")
+    do = harness.random_bits(333, (B, H, N, d), tensor="q")
+    mask = masks.empty(B, 1, N)
+    mask[..., 2], mask[..., 3] = 200, 520
+    mask[0, 0, 300:428, 0], mask[0, 0, 300:428, 1] = 0, N
+    qd, kd, vd, dod = (harness.to_device_bf16(x) for x in (q, k, v, do))
+    md = torch.from_numpy(mask).cuda()
+    o, lse = binding.fwd_colmask(qd, kd, vd, md, scale=0.1)
+    dq, dk, dv = binding.bwd_colmask(qd, kd, vd, o, dod, lse, md, scale=0.1)
+    assert binding.attn_status_sync(torch.cuda.current_stream().cuda_stream) == 0
+    assert torch.all(dk[:, :, 300:428] == 0) and torch.all(dv[:, :, 300:428] == 0)
+    assert torch.all(dq[:, :, 200:520] == 0)
+    f = inputs.bf16_bits_to_f64
+    ref = oracle.attn_bwd_colmask(f(q), f(k), f(v), f(do), 0.1, False, mask)
+    check_grads(tuple(x.float().cpu().numpy() for x in (dq, dk, dv)), ref, "hidden")

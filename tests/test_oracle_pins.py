@@ -32,6 +32,11 @@ def test_bwd_varlen_pin_catches_wrong_offsets():
         pins.pin_bwd_varlen_finite_differences(shifted, oracle.attn_varlen)
 
 
+@pytest.mark.parametrize("pin", pins.BWD_COLMASK_PINS, ids=[p.__name__ for p in pins.BWD_COLMASK_PINS])
+def test_oracle_bwd_colmask_pin(pin):
+    pin(oracle.attn_bwd_colmask_head, oracle.attn_rows_colmask)
+
+
 @pytest.mark.parametrize("pin", pins.COLMASK_PINS, ids=[p.__name__ for p in pins.COLMASK_PINS])
 def test_oracle_colmask_pin(pin):
     pin(oracle.attn_rows_colmask)
@@ -118,6 +123,9 @@ MUTANTS = {
     "cols_causal_ignored": ("(jb->causal && j > i)", "(0 && j > i)"),
     "cols_value_not_gathered": ("const double *vj = jb->v + jb->vis[t] * d;",
                                 "const double *vj = jb->v + t * d;"),
+    "bwd_cols_second_interval_ignored": ("(c[2] <= i && i < c[3]);\n            if (!hidden) vis[n++] = j;",
+                                         "(0 && i < c[3]);\n            if (!hidden) vis[n++] = j;"),
+    "bwd_cols_dv_not_gathered": ("dv[j * d + c] += p[t] * gi[c];", "dv[t * d + c] += p[t] * gi[c];"),
     "bwd_band_ignored": ("if (window_right >= 0 && i + window_right < hi) hi = i + window_right;",
                          "if (0) hi = i + window_right;"),
 }
@@ -187,17 +195,33 @@ def _build_mutant(tmp_path, name, old, new):
           int(wl), int(wr), dq.ctypes.data, dk.ctypes.data, dv.ctypes.data)
         return dq, dk, dv
 
-    return attn_rows, attn_rows_window, attn_bwd_head, attn_rows_colmask
+    bcm = cdll.oracle_attn_bwd_colmask_f64
+    bcm.restype = ctypes.c_int
+    bcm.argtypes = [ctypes.c_void_p] * 4 + [ctypes.c_int64] * 3 + [ctypes.c_double, ctypes.c_int] + \
+        [ctypes.c_void_p] * 4
+
+    def attn_bwd_colmask_head(q, k, v, dout, scale, causal, cols):
+        q, k, v, dout = (np.ascontiguousarray(x, dtype=np.float64) for x in (q, k, v, dout))
+        cols = np.ascontiguousarray(cols, dtype=np.int64)
+        nq, d = q.shape
+        nk = k.shape[0]
+        dq, dk, dv = np.empty((nq, d)), np.empty((nk, d)), np.empty((nk, d))
+        bcm(q.ctypes.data, k.ctypes.data, v.ctypes.data, dout.ctypes.data, nq, nk, d, float(scale),
+            int(causal), cols.ctypes.data, dq.ctypes.data, dk.ctypes.data, dv.ctypes.data)
+        return dq, dk, dv
+
+    return attn_rows, attn_rows_window, attn_bwd_head, attn_rows_colmask, attn_bwd_colmask_head
 
 
 @pytest.mark.parametrize("name", sorted(MUTANTS))
 def test_planted_mistake_is_caught(tmp_path, name):
     old, new = MUTANTS[name]
-    rows_fn, window_fn, bwd_fn, colmask_fn = _build_mutant(tmp_path, name, old, new)
+    rows_fn, window_fn, bwd_fn, colmask_fn, bwd_cm_fn = _build_mutant(tmp_path, name, old, new)
     failed = []
     for pin_set, args in ((PINS, (rows_fn,)), (pins.WINDOW_PINS, (window_fn,)),
                           (pins.BWD_PINS, (bwd_fn, window_fn)),
-                          (pins.COLMASK_PINS, (colmask_fn,))):
+                          (pins.COLMASK_PINS, (colmask_fn,)),
+                          (pins.BWD_COLMASK_PINS, (bwd_cm_fn, colmask_fn))):
         for pin in pin_set:
             try:
                 pin(*args)
