@@ -237,10 +237,10 @@ __device__ __forceinline__ int next_block(const uint32_t* vis, int blk) {
   return blk;
 }
 
-// Rows [lo, hi) of a warp's 32 rows starting at w0, as bits (lo, hi any ints).
-__device__ __forceinline__ uint32_t row_bits(int lo, int hi, int w0) {
-  const long long a = max(static_cast<long long>(lo) - w0, 0LL);
-  const long long b = min(static_cast<long long>(hi) - w0, 32LL);
+// Positions [lo, hi) of the 32 starting at base, as bits (bit i: base + i).
+__device__ __forceinline__ uint32_t span_bits(long long lo, long long hi, long long base) {
+  const long long a = max(lo - base, 0LL);
+  const long long b = min(hi - base, 32LL);
   if (b <= a) return 0u;
   const uint32_t upto = b >= 32 ? 0xffffffffu : ((1u << b) - 1u);
   return upto & ~((1u << a) - 1u);
@@ -543,8 +543,8 @@ __device__ __forceinline__ void softmax_role(const Smem<D, F8>& sm, uint32_t tme
         const int4 none = make_int4(0, 0, 0, 0);
         const int4 ia = lane < n_in ? __ldg(cm + lane) : none;
         const int4 ib = lane + 32 < n_in ? __ldg(cm + 32 + lane) : none;
-        const uint32_t ca = row_bits(ia.x, ia.y, rw0) | row_bits(ia.z, ia.w, rw0);
-        const uint32_t cb = row_bits(ib.x, ib.y, rw0) | row_bits(ib.z, ib.w, rw0);
+        const uint32_t ca = span_bits(ia.x, ia.y, rw0) | span_bits(ia.z, ia.w, rw0);
+        const uint32_t cb = span_bits(ib.x, ib.y, rw0) | span_bits(ib.z, ib.w, rw0);
 #pragma unroll
         for (int rr = 0; rr < 32; ++rr) {
           const uint32_t wa = __ballot_sync(0xffffffffu, (ca >> rr) & 1u);
@@ -555,6 +555,17 @@ __device__ __forceinline__ void softmax_role(const Smem<D, F8>& sm, uint32_t tme
           }
         }
       }
+    }
+    // the keys this row sees among the warp's 64, as two 32-bit words: below
+    // Nk, inside the band, and not hidden by a column interval (one bit test
+    // per score below instead of the comparisons themselves)
+    uint32_t keep[2] = {0xffffffffu, 0xffffffffu};
+    if (masked) {
+      const long long klo = MASK != kMaskNone ? static_cast<long long>(row) - prm.wl : 0;
+      const long long khi = MASK != kMaskNone ? min(static_cast<long long>(row) + prm.wr + 1, static_cast<long long>(Nk))
+                                              : static_cast<long long>(Nk);
+#pragma unroll
+      for (int k = 0; k < 2; ++k) keep[k] = span_bits(klo, khi, kv0 + 32 * k) & ~hid[k];
     }
     ok = warp_wait(sm.s_full(t), j & 1, timeout);
     // load 32 score columns [32*k, 32*k + 32) of this warp's half as fp32,
@@ -572,12 +583,8 @@ __device__ __forceinline__ void softmax_role(const Smem<D, F8>& sm, uint32_t tme
       }
       if (masked) {
 #pragma unroll
-        for (int c = 0; c < 32; ++c) {
-          const int key = kv0 + 32 * k + c;
-          if (key >= Nk || (MASK != kMaskNone && (key - row > prm.wr || row - key > prm.wl)) ||
-              (MASK == kMaskCols && ((hid[k] >> c) & 1u)))
-            x[c] = -INFINITY;
-        }
+        for (int c = 0; c < 32; ++c)
+          if (!((keep[k] >> c) & 1u)) x[c] = -INFINITY;
       }
     };
 
