@@ -302,6 +302,15 @@ __device__ __forceinline__ void walk_next(Walk& k, const BwdParams& prm, const W
   walk_settle<MASK>(k, prm, w, n_qtiles);
 }
 
+// Positions [lo, hi) of the 32 starting at base, as bits (bit i: base + i).
+__device__ __forceinline__ uint32_t span_bits(long long lo, long long hi, long long base) {
+  const long long a = max(lo - base, 0LL);
+  const long long b = min(hi - base, 32LL);
+  if (b <= a) return 0u;
+  const uint32_t upto = b >= 32 ? 0xffffffffu : ((1u << b) - 1u);
+  return upto & ~((1u << a) - 1u);
+}
+
 // Tensor-map coordinates (column, row, head) in the map's dimension order:
 // dense maps are [BH, N, d], packed maps [total, H, d].
 __device__ __forceinline__ void load_rows(uint32_t dst, const CUtensorMap* tm, int col, int row, int head,
@@ -509,6 +518,19 @@ __device__ __forceinline__ bool softmax_grad_role(const Smem<D>& sm, uint32_t tm
       reg_fence32(sv);
       reg_fence32(pv);
       uint32_t pp[16], dsp[16];
+      // the queries of these 32 columns this key is visible to (bit c: query
+      // q_base + 32k + c): inside the band key - wr <= q <= key + wl and outside
+      // the key's column intervals; one bit test per score below instead of
+      // the comparisons themselves
+      uint32_t keep = 0xffffffffu;
+      if (masked) {
+        const long long base = q_base + 32 * k;
+        keep = key_in ? span_bits(MASK != kMaskNone ? static_cast<long long>(key) - prm.wr : base,
+                                  MASK != kMaskNone ? static_cast<long long>(key) + prm.wl + 1 : base + 32,
+                                  base)
+                      : 0u;
+        if (MASK == kMaskCols) keep &= ~(span_bits(kiv.x, kiv.y, base) | span_bits(kiv.z, kiv.w, base));
+      }
 #pragma unroll
       for (int g = 0; g < 8; ++g) {  // query columns 32k + 4g .. 32k + 4g + 3
         const float4 nl = nl4[8 * k + g], dv = dd4[8 * k + g];
@@ -517,26 +539,11 @@ __device__ __forceinline__ bool softmax_grad_role(const Smem<D>& sm, uint32_t tm
         float2 xb = ffma2(make_float2(__uint_as_float(sv[4 * g + 2]), __uint_as_float(sv[4 * g + 3])),
                           sl2, make_float2(nl.z, nl.w));
         if (masked) {
-          // query q = q_base + 32k + 4g + e is outside the band of this key when
-          // key - q > wr or q - key > wl; with d0 = key - (q_base + 32k + 4g):
-          // d0 - e > wr or e - d0 > wl
-          const int d0 = key - (q_base + 32 * k + 4 * g);
-          const int hi = prm.wr, lo = -prm.wl;  // visible iff lo <= d0 - e <= hi
-          if (!key_in || d0 > hi || d0 < lo) xa.x = -INFINITY;
-          if (!key_in || d0 - 1 > hi || d0 - 1 < lo) xa.y = -INFINITY;
-          if (!key_in || d0 - 2 > hi || d0 - 2 < lo) xb.x = -INFINITY;
-          if (!key_in || d0 - 3 > hi || d0 - 3 < lo) xb.y = -INFINITY;
-          if (MASK == kMaskCols) {
-            // query q0 + e hidden from this key by one of its intervals
-            const int q0 = q_base + 32 * k + 4 * g;
-            auto hid = [&](int e) {
-              return (kiv.x <= q0 + e && q0 + e < kiv.y) || (kiv.z <= q0 + e && q0 + e < kiv.w);
-            };
-            if (hid(0)) xa.x = -INFINITY;
-            if (hid(1)) xa.y = -INFINITY;
-            if (hid(2)) xb.x = -INFINITY;
-            if (hid(3)) xb.y = -INFINITY;
-          }
+          const uint32_t kw = keep >> (4 * g);
+          if (!(kw & 1u)) xa.x = -INFINITY;
+          if (!(kw & 2u)) xa.y = -INFINITY;
+          if (!(kw & 4u)) xb.x = -INFINITY;
+          if (!(kw & 8u)) xb.y = -INFINITY;
         }
         float2 pa, pb;
         if ((g & 3) == 0) {  // a quarter of the exponentials on the FMA pipe
