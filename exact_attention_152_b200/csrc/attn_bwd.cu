@@ -38,6 +38,12 @@
 //    memory for the dQ GEMM.  Warps 8-11 drain each dQ tile from TMEM into the
 //    fp32 accumulator with vector reductions.  Warp 12 loads (TMA), warp 13
 //    issues the MMAs from one thread.
+//  * Variants (template arguments): key band (causal, sliding windows) or
+//    column intervals (attn_bwd_colmask; the query tiles every key of the
+//    block hides form at most two ranges per head and are stepped over), and
+//    packed variable-length batches (attn_bwd_varlen; per-sequence offsets,
+//    ragged dK/dV stores).  Masked scores are cleared by one bit test each
+//    against a per-key keep word.
 //  * Every wait is bounded; a timeout sets this file's status word and the CTA
 //    leaves its loops and exits cleanly.
 #include <cuda.h>
