@@ -54,7 +54,7 @@ def lib() -> ctypes.CDLL:
             l.attn_fwd_colmask.argtypes = [_P, _P, _P, _P, _P] + [_I] * 6 + [ctypes.c_float, _I, _P, _I,
                                                                           _P, ctypes.c_size_t, _P]
             l.attn_fwd_colmask.restype = _I
-            l.attn_colmask_workspace_size.argtypes = [_I] * 5
+            l.attn_colmask_workspace_size.argtypes = [_I, _I, _I]
             l.attn_colmask_workspace_size.restype = ctypes.c_size_t
             l.attn_fwd_varlen.argtypes = [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I,
                                           ctypes.c_float, _I, _I, _P]
@@ -109,8 +109,8 @@ def attn_fwd_colmask(q, k, v, o, lse, B, H, Hkv, Nq, Nk, d, scale, causal, mask,
                                   workspace, workspace_bytes, stream)
 
 
-def attn_colmask_workspace_size(B, H, Hm, Nq, Nk) -> int:
-    return lib().attn_colmask_workspace_size(B, H, Hm, Nq, Nk)
+def attn_colmask_workspace_size(B, Hm, Nk) -> int:
+    return lib().attn_colmask_workspace_size(B, Hm, Nk)
 
 
 def attn_fwd_varlen(q, k, v, o, lse, cu_seqlens_q, cu_seqlens_k, num_seqs, max_seqlen_q, total_q,
@@ -274,7 +274,7 @@ def fwd_colmask(q, k, v, mask, causal: bool = False, scale: float | None = None,
     an int32 CUDA mask [B, Hm, Nk, 4] (Hm = 1 or H): key j is hidden from query
     rows [mask[..., j, 0], mask[..., j, 1]) and [mask[..., j, 2], mask[..., j, 3]),
     and from rows i < j when causal.  workspace: a uint8 CUDA tensor of at least
-    attn_colmask_workspace_size(B, H, Hm, Nq, Nk) bytes (allocated when None).
+    attn_colmask_workspace_size(B, Hm, Nk) bytes (allocated when None).
     Returns (o, lse) on torch's current stream."""
     import torch
 
@@ -291,7 +291,7 @@ def fwd_colmask(q, k, v, mask, causal: bool = False, scale: float | None = None,
     Hm = mask.shape[1]
     if scale is None:
         scale = 1.0 / math.sqrt(d)
-    ws_bytes = attn_colmask_workspace_size(B, H, Hm, Nq, Nk)
+    ws_bytes = attn_colmask_workspace_size(B, Hm, Nk)
     if workspace is None:
         workspace = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=q.device)
     if out is None:

@@ -181,9 +181,6 @@ struct FwdParams {
   const int4* colsum;
   int mask_heads;    // 1 (one mask for all heads of a batch entry) or H
   int n_kblocks;     // key blocks per head: ceil(Nk / 128)
-  // column-interval mask: CTA order (tile of CTA i = perm[i], head-major), the
-  // most visited blocks first within each L2 head group; null: the order below
-  const int* perm;
 };
 
 // Where one CTA's sequence lives: lengths, first packed row (packed layout),
@@ -205,33 +202,6 @@ __device__ __forceinline__ void tma_load_rows(uint32_t dst, const CUtensorMap* t
                                               int head, bool packed, uint32_t bar) {
   if (packed) tma_load_3d(dst, tm, col, head, row, bar);
   else tma_load_3d(dst, tm, col, row, head, bar);
-}
-
-// KV tiles [j_lo, j_hi) that hold a key of the band for some of the rows of
-// query block qb; a block whose band holds none still visits one tile (fully
-// masked: O = 0, LSE = -inf).
-template <int MASK>
-__device__ __forceinline__ void kv_band_range(const FwdParams& prm, int Nq, int Nk, int qb, int* lo,
-                                              int* hi) {
-  const int n_all = max((Nk + kBlockN - 1) / kBlockN, 1);
-  int j_lo = 0, j_hi = n_all;
-  if (MASK != kMaskNone) {
-    // rows and bounds are below 2^31 and 2^30: the sums stay inside 64 bits
-    const long long r_lo = static_cast<long long>(qb) * kRowsPerCta;
-    const long long r_end = r_lo + kRowsPerCta < Nq ? r_lo + kRowsPerCta : Nq;
-    const long long r_hi = r_end - 1;
-    if (prm.wr < kUnbounded) {
-      const long long last = (r_hi + prm.wr) / kBlockN + 1;
-      if (last < j_hi) j_hi = static_cast<int>(last);
-    }
-    if (prm.wl < kUnbounded && r_lo - prm.wl > 0) j_lo = static_cast<int>((r_lo - prm.wl) / kBlockN);
-    if (j_lo >= j_hi) {
-      j_lo = min(j_lo, n_all - 1);
-      j_hi = j_lo + 1;
-    }
-  }
-  *lo = j_lo;
-  *hi = j_hi;
 }
 
 // Column-interval mask, block summaries (colmask_summary_kernel):
@@ -823,22 +793,17 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   // host so a group's K/V fits in L2), and within a group the heaviest query
   // blocks first, so short blocks fill the tail of each group while the next
   // group starts.
+  const int tile = blockIdx.x;
   int bh, qb;
-  if (MASK == kMaskCols && prm.perm != nullptr) {
-    // column intervals: the planned order (head-major tile numbers)
-    const int tile = __ldg(prm.perm + blockIdx.x);
-    bh = tile / prm.n_qblocks;
-    qb = tile % prm.n_qblocks;
-  } else if (prm.grouped) {
-    const int tile = blockIdx.x;
+  if (prm.grouped) {
     const int per_group = prm.hgroup * prm.n_qblocks;
     const int g = tile / per_group, w = tile % per_group;
     const int gsize = min(prm.hgroup, prm.BH - g * prm.hgroup);
     qb = prm.n_qblocks - 1 - w / gsize;
     bh = g * prm.hgroup + w % gsize;
   } else {
-    bh = blockIdx.x / prm.n_qblocks;
-    qb = blockIdx.x % prm.n_qblocks;
+    bh = tile / prm.n_qblocks;
+    qb = tile % prm.n_qblocks;
   }
   // grouped-query attention: query head h reads key/value head h / group of the
   // same batch entry (group = 1: one key/value head per query head)
@@ -879,8 +844,23 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     // KV tiles that hold a visible key for some row of this block; a block with
     // none (an empty band, an empty key set) still runs one fully masked tile,
     // which yields O = 0 and LSE = -inf.
-    int j_lo, j_hi;
-    kv_band_range<MASK>(prm, sv.Nq, sv.Nk, qb, &j_lo, &j_hi);
+    const int n_all = max((sv.Nk + kBlockN - 1) / kBlockN, 1);
+    int j_lo = 0, j_hi = n_all;
+    if (MASK != kMaskNone) {
+      // rows and bounds are below 2^31 and 2^30: the sums stay inside 64 bits
+      const long long r_lo = static_cast<long long>(qb) * kRowsPerCta;
+      const long long r_end = r_lo + kRowsPerCta < sv.Nq ? r_lo + kRowsPerCta : sv.Nq;
+      const long long r_hi = r_end - 1;
+      if (prm.wr < kUnbounded) {
+        const long long last = (r_hi + prm.wr) / kBlockN + 1;
+        if (last < j_hi) j_hi = static_cast<int>(last);
+      }
+      if (prm.wl < kUnbounded && r_lo - prm.wl > 0) j_lo = static_cast<int>((r_lo - prm.wl) / kBlockN);
+      if (j_lo >= j_hi) {
+        j_lo = min(j_lo, n_all - 1);
+        j_hi = j_lo + 1;
+      }
+    }
     sv.j_lo = j_lo;
     sv.n_kv = j_hi - j_lo;
     sv.mrow = 0;
@@ -1021,78 +1001,6 @@ __global__ void __launch_bounds__(128) colmask_summary_kernel(const int4* __rest
   }
 }
 
-// CTA order for column-interval masks: counting sort of the query blocks by
-// (L2 head group, most visited KV tiles first), so the long blocks of a group
-// start first and the short ones fill the tail.  One warp per query block
-// counts its visited tiles (the same test as the kernel's prologue) and bins
-// it; the histogram has kPlanBins bins per head group.
-constexpr int kPlanBins = 64;
-constexpr int kPlanMaxBins = 8192;  // shared-memory histogram of the scatter kernel
-
-template <int MASK>
-__global__ void __launch_bounds__(256) colmask_plan_count_kernel(const FwdParams prm, int* bin_of,
-                                                                 int* hist, int n_tiles) {
-  const int tile = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
-  if (tile >= n_tiles) return;
-  const int bh = tile / prm.n_qblocks, qb = tile % prm.n_qblocks;
-  const int hq = bh % prm.H, seq = bh / prm.H;
-  const int mrow = seq * prm.mask_heads + (prm.mask_heads == 1 ? 0 : hq);
-  int j_lo, j_hi;
-  kv_band_range<MASK>(prm, prm.Nq, prm.Nk, qb, &j_lo, &j_hi);
-  const int r0 = qb * kRowsPerCta, r1 = cta_row_end(qb, prm.Nq);
-  int cnt = 0;
-  for (int b = j_lo + lane; b < j_hi; b += 32) cnt += cols_hide_all(prm, mrow, b, r0, r1) ? 0 : 1;
-#pragma unroll
-  for (int off = 16; off > 0; off >>= 1) cnt += __shfl_xor_sync(0xffffffffu, cnt, off);
-  if (lane == 0) {
-    const int bin = (bh / prm.hgroup) * kPlanBins + (kPlanBins - 1 - min(cnt, kPlanBins - 1));
-    bin_of[tile] = bin;
-    atomicAdd(hist + bin, 1);
-  }
-}
-
-// One CTA: exclusive prefix sum of the histogram, then every query block takes
-// the next slot of its bin (the order inside a bin is arbitrary; each block
-// computes the same result wherever it runs).
-__global__ void __launch_bounds__(1024) colmask_plan_scatter_kernel(const int* bin_of, const int* hist,
-                                                                    int* perm, int n_tiles, int n_bins) {
-  __shared__ int off[kPlanMaxBins];
-  __shared__ int part[32];
-  const int t = threadIdx.x;
-  const int per = (n_bins + 1023) / 1024;
-  int sum = 0;
-  for (int i = t * per; i < min(n_bins, (t + 1) * per); ++i) sum += hist[i];
-  // exclusive scan of the 1024 partial sums: within each warp by shuffles,
-  // then over the 32 warp totals
-  const int lane = t & 31, w = t >> 5;
-  int inc = sum;
-#pragma unroll
-  for (int d = 1; d < 32; d <<= 1) {
-    const int y = __shfl_up_sync(0xffffffffu, inc, d);
-    if (lane >= d) inc += y;
-  }
-  if (lane == 31) part[w] = inc;
-  __syncthreads();
-  if (w == 0) {
-    const int tot = part[lane];
-    int winc = tot;
-#pragma unroll
-    for (int d = 1; d < 32; d <<= 1) {
-      const int y = __shfl_up_sync(0xffffffffu, winc, d);
-      if (lane >= d) winc += y;
-    }
-    part[lane] = winc - tot;  // exclusive prefix of the warp totals
-  }
-  __syncthreads();
-  int run = part[w] + inc - sum;
-  for (int i = t * per; i < min(n_bins, (t + 1) * per); ++i) {
-    off[i] = run;
-    run += hist[i];
-  }
-  __syncthreads();
-  for (int tile = t; tile < n_tiles; tile += 1024) perm[atomicAdd(&off[bin_of[tile]], 1)] = tile;
-}
-
 int launch_colmask_summary(const int* mask, void* sum, long long BHm, int Nk, cudaStream_t stream) {
   const int n_kblocks = (Nk + kBlockN - 1) / kBlockN;
   const unsigned grid = static_cast<unsigned>(BHm * n_kblocks);
@@ -1219,16 +1127,9 @@ struct ColMaskArgs {
   size_t workspace_bytes;
 };
 
-// Workspace of attn_fwd_colmask: the block summaries, then the CTA plan
-// (per query block its bin, the order, and the histogram).
-size_t colmask_summary_bytes(long long BHm, int Nk) {
+size_t colmask_workspace_bytes(long long BHm, int Nk) {
   const long long n_kblocks = (static_cast<long long>(Nk) + kBlockN - 1) / kBlockN;
   return static_cast<size_t>(BHm * n_kblocks) * 2 * sizeof(int4);
-}
-size_t colmask_workspace_bytes(long long BH, long long BHm, int Nq, int Nk) {
-  const long long n_tiles = BH * ((static_cast<long long>(Nq) + kRowsPerCta - 1) / kRowsPerCta);
-  const size_t sum = (colmask_summary_bytes(BHm, Nk) + 255) / 256 * 256;
-  return sum + static_cast<size_t>(n_tiles) * 8 + kPlanMaxBins * 4;
 }
 
 int fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
@@ -1264,7 +1165,7 @@ int fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, i
     if (cm->Hm != 1 && cm->Hm != H) return ATTN_ERR_INVALID_ARG;
     BHm = static_cast<long long>(B) * cm->Hm;
     mask_bytes = static_cast<size_t>(BHm) * Nk * sizeof(int4);
-    ws_need = colmask_workspace_bytes(BH, BHm, Nq, Nk);
+    ws_need = colmask_workspace_bytes(BHm, Nk);
     if (Nk > 0 && (!cm->mask || !cm->workspace)) return ATTN_ERR_INVALID_ARG;
     if (misaligned(cm->mask, 16) || misaligned(cm->workspace, 16)) return ATTN_ERR_INVALID_ARG;
     if (cm->workspace_bytes < ws_need) return ATTN_ERR_INVALID_ARG;
@@ -1318,28 +1219,6 @@ int fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, i
     prm.n_kblocks = (Nk + kBlockN - 1) / kBlockN;
     const int rc2 = launch_colmask_summary(cm->mask, cm->workspace, BHm, Nk, stream);
     if (rc2 != ATTN_OK) return rc2;
-    // CTA plan: the most visited query blocks of each L2 head group first (when
-    // the histogram fits; otherwise the grouped order below)
-    const int n_tiles = static_cast<int>(BH * n_qblocks);
-    const long long n_groups = (BH + prm.hgroup - 1) / prm.hgroup;
-    const long long n_bins = n_groups * kPlanBins;
-    if (n_bins <= kPlanMaxBins) {
-      uint8_t* base = static_cast<uint8_t*>(cm->workspace) + (colmask_summary_bytes(BHm, Nk) + 255) / 256 * 256;
-      int* bin_of = reinterpret_cast<int*>(base);
-      int* perm = bin_of + n_tiles;
-      int* hist = perm + n_tiles;
-      cudaError_t e = cudaMemsetAsync(hist, 0, static_cast<size_t>(n_bins) * 4, stream);
-      if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync");
-      const unsigned blocks = static_cast<unsigned>((n_tiles + 7) / 8);
-      colmask_plan_count_kernel<kMaskCols><<<blocks, 256, 0, stream>>>(prm, bin_of, hist, n_tiles);
-      e = cudaGetLastError();
-      if (e != cudaSuccess) return cuda_fail(e, "colmask_plan_count_kernel launch");
-      colmask_plan_scatter_kernel<<<1, 1024, 0, stream>>>(bin_of, hist, perm, n_tiles,
-                                                          static_cast<int>(n_bins));
-      e = cudaGetLastError();
-      if (e != cudaSuccess) return cuda_fail(e, "colmask_plan_scatter_kernel launch");
-      prm.perm = perm;
-    }
   }
   return launch_any(d, exp_mode, tq, tk, tv, to, prm, stream);
 }
@@ -1502,9 +1381,9 @@ int attn_fwd_window(const void* q, const void* k, const void* v, void* o, float*
                        eab::kDefaultThreshold, 1, nullptr, stream);
 }
 
-size_t attn_colmask_workspace_size(int B, int H, int Hm, int Nq, int Nk) {
-  if (B < 0 || H < 0 || Hm < 0 || Nq < 0 || Nk < 0) return 0;
-  return eab::colmask_workspace_bytes(static_cast<long long>(B) * H, static_cast<long long>(B) * Hm, Nq, Nk);
+size_t attn_colmask_workspace_size(int B, int Hm, int Nk) {
+  if (B < 0 || Hm < 0 || Nk < 0) return 0;
+  return eab::colmask_workspace_bytes(static_cast<long long>(B) * Hm, Nk);
 }
 
 int attn_fwd_colmask(const void* q, const void* k, const void* v, void* o, float* lse, int B,

@@ -132,19 +132,18 @@ int attn_fwd_window(const void *q, const void *k, const void *v, void *o, float 
  *          aligned; Hm == 1 (one mask per batch entry, shared by all heads) or
  *          Hm == H (one per query head).  Read only.
  *   workspace : DEVICE, 16-byte aligned, at least
- *          attn_colmask_workspace_size(B, H, Hm, Nq, Nk) bytes, owned by the
- *          caller; overwritten with per-128-key-block summaries of the mask
- *          and the CTA order, so it may not overlap any other argument.  Calls
- *          on different streams need different workspaces.
- * The call enqueues on `stream`: the block summaries; a plan that orders the
- * CTAs by the number of key blocks their rows see (most first within each
- * L2-sized group of heads); then the attention kernel, which skips every
- * 128-key block that hides all 256 query rows of a CTA and masks element-wise
- * only in blocks whose intervals meet a warp's 32 rows.  Errors as attn_fwd_gqa, plus ATTN_ERR_INVALID_ARG for a NULL
+ *          attn_colmask_workspace_size(B, Hm, Nk) bytes, owned by the caller;
+ *          overwritten with per-128-key-block summaries of the mask, so it may
+ *          not overlap any other argument.  Calls on different streams need
+ *          different workspaces.
+ * The call launches two kernels on `stream`: the block summaries, then the
+ * attention kernel, which skips every 128-key block that hides all 256 query
+ * rows of a CTA and masks element-wise only in blocks whose intervals meet a
+ * warp's 32 rows.  Errors as attn_fwd_gqa, plus ATTN_ERR_INVALID_ARG for a NULL
  * or misaligned mask or workspace, a workspace that is too small or overlaps
  * another argument, or Hm not in {1, H}.
  */
-size_t attn_colmask_workspace_size(int B, int H, int Hm, int Nq, int Nk);
+size_t attn_colmask_workspace_size(int B, int Hm, int Nk);
 int attn_fwd_colmask(const void *q, const void *k, const void *v, void *o, float *lse, int B,
                      int H, int Hkv, int Nq, int Nk, int d, float scale, int causal,
                      const int *mask, int Hm, void *workspace, size_t workspace_bytes,

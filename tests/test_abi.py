@@ -125,12 +125,10 @@ def test_colmask_validation():
     P = (ALIGNED, ALIGNED * 2, ALIGNED * 3, ALIGNED * 16, None)
     sizes = (1, 4, 2, 8, 8, 64, 0.1, 0)            # B, H, Hkv, Nq, Nk, d, scale, causal
     M, WS = ALIGNED * 40, ALIGNED * 48
-    need = binding.attn_colmask_workspace_size(1, 4, 1, 8, 8)
-    # one key block's two int4 summaries (padded to 256 B), per query block its
-    # bin and its slot in the order, and the plan's 8192-bin histogram
-    assert need == 256 + 4 * 8 + 8192 * 4
-    assert binding.attn_colmask_workspace_size(2, 4, 4, 300, 129) == 512 + 2 * 4 * 2 * 8 + 8192 * 4
-    assert binding.attn_colmask_workspace_size(-1, 4, 1, 8, 8) == 0
+    need = binding.attn_colmask_workspace_size(1, 1, 8)
+    assert need == 32                              # one key block: two int4 summaries
+    assert binding.attn_colmask_workspace_size(2, 4, 129) == 2 * 4 * 2 * 32
+    assert binding.attn_colmask_workspace_size(-1, 1, 8) == 0
 
     def call(ptrs=P, sz=sizes, mask=M, hm=1, ws=WS, ws_bytes=need):
         return C(*ptrs, *sz, mask, hm, ws, ws_bytes, None)
