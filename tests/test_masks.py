@@ -70,3 +70,14 @@ def test_prefix_lm():
     m = masks.prefix_lm(1, 12, 4)[0, 0]
     i, j = np.meshgrid(np.arange(12), np.arange(12), indexing="ij")
     assert np.array_equal(dense_visible(m, 12, False), (j < 4) | (j <= i))
+
+
+def test_document_workload_flops_closed_form():
+    """The document workload counts 4*d*H FLOPs per visible pair: for causal
+    documents that is sum over documents of n(n+1)/2 pairs per batch entry."""
+    from exact_attention_152_b200.workloads import WORKLOADS
+    w = WORKLOADS["docs_b2h16n8k_d128_causal"]
+    pairs = sum(n * (n + 1) // 2 for b in range(w.B) for n in w.doc_lengths(b))
+    assert w.flops == 4.0 * w.d * w.H * pairs
+    assert all(sum(w.doc_lengths(b)) == w.Nk for b in range(w.B))
+    assert all(256 <= n <= 4096 for b in range(w.B) for n in w.doc_lengths(b)[:-1])
