@@ -55,6 +55,8 @@ def parse_args(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--exp-mode", type=int, default=None, help="0 MUFU, 1 split, 2 polynomial")
     ap.add_argument("--threshold", type=float, default=None, help="rescale threshold (powers of 2)")
+    ap.add_argument("--count-rescales", action="store_true",
+                    help="after timing, one extra launch counts the (row, KV step) rescale events")
     ap.add_argument("--pass", dest="which", choices=["fwd", "bwd"], default="fwd",
                     help="time the forward (default) or the backward pass")
     return ap.parse_args(argv)
@@ -403,7 +405,7 @@ def run_ours(args):
         host_mask = mask = None
     stream = torch.cuda.current_stream(dev)
     sh = stream.cuda_stream
-    knobs = args.exp_mode is not None or args.threshold is not None
+    knobs = args.exp_mode is not None or args.threshold is not None or args.count_rescales
     thr = 8.0 if args.threshold is None else args.threshold
     em = 1 if args.exp_mode is None else args.exp_mode
     if knobs and (w.packed or w.window is not None or w.kv_heads != w.H or w.fp8 or w.colmask):
@@ -517,6 +519,30 @@ def run_ours(args):
               for x in (hq, hk, hv) + ((hc,) if w.packed else ()) + ((hm,) if w.colmask else ()))
     d2h = ho.numel() * ho.element_size() + hl.numel() * hl.element_size()
 
+    # rescale events of one launch (outside the timed region): rows whose
+    # reference max moved at a KV step after their first
+    rescales = None
+    if args.count_rescales:
+        cnt = torch.zeros(1, dtype=torch.int64, device=dev)
+        rc = binding.attn_fwd_config(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
+                                     w.B, w.H, w.Nq, w.Nk, w.d, w.scale, int(w.causal), thr, em,
+                                     cnt.data_ptr(), sh)
+        binding.check(rc, "attn_fwd_config")
+        binding.check(binding.attn_status_sync(sh), "rescale count")
+        n = int(cnt.item())
+        rows = w.B * w.H * w.Nq
+        # KV steps after the first, summed over rows: a CTA of 256 query rows
+        # visits KV tiles of 128 keys up to its last row's (causal) or all
+        n_all = (w.Nk + 127) // 128
+        steps = 0.0
+        for r0 in range(0, w.Nq, 256):
+            r1 = min(r0 + 256, w.Nq)
+            n_kv = min((r1 - 1) // 128 + 1, n_all) if w.causal else n_all
+            steps += (r1 - r0) * (n_kv - 1)
+        steps *= w.B * w.H
+        rescales = {"threshold": thr, "events": n, "rows": rows, "per_row": n / rows,
+                    "fraction_of_row_steps": n / steps if steps else 0.0}
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(w, args.cpu_seconds)
@@ -559,6 +585,8 @@ def run_ours(args):
     if knobs:
         line["config"]["rescale_threshold"] = thr
         line["config"]["exp_mode"] = em
+    if rescales is not None:
+        line["rescale_events"] = rescales
     print(json.dumps(line), flush=True)
     return 0
 
