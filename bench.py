@@ -198,9 +198,10 @@ def oracle_units(w):
                 w.to_f64(x, w.head_bits(x, w.kv_head_of(bh))) for x in "kv"))
 
 
-def time_oracle_rows(w, n_rows, seed_off):
+def time_oracle_rows(w, n_rows, seed_off, keep=None):
     """Time the oracle on n_rows seeded query rows, taken unit by unit (all rows
-    of a head, then the next) so large samples span several heads."""
+    of a head, then the next) so large samples span several heads.  keep: a
+    list that receives (unit tag, rows, O, LSE) of every unit."""
     import oracle
     from exact_attention_152_b200 import inputs, masks
     from exact_attention_152_b200.workloads import visible_keys
@@ -219,14 +220,16 @@ def time_oracle_rows(w, n_rows, seed_off):
         if cols_all is not None:
             cols = cols_all[tag // w.H, 0]
             t0 = time.perf_counter()
-            oracle.attn_rows_colmask(q, rows, k, v, w.scale, w.causal, cols)
+            res = oracle.attn_rows_colmask(q, rows, k, v, w.scale, w.causal, cols)
             tot_t += time.perf_counter() - t0
             tot_f += 4.0 * w.d * float(masks.visible_per_row(cols, rows, w.causal).sum())
         else:
             t0 = time.perf_counter()
-            oracle.attn_rows_window(q, rows, k, v, w.scale, wl, wr)
+            res = oracle.attn_rows_window(q, rows, k, v, w.scale, wl, wr)
             tot_t += time.perf_counter() - t0
             tot_f += 4.0 * w.d * float(visible_keys(rows, nk, wl, wr).sum())
+        if keep is not None:
+            keep.append((tag, rows) + tuple(res))
         done += len(rows)
         units += 1
     return tot_t, tot_f, done, units
@@ -241,15 +244,38 @@ def calibrate_rows(w, seconds):
     return max(16, min(total_rows(w), int(n * seconds / max(dt, 1e-6))))
 
 
-def cpu_baseline(w, seconds):
+def cpu_baseline(w, seconds, o_gpu=None, lse_gpu=None):
+    """The oracle timed on sampled rows; with the GPU's O and LSE of the same
+    inputs (host arrays in the workload's layout) the same rows also give the
+    errors of the GPU result."""
     import oracle
     n = calibrate_rows(w, seconds)
-    dt, flops, n, heads = time_oracle_rows(w, n, 2000)
-    return {"value": flops / dt / 1e12, "unit": UNIT, "cores": oracle.default_threads(),
-            "kind": "oracle",
-            "sample": f"{n} seeded query rows over {heads} head(s) of {w.name} (visible keys "
-                      f"of {mask_words(w)}), fp64, {dt:.1f} s of oracle time; "
-                      f"value = those rows' algorithmic FLOPs / time"}
+    units = []
+    dt, flops, n, heads = time_oracle_rows(w, n, 2000, keep=units if o_gpu is not None else None)
+    out = {"value": flops / dt / 1e12, "unit": UNIT, "cores": oracle.default_threads(),
+           "kind": "oracle",
+           "sample": f"{n} seeded query rows over {heads} head(s) of {w.name} (visible keys "
+                     f"of {mask_words(w)}), fp64, {dt:.1f} s of oracle time; "
+                     f"value = those rows' algorithmic FLOPs / time"}
+    if o_gpu is not None:
+        eo, el = [], []
+        for tag, rows, o_ref, l_ref in units:
+            if w.packed:
+                s_, h_ = tag
+                g = int(w.cu_seqlens[s_]) + rows
+                og, lg = o_gpu[g, h_], lse_gpu[h_, g]
+            else:
+                b_, h_ = divmod(tag, w.H)
+                og, lg = o_gpu[b_, h_, rows], lse_gpu[b_, h_, rows]
+            eo.append(np.abs(og.astype(np.float64) - o_ref).ravel())
+            both = np.isneginf(lg) & np.isneginf(l_ref)
+            el.append(np.abs(np.where(both, 0.0, lg) - np.where(both, 0.0, l_ref)))
+        eo, el = np.concatenate(eo), np.concatenate(el)
+        out["parity"] = {"rows": int(n), "max_abs_o": float(eo.max()), "mean_abs_o": float(eo.mean()),
+                         "max_abs_lse": float(el.max()),
+                         "bound": ("E4M3 inputs: the per-element bound of the FP8 parity tests" if w.fp8 else
+                                   "max|dO| <= 1e-2, mean|dO| <= 1e-3, max|dLSE| <= 1e-3")}
+    return out
 
 
 def mask_words(w):
@@ -545,7 +571,7 @@ def run_ours(args):
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cpu = cpu_baseline(w, args.cpu_seconds)
+        cpu = cpu_baseline(w, args.cpu_seconds, o.float().cpu().numpy(), lse.cpu().numpy())
 
     if world > 1:
         dist.destroy_process_group()
