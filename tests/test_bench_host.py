@@ -1,0 +1,78 @@
+"""Host-side pieces of bench.py (CPU): workload descriptions, entry-point names,
+kernel hashes, and the cpu_baseline leg's parity report."""
+import os
+import sys
+
+import numpy as np
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import bench  # noqa: E402
+import oracle  # noqa: E402
+from exact_attention_152_b200.workloads import HEADLINE, WORKLOADS  # noqa: E402
+
+
+@pytest.mark.parametrize("name", sorted(WORKLOADS))
+def test_workload_config_and_names(name):
+    w = WORKLOADS[name]
+    cfg = bench.workload_config(w, 1)
+    assert cfg["workload"] == name and cfg["per_gpu_problem"]
+    assert w.flops > 0
+    assert bench.launch_name(w).startswith("attn_fwd")
+    assert bench.bwd_launch_name(w).startswith("attn_bwd")
+    if w.colmask:
+        assert bench.launch_name(w) == "attn_fwd_colmask" and "doc_lengths" in cfg
+    if w.packed:
+        assert bench.launch_name(w) == "attn_fwd_varlen" and cfg["num_seqs"] == len(w.seqlens)
+
+
+def test_kernel_hash_ignores_comments_and_tracks_code(tmp_path, monkeypatch):
+    h_fwd, h_bwd = bench.kernel_source_hash("fwd"), bench.kernel_source_hash("bwd")
+    assert h_fwd != h_bwd and len(h_fwd) == 16
+    # a copy of the sources with an extra comment hashes the same; a code change does not
+    csrc = os.path.join(ROOT, "exact_attention_152_b200", "csrc")
+    fake = tmp_path / "exact_attention_152_b200" / "csrc"
+    fake.mkdir(parents=True)
+    for n in bench.KERNEL_SOURCES["fwd"]:
+        (fake / n).write_text(open(os.path.join(csrc, n)).read())
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    assert bench.kernel_source_hash("fwd") == h_fwd
+    src = (fake / "attn_fwd.cu").read_text()
+    (fake / "attn_fwd.cu").write_text(src + "\n// a comment\n/* another */\n")
+    assert bench.kernel_source_hash("fwd") == h_fwd
+    (fake / "attn_fwd.cu").write_text(src + "\nstatic int extra_code = 1;\n")
+    assert bench.kernel_source_hash("fwd") != h_fwd
+
+
+def test_recorded_traffic_matches_current_sources():
+    """profiles/ncu_traffic.json holds the headline's counters for the current
+    kernel sources (the bench reports them as roofline.traffic)."""
+    t = bench.recorded_traffic(HEADLINE, "fwd")
+    assert t is not None and 0.8e8 < t < 4e8
+    assert bench.recorded_traffic(HEADLINE, "bwd") is not None
+
+
+@pytest.mark.parametrize("name", ["tiny_b1h2n128d64", "varlen16_h16_d128_causal"])
+def test_cpu_baseline_parity_report(name):
+    """With the oracle's own result standing in for the GPU's, the parity report
+    is exactly zero (indexing of dense and packed layouts); with zeros it is
+    the oracle's magnitudes."""
+    w = WORKLOADS[name]
+    shape_o = (w.total, w.H, w.d) if w.packed else (w.B, w.H, w.Nq, w.d)
+    shape_l = (w.H, w.total) if w.packed else (w.B, w.H, w.Nq)
+    zeros = bench.cpu_baseline(w, 0.5, np.zeros(shape_o, np.float32), np.zeros(shape_l, np.float32))
+    assert zeros["parity"]["rows"] > 0 and zeros["parity"]["max_abs_o"] > 0.1
+    if not w.packed:
+        o = np.zeros(shape_o)
+        lse = np.zeros(shape_l)
+        for b in range(w.B):
+            for h in range(w.H):
+                bh = b * w.H + h
+                q = w.to_f64("q", w.head_bits("q", bh))
+                k, v = (w.to_f64(x, w.head_bits(x, w.kv_head_of(bh))) for x in "kv")
+                o[b, h], lse[b, h] = oracle.attn_rows(q, np.arange(w.Nq), k, v, w.scale, w.causal)
+        exact = bench.cpu_baseline(w, 0.5, o, lse)["parity"]
+        assert exact["max_abs_o"] == 0.0 and exact["max_abs_lse"] == 0.0
