@@ -228,3 +228,21 @@ def test_planted_mistake_is_caught(tmp_path, name):
             except AssertionError:
                 failed.append(pin.__name__)
     assert failed, f"no pin catches the planted mistake {name}"
+
+
+def test_bwd_colmask_per_head_masks_and_group_sums():
+    """attn_bwd_colmask with one mask per query head: a head whose mask hides
+    every key gets dQ = 0 and adds nothing to its key/value head's dK, dV,
+    which then equal the other head's alone (two query heads on one K/V head)."""
+    r = np.random.default_rng(350)
+    B, H, N, d = 1, 2, 6, 3
+    q, dout = r.standard_normal((B, H, N, d)), r.standard_normal((B, H, N, d))
+    k, v = r.standard_normal((B, 1, N, d)), r.standard_normal((B, 1, N, d))
+    mask = np.zeros((B, H, N, 4), dtype=np.int32)
+    mask[0, 1, :, 0], mask[0, 1, :, 1] = 0, N  # head 1 sees nothing
+    dq, dk, dv = oracle.attn_bwd_colmask(q, k, v, dout, 0.8, False, mask)
+    assert np.all(dq[0, 1] == 0.0)
+    a, bk, bv = oracle.attn_bwd_colmask_head(q[0, 0], k[0, 0], v[0, 0], dout[0, 0], 0.8, False, mask[0, 0])
+    np.testing.assert_array_equal(dq[0, 0], a)
+    np.testing.assert_array_equal(dk[0, 0], bk)
+    np.testing.assert_array_equal(dv[0, 0], bv)
