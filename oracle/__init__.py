@@ -1,4 +1,5 @@
-"""fp64 CPU oracle for exact attention (forward).
+"""fp64 CPU oracle for exact attention: forward and backward, dense, key
+bands, packed variable-length batches and column-interval masks.
 
 TEST INFRASTRUCTURE.  Only ``tests/``, ``__graft_entry__.smoke()`` and the
 ``cpu_baseline`` / ``--impl reference`` legs of ``bench.py`` may import this
@@ -8,7 +9,11 @@ this package never imports the product.
 The arithmetic lives in ``attn_oracle.c`` (plain C, fp64, one query row at a
 time, written straight from the definition -- see that file's header for the
 citations and the readings of the pages).  This module only compiles it with
-gcc, marshals numpy arrays and loops over (batch, head).
+gcc, marshals numpy arrays and loops over (batch, head) or (sequence, head).
+
+Pins (checks against facts that do not come from this code) live in
+``tests/oracle_pins.py``: brute force on tiny shapes, closed forms, invariants
+and finite differences for every function here; none is left unpinned.
 """
 from __future__ import annotations
 

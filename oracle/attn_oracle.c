@@ -1,5 +1,7 @@
 /*
- * Plain fp64 CPU oracle for exact scaled dot-product attention (forward).
+ * Plain fp64 CPU oracle for exact scaled dot-product attention (forward and
+ * backward: dense, key bands and column intervals; packed batches are composed
+ * per sequence by oracle/__init__.py).
  *
  * TEST INFRASTRUCTURE ONLY.  Nothing in the product path may link, load or call
  * this file; it exists so that tests, the smoke check and the CPU-baseline leg of
