@@ -394,8 +394,22 @@ def pin_colmask_two_intervals(attn_rows_colmask):
     assert np.all(o[8:] == 0.0) and np.all(lse[8:] == -np.inf)
 
 
+def pin_colmask_golden(attn_rows_colmask):
+    """Hand-derived closed forms under column intervals stored under tests/golden/."""
+    with open(os.path.join(os.path.dirname(GOLDEN), "colmask_closed_forms.json")) as f:
+        cases = json.load(f)["cases"]
+    for c in cases:
+        q, k, v = (np.array(c[x], dtype=np.float64) for x in ("q", "k", "v"))
+        cols = np.array(c["cols"], dtype=np.int64)
+        o, lse = attn_rows_colmask(q, np.arange(q.shape[0], dtype=np.int64), k, v, c["scale"], c["causal"],
+                                   cols)
+        want_lse = np.array([float(x) for x in c["lse"]])
+        np.testing.assert_allclose(o, np.array(c["o"]), rtol=1e-13, atol=1e-13, err_msg=c["name"])
+        np.testing.assert_allclose(lse, want_lse, rtol=1e-13, atol=1e-13, err_msg=c["name"])
+
+
 COLMASK_PINS = [pin_colmask_band, pin_colmask_documents, pin_colmask_empty_intervals,
-                pin_colmask_two_intervals]
+                pin_colmask_two_intervals, pin_colmask_golden]
 
 
 def pin_bwd_colmask_finite_differences(attn_bwd_colmask_head, attn_rows_colmask):
