@@ -614,8 +614,20 @@ def pin_bwd_dv_is_pt_dout(bwd, fwd):
         np.testing.assert_allclose(dv, p.T @ dout, rtol=1e-12, atol=1e-12)
 
 
+def pin_bwd_golden(bwd, fwd):
+    """Hand-derived gradients stored under tests/golden/."""
+    with open(os.path.join(os.path.dirname(GOLDEN), "bwd_closed_forms.json")) as f:
+        cases = json.load(f)["cases"]
+    for c in cases:
+        q, k, v, g = (np.array(c[x], dtype=np.float64) for x in ("q", "k", "v", "dout"))
+        dq, dk, dv = bwd(q, k, v, g, c["scale"], *c["window"])
+        for name, got in (("dq", dq), ("dk", dk), ("dv", dv)):
+            np.testing.assert_allclose(got, np.array(c[name]), rtol=1e-13, atol=1e-13,
+                                       err_msg=f"{c['name']} {name}")
+
+
 BWD_PINS = [pin_bwd_finite_differences, pin_bwd_single_key, pin_bwd_sums,
-            pin_bwd_linear_in_cotangent, pin_bwd_dv_is_pt_dout]
+            pin_bwd_linear_in_cotangent, pin_bwd_dv_is_pt_dout, pin_bwd_golden]
 
 
 # ---------------------------------------------------------------------------
