@@ -141,7 +141,8 @@ int attn_fwd_window(const void *q, const void *k, const void *v, void *o, float 
  * rows of a CTA and masks element-wise only in blocks whose intervals meet a
  * warp's 32 rows.  Errors as attn_fwd_gqa, plus ATTN_ERR_INVALID_ARG for a NULL
  * or misaligned mask or workspace, a workspace that is too small or overlaps
- * another argument, or Hm not in {1, H}.
+ * another argument, or Hm not in {1, H}, and ATTN_ERR_UNSUPPORTED for more than
+ * 65536 key blocks of 128 (8M keys: the kernel keeps one bit per key block).
  */
 size_t attn_colmask_workspace_size(int B, int Hm, int Nk);
 int attn_fwd_colmask(const void *q, const void *k, const void *v, void *o, float *lse, int B,
