@@ -146,6 +146,11 @@ def test_colmask_validation():
     assert call(sz=sizes[:5] + (96,) + sizes[6:]) == 2
     # nothing to compute: a no-op even with null pointers
     assert C(None, None, None, None, None, 0, 4, 2, 8, 8, 64, 0.1, 0, None, 1, None, 0, None) == 0
+    # more than 65536 key blocks of 128: unsupported (fake pointers far apart)
+    T = 1 << 40
+    nk = 65536 * 128 + 1
+    big = binding.attn_colmask_workspace_size(1, 1, nk)
+    assert C(T, 2 * T, 3 * T, 4 * T, None, 1, 1, 1, 8, nk, 64, 0.1, 0, 5 * T, 1, 6 * T, big, None) == 2
 
 
 def test_varlen_validation():
