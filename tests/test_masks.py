@@ -81,3 +81,38 @@ def test_document_workload_flops_closed_form():
     assert w.flops == 4.0 * w.d * w.H * pairs
     assert all(sum(w.doc_lengths(b)) == w.Nk for b in range(w.B))
     assert all(256 <= n <= 4096 for b in range(w.B) for n in w.doc_lengths(b)[:-1])
+
+
+def test_block_summary_rules_are_sound():
+    """The block summaries the kernels use decide two things per (128-key block,
+    row range): 'every key hides every row' (max lo <= r0 and min hi >= r1 for
+    one interval) lets a block be skipped, and 'no key's interval meets the
+    rows' (max hi <= r0 or min lo >= r1 for both intervals) lets a warp skip
+    element-wise masking.  Both must only fire when brute force agrees."""
+    rng = np.random.default_rng(7)
+    fired = {"hide_all": 0, "no_touch": 0}
+    for trial in range(40):
+        nq, nk = 300, 256
+        m = masks.random_intervals(100 + trial, 1, 1, nq, nk)[0, 0].astype(np.int64)
+        if trial % 3 == 0:  # documents too, where the rules fire often
+            m = masks.documents([[70, 50, 90, 46]], nk)[0, 0].astype(np.int64)
+        vis = dense_visible(m, nq, False)
+        for blk in range(nk // 128):
+            c = m[blk * 128:(blk + 1) * 128]
+            e1, e2 = c[:, 0] >= c[:, 1], c[:, 2] >= c[:, 3]
+            big, small = np.iinfo(np.int64).max, np.iinfo(np.int64).min
+            lo1, hi1 = np.where(e1, big, c[:, 0]), np.where(e1, small, c[:, 1])
+            lo2, hi2 = np.where(e2, big, c[:, 2]), np.where(e2, small, c[:, 3])
+            for _ in range(10):
+                r0 = int(rng.integers(0, nq - 1))
+                r1 = int(rng.integers(r0 + 1, min(nq, r0 + 64) + 1))
+                block = vis[r0:r1, blk * 128:(blk + 1) * 128]
+                hide_all = (lo1.max() <= r0 and hi1.min() >= r1) or (lo2.max() <= r0 and hi2.min() >= r1)
+                if hide_all:
+                    assert not block.any()
+                    fired["hide_all"] += 1
+                touch = not (hi1.max() <= r0 or lo1.min() >= r1) or not (hi2.max() <= r0 or lo2.min() >= r1)
+                if not touch:
+                    assert block.all()
+                    fired["no_touch"] += 1
+    assert fired["hide_all"] > 0 and fired["no_touch"] > 0, fired
