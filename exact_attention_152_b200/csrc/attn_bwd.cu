@@ -1214,18 +1214,58 @@ int bwd_varlen_impl(const void* q, const void* k, const void* v, const void* o, 
 constexpr size_t kStaticScratchBytes = size_t(96) << 20;  // 96 MiB per device
 __device__ __align__(256) unsigned char g_bwd_scratch[kStaticScratchBytes];
 
-// Device address of g_bwd_scratch on the current device, looked up once per device.
+// Device address of g_bwd_scratch in the current context.  The address
+// belongs to the copy of this module loaded into one context: a new context on
+// the same device (after cudaDeviceReset, or one the caller made current) loads
+// the module again, possibly elsewhere.  So the address is cached per device
+// together with the unique ID of the context it was looked up in, and looked up
+// again (cudaGetSymbolAddress: a lookup, no allocation) whenever that ID
+// changes or cannot be read.
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+using CtxGetIdFn = CUresult (*)(CUcontext, unsigned long long*);
+
+bool current_context_id(unsigned long long* id) {
+  static CtxGetCurrentFn get_current = nullptr;
+  static CtxGetIdFn get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_current = reinterpret_cast<CtxGetCurrentFn>(p);
+    p = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<CtxGetIdFn>(p);
+  });
+  CUcontext ctx = nullptr;
+  if (!get_current || !get_id || get_current(&ctx) != CUDA_SUCCESS || ctx == nullptr) return false;
+  return get_id(ctx, id) == CUDA_SUCCESS;
+}
+
 int static_scratch(void** ptr) {
-  static std::once_flag once[kMaxDeviceCount];
+  static std::mutex mu;
   static void* addr[kMaxDeviceCount];
-  static cudaError_t err[kMaxDeviceCount];
+  static unsigned long long ctx_id[kMaxDeviceCount];
+  static bool cached[kMaxDeviceCount];
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
   if (dev < 0 || dev >= kMaxDeviceCount) return ATTN_ERR_UNSUPPORTED;
-  std::call_once(once[dev], [&] { err[dev] = cudaGetSymbolAddress(&addr[dev], g_bwd_scratch); });
-  if (err[dev] != cudaSuccess) return cuda_fail(err[dev], "cudaGetSymbolAddress");
-  *ptr = addr[dev];
+  std::lock_guard<std::mutex> lk(mu);
+  unsigned long long id = 0;
+  if (current_context_id(&id) && cached[dev] && ctx_id[dev] == id) {
+    *ptr = addr[dev];
+    return ATTN_OK;
+  }
+  void* a = nullptr;
+  e = cudaGetSymbolAddress(&a, g_bwd_scratch);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress");
+  addr[dev] = a;
+  // the lookup made the device's context current if none was: read its ID now
+  cached[dev] = current_context_id(&ctx_id[dev]);
+  *ptr = a;
   return ATTN_OK;
 }
 

@@ -27,26 +27,32 @@
 //    memory stages filled by TMA.  Q, K and V are read through 3-D tensor maps
 //    [B*H, N, d] so out-of-range rows of one head read as zeros, never as the
 //    next head's data.
-//  * 20 warps.  Warps 0-15 do softmax, correction and epilogue: tile t uses
-//    warps 8t..8t+7; warp (t, h, q) owns TMEM lanes 32q..32q+31 (its 32 query
-//    rows) and the key columns [64h, 64h+64) of each S tile, and the output
-//    columns [h*d/2, (h+1)*d/2).  The two warps of a row pair swap their partial
-//    row maxima through shared memory.  Warp 16: TMA producer.  Warp 17: TMEM
-//    allocation and the single MMA-issuing thread.  Warps 18-19 idle (they
-//    complete the fifth warpgroup for the setmaxnreg split 104 / 40).
+//  * 12 warps.  Warps 0-7 do softmax, correction and epilogue, one thread per
+//    query row: tile t uses warpgroup t (warps 4t..4t+3), and warp (t, q) owns
+//    TMEM lanes 32q..32q+31 (its 32 rows) with all 128 key columns of each S
+//    tile and all d output columns.  A row's scores sit in one thread's
+//    registers, so its max needs no exchange between threads.  Warp 8: TMA
+//    producer.  Warp 9: TMEM allocation and the single MMA-issuing thread.
+//    Warps 10-11 idle (they complete the third warpgroup for the setmaxnreg
+//    split 232 / 40).
 //  * Tensor Memory (512 columns): S0 [0,128), S1 [128,256), O0 and O1 after
-//    column 256.  P (BF16 pairs) overwrites the first half of each warp's part
-//    of S and is the A operand of O += P V straight from TMEM, so P never
-//    touches shared memory.
+//    column 256.  P (BF16 pairs; E4M3 quadruples) overwrites the first columns
+//    of its tile's S and is the A operand of O += P V straight from TMEM, so P
+//    never touches shared memory.
 //  * The MMA thread issues, per KV tile j:  O0 += P0 V_{j-1};  S0 = Q0 K_j^T;
-//    O1 += P1 V_{j-1};  S1 = Q1 K_j^T.  Each O += P V is issued in two chunks,
-//    each as soon as the softmax warps have stored that chunk of P.  The
+//    O1 += P1 V_{j-1};  S1 = Q1 K_j^T.  Each O += P V is issued in four
+//    chunks of 32 keys, each as soon as the softmax warps have stored that
+//    chunk of P, so only the last chunk sits between a tile's softmax and its
+//    next S.  The
 //    commit that announces S_t(j) also covers O_t += P_t V_{j-1}, so when a
 //    softmax warp sees S_t(j) its O_t is final up to tile j-1 and it can
 //    rescale O_t in place without another wait.
 //  * MMAs are issued from fully unrolled code with descriptor offsets as
 //    immediates: the tensor core queues about one MMA ahead, so every cycle
 //    the issuing thread spends between MMAs is a cycle the tensor core idles.
+//    For the same reason the issuer looks at the barrier of its next MMA group
+//    (non-blocking) before issuing the current one, and K_j / V_{j-1} arrive
+//    on a single barrier per step.
 //  * Masks: the key tail, a key band i - wl <= j <= i + wr (causal, sliding
 //    windows), and column intervals (attn_fwd_colmask: each key hidden from up
 //    to two query-row intervals).  KV tiles outside the band are never
@@ -80,15 +86,21 @@ namespace eab {
 constexpr int kBlockM = 128;  // query rows per tile  (= TMEM lanes)
 constexpr int kBlockN = 128;  // keys per KV tile
 constexpr int kRowsPerCta = 2 * kBlockM;
-// 5 warpgroups: 4 softmax warpgroups (tile t, key half h -> warps 8t+4h .. 8t+4h+3)
-// and one for the TMA producer (warp 16), the MMA issuer (warp 17) and two idle
-// warps that complete the group for the register split.
-constexpr int kWarpLoad = 16;
-constexpr int kWarpMma = 17;
-constexpr int kNumThreads = 640;
-// setmaxnreg split of the 640 x 96 launch budget: 512 x 104 + 128 x 40 <= 61440.
-constexpr int kSoftmaxRegs = 104;
+// 3 warpgroups: one softmax warpgroup per query tile (warps 4t .. 4t+3) and one
+// for the TMA producer (warp 8), the MMA issuer (warp 9) and two idle warps
+// that complete the group for the register split.
+constexpr int kWarpLoad = 8;
+constexpr int kWarpMma = 9;
+constexpr int kNumThreads = 384;
+// setmaxnreg split of the 384 x 168 launch budget: 256 x 232 + 128 x 40 = 64512.
+// The host refuses to launch a build whose register count at launch is lower
+// (setmaxnreg.inc would wait for registers that are not there).
+constexpr int kLaunchRegs = 168;
+constexpr int kSoftmaxRegs = 232;
 constexpr int kProducerRegs = 40;
+static_assert(2 * 128 * kSoftmaxRegs + 128 * kProducerRegs <= kNumThreads * kLaunchRegs,
+              "register split exceeds the launch budget");
+constexpr int kPChunks = 4;  // P published in chunks of 32 keys
 constexpr uint32_t kTmemCols = 512;
 constexpr uint64_t kWaitTimeoutNs = 2000000000ull;  // 2 s per pipeline wait
 constexpr float kDefaultThreshold = 8.0f;           // powers of two
@@ -141,13 +153,10 @@ struct Cfg {
   static constexpr int kOTileBytes = kBlockM * D * 2;
   static constexpr int kOffO = F8 ? kOffKV + kStages * kTileBytes : kOffQ;
   static constexpr int kOffBar = F8 ? kOffO + 2 * kOTileBytes : kOffKV + kStages * kTileBytes;
-  static constexpr int kNumBars = 2 + 2 * kStages + 2 + 4 + 2 + 1;
+  static constexpr int kNumKvSteps = 4;  // step barriers, used round robin
+  static constexpr int kNumBars = 2 + kStages + kNumKvSteps + 2 + 2 * kPChunks + 2 + 1;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
-  // row-max / row-sum exchange between the two key halves of a row:
-  // float [tile 2][half 2][parity 2][row 128]
-  static constexpr int kOffXch = (kOffMisc + 16 + 15) / 16 * 16;
-  static constexpr int kXchBytes = 2 * 2 * 2 * kBlockM * 4;
-  static constexpr int kOffSeq = kOffXch + kXchBytes;  // this CTA's SeqView
+  static constexpr int kOffSeq = (kOffMisc + 16 + 15) / 16 * 16;  // this CTA's SeqView
   static constexpr int kSeqBytes = 64;
   // column-interval mask: one bit per 128-key block, set when the block is
   // visited (kMaxMaskBlocks blocks = 8M keys)
@@ -264,18 +273,26 @@ struct Smem {
   __device__ __forceinline__ uint32_t kv(int s) const { return sbase + Cfg<D, F8>::kOffKV + s * Cfg<D, F8>::kTileBytes; }
   __device__ __forceinline__ uint32_t bar(int i) const { return sbase + Cfg<D, F8>::kOffBar + 8 * i; }
   __device__ __forceinline__ uint32_t q_full(int t) const { return bar(t); }
-  __device__ __forceinline__ uint32_t kv_full(int s) const { return bar(2 + s); }
-  __device__ __forceinline__ uint32_t kv_empty(int s) const { return bar(2 + Cfg<D, F8>::kStages + s); }
-  __device__ __forceinline__ uint32_t s_full(int t) const { return bar(2 + 2 * Cfg<D, F8>::kStages + t); }
-  // chunk k of P_t (keys [32k, 32k+32) and [64+32k, 96+32k)) written to TMEM by
-  // all 8 warps of the tile (chunk 0 also marks O_t as rescaled)
-  __device__ __forceinline__ uint32_t p_full(int t, int k) const {
-    return bar(4 + 2 * Cfg<D, F8>::kStages + 2 * t + k);
+  // K/V slot s free again (its last reader, an MMA, has completed)
+  __device__ __forceinline__ uint32_t kv_empty(int s) const { return bar(2 + s); }
+  // MMA step j (0 .. n_kv): V(j-1) and K(j) both resident.  One barrier per
+  // step instead of one per tile halves the MMA thread's waits on data.
+  __device__ __forceinline__ uint32_t kvp(int j) const {
+    return bar(2 + Cfg<D, F8>::kStages + (j % Cfg<D, F8>::kNumKvSteps));
   }
-  __device__ __forceinline__ uint32_t o_full(int t) const { return bar(8 + 2 * Cfg<D, F8>::kStages + t); }
-  __device__ __forceinline__ uint32_t mma_done() const { return bar(10 + 2 * Cfg<D, F8>::kStages); }
-  __device__ __forceinline__ float* xch(int t, int h, int par) const {
-    return reinterpret_cast<float*>(base + Cfg<D, F8>::kOffXch) + ((t * 2 + h) * 2 + par) * kBlockM;
+  __device__ __forceinline__ uint32_t s_full(int t) const {
+    return bar(2 + Cfg<D, F8>::kStages + Cfg<D, F8>::kNumKvSteps + t);
+  }
+  // chunk k of P_t (keys [32k, 32k+32)) written to TMEM by all 4 warps of the
+  // tile (chunk 0 also marks O_t as rescaled)
+  __device__ __forceinline__ uint32_t p_full(int t, int k) const {
+    return bar(4 + Cfg<D, F8>::kStages + Cfg<D, F8>::kNumKvSteps + kPChunks * t + k);
+  }
+  __device__ __forceinline__ uint32_t o_full(int t) const {
+    return bar(4 + Cfg<D, F8>::kStages + Cfg<D, F8>::kNumKvSteps + 2 * kPChunks + t);
+  }
+  __device__ __forceinline__ uint32_t mma_done() const {
+    return bar(6 + Cfg<D, F8>::kStages + Cfg<D, F8>::kNumKvSteps + 2 * kPChunks);
   }
   __device__ __forceinline__ uint32_t* tmem_slot() const {
     return reinterpret_cast<uint32_t*>(base + Cfg<D, F8>::kOffMisc);
@@ -314,34 +331,55 @@ __device__ __forceinline__ void producer_role(const Smem<D, F8>& sm, const CUten
       tma_load_rows(sm.q(t) + b * C::kBoxBytes, tm_q, b * C::kBoxCols, sv.q0 + qb * kRowsPerCta + t * kBlockM,
                     sv.head_q, sv.packed, sm.q_full(t));
   };
-  auto load_kv = [&](const CUtensorMap* tm, int j) -> bool {
-    const uint32_t slot = it % C::kStages;
+  auto wait_slot = [&](uint32_t& slot) -> bool {
+    slot = it % C::kStages;
     const uint32_t phase = (it / C::kStages) & 1u;
-    if (!mbar_wait(sm.kv_empty(slot), phase ^ 1u, timeout)) return false;
-    mbar_arrive_expect_tx(sm.kv_full(slot), C::kTileBytes);
+    ++it;
+    return mbar_wait(sm.kv_empty(slot), phase ^ 1u, timeout);
+  };
+  auto issue_kv = [&](const CUtensorMap* tm, int j, uint32_t slot, uint32_t pbar) {
 #pragma unroll
     for (int b = 0; b < C::kBoxes; ++b)
       tma_load_rows(sm.kv(slot) + b * C::kBoxBytes, tm, b * C::kBoxCols, sv.k0 + j * kBlockN, sv.head_kv,
-                    sv.packed, sm.kv_full(slot));
-    ++it;
-    return true;
+                    sv.packed, pbar);
   };
 
   const uint32_t* vis = sm.vis();
   int blk = next_block<MASK>(vis, sv.j_lo - 1);
+  uint32_t s_k = 0, s_v = 0;
   load_q(0);
-  bool ok = load_kv(tm_k, blk);
+  bool ok = wait_slot(s_k);
+  if (ok) {
+    mbar_arrive_expect_tx(sm.kvp(0), C::kTileBytes);
+    issue_kv(tm_k, blk, s_k, sm.kvp(0));
+  }
   load_q(1);
-  ok = ok && load_kv(tm_v, blk);
+  int prev = blk;
+  int steps = ok ? 1 : 0;
   for (int j = 1; ok && j < sv.n_kv; ++j) {
     blk = next_block<MASK>(vis, blk);
-    ok = load_kv(tm_k, blk) && load_kv(tm_v, blk);
+    // V(j-1) and K(j) complete one barrier together
+    ok = wait_slot(s_v) && wait_slot(s_k);
+    if (!ok) break;
+    mbar_arrive_expect_tx(sm.kvp(j), 2 * C::kTileBytes);
+    issue_kv(tm_v, prev, s_v, sm.kvp(j));
+    issue_kv(tm_k, blk, s_k, sm.kvp(j));
+    prev = blk;
+    ++steps;
+  }
+  if (ok) {
+    ok = wait_slot(s_v);
+    if (ok) {
+      mbar_arrive_expect_tx(sm.kvp(sv.n_kv), C::kTileBytes);
+      issue_kv(tm_v, prev, s_v, sm.kvp(sv.n_kv));
+      ++steps;
+    }
   }
 
-  // Never leave the CTA with a copy in flight: wait for the latest fill of
-  // every slot and for both Q tiles (immediate on the normal path).
-  const uint32_t first = it > (uint32_t)C::kStages ? it - C::kStages : 0u;
-  for (uint32_t i = first; i < it; ++i) mbar_wait(sm.kv_full(i % C::kStages), (i / C::kStages) & 1u, timeout);
+  // Never leave the CTA with a copy in flight: wait for the latest steps
+  // (immediate on the normal path).
+  for (int i = steps > C::kNumKvSteps ? steps - C::kNumKvSteps : 0; i < steps; ++i)
+    mbar_wait(sm.kvp(i), (i / C::kNumKvSteps) & 1, timeout);
   mbar_wait(sm.q_full(0), 0, timeout);
   mbar_wait(sm.q_full(1), 0, timeout);
   if (!ok) atomicOr(&g_status, kStatusTimeout);
@@ -365,38 +403,38 @@ struct MmaUnroll {
       MmaUnroll<D, F8, KK + 1>::s(d, a_lo, a_hi, b_lo, b_hi, idesc);
     }
   }
-  // O += P V for P chunk CH.  BF16: K steps {2CH, 2CH+1} (keys [32CH, 32CH+32))
-  // and {4+2CH, 5+2CH} (keys [64+32CH, 96+32CH)); P of keys [64h, 64h+64) sits
-  // in TMEM columns [64h, 64h+32) (two per column); V rows of 16 keys = 2048
-  // bytes.  E4M3: K steps CH (keys [32CH, 32CH+32)) and 2+CH (keys
-  // [64+32CH, 96+32CH)); P of keys [64h, 64h+64) in columns [64h, 64h+16)
-  // (four per column); V rows of 32 keys = 4096 bytes.  KK counts the steps
-  // of the chunk.
+  // O += P V for P chunk CH (keys [32CH, 32CH+32)).  P of key pair / quad c
+  // sits in TMEM column c of the tile (BF16: two keys per column, E4M3: four),
+  // so K step s reads columns [8s, 8s+8) either way.  BF16: 16 keys per step,
+  // steps 2CH and 2CH+1, V rows of 16 keys = 2048 bytes per 64-column box.
+  // E4M3: 32 keys per step, step CH, V rows of 32 keys = 4096 bytes.  KK
+  // counts the steps of the chunk.
   template <int CH>
   __device__ __forceinline__ static void o(uint32_t d, uint32_t a_tmem, uint32_t b_lo, uint32_t b_hi,
                                            uint32_t idesc, uint32_t acc) {
-    if constexpr (F8) {
-      if constexpr (KK < 2) {
-        constexpr int step = 2 * KK + CH;  // K step among 0..3, 32 keys each
-        constexpr uint32_t a_off = (step >> 1) * 64 + (step & 1) * 8;
-        constexpr uint32_t b_off = (step * 4096) >> 4;
+    constexpr int kSteps = F8 ? 1 : 2;
+    if constexpr (KK < kSteps) {
+      constexpr int step = CH * kSteps + KK;
+      constexpr uint32_t a_off = step * 8;
+      constexpr uint32_t b_off = (step * (F8 ? 4096 : 2048)) >> 4;
+      if constexpr (F8)
         mma_ts_imm_f8<a_off, b_off>(d, a_tmem, b_lo, b_hi, idesc, (CH == 0 && KK == 0) ? acc : 1u);
-        MmaUnroll<D, F8, KK + 1>::template o<CH>(d, a_tmem, b_lo, b_hi, idesc, acc);
-      }
-    } else if constexpr (KK < 4) {
-      constexpr int step = (KK >> 1) * 4 + 2 * CH + (KK & 1);  // K step among 0..7
-      constexpr uint32_t a_off = (step >> 2) * 64 + (step & 3) * 8;
-      constexpr uint32_t b_off = (step * 2048) >> 4;
-      mma_ts_imm<a_off, b_off>(d, a_tmem, b_lo, b_hi, idesc, (CH == 0 && KK == 0) ? acc : 1u);
+      else
+        mma_ts_imm<a_off, b_off>(d, a_tmem, b_lo, b_hi, idesc, (CH == 0 && KK == 0) ? acc : 1u);
       MmaUnroll<D, F8, KK + 1>::template o<CH>(d, a_tmem, b_lo, b_hi, idesc, acc);
     }
   }
 };
 
 // ---------------------------------------------------------------------------
-// MMA issuer: one thread.  Per KV tile j it waits for V_{j-1} and K_j first
-// (normally long resident), so the only wait between a tile's P becoming
-// ready and its O += P V_{j-1}; S = Q K_j^T block is the P barrier itself.
+// MMA issuer: one thread.  The tensor core queues only about one MMA ahead of
+// the issuing thread, and a look at an mbarrier costs this thread ~50 cycles
+// alone and over 100 while TMA and the MMAs keep shared memory busy, so every
+// blocking look between two MMA groups idles the tensor core.  The thread
+// therefore starts a non-blocking look (test_wait) at the barrier the NEXT
+// group needs before it issues the current group, and only falls back to a
+// bounded blocking wait if that look failed.  Data for a step, V_{j-1} and
+// K_j, arrives on one barrier per step.
 // ---------------------------------------------------------------------------
 template <int D, bool F8>
 __device__ __forceinline__ void mma_role(const Smem<D, F8>& sm, uint32_t tmem, int n_kv,
@@ -408,12 +446,11 @@ __device__ __forceinline__ void mma_role(const Smem<D, F8>& sm, uint32_t tmem, i
                                   : idesc_bf16_f32(kBlockM, D, false, true);
   uint32_t it = 0;  // position in the K0, V0, K1, V1, ... ring order
 
-  auto wait_kv = [&](uint32_t& slot) -> bool {
+  auto next_slot = [&](uint32_t& slot) {
     slot = it % C::kStages;
-    const uint32_t phase = (it / C::kStages) & 1u;
     ++it;
-    return mbar_wait(sm.kv_full(slot), phase, timeout);
   };
+  auto wait_step = [&](int j) -> bool { return mbar_wait(sm.kvp(j), (j / C::kNumKvSteps) & 1, timeout); };
   // descriptors as 32-bit halves; stage and tile offsets go into the low word
   const uint64_t dq = sdesc_sw128(sm.q(0), 16, 1024);
   const uint64_t dk = sdesc_sw128(sm.kv(0), 16, 1024);
@@ -426,55 +463,80 @@ __device__ __forceinline__ void mma_role(const Smem<D, F8>& sm, uint32_t tmem, i
     MmaUnroll<D, F8, 0>::s(tmem + t * kBlockM, q_lo + t * kTileStep, q_hi, k_lo + slot * kTileStep,
                        k_hi, idesc_s);
   };
-  // O_t += P_t V in two chunks, each issued as soon as the softmax warps have
-  // stored it
-  auto mma_o = [&](int t, uint32_t slot, bool acc, uint32_t par) -> bool {
+  // settle a look taken earlier: block only if it failed
+  auto settle = [&](bool seen, uint32_t bar, uint32_t par) -> bool {
+    return seen || mbar_wait(bar, par, timeout);
+  };
+  // O_t += P_t V in four chunks; the next chunk's barrier is looked at before
+  // the current chunk is issued.  `pre` is the look at chunk 0 taken earlier
+  // (while the previous S group was issued).
+  auto mma_o = [&](int t, uint32_t slot, bool acc, uint32_t par, bool pre) -> bool {
     const uint32_t d = tmem + C::kTmemO + t * D, a = tmem + t * kBlockM;
     const uint32_t b_lo = v_lo + slot * kTileStep;
-    if (!mbar_wait(sm.p_full(t, 0), par, timeout)) return false;
+    if (!settle(pre, sm.p_full(t, 0), par)) return false;
     tc_fence_after();
+    bool nx = mbar_test(sm.p_full(t, 1), par);
     MmaUnroll<D, F8, 0>::template o<0>(d, a, b_lo, v_hi, idesc_o, acc ? 1u : 0u);
-    if (!mbar_wait(sm.p_full(t, 1), par, timeout)) return false;
+    if (!settle(nx, sm.p_full(t, 1), par)) return false;
     tc_fence_after();
+    nx = mbar_test(sm.p_full(t, 2), par);
     MmaUnroll<D, F8, 0>::template o<1>(d, a, b_lo, v_hi, idesc_o, 1u);
+    if (!settle(nx, sm.p_full(t, 2), par)) return false;
+    tc_fence_after();
+    nx = mbar_test(sm.p_full(t, 3), par);
+    MmaUnroll<D, F8, 0>::template o<2>(d, a, b_lo, v_hi, idesc_o, 1u);
+    if (!settle(nx, sm.p_full(t, 3), par)) return false;
+    tc_fence_after();
+    MmaUnroll<D, F8, 0>::template o<3>(d, a, b_lo, v_hi, idesc_o, 1u);
     return true;
   };
 
   uint32_t sK = 0, sV = 0;
-  bool ok = mbar_wait(sm.q_full(0), 0, timeout) && wait_kv(sK);
+  next_slot(sK);
+  bool ok = mbar_wait(sm.q_full(0), 0, timeout) && wait_step(0);
   if (ok) {
     tc_fence_after();
     mma_s(0, sK);
     tc_commit(sm.s_full(0));
     ok = mbar_wait(sm.q_full(1), 0, timeout);
   }
+  bool pk = false, pp = false;
   if (ok) {
     tc_fence_after();
+    if (n_kv > 1) pk = mbar_test(sm.kvp(1), 0);
+    pp = mbar_test(sm.p_full(0, 0), 0);
     mma_s(1, sK);
     tc_commit(sm.s_full(1));
     tc_commit(sm.kv_empty(sK));
   }
   for (int j = 1; ok && j < n_kv; ++j) {
     const uint32_t par = (j - 1) & 1;
-    ok = wait_kv(sV) && wait_kv(sK);
+    next_slot(sV);
+    next_slot(sK);
+    ok = settle(pk, sm.kvp(j), (j / C::kNumKvSteps) & 1);
     if (!ok) break;
-    ok = mma_o(0, sV, j > 1, par);
+    ok = mma_o(0, sV, j > 1, par, pp);
     if (!ok) break;
+    pp = mbar_test(sm.p_full(1, 0), par);
     mma_s(0, sK);
     tc_commit(sm.s_full(0));
-    ok = mma_o(1, sV, j > 1, par);
+    ok = mma_o(1, sV, j > 1, par, pp);
     if (!ok) break;
     tc_commit(sm.kv_empty(sV));
+    // the next step's K/V and chunk 0 of P0, looked at while S1 is issued
+    pk = mbar_test(sm.kvp(j + 1), ((j + 1) / C::kNumKvSteps) & 1);
+    pp = mbar_test(sm.p_full(0, 0), j & 1);
     mma_s(1, sK);
     tc_commit(sm.s_full(1));
     tc_commit(sm.kv_empty(sK));
   }
   if (ok) {
     const uint32_t par = (n_kv - 1) & 1;
-    ok = wait_kv(sV) && mma_o(0, sV, n_kv > 1, par);
+    next_slot(sV);
+    ok = settle(n_kv > 1 ? pk : false, sm.kvp(n_kv), (n_kv / C::kNumKvSteps) & 1) && mma_o(0, sV, n_kv > 1, par, pp);
     if (ok) {
       tc_commit(sm.o_full(0));
-      ok = mma_o(1, sV, n_kv > 1, par);
+      ok = mma_o(1, sV, n_kv > 1, par, false);
     }
     if (ok) {
       tc_commit(sm.o_full(1));
@@ -488,37 +550,29 @@ __device__ __forceinline__ void mma_role(const Smem<D, F8>& sm, uint32_t tmem, i
 }
 
 // ---------------------------------------------------------------------------
-// Softmax + correction + epilogue.  Tile t has 8 warps: warp (t, h, q) owns
-// TMEM lanes 32q..32q+31 (rows) and key columns [64h, 64h+64) of every S tile,
-// and output columns [h*d/2, (h+1)*d/2).  The two warps of a row pair (same t,
-// q) swap their partial row maxima (and at the end their partial sums) through
-// shared memory and a 64-thread named barrier that both reach unconditionally
-// every iteration; a failed wait travels through the same exchange as NaN, so
-// a pair always leaves its loop together.
+// Softmax + correction + epilogue, one thread per query row.  Tile t has the
+// four warps of warpgroup t: warp (t, q) owns TMEM lanes 32q..32q+31 (its 32
+// rows), all 128 key columns of every S tile and all d output columns.  A
+// warp waits only on pipeline mbarriers (bounded), never on another warp, so a
+// failed wait simply ends its loop; the MMA thread then gives up on the P
+// barrier that warp no longer signals.
 // ---------------------------------------------------------------------------
-__device__ __forceinline__ void pair_sync(int t, int q) {
-  asm volatile("bar.sync %0, 64;" ::"r"(1 + t * 4 + q) : "memory");
-}
-
 template <int D, int MASK, int POLY16, bool F8>
 __device__ __forceinline__ void softmax_role(const Smem<D, F8>& sm, uint32_t tmem,
                                              const CUtensorMap* tm_o, const FwdParams& prm,
                                              const SeqView& sv, int qb) {
   using C = Cfg<D, F8>;
-  constexpr int kCols = kBlockN / 2;  // key columns per warp
-  constexpr int kOCols = D / 2;       // output columns per warp
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int t = warp >> 3;        // query tile of this CTA
-  const int h = (warp >> 2) & 1;  // key half / output-column half
+  const int t = warp >> 2;        // query tile of this CTA
   const int q4 = warp & 3;        // TMEM lane quarter this warp may access
-  const int r = q4 * 32 + lane;
+  const int r = q4 * 32 + lane;   // row within the tile (= TMEM lane)
   const int tile_row0 = qb * kRowsPerCta + t * kBlockM;
   const int row = tile_row0 + r;
   const int rw0 = tile_row0 + q4 * 32;  // first row of this warp
   const int Nk = sv.Nk;
   const uint32_t lane_off = static_cast<uint32_t>(q4 * 32) << 16;
-  const uint32_t tS = tmem + lane_off + t * kBlockM + h * kCols;
-  const uint32_t tO = tmem + lane_off + C::kTmemO + t * D + h * kOCols;
+  const uint32_t tS = tmem + lane_off + t * kBlockM;
+  const uint32_t tO = tmem + lane_off + C::kTmemO + t * D;
   const uint64_t timeout = prm.timeout_ns;
 
   // scale <= 0: apply it first, then run with an effective scale of 1 (the
@@ -526,103 +580,94 @@ __device__ __forceinline__ void softmax_role(const Smem<D, F8>& sm, uint32_t tme
   const bool prescale = !(prm.scale_log2 > 0.0f);
   const float sl = prescale ? 1.0f : prm.scale_log2;
   float m_run = -INFINITY;  // running reference max, log2 units of scaled scores
-  float l_run = 0.0f;       // this half's running sum of 2^(score - m_run)
+  float l_run = 0.0f;       // running sum of 2^(score - m_run)
   bool ok = true;
 
   int blk = sv.j_lo - 1;
   for (int j = 0; j < sv.n_kv; ++j) {
     blk = next_block<MASK>(sm.vis(), blk);
-    const int kv0 = blk * kBlockN + h * kCols;
-    // mask needed: key tail, a band edge crossing this warp's 64 x 32 block, or
-    // a column interval meeting the warp's rows
-    bool masked = kv0 + kCols > Nk ||
-                  (MASK != kMaskNone && (kv0 + kCols - 1 - rw0 > prm.wr || rw0 + 31 - kv0 > prm.wl));
+    const int kv0 = blk * kBlockN;
+    // mask needed: key tail, a band edge crossing this warp's 32 x 128 block,
+    // or a column interval meeting the warp's rows
+    bool masked = kv0 + kBlockN > Nk ||
+                  (MASK != kMaskNone && (kv0 + kBlockN - 1 - rw0 > prm.wr || rw0 + 31 - kv0 > prm.wl));
     // column-interval mask: bit c of hid[k] = key kv0 + 32k + c hidden from this row
-    uint32_t hid[2] = {0u, 0u};
+    uint32_t hid[4] = {0u, 0u, 0u, 0u};
     if constexpr (MASK == kMaskCols) {
       if (cols_touch(prm, sv.mrow, blk, rw0, rw0 + 32)) {
         masked = true;
-        // lane l reads keys kv0 + l and kv0 + 32 + l (coalesced) and turns each
-        // into the set of the warp's 32 rows it is hidden from; 32 ballots
-        // transpose those into per-row words (bit c of row r: key 32k + c)
+        // lane l reads keys kv0 + 32k + l (coalesced) and turns each into the
+        // set of the warp's 32 rows it is hidden from; ballots transpose those
+        // into per-row words (bit c of row r's word k: key 32k + c)
         const int4* cm = prm.colmask + static_cast<size_t>(sv.mrow) * Nk + kv0;
-        const int n_in = min(kCols, Nk - kv0);
+        const int n_in = min(kBlockN, Nk - kv0);
         const int4 none = make_int4(0, 0, 0, 0);
-        const int4 ia = lane < n_in ? __ldg(cm + lane) : none;
-        const int4 ib = lane + 32 < n_in ? __ldg(cm + 32 + lane) : none;
-        const uint32_t ca = span_bits(ia.x, ia.y, rw0) | span_bits(ia.z, ia.w, rw0);
-        const uint32_t cb = span_bits(ib.x, ib.y, rw0) | span_bits(ib.z, ib.w, rw0);
+        uint32_t cb[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const int4 iv = 32 * k + lane < n_in ? __ldg(cm + 32 * k + lane) : none;
+          cb[k] = span_bits(iv.x, iv.y, rw0) | span_bits(iv.z, iv.w, rw0);
+        }
 #pragma unroll
         for (int rr = 0; rr < 32; ++rr) {
-          const uint32_t wa = __ballot_sync(0xffffffffu, (ca >> rr) & 1u);
-          const uint32_t wb = __ballot_sync(0xffffffffu, (cb >> rr) & 1u);
-          if (lane == rr) {
-            hid[0] = wa;
-            hid[1] = wb;
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const uint32_t w = __ballot_sync(0xffffffffu, (cb[k] >> rr) & 1u);
+            if (lane == rr) hid[k] = w;
           }
         }
       }
     }
-    // the keys this row sees among the warp's 64, as two 32-bit words: below
+    // the keys this row sees among the tile's 128, as four 32-bit words: below
     // Nk, inside the band, and not hidden by a column interval (one bit test
     // per score below instead of the comparisons themselves)
-    uint32_t keep[2] = {0xffffffffu, 0xffffffffu};
+    uint32_t keep[4] = {0xffffffffu, 0xffffffffu, 0xffffffffu, 0xffffffffu};
     if (masked) {
       const long long klo = MASK != kMaskNone ? static_cast<long long>(row) - prm.wl : 0;
       const long long khi = MASK != kMaskNone ? min(static_cast<long long>(row) + prm.wr + 1, static_cast<long long>(Nk))
                                               : static_cast<long long>(Nk);
 #pragma unroll
-      for (int k = 0; k < 2; ++k) keep[k] = span_bits(klo, khi, kv0 + 32 * k) & ~hid[k];
+      for (int k = 0; k < 4; ++k) keep[k] = span_bits(klo, khi, kv0 + 32 * k) & ~hid[k];
     }
     ok = warp_wait(sm.s_full(t), j & 1, timeout);
-    // load 32 score columns [32*k, 32*k + 32) of this warp's half as fp32,
-    // prescaled and masked
-    auto load_scores = [&](int k, float (&x)[32]) {
-      uint32_t s[32];
-      tmem_ld32(tS + 32 * k, s);
+    if (!ok) break;
+    tc_fence_after();
+
+    // the row's 128 scores: two loads, one wait
+    float x[128];
+    {
+      uint32_t s[128];
+      tmem_ld64(tS, s);
+      tmem_ld64(tS + 64, s + 64);
       tmem_ld_wait();
-      reg_fence32(s);
+      reg_fence64(s);
+      reg_fence64(s + 64);
 #pragma unroll
-      for (int c = 0; c < 32; ++c) x[c] = __uint_as_float(s[c]);
-      if (prescale) {
-#pragma unroll
-        for (int c = 0; c < 32; ++c) x[c] *= prm.scale_log2;
-      }
-      if (masked) {
-#pragma unroll
-        for (int c = 0; c < 32; ++c)
-          if (!((keep[k] >> c) & 1u)) x[c] = -INFINITY;
-      }
-    };
-
-    // pass 1: this half's row max
-    float mloc = __int_as_float(0x7fc00000);  // NaN marks a failed wait
-    if (ok) {
-      tc_fence_after();
-      float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-#pragma unroll
-      for (int k = 0; k < 2; ++k) {
-        float x[32];
-        load_scores(k, x);
-#pragma unroll
-        for (int c = 0; c < 32; c += 8) {
-#pragma unroll
-          for (int a = 0; a < 4; ++a) mx[a] = fmax3(mx[a], x[c + 2 * a], x[c + 2 * a + 1]);
-        }
-      }
-      mloc = fmax3(fmaxf(mx[0], mx[1]), mx[2], mx[3]);
+      for (int c = 0; c < 128; ++c) x[c] = __uint_as_float(s[c]);
     }
-    sm.xch(t, h, j & 1)[r] = mloc;
-    pair_sync(t, q4);
-    const float mother = sm.xch(t, h ^ 1, j & 1)[r];
-    if (!ok || isnan(mother)) {  // uniform across the pair
-      ok = false;
-      break;
+    if (prescale) {
+#pragma unroll
+      for (int c = 0; c < 128; ++c) x[c] *= prm.scale_log2;
     }
-    const float m_tile = fmaxf(mloc, mother) * sl;
+    if (masked) {
+#pragma unroll
+      for (int c = 0; c < 128; ++c)
+        if (!((keep[c >> 5] >> (c & 31)) & 1u)) x[c] = -INFINITY;
+    }
 
-    // adaptive rescaling: move the reference only on a jump beyond tau (both
-    // warps of the pair take the same decision from the same numbers)
+    // the tile's row max: eight independent chains of three-input maxima
+    float mx[8];
+#pragma unroll
+    for (int a = 0; a < 8; ++a) mx[a] = fmaxf(x[2 * a], x[2 * a + 1]);
+#pragma unroll
+    for (int c = 16; c < 128; c += 16) {
+#pragma unroll
+      for (int a = 0; a < 8; ++a) mx[a] = fmax3(mx[a], x[c + 2 * a], x[c + 2 * a + 1]);
+    }
+    const float m_tile =
+        fmax3(fmax3(mx[0], mx[1], mx[2]), fmax3(mx[3], mx[4], mx[5]), fmaxf(mx[6], mx[7])) * sl;
+
+    // adaptive rescaling: move the reference only on a jump beyond tau
     const bool resc = m_tile > m_run + prm.tau;
     float alpha = 1.0f;
     if (resc) {
@@ -631,15 +676,15 @@ __device__ __forceinline__ void softmax_role(const Smem<D, F8>& sm, uint32_t tme
     }
     l_run *= alpha;
 
-    // Correction: rescale this warp's half of the row's O accumulator (final up
-    // to tile j-1, see the MMA order) by alpha before O += P V_j is issued.
+    // Correction: rescale the row's O accumulator (final up to tile j-1, see
+    // the MMA order) by alpha before O += P V_j is issued.
     if (j > 0 && __any_sync(0xffffffffu, resc)) {
-      if (prm.rescale_count && h == 0) {
+      if (prm.rescale_count) {
         const unsigned n = __popc(__ballot_sync(0xffffffffu, resc));
         if (lane == 0) atomicAdd(prm.rescale_count, static_cast<unsigned long long>(n));
       }
 #pragma unroll
-      for (int cc = 0; cc < kOCols / 32; ++cc) {
+      for (int cc = 0; cc < D / 32; ++cc) {
         uint32_t o[32];
         tmem_ld32(tO + cc * 32, o);
         tmem_ld_wait();
@@ -650,25 +695,22 @@ __device__ __forceinline__ void softmax_role(const Smem<D, F8>& sm, uint32_t tme
       }
     }
 
-    // pass 2: P = 2^(x*sl - m), 32 scores at a time (re-read from TMEM) ->
-    // BF16 pairs in the first 32 TMEM columns of this warp's half of S_t.
-    // Chunk k's P lands in columns [16k, 16k+16), which chunk k has consumed,
-    // and is announced on its own barrier so its O += P V can start while the
-    // next chunk is being exponentiated.
+    // P = 2^(x*sl - m), 32 keys at a time -> BF16 pairs (E4M3 quadruples) in
+    // the tile's first TMEM columns, whose scores are already in registers.
+    // Chunk k is announced on its own barrier so its O += P V can start while
+    // the next chunk is being exponentiated.
     constexpr float kOff = F8 ? kP8Offset : 0.0f;
     const float neg_m = (m_run == -INFINITY) ? 0.0f : kOff - m_run;
     const float2 sl2 = make_float2(sl, sl), nm2 = make_float2(neg_m, neg_m);
     float2 sum2[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
                       make_float2(0.f, 0.f)};
 #pragma unroll
-    for (int k = 0; k < 2; ++k) {
-      float x[32];
-      load_scores(k, x);
+    for (int k = 0; k < kPChunks; ++k) {
       uint32_t p[16];
       float2 prev = make_float2(0.f, 0.f);
 #pragma unroll
       for (int i = 0; i < 16; ++i) {
-        const int c = 2 * i;
+        const int c = 32 * k + 2 * i;
         const float2 u = ffma2(make_float2(x[c], x[c + 1]), sl2, nm2);
         float2 e;
         if ((c & 15) < POLY16) {
@@ -700,25 +742,18 @@ __device__ __forceinline__ void softmax_role(const Smem<D, F8>& sm, uint32_t tme
     l_run += s03.x + s03.y;
   }
 
-  // Epilogue.  Both warps of the pair reach both exchanges below whatever
-  // happened above.
+  // Epilogue.
   const bool ok2 = ok && warp_wait(sm.o_full(t), 0, timeout);
-  sm.xch(t, h, 0)[r] = ok2 ? l_run : __int_as_float(0x7fc00000);
-  pair_sync(t, q4);
-  const float lother = sm.xch(t, h ^ 1, 0)[r];
-  const bool ok3 = ok2 && !isnan(lother);
   uint8_t* sOt = sm.base + C::kOffO + t * C::kOTileBytes;
-  const float l_tot = l_run + lother;
   const bool ragged = sv.packed && rw0 + 32 > sv.Nq;
-  if (ok3) {
+  if (ok2) {
     tc_fence_after();
     // O / l -> BF16 -> the tile's O staging (BF16 inputs: the tile's Q buffer,
     // whose last reader, the final S MMA, finished before the last O MMA) in
-    // the 128-byte swizzled layout the O tensor map expects.  Warp h writes
-    // output columns [h*d/2, (h+1)*d/2).
-    const float inv_l = l_tot > 0.0f ? prm.o_scale / l_tot : 0.0f;
+    // the 128-byte swizzled layout the O tensor map expects.
+    const float inv_l = l_run > 0.0f ? prm.o_scale / l_run : 0.0f;
 #pragma unroll
-    for (int cc = 0; cc < kOCols / 32; ++cc) {
+    for (int cc = 0; cc < D / 32; ++cc) {
       uint32_t o[32];
       tmem_ld32(tO + cc * 32, o);
       tmem_ld_wait();
@@ -727,7 +762,7 @@ __device__ __forceinline__ void softmax_role(const Smem<D, F8>& sm, uint32_t tme
 #pragma unroll
       for (int i = 0; i < 16; ++i)
         w[i] = pack_bf16x2(__uint_as_float(o[2 * i]) * inv_l, __uint_as_float(o[2 * i + 1]) * inv_l);
-      const int col0 = h * kOCols + cc * 32;  // first output column of this chunk
+      const int col0 = cc * 32;  // first output column of this chunk
       if (ragged) {
         // the warp's 32 rows cross the end of a packed sequence: a TMA store
         // would write into the next sequence, so each row stores itself
@@ -749,24 +784,24 @@ __device__ __forceinline__ void softmax_role(const Smem<D, F8>& sm, uint32_t tme
     }
     fence_proxy_async_smem();
   }
-  // d = 128: each warp stores its own 64-column box; d = 64: the pair shares
-  // one box, stored by the h = 0 warp after both halves are written.
-  if (D == 64) pair_sync(t, q4);
   __syncwarp();
-  if (ok3 && !ragged && lane == 0 && rw0 < sv.Nq && (D == 128 || h == 0)) {
-    const int box = D == 128 ? h : 0;
-    const uint32_t src = smem_u32(sOt + box * C::kBoxBytes + q4 * 32 * 128);
-    if (sv.packed) tma_store_3d(tm_o, src, box * 64, sv.head_q, sv.q0 + rw0);
-    else tma_store_3d(tm_o, src, box * 64, rw0, sv.head_q);
+  // each warp stores its 32 rows, one 64-column box at a time
+  if (ok2 && !ragged && lane == 0 && rw0 < sv.Nq) {
+#pragma unroll
+    for (int box = 0; box < D / 64; ++box) {
+      const uint32_t src = smem_u32(sOt + box * C::kBoxBytes + q4 * 32 * 128);
+      if (sv.packed) tma_store_3d(tm_o, src, box * 64, sv.head_q, sv.q0 + rw0);
+      else tma_store_3d(tm_o, src, box * 64, rw0, sv.head_q);
+    }
     bulk_commit_group();
     bulk_wait_group_read0();
   }
-  if (ok3 && h == 0 && sv.lse_row0 != nullptr && row < sv.Nq) {
+  if (ok2 && sv.lse_row0 != nullptr && row < sv.Nq) {
     // P carried 2^kOff: LSE = ln 2 * (m - kOff + log2 l)
     const float m_use = (m_run == -INFINITY) ? 0.0f : m_run - (F8 ? kP8Offset : 0.0f);
-    sv.lse_row0[row] = (m_use + log2f(l_tot)) * kLn2;
+    sv.lse_row0[row] = (m_use + log2f(l_run)) * kLn2;
   }
-  if (!ok3 && lane == 0) atomicOr(&g_status, kStatusTimeout);
+  if (!ok2 && lane == 0) atomicOr(&g_status, kStatusTimeout);
 }
 
 // ---------------------------------------------------------------------------
@@ -891,10 +926,9 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   if (threadIdx.x == 0) {
     for (int i = 0; i < C::kNumBars; ++i) {
       const uint32_t b = sm.bar(i);
-      // p_full: one arrival per softmax warp of the tile (8); everything else: one.
-      const bool pf = b == sm.p_full(0, 0) || b == sm.p_full(0, 1) || b == sm.p_full(1, 0) ||
-                      b == sm.p_full(1, 1);
-      mbar_init(b, pf ? 8u : 1u);
+      // p_full: one arrival per softmax warp of the tile (4); everything else: one.
+      const bool pf = b >= sm.p_full(0, 0) && b <= sm.p_full(1, kPChunks - 1);
+      mbar_init(b, pf ? 4u : 1u);
     }
     fence_barrier_init();
     fence_proxy_async_smem();
@@ -1037,11 +1071,22 @@ int launch_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& 
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  static int launch_regs[kMaxDevices];
   std::call_once(attr_once[dev], [&] {
     attr_err[dev] = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          Cfg<D, F8>::kSmemBytes);
+    cudaFuncAttributes fa;
+    if (attr_err[dev] == cudaSuccess) attr_err[dev] = cudaFuncGetAttributes(&fa, kern);
+    if (attr_err[dev] == cudaSuccess) launch_regs[dev] = fa.numRegs;
   });
   if (attr_err[dev] != cudaSuccess) return cuda_fail(attr_err[dev], "cudaFuncSetAttribute");
+  // the warpgroups' setmaxnreg shares must fit in the registers the block is
+  // launched with, or setmaxnreg.inc would never be granted
+  if (launch_regs[dev] * kNumThreads < 2 * 128 * kSoftmaxRegs + 128 * kProducerRegs) {
+    t_last_error = "attn_fwd_kernel: built with " + std::to_string(launch_regs[dev]) +
+                   " registers per thread, below the setmaxnreg split";
+    return ATTN_ERR_CUDA;
+  }
   const unsigned grid = static_cast<unsigned>(prm.BH) * static_cast<unsigned>(prm.n_qblocks);
   kern<<<grid, kNumThreads, Cfg<D, F8>::kSmemBytes, stream>>>(tq, tk, tv, to, prm);
   e = cudaGetLastError();

@@ -325,6 +325,15 @@ size_t attn_bwd_workspace_size(int B, int H, int Nq, int d);
  * anything else is done.  Every call on a device uses the same array: calls
  * must be ordered (one stream, or synchronised between streams).  Arguments
  * and results are otherwise those of attn_bwd.
+ *
+ * The array lives in the same device module as every backward kernel, so the
+ * 96 MiB are resident on a device as soon as any backward entry point
+ * (attn_bwd, attn_bwd_window, attn_bwd_varlen, attn_bwd_colmask or this one)
+ * has run there -- from context creation under CUDA_MODULE_LOADING=EAGER --
+ * whether or not attn_bwd_noalloc is ever called.  The array's device address
+ * is looked up once per device and context (again after cudaDeviceReset or
+ * when another context becomes current), on the first call there; make that
+ * first call before any stream capture.
  */
 int attn_bwd_noalloc(const void *q, const void *k, const void *v, const void *o, const void *dout,
                      const float *lse, void *dq, void *dk, void *dv, int B, int H, int Hkv, int Nq,

@@ -121,3 +121,150 @@ def compare_varlen(o_gpu, lse_gpu, ref, cu_q):
     return {"max_abs_o": float(eo.max()) if eo.size else 0.0,
             "mean_abs_o": float(eo.mean()) if eo.size else 0.0,
             "max_abs_lse": float(el.max()) if el.size else 0.0}
+
+
+# ---------------------------------------------------------------------------
+# Element-wise error bound of the BF16 backward
+# ---------------------------------------------------------------------------
+# Each gradient element is a sum of products in which at most one BF16-rounded
+# factor per product carries error, accumulated in fp32 (error ~2^-24 per add,
+# negligible), and is itself rounded to BF16 once:
+#   dV_j = sum_i P_ij dO_i          P rounded to BF16 before its GEMM:
+#        |err| <= u (sum_i P_ij |dO_i|) + u |dV_j|
+#   dS_ij = P_ij (dP_ij - D_i)       dS rounded to BF16 before its GEMMs, and
+#                                    D_i = <dO_i, O_i> formed from the forward's
+#                                    BF16 O, itself within u (|O| + P|V|) of O:
+#        |err dS_ij| <= u |dS_ij| + u P_ij sum_c |dO_ic| (|O_ic| + (P|V|)_ic)
+#   dK_j = scale sum_i dS_ij Q_i,  dQ_i = scale sum_j dS_ij K_j
+#        |err| <= scale sum |err dS| |Q or K| + u |dK_j or dQ_i|
+# with u = 2^-8 the unit roundoff of BF16 (8 significant bits, round to
+# nearest even).  The exponentials (MUFU, or the polynomial at 1.01e-4
+# relative) and the forward's LSE (within ~1e-5) move P by far less than u.
+# The GPU tests allow twice the sum (BWD_C = 2); tests/test_bwd_bound.py checks
+# that a CPU model of exactly these roundings stays within the sum itself.
+BWD_U = 2.0 ** -8
+BWD_C = 2.0
+
+
+def bwd_bound_head(q, k, v, do, scale, visible, chunk=512):
+    """Magnitude sums of the bound above for one head, fp64.
+
+    q, do [Nq, d]; k, v [Nk, d]; visible(r0, r1) -> bool [r1 - r0, Nk], the
+    keys each of rows r0..r1-1 sees.  Returns (mq [Nq, d], mk [Nk, d],
+    mv [Nk, d]) such that |err| <= u * (m + |grad|) element by element."""
+    Nq, d = q.shape
+    Nk = k.shape[0]
+    mq = np.zeros((Nq, d))
+    mk = np.zeros((Nk, d))
+    mv = np.zeros((Nk, d))
+    if Nq == 0 or Nk == 0:
+        return mq, mk, mv
+    ak, av = np.abs(k), np.abs(v)
+    for r0 in range(0, Nq, chunk):
+        r1 = min(Nq, r0 + chunk)
+        vis = visible(r0, r1)
+        s = scale * (q[r0:r1] @ k.T)
+        s = np.where(vis, s, -np.inf)
+        m = s.max(axis=1, keepdims=True)
+        m = np.where(np.isfinite(m), m, 0.0)
+        e = np.where(vis, np.exp(s - m), 0.0)
+        l = e.sum(axis=1, keepdims=True)
+        p = e / np.where(l > 0, l, 1.0)
+        o = p @ v
+        pv_abs = p @ av
+        g = do[r0:r1]
+        dp = g @ v.T
+        dd = (g * o).sum(axis=1, keepdims=True)
+        ds = p * (dp - dd)
+        dabs = (np.abs(g) * (np.abs(o) + pv_abs)).sum(axis=1, keepdims=True)
+        w = np.abs(ds) + p * dabs
+        mq[r0:r1] = scale * (w @ ak)
+        mk += scale * (w.T @ np.abs(q[r0:r1]))
+        mv += p.T @ np.abs(g)
+    return mq, mk, mv
+
+
+def band_visible(wl, wr, Nk):
+    """visible(r0, r1) for the key band i - wl <= j <= i + wr (-1: no bound)."""
+    j = np.arange(Nk)[None, :]
+
+    def vis(r0, r1):
+        i = np.arange(r0, r1)[:, None]
+        ok = np.ones((r1 - r0, Nk), dtype=bool)
+        if wl >= 0:
+            ok &= j >= i - wl
+        if wr >= 0:
+            ok &= j <= i + wr
+        return ok
+    return vis
+
+
+def colmask_visible(cols, causal):
+    """visible(r0, r1) for column intervals cols [Nk, 4] (lo1, hi1, lo2, hi2:
+    rows in [lo, hi) do not see the key) plus the causal rule j <= i."""
+    lo1, hi1, lo2, hi2 = (cols[:, c][None, :].astype(np.int64) for c in range(4))
+    Nk = cols.shape[0]
+    j = np.arange(Nk)[None, :]
+
+    def vis(r0, r1):
+        i = np.arange(r0, r1)[:, None]
+        hidden = ((i >= lo1) & (i < hi1)) | ((i >= lo2) & (i < hi2))
+        ok = ~hidden
+        if causal:
+            ok &= j <= i
+        return ok
+    return vis
+
+
+def bwd_bound_dense(q, k, v, do, scale, visible_of):
+    """Magnitude sums for [B, H, Nq, d] problems with [B, Hkv, Nk, d] keys and
+    values (grouped heads sum into their key/value head).  visible_of(b, h)
+    returns the visibility function of that query head."""
+    B, H, Nq, d = q.shape
+    Hkv = k.shape[1]
+    grp = H // Hkv
+    mq = np.zeros(q.shape)
+    mk = np.zeros(k.shape)
+    mv = np.zeros(v.shape)
+    for b in range(B):
+        for h in range(H):
+            a, bk, bv = bwd_bound_head(q[b, h], k[b, h // grp], v[b, h // grp], do[b, h], scale,
+                                       visible_of(b, h))
+            mq[b, h] = a
+            mk[b, h // grp] += bk
+            mv[b, h // grp] += bv
+    return mq, mk, mv
+
+
+def bwd_bound_varlen(q, k, v, do, cu_q, cu_k, scale, wl, wr):
+    """Magnitude sums for packed batches (q, do [total_q, H, d]; k, v
+    [total_k, Hkv, d]); positions count from 0 within each sequence."""
+    H, Hkv = q.shape[1], k.shape[1]
+    grp = H // Hkv
+    mq = np.zeros(q.shape)
+    mk = np.zeros(k.shape)
+    mv = np.zeros(v.shape)
+    for s in range(len(cu_q) - 1):
+        a0, a1, c0, c1 = int(cu_q[s]), int(cu_q[s + 1]), int(cu_k[s]), int(cu_k[s + 1])
+        for h in range(H):
+            a, bk, bv = bwd_bound_head(q[a0:a1, h], k[c0:c1, h // grp], v[c0:c1, h // grp],
+                                       do[a0:a1, h], scale, band_visible(wl, wr, c1 - c0))
+            mq[a0:a1, h] = a
+            mk[c0:c1, h // grp] += bk
+            mv[c0:c1, h // grp] += bv
+    return mq, mk, mv
+
+
+def check_grads_elementwise(got, ref, mags, label=""):
+    """|got - ref| <= BWD_C * u * (magnitude sums + |ref|) element by element,
+    plus a floor of 1e-6 of the problem's largest gradient for fp32 noise."""
+    top = max((np.abs(r).max() if r.size else 0.0) for r in ref)
+    for name, g, r, m in zip(("dq", "dk", "dv"), got, ref, mags):
+        g = np.asarray(g, dtype=np.float64)
+        assert np.all(np.isfinite(g)), (label, name)
+        err = np.abs(g - r)
+        lim = BWD_C * BWD_U * (m + np.abs(r)) + 1e-6 * top + 1e-12
+        worst = np.unravel_index(np.argmax(err / lim), err.shape) if err.size else None
+        if err.size:
+            print(label, name, "max err/bound", float((err / lim).max()), "at", worst)
+        assert np.all(err <= lim), (label, name, worst, float(err[worst]), float(lim[worst]))

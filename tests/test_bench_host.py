@@ -76,3 +76,19 @@ def test_cpu_baseline_parity_report(name):
                 o[b, h], lse[b, h] = oracle.attn_rows(q, np.arange(w.Nq), k, v, w.scale, w.causal)
         exact = bench.cpu_baseline(w, 0.5, o, lse)["parity"]
         assert exact["max_abs_o"] == 0.0 and exact["max_abs_lse"] == 0.0
+
+
+def test_peak_follows_the_timed_window():
+    """A short window with no power-cap samples is a burst; a seconds-long
+    window, or one that saw sw_power_cap, takes the sustained figure."""
+    peaks = {"burst": 1636.8, "sustained": 1388.9, "hbm_gbs": 6551.4, "source": "measured"}
+    cool = {"sm_mhz": 1965.0, "reasons": []}
+    capped = {"sm_mhz": 1620.0, "reasons": ["sw_power_cap"]}
+    assert bench.pick_peak(peaks, 18.0, cool)[0] == 1636.8
+    assert bench.pick_peak(peaks, 18.0, None)[0] == 1636.8
+    assert bench.pick_peak(peaks, 18.0, capped)[0] == 1388.9
+    assert bench.pick_peak(peaks, 1800.0, cool)[0] == 1388.9
+    assert bench.pick_peak(peaks, 18.0, cool, ratio=2.0)[0] == 2 * 1636.8
+    # 148 SMs x 8192 FLOP/clk at 1965 MHz
+    assert abs(bench.clock_peak(cool) - 2382.4) < 0.1
+    assert bench.clock_peak(None) is None
