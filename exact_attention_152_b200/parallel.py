@@ -5,9 +5,11 @@ path shards with no exchange inside it:
 
 * ``bench.py --gpus N`` runs one independent problem per GPU (weak scaling) and
   only reduces the timings (max over ranks);
-* ``fwd_sharded`` splits the B*H heads of ONE problem into contiguous per-rank
-  ranges, runs the CUDA forward on the local range and, if asked, all-gathers
-  O and LSE so every rank holds the full result.
+* ``fwd_sharded`` splits ONE problem by key/value-head groups: a rank owns
+  whole groups -- one key/value head with the H/Hkv query heads that read it
+  (grouped-query attention; H/Hkv = 1 for multi-head attention) -- so it needs
+  only its own K/V heads.  It runs the CUDA forward on that range and, if
+  asked, all-gathers O and LSE so every rank holds the full result.
 
 Nothing here does attention arithmetic; the local compute is the C-ABI call.
 """
@@ -79,28 +81,47 @@ def gather_heads(local: torch.Tensor, plan, n_units: int, group=None) -> torch.T
     return full
 
 
-def fwd_sharded(q, k, v, causal: bool = False, scale: float | None = None, gather: bool = True):
-    """Forward attention of one [B,H,N,d] problem split over the ranks by heads.
+def group_plan(B: int, H: int, Hkv: int, world: int):
+    """Per-rank ranges for a problem of B*H query heads over B*Hkv key/value
+    heads: the key/value heads are split into contiguous ranges (shard_plan),
+    and a rank's query heads are those of its key/value heads.  Query head h
+    of batch entry b reads key/value head h // (H // Hkv), so in the flattened
+    B*H axis the query heads of key/value heads [s, e) are [s*G, e*G) with
+    G = H // Hkv.  Returns (kv_plan, q_plan)."""
+    if Hkv <= 0 or H % Hkv != 0:
+        raise ValueError("H must be a positive multiple of Hkv")
+    G = H // Hkv
+    kv_plan = shard_plan(B * Hkv, world)
+    q_plan = [(s * G, e * G) for s, e in kv_plan]
+    return kv_plan, q_plan
 
-    Each rank computes its contiguous range of the B*H heads with the CUDA
-    kernel (``binding.fwd``); with ``gather`` every rank receives the full O
-    [B,H,Nq,d] and LSE [B,H,Nq], otherwise each rank returns (o_local,
+
+def fwd_sharded(q, k, v, causal: bool = False, scale: float | None = None, gather: bool = True,
+                window=None):
+    """Forward attention of one problem, q [B,H,Nq,d] and k/v [B,Hkv,Nk,d]
+    (Hkv divides H), split over the ranks by key/value-head groups.
+
+    Each rank computes the query heads of its contiguous range of key/value
+    heads with the CUDA kernel (``binding.fwd``: attn_fwd, attn_fwd_gqa or
+    attn_fwd_window); every load stays in the rank's own memory.  With
+    ``gather`` every rank receives the full O [B,H,Nq,d] and LSE [B,H,Nq]
+    (one NCCL all-gather each); otherwise each rank returns (o_local,
     lse_local, (start, end)) for its range of the flattened B*H axis.
     """
     from . import binding
 
     B, H, Nq, d = q.shape
-    Nk = k.shape[2]
+    Hkv, Nk = k.shape[1], k.shape[2]
     world = dist.get_world_size() if dist.is_initialized() else 1
     rank = dist.get_rank() if dist.is_initialized() else 0
-    plan = shard_plan(B * H, world)
-    s, e = plan[rank]
-    q2 = q.reshape(B * H, 1, Nq, d)[s:e].reshape(1, e - s, Nq, d)
-    k2 = k.reshape(B * H, 1, Nk, d)[s:e].reshape(1, e - s, Nk, d)
-    v2 = v.reshape(B * H, 1, Nk, d)[s:e].reshape(1, e - s, Nk, d)
+    kv_plan, q_plan = group_plan(B, H, Hkv, world)
+    ks, ke = kv_plan[rank]
+    s, e = q_plan[rank]
     if e > s:
-        o2, l2 = binding.fwd(q2.contiguous(), k2.contiguous(), v2.contiguous(), causal=causal,
-                             scale=scale)
+        q2 = q.reshape(B * H, Nq, d)[s:e].reshape(1, e - s, Nq, d).contiguous()
+        k2 = k.reshape(B * Hkv, Nk, d)[ks:ke].reshape(1, ke - ks, Nk, d).contiguous()
+        v2 = v.reshape(B * Hkv, Nk, d)[ks:ke].reshape(1, ke - ks, Nk, d).contiguous()
+        o2, l2 = binding.fwd(q2, k2, v2, causal=causal, scale=scale, window=window)
         o2 = o2.reshape(e - s, Nq, d)
         l2 = l2.reshape(e - s, Nq)
     else:
@@ -108,6 +129,6 @@ def fwd_sharded(q, k, v, causal: bool = False, scale: float | None = None, gathe
         l2 = torch.empty((0, Nq), dtype=torch.float32, device=q.device)
     if not gather:
         return o2, l2, (s, e)
-    o = gather_heads(o2, plan, B * H).reshape(B, H, Nq, d)
-    lse = gather_heads(l2, plan, B * H).reshape(B, H, Nq)
+    o = gather_heads(o2, q_plan, B * H).reshape(B, H, Nq, d)
+    lse = gather_heads(l2, q_plan, B * H).reshape(B, H, Nq)
     return o, lse
