@@ -7,9 +7,11 @@
 namespace eab {
 
 // exp2 on the FMA pipe: 2^x = 2^n * p(f), n = round-to-nearest(x), f = x - n in
-// [-1/2, 1/2].  p is a cubic with p(0) = 1 exactly, fitted by this library for
-// minimum max relative error (1.01e-4, below BF16's 2^-9 half ulp) -- see
-// fit_exp2_poly.py.  n is read out of the low mantissa bits of x + 1.5*2^23
+// [-1/2, 1/2].  p is a cubic with p(0) = 1 exactly whose other coefficients
+// minimise the maximum relative error |p(f)/2^f - 1| on [-1/2, 1/2] (a linear
+// program on a dense grid, rounded to fp32; tests/test_exp2_coeffs.py solves
+// it again): 1.01e-4, far below BF16's unit roundoff 2^-8.  n is read out of
+// the low mantissa bits of x + 1.5*2^23
 // and added straight into the exponent field.  x is clamped at -127, where the
 // result is exactly +0 (so masked scores give weight 0).
 constexpr float kExpC1 = 0x1.62f5fap-1f;
