@@ -1220,30 +1220,7 @@ __device__ __align__(256) unsigned char g_bwd_scratch[kStaticScratchBytes];
 // the module again, possibly elsewhere.  So the address is cached per device
 // together with the unique ID of the context it was looked up in, and looked up
 // again (cudaGetSymbolAddress: a lookup, no allocation) whenever that ID
-// changes or cannot be read.
-using CtxGetCurrentFn = CUresult (*)(CUcontext*);
-using CtxGetIdFn = CUresult (*)(CUcontext, unsigned long long*);
-
-bool current_context_id(unsigned long long* id) {
-  static CtxGetCurrentFn get_current = nullptr;
-  static CtxGetIdFn get_id = nullptr;
-  static std::once_flag once;
-  std::call_once(once, [] {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      get_current = reinterpret_cast<CtxGetCurrentFn>(p);
-    p = nullptr;
-    if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      get_id = reinterpret_cast<CtxGetIdFn>(p);
-  });
-  CUcontext ctx = nullptr;
-  if (!get_current || !get_id || get_current(&ctx) != CUDA_SUCCESS || ctx == nullptr) return false;
-  return get_id(ctx, id) == CUDA_SUCCESS;
-}
-
+// changes or cannot be read (current_context_id, host_common.h).
 int static_scratch(void** ptr) {
   static std::mutex mu;
   static void* addr[kMaxDeviceCount];
