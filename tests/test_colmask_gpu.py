@@ -235,3 +235,38 @@ def test_colmask_bwd_hidden_blocks():
     mags = harness.bwd_bound_dense(f(q), f(k), f(v), f(do), 0.1,
                                    lambda b, h: harness.colmask_visible(mask[b, 0], False))
     check_grads(tuple(x.float().cpu().numpy() for x in (dq, dk, dv)), ref, mags, "hidden")
+
+
+def test_colmask_bwd_both_hidden_ranges_ragged():
+    """Both hidden query-tile ranges of a key block, a partial last key block
+    and a partial last query tile at once (Nq = 650, Nk = 333): every key
+    hides rows [128, 384) by its first interval and [512, Nq) by its second,
+    with per-key jitter in the middle block so the block summaries (max lo,
+    min hi) differ from the keys' own bounds.  The backward skips tiles 1-2
+    and 4-5 for the blocks where every key hides them; the result matches the
+    oracle under the element-wise bound, and keys past Nk do not exist."""
+    import torch
+    from exact_attention_152_b200 import binding
+    from test_bwd_gpu import check_grads
+    B, H, Nq, Nk, d = 1, 2, 650, 333, 128
+    q, k, v = (harness.random_bits(334, (B, H, n, d), tensor=t) for t, n in (("q", Nq), ("k", Nk), ("v", Nk)))
+    do = harness.random_bits(335, (B, H, Nq, d), tensor="q")
+    mask = masks.empty(B, 1, Nk)
+    mask[..., 0], mask[..., 1] = 128, 384
+    mask[..., 2], mask[..., 3] = 512, Nq
+    rng = np.random.default_rng(5)
+    mid = slice(128, 256)
+    mask[0, 0, mid, 0] = 128 - rng.integers(0, 40, 128)     # max lo stays 128: tiles 1-2 still hidden
+    mask[0, 0, mid, 1] = 384 + rng.integers(0, 40, 128)
+    mask[0, 0, mid, 3] = Nq + rng.integers(0, 40, 128)       # ends past Nq: the last tile stays hidden
+    qd, kd, vd, dod = (harness.to_device_bf16(x) for x in (q, k, v, do))
+    md = torch.from_numpy(mask).cuda()
+    o, lse = binding.fwd_colmask(qd, kd, vd, md, scale=0.1)
+    dq, dk, dv = binding.bwd_colmask(qd, kd, vd, o, dod, lse, md, scale=0.1)
+    assert binding.attn_status_sync(torch.cuda.current_stream().cuda_stream) == 0
+    assert torch.all(dq[:, :, 128:384] == 0) and torch.all(dq[:, :, 512:] == 0)
+    f = inputs.bf16_bits_to_f64
+    ref = oracle.attn_bwd_colmask(f(q), f(k), f(v), f(do), 0.1, False, mask)
+    mags = harness.bwd_bound_dense(f(q), f(k), f(v), f(do), 0.1,
+                                   lambda b, h: harness.colmask_visible(mask[b, 0], False))
+    check_grads(tuple(x.float().cpu().numpy() for x in (dq, dk, dv)), ref, mags, "two ranges, ragged")

@@ -121,26 +121,29 @@ def test_block_summary_rules_are_sound():
 def test_backward_hidden_tile_ranges_are_sound():
     """The backward skips, per 128-key block, the query tiles t in
     [ceil(max lo / 128), (min hi >= Nq ? last : min hi // 128 - 1)] of each
-    interval: every key of the block hides all rows of those tiles."""
-    for trial in range(30):
-        nq, nk = 700, 384
-        if trial % 2:
-            m = masks.random_intervals(200 + trial, 1, 1, nq, nk)[0, 0].astype(np.int64)
-        else:
-            m = masks.documents([[100, 130, 90, 64]], nk, bidirectional=True)[0, 0].astype(np.int64)
-        vis = dense_visible(m, nq, False)
-        n_qtiles = (nq + 127) // 128
-        fired = 0
-        for blk in range(nk // 128):
-            c = m[blk * 128:(blk + 1) * 128]
-            for lo_col, hi_col in ((0, 1), (2, 3)):
-                empty = c[:, lo_col] >= c[:, hi_col]
-                lo = np.where(empty, np.iinfo(np.int64).max, c[:, lo_col]).max()
-                hi = np.where(empty, np.iinfo(np.int64).min, c[:, hi_col]).min()
-                first = 0 if lo <= 0 else -(-lo // 128)
-                last = n_qtiles - 1 if hi >= nq else hi // 128 - 1
-                for t in range(max(first, 0), min(last, n_qtiles - 1) + 1):
-                    assert not vis[128 * t:min(128 * t + 128, nq), blk * 128:(blk + 1) * 128].any()
-                    fired += 1
-        if trial % 2 == 0:
-            assert fired > 0
+    interval: every key of the block hides all rows of those tiles.  Key and
+    query lengths that are not multiples of 128 leave a partial last key block
+    (keys past Nk take no part in its summary) and a partial last query tile."""
+    for nq, nk in ((700, 384), (650, 333), (513, 200), (129, 129)):
+        for trial in range(24):
+            if trial % 2:
+                m = masks.random_intervals(200 + trial + nq, 1, 1, nq, nk)[0, 0].astype(np.int64)
+            else:
+                m = masks.documents([masks.document_lengths(300 + trial, nk, 30, 160)], nk,
+                                    bidirectional=True)[0, 0].astype(np.int64)
+            vis = dense_visible(m, nq, False)
+            n_qtiles = (nq + 127) // 128
+            fired = 0
+            for blk in range((nk + 127) // 128):
+                c = m[blk * 128:min(nk, (blk + 1) * 128)]
+                for lo_col, hi_col in ((0, 1), (2, 3)):
+                    empty = c[:, lo_col] >= c[:, hi_col]
+                    lo = np.where(empty, np.iinfo(np.int64).max, c[:, lo_col]).max()
+                    hi = np.where(empty, np.iinfo(np.int64).min, c[:, hi_col]).min()
+                    first = 0 if lo <= 0 else -(-lo // 128)
+                    last = n_qtiles - 1 if hi >= nq else hi // 128 - 1
+                    for t in range(max(first, 0), min(last, n_qtiles - 1) + 1):
+                        assert not vis[128 * t:min(128 * t + 128, nq), blk * 128:min(nk, (blk + 1) * 128)].any()
+                        fired += 1
+            if trial % 2 == 0 and nq >= 500:
+                assert fired > 0, (nq, nk, trial)
