@@ -22,22 +22,32 @@
 //    the block stay in shared memory; the CTA walks every query tile (128
 //    rows) of every query head that reads this key/value head (with a key
 //    band such as causal, only the tiles whose queries see one of the block's
-//    keys), double-buffering Q and dO by TMA.
+//    keys), loading Q (two stages) and dO (one stage, refilled between the
+//    tile's dV GEMM and the next tile's dP^T GEMM) by TMA.  Shared memory at
+//    d = 128: K, V, two Q stages, dO, dS and the dQ drain's staging, 32 KiB
+//    each.
 //  * Per query tile, five BF16 GEMMs on the tensor cores, all with M = 128
 //    keys or queries:
 //        S^T  = K Q^T          (keys x queries, TMEM columns [0, 128))
 //        dP^T = V dO^T         (TMEM columns [128, 256))
 //        dV  += P^T dO         (A = P^T straight from TMEM; TMEM [256, 256+d))
 //        dK  += dS^T Q         (A = dS^T from TMEM;          TMEM [256+d, 256+2d))
-//        dQ_i = dS K           (A = dS from shared memory, MN-major; TMEM [0, d))
+//        dQ_i = dS K           (A = dS from shared memory, MN-major; TMEM [128, 128+d))
 //    Because the tiles are computed transposed (keys on the TMEM lanes), P^T
 //    and dS^T are the A operands of the dV and dK GEMMs as they stand.
 //  * Warps 0-7 turn S^T and dP^T into P^T and dS^T (one key row per thread,
-//    half of the query columns per warp) and write them back to TMEM as BF16
-//    pairs over the first half of their own columns; dS also goes to shared
-//    memory for the dQ GEMM.  Warps 8-11 drain each dQ tile from TMEM into the
-//    fp32 accumulator with vector reductions.  Warp 12 loads (TMA), warp 13
-//    issues the MMAs from one thread.
+//    half of the query columns per warp).  S^T is taken into registers first
+//    and its columns handed back at once, so the next tile's S^T GEMM runs
+//    while the exponentials are computed; P^T and dS^T go back to TMEM as
+//    BF16 pairs in the dP^T columns (each 32-query chunk as 16 columns of P^T
+//    then 16 of dS^T), where dQ accumulates once dK has read them.  dS also
+//    goes to shared memory for the dQ GEMM.  Warps 8-11 drain each dQ tile
+//    from TMEM into the fp32 accumulator with TMA reduce-adds, 32 columns at a
+//    time through two alternating staging slots.  Warp 12 loads (TMA), warp
+//    13 issues the MMAs from one thread, in the order
+//        S(0) dP(0) | S(t+1) | dV(t) dK(t) | dQ(t) | dP(t+1) | ...
+//    so the tensor pipe has the next tile's S^T to compute while the
+//    element-wise warps work on this one.
 //  * Variants (template arguments): key band (causal, sliding windows) or
 //    column intervals (attn_bwd_colmask; the query tiles every key of the
 //    block hides form at most two ranges per head and are stepped over), and
@@ -102,12 +112,15 @@ struct Cfg {
   static constexpr int kOffK = 0;
   static constexpr int kOffV = kTileBytes;
   static constexpr int kOffQ = 2 * kTileBytes;      // 2 stages
-  static constexpr int kOffDO = 4 * kTileBytes;     // 2 stages
-  static constexpr int kOffDS = 6 * kTileBytes;     // dS, 128 queries x 128 keys, MN-major
+  static constexpr int kOffDO = 4 * kTileBytes;     // 1 stage: refilled between dV and the next dP^T
+  static constexpr int kOffDS = 5 * kTileBytes;     // dS, 128 queries x 128 keys, MN-major
   static constexpr int kDSBytes = 2 * kBoxBytes;
-  static constexpr int kOffRow = kOffDS + kDSBytes; // per stage: LSE*log2e [128], D [128]
+  // dQ drain staging: per drain warp two 4 KiB slots (32 rows x 32 fp32)
+  static constexpr int kOffStage = kOffDS + kDSBytes;
+  static constexpr int kStageBytes = 4 * 2 * 4096;
+  static constexpr int kOffRow = kOffStage + kStageBytes;  // per stage: LSE*log2e [128], D [128]
   static constexpr int kRowBytes = 2 * 2 * kBlockQ * 4;
-  static constexpr int kNumBars = 13;
+  static constexpr int kNumBars = 16;
   static constexpr int kOffBar = kOffRow + kRowBytes;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
   static constexpr int kSmemBytes = kOffMisc + 16;
@@ -144,7 +157,7 @@ struct Smem {
   __device__ __forceinline__ uint32_t k() const { return sbase + Cfg<D>::kOffK; }
   __device__ __forceinline__ uint32_t v() const { return sbase + Cfg<D>::kOffV; }
   __device__ __forceinline__ uint32_t q(int s) const { return sbase + Cfg<D>::kOffQ + s * Cfg<D>::kTileBytes; }
-  __device__ __forceinline__ uint32_t dout(int s) const { return sbase + Cfg<D>::kOffDO + s * Cfg<D>::kTileBytes; }
+  __device__ __forceinline__ uint32_t dout() const { return sbase + Cfg<D>::kOffDO; }
   __device__ __forceinline__ uint32_t ds() const { return sbase + Cfg<D>::kOffDS; }
   // -LSE * log2(e) of the stage's 128 query rows, then their D
   __device__ __forceinline__ float* lse2(int s) const {
@@ -161,10 +174,16 @@ struct Smem {
   __device__ __forceinline__ uint32_t dq_full() const { return bar(8); }
   __device__ __forceinline__ uint32_t dq_free() const { return bar(9); }
   __device__ __forceinline__ uint32_t done() const { return bar(10); }
-  // the dQ drain no longer stages in the dS buffer (its reductions have read it)
+  // the dQ GEMM has read dS from shared memory (the next dS may be written)
   __device__ __forceinline__ uint32_t ds_free() const { return bar(11); }
   // dS of the current tile is in shared memory (the dQ GEMM may start)
   __device__ __forceinline__ uint32_t ds_ready() const { return bar(12); }
+  // the element-wise warps hold the tile's S^T in registers (its columns may
+  // take the next tile's S^T)
+  __device__ __forceinline__ uint32_t s_free() const { return bar(13); }
+  // dO of the tile is in shared memory / has been read by dP^T and dV
+  __device__ __forceinline__ uint32_t do_full() const { return bar(14); }
+  __device__ __forceinline__ uint32_t do_empty() const { return bar(15); }
   __device__ __forceinline__ uint32_t* tmem_slot() const {
     return reinterpret_cast<uint32_t*>(base + Cfg<D>::kOffMisc);
   }
@@ -207,17 +226,6 @@ struct Mma {
       Mma<D, KK + 1>::kmajor(d, a_lo, a_hi, b_lo, b_hi, idesc);
     }
   }
-  // A from TMEM (BF16 pairs; queries [64h, 64h+64) in columns [64h, 64h+32)),
-  // B MN-major (rows of 16 queries = 2048 bytes per K step): dV, dK.
-  __device__ __forceinline__ static void tmem_a(uint32_t d, uint32_t a_tmem, uint32_t b_lo,
-                                                uint32_t b_hi, uint32_t idesc, uint32_t acc) {
-    if constexpr (KK < kBlockQ / 16) {
-      constexpr uint32_t a_off = (KK >> 2) * 64 + (KK & 3) * 8;
-      constexpr uint32_t b_off = (KK * 2048) >> 4;
-      mma_ts_imm<a_off, b_off>(d, a_tmem, b_lo, b_hi, idesc, KK == 0 ? acc : 1u);
-      Mma<D, KK + 1>::tmem_a(d, a_tmem, b_lo, b_hi, idesc, acc);
-    }
-  }
   // A and B both MN-major, K = 128 keys, 2048 bytes per K step: dQ = dS K.
   __device__ __forceinline__ static void mnmajor(uint32_t d, uint32_t a_lo, uint32_t a_hi, uint32_t b_lo,
                                                  uint32_t b_hi, uint32_t idesc) {
@@ -225,6 +233,24 @@ struct Mma {
       constexpr uint32_t off = (KK * 2048) >> 4;
       mma_ss_imm<off, off, KK == 0 ? 0u : 1u>(d, a_lo, a_hi, b_lo, b_hi, idesc);
       Mma<D, KK + 1>::mnmajor(d, a_lo, a_hi, b_lo, b_hi, idesc);
+    }
+  }
+};
+
+// A from TMEM, B MN-major (rows of 16 queries = 2048 bytes per K step): dV
+// (SUB = 0, A = P^T) and dK (SUB = 16, A = dS^T).  The element-wise warps write
+// queries [64h + 32c, 64h + 32c + 32) as 16 columns of BF16 pairs at
+// 64h + 32c + SUB, so the K step of queries [16KK, 16KK + 16) reads 8 columns
+// at 64 (KK / 4) + 32 ((KK / 2) % 2) + 8 (KK % 2) + SUB.
+template <int D, int KK, uint32_t SUB>
+struct MmaTs {
+  __device__ __forceinline__ static void run(uint32_t d, uint32_t a_tmem, uint32_t b_lo, uint32_t b_hi,
+                                             uint32_t idesc, uint32_t acc) {
+    if constexpr (KK < kBlockQ / 16) {
+      constexpr uint32_t a_off = (KK >> 2) * 64 + ((KK >> 1) & 1) * 32 + (KK & 1) * 8 + SUB;
+      constexpr uint32_t b_off = (KK * 2048) >> 4;
+      mma_ts_imm<a_off, b_off>(d, a_tmem, b_lo, b_hi, idesc, KK == 0 ? acc : 1u);
+      MmaTs<D, KK + 1, SUB>::run(d, a_tmem, b_lo, b_hi, idesc, acc);
     }
   }
 };
@@ -346,7 +372,7 @@ __device__ __forceinline__ void producer_role(const Smem<D>& sm, const CUtensorM
     }
   }
   bool ok = true;
-  int it = 0;
+  int it = 0, n_q = 0, n_do = 0;  // tiles whose Q / dO loads were issued
   Walk wk;
   walk_start<MASK>(wk, prm, w, w.n_qtiles);
   for (; it < w.n_it; ++it) {
@@ -383,24 +409,33 @@ __device__ __forceinline__ void producer_role(const Smem<D>& sm, const CUtensorM
         dd[r] = in ? prm.dsum[row] : 0.0f;
       }
     }
+    const int qh = w.packed ? h : bh;
     if (lane == 0) {
-      mbar_arrive_expect_tx(sm.q_full(s), 2 * C::kTileBytes);
-      const int qh = w.packed ? h : bh;
+      mbar_arrive_expect_tx(sm.q_full(s), C::kTileBytes);
 #pragma unroll
-      for (int b = 0; b < C::kBoxes; ++b) {
+      for (int b = 0; b < C::kBoxes; ++b)
         load_rows(sm.q(s) + b * C::kBoxBytes, tm_q, b * 64, w.row_q0() + q0, qh, w.packed, sm.q_full(s));
-        load_rows(sm.dout(s) + b * C::kBoxBytes, tm_do, b * 64, w.row_q0() + q0, qh, w.packed,
-                  sm.q_full(s));
-      }
     } else {
       mbar_arrive(sm.q_full(s));
     }
+    ++n_q;
+    // dO, single-buffered: once the previous tile's dV has read it
+    ok = warp_wait(sm.do_empty(), (it & 1) ^ 1u, prm.timeout_ns);
+    if (!ok) break;
+    if (lane == 0) {
+      mbar_arrive_expect_tx(sm.do_full(), C::kTileBytes);
+#pragma unroll
+      for (int b = 0; b < C::kBoxes; ++b)
+        load_rows(sm.dout() + b * C::kBoxBytes, tm_do, b * 64, w.row_q0() + q0, qh, w.packed, sm.do_full());
+    }
+    ++n_do;
   }
-  // never leave with a copy in flight
+  // never leave with a copy in flight: the last two Q loads and the last dO load
   if (lane == 0) {
     mbar_wait(sm.kv_full(), 0, prm.timeout_ns);
-    for (int i = it > 2 ? it - 2 : 0; i < it; ++i)
+    for (int i = n_q > 2 ? n_q - 2 : 0; i < n_q; ++i)
       mbar_wait(sm.q_full(i & 1), (i >> 1) & 1, prm.timeout_ns);
+    if (n_do > 0) mbar_wait(sm.do_full(), (n_do - 1) & 1, prm.timeout_ns);
     if (!ok) atomicOr(&g_status_bwd, kStatusTimeout);
   }
 }
@@ -416,47 +451,65 @@ __device__ __forceinline__ void mma_role(const Smem<D>& sm, uint32_t tmem, const
   constexpr uint32_t id_kv = idesc_bf16_f32(kBlockK, D, false, true);         // dV, dK
   constexpr uint32_t id_q = idesc_bf16_f32(kBlockQ, D, true, true);           // dQ
   const uint64_t dk_ = sdesc_sw128(sm.k(), 16, 1024), dv_ = sdesc_sw128(sm.v(), 16, 1024);
-  const uint64_t dq_ = sdesc_sw128(sm.q(0), 16, 1024), do_ = sdesc_sw128(sm.dout(0), 16, 1024);
+  const uint64_t dq_ = sdesc_sw128(sm.q(0), 16, 1024), do_ = sdesc_sw128(sm.dout(), 16, 1024);
   // MN-major views: Q, dO and K as B operands along d; dS as the A operand
   const uint64_t qmn = sdesc_sw128(sm.q(0), C::kBoxBytes, 1024);
-  const uint64_t domn = sdesc_sw128(sm.dout(0), C::kBoxBytes, 1024);
+  const uint64_t domn = sdesc_sw128(sm.dout(), C::kBoxBytes, 1024);
   const uint64_t kmn = sdesc_sw128(sm.k(), C::kBoxBytes, 1024);
   const uint64_t dsmn = sdesc_sw128(sm.ds(), Cfg<D>::kBoxBytes, 1024);
   auto lo = [](uint64_t x) { return static_cast<uint32_t>(x); };
   auto hi = [](uint64_t x) { return static_cast<uint32_t>(x >> 32); };
   constexpr uint32_t kStageStep = C::kTileBytes >> 4;
 
-  bool ok = mbar_wait(sm.kv_full(), 0, timeout);
-  for (int it = 0; ok && it < w.n_it; ++it) {
-    const int s = it & 1;
-    ok = mbar_wait(sm.q_full(s), (it >> 1) & 1, timeout);
-    if (!ok) break;
+  bool ok = mbar_wait(sm.kv_full(), 0, timeout) && mbar_wait(sm.q_full(0), 0, timeout);
+  if (ok) {
     tc_fence_after();
-    // dP^T = V dO^T (its columns were last read by dK of the previous tile,
-    // issued earlier by this thread: MMAs execute in issue order)
-    Mma<D, 0>::kmajor(tmem + C::kTmemDP, lo(dv_), hi(dv_), lo(do_) + s * kStageStep, hi(do_), id_sq);
+    // the first tile's S^T = K Q^T and dP^T = V dO^T
+    Mma<D, 0>::kmajor(tmem, lo(dk_), hi(dk_), lo(dq_), hi(dq_), id_sq);
+    tc_commit(sm.s_full());
+    ok = mbar_wait(sm.do_full(), 0, timeout);
+  }
+  if (ok) {
+    tc_fence_after();
+    Mma<D, 0>::kmajor(tmem + C::kTmemDP, lo(dv_), hi(dv_), lo(do_), hi(do_), id_sq);
     tc_commit(sm.dp_full());
-    // S^T = K Q^T into the columns of the previous dQ tile, once it is drained
-    if (it > 0) {
-      ok = mbar_wait(sm.dq_free(), (it - 1) & 1, timeout);
+  }
+  for (int it = 0; ok && it < w.n_it; ++it) {
+    const int s = it & 1, sn = s ^ 1;
+    const bool next = it + 1 < w.n_it;
+    if (next) {
+      // the next tile's S^T, as soon as the element-wise warps hold this one's
+      // in registers: it runs while they compute the exponentials
+      ok = mbar_wait(sm.q_full(sn), ((it + 1) >> 1) & 1, timeout) && mbar_wait(sm.s_free(), it & 1, timeout);
       if (!ok) break;
       tc_fence_after();
+      Mma<D, 0>::kmajor(tmem, lo(dk_), hi(dk_), lo(dq_) + sn * kStageStep, hi(dq_), id_sq);
+      tc_commit(sm.s_full());
     }
-    Mma<D, 0>::kmajor(tmem, lo(dk_), hi(dk_), lo(dq_) + s * kStageStep, hi(dq_), id_sq);
-    tc_commit(sm.s_full());
     ok = mbar_wait(sm.p_ready(), it & 1, timeout);
     if (!ok) break;
     tc_fence_after();
     const uint32_t acc = it > 0 ? 1u : 0u;
-    Mma<D, 0>::tmem_a(tmem + C::kTmemDV, tmem, lo(domn) + s * kStageStep, hi(domn), id_kv, acc);
-    Mma<D, 0>::tmem_a(tmem + C::kTmemDK, tmem + C::kTmemDP, lo(qmn) + s * kStageStep, hi(qmn), id_kv,
-                      acc);
+    MmaTs<D, 0, 0>::run(tmem + C::kTmemDV, tmem + C::kTmemDP, lo(domn), hi(domn), id_kv, acc);
+    tc_commit(sm.do_empty());  // dO may be refilled once dV has read it
+    MmaTs<D, 0, 16>::run(tmem + C::kTmemDK, tmem + C::kTmemDP, lo(qmn) + s * kStageStep, hi(qmn), id_kv, acc);
     tc_commit(sm.q_empty(s));
     ok = mbar_wait(sm.ds_ready(), it & 1, timeout);
     if (!ok) break;
     tc_fence_after();
-    Mma<D, 0>::mnmajor(tmem, lo(dsmn), hi(dsmn), lo(kmn), hi(kmn), id_q);
+    // dQ into the dP^T columns, whose P^T and dS^T the two GEMMs above read
+    // first (MMAs from one thread execute in issue order)
+    Mma<D, 0>::mnmajor(tmem + C::kTmemDP, lo(dsmn), hi(dsmn), lo(kmn), hi(kmn), id_q);
     tc_commit(sm.dq_full());
+    tc_commit(sm.ds_free());
+    if (next) {
+      // the next tile's dP^T, once dQ has left those columns and its dO is in
+      ok = mbar_wait(sm.dq_free(), it & 1, timeout) && mbar_wait(sm.do_full(), (it + 1) & 1, timeout);
+      if (!ok) break;
+      tc_fence_after();
+      Mma<D, 0>::kmajor(tmem + C::kTmemDP, lo(dv_), hi(dv_), lo(do_), hi(do_), id_sq);
+      tc_commit(sm.dp_full());
+    }
   }
   tc_commit(sm.done());
   mbar_wait(sm.done(), 0, timeout);
@@ -497,10 +550,20 @@ __device__ __forceinline__ bool softmax_grad_role(const Smem<D>& sm, uint32_t tm
     // below (long complete by now); it cannot run two phases ahead, since the
     // stage is refilled only after this tile's p_ready.
     ok = warp_wait(sm.q_full(s), (it >> 1) & 1, prm.timeout_ns) &&
-         warp_wait(sm.s_full(), it & 1, prm.timeout_ns) &&
-         warp_wait(sm.dp_full(), it & 1, prm.timeout_ns);
+         warp_wait(sm.s_full(), it & 1, prm.timeout_ns);
     if (!ok) break;
     tc_fence_after();
+    // this warp's 64 columns of S^T into registers; then the columns are free
+    // for the next tile's S^T GEMM
+    uint32_t sv[2][32];
+    tmem_ld32(tS, sv[0]);
+    tmem_ld32(tS + 32, sv[1]);
+    tmem_ld_wait();
+    reg_fence32(sv[0]);
+    reg_fence32(sv[1]);
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(sm.s_free());
     const int q_base = wk.t * kBlockQ + c * 64;  // first query of this warp's columns
     // masking: key tail, a band edge crossing this warp's 32 keys x 64 queries,
     // or a key interval meeting the warp's queries
@@ -514,16 +577,9 @@ __device__ __forceinline__ bool softmax_grad_role(const Smem<D>& sm, uint32_t tm
     const float4* nl4 = reinterpret_cast<const float4*>(sm.lse2(s) + c * 64);
     const float4* dd4 = reinterpret_cast<const float4*>(sm.dsum(s) + c * 64);
     const float2 sl2 = make_float2(prm.scale_log2, prm.scale_log2);
-    uint32_t dsk[2][16];  // this thread's dS row (BF16 pairs), written to shared memory last
+    // P = exp2(scale log2(e) S - LSE log2(e)) in fp32, in place of S
 #pragma unroll
     for (int k = 0; k < 2; ++k) {
-      uint32_t sv[32], pv[32];
-      tmem_ld32(tS + 32 * k, sv);
-      tmem_ld32(tP + 32 * k, pv);
-      tmem_ld_wait();
-      reg_fence32(sv);
-      reg_fence32(pv);
-      uint32_t pp[16], dsp[16];
       // the queries of these 32 columns this key is visible to (bit c: query
       // q_base + 32k + c): inside the band key - wr <= q <= key + wl and outside
       // the key's column intervals; one bit test per score below instead of
@@ -539,10 +595,10 @@ __device__ __forceinline__ bool softmax_grad_role(const Smem<D>& sm, uint32_t tm
       }
 #pragma unroll
       for (int g = 0; g < 8; ++g) {  // query columns 32k + 4g .. 32k + 4g + 3
-        const float4 nl = nl4[8 * k + g], dv = dd4[8 * k + g];
-        float2 xa = ffma2(make_float2(__uint_as_float(sv[4 * g]), __uint_as_float(sv[4 * g + 1])), sl2,
+        const float4 nl = nl4[8 * k + g];
+        float2 xa = ffma2(make_float2(__uint_as_float(sv[k][4 * g]), __uint_as_float(sv[k][4 * g + 1])), sl2,
                           make_float2(nl.x, nl.y));
-        float2 xb = ffma2(make_float2(__uint_as_float(sv[4 * g + 2]), __uint_as_float(sv[4 * g + 3])),
+        float2 xb = ffma2(make_float2(__uint_as_float(sv[k][4 * g + 2]), __uint_as_float(sv[k][4 * g + 3])),
                           sl2, make_float2(nl.z, nl.w));
         if (masked) {
           const uint32_t kw = keep >> (4 * g);
@@ -559,6 +615,30 @@ __device__ __forceinline__ bool softmax_grad_role(const Smem<D>& sm, uint32_t tm
           pa = make_float2(ex2_mufu(xa.x), ex2_mufu(xa.y));
           pb = make_float2(ex2_mufu(xb.x), ex2_mufu(xb.y));
         }
+        sv[k][4 * g] = __float_as_uint(pa.x);
+        sv[k][4 * g + 1] = __float_as_uint(pa.y);
+        sv[k][4 * g + 2] = __float_as_uint(pb.x);
+        sv[k][4 * g + 3] = __float_as_uint(pb.y);
+      }
+    }
+    // dS = P (dP - D); P^T and dS^T back into the dP^T columns this warp has
+    // just read, 16 columns each per 32-query chunk
+    ok = warp_wait(sm.dp_full(), it & 1, prm.timeout_ns);
+    if (!ok) break;
+    tc_fence_after();
+    uint32_t dsk[2][16];  // this thread's dS row (BF16 pairs), written to shared memory last
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+      uint32_t pv[32];
+      tmem_ld32(tP + 32 * k, pv);
+      tmem_ld_wait();
+      reg_fence32(pv);
+      uint32_t pp[16];
+#pragma unroll
+      for (int g = 0; g < 8; ++g) {
+        const float4 dv = dd4[8 * k + g];
+        const float2 pa = make_float2(__uint_as_float(sv[k][4 * g]), __uint_as_float(sv[k][4 * g + 1]));
+        const float2 pb = make_float2(__uint_as_float(sv[k][4 * g + 2]), __uint_as_float(sv[k][4 * g + 3]));
         const float2 da = fmul2(pa, fsub2(make_float2(__uint_as_float(pv[4 * g]), __uint_as_float(pv[4 * g + 1])),
                                           make_float2(dv.x, dv.y)));
         const float2 db = fmul2(pb, fsub2(make_float2(__uint_as_float(pv[4 * g + 2]),
@@ -566,22 +646,19 @@ __device__ __forceinline__ bool softmax_grad_role(const Smem<D>& sm, uint32_t tm
                                           make_float2(dv.z, dv.w)));
         pp[2 * g] = pack_bf16x2(pa.x, pa.y);
         pp[2 * g + 1] = pack_bf16x2(pb.x, pb.y);
-        dsp[2 * g] = pack_bf16x2(da.x, da.y);
-        dsp[2 * g + 1] = pack_bf16x2(db.x, db.y);
+        dsk[k][2 * g] = pack_bf16x2(da.x, da.y);
+        dsk[k][2 * g + 1] = pack_bf16x2(db.x, db.y);
       }
-      tmem_st16(tS + 16 * k, pp);
-      tmem_st16(tP + 16 * k, dsp);
-#pragma unroll
-      for (int i = 0; i < 16; ++i) dsk[k][i] = dsp[i];
+      tmem_st16(tP + 32 * k, pp);
+      tmem_st16(tP + 32 * k + 16, dsk[k]);
     }
     // P^T and dS^T are in TMEM: the dV and dK GEMMs may start
     tmem_st_wait();
     tc_fence_before();
     __syncwarp();
     if (lane == 0) mbar_arrive(sm.p_ready());
-    // dS for the dQ GEMM, once the previous dQ tile's reductions have read the
-    // buffer they staged in: key row r of the 64-query block c, 16-byte chunks,
-    // 128-byte swizzle
+    // dS for the dQ GEMM, once the previous dQ GEMM has read the buffer: key
+    // row r of the 64-query block c, 16-byte chunks, 128-byte swizzle
     if (it > 0 && !warp_wait(sm.ds_free(), (it - 1) & 1, prm.timeout_ns)) {
       ok = false;
       break;
@@ -603,20 +680,23 @@ __device__ __forceinline__ bool softmax_grad_role(const Smem<D>& sm, uint32_t tm
 }
 
 // Warps 8-11: dQ tile (queries on the TMEM lanes) -> fp32 accumulator by TMA
-// reduce-add.  Each warp stages its 32 rows, 64 columns at a time, as two
-// 32-column x 32-row boxes (128-byte swizzle) in its 8 KiB of the dS buffer,
-// which the dQ GEMM has finished reading and the next dS is not written until
-// ds_free.  TMEM is released (dq_free) as soon as the last columns are in
-// registers, so the next S^T GEMM overlaps the reductions.
+// reduce-add.  Each warp stages its 32 rows in 32-column x 32-row boxes
+// (128-byte swizzle, 4 KiB) through two alternating slots of its own 8 KiB of
+// staging; a slot is refilled once the reduction issued from it two boxes
+// earlier has read it, so the next reduction is always queued behind the
+// current one, across tiles too.  The reductions are bound by the SM's write
+// path to L2 (about 25 bytes per clock), so they run on their own buffer,
+// overlapping everything else.  TMEM is released (dq_free) as soon as the
+// whole tile is in registers, so the next dP^T GEMM overlaps the reductions.
 template <int D, int MASK>
 __device__ __forceinline__ bool dq_drain_role(const Smem<D>& sm, uint32_t tmem, const CUtensorMap* tm_dq,
                                               const BwdParams& prm, const Work& w) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int q4 = warp & 3;
-  const uint32_t tQ = tmem + (static_cast<uint32_t>(q4 * 32) << 16);
-  uint8_t* stage = sm.base + Cfg<D>::kOffDS + q4 * 8192;
+  const uint32_t tQ = tmem + (static_cast<uint32_t>(q4 * 32) << 16) + Cfg<D>::kTmemDP;
+  uint8_t* stage = sm.base + Cfg<D>::kOffStage + q4 * 8192;
   const uint32_t stage_s = smem_u32(stage);
-  constexpr int kHalves = D / 64;
+  constexpr int kBoxes = D / 32;
   bool ok = true;
   Walk wk;
   walk_start<MASK>(wk, prm, w, w.n_qtiles);
@@ -631,51 +711,36 @@ __device__ __forceinline__ bool dq_drain_role(const Smem<D>& sm, uint32_t tmem, 
     // the next sequence's rows, which leaves them unchanged
     const int row0 = w.row_q0() + wk.t * kBlockQ + q4 * 32;
     // all of this warp's dQ columns into registers, then TMEM is free
-    uint32_t v[kHalves][2][32];
+    uint32_t v[kBoxes][32];
 #pragma unroll
-    for (int hf = 0; hf < kHalves; ++hf) {
-      tmem_ld32(tQ + 64 * hf, v[hf][0]);
-      tmem_ld32(tQ + 64 * hf + 32, v[hf][1]);
-    }
+    for (int bx = 0; bx < kBoxes; ++bx) tmem_ld32(tQ + 32 * bx, v[bx]);
     tmem_ld_wait();
 #pragma unroll
-    for (int hf = 0; hf < kHalves; ++hf) {
-      reg_fence32(v[hf][0]);
-      reg_fence32(v[hf][1]);
-    }
+    for (int bx = 0; bx < kBoxes; ++bx) reg_fence32(v[bx]);
     tc_fence_before();
     __syncwarp();
     if (lane == 0) mbar_arrive(sm.dq_free());
 #pragma unroll
-    for (int hf = 0; hf < kHalves; ++hf) {
-      if (hf > 0) {  // the previous half's reductions must have read the staging
-        if (lane == 0) bulk_wait_group_read0();
-        __syncwarp();
-      }
-      uint8_t* row = stage + lane * 128;
+    for (int bx = 0; bx < kBoxes; ++bx) {
+      const uint32_t slot = static_cast<uint32_t>(bx & 1) * 4096u;
+      // the reduction issued from this slot two boxes ago has read it
+      if (lane == 0) bulk_wait_group_read1();
+      __syncwarp();
+      uint8_t* row = stage + slot + lane * 128;
 #pragma unroll
-      for (int c = 0; c < 8; ++c) {
+      for (int c = 0; c < 8; ++c)
         *reinterpret_cast<uint4*>(row + ((c ^ (lane & 7)) * 16)) =
-            make_uint4(v[hf][0][4 * c], v[hf][0][4 * c + 1], v[hf][0][4 * c + 2], v[hf][0][4 * c + 3]);
-        *reinterpret_cast<uint4*>(row + 4096 + ((c ^ (lane & 7)) * 16)) =
-            make_uint4(v[hf][1][4 * c], v[hf][1][4 * c + 1], v[hf][1][4 * c + 2], v[hf][1][4 * c + 3]);
-      }
+            make_uint4(v[bx][4 * c], v[bx][4 * c + 1], v[bx][4 * c + 2], v[bx][4 * c + 3]);
       fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) {
-        if (w.packed) {
-          tma_reduce_add_3d(tm_dq, stage_s, 64 * hf, qh, row0);
-          tma_reduce_add_3d(tm_dq, stage_s + 4096, 64 * hf + 32, qh, row0);
-        } else {
-          tma_reduce_add_3d(tm_dq, stage_s, 64 * hf, row0, qh);
-          tma_reduce_add_3d(tm_dq, stage_s + 4096, 64 * hf + 32, row0, qh);
-        }
+        if (w.packed)
+          tma_reduce_add_3d(tm_dq, stage_s + slot, 32 * bx, qh, row0);
+        else
+          tma_reduce_add_3d(tm_dq, stage_s + slot, 32 * bx, row0, qh);
         bulk_commit_group();
       }
     }
-    if (lane == 0) bulk_wait_group_read0();
-    __syncwarp();
-    if (lane == 0) mbar_arrive(sm.ds_free());
   }
   if (lane == 0) bulk_wait_group0();  // every reduction complete before the CTA exits
   return ok;
@@ -843,8 +908,8 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       const uint32_t b = sm.bar(i);
       uint32_t count = 1;
       if (b == sm.q_full(0) || b == sm.q_full(1)) count = 32;  // every producer lane
-      if (b == sm.p_ready() || b == sm.ds_ready()) count = 8;
-      if (b == sm.dq_free() || b == sm.ds_free()) count = 4;
+      if (b == sm.p_ready() || b == sm.ds_ready() || b == sm.s_free()) count = 8;
+      if (b == sm.dq_free()) count = 4;
       mbar_init(b, count);
     }
     fence_barrier_init();
@@ -865,16 +930,16 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   tc_fence_after();
   const uint32_t tmem = *sm.tmem_slot();
 
-  // register split of the 512 x 128 launch budget: element-wise warpgroups 144,
-  // the drain 176 (a whole dQ row in registers), load/MMA 48
-  // (2 x 128 x 144 + 128 x 176 + 128 x 48 = 65536)
+  // register split of the 512 x 128 launch budget: element-wise warpgroups 152
+  // (P of 64 queries in fp32 while dP^T is read), the drain 160 (a whole dQ
+  // row in registers), load/MMA 48 (2 x 128 x 152 + 128 x 160 + 128 x 48 = 65536)
   if (warp < kWarpDrain) {
-    setmaxnreg_inc<144>();
+    setmaxnreg_inc<152>();
     bool ok = softmax_grad_role<D, MASK>(sm, tmem, prm, w);
     ok = epilogue<D>(sm, tmem, &tm_dk, &tm_dv, prm, w, ok);
     if (!ok && lane == 0) atomicOr(&g_status_bwd, kStatusTimeout);
   } else if (warp < kWarpLoad) {
-    setmaxnreg_inc<176>();
+    setmaxnreg_inc<160>();
     const bool ok = dq_drain_role<D, MASK>(sm, tmem, &tm_dq, prm, w);
     if (!ok && lane == 0) atomicOr(&g_status_bwd, kStatusTimeout);
   } else {
