@@ -351,6 +351,7 @@ __device__ __forceinline__ void load_rows(uint32_t dst, const CUtensorMap* tm, i
   else tma_load_3d(dst, tm, col, row, head, bar);
 }
 
+
 // ---------------------------------------------------------------------------
 // Producer warp: K, V once; then Q, dO (TMA) and LSE, D (plain loads) per tile.
 // ---------------------------------------------------------------------------
@@ -384,6 +385,16 @@ __device__ __forceinline__ void producer_role(const Smem<D>& sm, const CUtensorM
     const int h = w.hkv * prm.group + wk.hh;  // query head within the batch entry
     const int bh = w.b * prm.H + h;
     const int q0 = wk.t * kBlockQ;
+    const int qh = w.packed ? h : bh;
+    // Q first (its transaction count raised without arriving), then the rows
+    // below, so the copy does not wait behind their global loads; every lane
+    // arrives once its rows are in shared memory
+    if (lane == 0) {
+      mbar_expect_tx(sm.q_full(s), C::kTileBytes);
+#pragma unroll
+      for (int b = 0; b < C::kBoxes; ++b)
+        load_rows(sm.q(s) + b * C::kBoxBytes, tm_q, b * 64, w.row_q0() + q0, qh, w.packed, sm.q_full(s));
+    }
     // -LSE * log2(e) per query row (rows past the sequence: -inf, so P = 0
     // there), and D.  Dense: both [B*H, Nq]; packed: LSE [H, total_q], D
     // [total_q, H].
@@ -409,15 +420,7 @@ __device__ __forceinline__ void producer_role(const Smem<D>& sm, const CUtensorM
         dd[r] = in ? prm.dsum[row] : 0.0f;
       }
     }
-    const int qh = w.packed ? h : bh;
-    if (lane == 0) {
-      mbar_arrive_expect_tx(sm.q_full(s), C::kTileBytes);
-#pragma unroll
-      for (int b = 0; b < C::kBoxes; ++b)
-        load_rows(sm.q(s) + b * C::kBoxBytes, tm_q, b * 64, w.row_q0() + q0, qh, w.packed, sm.q_full(s));
-    } else {
-      mbar_arrive(sm.q_full(s));
-    }
+    mbar_arrive(sm.q_full(s));
     ++n_q;
     // dO, single-buffered: once the previous tile's dV has read it
     ok = warp_wait(sm.do_empty(), (it & 1) ^ 1u, prm.timeout_ns);
