@@ -19,6 +19,7 @@ workload, in the same metric.
 from __future__ import annotations
 
 import argparse
+import datetime
 import hashlib
 import json
 import math
@@ -149,15 +150,21 @@ def recorded_traffic(workload_name, kind="fwd"):
 # nvidia-smi clock sampling during the timed region
 # ---------------------------------------------------------------------------
 class ClockSampler:
-    FIELDS = ["clocks.sm", "clocks.max.sm", "power.draw", "utilization.gpu",
+    """nvidia-smi samples every 20 ms while a region is timed.  Each sample
+    carries nvidia-smi's own timestamp, and the report uses the samples taken
+    within 60 ms of the timed region (all samples if none falls there)."""
+    FIELDS = ["timestamp", "clocks.sm", "clocks.max.sm", "power.draw", "utilization.gpu",
               "clocks_event_reasons.hw_slowdown", "clocks_event_reasons.hw_thermal_slowdown",
               "clocks_event_reasons.sw_thermal_slowdown", "clocks_event_reasons.sw_power_cap"]
     REASONS = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+    INTERVAL_MS = 20
+    MARGIN_S = 0.06
 
     def __init__(self, gpu_id: str):
         self.gpu_id = gpu_id
         self.proc = None
         self.path = None
+        self.t0 = self.t1 = None
 
     def start(self):
         try:
@@ -166,11 +173,53 @@ class ClockSampler:
             self.out = open(self.path, "w")
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", self.gpu_id, f"--query-gpu={','.join(self.FIELDS)}",
-                 "--format=csv,noheader,nounits", "-lms", "100"],
+                 "--format=csv,noheader,nounits", "-lms", str(self.INTERVAL_MS)],
                 stdout=self.out, stderr=subprocess.DEVNULL)
-            time.sleep(0.3)
+            # nvidia-smi's first start on a fresh box can take seconds: wait for
+            # its first row, so a short timed region is not over before sampling
+            t0 = time.time()
+            while time.time() - t0 < 15.0 and os.path.getsize(self.path) == 0 \
+                    and self.proc.poll() is None:
+                time.sleep(0.01)
         except Exception:
             self.proc = None
+
+    def mark_start(self):
+        self.t0 = datetime.datetime.now()
+
+    def mark_end(self):
+        self.t1 = datetime.datetime.now()
+        time.sleep(2 * self.INTERVAL_MS / 1e3)  # a sample after the region's end
+
+    @staticmethod
+    def parse(lines, t0=None, t1=None, margin_s=0.06):
+        """Summary of nvidia-smi CSV rows (the FIELDS order); rows stamped
+        within margin_s of [t0, t1] when there are any."""
+        rows = []
+        for line in lines:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) != len(ClockSampler.FIELDS):
+                continue
+            try:
+                ts = datetime.datetime.strptime(parts[0], "%Y/%m/%d %H:%M:%S.%f")
+                rows.append((ts, float(parts[1]), float(parts[2]), float(parts[3]), float(parts[4]),
+                             parts[5:]))
+            except ValueError:
+                continue
+        if not rows:
+            return None
+        sel = rows
+        if t0 is not None and t1 is not None:
+            m = datetime.timedelta(seconds=margin_s)
+            near = [r for r in rows if t0 - m <= r[0] <= t1 + m]
+            sel = near or rows
+        reasons = sorted({ClockSampler.REASONS[i] for r in sel for i, s in enumerate(r[5])
+                          if s.lower().startswith("active")})
+        return {"sm_mhz": statistics.median(r[1] for r in sel),
+                "sm_max_mhz": max(r[2] for r in sel),
+                "power_w_max": max(r[3] for r in sel),
+                "samples": len(sel), "samples_in_window": len(sel) if sel is not rows else 0,
+                "reasons": reasons}
 
     def stop(self):
         if self.proc is None:
@@ -181,27 +230,10 @@ class ClockSampler:
         except Exception:
             self.proc.kill()
         self.out.close()
-        rows = []
         with open(self.path) as f:
-            for line in f:
-                parts = [p.strip() for p in line.split(",")]
-                if len(parts) != len(self.FIELDS):
-                    continue
-                try:
-                    rows.append((float(parts[0]), float(parts[1]), float(parts[2]), float(parts[3]),
-                                 parts[4:]))
-                except ValueError:
-                    continue
+            lines = f.readlines()
         os.unlink(self.path)
-        if not rows:
-            return None
-        loaded = [r for r in rows if r[3] >= 50.0] or rows
-        reasons = sorted({self.REASONS[i] for r in loaded for i, s in enumerate(r[4])
-                          if s.lower().startswith("active")})
-        return {"sm_mhz": statistics.median(r[0] for r in loaded),
-                "sm_max_mhz": max(r[1] for r in loaded),
-                "power_w_max": max(r[2] for r in loaded),
-                "samples": len(loaded), "reasons": reasons}
+        return self.parse(lines, self.t0, self.t1, self.MARGIN_S)
 
 
 # ---------------------------------------------------------------------------
@@ -508,15 +540,17 @@ def run_ours(args):
     sampler = ClockSampler(gpu_id)
     K = args.steps
     evs = [torch.cuda.Event(enable_timing=True) for _ in range(K + 1)]
+    sampler.start()
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize(dev)
-    sampler.start()
+    sampler.mark_start()
     evs[0].record(stream)
     for i in range(K):
         launch()
         evs[i + 1].record(stream)
     torch.cuda.synchronize(dev)
+    sampler.mark_end()
     if world > 1:
         dist.barrier()
     clocks = sampler.stop()
@@ -761,13 +795,15 @@ def run_ours_bwd(args):
     sampler = ClockSampler("GPU-" + str(torch.cuda.get_device_properties(dev).uuid))
     K = args.steps
     evs = [torch.cuda.Event(enable_timing=True) for _ in range(K + 1)]
-    torch.cuda.synchronize(dev)
     sampler.start()
+    torch.cuda.synchronize(dev)
+    sampler.mark_start()
     evs[0].record(stream)
     for i in range(K):
         launch()
         evs[i + 1].record(stream)
     torch.cuda.synchronize(dev)
+    sampler.mark_end()
     clocks = sampler.stop()
     binding.check(binding.attn_status_sync(sh), "timed region")
     total_ms = evs[0].elapsed_time(evs[K])

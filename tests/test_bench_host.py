@@ -92,3 +92,25 @@ def test_peak_follows_the_timed_window():
     # 148 SMs x 8192 FLOP/clk at 1965 MHz
     assert abs(bench.clock_peak(cool) - 2382.4) < 0.1
     assert bench.clock_peak(None) is None
+
+
+def test_clock_samples_near_the_timed_region():
+    """The clock summary keeps the nvidia-smi rows stamped within the margin of
+    the timed region, and falls back to every row when none is."""
+    import datetime
+    rows = [
+        "2026/12/03 10:00:00.000, 1965, 1965, 300.0, 0, Not Active, Not Active, Not Active, Not Active",
+        "2026/12/03 10:00:00.500, 1600, 1965, 900.0, 100, Not Active, Not Active, Not Active, Active",
+        "2026/12/03 10:00:00.520, 1620, 1965, 910.0, 100, Not Active, Not Active, Not Active, Active",
+        "2026/12/03 10:00:02.000, 1965, 1965, 250.0, 0, Not Active, Not Active, Not Active, Not Active",
+        "garbage line",
+    ]
+    t0 = datetime.datetime(2026, 12, 3, 10, 0, 0, 480000)
+    t1 = datetime.datetime(2026, 12, 3, 10, 0, 0, 500000)
+    c = bench.ClockSampler.parse(rows, t0, t1, 0.06)
+    assert c["samples"] == 2 and c["samples_in_window"] == 2
+    assert c["sm_mhz"] == 1610.0 and c["reasons"] == ["sw_power_cap"] and c["power_w_max"] == 910.0
+    far = datetime.datetime(2026, 12, 3, 11, 0, 0)
+    c = bench.ClockSampler.parse(rows, far, far, 0.06)
+    assert c["samples"] == 4 and c["samples_in_window"] == 0
+    assert bench.ClockSampler.parse(["x"], t0, t1) is None
