@@ -596,24 +596,34 @@ __device__ __forceinline__ void softmax_role(const Smem<D, F8>& sm, uint32_t tme
     if constexpr (MASK == kMaskCols) {
       if (cols_touch(prm, sv.mrow, blk, rw0, rw0 + 32)) {
         masked = true;
-        // lane l reads keys kv0 + 32k + l (coalesced) and turns each into the
-        // set of the warp's 32 rows it is hidden from; ballots transpose those
-        // into per-row words (bit c of row r's word k: key 32k + c)
+        // lane l reads keys kv0 + 32k + l (coalesced).  A 32-key chunk whose
+        // keys all carry the same intervals (a chunk inside one document)
+        // hides a row from all 32 keys or from none, so each lane tests its
+        // own row.  Otherwise each key becomes the set of the warp's 32 rows
+        // it is hidden from, and ballots transpose those into per-row words
+        // (bit c of row r's word k: key 32k + c).
         const int4* cm = prm.colmask + static_cast<size_t>(sv.mrow) * Nk + kv0;
         const int n_in = min(kBlockN, Nk - kv0);
         const int4 none = make_int4(0, 0, 0, 0);
-        uint32_t cb[4];
+        int4 iv[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) iv[k] = 32 * k + lane < n_in ? __ldg(cm + 32 * k + lane) : none;
+        const int row_l = rw0 + lane;
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
-          const int4 iv = 32 * k + lane < n_in ? __ldg(cm + 32 * k + lane) : none;
-          cb[k] = span_bits(iv.x, iv.y, rw0) | span_bits(iv.z, iv.w, rw0);
-        }
+          const int4 i0 = make_int4(__shfl_sync(0xffffffffu, iv[k].x, 0), __shfl_sync(0xffffffffu, iv[k].y, 0),
+                                    __shfl_sync(0xffffffffu, iv[k].z, 0), __shfl_sync(0xffffffffu, iv[k].w, 0));
+          const bool same = iv[k].x == i0.x && iv[k].y == i0.y && iv[k].z == i0.z && iv[k].w == i0.w;
+          if (__all_sync(0xffffffffu, same)) {
+            const bool h = (row_l >= i0.x && row_l < i0.y) || (row_l >= i0.z && row_l < i0.w);
+            hid[k] = h ? 0xffffffffu : 0u;
+          } else {
+            const uint32_t cb = span_bits(iv[k].x, iv[k].y, rw0) | span_bits(iv[k].z, iv[k].w, rw0);
 #pragma unroll
-        for (int rr = 0; rr < 32; ++rr) {
-#pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            const uint32_t w = __ballot_sync(0xffffffffu, (cb[k] >> rr) & 1u);
-            if (lane == rr) hid[k] = w;
+            for (int rr = 0; rr < 32; ++rr) {
+              const uint32_t w = __ballot_sync(0xffffffffu, (cb >> rr) & 1u);
+              if (lane == rr) hid[k] = w;
+            }
           }
         }
       }
