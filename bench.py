@@ -237,6 +237,67 @@ class ClockSampler:
 
 
 # ---------------------------------------------------------------------------
+# End-to-end timing with host buffers
+# ---------------------------------------------------------------------------
+E2E_PATTERN = ("two buffer slots on three streams: step i+1's host-to-device copies overlap "
+               "step i's call and its device-to-host read (PCIe is full duplex)")
+
+
+def pipelined_e2e(comp, slots, n_steps, warmup=2):
+    """Device milliseconds for n_steps end-to-end steps.  Each step copies its
+    inputs from pinned host memory (upload stream), runs the call on `comp`
+    (the stream the C-ABI call is given) and reads its results back to pinned
+    host memory (download stream).  Steps alternate between two slots, each a
+    dict with 'h2d' [(device dst, host src)], 'run' (issues the call on comp)
+    and 'd2h' [(host dst, device src)]; a slot's inputs are rewritten only
+    after the call two steps back has read them, and its outputs only after
+    their read-back."""
+    import torch
+    up, down = torch.cuda.Stream(comp.device), torch.cuda.Stream(comp.device)
+    in_free, out_free = [None, None], [None, None]
+    last = [None]
+
+    def step(i):
+        s = i % 2
+        sl = slots[s]
+        if in_free[s] is not None:
+            up.wait_event(in_free[s])
+        with torch.cuda.stream(up):
+            for dst, src in sl["h2d"]:
+                dst.copy_(src, non_blocking=True)
+        ready = torch.cuda.Event()
+        ready.record(up)
+        comp.wait_event(ready)
+        if out_free[s] is not None:
+            comp.wait_event(out_free[s])
+        sl["run"]()
+        done = torch.cuda.Event()
+        done.record(comp)
+        in_free[s] = done
+        down.wait_event(done)
+        with torch.cuda.stream(down):
+            for dst, src in sl["d2h"]:
+                dst.copy_(src, non_blocking=True)
+        back = torch.cuda.Event()
+        back.record(down)
+        out_free[s] = back
+        last[0] = back
+
+    for i in range(warmup):
+        step(i)
+    torch.cuda.synchronize(comp.device)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(comp)
+    up.wait_event(e0)
+    for i in range(n_steps):
+        step(warmup + i)
+    comp.wait_event(last[0])
+    e1.record(comp)
+    torch.cuda.synchronize(comp.device)
+    return e0.elapsed_time(e1)
+
+
+# ---------------------------------------------------------------------------
 # CPU oracle timing (baseline / reference arm)
 # ---------------------------------------------------------------------------
 def oracle_units(w):
@@ -564,47 +625,39 @@ def run_ours(args):
 
     # end to end through the public API: pinned host inputs -> H2D, attn_fwd, D2H
     hq, hk, hv = (as_tensor(host[x]).pin_memory() for x in "qkv")
-    ho = torch.empty(o.shape, dtype=torch.bfloat16).pin_memory()
-    hl = torch.empty(lse.shape, dtype=torch.float32).pin_memory()
-    qd, kd, vd = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
     hc = host_cu.pin_memory() if w.packed else None
-    cd = torch.empty_like(cu) if w.packed else None
     hm = host_mask.pin_memory() if w.colmask else None
-    md = torch.empty_like(mask) if w.colmask else None
     KE = args.e2e_steps
-
-    def e2e_step():
-        qd.copy_(hq, non_blocking=True)
-        kd.copy_(hk, non_blocking=True)
-        vd.copy_(hv, non_blocking=True)
-        if w.packed:
-            cd.copy_(hc, non_blocking=True)
-        if w.colmask:
-            md.copy_(hm, non_blocking=True)
-        launch(qd, kd, vd, o, lse, cd, md)
-        ho.copy_(o, non_blocking=True)
-        hl.copy_(lse, non_blocking=True)
-
-    for _ in range(2):
-        e2e_step()
-    torch.cuda.synchronize(dev)
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    slots = []
+    for s_ in range(2):
+        qd, kd, vd = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+        od, ld = (o, lse) if s_ == 0 else (torch.empty_like(o), torch.empty_like(lse))
+        cd = torch.empty_like(cu) if w.packed else None
+        md = torch.empty_like(mask) if w.colmask else None
+        ho = torch.empty(o.shape, dtype=torch.bfloat16).pin_memory()
+        hl = torch.empty(lse.shape, dtype=torch.float32).pin_memory()
+        h2d_pairs = [(qd, hq), (kd, hk), (vd, hv)] + ([(cd, hc)] if w.packed else []) + \
+            ([(md, hm)] if w.colmask else [])
+        slots.append({"h2d": h2d_pairs, "d2h": [(ho, od), (hl, ld)],
+                      "run": (lambda a=(qd, kd, vd, od, ld, cd, md): launch(*a))})
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize(dev)
-    e0.record(stream)
-    for _ in range(KE):
-        e2e_step()
-    e1.record(stream)
-    torch.cuda.synchronize(dev)
+    te_ms = pipelined_e2e(stream, slots, KE)
     if world > 1:
         dist.barrier()
     binding.check(binding.attn_status_sync(sh), "e2e region")
-    (te_ms,) = parallel.max_over_ranks([e0.elapsed_time(e1)], dev)
+    # the results read back through both slots equal the device-resident one
+    for sl in slots:
+        for h_, d_ in zip((sl["d2h"][0][0], sl["d2h"][1][0]), (o, lse)):
+            assert torch.equal(h_.view(torch.int16) if h_.dtype == torch.bfloat16 else h_,
+                               d_.cpu().view(torch.int16) if d_.dtype == torch.bfloat16 else d_.cpu()), \
+                "end-to-end read-back differs from the device result"
+    (te_ms,) = parallel.max_over_ranks([te_ms], dev)
     e2e_value = world * w.flops * KE / (te_ms / 1e3) / 1e12
     h2d = sum(x.numel() * x.element_size()
               for x in (hq, hk, hv) + ((hc,) if w.packed else ()) + ((hm,) if w.colmask else ()))
-    d2h = ho.numel() * ho.element_size() + hl.numel() * hl.element_size()
+    d2h = o.numel() * o.element_size() + lse.numel() * lse.element_size()
 
     # rescale events of one launch (outside the timed region): rows whose
     # reference max moved at a KV step after their first
@@ -663,7 +716,7 @@ def run_ours(args):
                                       else "attention kernel")},
         "cpu_baseline": cpu,
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                "steps": KE, "path": f"pinned host Q/K/V{' + offsets' if w.packed else ''}"
+                "steps": KE, "pattern": E2E_PATTERN, "path": f"pinned host Q/K/V{' + offsets' if w.packed else ''}"
                         f"{' + mask' if w.colmask else ''} -> H2D -> "
                         f"{launch_name(w)} (C-ABI) -> D2H of O and LSE"},
         # attn_fwd_colmask launches a summary kernel before the attention kernel
@@ -814,27 +867,23 @@ def run_ours_bwd(args):
     pin = lambda t: t.cpu().pin_memory()  # noqa: E731
     ins = (q, k, v, o, do, lse) + ((cu,) if w.packed else ()) + ((mask,) if w.colmask else ())
     h_in = [pin(t) for t in ins]
-    h_out = [torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in (dq, dk, dv)]
-    d_in = [torch.empty_like(t) for t in ins]
-
-    def e2e_step():
-        for d_, h_ in zip(d_in, h_in):
-            d_.copy_(h_, non_blocking=True)
-        launch(tuple(d_in) + ((None,) if not (w.packed or w.colmask) else ()))
-        for h_, d_ in zip(h_out, (dq, dk, dv)):
-            h_.copy_(d_, non_blocking=True)
-
-    for _ in range(2):
-        e2e_step()
-    torch.cuda.synchronize(dev)
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(args.e2e_steps):
-        e2e_step()
-    e1.record(stream)
-    torch.cuda.synchronize(dev)
+    slots = []
+    for s_ in range(2):
+        d_in = [torch.empty_like(t) for t in ins]
+        d_out = (dq, dk, dv) if s_ == 0 else tuple(torch.empty_like(t) for t in (dq, dk, dv))
+        h_out = [torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in d_out]
+        args_in = tuple(d_in) + ((None,) if not (w.packed or w.colmask) else ())
+        slots.append({"h2d": list(zip(d_in, h_in)), "d2h": list(zip(h_out, d_out)),
+                      "run": (lambda a=args_in, o_=d_out: launch(a, o_))})
+    te_ms = pipelined_e2e(stream, slots, args.e2e_steps)
     binding.check(binding.attn_status_sync(sh), "e2e region")
-    e2e_value = flops * args.e2e_steps / (e0.elapsed_time(e1) / 1e3) / 1e12
+    # dK and dV read back through both slots equal the device-resident ones
+    # (dQ's fp32 reductions may land in another order)
+    for sl in slots:
+        for (h_, _), d_ in zip(sl["d2h"][1:], (dk, dv)):
+            assert torch.equal(h_.view(torch.int16), d_.cpu().view(torch.int16)), \
+                "end-to-end read-back differs from the device result"
+    e2e_value = flops * args.e2e_steps / (te_ms / 1e3) / 1e12
     cpu = None if args.no_cpu_baseline else bwd_cpu_baseline(w, args.cpu_seconds)
     peak, peak_kind = pick_peak(peaks, total_ms, clocks)
     cpk = clock_peak(clocks)
@@ -857,8 +906,8 @@ def run_ours_bwd(args):
         "cpu_baseline": cpu,
         "e2e": {"value": e2e_value, "unit": UNIT,
                 "h2d_bytes_per_step": sum(t.numel() * t.element_size() for t in h_in),
-                "d2h_bytes_per_step": sum(t.numel() * t.element_size() for t in h_out),
-                "steps": args.e2e_steps,
+                "d2h_bytes_per_step": sum(t.numel() * t.element_size() for t in (dq, dk, dv)),
+                "steps": args.e2e_steps, "pattern": E2E_PATTERN,
                 "path": f"pinned host Q/K/V/O/dO/LSE{' + offsets' if w.packed else ''}"
                         f"{' + mask' if w.colmask else ''} -> H2D -> "
                         f"{bwd_launch_name(w)} (C-ABI) -> D2H of dQ/dK/dV"},
