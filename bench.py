@@ -236,6 +236,17 @@ class ClockSampler:
         return self.parse(lines, self.t0, self.t1, self.MARGIN_S)
 
 
+def colmask_launches(w, Hm=1):
+    """Kernels one attn_fwd_colmask call launches with a workspace of
+    attn_colmask_workspace_size bytes: the mask summaries, the CTA plan when it
+    fits (at most 8192 (mask row, 256-row block) units, fewer than 2048 key
+    blocks, Nq <= 4 Nk), and the attention kernel."""
+    units = w.B * Hm * math.ceil(w.Nq / 256)
+    n_kb = math.ceil(w.Nk / 128)
+    fits = 0 < units <= 8192 and n_kb + 1 <= 2048 and w.Nq <= 4 * w.Nk
+    return 3 if fits else 2
+
+
 # ---------------------------------------------------------------------------
 # End-to-end timing with host buffers
 # ---------------------------------------------------------------------------
@@ -712,15 +723,16 @@ def run_ours(args):
                      "frac_of_clock_peak": achieved / cpk if cpk else None,
                      "frac_of_spec": achieved / (SPEC_DENSE_BF16_TFLOPS * ratio),
                      "algorithmic_flops_per_launch": w.flops,
-                     "timed_window": ("mask-summary + attention kernels" if w.colmask
+                     "timed_window": ("mask-summary + CTA-plan + attention kernels" if w.colmask
                                       else "attention kernel")},
         "cpu_baseline": cpu,
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "steps": KE, "pattern": E2E_PATTERN, "path": f"pinned host Q/K/V{' + offsets' if w.packed else ''}"
                         f"{' + mask' if w.colmask else ''} -> H2D -> "
                         f"{launch_name(w)} (C-ABI) -> D2H of O and LSE"},
-        # attn_fwd_colmask launches a summary kernel before the attention kernel
-        "gpu_launches": 2 * K if w.colmask else K,
+        # attn_fwd_colmask launches the mask summaries (and, when it fits, the
+        # CTA plan) before the attention kernel
+        "gpu_launches": colmask_launches(w) * K if w.colmask else K,
         "clocks": clocks,
         "kernel_src_sha": kernel_source_hash("fwd"),
     }

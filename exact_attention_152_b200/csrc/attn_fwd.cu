@@ -190,6 +190,9 @@ struct FwdParams {
   const int4* colsum;
   int mask_heads;    // 1 (one mask for all heads of a batch entry) or H
   int n_kblocks;     // key blocks per head: ceil(Nk / 128)
+  // column-interval mask: CTA order by (mask row, query block) units, most
+  // visited key blocks first (colmask_plan_kernel); null: the order below
+  const int* uperm;
 };
 
 // Where one CTA's sequence lives: lengths, first packed row (packed layout),
@@ -228,6 +231,33 @@ __device__ __forceinline__ bool cols_touch(const FwdParams& prm, int mrow, int b
                                            int r1) {
   const int4 b = __ldg(prm.colsum + (static_cast<size_t>(mrow) * prm.n_kblocks + blk) * 2 + 1);
   return !(b.y <= r0 || b.x >= r1) || !(b.w <= r0 || b.z >= r1);
+}
+
+// KV tiles [j_lo, j_hi) that hold a key of the band for some of the rows of
+// query block qb; a block whose band holds none still visits one tile (fully
+// masked: O = 0, LSE = -inf).
+template <int MASK>
+__device__ __forceinline__ void kv_band_range(const FwdParams& prm, int Nq, int Nk, int qb, int* lo,
+                                              int* hi) {
+  const int n_all = max((Nk + kBlockN - 1) / kBlockN, 1);
+  int j_lo = 0, j_hi = n_all;
+  if (MASK != kMaskNone) {
+    // rows and bounds are below 2^31 and 2^30: the sums stay inside 64 bits
+    const long long r_lo = static_cast<long long>(qb) * kRowsPerCta;
+    const long long r_end = r_lo + kRowsPerCta < Nq ? r_lo + kRowsPerCta : Nq;
+    const long long r_hi = r_end - 1;
+    if (prm.wr < kUnbounded) {
+      const long long last = (r_hi + prm.wr) / kBlockN + 1;
+      if (last < j_hi) j_hi = static_cast<int>(last);
+    }
+    if (prm.wl < kUnbounded && r_lo - prm.wl > 0) j_lo = static_cast<int>((r_lo - prm.wl) / kBlockN);
+    if (j_lo >= j_hi) {
+      j_lo = min(j_lo, n_all - 1);
+      j_hi = j_lo + 1;
+    }
+  }
+  *lo = j_lo;
+  *hi = j_hi;
 }
 
 // Query rows [r0, r1) of a CTA's block qb (r1 clipped to the sequence).
@@ -840,7 +870,15 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   // group starts.
   const int tile = blockIdx.x;
   int bh, qb;
-  if (prm.grouped) {
+  if (MASK == kMaskCols && prm.uperm != nullptr) {
+    // the planned order: CTA i takes unit uperm[i / hper] (a mask row and a
+    // query block) for the i % hper-th query head reading that mask row
+    const int hper = prm.mask_heads == 1 ? prm.H : 1;
+    const int u = __ldg(prm.uperm + blockIdx.x / hper);
+    const int mrow = u / prm.n_qblocks;
+    qb = u % prm.n_qblocks;
+    bh = prm.mask_heads == 1 ? mrow * prm.H + static_cast<int>(blockIdx.x % hper) : mrow;
+  } else if (prm.grouped) {
     const int per_group = prm.hgroup * prm.n_qblocks;
     const int g = tile / per_group, w = tile % per_group;
     const int gsize = min(prm.hgroup, prm.BH - g * prm.hgroup);
@@ -889,23 +927,8 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     // KV tiles that hold a visible key for some row of this block; a block with
     // none (an empty band, an empty key set) still runs one fully masked tile,
     // which yields O = 0 and LSE = -inf.
-    const int n_all = max((sv.Nk + kBlockN - 1) / kBlockN, 1);
-    int j_lo = 0, j_hi = n_all;
-    if (MASK != kMaskNone) {
-      // rows and bounds are below 2^31 and 2^30: the sums stay inside 64 bits
-      const long long r_lo = static_cast<long long>(qb) * kRowsPerCta;
-      const long long r_end = r_lo + kRowsPerCta < sv.Nq ? r_lo + kRowsPerCta : sv.Nq;
-      const long long r_hi = r_end - 1;
-      if (prm.wr < kUnbounded) {
-        const long long last = (r_hi + prm.wr) / kBlockN + 1;
-        if (last < j_hi) j_hi = static_cast<int>(last);
-      }
-      if (prm.wl < kUnbounded && r_lo - prm.wl > 0) j_lo = static_cast<int>((r_lo - prm.wl) / kBlockN);
-      if (j_lo >= j_hi) {
-        j_lo = min(j_lo, n_all - 1);
-        j_hi = j_lo + 1;
-      }
-    }
+    int j_lo, j_hi;
+    kv_band_range<MASK>(prm, sv.Nq, sv.Nk, qb, &j_lo, &j_hi);
     sv.j_lo = j_lo;
     sv.n_kv = j_hi - j_lo;
     sv.mrow = 0;
@@ -1045,6 +1068,75 @@ __global__ void __launch_bounds__(128) colmask_summary_kernel(const int4* __rest
   }
 }
 
+// CTA order for column-interval masks, longest first.  For every (mask row,
+// query block) unit the number of key blocks the attention kernel will visit
+// (the band range and block-summary test of its prologue: one warp per unit,
+// lanes over the blocks), then a counting sort of the units by that number,
+// most first: uperm[i] is the unit of the i-th group of CTAs.  Units with
+// equal counts keep no particular order; the results do not depend on it.
+constexpr int kPlanThreads = 1024;
+constexpr int kPlanMaxUnits = 8192;   // per-unit bins in shared memory
+constexpr int kPlanMaxBins = 2048;    // counts 0 .. n_kblocks
+
+__global__ void __launch_bounds__(kPlanThreads) colmask_plan_kernel(const FwdParams prm, int* __restrict__ uperm,
+                                                                    int n_units) {
+  __shared__ int ubin[kPlanMaxUnits];
+  __shared__ int off[kPlanMaxBins];
+  __shared__ int wsum[kPlanThreads / 32];
+  const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
+  const int n_bins = prm.n_kblocks + 1;
+  for (int i = t; i < n_bins; i += kPlanThreads) off[i] = 0;
+  __syncthreads();
+  for (int u = warp; u < n_units; u += kPlanThreads / 32) {
+    const int mrow = u / prm.n_qblocks, qb = u % prm.n_qblocks;
+    int j_lo, j_hi;
+    kv_band_range<kMaskCols>(prm, prm.Nq, prm.Nk, qb, &j_lo, &j_hi);
+    const int r0 = qb * kRowsPerCta, r1 = cta_row_end(qb, prm.Nq);
+    int cnt = 0;
+    for (int b = j_lo + lane; b < j_hi; b += 32) cnt += cols_hide_all(prm, mrow, b, r0, r1) ? 0 : 1;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) cnt += __shfl_xor_sync(0xffffffffu, cnt, o);
+    if (lane == 0) {
+      const int bin = prm.n_kblocks - min(cnt, prm.n_kblocks);  // most visited first
+      ubin[u] = bin;
+      atomicAdd(&off[bin], 1);
+    }
+  }
+  __syncthreads();
+  // exclusive prefix sum of the bin sizes: thread t owns bins [b0, b1)
+  const int per = (n_bins + kPlanThreads - 1) / kPlanThreads;
+  const int b0 = min(t * per, n_bins), b1 = min(b0 + per, n_bins);
+  int run = 0;
+  for (int b = b0; b < b1; ++b) run += off[b];
+  int incl = run;
+#pragma unroll
+  for (int d = 1; d < 32; d <<= 1) {
+    const int v = __shfl_up_sync(0xffffffffu, incl, d);
+    if (lane >= d) incl += v;
+  }
+  if (lane == 31) wsum[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    const int w = wsum[lane];
+    int wi = w;
+#pragma unroll
+    for (int d = 1; d < 32; d <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, wi, d);
+      if (lane >= d) wi += v;
+    }
+    wsum[lane] = wi - w;
+  }
+  __syncthreads();
+  int base = wsum[warp] + incl - run;
+  for (int b = b0; b < b1; ++b) {
+    const int c = off[b];
+    off[b] = base;
+    base += c;
+  }
+  __syncthreads();
+  for (int u = t; u < n_units; u += kPlanThreads) uperm[atomicAdd(&off[ubin[u]], 1)] = u;
+}
+
 int launch_colmask_summary(const int* mask, void* sum, long long BHm, int Nk, cudaStream_t stream) {
   const int n_kblocks = (Nk + kBlockN - 1) / kBlockN;
   const unsigned grid = static_cast<unsigned>(BHm * n_kblocks);
@@ -1182,9 +1274,17 @@ struct ColMaskArgs {
   size_t workspace_bytes;
 };
 
-size_t colmask_workspace_bytes(long long BHm, int Nk) {
+// Column-interval workspace: the block summaries (required), then room for the
+// CTA plan of colmask_plan_kernel, one int per (mask row, 256-row query block)
+// for up to 4 Nk query rows (a call whose plan does not fit keeps the fixed
+// CTA order).
+size_t colmask_summary_bytes(long long BHm, int Nk) {
   const long long n_kblocks = (static_cast<long long>(Nk) + kBlockN - 1) / kBlockN;
   return static_cast<size_t>(BHm * n_kblocks) * 2 * sizeof(int4);
+}
+size_t colmask_workspace_bytes(long long BHm, int Nk) {
+  const long long plan_units = BHm * ((4LL * Nk + kRowsPerCta - 1) / kRowsPerCta);
+  return colmask_summary_bytes(BHm, Nk) + ((static_cast<size_t>(plan_units) * 4 + 15) & ~static_cast<size_t>(15));
 }
 
 int fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
@@ -1216,11 +1316,17 @@ int fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, i
   if (n_qblocks * BH > 0x7fffffffLL) return ATTN_ERR_INVALID_ARG;
   long long BHm = 0;
   size_t mask_bytes = 0, ws_need = 0;
+  bool plan = false;  // longest-first CTA order (colmask_plan_kernel)
   if (cm) {
     if (cm->Hm != 1 && cm->Hm != H) return ATTN_ERR_INVALID_ARG;
     BHm = static_cast<long long>(B) * cm->Hm;
     mask_bytes = static_cast<size_t>(BHm) * Nk * sizeof(int4);
-    ws_need = colmask_workspace_bytes(BHm, Nk);
+    ws_need = colmask_summary_bytes(BHm, Nk);
+    const long long units = BHm * n_qblocks;
+    const long long n_kb = (static_cast<long long>(Nk) + kBlockN - 1) / kBlockN;
+    plan = units > 0 && units <= kPlanMaxUnits && n_kb + 1 <= kPlanMaxBins &&
+           cm->workspace_bytes >= ws_need + static_cast<size_t>(units) * 4;
+    if (plan) ws_need += static_cast<size_t>(units) * 4;  // the region written
     if (Nk > 0 && (!cm->mask || !cm->workspace)) return ATTN_ERR_INVALID_ARG;
     if (misaligned(cm->mask, 16) || misaligned(cm->workspace, 16)) return ATTN_ERR_INVALID_ARG;
     if (cm->workspace_bytes < ws_need) return ATTN_ERR_INVALID_ARG;
@@ -1274,6 +1380,13 @@ int fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, i
     prm.n_kblocks = (Nk + kBlockN - 1) / kBlockN;
     const int rc2 = launch_colmask_summary(cm->mask, cm->workspace, BHm, Nk, stream);
     if (rc2 != ATTN_OK) return rc2;
+    if (plan) {
+      int* uperm = reinterpret_cast<int*>(static_cast<uint8_t*>(cm->workspace) + colmask_summary_bytes(BHm, Nk));
+      colmask_plan_kernel<<<1, kPlanThreads, 0, stream>>>(prm, uperm, static_cast<int>(BHm * n_qblocks));
+      const cudaError_t e = cudaGetLastError();
+      if (e != cudaSuccess) return cuda_fail(e, "colmask_plan_kernel launch");
+      prm.uperm = uperm;
+    }
   }
   return launch_any(d, exp_mode, tq, tk, tv, to, prm, stream);
 }

@@ -131,15 +131,21 @@ int attn_fwd_window(const void *q, const void *k, const void *v, void *o, float 
  *   mask : DEVICE int32 [B, Hm, Nk, 4], each key's (lo1, hi1, lo2, hi2), 16-byte
  *          aligned; Hm == 1 (one mask per batch entry, shared by all heads) or
  *          Hm == H (one per query head).  Read only.
- *   workspace : DEVICE, 16-byte aligned, at least
- *          attn_colmask_workspace_size(B, Hm, Nk) bytes, owned by the caller;
- *          overwritten with per-128-key-block summaries of the mask, so it may
- *          not overlap any other argument.  Calls on different streams need
- *          different workspaces.
- * The call launches two kernels on `stream`: the block summaries, then the
- * attention kernel, which skips every 128-key block that hides all 256 query
- * rows of a CTA and masks element-wise only in blocks whose intervals meet a
- * warp's 32 rows.  Errors as attn_fwd_gqa, plus ATTN_ERR_INVALID_ARG for a NULL
+ *   workspace : DEVICE, 16-byte aligned, owned by the caller; give it
+ *          attn_colmask_workspace_size(B, Hm, Nk) bytes.  The call overwrites
+ *          it with per-128-key-block summaries of the mask (32 bytes per mask
+ *          row and key block: the minimum accepted) and, where the workspace
+ *          has room for one int per mask row and 256-row query block (the size
+ *          function allows for Nq <= 4 Nk; up to 8192 such units and 2047 key
+ *          blocks), with an
+ *          order of the attention kernel's CTAs.  It may not overlap any other
+ *          argument.  Calls on different streams need different workspaces.
+ * The call launches two or three kernels on `stream`: the block summaries;
+ * when the workspace has room for it, a one-CTA kernel that orders the query
+ * blocks by the number of key blocks they visit, longest first (the order
+ * changes no result); then the attention kernel, which skips every 128-key
+ * block that hides all 256 query rows of a CTA and masks element-wise only in
+ * blocks whose intervals meet a warp's 32 rows.  Errors as attn_fwd_gqa, plus ATTN_ERR_INVALID_ARG for a NULL
  * or misaligned mask or workspace, a workspace that is too small or overlaps
  * another argument, or Hm not in {1, H}, and ATTN_ERR_UNSUPPORTED for more than
  * 65536 key blocks of 128 (8M keys: the kernel keeps one bit per key block).

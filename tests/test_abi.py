@@ -126,8 +126,11 @@ def test_colmask_validation():
     sizes = (1, 4, 2, 8, 8, 64, 0.1, 0)            # B, H, Hkv, Nq, Nk, d, scale, causal
     M, WS = ALIGNED * 40, ALIGNED * 48
     need = binding.attn_colmask_workspace_size(1, 1, 8)
-    assert need == 32                              # one key block: two int4 summaries
-    assert binding.attn_colmask_workspace_size(2, 4, 129) == 2 * 4 * 2 * 32
+    # one key block: two int4 summaries (32 bytes, the minimum), then the CTA
+    # plan's room: one int per mask row and 256-row block of up to 4 Nk query
+    # rows, padded to 16 bytes
+    assert need == 32 + 16
+    assert binding.attn_colmask_workspace_size(2, 4, 129) == 2 * 4 * 2 * 32 + 2 * 4 * 3 * 4
     assert binding.attn_colmask_workspace_size(-1, 1, 8) == 0
 
     def call(ptrs=P, sz=sizes, mask=M, hm=1, ws=WS, ws_bytes=need):
@@ -138,7 +141,7 @@ def test_colmask_validation():
     assert call(ws=None) == 1
     assert call(mask=M + 4) == 1                   # misaligned mask
     assert call(ws=WS + 8) == 1                    # misaligned workspace
-    assert call(ws_bytes=need - 16) == 1           # workspace too small
+    assert call(ws_bytes=32 - 16) == 1             # workspace below the summaries
     assert call(ws=ALIGNED * 16) == 1              # workspace inside o
     assert call(ws=M) == 1                         # workspace over the mask
     assert call(mask=ALIGNED * 16) == 1            # mask inside o

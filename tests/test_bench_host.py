@@ -114,3 +114,14 @@ def test_clock_samples_near_the_timed_region():
     c = bench.ClockSampler.parse(rows, far, far, 0.06)
     assert c["samples"] == 4 and c["samples_in_window"] == 0
     assert bench.ClockSampler.parse(["x"], t0, t1) is None
+
+
+def test_colmask_launch_count():
+    """The document workload's calls launch the mask summaries, the CTA plan
+    and the attention kernel; a problem with more units than the plan holds
+    launches two kernels."""
+    import types
+    w = WORKLOADS["docs_b2h16n8k_d128_causal"]
+    assert bench.colmask_launches(w) == 3
+    big = types.SimpleNamespace(B=64, Nq=65536, Nk=65536)
+    assert bench.colmask_launches(big) == 2
