@@ -239,11 +239,11 @@ class ClockSampler:
 def colmask_launches(w, Hm=1):
     """Kernels one attn_fwd_colmask call launches with a workspace of
     attn_colmask_workspace_size bytes: the mask summaries, the CTA plan when it
-    fits (at most 8192 (mask row, 256-row block) units, fewer than 2048 key
-    blocks, Nq <= 4 Nk), and the attention kernel."""
+    fits (at most 8192 (mask row, 256-row block) units, mask rows x (key
+    blocks + 1) at most 4096, Nq <= 4 Nk), and the attention kernel."""
     units = w.B * Hm * math.ceil(w.Nq / 256)
     n_kb = math.ceil(w.Nk / 128)
-    fits = 0 < units <= 8192 and n_kb + 1 <= 2048 and w.Nq <= 4 * w.Nk
+    fits = 0 < units <= 8192 and w.B * Hm * (n_kb + 1) <= 4096 and w.Nq <= 4 * w.Nk
     return 3 if fits else 2
 
 

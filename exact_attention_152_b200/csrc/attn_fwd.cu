@@ -1068,23 +1068,26 @@ __global__ void __launch_bounds__(128) colmask_summary_kernel(const int4* __rest
   }
 }
 
-// CTA order for column-interval masks, longest first.  For every (mask row,
-// query block) unit the number of key blocks the attention kernel will visit
-// (the band range and block-summary test of its prologue: one warp per unit,
-// lanes over the blocks), then a counting sort of the units by that number,
-// most first: uperm[i] is the unit of the i-th group of CTAs.  Units with
-// equal counts keep no particular order; the results do not depend on it.
+// CTA order for column-interval masks, longest first within each mask row.
+// For every (mask row, query block) unit the number of key blocks the
+// attention kernel will visit (the band range and block-summary test of its
+// prologue: one warp per unit, lanes over the blocks), then a counting sort of
+// the units by (mask row, that number, most first): uperm[i] is the unit of
+// the i-th group of CTAs.  Keeping the mask rows apart keeps the K/V of one
+// batch entry's heads (mask row shared by all heads) or of one head (a mask
+// per head) in flight together, so L2 holds them.  Units of equal key keep
+// no particular order; the results do not depend on it.
 constexpr int kPlanThreads = 1024;
 constexpr int kPlanMaxUnits = 8192;   // per-unit bins in shared memory
-constexpr int kPlanMaxBins = 2048;    // counts 0 .. n_kblocks
+constexpr int kPlanMaxBins = 4096;    // mask rows x (counts 0 .. n_kblocks)
 
 __global__ void __launch_bounds__(kPlanThreads) colmask_plan_kernel(const FwdParams prm, int* __restrict__ uperm,
                                                                     int n_units) {
-  __shared__ int ubin[kPlanMaxUnits];
+  __shared__ uint16_t ubin[kPlanMaxUnits];
   __shared__ int off[kPlanMaxBins];
   __shared__ int wsum[kPlanThreads / 32];
   const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
-  const int n_bins = prm.n_kblocks + 1;
+  const int n_bins = (n_units / prm.n_qblocks) * (prm.n_kblocks + 1);
   for (int i = t; i < n_bins; i += kPlanThreads) off[i] = 0;
   __syncthreads();
   for (int u = warp; u < n_units; u += kPlanThreads / 32) {
@@ -1097,8 +1100,9 @@ __global__ void __launch_bounds__(kPlanThreads) colmask_plan_kernel(const FwdPar
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) cnt += __shfl_xor_sync(0xffffffffu, cnt, o);
     if (lane == 0) {
-      const int bin = prm.n_kblocks - min(cnt, prm.n_kblocks);  // most visited first
-      ubin[u] = bin;
+      // mask row first, then most visited first
+      const int bin = mrow * (prm.n_kblocks + 1) + prm.n_kblocks - min(cnt, prm.n_kblocks);
+      ubin[u] = static_cast<uint16_t>(bin);
       atomicAdd(&off[bin], 1);
     }
   }
@@ -1324,7 +1328,7 @@ int fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, i
     ws_need = colmask_summary_bytes(BHm, Nk);
     const long long units = BHm * n_qblocks;
     const long long n_kb = (static_cast<long long>(Nk) + kBlockN - 1) / kBlockN;
-    plan = units > 0 && units <= kPlanMaxUnits && n_kb + 1 <= kPlanMaxBins &&
+    plan = units > 0 && units <= kPlanMaxUnits && BHm * (n_kb + 1) <= kPlanMaxBins &&
            cm->workspace_bytes >= ws_need + static_cast<size_t>(units) * 4;
     if (plan) ws_need += static_cast<size_t>(units) * 4;  // the region written
     if (Nk > 0 && (!cm->mask || !cm->workspace)) return ATTN_ERR_INVALID_ARG;

@@ -136,14 +136,14 @@ int attn_fwd_window(const void *q, const void *k, const void *v, void *o, float 
  *          it with per-128-key-block summaries of the mask (32 bytes per mask
  *          row and key block: the minimum accepted) and, where the workspace
  *          has room for one int per mask row and 256-row query block (the size
- *          function allows for Nq <= 4 Nk; up to 8192 such units and 2047 key
- *          blocks), with an
+ *          function allows for Nq <= 4 Nk; up to 8192 such units, and mask
+ *          rows x (key blocks + 1) up to 4096), with an
  *          order of the attention kernel's CTAs.  It may not overlap any other
  *          argument.  Calls on different streams need different workspaces.
  * The call launches two or three kernels on `stream`: the block summaries;
  * when the workspace has room for it, a one-CTA kernel that orders the query
- * blocks by the number of key blocks they visit, longest first (the order
- * changes no result); then the attention kernel, which skips every 128-key
+ * blocks of each mask row by the number of key blocks they visit, longest
+ * first (the order changes no result); then the attention kernel, which skips every 128-key
  * block that hides all 256 query rows of a CTA and masks element-wise only in
  * blocks whose intervals meet a warp's 32 rows.  Errors as attn_fwd_gqa, plus ATTN_ERR_INVALID_ARG for a NULL
  * or misaligned mask or workspace, a workspace that is too small or overlaps
