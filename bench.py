@@ -247,6 +247,20 @@ def colmask_launches(w, Hm=1):
     return 3 if fits else 2
 
 
+def bwd_colmask_launches(w):
+    """Kernels one attn_bwd_colmask call launches with a workspace of
+    attn_bwd_colmask_workspace_size bytes: row sums, mask summaries, the CTA
+    plan when it fits (at most 8192 CTAs, groups of key/value heads x (query
+    tiles per CTA + 1) at most 4096 bins), the main kernel, dQ rounding."""
+    hkv, group = w.kv_heads, w.H // w.kv_heads
+    n_kb, n_qt = math.ceil(w.Nk / 128), math.ceil(w.Nq / 128)
+    per_kv = group * w.Nq * w.d * 8
+    g = max([c for c in range(1, hkv + 1) if hkv % c == 0 and c * per_kv <= 48 << 20] or [1])
+    units = w.B * hkv * n_kb
+    bins = math.ceil(w.B * hkv / g) * (group * n_qt + 1)
+    return 5 if units <= 8192 and bins <= 4096 else 4
+
+
 # ---------------------------------------------------------------------------
 # End-to-end timing with host buffers
 # ---------------------------------------------------------------------------
@@ -924,7 +938,7 @@ def run_ours_bwd(args):
                         f"{' + mask' if w.colmask else ''} -> H2D -> "
                         f"{bwd_launch_name(w)} (C-ABI) -> D2H of dQ/dK/dV"},
         # row sums, main kernel, dQ rounding (+ the mask summaries for column intervals)
-        "gpu_launches": (4 if w.colmask else 3) * K,
+        "gpu_launches": (bwd_colmask_launches(w) if w.colmask else 3) * K,
         "clocks": clocks,
         "kernel_src_sha": kernel_source_hash("bwd"),
     }

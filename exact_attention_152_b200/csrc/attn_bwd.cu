@@ -143,6 +143,9 @@ struct BwdParams {
   const int4* colmask;
   const int4* colsum;
   int mask_heads;      // 1 or H
+  // column intervals: CTA order, longest first within groups of key/value
+  // heads (colmask_bwd_plan_kernel); null: the order of blockIdx
+  const int* uperm;
   uint64_t timeout_ns;
   int Nq, Nk, H, group, n_kblocks, n_qtiles;  // packed: Nq, Nk = total_q, total_k
   int wl, wr;          // key band i - wl <= j <= i + wr (kUnbounded: no bound)
@@ -353,6 +356,43 @@ __device__ __forceinline__ void load_rows(uint32_t dst, const CUtensorMap* tm, i
 
 
 // ---------------------------------------------------------------------------
+// The query tiles a CTA iterates over (w.bh_kv, w.j, w.b, w.hkv and the packed
+// fields set): with a key band, the tiles whose queries i see a key j of the
+// block, i - wl <= j <= i + wr; with column intervals, those minus the tiles
+// every key of the block hides, per query head of the group.  A block no
+// query sees still runs one fully masked tile, so dK = dV = 0 come out of TMEM.
+template <int MASK>
+__device__ __forceinline__ void work_extent(const BwdParams& prm, Work& w, int n_qtiles) {
+  w.n_qtiles = n_qtiles;
+  w.force = false;
+  w.i_lo = 0;
+  w.tiles_per_head = n_qtiles;
+  if (MASK != kMaskNone) {
+    const long long j0 = static_cast<long long>(w.j) * kBlockK;
+    long long lo = 0, hi = n_qtiles - 1;
+    if (prm.wr < kUnbounded && j0 - prm.wr > 0) lo = (j0 - prm.wr) / kBlockQ;
+    if (prm.wl < kUnbounded) {
+      const long long last = (j0 + kBlockK - 1 + prm.wl) / kBlockQ;
+      if (last < hi) hi = last;
+    }
+    if (lo > hi) lo = hi = (lo < n_qtiles - 1 ? lo : n_qtiles - 1);
+    w.i_lo = static_cast<int>(lo);
+    w.tiles_per_head = static_cast<int>(hi - lo + 1);
+  }
+  w.n_it = prm.group * w.tiles_per_head;
+  if constexpr (MASK == kMaskCols) {
+    const int i_hi = w.i_lo + w.tiles_per_head - 1;
+    int n = 0;
+    Walk k;
+    for (k.hh = 0; k.hh < prm.group; ++k.hh) {
+      walk_head(k, prm, w, n_qtiles);
+      n += visible_count(k, w.i_lo, i_hi);
+    }
+    w.force = n == 0;
+    w.n_it = n > 0 ? n : 1;
+  }
+}
+
 // Producer warp: K, V once; then Q, dO (TMA) and LSE, D (plain loads) per tile.
 // ---------------------------------------------------------------------------
 template <int D, int MASK>
@@ -840,8 +880,10 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   Work w;
-  w.bh_kv = blockIdx.x / prm.n_kblocks;
-  w.j = blockIdx.x % prm.n_kblocks;
+  const int cta = (MASK == kMaskCols && prm.uperm != nullptr) ? __ldg(prm.uperm + blockIdx.x)
+                                                              : static_cast<int>(blockIdx.x);
+  w.bh_kv = cta / prm.n_kblocks;
+  w.j = cta % prm.n_kblocks;
   const int hkv_per_b = prm.H / prm.group;
   w.b = w.bh_kv / hkv_per_b;
   w.hkv = w.bh_kv % hkv_per_b;
@@ -871,40 +913,7 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   // query tiles (packed: at least one -- a sequence without queries still runs
   // one fully masked tile, so dK = dV = 0 come out of TMEM)
   const int n_qtiles = PACKED ? (w.Nq > 0 ? (w.Nq + kBlockQ - 1) / kBlockQ : 1) : prm.n_qtiles;
-  // query tiles that can see a key of this block: i - wl <= j <= i + wr for
-  // some key j in [j0, j0 + 127] and query i of the tile; a block no query
-  // sees still runs one fully masked tile, so dK = dV = 0 come out of TMEM
-  w.n_qtiles = n_qtiles;
-  w.force = false;
-  w.i_lo = 0;
-  w.tiles_per_head = n_qtiles;
-  if (MASK != kMaskNone) {
-    const long long j0 = static_cast<long long>(w.j) * kBlockK;
-    long long lo = 0, hi = n_qtiles - 1;
-    if (prm.wr < kUnbounded && j0 - prm.wr > 0) lo = (j0 - prm.wr) / kBlockQ;
-    if (prm.wl < kUnbounded) {
-      const long long last = (j0 + kBlockK - 1 + prm.wl) / kBlockQ;
-      if (last < hi) hi = last;
-    }
-    if (lo > hi) lo = hi = (lo < n_qtiles - 1 ? lo : n_qtiles - 1);
-    w.i_lo = static_cast<int>(lo);
-    w.tiles_per_head = static_cast<int>(hi - lo + 1);
-  }
-  w.n_it = prm.group * w.tiles_per_head;
-  if constexpr (MASK == kMaskCols) {
-    // visible (head, tile) pairs: per head, the band's tiles minus the ones
-    // every key of this block hides; none at all: one fully masked tile, so
-    // dK = dV = 0 come out of TMEM
-    const int i_hi = w.i_lo + w.tiles_per_head - 1;
-    int n = 0;
-    Walk k;
-    for (k.hh = 0; k.hh < prm.group; ++k.hh) {
-      walk_head(k, prm, w, n_qtiles);
-      n += visible_count(k, w.i_lo, i_hi);
-    }
-    w.force = n == 0;
-    w.n_it = n > 0 ? n : 1;
-  }
+  work_extent<MASK>(prm, w, n_qtiles);
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < C::kNumBars; ++i) {
@@ -983,6 +992,76 @@ __global__ void row_dot_kernel(const __nv_bfloat16* __restrict__ o, const __nv_b
     for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
     if (lane == 0) dsum[row] = acc;
   }
+}
+
+// CTA order for column intervals: for every CTA (key/value head, key block)
+// the query tiles it will visit (work_extent, as its prologue computes it),
+// then a counting sort by (group of hgroup key/value heads, that number, most
+// first): uperm[i] is the CTA index the i-th launched CTA takes.  A group's
+// Q, dO and dQ accumulator are sized to stay in L2 together; longest first
+// within it evens out the end of the launch.  CTAs of equal key keep no
+// particular order; the results do not depend on it.  One CTA.
+constexpr int kPlanThreads = 1024;
+constexpr int kPlanMaxUnits = 8192;
+constexpr int kPlanMaxBins = 4096;
+
+__global__ void __launch_bounds__(kPlanThreads) colmask_bwd_plan_kernel(const BwdParams prm, int* __restrict__ uperm,
+                                                                        int n_units, int hgroup, int max_n) {
+  __shared__ uint16_t ubin[kPlanMaxUnits];
+  __shared__ int off[kPlanMaxBins];
+  __shared__ int wsum[kPlanThreads / 32];
+  const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
+  const int n_bh = n_units / prm.n_kblocks;
+  const int n_bins = ((n_bh + hgroup - 1) / hgroup) * (max_n + 1);
+  for (int i = t; i < n_bins; i += kPlanThreads) off[i] = 0;
+  __syncthreads();
+  const int hkv_per_b = prm.H / prm.group;
+  for (int u = t; u < n_units; u += kPlanThreads) {
+    Work w;
+    w.bh_kv = u / prm.n_kblocks;
+    w.j = u % prm.n_kblocks;
+    w.b = w.bh_kv / hkv_per_b;
+    w.hkv = w.bh_kv % hkv_per_b;
+    w.packed = false;
+    w.Nq = w.Nk = w.q0 = w.k0 = 0;
+    work_extent<kMaskCols>(prm, w, prm.n_qtiles);
+    const int bin = (w.bh_kv / hgroup) * (max_n + 1) + max_n - min(w.n_it, max_n);
+    ubin[u] = static_cast<uint16_t>(bin);
+    atomicAdd(&off[bin], 1);
+  }
+  __syncthreads();
+  // exclusive prefix sum of the bin sizes: thread t owns bins [b0, b1)
+  const int per = (n_bins + kPlanThreads - 1) / kPlanThreads;
+  const int b0 = min(t * per, n_bins), b1 = min(b0 + per, n_bins);
+  int run = 0;
+  for (int b = b0; b < b1; ++b) run += off[b];
+  int incl = run;
+#pragma unroll
+  for (int d = 1; d < 32; d <<= 1) {
+    const int v = __shfl_up_sync(0xffffffffu, incl, d);
+    if (lane >= d) incl += v;
+  }
+  if (lane == 31) wsum[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    const int w = wsum[lane];
+    int wi = w;
+#pragma unroll
+    for (int d = 1; d < 32; d <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, wi, d);
+      if (lane >= d) wi += v;
+    }
+    wsum[lane] = wi - w;
+  }
+  __syncthreads();
+  int base = wsum[warp] + incl - run;
+  for (int b = b0; b < b1; ++b) {
+    const int c = off[b];
+    off[b] = base;
+    base += c;
+  }
+  __syncthreads();
+  for (int u = t; u < n_units; u += kPlanThreads) uperm[atomicAdd(&off[ubin[u]], 1)] = u;
 }
 
 // dQ = BF16(scale * accumulator), 4 elements per thread per step.
@@ -1078,8 +1157,14 @@ struct ColMaskArgs {
   int Hm;
 };
 
+// Column intervals: attn_bwd's workspace, the block summaries (together the
+// minimum), then room for the CTA plan, one int per (head, key block) (an
+// upper bound: the CTAs are per key/value head).
 size_t colmask_workspace_bytes(long long BH, long long Nq, int d, long long BHm, long long Nk) {
   return align256(workspace_bytes(BH, Nq, d)) + static_cast<size_t>(BHm * ((Nk + kBlockK - 1) / kBlockK)) * 32;
+}
+size_t colmask_plan_bytes(long long BH, long long Nk) {
+  return (static_cast<size_t>(BH * ((Nk + kBlockK - 1) / kBlockK)) * 4 + 15) & ~static_cast<size_t>(15);
 }
 
 int bwd_impl(const void* q, const void* k, const void* v, const void* o, const void* dout,
@@ -1101,8 +1186,30 @@ int bwd_impl(const void* q, const void* k, const void* v, const void* o, const v
     return ATTN_ERR_INVALID_ARG;
   if (cm && cm->Hm != 1 && cm->Hm != H) return ATTN_ERR_INVALID_ARG;
   const long long BHm = cm ? static_cast<long long>(B) * cm->Hm : 0;
-  const size_t need = cm ? colmask_workspace_bytes(BH, Nq, d, BHm, Nk) : workspace_bytes(BH, Nq, d);
+  size_t need = cm ? colmask_workspace_bytes(BH, Nq, d, BHm, Nk) : workspace_bytes(BH, Nq, d);
   if (any_q && any_k && (!workspace || ws_bytes < need)) return ATTN_ERR_INVALID_ARG;
+  // column intervals: the longest-first CTA plan when the workspace has room for it
+  int plan_hgroup = 0, plan_max_n = 0;
+  long long plan_units = 0;
+  if (cm && any_q && any_k) {
+    const long long n_kb = (static_cast<long long>(Nk) + kBlockK - 1) / kBlockK;
+    const long long n_qt = (static_cast<long long>(Nq) + kBlockQ - 1) / kBlockQ;
+    const long long group = H / Hkv, hkv_per_b = Hkv;
+    // key/value heads per group: the largest divisor of a batch entry's whose
+    // query heads' Q, dO (BF16) and fp32 dQ accumulator fit in ~48 MiB
+    const long long per_kv = group * static_cast<long long>(Nq) * d * 8;
+    long long g = 1;
+    for (long long c = 1; c <= hkv_per_b; ++c)
+      if (hkv_per_b % c == 0 && c * per_kv <= (48LL << 20)) g = c;
+    plan_units = BHkv * n_kb;
+    const long long max_n = group * n_qt;
+    const long long bins = ((BHkv + g - 1) / g) * (max_n + 1);
+    if (plan_units <= kPlanMaxUnits && bins <= kPlanMaxBins && ws_bytes >= need + plan_units * 4) {
+      plan_hgroup = static_cast<int>(g);
+      plan_max_n = static_cast<int>(max_n);
+      need += static_cast<size_t>(plan_units) * 4;  // the region written
+    }
+  }
   if (cm && any_k && (!cm->mask || misaligned(cm->mask, 16))) return ATTN_ERR_INVALID_ARG;
   if (misaligned(q, 16) || misaligned(k, 16) || misaligned(v, 16) || misaligned(o, 16) ||
       misaligned(dout, 16) || misaligned(dq, 16) || misaligned(dk, 16) || misaligned(dv, 16) ||
@@ -1177,6 +1284,14 @@ int bwd_impl(const void* q, const void* k, const void* v, const void* o, const v
     prm.mask_heads = cm->Hm;
     rc = launch_colmask_summary(cm->mask, sum, BHm, Nk, stream);
     if (rc != ATTN_OK) return rc;
+    if (plan_hgroup > 0) {
+      int* uperm = reinterpret_cast<int*>(static_cast<uint8_t*>(sum) + static_cast<size_t>(BHm * n_kblocks) * 32);
+      colmask_bwd_plan_kernel<<<1, kPlanThreads, 0, stream>>>(prm, uperm, static_cast<int>(plan_units), plan_hgroup,
+                                                              plan_max_n);
+      const cudaError_t pe = cudaGetLastError();
+      if (pe != cudaSuccess) return cuda_fail(pe, "colmask_bwd_plan_kernel launch");
+      prm.uperm = uperm;
+    }
   }
   return run_bwd(maps, prm, o, dout, dq, static_cast<size_t>(BH) * Nq, d, mask,
                  static_cast<int>(n_kblocks * BHkv), stream);
@@ -1365,7 +1480,8 @@ int attn_bwd_window(const void* q, const void* k, const void* v, const void* o, 
 size_t attn_bwd_colmask_workspace_size(int B, int H, int Nq, int d, int Hm, int Nk) {
   if (B < 0 || H < 0 || Nq < 0 || Hm < 0 || Nk < 0 || (d != 64 && d != 128)) return 0;
   return eab::bwd::colmask_workspace_bytes(static_cast<long long>(B) * H, Nq, d,
-                                           static_cast<long long>(B) * Hm, Nk);
+                                           static_cast<long long>(B) * Hm, Nk) +
+         eab::bwd::colmask_plan_bytes(static_cast<long long>(B) * H, Nk);
 }
 
 int attn_bwd_colmask(const void* q, const void* k, const void* v, const void* o, const void* dout,

@@ -300,11 +300,16 @@ int attn_bwd_window(const void *q, const void *k, const void *v, const void *o, 
  *   q, o, dout, dq : BF16 [B, H, Nq, d]    k, v, dk, dv : BF16 [B, Hkv, Nk, d]
  *   lse  : FP32 [B, H, Nq] from attn_fwd_colmask
  *   mask, Hm, causal : as attn_fwd_colmask
- *   workspace : DEVICE, 256-byte aligned, at least
- *       attn_bwd_colmask_workspace_size(B, H, Nq, d, Hm, Nk) bytes (attn_bwd's
- *       workspace followed by the mask's block summaries), overwritten
+ *   workspace : DEVICE, 256-byte aligned; give it
+ *       attn_bwd_colmask_workspace_size(B, H, Nq, d, Hm, Nk) bytes: attn_bwd's
+ *       workspace followed by the mask's block summaries (together the
+ *       minimum accepted), then room for an order of the CTAs (one int per
+ *       head and 128-key block); overwritten
  * Each CTA owns a 128-key block; the query tiles that every key of the block
  * hides form at most two ranges per query head, which are skipped outright.
+ * When the workspace has room (and the problem has at most 8192 CTAs), a
+ * one-CTA kernel orders the CTAs by the query tiles they visit, longest first
+ * within groups of key/value heads (the order changes no result).
  * Errors as attn_bwd, plus ATTN_ERR_INVALID_ARG for a NULL or misaligned mask,
  * Hm not in {1, H}, or a mask overlapping an output or the workspace.
  */

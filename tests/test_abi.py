@@ -222,14 +222,15 @@ def test_bwd_colmask_validation():
     ptrs = (A, A * 2, A * 3, A * 4, A * 5, A * 6, A * 7, A * 8, A * 9, A * 16)
     base = binding.attn_bwd_workspace_size(1, 2, 64, 64)
     need = binding.attn_bwd_colmask_workspace_size(1, 2, 64, 64, 1, 64)
-    assert need == (base + 255) // 256 * 256 + 32     # + one key block's two int4 summaries
+    minimum = (base + 255) // 256 * 256 + 32           # + one key block's two int4 summaries
+    assert need == minimum + 16                        # + the CTA plan: 2 ints, padded to 16 bytes
     assert binding.attn_bwd_colmask_workspace_size(1, 2, 64, 96, 1, 64) == 0
     M = A * 40
     sizes = (1, 2, 2, 64, 64, 64, 0.1, 0)
 
     def call(ws=need, mask=M, hm=1, sz=sizes, p=ptrs):
         return BC(*p, ws, *sz, mask, hm, None)
-    assert call(ws=need - 1) == 1                      # workspace too small
+    assert call(ws=minimum - 1) == 1                   # workspace too small
     assert call(ws=base) == 1                          # room for attn_bwd only
     assert call(mask=None) == 1
     assert call(mask=M + 4) == 1                       # misaligned mask

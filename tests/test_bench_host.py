@@ -125,3 +125,9 @@ def test_colmask_launch_count():
     assert bench.colmask_launches(w) == 3
     big = types.SimpleNamespace(B=64, Nq=65536, Nk=65536)
     assert bench.colmask_launches(big) == 2
+
+
+def test_bwd_colmask_launch_count():
+    """The document workload's backward launches row sums, mask summaries, the
+    CTA plan, the main kernel and the dQ rounding."""
+    assert bench.bwd_colmask_launches(WORKLOADS["docs_b2h16n8k_d128_causal"]) == 5
