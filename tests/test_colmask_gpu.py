@@ -270,3 +270,33 @@ def test_colmask_bwd_both_hidden_ranges_ragged():
     mags = harness.bwd_bound_dense(f(q), f(k), f(v), f(do), 0.1,
                                    lambda b, h: harness.colmask_visible(mask[b, 0], False))
     check_grads(tuple(x.float().cpu().numpy() for x in (dq, dk, dv)), ref, mags, "two ranges, ragged")
+
+
+def test_colmask_plan_order_changes_nothing():
+    """A workspace of the required size (block summaries only) keeps the launch
+    order; the full size runs the longest-first CTA plans.  Both give the same
+    forward output bit for bit and the same dK and dV (dQ's fp32 reductions
+    may land in another order)."""
+    import torch
+    from exact_attention_152_b200 import binding
+    B, H, N, d = 2, 4, 1000, 128
+    g = torch.Generator().manual_seed(21)
+    q, k, v, do = (torch.randn(B, H, N, d, generator=g).to(torch.bfloat16).cuda() for _ in range(4))
+    mask = torch.from_numpy(masks.documents([masks.document_lengths(31 + b, N, 40, 400) for b in range(B)],
+                                            N)).cuda()
+    n_kb = (N + 127) // 128
+    o_plan, l_plan = binding.fwd_colmask(q, k, v, mask, causal=True)
+    ws_min = torch.empty(B * n_kb * 32, dtype=torch.uint8, device="cuda")
+    o_fix, l_fix = binding.fwd_colmask(q, k, v, mask, causal=True, workspace=ws_min)
+    torch.cuda.synchronize()
+    assert torch.equal(o_plan.view(torch.int16), o_fix.view(torch.int16))
+    assert torch.equal(l_plan, l_fix)
+    dq_p, dk_p, dv_p = binding.bwd_colmask(q, k, v, o_plan, do, l_plan, mask, causal=True)
+    base = binding.attn_bwd_workspace_size(B, H, N, d)
+    ws_bmin = torch.empty((base + 255) // 256 * 256 + B * n_kb * 32, dtype=torch.uint8, device="cuda")
+    dq_f, dk_f, dv_f = binding.bwd_colmask(q, k, v, o_plan, do, l_plan, mask, causal=True, workspace=ws_bmin)
+    torch.cuda.synchronize()
+    assert torch.equal(dk_p.view(torch.int16), dk_f.view(torch.int16))
+    assert torch.equal(dv_p.view(torch.int16), dv_f.view(torch.int16))
+    assert torch.allclose(dq_p.float(), dq_f.float(), rtol=1e-2, atol=1e-3)
+    assert binding.attn_status_sync(torch.cuda.current_stream().cuda_stream) == 0
