@@ -16,8 +16,10 @@
 //
 // Design (this library's, for sm_100a):
 //  * Three launches: a row-sum kernel for D (and dQ's fp32 accumulator is
-//    zeroed), the main kernel, and a kernel that scales and rounds dQ to BF16.
-//    D and the dQ accumulator live in a caller-provided workspace.
+//    zeroed), the main kernel, and a kernel that scales and rounds dQ to BF16
+//    (column intervals add the mask summaries and, when the workspace has
+//    room, a one-CTA plan that orders the CTAs longest first).  D and the dQ
+//    accumulator live in a caller-provided workspace.
 //  * Main kernel: one CTA per (b, key/value head, 128-key block).  K and V of
 //    the block stay in shared memory; the CTA walks every query tile (128
 //    rows) of every query head that reads this key/value head (with a key

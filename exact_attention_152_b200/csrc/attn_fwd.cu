@@ -57,9 +57,10 @@
 //    windows), and column intervals (attn_fwd_colmask: each key hidden from up
 //    to two query-row intervals).  KV tiles outside the band are never
 //    visited; under column intervals a per-CTA bitmap, built from per-block
-//    summaries, lists the tiles some row sees.  A warp whose 64 x 32 block is
-//    cut by a mask folds it into two 32-bit keep words per row and tests one
-//    bit per score.
+//    summaries, lists the tiles some row sees, and a one-CTA plan kernel
+//    orders the CTAs by those counts, longest first within each mask row.  A
+//    warp whose 64 x 32 block is cut by a mask folds it into two 32-bit keep
+//    words per row and tests one bit per score.
 //  * Every wait is bounded (see sm100.cuh); a timeout sets the per-device
 //    status word and the CTA leaves its loops and exits cleanly.
 #include <cuda.h>
